@@ -1,0 +1,522 @@
+/*
+ * fg_oracle.c -- plain, slow, obviously-correct CPU oracle for the group-wise
+ * 4-bit ("W4 KV4") OPT decode step.
+ *
+ * TEST INFRASTRUCTURE.  Only the test-suite, the smoke check and the
+ * benchmark's CPU-baseline leg load this library.  It shares no code, header,
+ * table or constant with the CUDA library and never calls it.
+ *
+ * What it follows (the web pages the method is described on):
+ *   [G3]  "FlexGen Guide: High-Throughput LLM Offloading on One GPU",
+ *         section "3. Group-Wise 4-Bit Quantization for Weights and KV Cache":
+ *         weights and KV cache compressed to 4-bit integers, per-group scaling
+ *         over small contiguous groups (64), dequantised to FP16 for compute.
+ *   [G2]  same page, section "2. The Zig-Zag Block Schedule": a loaded layer
+ *         is reused for every micro-batch of the block, so a row's result
+ *         does not depend on the batch split.
+ *   [OPT] the OPT entry in the PIPO paper's list of references (model family):
+ *         pre-LayerNorm decoder layer, multi-head attention, ReLU FFN.
+ *
+ * Readings where the pages are silent (all listed in the design notes):
+ *   - asymmetric min-max per group: scale = fp16((max-min)/15), codes
+ *     round-half-even of (x-min)*(1/scale) in fp32, clamp to [0,15], two
+ *     codes per byte with the even element in the low nibble, fp16 min and
+ *     fp16 scale stored in separate planar arrays;
+ *   - a zero scale (constant group, or a scale that underflows fp16) gives
+ *     all codes 0 and a stored +0 scale; -0 min is stored as +0;
+ *   - dequantised value = min + code*scale computed exactly, rounded once to
+ *     fp16 (the FP16 fused multiply-add);
+ *   - the layer is evaluated in float64 from the fp16 inputs and the
+ *     dequantised fp16 weights; the new token's k and v are rounded to fp16,
+ *     appended to the cache in 4-bit form, and attention runs over the
+ *     dequantised cache including the new token; q is scaled by d^-1/2
+ *     after its bias; LayerNorm eps as passed (1e-5 for OPT).
+ *
+ * Build: gcc -O2 -ffp-contract=off -fPIC -shared -pthread (no fast-math), so
+ * every float operation below is one IEEE-754 operation rounded to nearest.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_GROUP 64
+
+/* ------------------------------------------------------------------------- */
+/* binary16 conversions, written from the IEEE 754 binary16 format:          */
+/* 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits.                  */
+/* ------------------------------------------------------------------------- */
+
+double oracle_f16_to_f64(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int m = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);                 /* subnormal: m * 2^-24 */
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(m | 0x400), e - 25);    /* (1024+m) * 2^(e-15-10) */
+    return sign ? -v : v;
+}
+
+float oracle_f16_to_f32(uint16_t h) { return (float)oracle_f16_to_f64(h); } /* exact */
+
+/* Round a binary64 value to the nearest binary16, ties to even. */
+uint16_t oracle_f64_to_f16(double x)
+{
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs(x);
+    if (isnan(x)) return 0x7e00;
+    /* 65504 is the largest finite half; halfway to 2^16 is 65520, and a tie
+       there goes to the even neighbour 2^16, i.e. overflows to infinity. */
+    if (a >= 65520.0) return sign | 0x7c00;
+    if (a == 0.0) return sign;
+    int e2;
+    frexp(a, &e2);            /* a = f * 2^e2, f in [0.5, 1) */
+    int E = e2 - 1;           /* unbiased exponent: 2^E <= a < 2^(E+1) */
+    if (E < -14) E = -14;     /* subnormal range shares the 2^-24 spacing */
+    double ulp = ldexp(1.0, E - 10);
+    double r = nearbyint(a / ulp);   /* a/ulp is exact (power-of-two scale) */
+    /* r is an integer multiple count of ulp; r may equal 2048 (next binade). */
+    long n = (long)r;
+    uint16_t bits;
+    if (E == -14 && n < 1024) {
+        bits = (uint16_t)n;                          /* subnormal (or 0) */
+    } else {
+        if (n >= 2048) { n >>= 1; E += 1; }          /* carried into next binade */
+        if (E > 15) return sign | 0x7c00;
+        bits = (uint16_t)(((E + 15) << 10) | (n - 1024));
+    }
+    return sign | bits;
+}
+
+uint16_t oracle_f32_to_f16(float x) { return oracle_f64_to_f16((double)x); } /* float->double exact */
+
+void oracle_f16_to_f64_array(const uint16_t *h, double *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = oracle_f16_to_f64(h[i]);
+}
+
+void oracle_f64_to_f16_array(const double *x, uint16_t *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = oracle_f64_to_f16(x[i]);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Group-wise 4-bit min-max quantisation [G3]                                 */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * One group of 64 fp16 values x[i*xs] -> 32 packed bytes codes[j*cs]
+ * (byte j = code(2j) | code(2j+1) << 4), fp16 min and fp16 scale.
+ * Steps, in this order, each one IEEE fp32 operation:
+ *   1. mn = min(x), mx = max(x);  mn = mn + 0  (turns -0 into +0)
+ *   2. d = mx - mn
+ *   3. scale_h = fp16_rn(d / 15)
+ *   4. scale_h == 0  ->  every code 0, stored scale +0
+ *   5. inv = 1 / scale_h
+ *   6. t = (x - mn) * inv    (two roundings, no fused multiply-add)
+ *   7. code = clamp(round_half_even(t), 0, 15)
+ *   8. min_h = fp16(mn)      (exact: mn is one of the fp16 inputs)
+ */
+static void quantize_group(const uint16_t *x, ptrdiff_t xs, uint8_t *codes, ptrdiff_t cs,
+                           uint16_t *min_out, uint16_t *scale_out)
+{
+    float v[OR_GROUP];
+    for (int i = 0; i < OR_GROUP; i++) v[i] = oracle_f16_to_f32(x[i * xs]);
+    float mn = v[0], mx = v[0];
+    for (int i = 1; i < OR_GROUP; i++) {
+        if (v[i] < mn) mn = v[i];
+        if (v[i] > mx) mx = v[i];
+    }
+    mn = mn + 0.0f;
+    float d = mx - mn;
+    float q15 = d / 15.0f;
+    uint16_t scale_h = oracle_f32_to_f16(q15);
+    float s = oracle_f16_to_f32(scale_h);
+    int q[OR_GROUP];
+    if (s == 0.0f) {
+        scale_h = 0;
+        for (int i = 0; i < OR_GROUP; i++) q[i] = 0;
+    } else {
+        float inv = 1.0f / s;
+        for (int i = 0; i < OR_GROUP; i++) {
+            float diff = v[i] - mn;
+            float t = diff * inv;
+            float r = nearbyintf(t);          /* default mode: nearest, ties to even */
+            int c = (int)r;
+            if (c < 0) c = 0;
+            if (c > 15) c = 15;
+            q[i] = c;
+        }
+    }
+    for (int j = 0; j < OR_GROUP / 2; j++)
+        codes[j * cs] = (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
+    *min_out = oracle_f32_to_f16(mn);
+    *scale_out = scale_h;
+}
+
+/* Dequantised value of one code: fp16_rn(mn + q*s), exact before the rounding
+   (q*s has at most 15 significant bits and every term is a multiple of 2^-24
+   below 2^18, so the float64 sum is exact). */
+static uint16_t dequant_one(int q, uint16_t min_h, uint16_t scale_h)
+{
+    double s = oracle_f16_to_f64(scale_h);
+    double m = oracle_f16_to_f64(min_h);
+    return oracle_f64_to_f16((double)q * s + m);
+}
+
+/*
+ * x viewed as [outer, n, inner]; groups of 64 consecutive elements along n.
+ * codes: [outer, n/2, inner]   mins, scales: [outer, n/64, inner].
+ * Returns 0, or -1 when n is not a multiple of 64.
+ */
+int oracle_quantize(const uint16_t *x, int64_t outer, int64_t n, int64_t inner,
+                    uint8_t *codes, uint16_t *mins, uint16_t *scales)
+{
+    if (n % OR_GROUP) return -1;
+    int64_t ng = n / OR_GROUP;
+    for (int64_t o = 0; o < outer; o++)
+        for (int64_t g = 0; g < ng; g++)
+            for (int64_t i = 0; i < inner; i++) {
+                const uint16_t *xp = x + (o * n + g * OR_GROUP) * inner + i;
+                uint8_t *cp = codes + (o * (n / 2) + g * (OR_GROUP / 2)) * inner + i;
+                int64_t m = (o * ng + g) * inner + i;
+                quantize_group(xp, inner, cp, inner, &mins[m], &scales[m]);
+            }
+    return 0;
+}
+
+int oracle_dequantize(const uint8_t *codes, const uint16_t *mins, const uint16_t *scales,
+                      int64_t outer, int64_t n, int64_t inner, uint16_t *y)
+{
+    if (n % OR_GROUP) return -1;
+    int64_t ng = n / OR_GROUP;
+    for (int64_t o = 0; o < outer; o++)
+        for (int64_t e = 0; e < n; e++)
+            for (int64_t i = 0; i < inner; i++) {
+                uint8_t byte = codes[(o * (n / 2) + e / 2) * inner + i];
+                int q = (e & 1) ? (byte >> 4) : (byte & 15);
+                int64_t m = (o * ng + e / OR_GROUP) * inner + i;
+                y[(o * n + e) * inner + i] = dequant_one(q, mins[m], scales[m]);
+            }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* OPT layer pieces, float64 [OPT]                                            */
+/* ------------------------------------------------------------------------- */
+
+/* y = (x - mean) / sqrt(var + eps) * gamma + beta, var the biased variance. */
+static void layernorm_row(const double *x, int h, const double *g, const double *b, double eps, double *y)
+{
+    double mean = 0.0;
+    for (int i = 0; i < h; i++) mean += x[i];
+    mean /= h;
+    double var = 0.0;
+    for (int i = 0; i < h; i++) var += (x[i] - mean) * (x[i] - mean);
+    var /= h;
+    double rstd = 1.0 / sqrt(var + eps);
+    for (int i = 0; i < h; i++) y[i] = (x[i] - mean) * rstd * g[i] + b[i];
+}
+
+/* y[n] = sum_k W[n][k] * x[k] + b[n]  (W row-major [N][K], PyTorch Linear orientation) */
+static void linear_row(const float *W, const double *b, const double *x, int N, int K, double *y)
+{
+    for (int n = 0; n < N; n++) {
+        const float *w = W + (int64_t)n * K;
+        double acc = 0.0;
+        for (int k = 0; k < K; k++) acc += (double)w[k] * x[k];
+        y[n] = acc + (b ? b[n] : 0.0);
+    }
+}
+
+/* Dequantise a [N][K] weight (groups along K) into float (exact for fp16 values). */
+static float *dequant_weight(const uint8_t *codes, const uint16_t *mins, const uint16_t *scales, int N, int K)
+{
+    float *W = (float *)malloc(sizeof(float) * (size_t)N * K);
+    if (!W) return NULL;
+    int ng = K / OR_GROUP;
+    for (int64_t n = 0; n < N; n++)
+        for (int k = 0; k < K; k++) {
+            uint8_t byte = codes[n * (K / 2) + k / 2];
+            int q = (k & 1) ? (byte >> 4) : (byte & 15);
+            int64_t m = n * ng + k / OR_GROUP;
+            W[n * K + k] = (float)oracle_f16_to_f64(dequant_one(q, mins[m], scales[m]));
+        }
+    return W;
+}
+
+static double *f16_vec(const uint16_t *h, int64_t n, double dflt)
+{
+    double *v = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    for (int64_t i = 0; i < n; i++) v[i] = h ? oracle_f16_to_f64(h[i]) : dflt;
+    return v;
+}
+
+/* y[m][n] = epilogue(sum_k x[m][k] * deq(W)[n][k] + b[n]) in float64.
+   relu: max(0, .);  residual (fp16 [M][N]) added after the activation;
+   the first qscale_cols outputs of each row are multiplied by qscale after the bias. */
+int oracle_linear(const uint16_t *x, int M, int K,
+                  const uint8_t *codes, const uint16_t *mins, const uint16_t *scales, int N,
+                  const uint16_t *bias, const uint16_t *residual, int relu,
+                  int qscale_cols, double qscale, double *y)
+{
+    if (K % OR_GROUP) return -1;
+    float *W = dequant_weight(codes, mins, scales, N, K);
+    double *b = f16_vec(bias, N, 0.0);
+    double *xr = (double *)malloc(sizeof(double) * (size_t)K);
+    if (!W || !b || !xr) return -2;
+    for (int64_t m = 0; m < M; m++) {
+        for (int k = 0; k < K; k++) xr[k] = oracle_f16_to_f64(x[m * K + k]);
+        double *yr = y + m * N;
+        linear_row(W, b, xr, N, K, yr);
+        for (int n = 0; n < N; n++) {
+            double v = yr[n];
+            if (n < qscale_cols) v *= qscale;
+            if (relu && v < 0.0) v = 0.0;
+            if (residual) v += oracle_f16_to_f64(residual[m * N + n]);
+            yr[n] = v;
+        }
+    }
+    free(W); free(b); free(xr);
+    return 0;
+}
+
+int oracle_layernorm(const uint16_t *x, int M, int h, const uint16_t *gamma, const uint16_t *beta,
+                     double eps, double *y)
+{
+    double *g = f16_vec(gamma, h, 1.0), *b = f16_vec(beta, h, 0.0);
+    double *xr = (double *)malloc(sizeof(double) * (size_t)h);
+    for (int64_t m = 0; m < M; m++) {
+        for (int i = 0; i < h; i++) xr[i] = oracle_f16_to_f64(x[m * h + i]);
+        layernorm_row(xr, h, g, b, eps, y + m * h);
+    }
+    free(g); free(b); free(xr);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* 4-bit KV cache [G3]: per layer, for each (sequence, head, position) the    */
+/* head_dim values are quantised in groups of 64 along head_dim.              */
+/*   codes [S][H][maxL][d/2], mins/scales [S][H][maxL][d/64]                  */
+/* ------------------------------------------------------------------------- */
+
+typedef struct {
+    uint8_t *kc; uint16_t *km, *ks;
+    uint8_t *vc; uint16_t *vm, *vs;
+    int S, H, d, maxL;
+} kv_t;
+
+static void kv_store(const kv_t *kv, int s, int head, int pos, const uint16_t *k16, const uint16_t *v16)
+{
+    int64_t slot = ((int64_t)s * kv->H + head) * kv->maxL + pos;
+    int ng = kv->d / OR_GROUP;
+    for (int g = 0; g < ng; g++) {
+        quantize_group(k16 + g * OR_GROUP, 1, kv->kc + slot * (kv->d / 2) + g * 32, 1,
+                       &kv->km[slot * ng + g], &kv->ks[slot * ng + g]);
+        quantize_group(v16 + g * OR_GROUP, 1, kv->vc + slot * (kv->d / 2) + g * 32, 1,
+                       &kv->vm[slot * ng + g], &kv->vs[slot * ng + g]);
+    }
+}
+
+static void kv_load(const uint8_t *c, const uint16_t *mn, const uint16_t *sc, int64_t slot, int d, double *out)
+{
+    int ng = d / OR_GROUP;
+    for (int i = 0; i < d; i++) {
+        uint8_t byte = c[slot * (d / 2) + i / 2];
+        int q = (i & 1) ? (byte >> 4) : (byte & 15);
+        int64_t m = slot * ng + i / OR_GROUP;
+        out[i] = oracle_f16_to_f64(dequant_one(q, mn[m], sc[m]));
+    }
+}
+
+/* Append fp16 k, v rows [R][H*d] (row stride ld) at positions pos_of_row[r] of
+   sequence seq_of_row[r]. */
+int oracle_kv_append(const uint16_t *k, const uint16_t *v, int64_t ld, int R,
+                     const int *seq_of_row, const int *pos_of_row,
+                     uint8_t *kc, uint16_t *km, uint16_t *ks, uint8_t *vc, uint16_t *vm, uint16_t *vs,
+                     int S, int H, int d, int maxL)
+{
+    if (d % OR_GROUP) return -1;
+    kv_t kv = {kc, km, ks, vc, vm, vs, S, H, d, maxL};
+    for (int r = 0; r < R; r++) {
+        if (pos_of_row[r] < 0 || pos_of_row[r] >= maxL || seq_of_row[r] < 0 || seq_of_row[r] >= S) return -2;
+        for (int hd = 0; hd < H; hd++)
+            kv_store(&kv, seq_of_row[r], hd, pos_of_row[r], k + (int64_t)r * ld + hd * d, v + (int64_t)r * ld + hd * d);
+    }
+    return 0;
+}
+
+/* Softmax attention of one query head over cached positions 0..L-1:
+   p_j = exp(q.K_j - max) / sum, o = sum_j p_j V_j   (q already scaled). */
+static void attend_head(const kv_t *kv, int s, int head, int L, const double *q, double *o, double *kbuf, double *scores)
+{
+    int d = kv->d;
+    int64_t base = ((int64_t)s * kv->H + head) * kv->maxL;
+    double mx = -INFINITY;
+    for (int j = 0; j < L; j++) {
+        kv_load(kv->kc, kv->km, kv->ks, base + j, d, kbuf);
+        double acc = 0.0;
+        for (int i = 0; i < d; i++) acc += q[i] * kbuf[i];
+        scores[j] = acc;
+        if (acc > mx) mx = acc;
+    }
+    double sum = 0.0;
+    for (int j = 0; j < L; j++) { scores[j] = exp(scores[j] - mx); sum += scores[j]; }
+    for (int i = 0; i < d; i++) o[i] = 0.0;
+    for (int j = 0; j < L; j++) {
+        kv_load(kv->vc, kv->vm, kv->vs, base + j, d, kbuf);
+        double p = scores[j] / sum;
+        for (int i = 0; i < d; i++) o[i] += p * kbuf[i];
+    }
+}
+
+/* q: fp16 rows [R][H*d] (row stride ld); each row attends over positions
+   0..len_of_row[r]-1 of sequence seq_of_row[r].  out: float64 [R][H*d]. */
+int oracle_attention(const uint16_t *q16, int64_t ld, int R, const int *seq_of_row, const int *len_of_row,
+                     const uint8_t *kc, const uint16_t *km, const uint16_t *ks,
+                     const uint8_t *vc, const uint16_t *vm, const uint16_t *vs,
+                     int S, int H, int d, int maxL, double *out)
+{
+    kv_t kv = {(uint8_t *)kc, (uint16_t *)km, (uint16_t *)ks, (uint8_t *)vc, (uint16_t *)vm, (uint16_t *)vs, S, H, d, maxL};
+    double *q = malloc(sizeof(double) * d), *kb = malloc(sizeof(double) * d);
+    double *sc = malloc(sizeof(double) * (maxL > 0 ? maxL : 1));
+    for (int r = 0; r < R; r++) {
+        if (len_of_row[r] < 1 || len_of_row[r] > maxL) { free(q); free(kb); free(sc); return -2; }
+        for (int hd = 0; hd < H; hd++) {
+            for (int i = 0; i < d; i++) q[i] = oracle_f16_to_f64(q16[(int64_t)r * ld + hd * d + i]);
+            attend_head(&kv, seq_of_row[r], hd, len_of_row[r], q, out + (int64_t)r * H * d + hd * d, kb, sc);
+        }
+    }
+    free(q); free(kb); free(sc);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* One OPT decoder layer, row by row [OPT][G3][G2]                            */
+/* ------------------------------------------------------------------------- */
+
+typedef struct {
+    int h, H, d, F;
+    double eps;
+    float *Wqkv, *Wo, *W1, *W2;           /* dequantised, [out][in] */
+    double *bqkv, *bo, *b1, *b2, *g1, *be1, *g2, *be2;
+    kv_t kv;
+    const uint16_t *x;                    /* [R][h] */
+    const int *seq_of_row, *pos_of_row;
+    int R, kv_only, nthreads;
+    double *out, *attn;                   /* [R][h] each (attn may be NULL) */
+} layer_ctx;
+
+typedef struct { layer_ctx *c; int tid; } layer_job;
+
+/* The rows of one sequence are processed in the order given, so a prompt
+   (positions 0..P-1) appends each token before the next one attends. */
+static void *layer_worker(void *arg)
+{
+    layer_job *job = (layer_job *)arg;
+    layer_ctx *c = job->c;
+    int h = c->h, H = c->H, d = c->d, F = c->F;
+    double *x = malloc(sizeof(double) * h), *a = malloc(sizeof(double) * h);
+    double *qkv = malloc(sizeof(double) * 3 * h), *o = malloc(sizeof(double) * h);
+    double *h1 = malloc(sizeof(double) * h), *a2 = malloc(sizeof(double) * h);
+    double *f = malloc(sizeof(double) * F), *y = malloc(sizeof(double) * h);
+    double *tmp = malloc(sizeof(double) * h), *kb = malloc(sizeof(double) * d);
+    double *sc = malloc(sizeof(double) * c->kv.maxL);
+    uint16_t *k16 = malloc(sizeof(uint16_t) * d), *v16 = malloc(sizeof(uint16_t) * d);
+    double qscale = 1.0 / sqrt((double)d);
+    for (int r = 0; r < c->R; r++) {
+        int s = c->seq_of_row[r], pos = c->pos_of_row[r];
+        if (s % c->nthreads != job->tid) continue;
+        for (int i = 0; i < h; i++) x[i] = oracle_f16_to_f64(c->x[(int64_t)r * h + i]);
+        /* 1. a = LN1(x) */
+        layernorm_row(x, h, c->g1, c->be1, c->eps, a);
+        /* 2. [q k v] = a Wqkv^T + b;  q *= d^-1/2 */
+        linear_row(c->Wqkv, c->bqkv, a, 3 * h, h, qkv);
+        for (int i = 0; i < h; i++) qkv[i] *= qscale;
+        /* 3. append k, v (rounded to fp16) to the 4-bit cache at pos */
+        for (int hd = 0; hd < H; hd++) {
+            for (int i = 0; i < d; i++) {
+                k16[i] = oracle_f64_to_f16(qkv[h + hd * d + i]);
+                v16[i] = oracle_f64_to_f16(qkv[2 * h + hd * d + i]);
+            }
+            kv_store(&c->kv, s, hd, pos, k16, v16);
+        }
+        if (c->kv_only) continue;
+        /* 4-5. attention of each head over cached positions 0..pos */
+        for (int hd = 0; hd < H; hd++)
+            attend_head(&c->kv, s, hd, pos + 1, qkv + hd * d, o + hd * d, kb, sc);
+        if (c->attn) memcpy(c->attn + (int64_t)r * h, o, sizeof(double) * h);
+        /* 6. h1 = x + o Wo^T + bo */
+        linear_row(c->Wo, c->bo, o, h, h, tmp);
+        for (int i = 0; i < h; i++) h1[i] = x[i] + tmp[i];
+        /* 7. y = h1 + relu(LN2(h1) W1^T + b1) W2^T + b2 */
+        layernorm_row(h1, h, c->g2, c->be2, c->eps, a2);
+        linear_row(c->W1, c->b1, a2, F, h, f);
+        for (int i = 0; i < F; i++) if (f[i] < 0.0) f[i] = 0.0;
+        linear_row(c->W2, c->b2, f, h, F, tmp);
+        for (int i = 0; i < h; i++) y[i] = h1[i] + tmp[i];
+        memcpy(c->out + (int64_t)r * h, y, sizeof(double) * h);
+    }
+    free(x); free(a); free(qkv); free(o); free(h1); free(a2); free(f); free(y); free(tmp); free(kb); free(sc);
+    free(k16); free(v16);
+    return NULL;
+}
+
+/*
+ * dims = {hidden, heads, head_dim, ffn}.  Weights as packed 4-bit tensors
+ * quantised along the input dim: wqkv [3h][h], wo [h][h], w1 [F][h], w2 [h][F]
+ * (codes, mins, scales each); biases and LayerNorm parameters fp16 (NULL = 0,
+ * gamma NULL = 1).  The KV cache arrays are read and written in place.
+ * kv_only = 1 stops after step 3 (cache fill for prompts).
+ */
+int oracle_layer_rows(const int *dims, double eps,
+                      const uint8_t *qkv_c, const uint16_t *qkv_m, const uint16_t *qkv_s, const uint16_t *bqkv,
+                      const uint8_t *o_c, const uint16_t *o_m, const uint16_t *o_s, const uint16_t *bo,
+                      const uint8_t *f1_c, const uint16_t *f1_m, const uint16_t *f1_s, const uint16_t *b1,
+                      const uint8_t *f2_c, const uint16_t *f2_m, const uint16_t *f2_s, const uint16_t *b2,
+                      const uint16_t *ln1_g, const uint16_t *ln1_b, const uint16_t *ln2_g, const uint16_t *ln2_b,
+                      uint8_t *kc, uint16_t *km, uint16_t *ks, uint8_t *vc, uint16_t *vm, uint16_t *vs,
+                      int S, int maxL,
+                      const uint16_t *x, int R, const int *seq_of_row, const int *pos_of_row,
+                      int kv_only, double *out, double *attn, int nthreads)
+{
+    layer_ctx c;
+    memset(&c, 0, sizeof(c));
+    c.h = dims[0]; c.H = dims[1]; c.d = dims[2]; c.F = dims[3]; c.eps = eps;
+    if (c.h != c.H * c.d || c.h % OR_GROUP || c.F % OR_GROUP || c.d % OR_GROUP) return -1;
+    for (int r = 0; r < R; r++)
+        if (seq_of_row[r] < 0 || seq_of_row[r] >= S || pos_of_row[r] < 0 || pos_of_row[r] >= maxL) return -2;
+    c.Wqkv = dequant_weight(qkv_c, qkv_m, qkv_s, 3 * c.h, c.h);
+    c.Wo = kv_only ? NULL : dequant_weight(o_c, o_m, o_s, c.h, c.h);
+    c.W1 = kv_only ? NULL : dequant_weight(f1_c, f1_m, f1_s, c.F, c.h);
+    c.W2 = kv_only ? NULL : dequant_weight(f2_c, f2_m, f2_s, c.h, c.F);
+    c.bqkv = f16_vec(bqkv, 3 * c.h, 0.0); c.bo = f16_vec(bo, c.h, 0.0);
+    c.b1 = f16_vec(b1, c.F, 0.0); c.b2 = f16_vec(b2, c.h, 0.0);
+    c.g1 = f16_vec(ln1_g, c.h, 1.0); c.be1 = f16_vec(ln1_b, c.h, 0.0);
+    c.g2 = f16_vec(ln2_g, c.h, 1.0); c.be2 = f16_vec(ln2_b, c.h, 0.0);
+    kv_t kv = {kc, km, ks, vc, vm, vs, S, c.H, c.d, maxL};
+    c.kv = kv;
+    c.x = x; c.seq_of_row = seq_of_row; c.pos_of_row = pos_of_row; c.R = R;
+    c.kv_only = kv_only; c.out = out; c.attn = attn;
+    if (nthreads < 1) nthreads = 1;
+    c.nthreads = nthreads;
+    pthread_t *th = malloc(sizeof(pthread_t) * nthreads);
+    layer_job *jobs = malloc(sizeof(layer_job) * nthreads);
+    for (int t = 0; t < nthreads; t++) {
+        jobs[t].c = &c; jobs[t].tid = t;
+        if (t > 0) pthread_create(&th[t], NULL, layer_worker, &jobs[t]);
+    }
+    layer_worker(&jobs[0]);
+    for (int t = 1; t < nthreads; t++) pthread_join(th[t], NULL);
+    free(th); free(jobs);
+    free(c.Wqkv); free(c.Wo); free(c.W1); free(c.W2);
+    free(c.bqkv); free(c.bo); free(c.b1); free(c.b2); free(c.g1); free(c.be1); free(c.g2); free(c.be2);
+    return 0;
+}
