@@ -26,11 +26,15 @@
  *     all codes 0 and a stored +0 scale; -0 min is stored as +0;
  *   - dequantised value = min + code*scale computed exactly, rounded once to
  *     fp16 (the FP16 fused multiply-add);
- *   - the layer is evaluated in float64 from the fp16 inputs and the
- *     dequantised fp16 weights; the new token's k and v are rounded to fp16,
- *     appended to the cache in 4-bit form, and attention runs over the
- *     dequantised cache including the new token; q is scaled by d^-1/2
- *     after its bias; LayerNorm eps as passed (1e-5 for OPT).
+ *   - the layer is an FP16 layer: every op is evaluated in float64 from fp16
+ *     operands (the dequantised fp16 weights and fp16 activations), and every
+ *     activation tensor one op hands to the next is rounded to fp16: the
+ *     LayerNorm outputs, q (after its bias and the d^-1/2 scale), k and v,
+ *     the attention output, the residual stream h1 and the ReLU output.  The
+ *     layer output itself is returned unrounded (float64).  The new token's
+ *     k and v are appended to the cache in 4-bit form before attention, which
+ *     runs over the dequantised cache including the new token.  LayerNorm eps
+ *     as passed (1e-5 for OPT).
  *
  * Build: gcc -O2 -ffp-contract=off -fPIC -shared -pthread (no fast-math), so
  * every float operation below is one IEEE-754 operation rounded to nearest.
@@ -252,6 +256,14 @@ static float *dequant_weight(const uint8_t *codes, const uint16_t *mins, const u
     return W;
 }
 
+/* The fp16 value nearest to x, as a double (an activation stored in fp16). */
+static double round16(double x) { return oracle_f16_to_f64(oracle_f64_to_f16(x)); }
+
+static void round16_vec(double *v, int64_t n)
+{
+    for (int64_t i = 0; i < n; i++) v[i] = round16(v[i]);
+}
+
 static double *f16_vec(const uint16_t *h, int64_t n, double dflt)
 {
     double *v = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
@@ -435,12 +447,14 @@ static void *layer_worker(void *arg)
         int s = c->seq_of_row[r], pos = c->pos_of_row[r];
         if (s % c->nthreads != job->tid) continue;
         for (int i = 0; i < h; i++) x[i] = oracle_f16_to_f64(c->x[(int64_t)r * h + i]);
-        /* 1. a = LN1(x) */
+        /* 1. a = fp16(LN1(x)) */
         layernorm_row(x, h, c->g1, c->be1, c->eps, a);
-        /* 2. [q k v] = a Wqkv^T + b;  q *= d^-1/2 */
+        round16_vec(a, h);
+        /* 2. [q k v] = a Wqkv^T + b;  q = fp16(q * d^-1/2), k = fp16(k), v = fp16(v) */
         linear_row(c->Wqkv, c->bqkv, a, 3 * h, h, qkv);
         for (int i = 0; i < h; i++) qkv[i] *= qscale;
-        /* 3. append k, v (rounded to fp16) to the 4-bit cache at pos */
+        round16_vec(qkv, 3 * h);
+        /* 3. append k, v to the 4-bit cache at pos */
         for (int hd = 0; hd < H; hd++) {
             for (int i = 0; i < d; i++) {
                 k16[i] = oracle_f64_to_f16(qkv[h + hd * d + i]);
@@ -449,17 +463,19 @@ static void *layer_worker(void *arg)
             kv_store(&c->kv, s, hd, pos, k16, v16);
         }
         if (c->kv_only) continue;
-        /* 4-5. attention of each head over cached positions 0..pos */
+        /* 4-5. o = fp16(attention of each head over cached positions 0..pos) */
         for (int hd = 0; hd < H; hd++)
             attend_head(&c->kv, s, hd, pos + 1, qkv + hd * d, o + hd * d, kb, sc);
+        round16_vec(o, h);
         if (c->attn) memcpy(c->attn + (int64_t)r * h, o, sizeof(double) * h);
-        /* 6. h1 = x + o Wo^T + bo */
+        /* 6. h1 = fp16(x + o Wo^T + bo) */
         linear_row(c->Wo, c->bo, o, h, h, tmp);
-        for (int i = 0; i < h; i++) h1[i] = x[i] + tmp[i];
-        /* 7. y = h1 + relu(LN2(h1) W1^T + b1) W2^T + b2 */
+        for (int i = 0; i < h; i++) h1[i] = round16(x[i] + tmp[i]);
+        /* 7. y = h1 + fp16(relu(fp16(LN2(h1)) W1^T + b1)) W2^T + b2 */
         layernorm_row(h1, h, c->g2, c->be2, c->eps, a2);
+        round16_vec(a2, h);
         linear_row(c->W1, c->b1, a2, F, h, f);
-        for (int i = 0; i < F; i++) if (f[i] < 0.0) f[i] = 0.0;
+        for (int i = 0; i < F; i++) f[i] = f[i] < 0.0 ? 0.0 : round16(f[i]);
         linear_row(c->W2, c->b2, f, h, F, tmp);
         for (int i = 0; i < h; i++) y[i] = h1[i] + tmp[i];
         memcpy(c->out + (int64_t)r * h, y, sizeof(double) * h);
