@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Decode throughput of one OPT layer block with 4-bit weights and a 4-bit KV cache.
+
+Default workload (one GPU): the OPT-6.7B-shaped layer -- hidden 4096, 32 heads x 128,
+FFN 16384 -- over a zig-zag block of 8 GPU batches x 64 sequences, prompt 512 (prefilled,
+untimed), then decode steps at positions 512, 513, ...  A step is one fg_layer_decode
+over the whole block: LN1, QKV W4A16 GEMM, 4-bit KV append, decode attention over the
+4-bit cache, out-proj GEMM + residual, LN2, FC1 GEMM + ReLU, FC2 GEMM + residual.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload ...]
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own block of
+sequences (independent replicas, weak scaling, no collective on the data path); the
+timed region is bracketed by barriers and the time is the max over ranks.
+The reference arm (--impl reference) times the CPU oracle on a bounded sample of the
+same workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    "opt-6.7b-layer": dict(hidden=4096, heads=32, ffn=16384, nb=8, gbs=64, prompt=512, steps=32),
+    "opt-125m-layer": dict(hidden=768, heads=12, ffn=3072, nb=1, gbs=4, prompt=32, steps=8),
+}
+METRIC = "decode tokens/s per OPT layer block (W4 KV4)"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], tc_burst=d["bf16_tflops"], tc_sustained=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, tc_burst=1590.0, tc_sustained=1400.0, source="fallback")
+
+
+def kernel_work(wl, S, L_avg):
+    """Algorithmic work per launch of each kernel of one decode step (bytes or flops)."""
+    h, F, H = wl["hidden"], wl["ffn"], wl["heads"]
+    d = h // H
+    kv_tok = 2 * (d // 2 + 4 * (d // 64))            # K and V codes + fp16 min/scale per (seq, head, token)
+    w4 = lambda n, k: n * k // 2 + n * (k // 64) * 4  # packed weight bytes
+    return {
+        "ln1": ("hbm", 2 * S * h * 2 + 4 * h),
+        "qkv_gemm": ("tensor", 2 * S * 3 * h * h),
+        "kv_append": ("hbm", S * 2 * h * 2 + S * H * kv_tok),
+        "attention": ("hbm", S * H * L_avg * kv_tok + 2 * S * h * 2),
+        "out_gemm": ("tensor", 2 * S * h * h),
+        "ln2": ("hbm", 2 * S * h * 2 + 4 * h),
+        "fc1_gemm": ("tensor", 2 * S * F * h),
+        "fc2_gemm": ("tensor", 2 * S * h * F),
+    }, {"w4_bytes": w4(3 * h, h) + w4(h, h) + w4(F, h) + w4(h, F), "kv_bytes_per_token": kv_tok}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while active."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows]
+        reasons = set()
+        for r in rows:
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                 r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "samples": len(rows),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------------------
+# CPU oracle baseline (test infrastructure; only this leg of the benchmark loads it)
+# ----------------------------------------------------------------------------------------
+
+class OracleSample:
+    """One oracle decode step for `n_seqs` sequences at position `prompt`.
+
+    Set-up (untimed): the layer's seeded fp16 weights quantised by the oracle, and the
+    sampled sequences' caches filled with `prompt` tokens of seeded N(0,1) k/v in 4-bit
+    form (the decode step's work does not depend on how they were produced).
+    step() times oracle.layer_rows as it stands (it dequantises the weights, then runs
+    the rows on `threads` threads)."""
+
+    def __init__(self, wl, n_seqs: int, threads: int, seed: int = 0):
+        import oracle
+        import seeded_inputs as si
+        self.oracle = oracle
+        h, H, F, P = wl["hidden"], wl["heads"], wl["ffn"], wl["prompt"]
+        self.H, self.P, self.n, self.threads = H, P, n_seqs, threads
+        maxL = (P + wl["steps"] + 63) // 64 * 64
+        self.W = oracle.LayerWeights(si.layer_weights_f16(seed, h, F))
+        self.cache = oracle.KVCache(n_seqs, H, h // H, maxL)
+        for s in range(n_seqs):
+            k = si.normal_f16(seed, si.STREAM["k_new"], (P, h), 1.0, start=s * P * h)
+            v = si.normal_f16(seed, si.STREAM["v_new"], (P, h), 1.0, start=s * P * h)
+            oracle.kv_append(self.cache, k, v, np.full(P, s), np.arange(P))
+        self.x = si.decode_inputs(seed, 0, n_seqs, h)
+
+    def step(self) -> float:
+        t0 = time.perf_counter()
+        self.oracle.layer_rows(self.W, self.H, self.cache, self.x, np.arange(self.n), np.full(self.n, self.P),
+                               nthreads=self.threads)
+        return time.perf_counter() - t0
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    threads = os.cpu_count() or 1
+    n_seqs = max(1, min(threads, 8))
+    sample = OracleSample(wl, n_seqs, threads)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = sample.step()
+        if i >= args.warmup:
+            times.append(t)
+    mean = sum(times) / len(times)
+    value = n_seqs / mean
+    S = wl["nb"] * wl["gbs"]
+    desc = (f"{n_seqs} of {S} sequences, one decode step at position {wl['prompt']} per step "
+            f"(cache of {wl['prompt']} tokens); {threads} threads")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "block": f"{wl['nb']}x{wl['gbs']}", "hidden": wl["hidden"],
+                   "prompt": wl["prompt"]},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ----------------------------------------------------------------------------------------
+# GPU path
+# ----------------------------------------------------------------------------------------
+
+def read_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if it matches the current sources."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(kernel)
+    if not e:
+        return None
+    import hashlib
+    src = os.path.join(ROOT, "bit_compressed_decode_b200", "csrc", e["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != e["source_sha"]:
+            return None
+    return e["dram_bytes_per_launch"]
+
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    import bit_compressed_decode_b200 as fg
+    import seeded_inputs as si
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    h, H, F, P = wl["hidden"], wl["heads"], wl["ffn"], wl["prompt"]
+    nb, gbs = wl["nb"], wl["gbs"]
+    S = nb * gbs
+    d = h // H
+    nsteps_cfg = wl["steps"]
+    maxL = (P + nsteps_cfg + 63) // 64 * 64
+    cfg = fg.LayerConfig(h, H, F)
+
+    # weights: the shared seeded host generator (same on every rank: replicas)
+    w16 = si.layer_weights_f16(0, h, F)
+    lw = fg.LayerWeights.from_fp16(cfg, w16, device=dev)
+    del w16
+    cache = fg.KVCache(S, H, d, maxL, device=dev)
+    # prompt hidden states: seeded device generator (bulk synthetic N(0,1)), per rank
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + rank)
+    zero = torch.zeros(S, dtype=torch.int32, device=dev)
+    chunk = max(1, 65536 // P)
+    pws = torch.empty(cfg.workspace_bytes(chunk * P), dtype=torch.uint8, device=dev)
+    for s0 in range(0, S, chunk):
+        n = min(chunk, S - s0)
+        xp = torch.randn((n, P, h), generator=g, device=dev, dtype=torch.float16)
+        fg.fg_layer_prefill(cfg, lw, cache.view(s0, n), xp, zero[:n], workspace=pws)
+        del xp
+    del pws
+    fg.fg_sync_status()
+
+    xs = [torch.randn((S, h), generator=g, device=dev, dtype=torch.float16) for _ in range(4)]
+    pos = [torch.full((S,), P + t, dtype=torch.int32, device=dev) for t in range(nsteps_cfg)]
+    out = torch.empty((S, h), dtype=torch.float16, device=dev)
+    ws = torch.empty(cfg.workspace_bytes(S), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i, x=None, o=None, p=None):
+        fg.fg_layer_decode(cfg, lw, cache, xs[i % 4] if x is None else x, pos[i % nsteps_cfg] if p is None else p,
+                           num_gpu_batches=nb, gpu_batch_size=gbs, out=out if o is None else o, workspace=ws,
+                           stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        step(i)
+    fg.fg_sync_status()
+
+    # ---- timed region (device time, CUDA events on the launching stream) ----
+    sampler = ClockSampler(dev.index if world == 1 else local)
+    sampler.start()
+    time.sleep(0.3)
+    fg.fg_profile_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    fg.fg_profile_enable(False)
+    clocks = sampler.stop()
+    prof = fg.fg_profile_collect()
+    fg.fg_sync_status()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * S * args.steps / (ms / 1e3)
+
+    # ---- end to end through host buffers: H2D inputs, decode, D2H result, every step ----
+    xh = [torch.empty((S, h), dtype=torch.float16, pin_memory=True) for _ in range(2)]
+    for i in range(2):
+        xh[i].copy_(xs[i])
+    ph = [torch.full((S,), P + t, dtype=torch.int32).pin_memory() for t in range(nsteps_cfg)]
+    oh = torch.empty((S, h), dtype=torch.float16, pin_memory=True)
+    xd = torch.empty((S, h), dtype=torch.float16, device=dev)
+    pd = torch.empty((S,), dtype=torch.int32, device=dev)
+    barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for i in range(args.steps):
+        xd.copy_(xh[i % 2], non_blocking=True)
+        pd.copy_(ph[(args.warmup + i) % nsteps_cfg], non_blocking=True)
+        step(0, x=xd, p=pd)
+        oh.copy_(out, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ems = f0.elapsed_time(f1)
+    if world > 1:
+        t = torch.tensor([ems], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ems = float(t.item())
+    e2e_value = world * S * args.steps / (ems / 1e3)
+    h2d = S * h * 2 + S * 4
+    d2h = S * h * 2
+
+    # ---- roofline of the dominant kernel (and of every kernel) ----
+    peaks = load_peaks()
+    L_avg = P + (args.warmup + (args.steps - 1) / 2.0) % nsteps_cfg + 1
+    work, totals = kernel_work(wl, S, L_avg)
+    kernels = {}
+    for name, (tot_ms, cnt) in prof.items():
+        if cnt == 0:
+            continue
+        avg_s = tot_ms / cnt / 1e3
+        bound, units = work[name]
+        if bound == "tensor":
+            ach, peak, unit = units / avg_s / 1e12, peaks["tc_sustained"], "TFLOP/s"
+        else:
+            ach, peak, unit = units / avg_s / 1e9, peaks["hbm"], "GB/s"
+        kernels[name] = {"bound": bound, "avg_us": round(avg_s * 1e6, 2), "launches": cnt,
+                         "share": round(tot_ms / max(1e-9, sum(v[0] for v in prof.values())), 4),
+                         "achieved": round(ach, 1), "peak": peak, "unit": unit, "frac": round(ach / peak, 4)}
+    dom = max(kernels, key=lambda k: kernels[k]["share"])
+    kd = kernels[dom]
+    roofline = {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"],
+                "unit": kd["unit"], "frac": kd["frac"],
+                "traffic": read_traffic(dom, args.workload),
+                "peak_source": f"{peaks['source']} ({'sustained bf16' if kd['bound'] == 'tensor' else 'copy'})"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        n = max(1, min(threads, 8))
+        osample = OracleSample(wl, n, threads)
+        t = min(osample.step() for _ in range(2))
+        cpu = {"value": n / t, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} of {S} sequences, one decode step at position {P} ({threads} threads)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": args.workload, "block": f"{nb}x{gbs}", "sequences_per_gpu": S, "hidden": h,
+                       "heads": H, "ffn": F, "prompt": P, "positions": f"{P}..{P + nsteps_cfg - 1} (cycled)",
+                       "weights": "W4 g64", "kv": "KV4 g64", "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (KV4 cache %.2f GB + W4 %.0f MB per step)" % (
+                           cache.nbytes() / 1e9, totals["w4_bytes"] / 1e6)},
+            "roofline": roofline,
+            "kernels": kernels,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": sum(v[1] for v in prof.values()),
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="opt-6.7b-layer")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

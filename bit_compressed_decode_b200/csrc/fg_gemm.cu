@@ -1,0 +1,479 @@
+// fg_gemm.cu -- W4A16 linear layer on the 5th-generation tensor cores (tcgen05/TMEM).
+//
+// y[m][n] = epi( sum_k x[m][k] * deq(W)[n][k] + b[n] ),  W packed 4-bit along k.
+//
+// "FlexGen Guide: High-Throughput LLM Offloading on One GPU", section 3: weights stay
+// in 4-bit form and are dequantised on the fly so the tensor cores compute in FP16.
+// Here the dequantisation target is shared memory, in the tensor cores' operand layout:
+//
+//   CTA tile: 256 output features (two 128-row MMA accumulators) x NT tokens x a k-range.
+//   warps 0..7   dequantise: thread t owns weight row n0+t; per 64-wide k-tile it loads
+//                32 code bytes + the group's fp16 min/scale (prefetched 3 tiles ahead),
+//                expands them with fp16 FMAs (exactly round(min + code*scale)) and stores
+//                128 bytes into the 128-byte-swizzled K-major A tile; then the epilogue.
+//   warp 8       TMA: the x tile [NT tokens x 64] (128-byte swizzle) per k-tile.
+//   warp 9       one lane issues tcgen05.mma (M=128, N=NT, K=16, fp16 in, fp32 in TMEM),
+//                A = dequantised W tile, B = x tile, and commits each stage back.
+//   The accumulators D[feature][token] live in TMEM (2*NT columns); the epilogue reads
+//   them with tcgen05.ld, adds bias / q-scale / ReLU / residual and stores fp16.
+//   When the k-range is split, the splits of one output tile run as one thread-block
+//   cluster: each CTA copies its partial accumulator, 32 token columns at a time, into
+//   its own shared memory, and the owner of each 32-column chunk adds the partials of
+//   all CTAs of the cluster over distributed shared memory in cluster-rank order
+//   (deterministic) before the epilogue -- no partial sums go through global memory.
+// Every mbarrier wait is bounded (FG_WAIT_TIMEOUT_NS) and reports FG_ERR_TIMEOUT.
+#include <stdio.h>
+
+#include "fg_internal.cuh"
+
+namespace {
+
+constexpr int kBK = 64;                      // k-tile = one quantisation group
+constexpr int kNAcc = 2;                     // accumulators (128 features each) per CTA
+constexpr int kBM = 128 * kNAcc;             // features per CTA
+constexpr int kDeqWarps = 4 * kNAcc;         // dequant / epilogue warps
+constexpr int kTmaWarp = kDeqWarps;
+constexpr int kMmaWarp = kDeqWarps + 1;
+constexpr int kThreads = (kDeqWarps + 2) * 32;
+constexpr int kPrefetch = 3;                 // k-tiles of codes in flight per dequant thread
+
+template <int NT>
+struct Cfg {
+  static constexpr int STAGES = NT >= 256 ? 3 : 4;
+  static constexpr int A_BYTES = 128 * 128;  // one accumulator's A tile: 128 rows x 128 B
+  static constexpr int B_BYTES = NT * 128;   // x tile: NT rows x 128 B
+  static constexpr int STAGE = kNAcc * A_BYTES + B_BYTES;
+  static constexpr int SMEM = STAGES * STAGE + 1024;  // + alignment slack
+  static constexpr int COLS = kNAcc * NT < 32 ? 32 : kNAcc * NT;
+  static constexpr uint32_t IDESC = umma_idesc_f16_f32(128, NT);
+};
+
+struct GemmArgs {
+  const uint8_t *wc;   // codes [N][K/2]
+  const __half *wm;    // mins  [N][K/64]
+  const __half *ws;    // scales[N][K/64]
+  const __half *bias;  // [N] or null
+  const __half *res;   // [M][N] or null
+  __half *y;           // [M][N]
+  int M, N, K;
+  int relu, qcols;
+  float qscale;
+  int splits;
+  unsigned int *err;
+};
+
+__device__ __forceinline__ float epilogue(float v, int m, int n, const GemmArgs &a) {
+  if (a.bias) v += __half2float(a.bias[n]);
+  if (n < a.qcols) v *= a.qscale;
+  if (a.relu) v = fmaxf(v, 0.f);
+  if (a.res) v += __half2float(a.res[static_cast<int64_t>(m) * a.N + n]);
+  return v;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                 const GemmArgs a) {
+  using C = Cfg<NT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_a[C::STAGES], full_b[C::STAGES], empty[C::STAGES], accum_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * kBM, t0 = blockIdx.y * NT, split = blockIdx.z;
+  const int ktiles = a.K / kBK;
+  const int kt0 = static_cast<int>((static_cast<int64_t>(split) * ktiles) / a.splits);
+  const int kt1 = static_cast<int>((static_cast<int64_t>(split + 1) * ktiles) / a.splits);
+  const int nk = kt1 - kt0;
+  volatile int *abortp = &abort_flag;
+
+  auto a_tile = [&](int st, int acc) { return smem + st * C::STAGE + acc * C::A_BYTES; };
+  auto b_tile = [&](int st) { return smem + st * C::STAGE + kNAcc * C::A_BYTES; };
+
+  if (tid == 0) {
+    for (int i = 0; i < C::STAGES; i++) {
+      mbar_init(smem_u32(&full_a[i]), kDeqWarps);
+      mbar_init(smem_u32(&full_b[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    mbar_init(smem_u32(&accum_bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(&tmem_slot), C::COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp < kDeqWarps) {
+    // ---------------- dequantise producer: one weight row per thread ----------------
+    const int row = tid;  // 0..255
+    const int n = n0 + row;
+    const bool live = n < a.N;
+    const int acc = row >> 7, r = row & 127;
+    const uint4 *crow = reinterpret_cast<const uint4 *>(a.wc + static_cast<int64_t>(live ? n : 0) * (a.K / 2));
+    const __half *mrow = a.wm + static_cast<int64_t>(live ? n : 0) * (a.K / kBK);
+    const __half *srow = a.ws + static_cast<int64_t>(live ? n : 0) * (a.K / kBK);
+    uint4 cb[kPrefetch][2];
+    __half mb[kPrefetch], sb[kPrefetch];
+#pragma unroll
+    for (int j = 0; j < kPrefetch; j++) {
+      if (j < nk && live) {
+        const int kt = kt0 + j;
+        cb[j][0] = crow[kt * 2];
+        cb[j][1] = crow[kt * 2 + 1];
+        mb[j] = mrow[kt];
+        sb[j] = srow[kt];
+      } else {
+        cb[j][0] = cb[j][1] = make_uint4(0, 0, 0, 0);
+        mb[j] = sb[j] = __ushort_as_half(0);
+      }
+    }
+    for (int i = 0; i < nk; i++) {
+      const int st = i % C::STAGES;
+      const uint4 c0 = cb[0][0], c1 = cb[0][1];
+      const __half m0 = mb[0], s0 = sb[0];
+#pragma unroll
+      for (int j = 0; j + 1 < kPrefetch; j++) {
+        cb[j][0] = cb[j + 1][0];
+        cb[j][1] = cb[j + 1][1];
+        mb[j] = mb[j + 1];
+        sb[j] = sb[j + 1];
+      }
+      if (i + kPrefetch < nk && live) {
+        const int kt = kt0 + i + kPrefetch;
+        cb[kPrefetch - 1][0] = crow[kt * 2];
+        cb[kPrefetch - 1][1] = crow[kt * 2 + 1];
+        mb[kPrefetch - 1] = mrow[kt];
+        sb[kPrefetch - 1] = srow[kt];
+      }
+      if (i >= C::STAGES && !mbar_wait_bounded(smem_u32(&empty[st]), ((i / C::STAGES) - 1) & 1, abortp, a.err))
+        break;
+      const __half2 s2 = __half2half2(s0), m2 = __half2half2(m0);
+      uint8_t *at = a_tile(st, acc);
+      const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+      for (int c = 0; c < 8; c++) {
+        const uint4 v = live ? dequant8(words[c], s2, m2) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(at + sw128_offset(r, c)) = v;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&full_a[st]));
+    }
+  } else if (warp == kTmaWarp) {
+    // ---------------- TMA producer for the x tiles ----------------
+    if (lane == 0) {
+      prefetch_tmap(&xmap);
+      int issued = 0;
+      for (int i = 0; i < nk; i++) {
+        const int st = i % C::STAGES;
+        if (i >= C::STAGES && !mbar_wait_bounded(smem_u32(&empty[st]), ((i / C::STAGES) - 1) & 1, abortp, a.err))
+          break;
+        const uint32_t bar = smem_u32(&full_b[st]);
+        mbar_arrive_expect_tx(bar, C::B_BYTES);
+        tma_load_2d(smem_u32(b_tile(st)), &xmap, (kt0 + i) * kBK, t0, bar);
+        issued = i + 1;
+      }
+      if (*abortp) {  // let copies still in flight land before the CTA exits
+        for (int j = issued > C::STAGES ? issued - C::STAGES : 0; j < issued; j++)
+          mbar_wait_bounded(smem_u32(&full_b[j % C::STAGES]), (j / C::STAGES) & 1, nullptr, nullptr);
+      }
+    }
+  } else {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      for (int i = 0; i < nk; i++) {
+        const int st = i % C::STAGES;
+        const uint32_t par = (i / C::STAGES) & 1;
+        if (!mbar_wait_bounded(smem_u32(&full_a[st]), par, abortp, a.err)) break;
+        if (!mbar_wait_bounded(smem_u32(&full_b[st]), par, abortp, a.err)) break;
+        tc_fence_after();
+        const uint32_t bbase = smem_u32(b_tile(st));
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; kk++) {
+          const uint64_t bdesc = umma_desc_sw128(bbase + kk * 32);
+#pragma unroll
+          for (int acc = 0; acc < kNAcc; acc++) {
+            const uint64_t adesc = umma_desc_sw128(smem_u32(a_tile(st, acc)) + kk * 32);
+            umma_f16(tmem + acc * NT, adesc, bdesc, C::IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(smem_u32(&empty[st]));
+      }
+      umma_commit(smem_u32(&accum_bar));  // also tracks completion if the loop stopped early
+    }
+  }
+
+  // ---------------- epilogue: TMEM -> registers -> global ----------------
+  constexpr int kChunks = NT >= 32 ? NT / 32 : 1;  // 32-column chunks of the accumulator
+  constexpr int kCW = NT >= 32 ? 32 : NT;          // columns per chunk
+  bool ready = false;
+  if (warp < kDeqWarps) {
+    ready = mbar_wait_bounded(smem_u32(&accum_bar), 0, nullptr, a.err) && !*abortp;
+    tc_fence_after();
+  }
+  const int acc = (warp & 7) >> 2, q = warp & 3;
+  const int n = n0 + acc * 128 + q * 32 + lane;
+  const bool nlive = n < a.N;
+  auto load_chunk = [&](int ch, uint32_t (&v)[32]) {
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * NT + ch * kCW;
+    if constexpr (NT >= 32) {
+      tmem_ld_32x32b_x32(taddr, v);
+    } else {
+      tmem_ld_32x32b_x16(taddr, v);  // NT == 16: this accumulator's 16 columns only
+    }
+    tmem_wait_ld();
+  };
+  if (a.splits == 1) {
+    if (warp < kDeqWarps) {
+      for (int ch = 0; ch < kChunks; ch++) {
+        uint32_t v[32];
+        load_chunk(ch, v);
+        if (!ready) continue;
+#pragma unroll
+        for (int j = 0; j < kCW; j++) {
+          const int m = t0 + ch * kCW + j;
+          if (m < a.M && nlive)
+            a.y[static_cast<int64_t>(m) * a.N + n] = __float2half_rn(epilogue(__uint_as_float(v[j]), m, n, a));
+        }
+      }
+    }
+  } else {
+    // Cluster reduction of the k-split partial sums.  Chunks are staged kRound at a time
+    // in the (now idle) pipeline buffers as [chunk][column][feature] fp32; chunk ch is
+    // reduced by cluster rank ch % splits.  Every thread of every CTA takes the same
+    // cluster barriers.
+    constexpr int kChunkBytes = kCW * kBM * 4;
+    constexpr int kRound = (C::STAGES * C::STAGE) / kChunkBytes < kChunks ? (C::STAGES * C::STAGE) / kChunkBytes
+                                                                           : kChunks;
+    static_assert(kRound >= 1, "reduction buffer");
+    const uint32_t rank = cluster_ctarank();
+    float *buf = reinterpret_cast<float *>(smem);
+    const int feat = tid;  // reducer thread -> feature row of the tile (epilogue warps only)
+    for (int r0 = 0; r0 < kChunks; r0 += kRound) {
+      if (warp < kDeqWarps) {
+        for (int i = 0; i < kRound && r0 + i < kChunks; i++) {
+          uint32_t v[32];
+          load_chunk(r0 + i, v);
+          float *cb = buf + i * (kCW * kBM);
+          const int f = acc * 128 + q * 32 + lane;
+#pragma unroll
+          for (int j = 0; j < kCW; j++) cb[j * kBM + f] = __uint_as_float(v[j]);
+        }
+      }
+      __syncwarp();
+      cluster_sync_all();
+      if (warp < kDeqWarps && ready) {
+        const int nn = n0 + feat;
+        for (int i = 0; i < kRound && r0 + i < kChunks; i++) {
+          const int ch = r0 + i;
+          if (ch % a.splits != static_cast<int>(rank)) continue;
+          const uint32_t base = smem_u32(buf + i * (kCW * kBM) + feat);
+          constexpr int kU = kCW < 8 ? kCW : 8;
+          for (int j0 = 0; j0 < kCW; j0 += kU) {
+            float sum[kU];
+#pragma unroll
+            for (int u = 0; u < kU; u++) sum[u] = 0.f;
+#pragma unroll
+            for (int sp = 0; sp < 8; sp++) {  // cluster-rank order: deterministic
+              if (sp < a.splits) {
+                const uint32_t rb = mapa_shared(base + j0 * kBM * 4, sp);
+#pragma unroll
+                for (int u = 0; u < kU; u++) sum[u] += ld_shared_cluster_f32(rb + u * kBM * 4);
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < kU; u++) {
+              const int m = t0 + ch * kCW + j0 + u;
+              if (m < a.M && nn < a.N)
+                a.y[static_cast<int64_t>(m) * a.N + nn] = __float2half_rn(epilogue(sum[u], m, nn, a));
+            }
+          }
+        }
+      }
+      __syncwarp();
+      cluster_sync_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::COLS);
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+int pick_nt(int M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  if (M <= 128) return 128;
+  return 256;
+}
+
+struct Plan {
+  int nt, n_tiles, t_tiles, splits;
+};
+
+// Split the k-range over the CTAs of a cluster only to fill the SMs: minimise
+// waves * k-tiles per CTA, with a small charge per extra split for the cluster reduction.
+Plan make_plan(int M, int N, int K) {
+  Plan p;
+  p.nt = pick_nt(M);
+  p.n_tiles = (N + kBM - 1) / kBM;
+  p.t_tiles = (M + p.nt - 1) / p.nt;
+  const int ktiles = K / kBK;
+  const int base = p.n_tiles * p.t_tiles;
+  const int nsm = sm_count();
+  double best = 1e30;
+  p.splits = 1;
+  for (int s = 1; s <= 8; s++) {
+    if (s > 1 && ktiles / s < 8) break;
+    const int waves = (base * s + nsm - 1) / nsm;
+    const double cost = static_cast<double>(waves) * ((ktiles + s - 1) / s) * (1.0 + 0.05 * (s - 1));
+    if (cost < best - 1e-9) {
+      best = cost;
+      p.splits = s;
+    }
+  }
+  return p;
+}
+
+template <int NT>
+fg_status launch_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st) {
+  using C = Cfg<NT>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    fg_status rc = fg_cuda_check(
+        cudaFuncSetAttribute(w4a16_gemm_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    if (rc != FG_OK) return rc;
+    attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(p.n_tiles, p.t_tiles, p.splits);
+  lc.blockDim = dim3(kThreads, 1, 1);
+  lc.dynamicSmemBytes = C::SMEM;
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = p.splits;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  fg_status rc = fg_cuda_check(cudaLaunchKernelEx(&lc, w4a16_gemm_kernel<NT>, map, a));
+  if (rc != FG_OK) return rc;
+  return fg_launch_check();
+}
+
+}  // namespace
+
+// No global scratch: split-k partial sums are reduced inside the cluster.
+size_t fg_linear_ws_bytes(int, int, int) { return 0; }
+
+fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, const fg_half *bias,
+                           const fg_half *residual, int flags, int qscale_cols, float qscale, fg_half *y,
+                           void *workspace, size_t ws_bytes, cudaStream_t st) {
+  const int N = static_cast<int>(w->shape[0]);
+  if (M == 0) return FG_OK;
+  (void)workspace;
+  (void)ws_bytes;
+  Plan p = make_plan(M, N, K);
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FG_ERR_CUDA;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {kBK, static_cast<cuuint32_t>(p.nt)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<fg_half *>(x), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return FG_ERR_INVALID;
+  GemmArgs a;
+  a.wc = w->codes;
+  a.wm = reinterpret_cast<const __half *>(w->mins);
+  a.ws = reinterpret_cast<const __half *>(w->scales);
+  a.bias = reinterpret_cast<const __half *>(bias);
+  a.res = (flags & FG_EPI_RESIDUAL) ? reinterpret_cast<const __half *>(residual) : nullptr;
+  a.y = reinterpret_cast<__half *>(y);
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.relu = (flags & FG_EPI_RELU) ? 1 : 0;
+  a.qcols = qscale_cols;
+  a.qscale = qscale;
+  a.splits = p.splits;
+  a.err = fg_error_word_ptr();
+  if (!a.err) return FG_ERR_CUDA;
+  switch (p.nt) {
+    case 16: return launch_nt<16>(map, a, p, st);
+    case 32: return launch_nt<32>(map, a, p, st);
+    case 64: return launch_nt<64>(map, a, p, st);
+    case 128: return launch_nt<128>(map, a, p, st);
+    default: return launch_nt<256>(map, a, p, st);
+  }
+}
+
+extern "C" size_t fg_linear_workspace_bytes(int M, int N, int K) { return fg_linear_ws_bytes(M, N, K); }
+
+extern "C" fg_status fg_linear_w4a16(const fg_half *x, int M, int K, const fg_qtensor *w, const fg_half *bias,
+                                     const fg_half *residual, int flags, int qscale_cols, float qscale, fg_half *y,
+                                     void *workspace, size_t workspace_bytes, void *stream) {
+  if (!w || M < 0 || K <= 0) return FG_ERR_INVALID;
+  if (w->bits != 4 || w->group != 64) return FG_ERR_UNSUPPORTED;
+  if (w->ndim != 2 || w->dim != 1 || w->shape[1] != K) return FG_ERR_SHAPE;
+  const int64_t N = w->shape[0];
+  if (K % 64 || N <= 0 || N % 128 || N > (1 << 30)) return FG_ERR_SHAPE;
+  if (flags & ~(FG_EPI_RELU | FG_EPI_RESIDUAL)) return FG_ERR_INVALID;
+  if (M == 0) return FG_OK;
+  if (!x || !y || !w->codes || !w->mins || !w->scales) return FG_ERR_INVALID;
+  if (!fg_aligned16(x) || !fg_aligned16(y) || !fg_aligned16(w->codes)) return FG_ERR_INVALID;
+  if ((flags & FG_EPI_RESIDUAL) && !residual) return FG_ERR_INVALID;
+  return fg_linear_launch(x, M, K, w, bias, residual, flags, qscale_cols, qscale, y, workspace, workspace_bytes,
+                          static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,316 @@
+// fg_internal.cuh -- shared device/host helpers of the sm_100a library.
+// Inline PTX for mbarriers, bulk/tensor copies (TMA) and the 5th-generation
+// tensor-core instructions (tcgen05), plus bounded waits that report through
+// the device error word instead of hanging.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fg.h"
+
+// Bits of the device error word.
+#define FG_DEVERR_RANGE 1u
+#define FG_DEVERR_TIMEOUT 2u
+
+// Every pipeline wait gives up after this many nanoseconds of device time.
+#define FG_WAIT_TIMEOUT_NS 2000000000ull
+
+// Host helpers (fg_status.cu).
+unsigned int *fg_error_word_ptr();  // device address of this device's error word (nullptr on failure)
+fg_status fg_cuda_check(cudaError_t e);  // records the error text, maps to FG_ERR_CUDA
+fg_status fg_launch_check();             // cudaGetLastError after a launch
+
+static inline bool fg_aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// --------------------------------------------------------------------------------------
+// device helpers
+// --------------------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\t"
+      "mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\t"
+      "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+      "r"(bytes)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for phase `parity` of an mbarrier.  Gives up (returns false) when the
+// shared abort flag is raised by another thread or after FG_WAIT_TIMEOUT_NS,
+// in which case it raises the abort flag and the device error word.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                                  unsigned int *err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (abort_flag && *abort_flag) return false;
+    if (globaltimer_ns() - t0 > FG_WAIT_TIMEOUT_NS) {
+      if (abort_flag) *abort_flag = 1;
+      if (err) atomicOr(err, FG_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// 1-D bulk copy global -> shared, completion counted on an mbarrier (bytes % 16 == 0,
+// both addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// 2-D tiled tensor copy global -> shared (no multicast).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---- thread-block clusters / distributed shared memory --------------------------------
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Every thread of every CTA in the cluster arrives (release) and waits (acquire).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+// ---- tcgen05 (5th-gen tensor cores, TMEM accumulators) -------------------------------
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, fp16 inputs, fp32 accumulation.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on an mbarrier once every previously issued tcgen05.mma of this thread has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp gets lane (base+i), columns col..col+31.
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+        "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+        "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor of a K-major operand tile laid out in the
+// 128-byte swizzle pattern: rows of 128 bytes, 8-row (1024-byte) atoms stacked
+// along M/N (stride 1024 bytes), atom base 1024-byte aligned.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);  // start address
+  d |= static_cast<uint64_t>(1u) << 16;                     // leading byte offset (unused for swizzled K-major)
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;             // stride byte offset: 8 rows * 128 B
+  d |= static_cast<uint64_t>(1u) << 46;                     // descriptor version (sm_100)
+  d |= static_cast<uint64_t>(2u) << 61;                     // layout: 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor: kind::f16 with fp16 A and B, fp32 D, both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_f16_f32(int M, int N) {
+  return (1u << 4)                                   // D format: f32
+         | (0u << 7) | (0u << 10)                    // A, B format: f16
+         | (0u << 15) | (0u << 16)                   // A, B K-major
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
+  return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+// ---- 4-bit group helpers shared by the quantise kernels --------------------------------
+
+// fp16 value of 1024 + n for a nibble n in bits 0..3 and 16..19 of `bits` (magic-number
+// conversion: 0x6400 is 1024.0 in binary16 and the nibble fills the low mantissa bits).
+__device__ __forceinline__ __half2 nib2_plus1024(uint32_t bits) {
+  uint32_t v = (bits & 0x000F000Fu) | 0x64006400u;
+  return *reinterpret_cast<__half2 *>(&v);
+}
+
+// Dequantise 8 codes of one 32-bit word (element 2j in the low nibble of byte j)
+// into 8 fp16 values in element order: round_to_fp16(min + code * scale), exactly
+// rounded once (hfma2).  Each pair (e_2j, e_2j+1) is gathered with one byte
+// permute (byte j of w -> bits 0..7, byte j of w>>4 -> bits 16..23); the mask in
+// nib2_plus1024 keeps the low nibble of each half.
+__device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 scale2, __half2 min2) {
+  const __half2 k1024 = __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400));
+  const uint32_t s = w >> 4;
+  __half2 c01 = __hsub2(nib2_plus1024(__byte_perm(w, s, 0x0400)), k1024);
+  __half2 c23 = __hsub2(nib2_plus1024(__byte_perm(w, s, 0x0501)), k1024);
+  __half2 c45 = __hsub2(nib2_plus1024(__byte_perm(w, s, 0x0602)), k1024);
+  __half2 c67 = __hsub2(nib2_plus1024(__byte_perm(w, s, 0x0703)), k1024);
+  __half2 y01 = __hfma2(c01, scale2, min2);
+  __half2 y23 = __hfma2(c23, scale2, min2);
+  __half2 y45 = __hfma2(c45, scale2, min2);
+  __half2 y67 = __hfma2(c67, scale2, min2);
+  uint4 r;
+  r.x = *reinterpret_cast<uint32_t *>(&y01);
+  r.y = *reinterpret_cast<uint32_t *>(&y23);
+  r.z = *reinterpret_cast<uint32_t *>(&y45);
+  r.w = *reinterpret_cast<uint32_t *>(&y67);
+  return r;
+}
+
+// Cooperative quantisation of one group of 64 fp16 values held by 8 consecutive
+// lanes (lane j of the 8 holds elements 8j..8j+7 in v).  Steps and fp32 operation
+// order as stated in fg.h: min/max over the group, mn += 0, d = mx - mn,
+// scale = fp16_rn(d/15), inv = 1/scale, code = clamp(rint((x - mn) * inv), 0, 15).
+// Returns this lane's 8 codes packed into one 32-bit word (element 8j+2i in the low
+// nibble of byte i) and the group's fp16 min and scale.  All 32 lanes of the warp
+// must call it together.
+__device__ __forceinline__ uint32_t quant_group8(const uint4 v, __half &min_h, __half &scale_h) {
+  float x[8];
+  {
+    const __half2 *h2 = reinterpret_cast<const __half2 *>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      float2 f = __half22float2(h2[i]);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < 8; i++) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  mn = __fadd_rn(mn, 0.0f);
+  const float d = __fsub_rn(mx, mn);
+  __half sh = __float2half_rn(__fdiv_rn(d, 15.0f));
+  const float s = __half2float(sh);
+  uint32_t word = 0;
+  if (s != 0.0f) {
+    const float inv = __fdiv_rn(1.0f, s);
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      int c = __float2int_rn(__fmul_rn(__fsub_rn(x[i], mn), inv));
+      c = min(max(c, 0), 15);
+      word |= static_cast<uint32_t>(c) << (4 * i);
+    }
+  } else {
+    sh = __ushort_as_half(0);
+  }
+  min_h = __float2half_rn(mn);
+  scale_h = sh;
+  return word;
+}

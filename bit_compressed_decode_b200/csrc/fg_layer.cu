@@ -1,0 +1,260 @@
+// fg_layer.cu -- one OPT decoder layer over a block of GPU batches, W4 weights, KV4 cache.
+//
+// "FlexGen Guide: High-Throughput LLM Offloading on One GPU", section 2 (The Zig-Zag Block
+// Schedule): the layer's weights are loaded once and reused by every GPU batch of the
+// block.  On this GPU the reuse happens inside each GEMM: one launch covers all rows of
+// the block, so every weight tile is read from HBM once per step and applied to all
+// num_gpu_batches * gpu_batch_size sequences.  Section 3: weights and KV cache are 4-bit.
+// Layer math (OPT, pre-LayerNorm, ReLU): see fg_layer_decode in fg.h.
+#include <math.h>
+
+#include "fg_internal.cuh"
+
+// kernels/launchers of the other translation units
+fg_status fg_layernorm_launch(const fg_half *x, int M, int h, const fg_half *gamma, const fg_half *beta, float eps,
+                              fg_half *y, cudaStream_t st);
+fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, const fg_half *bias,
+                           const fg_half *residual, int flags, int qscale_cols, float qscale, fg_half *y,
+                           void *workspace, size_t ws_bytes, cudaStream_t st);
+size_t fg_linear_ws_bytes(int M, int N, int K);
+fg_status fg_kv_validate(const fg_kv_cache *kv);
+fg_status fg_kv_append_launch(const fg_kv_cache *kv, const fg_half *k, const fg_half *v, int64_t ld, int rows,
+                              int rows_per_seq, const int32_t *positions, cudaStream_t st);
+fg_status fg_attention_launch(const fg_kv_cache *kv, const fg_half *q, int64_t ldq, fg_half *out, int64_t ldo,
+                              int rows, int rows_per_seq, const int32_t *positions, cudaStream_t st);
+
+int fg_profile_begin(int slot, cudaStream_t st);
+void fg_profile_end(int idx, cudaStream_t st);
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool config_ok(const fg_layer_config *c) {
+  if (!c) return false;
+  if (c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256) return false;
+  if (c->num_heads < 1 || c->hidden != c->num_heads * c->head_dim) return false;
+  if (c->hidden % 128 || c->ffn % 128 || c->ffn <= 0 || c->hidden > 16384) return false;
+  return true;
+}
+
+struct Matrix {
+  int64_t n, k;
+};
+
+// Offsets of every array inside the layer blob (256-byte aligned).
+struct BlobLayout {
+  size_t off[4][3];  // [matrix][codes, mins, scales]
+  size_t vec[8];     // bqkv, bo, b1, b2, ln1_g, ln1_b, ln2_g, ln2_b
+  size_t total;
+  Matrix mat[4];
+};
+
+BlobLayout blob_layout(const fg_layer_config *c) {
+  BlobLayout L;
+  const int64_t h = c->hidden, F = c->ffn;
+  L.mat[0] = {3 * h, h};
+  L.mat[1] = {h, h};
+  L.mat[2] = {F, h};
+  L.mat[3] = {h, F};
+  size_t p = 0;
+  for (int i = 0; i < 4; i++) {
+    const size_t numel = static_cast<size_t>(L.mat[i].n * L.mat[i].k);
+    L.off[i][0] = p;
+    p = align256(p + numel / 2);
+    L.off[i][1] = p;
+    p = align256(p + numel / 64 * 2);
+    L.off[i][2] = p;
+    p = align256(p + numel / 64 * 2);
+  }
+  const int64_t vlen[8] = {3 * h, h, F, h, h, h, h, h};
+  for (int i = 0; i < 8; i++) {
+    L.vec[i] = p;
+    p = align256(p + vlen[i] * 2);
+  }
+  L.total = p;
+  return L;
+}
+
+struct WsLayout {
+  size_t a, qkv, o, h1, f, gemm, total;
+};
+
+WsLayout ws_layout(const fg_layer_config *c, int rows) {
+  WsLayout w;
+  const size_t R = static_cast<size_t>(rows), h = c->hidden, F = c->ffn;
+  size_t p = 0;
+  w.a = p;
+  p = align256(p + R * h * 2);
+  w.qkv = p;
+  p = align256(p + R * 3 * h * 2);
+  w.o = p;
+  p = align256(p + R * h * 2);
+  w.h1 = p;
+  p = align256(p + R * h * 2);
+  w.f = p;
+  p = align256(p + R * F * 2);
+  w.gemm = p;
+  size_t g = fg_linear_ws_bytes(rows, 3 * c->hidden, c->hidden);
+  g = g > fg_linear_ws_bytes(rows, c->hidden, c->hidden) ? g : fg_linear_ws_bytes(rows, c->hidden, c->hidden);
+  g = g > fg_linear_ws_bytes(rows, c->ffn, c->hidden) ? g : fg_linear_ws_bytes(rows, c->ffn, c->hidden);
+  g = g > fg_linear_ws_bytes(rows, c->hidden, c->ffn) ? g : fg_linear_ws_bytes(rows, c->hidden, c->ffn);
+  p = align256(p + g);
+  w.total = p;
+  return w;
+}
+
+bool weights_ok(const fg_layer_config *c, const fg_layer_weights *w) {
+  const int64_t h = c->hidden, F = c->ffn;
+  const fg_qtensor *m[4] = {&w->wqkv, &w->wo, &w->w1, &w->w2};
+  const int64_t shp[4][2] = {{3 * h, h}, {h, h}, {F, h}, {h, F}};
+  for (int i = 0; i < 4; i++) {
+    if (m[i]->ndim != 2 || m[i]->dim != 1 || m[i]->bits != 4 || m[i]->group != 64) return false;
+    if (m[i]->shape[0] != shp[i][0] || m[i]->shape[1] != shp[i][1]) return false;
+    if (!m[i]->codes || !m[i]->mins || !m[i]->scales || !fg_aligned16(m[i]->codes)) return false;
+  }
+  return true;
+}
+
+// The layer over `rows` hidden-state rows; row r is token r % rows_per_seq of
+// sequence r / rows_per_seq of `kv` (a view starting at the first sequence).
+fg_status run_layer(const fg_layer_config *c, const fg_layer_weights *w, const fg_kv_cache *kv, const fg_half *x_in,
+                    fg_half *x_out, const int32_t *positions, int rows, int rows_per_seq, uint8_t *ws,
+                    size_t ws_bytes, cudaStream_t st) {
+  const WsLayout L = ws_layout(c, rows);
+  if (ws_bytes < L.total) return FG_ERR_WORKSPACE;
+  const int h = c->hidden, F = c->ffn;
+  fg_half *a = reinterpret_cast<fg_half *>(ws + L.a);
+  fg_half *qkv = reinterpret_cast<fg_half *>(ws + L.qkv);
+  fg_half *o = reinterpret_cast<fg_half *>(ws + L.o);
+  fg_half *h1 = reinterpret_cast<fg_half *>(ws + L.h1);
+  fg_half *f = reinterpret_cast<fg_half *>(ws + L.f);
+  void *gws = ws + L.gemm;
+  const size_t gbytes = L.total - L.gemm;
+  const float qscale = 1.0f / sqrtf(static_cast<float>(c->head_dim));
+  fg_status rc;
+  int ev;
+#define FG_STEP(slot, call)                    \
+  ev = fg_profile_begin(slot, st);             \
+  if ((rc = (call)) != FG_OK) return rc;       \
+  fg_profile_end(ev, st);
+  // a = LN1(x)
+  FG_STEP(0, fg_layernorm_launch(x_in, rows, h, w->ln1_g, w->ln1_b, c->ln_eps, a, st));
+  // [q k v] = a Wqkv^T + bqkv; q *= d^-1/2
+  FG_STEP(1, fg_linear_launch(a, rows, h, &w->wqkv, w->bqkv, nullptr, 0, h, qscale, qkv, gws, gbytes, st));
+  // append k, v (4-bit) at the sequences' positions
+  FG_STEP(2, fg_kv_append_launch(kv, qkv + h, qkv + 2 * h, 3 * h, rows, rows_per_seq, positions, st));
+  // o = softmax(q K^T) V over the 4-bit cache
+  FG_STEP(3, fg_attention_launch(kv, qkv, 3 * h, o, h, rows, rows_per_seq, positions, st));
+  // h1 = x + o Wo^T + bo
+  FG_STEP(4, fg_linear_launch(o, rows, h, &w->wo, w->bo, x_in, FG_EPI_RESIDUAL, 0, 1.f, h1, gws, gbytes, st));
+  // a = LN2(h1)
+  FG_STEP(5, fg_layernorm_launch(h1, rows, h, w->ln2_g, w->ln2_b, c->ln_eps, a, st));
+  // f = relu(a W1^T + b1)
+  FG_STEP(6, fg_linear_launch(a, rows, h, &w->w1, w->b1, nullptr, FG_EPI_RELU, 0, 1.f, f, gws, gbytes, st));
+  // x_out = h1 + f W2^T + b2
+  FG_STEP(7, fg_linear_launch(f, rows, F, &w->w2, w->b2, h1, FG_EPI_RESIDUAL, 0, 1.f, x_out, gws, gbytes, st));
+#undef FG_STEP
+  return FG_OK;
+}
+
+fg_kv_cache kv_view(const fg_kv_cache *kv, int s0, int n) {
+  fg_kv_cache v = *kv;
+  const size_t slots = static_cast<size_t>(s0) * kv->num_heads * kv->max_len;
+  v.k_codes += slots * (kv->head_dim / 2);
+  v.v_codes += slots * (kv->head_dim / 2);
+  v.k_mins += slots * (kv->head_dim / 64);
+  v.k_scales += slots * (kv->head_dim / 64);
+  v.v_mins += slots * (kv->head_dim / 64);
+  v.v_scales += slots * (kv->head_dim / 64);
+  v.num_seqs = n;
+  return v;
+}
+
+fg_status check_common(const fg_layer_config *c, const fg_layer_weights *w, const fg_kv_cache *kv,
+                       const fg_half *x_in, fg_half *x_out, const int32_t *positions, int nb, int gbs) {
+  if (!config_ok(c)) return FG_ERR_UNSUPPORTED;
+  if (!w || !weights_ok(c, w)) return FG_ERR_INVALID;
+  fg_status rc = fg_kv_validate(kv);
+  if (rc != FG_OK) return rc;
+  if (kv->num_heads != c->num_heads || kv->head_dim != c->head_dim) return FG_ERR_SHAPE;
+  if (nb < 0 || gbs < 0) return FG_ERR_INVALID;
+  if (static_cast<int64_t>(nb) * gbs != kv->num_seqs) return FG_ERR_SHAPE;
+  if (kv->num_seqs == 0) return FG_OK;
+  if (!x_in || !x_out || !positions || !fg_aligned16(x_in) || !fg_aligned16(x_out)) return FG_ERR_INVALID;
+  return FG_OK;
+}
+
+}  // namespace
+
+extern "C" size_t fg_layer_blob_bytes(const fg_layer_config *c) {
+  if (!config_ok(c)) return 0;
+  return blob_layout(c).total;
+}
+
+extern "C" fg_status fg_layer_weights_from_blob(const fg_layer_config *c, void *blob, fg_layer_weights *out) {
+  if (!config_ok(c)) return FG_ERR_UNSUPPORTED;
+  if (!blob || !out || (reinterpret_cast<uintptr_t>(blob) & 255)) return FG_ERR_INVALID;
+  const BlobLayout L = blob_layout(c);
+  uint8_t *b = static_cast<uint8_t *>(blob);
+  fg_qtensor *m[4] = {&out->wqkv, &out->wo, &out->w1, &out->w2};
+  for (int i = 0; i < 4; i++) {
+    m[i]->codes = b + L.off[i][0];
+    m[i]->mins = reinterpret_cast<fg_half *>(b + L.off[i][1]);
+    m[i]->scales = reinterpret_cast<fg_half *>(b + L.off[i][2]);
+    m[i]->ndim = 2;
+    m[i]->shape[0] = L.mat[i].n;
+    m[i]->shape[1] = L.mat[i].k;
+    m[i]->shape[2] = m[i]->shape[3] = 1;
+    m[i]->dim = 1;
+    m[i]->bits = 4;
+    m[i]->group = 64;
+  }
+  fg_half **v[8] = {&out->bqkv, &out->bo, &out->b1, &out->b2, &out->ln1_g, &out->ln1_b, &out->ln2_g, &out->ln2_b};
+  for (int i = 0; i < 8; i++) *v[i] = reinterpret_cast<fg_half *>(b + L.vec[i]);
+  return FG_OK;
+}
+
+extern "C" size_t fg_layer_workspace_bytes(const fg_layer_config *c, int rows) {
+  if (!config_ok(c) || rows < 0) return 0;
+  return ws_layout(c, rows).total;
+}
+
+extern "C" fg_status fg_layer_decode(const fg_layer_config *c, const fg_layer_weights *w, const fg_kv_cache *kv,
+                                     const fg_half *x_in, fg_half *x_out, const int32_t *positions,
+                                     int num_gpu_batches, int gpu_batch_size, void *workspace,
+                                     size_t workspace_bytes, void *stream) {
+  fg_status rc = check_common(c, w, kv, x_in, x_out, positions, num_gpu_batches, gpu_batch_size);
+  if (rc != FG_OK || kv->num_seqs == 0) return rc;
+  if (!workspace || !fg_aligned16(workspace)) return FG_ERR_INVALID;
+  return run_layer(c, w, kv, x_in, x_out, positions, kv->num_seqs, 1, static_cast<uint8_t *>(workspace),
+                   workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" fg_status fg_layer_prefill(const fg_layer_config *c, const fg_layer_weights *w, const fg_kv_cache *kv,
+                                      const fg_half *x_in, fg_half *x_out, const int32_t *positions, int prompt_len,
+                                      int num_gpu_batches, int gpu_batch_size, void *workspace,
+                                      size_t workspace_bytes, void *stream) {
+  fg_status rc = check_common(c, w, kv, x_in, x_out, positions, num_gpu_batches, gpu_batch_size);
+  if (rc != FG_OK || kv->num_seqs == 0) return rc;
+  if (prompt_len < 1) return FG_ERR_SHAPE;
+  if (prompt_len > kv->max_len) return FG_ERR_RANGE;
+  if (!workspace || !fg_aligned16(workspace)) return FG_ERR_INVALID;
+  // Process whole sequences in chunks that fit the workspace given.
+  const int S = kv->num_seqs;
+  int chunk = S;
+  while (chunk > 0 && ws_layout(c, chunk * prompt_len).total > workspace_bytes) chunk = chunk > 1 ? chunk / 2 : 0;
+  if (chunk == 0) return FG_ERR_WORKSPACE;
+  if (static_cast<int64_t>(chunk) * prompt_len > (1 << 30)) return FG_ERR_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t h = c->hidden;
+  for (int s0 = 0; s0 < S; s0 += chunk) {
+    const int n = chunk < S - s0 ? chunk : S - s0;
+    const fg_kv_cache sub = kv_view(kv, s0, n);
+    const int64_t off = static_cast<int64_t>(s0) * prompt_len * h;
+    rc = run_layer(c, w, &sub, x_in + off, x_out + off, positions + s0, n * prompt_len, prompt_len,
+                   static_cast<uint8_t *>(workspace), workspace_bytes, st);
+    if (rc != FG_OK) return rc;
+  }
+  return FG_OK;
+}

@@ -1,0 +1,296 @@
+/*
+ * fg.h -- C ABI of the B200 (sm_100a) group-wise 4-bit decode library.
+ *
+ * What the library computes follows these web pages:
+ *   [G2] "FlexGen Guide: High-Throughput LLM Offloading on One GPU",
+ *        section "2. The Zig-Zag Block Schedule" -- a loaded layer is reused for
+ *        every GPU batch of a block before the next layer is loaded.
+ *   [G3] same page, section "3. Group-Wise 4-Bit Quantization for Weights and KV
+ *        Cache" -- weights and KV cache held as 4-bit integers with per-group
+ *        scaling over contiguous groups, dequantised on the fly for FP16 compute.
+ *   [G1] same page, section "1. Three-Tier Storage Hierarchy" -- weights kept in
+ *        CPU memory and moved to the GPU layer by layer.
+ *   [OPT] the OPT entry of the PIPO paper's reference list -- the model family
+ *        (pre-LayerNorm decoder layer, multi-head attention, ReLU FFN).
+ *
+ * The 4-bit format (the pages give no formula; this is the reading the whole
+ * library and its tests use).  For every group of 64 consecutive fp16 values
+ * x_0..x_63 along the grouping dim, each step one IEEE fp32 operation:
+ *   mn = min(x) + 0 (so -0 becomes +0);  d = max(x) - mn;
+ *   scale = fp16_rn(d / 15);  if scale == 0: every code 0, stored scale +0;
+ *   inv = 1 / scale;  code_i = clamp(round_half_even((x_i - mn) * inv), 0, 15);
+ *   byte j of the group = code_{2j} | code_{2j+1} << 4  (even element low);
+ *   min and scale are stored as fp16 in two planar arrays.
+ * Dequantised value: fp16_rn(mn + code * scale), the exact value rounded once
+ * (an fp16 fused multiply-add).
+ *
+ * Conventions for every call:
+ *   - fp16 values travel as their binary16 bit patterns (fg_half).
+ *   - The caller owns all memory.  Pointers named "device" must point to
+ *     device memory of the current CUDA device (or memory mapped into it);
+ *     the library never allocates or frees device memory.
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Work is enqueued asynchronously; argument errors are returned before
+ *     anything is launched.  Faults detected inside kernels (a cache position
+ *     out of range, a pipeline wait that timed out) set a device error word
+ *     that fg_sync_status() reports and clears.
+ *   - Device pointers must be 16-byte aligned unless stated otherwise;
+ *     a misaligned pointer returns FG_ERR_INVALID.
+ *   - No call throws, exits or prints.
+ */
+#ifndef FG_H_
+#define FG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FG_API __attribute__((visibility("default")))
+#else
+#define FG_API
+#endif
+
+typedef uint16_t fg_half;  /* IEEE 754 binary16 bit pattern */
+
+typedef enum {
+    FG_OK = 0,
+    FG_ERR_INVALID = 1,     /* null/misaligned pointer, bad enum, negative size */
+    FG_ERR_SHAPE = 2,       /* size not a multiple of the group, inconsistent dims */
+    FG_ERR_UNSUPPORTED = 3, /* bits != 4, group != 64, dims the kernels do not cover */
+    FG_ERR_RANGE = 4,       /* a cache position outside [0, max_len) (host or device check) */
+    FG_ERR_CUDA = 5,        /* a CUDA runtime call failed (launch, copy, event) */
+    FG_ERR_TIMEOUT = 6,     /* a bounded wait inside a kernel gave up */
+    FG_ERR_WORKSPACE = 7    /* workspace too small */
+} fg_status;
+
+/* Human-readable name of a status (static string). */
+FG_API const char *fg_status_string(fg_status s);
+
+/* Synchronises `stream`, then reads and clears the current device's error
+ * word.  Returns FG_ERR_RANGE or FG_ERR_TIMEOUT if a kernel flagged one since
+ * the last call, FG_ERR_CUDA if the stream reported an error, else FG_OK. */
+FG_API fg_status fg_sync_status(void *stream);
+
+/* Text of the last CUDA runtime error seen by this library on this thread. */
+FG_API const char *fg_last_cuda_error(void);
+
+/* ---------------------------------------------------------------------- */
+/* Packed 4-bit tensors [G3]                                               */
+/* ---------------------------------------------------------------------- */
+
+/* A tensor of `shape` quantised in groups of `group` along `dim`.
+ * codes:  uint8, shape with shape[dim] halved  (even element in the low nibble)
+ * mins, scales: fp16, shape with shape[dim] divided by `group`.
+ * All three are row-major (C order) and caller-owned (device memory). */
+typedef struct {
+    uint8_t *codes;
+    fg_half *mins;
+    fg_half *scales;
+    int32_t ndim;        /* 1..4 */
+    int64_t shape[4];
+    int32_t dim;         /* grouping dim, 0..ndim-1 */
+    int32_t bits;        /* 4 */
+    int32_t group;       /* 64 */
+} fg_qtensor;
+
+/* Byte sizes of the codes array and of each of the mins/scales arrays. */
+FG_API fg_status fg_qtensor_bytes(int ndim, const int64_t *shape, int dim, int bits, int group,
+                           size_t *codes_bytes, size_t *meta_bytes);
+
+/* Quantise fp16 `x` (device, row-major `shape`) along `dim` into out->codes,
+ * out->mins, out->scales (device buffers set by the caller; their sizes from
+ * fg_qtensor_bytes).  Fills out->ndim/shape/dim/bits/group.
+ * Errors: FG_ERR_SHAPE if shape[dim] % 64 != 0; FG_ERR_UNSUPPORTED if
+ * bits != 4 or group != 64.  [G3] */
+FG_API fg_status fg_quantize(const fg_half *x, int ndim, const int64_t *shape, int dim, int bits, int group,
+                      fg_qtensor *out, void *stream);
+
+/* Dequantise q into fp16 `y` (device, row-major q->shape).  [G3] */
+FG_API fg_status fg_dequantize(const fg_qtensor *q, fg_half *y, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* 4-bit KV cache of one layer [G3]                                        */
+/* ---------------------------------------------------------------------- */
+
+/* For sequence s, head h, position p the head_dim values of k (and of v) are
+ * quantised in groups of 64 along head_dim:
+ *   k_codes  uint8 [num_seqs][num_heads][max_len][head_dim/2]
+ *   k_mins, k_scales fp16 [num_seqs][num_heads][max_len][head_dim/64]
+ * and the same for v.  Device memory, caller-owned.
+ * Requirements: head_dim in {64, 128, 256}; max_len % 64 == 0. */
+typedef struct {
+    uint8_t *k_codes;
+    fg_half *k_mins;
+    fg_half *k_scales;
+    uint8_t *v_codes;
+    fg_half *v_mins;
+    fg_half *v_scales;
+    int32_t num_seqs;
+    int32_t num_heads;
+    int32_t head_dim;
+    int32_t max_len;
+} fg_kv_cache;
+
+/* Byte sizes of one codes array and of one mins/scales array. */
+FG_API fg_status fg_kv_cache_bytes(int num_seqs, int num_heads, int head_dim, int max_len,
+                            size_t *codes_bytes, size_t *meta_bytes);
+
+/* Quantise and append new k, v rows.  k, v: fp16 device rows, row r at
+ * k + r*ld holding num_heads*head_dim values (head-major).  Row r belongs to
+ * sequence s = r / rows_per_seq and is written at position
+ * positions[s] + r % rows_per_seq (positions: int32 device [num_seqs]).
+ * rows must be a multiple of rows_per_seq.  Decode: rows_per_seq = 1;
+ * a prompt of P tokens: rows_per_seq = P, positions = start positions.
+ * A position outside [0, max_len) is skipped and flags FG_ERR_RANGE
+ * (reported by fg_sync_status).  [G3] */
+FG_API fg_status fg_kv_append(const fg_kv_cache *kv, const fg_half *k, const fg_half *v, int64_t ld,
+                       int rows, int rows_per_seq, const int32_t *positions, void *stream);
+
+/* Softmax attention of query rows over the 4-bit cache.  q: fp16 device rows
+ * (row stride ldq), already scaled by head_dim^-1/2; out: fp16 device rows
+ * (row stride ldo).  Row r (sequence s = r / rows_per_seq) attends over
+ * positions 0 .. positions[s] + r % rows_per_seq of its sequence, inclusive,
+ * reading K and V from their 4-bit form.  ([G3]; attention of OPT [OPT]) */
+FG_API fg_status fg_attention_decode(const fg_kv_cache *kv, const fg_half *q, int64_t ldq, fg_half *out, int64_t ldo,
+                              int rows, int rows_per_seq, const int32_t *positions, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* W4A16 linear layer and LayerNorm                                         */
+/* ---------------------------------------------------------------------- */
+
+enum {
+    FG_EPI_RELU = 1,      /* y = max(0, .) after the bias (and q-scale) */
+    FG_EPI_RESIDUAL = 2,  /* y += residual[m][n] after the activation */
+};
+
+/* y[m][n] = epi( sum_k x[m][k] * deq(w)[n][k] + bias[n] ), fp32 accumulation,
+ * fp16 output.  x: fp16 device [M][K]; w: packed along K, shape [N][K]
+ * (PyTorch Linear orientation); bias: fp16 [N] or NULL; residual: fp16 [M][N]
+ * (with FG_EPI_RESIDUAL); the first qscale_cols outputs of each row are
+ * multiplied by qscale after the bias.  K % 64 == 0, N % 128 == 0.
+ * workspace: device scratch of fg_linear_workspace_bytes(M, N, K) bytes
+ * (split-K partial sums and tile counters; may be NULL when that is 0).
+ * Tensor cores dequantise W tiles in shared memory ([G3]: on-the-fly
+ * dequantisation for FP16 compute). */
+FG_API size_t fg_linear_workspace_bytes(int M, int N, int K);
+FG_API fg_status fg_linear_w4a16(const fg_half *x, int M, int K, const fg_qtensor *w, const fg_half *bias,
+                          const fg_half *residual, int flags, int qscale_cols, float qscale,
+                          fg_half *y, void *workspace, size_t workspace_bytes, void *stream);
+
+/* y = (x - mean) / sqrt(var + eps) * gamma + beta per row (fp32 statistics,
+ * biased variance), fp16 in/out, gamma/beta fp16 [h] (NULL = 1 / 0).
+ * h % 8 == 0.  [OPT] */
+FG_API fg_status fg_layernorm(const fg_half *x, int M, int h, const fg_half *gamma, const fg_half *beta,
+                       float eps, fg_half *y, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* One OPT decoder layer over a block of GPU batches [G2][G3][OPT]         */
+/* ---------------------------------------------------------------------- */
+
+typedef struct {
+    int32_t hidden;     /* h = num_heads * head_dim, multiple of 128 */
+    int32_t num_heads;
+    int32_t head_dim;   /* 64, 128 or 256 */
+    int32_t ffn;        /* F, multiple of 128 */
+    float ln_eps;       /* 1e-5 for OPT */
+} fg_layer_config;
+
+/* Compressed weights of one layer.  Matrices are packed along their input
+ * dim (dim 1): wqkv [3h][h] (rows: q, then k, then v, each head-major),
+ * wo [h][h], w1 [F][h], w2 [h][F].  Vectors fp16: bqkv [3h], bo [h], b1 [F],
+ * b2 [h], ln1_g/ln1_b/ln2_g/ln2_b [h].  All device pointers. */
+typedef struct {
+    fg_qtensor wqkv, wo, w1, w2;
+    fg_half *bqkv, *bo, *b1, *b2;
+    fg_half *ln1_g, *ln1_b, *ln2_g, *ln2_b;
+} fg_layer_weights;
+
+/* Size of one layer's contiguous weight blob (every array at a 256-byte
+ * aligned offset), so a layer moves host->device with one copy [G1]. */
+FG_API size_t fg_layer_blob_bytes(const fg_layer_config *c);
+
+/* Points `out` into a blob of fg_layer_blob_bytes(c) bytes at `blob`
+ * (any memory; no data is touched). */
+FG_API fg_status fg_layer_weights_from_blob(const fg_layer_config *c, void *blob, fg_layer_weights *out);
+
+/* Device scratch needed by fg_layer_decode / fg_layer_prefill for `rows`
+ * hidden-state rows (the block's sequences, or sequences * prompt length). */
+FG_API size_t fg_layer_workspace_bytes(const fg_layer_config *c, int rows);
+
+/* One decode step of one layer for every sequence of a block of
+ * num_gpu_batches * gpu_batch_size sequences (batch j = rows
+ * [j*gpu_batch_size, (j+1)*gpu_batch_size)).  The layer's weights are loaded
+ * once and reused by all batches of the block [G2]: each GEMM runs over all
+ * the block's rows, so the result of a row does not depend on the batch split.
+ *   x_in, x_out: fp16 device [S][h] (S = num_gpu_batches * gpu_batch_size)
+ *   positions: int32 device [S], the cache position of the new token of each
+ *              sequence (= number of tokens already cached).
+ * Steps: a = LN1(x); [q k v] = a Wqkv^T + bqkv, q *= head_dim^-1/2;
+ * append k, v to the 4-bit cache at positions; o = attention over positions
+ * 0..pos; h1 = x + o Wo^T + bo; x_out = h1 + relu(LN2(h1) W1^T + b1) W2^T + b2.
+ * kv->num_seqs must equal S.  Positions are not advanced by the call. */
+FG_API fg_status fg_layer_decode(const fg_layer_config *c, const fg_layer_weights *w, const fg_kv_cache *kv,
+                          const fg_half *x_in, fg_half *x_out, const int32_t *positions,
+                          int num_gpu_batches, int gpu_batch_size,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/* The same layer over a prompt of prompt_len tokens per sequence:
+ * x_in, x_out fp16 device [S][prompt_len][h]; token t of sequence s is
+ * appended at positions[s] + t and attends over 0 .. positions[s] + t. */
+FG_API fg_status fg_layer_prefill(const fg_layer_config *c, const fg_layer_weights *w, const fg_kv_cache *kv,
+                           const fg_half *x_in, fg_half *x_out, const int32_t *positions, int prompt_len,
+                           int num_gpu_batches, int gpu_batch_size,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* Per-kernel timing of layer calls.  While enabled, each kernel that
+ * fg_layer_decode / fg_layer_prefill launch is bracketed by CUDA events on
+ * the call's stream (no synchronisation added).  fg_profile_collect waits for
+ * those events and writes, per kernel slot, the summed milliseconds and the
+ * number of launches, then forgets them.  Slots: 0 LN1, 1 QKV GEMM, 2 KV
+ * append, 3 attention, 4 out-proj GEMM, 5 LN2, 6 FC1 GEMM, 7 FC2 GEMM. */
+#define FG_PROFILE_SLOTS 8
+FG_API fg_status fg_profile_enable(int enable);
+FG_API fg_status fg_profile_collect(float *ms, int *count, int nslots);
+
+/* ---------------------------------------------------------------------- */
+/* Layer stack with weights streamed from pinned host memory [G1][G2]      */
+/* ---------------------------------------------------------------------- */
+
+typedef struct fg_stack fg_stack;  /* opaque */
+
+/* Prepares a stack of num_layers layers whose blobs live in host memory
+ * (host_blobs[l], fg_layer_blob_bytes(c) each; pinned for overlap).
+ * dev_staging[0..1]: two device buffers of fg_layer_blob_bytes(c) bytes that
+ * the next layer is prefetched into while the current one computes.
+ * Creates CUDA events only (no memory allocation).  *out is released with
+ * fg_stack_destroy. */
+FG_API fg_status fg_stack_create(const fg_layer_config *c, int num_layers, void *const *host_blobs,
+                          void *dev_staging0, void *dev_staging1, fg_stack **out);
+
+/* One decode step through all layers: layer l computes on compute_stream
+ * from staging buffer l%2 while copy_stream copies layer l+1's blob into the
+ * other buffer (events order the two).  kv: array of num_layers caches.
+ * x_in/x_out/positions/block as fg_layer_decode; x_in and x_out may alias. */
+FG_API fg_status fg_stack_decode(fg_stack *st, const fg_kv_cache *kv, const fg_half *x_in, fg_half *x_out,
+                          const int32_t *positions, int num_gpu_batches, int gpu_batch_size,
+                          void *workspace, size_t workspace_bytes, void *compute_stream, void *copy_stream);
+
+/* As fg_stack_decode for a prompt (see fg_layer_prefill). */
+FG_API fg_status fg_stack_prefill(fg_stack *st, const fg_kv_cache *kv, const fg_half *x_in, fg_half *x_out,
+                           const int32_t *positions, int prompt_len, int num_gpu_batches, int gpu_batch_size,
+                           void *workspace, size_t workspace_bytes, void *compute_stream, void *copy_stream);
+
+/* Test hook: the next `count` blob copies of this stack report a copy
+ * failure (no copy is issued), as if cudaMemcpyAsync had failed. */
+FG_API fg_status fg_stack_inject_copy_failure(fg_stack *st, int count);
+
+FG_API fg_status fg_stack_destroy(fg_stack *st);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FG_H_ */

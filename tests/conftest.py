@@ -19,3 +19,14 @@ GOLDEN = os.path.join(ROOT, "tests", "golden")
 @pytest.fixture(scope="session")
 def golden_dir():
     return GOLDEN
+
+
+@pytest.fixture(scope="session")
+def fg_lib():
+    """The CUDA library's binding; raises if the library is missing (no CPU path)."""
+    import torch
+
+    import bit_compressed_decode_b200 as m
+    if not torch.cuda.is_available():
+        raise RuntimeError("GPU tests need a CUDA device")
+    return m

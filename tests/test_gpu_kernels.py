@@ -1,0 +1,269 @@
+"""GPU parity of the individual kernels against the CPU oracle (through the C ABI).
+
+Bit-exact: quantise (codes, mins, scales), dequantise, KV append.
+Tolerance (floating point): attention, W4A16 linear, LayerNorm -- the fp16
+output rounding (2^-11 relative) plus fp32 accumulation, checked as
+max|gpu - oracle| <= tol * max|oracle|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import seeded_inputs as si
+
+pytestmark = pytest.mark.gpu
+
+fg = None
+
+
+@pytest.fixture(autouse=True)
+def _bind_library(fg_lib):
+    global fg
+    fg = fg_lib
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    return t.cpu().numpy()
+
+
+def u16(a):
+    return np.ascontiguousarray(a).view(np.uint16)
+
+
+# ------------------------------------------------------------------ quantise ----------
+
+def _check_quant_equal(x16, dim=-1):
+    q = fg.fg_quantize(dev(x16), dim=dim)
+    r = oracle.quantize(x16, dim=dim)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(q.codes), r.codes)
+    assert np.array_equal(u16(host(q.mins)), u16(r.mins))
+    assert np.array_equal(u16(host(q.scales)), u16(r.scales))
+    y = fg.fg_dequantize(q)
+    assert np.array_equal(u16(host(y)), u16(oracle.dequantize(r)))
+    return q
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 64), (3, 128), (17, 4096), (256, 4096), (5, 768 * 4)])
+def test_quantize_lastdim_bit_exact(rows, cols):
+    _check_quant_equal(si.sweep_tensor(7, rows * cols, row=cols) if cols % 64 == 0 and rows * cols >= 128
+                       else si.normal_f16(7, 1, (rows, cols), 0.02))
+
+
+def test_quantize_sweep_2pow20_bit_exact():
+    _check_quant_equal(si.sweep_tensor(0, 1 << 20, row=4096))
+
+
+def test_quantize_wide_ranges_and_specials():
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((2048, 64)) * 10.0 ** rng.integers(-7, 4, (2048, 1))).astype(np.float16)
+    x[0] = 0
+    x[1] = -0.0
+    x[2] = np.where(np.arange(64) % 3 == 0, np.float16(-0.0), np.float16(0.0))
+    x[3] = 65504
+    x[4, :32] = -65504
+    x[4, 32:] = 65504
+    x[5] = np.arange(64)
+    _check_quant_equal(x)
+
+
+@pytest.mark.parametrize("shape,dim", [((6, 128, 5), 1), ((64, 3), 0), ((2, 3, 192, 4), 2)])
+def test_quantize_strided_dims_bit_exact(shape, dim):
+    _check_quant_equal(si.normal_f16(8, 2, shape, 1.0), dim=dim)
+
+
+def test_quantize_empty_and_errors():
+    x = torch.empty((0, 64), dtype=torch.float16, device="cuda")
+    q = fg.fg_quantize(x)
+    assert q.codes.numel() == 0
+    with pytest.raises(fg.FgError, match="SHAPE"):
+        fg.fg_quantize(torch.zeros((2, 96), dtype=torch.float16, device="cuda"))
+    with pytest.raises(fg.FgError, match="UNSUPPORTED"):
+        fg.fg_quantize(torch.zeros((2, 64), dtype=torch.float16, device="cuda"), bits=8)
+
+
+@pytest.mark.slow
+def test_quantize_2pow30_sampled_bit_exact():
+    # full-size sweep point, in the launch the benchmark times; sampled groups checked by the oracle
+    n = 1 << 30
+    x = si.sweep_tensor(0, n, row=4096)
+    q = fg.fg_quantize(dev(x))
+    torch.cuda.synchronize()
+    G = n // 64
+    rng = np.random.default_rng(1)
+    sel = np.unique(np.concatenate([[0, 1, 2, G - 1], rng.integers(0, G, 20000)]))
+    xs = x.reshape(-1, 64)[sel]
+    r = oracle.quantize(xs)
+    codes = q.codes.view(-1, 32)[torch.from_numpy(sel).cuda()].cpu().numpy()
+    assert np.array_equal(codes, r.codes)
+    assert np.array_equal(u16(q.mins.view(-1)[torch.from_numpy(sel).cuda()].cpu().numpy()), u16(r.mins[:, 0]))
+    assert np.array_equal(u16(q.scales.view(-1)[torch.from_numpy(sel).cuda()].cpu().numpy()), u16(r.scales[:, 0]))
+    y = fg.fg_dequantize(q).view(-1, 64)[torch.from_numpy(sel).cuda()].cpu().numpy()
+    assert np.array_equal(u16(y), u16(oracle.dequantize(r)))
+
+
+# ------------------------------------------------------------------ KV append ---------
+
+@pytest.mark.parametrize("H,d", [(2, 64), (3, 128), (1, 256)])
+def test_kv_append_bit_exact(H, d):
+    S, maxL = 5, 128
+    g = fg.KVCache(S, H, d, maxL)
+    o = oracle.KVCache(S, H, d, maxL)
+    pos = np.array([0, 7, 63, 64, 127], dtype=np.int32)
+    k = si.normal_f16(9, 1, (S, 3 * H * d), 1.0)      # rows with a stride, like the QKV buffer
+    kk, vv = k[:, H * d:2 * H * d], k[:, 2 * H * d:]
+    kd = dev(k)
+    fg.fg_kv_append(g, kd[:, H * d:], kd[:, 2 * H * d:], dev(pos), ld=3 * H * d)
+    oracle.kv_append(o, kk, vv, np.arange(S), pos)
+    fg.fg_sync_status()
+    for a, b in zip(g.arrays(), o.arrays()):
+        assert np.array_equal(u16(host(a)) if a.dtype == torch.float16 else host(a), b)
+
+
+def test_kv_append_prompt_rows_and_range_error():
+    S, H, d, maxL, P = 3, 2, 128, 64, 10
+    g = fg.KVCache(S, H, d, maxL)
+    o = oracle.KVCache(S, H, d, maxL)
+    k = si.normal_f16(10, 1, (S * P, H * d), 1.0)
+    v = si.normal_f16(10, 2, (S * P, H * d), 1.0)
+    start = np.array([0, 5, 58], dtype=np.int32)        # the last sequence runs past max_len (58+9 > 63)
+    fg.fg_kv_append(g, dev(k), dev(v), dev(start), rows_per_seq=P)
+    with pytest.raises(fg.FgError, match="RANGE"):
+        fg.fg_sync_status()
+    fg.fg_sync_status()                                  # the error word was cleared
+    seq = np.repeat(np.arange(S), P)
+    pos = start[seq] + np.tile(np.arange(P), S)
+    ok = pos < maxL
+    oracle.kv_append(o, k[ok], v[ok], seq[ok], pos[ok])
+    for a, b in zip(g.arrays(), o.arrays()):
+        assert np.array_equal(u16(host(a)) if a.dtype == torch.float16 else host(a), b)
+
+
+# ------------------------------------------------------------------ attention ---------
+
+def _cache_pair(S, H, d, maxL, lens, seed):
+    o = oracle.KVCache(S, H, d, maxL)
+    for s in range(S):
+        L = lens[s]
+        k = si.normal_f16(seed, 100 + s, (L, H * d), 1.0)
+        v = si.normal_f16(seed, 200 + s, (L, H * d), 1.0)
+        oracle.kv_append(o, k, v, np.full(L, s), np.arange(L))
+    arrays = [dev(a.view(np.float16) if a.dtype == np.uint16 else a) for a in o.arrays()]
+    return o, fg.KVCache(S, H, d, maxL, arrays=arrays)
+
+
+@pytest.mark.parametrize("H,d", [(4, 64), (3, 128), (2, 256)])
+def test_attention_decode_matches_oracle(H, d):
+    S, maxL = 6, 320
+    lens = np.array([1, 2, 63, 64, 65, 300], dtype=np.int32)   # ragged: 1 token, chunk edges, several chunks
+    o, g = _cache_pair(S, H, d, maxL, lens, seed=11)
+    q = (si.normal_f16(11, 1, (S, H * d), 1.0).astype(np.float32) / np.sqrt(d)).astype(np.float16)
+    out = fg.fg_attention_decode(g, dev(q), dev(lens - 1))
+    ref = oracle.attention(o, q, np.arange(S), lens)
+    got = host(out).astype(np.float64)
+    for s in range(S):
+        for h in range(H):
+            sl = slice(h * d, (h + 1) * d)
+            err = np.max(np.abs(got[s, sl] - ref[s, sl]))
+            assert err <= 2e-3 * np.max(np.abs(ref[s, sl])) + 1e-4, (s, h, err)
+
+
+def test_attention_peaked_scores():
+    # large query norms make the softmax nearly one-hot: catches masking and max handling
+    S, H, d, maxL = 2, 2, 128, 256
+    lens = np.array([130, 200], dtype=np.int32)
+    o, g = _cache_pair(S, H, d, maxL, lens, seed=12)
+    q = si.normal_f16(12, 1, (S, H * d), 3.0)
+    out = fg.fg_attention_decode(g, dev(q), dev(lens - 1))
+    ref = oracle.attention(o, q, np.arange(S), lens)
+    assert np.max(np.abs(host(out).astype(np.float64) - ref)) <= 5e-3 * np.max(np.abs(ref))
+
+
+def test_attention_prompt_rows_causal():
+    S, H, d, maxL, P = 2, 2, 128, 128, 70
+    lens = np.array([P, P], dtype=np.int32)
+    o, g = _cache_pair(S, H, d, maxL, lens, seed=13)
+    q = (si.normal_f16(13, 1, (S * P, H * d), 1.0).astype(np.float32) / np.sqrt(d)).astype(np.float16)
+    out = fg.fg_attention_decode(g, dev(q), dev(np.zeros(S, np.int32)), rows_per_seq=P)
+    seq = np.repeat(np.arange(S), P)
+    ref = oracle.attention(o, q, seq, np.tile(np.arange(P), S) + 1)
+    assert np.max(np.abs(host(out).astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref))
+
+
+# ------------------------------------------------------------------ linear -------------
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 64), (4, 256, 768), (16, 384, 128), (17, 256, 192), (100, 512, 1024),
+                                   (256, 768, 768), (300, 1280, 512), (512, 2304, 768), (40, 768, 3072)])
+def test_linear_matches_oracle(M, N, K):
+    x = si.normal_f16(14, 1, (M, K), 1.0)
+    w16 = si.normal_f16(14, 2, (N, K), 0.02)
+    b = si.normal_f16(14, 3, (N,), 0.1)
+    wq = fg.fg_quantize(dev(w16), dim=1)
+    y = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b))
+    ref = oracle.linear(x, oracle.quantize(w16, 1), bias=b)
+    err = np.max(np.abs(host(y).astype(np.float64) - ref))
+    assert err <= 2e-3 * np.max(np.abs(ref)), err
+
+
+def test_linear_epilogues():
+    M, N, K = 70, 512, 256
+    x = si.normal_f16(15, 1, (M, K), 1.0)
+    w16 = si.normal_f16(15, 2, (N, K), 0.05)
+    b = si.normal_f16(15, 3, (N,), 0.1)
+    r = si.normal_f16(15, 4, (M, N), 1.0)
+    wq = fg.fg_quantize(dev(w16), dim=1)
+    wo = oracle.quantize(w16, 1)
+    for kw, okw in [(dict(relu=True), dict(relu=True)), (dict(residual=dev(r)), dict(residual=r)),
+                    (dict(qscale_cols=128, qscale=0.125), dict(qscale_cols=128, qscale=0.125))]:
+        y = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), **kw)
+        ref = oracle.linear(x, wo, bias=b, **okw)
+        assert np.max(np.abs(host(y).astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref)), kw
+
+
+def test_linear_permutation_weight_exact():
+    # weights {0, 15} per group are stored exactly; y = 15 * x[:, cols] + b up to the fp16 output rounding
+    M, N, K = 33, 256, 512
+    cols = np.random.default_rng(2).integers(0, K, N)
+    w16 = np.zeros((N, K), np.float16)
+    w16[np.arange(N), cols] = 15
+    x = si.normal_f16(16, 1, (M, K), 1.0)
+    y = fg.fg_linear_w4a16(dev(x), fg.fg_quantize(dev(w16), dim=1))
+    assert np.array_equal(host(y), (15.0 * x.astype(np.float64)[:, cols]).astype(np.float16))
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 256, 8192), (512, 4096, 4096), (40, 384, 16384)])
+def test_linear_split_k_deterministic(M, N, K):
+    # few output tiles and a long k-range take the cluster split-k path; two runs give identical bits
+    x = dev(si.normal_f16(17, 1, (M, K), 1.0))
+    w16 = si.normal_f16(17, 2, (N, K), 0.02)
+    wq = fg.fg_quantize(dev(w16), dim=1)
+    assert fg.fg_linear_workspace_bytes(M, N, K) == 0       # partial sums stay on chip
+    y1 = fg.fg_linear_w4a16(x, wq)
+    y2 = fg.fg_linear_w4a16(x, wq)
+    assert torch.equal(y1, y2)
+    ref = oracle.linear(host(x), oracle.quantize(w16, 1))
+    assert np.max(np.abs(host(y1).astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref))
+
+
+def test_linear_errors():
+    x = torch.zeros((4, 64), dtype=torch.float16, device="cuda")
+    w = fg.fg_quantize(torch.zeros((64, 64), dtype=torch.float16, device="cuda"), dim=1)
+    with pytest.raises(fg.FgError, match="SHAPE"):
+        fg.fg_linear_w4a16(x, w)                             # N = 64 is not a multiple of 128
+
+
+# ------------------------------------------------------------------ layernorm ----------
+
+@pytest.mark.parametrize("M,h", [(1, 768), (7, 4096), (3, 12288), (5, 64)])
+def test_layernorm_matches_oracle(M, h):
+    x = si.normal_f16(18, 1, (M, h), 1.0)
+    g = (1 + si.normal_f16(18, 2, (h,), 0.1).astype(np.float32)).astype(np.float16)
+    b = si.normal_f16(18, 3, (h,), 0.1)
+    y = fg.fg_layernorm(dev(x), dev(g), dev(b))
+    ref = oracle.layernorm(x, g, b)
+    assert np.max(np.abs(host(y).astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref))
