@@ -83,6 +83,8 @@ _decl("fg_layer_decode", c_int, POINTER(fg_layer_config), POINTER(fg_layer_weigh
       c_int, c_int, P, c_size_t, P)
 _decl("fg_layer_prefill", c_int, POINTER(fg_layer_config), POINTER(fg_layer_weights), POINTER(fg_kv_cache), P, P, P,
       c_int, c_int, c_int, P, c_size_t, P)
+_decl("fg_layer_decode_noalloc", c_int, POINTER(fg_layer_config), POINTER(fg_layer_weights), POINTER(fg_kv_cache),
+      P, P, P, c_int, c_int, P)
 _decl("fg_profile_enable", c_int, c_int)
 _decl("fg_profile_collect", c_int, POINTER(c_float), POINTER(c_int), c_int)
 _decl("fg_stack_create", c_int, POINTER(fg_layer_config), c_int, POINTER(c_void_p), P, P, POINTER(c_void_p))
@@ -370,6 +372,27 @@ def fg_layer_decode(cfg: LayerConfig, w: LayerWeights, cache: KVCache, x: torch.
     _check(_lib.fg_layer_decode(ctypes.byref(c), ctypes.byref(ws), ctypes.byref(kv), _ptr(x), _ptr(out),
                                 _ptr(positions), num_gpu_batches, gpu_batch_size, _ptr(workspace),
                                 workspace.numel(), _stream(stream)), "fg_layer_decode")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 48 << 20
+
+
+def fg_layer_decode_noalloc(cfg: LayerConfig, w: LayerWeights, cache: KVCache, x: torch.Tensor,
+                            positions: torch.Tensor, num_gpu_batches: int = 1, gpu_batch_size: int | None = None,
+                            out=None, stream=None):
+    """fg_layer_decode with the library's static scratch instead of a caller workspace."""
+    S = x.shape[0]
+    if gpu_batch_size is None:
+        gpu_batch_size = S // num_gpu_batches
+    if out is None:
+        out = torch.empty_like(x)
+    c = cfg.struct()
+    ws = w.struct()
+    kv = cache.struct()
+    _check(_lib.fg_layer_decode_noalloc(ctypes.byref(c), ctypes.byref(ws), ctypes.byref(kv), _ptr(x), _ptr(out),
+                                        _ptr(positions), num_gpu_batches, gpu_batch_size, _stream(stream)),
+           "fg_layer_decode_noalloc")
     return out
 
 

@@ -246,6 +246,30 @@ FG_API fg_status fg_layer_prefill(const fg_layer_config *c, const fg_layer_weigh
                            int num_gpu_batches, int gpu_batch_size,
                            void *workspace, size_t workspace_bytes, void *stream);
 
+/* fg_layer_decode for callers that cannot allocate device memory -- a serving
+ * process that reserved all device memory up front, a host that only passes
+ * pointers it already owns, or a loop that must not allocate between steps.
+ * (The pages have no counterpart: this is a deployment convenience.)  The step's
+ * scratch lives in a static device array of FG_NOALLOC_SCRATCH_BYTES that every
+ * GPU loading the library holds until the process exits; the caller still
+ * passes weights, cache, inputs and outputs, as for fg_layer_decode, whose
+ * computation this is.
+ *   - Returns FG_ERR_WORKSPACE when the block needs more scratch than that
+ *     (fg_layer_workspace_bytes(c, S) > FG_NOALLOC_SCRATCH_BYTES), before any
+ *     launch.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents;
+ *     nothing in it has to start at zero (each step writes what it reads).
+ *     Calls whose work overlaps on the GPU (other streams, other threads)
+ *     race on it: serialise them.
+ *   - Allocates nothing (keep fg_profile_enable off: profiling creates events). */
+#define FG_NOALLOC_SCRATCH_BYTES (48u << 20)
+FG_API fg_status fg_layer_decode_noalloc(const fg_layer_config *c, const fg_layer_weights *w,
+                                         const fg_kv_cache *kv, const fg_half *x_in, fg_half *x_out,
+                                         const int32_t *positions, int num_gpu_batches, int gpu_batch_size,
+                                         void *stream);
+
 /* Per-kernel timing of layer calls.  While enabled, each kernel that
  * fg_layer_decode / fg_layer_prefill launch is bracketed by CUDA events on
  * the call's stream (no synchronisation added).  fg_profile_collect waits for
