@@ -210,22 +210,20 @@ def run_ours(args, wl):
 
     import bit_compressed_decode_b200 as fg
     import seeded_inputs as si
+    from bit_compressed_decode_b200 import replicas
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = replicas.env_ranks()
     if world > 1:
-        import datetime
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        replicas.init("nccl", timeout_s=300, device=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
 
     h, H, F, P = wl["hidden"], wl["heads"], wl["ffn"], wl["prompt"]
     nb, gbs = wl["nb"], wl["gbs"]
-    S = nb * gbs
+    S = nb * gbs                      # sequences of this rank: its block
+    seq0, _ = replicas.shard(world * S, world, rank)
     d = h // H
     nsteps_cfg = wl["steps"]
     maxL = (P + nsteps_cfg + 63) // 64 * 64
@@ -238,7 +236,7 @@ def run_ours(args, wl):
     cache = fg.KVCache(S, H, d, maxL, device=dev)
     # prompt hidden states: seeded device generator (bulk synthetic N(0,1)), per rank
     g = torch.Generator(device=dev)
-    g.manual_seed(1000 + rank)
+    g.manual_seed(1000 + seq0)
     zero = torch.zeros(S, dtype=torch.int32, device=dev)
     chunk = max(1, 65536 // P)
     pws = torch.empty(cfg.workspace_bytes(chunk * P), dtype=torch.uint8, device=dev)
@@ -287,11 +285,7 @@ def run_ours(args, wl):
     clocks = sampler.stop()
     prof = fg.fg_profile_collect()
     fg.fg_sync_status()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = replicas.max_over_ranks(e0.elapsed_time(e1), device=dev)
     ms_per_step = ms / args.steps
     value = world * S * args.steps / (ms / 1e3)
 
@@ -315,11 +309,7 @@ def run_ours(args, wl):
     f1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ems = f0.elapsed_time(f1)
-    if world > 1:
-        t = torch.tensor([ems], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ems = float(t.item())
+    ems = replicas.max_over_ranks(f0.elapsed_time(f1), device=dev)
     e2e_value = world * S * args.steps / (ems / 1e3)
     h2d = S * h * 2 + S * 4
     d2h = S * h * 2

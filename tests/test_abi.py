@@ -1,0 +1,156 @@
+"""The C ABI library loads, exports every symbol include/fg.h declares, and validates
+arguments on the host (CPU only: no call here reaches a CUDA launch)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import bit_compressed_decode_b200 as fg
+from bit_compressed_decode_b200 import _binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fg.h")
+
+
+def declared():
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"FG_API\s+[\w\s\*]*?\b(fg_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared()
+    for must in ("fg_quantize", "fg_dequantize", "fg_kv_append", "fg_layer_decode", "fg_layer_prefill",
+                 "fg_attention_decode", "fg_linear_w4a16", "fg_sync_status", "fg_stack_decode",
+                 "fg_layer_decode_noalloc"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", fg.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (fg_\w+)", out))
+    missing = [n for n in declared() if n not in exported]
+    assert not missing, missing
+    for n in declared():
+        assert hasattr(B.lib(), n)
+
+
+def test_status_strings():
+    for code, name in B.STATUS.items():
+        assert fg.fg_status_string(code) == name
+    assert fg.fg_status_string(99) == "FG_ERR_UNKNOWN"
+
+
+def _rc(fn, *args):
+    return getattr(B.lib(), fn)(*args)
+
+
+def test_qtensor_bytes_and_errors():
+    assert fg.fg_qtensor_bytes((8, 4096)) == (8 * 4096 // 2, 8 * 4096 // 64 * 2)
+    assert fg.fg_qtensor_bytes((6, 128, 5), dim=1) == (6 * 128 * 5 // 2, 6 * 2 * 5 * 2)
+    with pytest.raises(fg.FgError, match="SHAPE"):
+        fg.fg_qtensor_bytes((8, 96))
+    with pytest.raises(fg.FgError, match="UNSUPPORTED"):
+        fg.fg_qtensor_bytes((8, 64), bits=8)
+    with pytest.raises(fg.FgError, match="UNSUPPORTED"):
+        fg.fg_qtensor_bytes((8, 128), group=128)
+    with pytest.raises(fg.FgError, match="INVALID"):
+        fg.fg_qtensor_bytes((1, 2, 3, 4, 64))
+
+
+def test_quantize_validates_before_launch():
+    q = B.fg_qtensor()
+    shape = (ctypes.c_int64 * 2)(4, 96)
+    assert _rc("fg_quantize", None, 2, shape, 1, 4, 64, ctypes.byref(q), None) == 2   # SHAPE
+    shape = (ctypes.c_int64 * 2)(4, 64)
+    assert _rc("fg_quantize", None, 2, shape, 1, 4, 64, ctypes.byref(q), None) == 1   # null buffers
+    assert _rc("fg_quantize", None, 2, shape, 1, 4, 64, None, None) == 1
+    misaligned = ctypes.c_void_p(0x1008)
+    q.codes, q.mins, q.scales = 0x1000, 0x2000, 0x3000
+    assert _rc("fg_quantize", misaligned, 2, shape, 1, 4, 64, ctypes.byref(q), None) == 1
+
+
+def test_kv_cache_bytes_rules():
+    cb, mb = ctypes.c_size_t(), ctypes.c_size_t()
+    assert _rc("fg_kv_cache_bytes", 512, 32, 128, 576, ctypes.byref(cb), ctypes.byref(mb)) == 0
+    assert cb.value == 512 * 32 * 576 * 64 and mb.value == 512 * 32 * 576 * 2 * 2
+    assert _rc("fg_kv_cache_bytes", 4, 12, 96, 64, ctypes.byref(cb), ctypes.byref(mb)) == 3     # head_dim
+    assert _rc("fg_kv_cache_bytes", 4, 12, 64, 100, ctypes.byref(cb), ctypes.byref(mb)) == 2    # max_len % 64
+
+
+def _align(x, a=256):
+    return (x + a - 1) // a * a
+
+
+@pytest.mark.parametrize("h,H,F", [(768, 12, 3072), (4096, 32, 16384), (7168, 56, 28672), (12288, 96, 49152)])
+def test_layer_blob_layout(h, H, F):
+    cfg = fg.LayerConfig(h, H, F)
+    # the blob holds 4 packed matrices (codes n*k/2, mins and scales n*k/64*2 each) and
+    # 8 fp16 vectors, every array 256-byte aligned
+    want = 0
+    for n, k in ((3 * h, h), (h, h), (F, h), (h, F)):
+        want += _align(n * k // 2) + 2 * _align(n * k // 64 * 2)
+    for n in (3 * h, h, F, h, h, h, h, h):
+        want += _align(2 * n)
+    assert cfg.blob_bytes() == want
+    blob = np.zeros(want + 256, dtype=np.uint8)
+    base = (blob.ctypes.data + 255) // 256 * 256
+    w = B.fg_layer_weights()
+    c = cfg.struct()
+    assert _rc("fg_layer_weights_from_blob", ctypes.byref(c), ctypes.c_void_p(base), ctypes.byref(w)) == 0
+    spans = []
+    for name, (n, k) in zip(("wqkv", "wo", "w1", "w2"), ((3 * h, h), (h, h), (F, h), (h, F))):
+        t = getattr(w, name)
+        assert (t.shape[0], t.shape[1], t.dim, t.bits, t.group) == (n, k, 1, 4, 64)
+        spans += [(t.codes, n * k // 2), (t.mins, n * k // 32), (t.scales, n * k // 32)]
+    for name, n in zip(("bqkv", "bo", "b1", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b"),
+                       (3 * h, h, F, h, h, h, h, h)):
+        spans.append((getattr(w, name), 2 * n))
+    spans.sort()
+    for (p, nbytes), (q, _) in zip(spans, spans[1:]):
+        assert p % 256 == 0 and p + nbytes <= q
+    assert spans[-1][0] + spans[-1][1] <= base + want
+
+
+def test_opt6p7b_sizes():
+    cfg = fg.LayerConfig(4096, 32, 16384)
+    # 12 h^2 parameters at 4.5 bits (codes + fp16 min and scale per 64): 113.2 MB + vectors
+    assert abs(cfg.blob_bytes() - 12 * 4096 ** 2 * (0.5 + 4 / 64)) < 0.2e6
+    # scratch per decode step: a, o, h1 [S,h] + qkv [S,3h] + ffn [S,F] in fp16
+    assert cfg.workspace_bytes(512) == 512 * (6 * 4096 + 16384) * 2
+    assert fg.fg_linear_workspace_bytes(512, 12288, 4096) == 0
+
+
+def test_layer_entry_points_validate_config():
+    bad = B.fg_layer_config(4096, 32, 100, 16384, 1e-5)     # head_dim inconsistent
+    assert B.lib().fg_layer_blob_bytes(ctypes.byref(bad)) == 0
+    w = B.fg_layer_weights()
+    kv = B.fg_kv_cache()
+    rc = _rc("fg_layer_decode", ctypes.byref(bad), ctypes.byref(w), ctypes.byref(kv), None, None, None, 1, 1, None,
+             0, None)
+    assert rc == 3
+
+
+def test_noalloc_rejects_oversized_block_on_host():
+    cfg = fg.LayerConfig(4096, 32, 16384)
+    c = cfg.struct()
+    w = B.fg_layer_weights()
+    kv = B.fg_kv_cache()
+    assert cfg.workspace_bytes(1024) > fg.NOALLOC_SCRATCH_BYTES
+    rc = _rc("fg_layer_decode_noalloc", ctypes.byref(c), ctypes.byref(w), ctypes.byref(kv), None, None, None, 1,
+             1024, None)
+    assert rc == 7                                          # FG_ERR_WORKSPACE, before any CUDA call
+
+
+def test_stack_create_validates():
+    cfg = fg.LayerConfig(768, 12, 3072)
+    c = cfg.struct()
+    h = ctypes.c_void_p()
+    blobs = (ctypes.c_void_p * 2)(None, None)
+    assert _rc("fg_stack_create", ctypes.byref(c), 2, blobs, ctypes.c_void_p(256), ctypes.c_void_p(512),
+               ctypes.byref(h)) == 1
+    assert _rc("fg_stack_create", ctypes.byref(c), 0, blobs, ctypes.c_void_p(256), ctypes.c_void_p(512),
+               ctypes.byref(h)) == 1
