@@ -370,6 +370,72 @@ def run_ours(args, wl):
         dist.destroy_process_group()
 
 
+def run_kernel(args, wl):
+    """Standalone launches of one kernel of the decode step on the workload's shapes,
+    timed with CUDA events (used for per-kernel measurements and small ncu captures)."""
+    import torch
+
+    import bit_compressed_decode_b200 as fg
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    h, H, F, P = wl["hidden"], wl["heads"], wl["ffn"], wl["prompt"]
+    S = args.seqs or wl["nb"] * wl["gbs"]
+    d = h // H
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+    if args.kernel == "attention":
+        maxL = (P + wl["steps"] + 63) // 64 * 64
+        ng = d // 64
+        cache = fg.KVCache(S, H, d, maxL, device=dev, arrays=[
+            torch.randint(0, 256, (S, H, maxL, d // 2), generator=g, device=dev, dtype=torch.uint8),
+            torch.randn((S, H, maxL, ng), generator=g, device=dev, dtype=torch.float16),
+            (torch.rand((S, H, maxL, ng), generator=g, device=dev) * 0.2).half(),
+            torch.randint(0, 256, (S, H, maxL, d // 2), generator=g, device=dev, dtype=torch.uint8),
+            torch.randn((S, H, maxL, ng), generator=g, device=dev, dtype=torch.float16),
+            (torch.rand((S, H, maxL, ng), generator=g, device=dev) * 0.2).half()])
+        qkv = torch.randn((S, 3 * h), generator=g, device=dev, dtype=torch.float16) * 0.1
+        out = torch.empty((S, h), dtype=torch.float16, device=dev)
+        pos = torch.full((S,), P, dtype=torch.int32, device=dev)
+        run = lambda: fg.fg_attention_decode(cache, qkv[:, :h], pos, out=out, stream=stream)
+        work, unit, peak = S * H * (P + 1) * 2 * (d // 2 + 4 * ng) + 2 * S * h * 2, "GB/s", peaks["hbm"]
+    elif args.kernel.endswith("_gemm"):
+        N, K = {"qkv_gemm": (3 * h, h), "out_gemm": (h, h), "fc1_gemm": (F, h), "fc2_gemm": (h, F)}[args.kernel]
+        x = torch.randn((S, K), generator=g, device=dev, dtype=torch.float16)
+        wq = fg.fg_quantize(torch.randn((N, K), generator=g, device=dev, dtype=torch.float16) * 0.02, dim=1)
+        y = torch.empty((S, N), dtype=torch.float16, device=dev)
+        run = lambda: fg.fg_linear_w4a16(x, wq, out=y, stream=stream)
+        work, unit, peak = 2 * S * N * K, "TFLOP/s", peaks["tc_burst"]
+    elif args.kernel in ("quantize", "dequantize"):
+        n = 1 << args.log2_elems
+        x = torch.randn((n // 4096, 4096), generator=g, device=dev, dtype=torch.float16) * 0.02
+        q = fg.fg_quantize(x)
+        if args.kernel == "quantize":
+            run = lambda: fg.fg_quantize(x, out=q, stream=stream)
+        else:
+            run = lambda: fg.fg_dequantize(q, stream=stream)
+        work, unit, peak = n * 2.5625, "GB/s", peaks["hbm"]
+    else:
+        raise SystemExit(f"unknown kernel {args.kernel}")
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in ev:
+        a.record(stream)
+        run()
+        b.record(stream)
+    torch.cuda.synchronize()
+    fg.fg_sync_status()
+    t = sorted(a.elapsed_time(b) / 1e3 for a, b in ev)
+    med = t[len(t) // 2]
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    print(json.dumps({"kernel": args.kernel, "workload": args.workload, "seqs": S, "median_us": med * 1e6,
+                      "min_us": t[0] * 1e6, "achieved": work / med / scale, "unit": unit, "peak": peak,
+                      "frac": work / med / scale / peak}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -378,9 +444,16 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="opt-6.7b-layer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", default=None,
+                    help="time one kernel alone: attention, qkv_gemm, out_gemm, fc1_gemm, fc2_gemm, quantize, "
+                         "dequantize")
+    ap.add_argument("--seqs", type=int, default=0, help="--kernel: sequences (default: the workload's block)")
+    ap.add_argument("--log2-elems", type=int, default=28, help="--kernel quantize/dequantize: tensor size")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
-    if args.impl == "reference":
+    if args.kernel:
+        run_kernel(args, wl)
+    elif args.impl == "reference":
         run_reference(args, wl)
     else:
         run_ours(args, wl)

@@ -62,12 +62,12 @@ struct GemmArgs {
   unsigned int *err;
 };
 
-__device__ __forceinline__ float epilogue(float v, int m, int n, const GemmArgs &a) {
-  if (a.bias) v += __half2float(a.bias[n]);
+// ((acc + bias) * qscale if n < qcols) -> ReLU if set -> + residual (0 when unused).
+__device__ __forceinline__ float epilogue(float v, float bias, float res, int n, const GemmArgs &a) {
+  v += bias;
   if (n < a.qcols) v *= a.qscale;
   if (a.relu) v = fmaxf(v, 0.f);
-  if (a.res) v += __half2float(a.res[static_cast<int64_t>(m) * a.N + n]);
-  return v;
+  return v + res;
 }
 
 template <int NT>
@@ -233,15 +233,22 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
   };
   if (a.splits == 1) {
     if (warp < kDeqWarps) {
+      const float bias = (a.bias && nlive) ? __half2float(a.bias[n]) : 0.f;
       for (int ch = 0; ch < kChunks; ch++) {
         uint32_t v[32];
         load_chunk(ch, v);
-        if (!ready) continue;
+        if (!ready || !nlive) continue;
+        float res[kCW];
+#pragma unroll
+        for (int j = 0; j < kCW; j++) {  // every residual load is issued before any store
+          const int m = t0 + ch * kCW + j;
+          res[j] = (a.res && m < a.M) ? __half2float(a.res[static_cast<int64_t>(m) * a.N + n]) : 0.f;
+        }
 #pragma unroll
         for (int j = 0; j < kCW; j++) {
           const int m = t0 + ch * kCW + j;
-          if (m < a.M && nlive)
-            a.y[static_cast<int64_t>(m) * a.N + n] = __float2half_rn(epilogue(__uint_as_float(v[j]), m, n, a));
+          if (m < a.M)
+            a.y[static_cast<int64_t>(m) * a.N + n] = __float2half_rn(epilogue(__uint_as_float(v[j]), bias, res[j], n, a));
         }
       }
     }
@@ -272,6 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
       cluster_sync_all();
       if (warp < kDeqWarps && ready) {
         const int nn = n0 + feat;
+        const float rbias = (a.bias && nn < a.N) ? __half2float(a.bias[nn]) : 0.f;
         for (int i = 0; i < kRound && r0 + i < kChunks; i++) {
           const int ch = r0 + i;
           if (ch % a.splits != static_cast<int>(rank)) continue;
@@ -289,11 +297,17 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
                 for (int u = 0; u < kU; u++) sum[u] += ld_shared_cluster_f32(rb + u * kBM * 4);
               }
             }
+            float res[kU];
+#pragma unroll
+            for (int u = 0; u < kU; u++) {
+              const int m = t0 + ch * kCW + j0 + u;
+              res[u] = (a.res && m < a.M && nn < a.N) ? __half2float(a.res[static_cast<int64_t>(m) * a.N + nn]) : 0.f;
+            }
 #pragma unroll
             for (int u = 0; u < kU; u++) {
               const int m = t0 + ch * kCW + j0 + u;
               if (m < a.M && nn < a.N)
-                a.y[static_cast<int64_t>(m) * a.N + nn] = __float2half_rn(epilogue(sum[u], m, nn, a));
+                a.y[static_cast<int64_t>(m) * a.N + nn] = __float2half_rn(epilogue(sum[u], rbias, res[u], nn, a));
             }
           }
         }
