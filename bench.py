@@ -34,6 +34,9 @@ sys.path.insert(0, ROOT)
 WORKLOADS = {
     "opt-6.7b-layer": dict(hidden=4096, heads=32, ffn=16384, nb=8, gbs=64, prompt=512, steps=32),
     "opt-125m-layer": dict(hidden=768, heads=12, ffn=3072, nb=1, gbs=4, prompt=32, steps=8),
+    # OPT-30B-shaped stack: 48 layers whose W4 blobs stay in pinned host memory and are
+    # prefetched layer by layer on a side stream; KV4 caches resident in HBM
+    "opt-30b-stack": dict(hidden=7168, heads=56, ffn=28672, nb=4, gbs=64, prompt=512, steps=32, layers=48),
 }
 METRIC = "decode tokens/s per OPT layer block (W4 KV4)"
 
@@ -64,6 +67,13 @@ def kernel_work(wl, S, L_avg):
         "fc1_gemm": ("tensor", 2 * S * F * h),
         "fc2_gemm": ("tensor", 2 * S * h * F),
     }, {"w4_bytes": w4(3 * h, h) + w4(h, h) + w4(F, h) + w4(h, F), "kv_bytes_per_token": kv_tok}
+
+
+def kernel_units(wl, S, L_avg):
+    """Units one launch of each kernel processes, the scale for traffic taken on a smaller case."""
+    h, F, H = wl["hidden"], wl["ffn"], wl["heads"]
+    return {"ln1": S, "qkv_gemm": S, "kv_append": S, "attention": S * H * L_avg, "out_gemm": S, "ln2": S,
+            "fc1_gemm": S, "fc2_gemm": S}
 
 
 class ClockSampler:
@@ -184,8 +194,11 @@ def run_reference(args, wl):
 # GPU path
 # ----------------------------------------------------------------------------------------
 
-def read_traffic(kernel: str, workload: str):
-    """Per-launch DRAM bytes from a committed ncu summary, if it matches the current sources."""
+def read_traffic(kernel: str, workload: str, units: float):
+    """Per-launch DRAM bytes (read + write) from a committed ncu capture, if it was taken on the
+    current source of the kernel.  A capture of a smaller case is scaled by the units one launch
+    processes (for attention: sequence x head x context-token triples), the kernel's traffic
+    being proportional to them."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
@@ -201,7 +214,7 @@ def read_traffic(kernel: str, workload: str):
     with open(src, "rb") as f:
         if hashlib.sha256(f.read()).hexdigest()[:16] != e["source_sha"]:
             return None
-    return e["dram_bytes_per_launch"]
+    return round(e["dram_bytes_per_launch"] * units / e["units_per_launch"])
 
 
 def run_ours(args, wl):
@@ -335,7 +348,7 @@ def run_ours(args, wl):
     kd = kernels[dom]
     roofline = {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"],
                 "unit": kd["unit"], "frac": kd["frac"],
-                "traffic": read_traffic(dom, args.workload),
+                "traffic": read_traffic(dom, args.workload, kernel_units(wl, S, L_avg)[dom]),
                 "peak_source": f"{peaks['source']} ({'sustained bf16' if kd['bound'] == 'tensor' else 'copy'})"}
 
     cpu = None
@@ -368,6 +381,103 @@ def run_ours(args, wl):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_stack(args, wl):
+    """One decode step = all layers of the stack for every sequence of the block, each layer's
+    packed weights copied from pinned host memory (fg_stack_decode, double-buffered prefetch)."""
+    import torch
+
+    import bit_compressed_decode_b200 as fg
+    from bit_compressed_decode_b200 import replicas
+
+    rank, world, local = replicas.env_ranks()
+    if world > 1:
+        torch.cuda.set_device(local)
+        replicas.init("nccl", timeout_s=600, device=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    h, H, F, P, nl = wl["hidden"], wl["heads"], wl["ffn"], wl["prompt"], args.layers or wl["layers"]
+    nb, gbs = wl["nb"], wl["gbs"]
+    S, d = nb * gbs, h // H
+    maxL = (P + wl["steps"] + 63) // 64 * 64
+    cfg = fg.LayerConfig(h, H, F)
+    g = torch.Generator(device=dev)
+    g.manual_seed(2000 + rank)
+    # weights: seeded device draws N(0, 0.02) (biases 0, LayerNorm 1/0), quantised by fg_quantize,
+    # then parked in pinned host memory -- the stack streams them back every step
+    host = []
+    tmp = fg.LayerWeights(cfg, torch.empty(cfg.blob_bytes(), dtype=torch.uint8, device=dev))
+    for _ in range(nl):
+        for name, shape in (("wqkv", (3 * h, h)), ("wo", (h, h)), ("w1", (F, h)), ("w2", (h, F))):
+            w = torch.randn(shape, generator=g, device=dev, dtype=torch.float16) * 0.02
+            fg.fg_quantize(w, dim=1, out=tmp.matrix(name))
+            del w
+        for name in ("bqkv", "bo", "b1", "b2", "ln1_b", "ln2_b"):
+            tmp.vector(name).zero_()
+        tmp.vector("ln1_g").fill_(1.0)
+        tmp.vector("ln2_g").fill_(1.0)
+        hb = torch.empty(cfg.blob_bytes(), dtype=torch.uint8, pin_memory=True)
+        hb.copy_(tmp.blob)
+        host.append(hb)
+    del tmp
+    torch.cuda.synchronize()
+    st = fg.Stack(cfg, host, device=dev)
+    caches = [fg.KVCache(S, H, d, maxL, device=dev) for _ in range(nl)]
+    compute = torch.cuda.current_stream()
+    copy = torch.cuda.Stream(device=dev)
+    # prefill (untimed): the prompt through all layers, in sequence chunks
+    chunk = max(1, 32768 // P)
+    for s0 in range(0, S, chunk):
+        n = min(chunk, S - s0)
+        x = torch.randn((n, P, h), generator=g, device=dev, dtype=torch.float16)
+        st.prefill([c.view(s0, n) for c in caches], x, torch.zeros(n, dtype=torch.int32, device=dev),
+                   compute_stream=compute, copy_stream=copy)
+        del x
+    fg.fg_sync_status()
+    xs = [torch.randn((S, h), generator=g, device=dev, dtype=torch.float16) for _ in range(2)]
+    pos = [torch.full((S,), P + t, dtype=torch.int32, device=dev) for t in range(wl["steps"])]
+    out = torch.empty((S, h), dtype=torch.float16, device=dev)
+    ws = torch.empty(st.workspace_bytes(S), dtype=torch.uint8, device=dev)
+
+    def step(i):
+        st.decode(caches, xs[i % 2], pos[i % wl["steps"]], num_gpu_batches=nb, gpu_batch_size=gbs, out=out,
+                  workspace=ws, compute_stream=compute, copy_stream=copy)
+
+    for i in range(args.warmup):
+        step(i)
+    fg.fg_sync_status()
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(compute)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    e1.record(compute)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = replicas.max_over_ranks(e0.elapsed_time(e1), device=dev)
+    fg.fg_sync_status()
+    blob_gb = cfg.blob_bytes() * nl / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "decode tokens/s of the OPT layer stack (W4 weights streamed from pinned host, KV4 in HBM)",
+            "value": world * S * args.steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "dtype": "f16", "data": "synthetic",
+            "config": {"workload": args.workload, "layers": nl, "block": f"{nb}x{gbs}", "hidden": h, "prompt": P,
+                       "weights_streamed_gb_per_step": round(blob_gb, 3),
+                       "kv_gb_in_hbm": round(sum(c.nbytes() for c in caches) / 1e9, 2)},
+            "host_link_gbs": round(blob_gb / (ms / args.steps / 1e3), 1),
+            "clocks": clocks,
+        }), flush=True)
+    st.close()
 
 
 def run_kernel(args, wl):
@@ -449,10 +559,13 @@ def main():
                          "dequantize")
     ap.add_argument("--seqs", type=int, default=0, help="--kernel: sequences (default: the workload's block)")
     ap.add_argument("--log2-elems", type=int, default=28, help="--kernel quantize/dequantize: tensor size")
+    ap.add_argument("--layers", type=int, default=0, help="stack workloads: number of layers (default: the model's)")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
     if args.kernel:
         run_kernel(args, wl)
+    elif "layers" in wl and args.impl == "ours":
+        run_stack(args, wl)
     elif args.impl == "reference":
         run_reference(args, wl)
     else:
