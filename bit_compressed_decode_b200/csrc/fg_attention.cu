@@ -7,12 +7,26 @@
 //
 // One CTA (4 warps) per (query row, head).  The row's cached K/V codes and group
 // metadata stream through shared memory in chunks of 64 tokens with 1-D bulk copies
-// (cp.async.bulk, completion on an mbarrier), STAGES chunks in flight.  Each token
-// is handled by D/32 lanes (16 code bytes = 32 dims each, half a 64-group).
-// Scores use the group decomposition
-//     q . k = sum_g ( min_g * sum_{d in g} q_d  +  scale_g * sum_{d in g} q_d * code_d ),
-// so the per-element work is one FMA with the integer code; V is accumulated the same
-// way (sum_t p_t * min_t and sum_t (p_t * scale_t) * code_t,d), all in fp32.
+// (cp.async.bulk, completion on an mbarrier), kStages chunks in flight; each warp takes
+// 16 tokens of every chunk.
+//
+// Both products run on the tensor cores (mma.sync m16n8k16, fp16 operands, fp32
+// accumulation) directly on the codes, through the group decomposition
+//     q . k_t = sum_g ( min_tg * sum_{d in g} q_d  +  scale_tg * sum_{d in g} q_d c_td )
+//     o_d     = sum_t p_t min_t,g(d)  +  sum_t (p_t scale_t,g(d)) c_td
+// so the per-element work is one AND per pair of codes: a nibble left in bits 0-3 of a
+// 16-bit half is the fp16 subnormal c * 2^-24, one in bits 4-7 is c * 2^-20, both exact,
+// and the fp32 results are rescaled by the matching power of two.
+//   scores: A = K codes (16 tokens x 16 dims per MMA), B = q (16 dims x 8 columns;
+//           column n holds q on the dims of one group, zero elsewhere) -> the group sums
+//           sum_{d in g} q_d c_td of every token, each group in 8/NG columns, so that every
+//           lane of a quad sees all groups of its two tokens and the four lanes split the
+//           per-token work;
+//   output: A = V codes transposed (16 dims x 16 tokens), B = w (16 tokens x 8 columns;
+//           column g is p_t * scale_tg rounded to fp16) -> row d, column g(d).
+// Dims may take any order along an MMA's k dimension as long as q takes the same order
+// (tokens likewise for V), which lets every lane build its operands from whole 32-bit
+// words of codes.  Scores, the softmax state and every sum stay in fp32.
 #include <math.h>
 
 #include "fg_internal.cuh"
@@ -22,6 +36,10 @@ namespace {
 constexpr int kChunk = 64;
 constexpr int kStages = 4;
 constexpr int kWarps = 4;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kSlack = 2.0f;
+constexpr uint32_t kLoNib = 0x000F000Fu;  // bits 0-3 of both halves: c * 2^-24
+constexpr uint32_t kHiNib = 0x00F000F0u;  // bits 4-7 of both halves: c * 2^-20
 
 struct AttnArgs {
   const __half *q;
@@ -37,32 +55,117 @@ struct AttnArgs {
 
 template <int D>
 struct AttnShape {
-  static constexpr int LPT = D / 32;                // lanes per token
-  static constexpr int TPW = 32 / LPT;              // tokens per warp per sub-step
   static constexpr int NG = D / 64;                 // 64-groups per head
-  static constexpr int SUB = kChunk / kWarps / TPW; // sub-steps per warp per chunk
-  static constexpr int CODE_B = kChunk * D / 2;     // code bytes per chunk (K or V)
+  static constexpr int RB = D / 2;                  // code bytes per token row
+  static constexpr int KW = D / 32;                 // K code words per lane per token
+  static constexpr int VW = D / 64;                 // V code words per lane per token
+  static constexpr int MT = D / 16;                 // 16-dim output tiles
+  static constexpr int CODE_B = kChunk * RB;        // code bytes per chunk (K or V)
   static constexpr int META_B = kChunk * NG * 2;    // bytes of one metadata array per chunk
   static constexpr int STAGE_B = 2 * CODE_B + 4 * META_B;
   static constexpr int SMEM = kStages * STAGE_B;
 };
 
-// code (0..15) of nibble i of w as an fp32 value: byte-permute the nibble-holding byte
-// into the low byte of 2^23 (0x4B000000), subtract 2^23.
-__device__ __forceinline__ float code_f(uint32_t lo_bytes, int byte_idx) {
-  const uint32_t bits = __byte_perm(lo_bytes, 0x4B000000u, 0x7540 + byte_idx);
-  return __int_as_float(bits) - 8388608.0f;
+// Byte offset in a K code row of word j of lane class c (lane % 4): the dims that lane
+// class feeds to the score MMAs.  Always inside one 64-group (32 bytes).
+template <int D>
+__device__ __forceinline__ int kword_off(int c, int j) {
+  return D == 64 ? 8 * c + 4 * j : 64 * (j >> 2) + 16 * c + 4 * (j & 3);
+}
+
+// Group held by column n of the score MMAs.  Lane (gid, c) reads columns 2c and 2c+1; the
+// map puts the group(s) lane c finishes (c % 2 for NG = 2; 2 (c % 2) + {0, 1} for NG = 4)
+// in those columns, the first of them in column 2c.
+template <int NG>
+__device__ __forceinline__ int col_group(int n) {
+  return NG == 1 ? 0 : NG == 2 ? ((n >> 1) ^ n) & 1 : n & 3;
+}
+
+template <int D>
+__device__ __forceinline__ void load_krow(const uint8_t *row, int c, uint32_t (&w)[D / 32]) {
+  if constexpr (D == 64) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(row + 8 * c);
+    w[0] = v.x;
+    w[1] = v.y;
+  } else {
+#pragma unroll
+    for (int u = 0; u < D / 128; u++) {
+      const uint4 v = *reinterpret_cast<const uint4 *>(row + 64 * u + 16 * c);
+      w[4 * u] = v.x;
+      w[4 * u + 1] = v.y;
+      w[4 * u + 2] = v.z;
+      w[4 * u + 3] = v.w;
+    }
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void load_words(const uint8_t *p, uint32_t (&w)[N]) {
+  if constexpr (N == 1) {
+    w[0] = *reinterpret_cast<const uint32_t *>(p);
+  } else if constexpr (N == 2) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(p);
+    w[0] = v.x;
+    w[1] = v.y;
+  } else {
+    const uint4 v = *reinterpret_cast<const uint4 *>(p);
+    w[0] = v.x;
+    w[1] = v.y;
+    w[2] = v.z;
+    w[3] = v.w;
+  }
+}
+
+// d += A * B for one m16n8k16 tile, fp16 operands and fp32 accumulators, in the PTX
+// fragment layout: a0/a1 = rows gid/gid+8 at k = 2c..2c+1, a2/a3 = the same rows at
+// k = 2c+8..2c+9; b0/b1 = column gid at k = 2c..2c+1 / 2c+8..2c+9; d = rows gid, gid+8 x
+// columns 2c, 2c+1 (gid = lane / 4, c = lane % 4).
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// d = A * B (fresh accumulators)
+__device__ __forceinline__ void mma_f16_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+// 2^x by the hardware approximation (relative error ~2^-22); results below 2^-126 are 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
+  const __half2 h = __halves2half2(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&h);
 }
 
 template <int D>
 __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs a) {
   using S = AttnShape<D>;
+  constexpr int NG = S::NG, RB = S::RB, KW = S::KW, VW = S::VW, MT = S::MT;
+  constexpr float kS24 = 16777216.0f, kS20 = 1048576.0f;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ float red_m[kWarps], red_l[kWarps];
   __shared__ float red_o[kWarps][D];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, c = lane & 3;
   const int r = blockIdx.x / a.H, hd = blockIdx.x % a.H;
   const int s = r / a.rows_per_seq;
   const int L = a.positions[s] + r % a.rows_per_seq + 1;
@@ -76,21 +179,21 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
   const int64_t slot0 = (static_cast<int64_t>(s) * a.H + hd) * a.maxL;
 
   auto stage_ptr = [&](int st) { return smem + st * S::STAGE_B; };
-  auto issue = [&](int c) {
-    const int st = c % kStages;
-    const int nt = min(kChunk, L - c * kChunk);
+  auto issue = [&](int ch) {
+    const int st = ch % kStages;
+    const int nt = min(kChunk, L - ch * kChunk);
     const int ntr = (nt + 7) & ~7;  // whole 16-byte metadata rows; stays below max_len (multiple of 64)
-    const uint32_t cb = ntr * (D / 2), mb = ntr * S::NG * 2;
+    const uint32_t cb = ntr * RB, mb = ntr * NG * 2;
     const uint32_t bar = smem_u32(&full_bar[st]);
     mbar_arrive_expect_tx(bar, 2 * cb + 4 * mb);
-    const int64_t t0 = slot0 + static_cast<int64_t>(c) * kChunk;
+    const int64_t t0 = slot0 + static_cast<int64_t>(ch) * kChunk;
     uint8_t *p = stage_ptr(st);
-    bulk_g2s(smem_u32(p), a.kc + t0 * (D / 2), cb, bar);
-    bulk_g2s(smem_u32(p + S::CODE_B), a.vc + t0 * (D / 2), cb, bar);
-    bulk_g2s(smem_u32(p + 2 * S::CODE_B + 0 * S::META_B), a.km + t0 * S::NG, mb, bar);
-    bulk_g2s(smem_u32(p + 2 * S::CODE_B + 1 * S::META_B), a.ks + t0 * S::NG, mb, bar);
-    bulk_g2s(smem_u32(p + 2 * S::CODE_B + 2 * S::META_B), a.vm + t0 * S::NG, mb, bar);
-    bulk_g2s(smem_u32(p + 2 * S::CODE_B + 3 * S::META_B), a.vs + t0 * S::NG, mb, bar);
+    bulk_g2s(smem_u32(p), a.kc + t0 * RB, cb, bar);
+    bulk_g2s(smem_u32(p + S::CODE_B), a.vc + t0 * RB, cb, bar);
+    bulk_g2s(smem_u32(p + 2 * S::CODE_B + 0 * S::META_B), a.km + t0 * NG, mb, bar);
+    bulk_g2s(smem_u32(p + 2 * S::CODE_B + 1 * S::META_B), a.ks + t0 * NG, mb, bar);
+    bulk_g2s(smem_u32(p + 2 * S::CODE_B + 2 * S::META_B), a.vm + t0 * NG, mb, bar);
+    bulk_g2s(smem_u32(p + 2 * S::CODE_B + 3 * S::META_B), a.vs + t0 * NG, mb, bar);
   };
 
   if (tid == 0) {
@@ -100,124 +203,209 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
   }
   __syncthreads();
   if (tid == 0)
-    for (int c = 0; c < min(kStages, nchunks); c++) issue(c);
+    for (int ch = 0; ch < min(kStages, nchunks); ch++) issue(ch);
 
-  // this lane's 32 query dims (scaled by log2(e) so the softmax can use exp2)
-  const int p = lane % S::LPT, ts = lane / S::LPT, g = p >> 1;
-  float qf[32];
-  {
-    const uint4 *qp = reinterpret_cast<const uint4 *>(a.q + static_cast<int64_t>(r) * a.ldq + hd * D + p * 32);
+  // ---- q as the B operand of the score MMAs, in the dim order of kword_off ----
+  // Word j of lane class c holds, per 16-bit half, nibbles (bits 0-3, 4-7, 8-11, 12-15) =
+  // dims 2o+{0,1,2,3} (low half) and 2o+{4,5,6,7} (high half), o = kword_off(c, j).
+  // Low-nibble MMA (bits 0-3 of w and of w >> 8): k slots (2c, 2c+1) = dims (2o, 2o+4),
+  // (2c+8, 2c+9) = (2o+2, 2o+6); high-nibble MMA: the same + 1.
+  const __half *qrow = a.q + static_cast<int64_t>(r) * a.ldq + hd * D;
+  uint32_t qlo[KW][2], qhi[KW][2];
 #pragma unroll
-    for (int i = 0; i < 4; i++) {
-      uint4 v = qp[i];
-      const __half2 *h2 = reinterpret_cast<const __half2 *>(&v);
-#pragma unroll
-      for (int j = 0; j < 4; j++) {
-        float2 f = __half22float2(h2[j]);
-        qf[8 * i + 2 * j] = f.x * 1.4426950408889634f;
-        qf[8 * i + 2 * j + 1] = f.y * 1.4426950408889634f;
-      }
+  for (int j = 0; j < KW; j++) {
+    const int o = kword_off<D>(c, j);
+    if (col_group<NG>(gid) == o / 32) {
+      const uint4 v = *reinterpret_cast<const uint4 *>(qrow + 2 * o);
+      const __half *e = reinterpret_cast<const __half *>(&v);
+      qlo[j][0] = pack_h2(e[0], e[4]);
+      qlo[j][1] = pack_h2(e[2], e[6]);
+      qhi[j][0] = pack_h2(e[1], e[5]);
+      qhi[j][1] = pack_h2(e[3], e[7]);
+    } else {
+      qlo[j][0] = qlo[j][1] = qhi[j][0] = qhi[j][1] = 0u;
     }
   }
-  float qsum = 0.f;
+  // Lane (gid, c) finishes token gid + 8 * (c >> 1) on the groups of its column pair
+  // (2c, 2c+1): g0 = (c & 1) * NG / 2 and, for NG = 4, g0 + 1; the other lane of its pair
+  // (c ^ 1) holds the remaining groups.
+  const int g0 = (c & 1) * (NG / 2);
+  constexpr int GPL = NG == 4 ? 2 : 1;  // groups per lane
+  float ql[GPL];                         // sum of q over those groups, times log2(e)
+  {
+    constexpr int PER = D / 32, LPG = 64 / PER;  // dims per lane, lanes per group
+    float qs = 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; i++) qsum += qf[i];
-  const float Qg = qsum + __shfl_xor_sync(0xffffffffu, qsum, 1);
-
-  float m = -INFINITY, l = 0.f, accmin = 0.f;
-  float acc[32];
+    for (int i = 0; i < PER; i++) qs += __half2float(qrow[lane * PER + i]);
 #pragma unroll
-  for (int i = 0; i < 32; i++) acc[i] = 0.f;
+    for (int o = 1; o < LPG; o <<= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
+#pragma unroll
+    for (int e = 0; e < GPL; e++) ql[e] = __shfl_sync(0xffffffffu, qs, (g0 + e) * LPG) * kLog2e;
+  }
+  const int tq = gid + 8 * (c >> 1);  // this lane's token within a warp tile
 
-  volatile int *no_abort = nullptr;
+  float m = -INFINITY, l = 0.f;
+  float vmin[GPL];  // sum_t p_t * min_t,g over this lane's tokens, for its groups
+  float ov[MT][4];
+#pragma unroll
+  for (int e = 0; e < GPL; e++) vmin[e] = 0.f;
+#pragma unroll
+  for (int t = 0; t < MT; t++) ov[t][0] = ov[t][1] = ov[t][2] = ov[t][3] = 0.f;
+
   bool ok = true;
-  for (int c = 0; c < nchunks; c++) {
-    const int st = c % kStages;
-    if (ok && !mbar_wait_bounded(smem_u32(&full_bar[st]), (c / kStages) & 1, no_abort, a.err)) ok = false;
+  for (int ch = 0; ch < nchunks; ch++) {
+    const int st = ch % kStages;
+    if (ok && !mbar_wait_bounded(smem_u32(&full_bar[st]), (ch / kStages) & 1, nullptr, a.err)) ok = false;
     if (ok) {
       const uint8_t *base = stage_ptr(st);
-      const uint4 *Kc = reinterpret_cast<const uint4 *>(base);
-      const uint4 *Vc = reinterpret_cast<const uint4 *>(base + S::CODE_B);
+      const uint8_t *Kc = base, *Vc = base + S::CODE_B;
       const __half *Km = reinterpret_cast<const __half *>(base + 2 * S::CODE_B);
-      const __half *Ks = Km + kChunk * S::NG;
-      const __half *Vm = Ks + kChunk * S::NG;
-      const __half *Vs = Vm + kChunk * S::NG;
-      float sc[S::SUB];
-      float cmax = -INFINITY;
+      const __half *Ks = Km + kChunk * NG;
+      const __half *Vm = Ks + kChunk * NG;
+      const __half *Vs = Vm + kChunk * NG;
+      const int t0 = warp * 16;  // this warp's tokens in the chunk: t0 .. t0+15
+
+      // ---- group sums of q . c for tokens t0+gid and t0+gid+8 ----
+      float slo[4], shi[4];
+      {
+        uint32_t k0[KW], k1[KW];
+        load_krow<D>(Kc + (t0 + gid) * RB, c, k0);
+        load_krow<D>(Kc + (t0 + gid + 8) * RB, c, k1);
 #pragma unroll
-      for (int u = 0; u < S::SUB; u++) {
-        const int tl = warp * (kChunk / kWarps) + u * S::TPW + ts;
-        const bool valid = c * kChunk + tl < L;
-        const uint4 kw = Kc[tl * S::LPT + p];
-        float dot = 0.f;
-        const uint32_t words[4] = {kw.x, kw.y, kw.z, kw.w};
-#pragma unroll
-        for (int wi = 0; wi < 4; wi++) {
-          const uint32_t lo = words[wi] & 0x0F0F0F0Fu, hi = (words[wi] >> 4) & 0x0F0F0F0Fu;
-#pragma unroll
-          for (int b = 0; b < 4; b++) {
-            dot = fmaf(qf[8 * wi + 2 * b], code_f(lo, b), dot);
-            dot = fmaf(qf[8 * wi + 2 * b + 1], code_f(hi, b), dot);
+        for (int j = 0; j < KW; j++) {
+          const uint32_t x0 = k0[j], x1 = k1[j], y0 = x0 >> 8, y1 = x1 >> 8;
+          if (j == 0) {
+            mma_f16_z(slo, x0 & kLoNib, x1 & kLoNib, y0 & kLoNib, y1 & kLoNib, qlo[j][0], qlo[j][1]);
+            mma_f16_z(shi, x0 & kHiNib, x1 & kHiNib, y0 & kHiNib, y1 & kHiNib, qhi[j][0], qhi[j][1]);
+          } else {
+            mma_f16(slo, x0 & kLoNib, x1 & kLoNib, y0 & kLoNib, y1 & kLoNib, qlo[j][0], qlo[j][1]);
+            mma_f16(shi, x0 & kHiNib, x1 & kHiNib, y0 & kHiNib, y1 & kHiNib, qhi[j][0], qhi[j][1]);
           }
         }
-        dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-        float sg = __half2float(Km[tl * S::NG + g]) * Qg + __half2float(Ks[tl * S::NG + g]) * dot;
-#pragma unroll
-        for (int o = 2; o < S::LPT; o <<= 1) sg += __shfl_xor_sync(0xffffffffu, sg, o);
-        sc[u] = valid ? sg : -INFINITY;
-        cmax = fmaxf(cmax, sc[u]);
       }
+      // ---- score (log2 units) of token t0+tq ----
+      const bool valid = ch * kChunk + t0 + tq < L;
+      float sc;
+      {
+        const int i0 = (t0 + tq) * NG + g0;
+        float part = 0.f;
 #pragma unroll
-      for (int o = S::LPT; o < 32; o <<= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
-      const float m_new = fmaxf(m, cmax);
-      if (m_new != -INFINITY) {
-        const float alpha = exp2f(m - m_new);  // 0 when m is -inf
+        for (int e = 0; e < GPL; e++) {
+          // C element of token row tq (gid or gid+8), column 2c + e
+          const bool r8 = c & 2;
+          const float lo = r8 ? slo[2 + e] : slo[e], hi = r8 ? shi[2 + e] : shi[e];
+          const float dot = lo * (kS24 * kLog2e) + hi * (kS20 * kLog2e);
+          part += __half2float(Km[i0 + e]) * ql[e] + __half2float(Ks[i0 + e]) * dot;
+        }
+        if constexpr (NG > 1) part += __shfl_xor_sync(0xffffffffu, part, 1);
+        sc = valid ? part : -INFINITY;
+      }
+      float cmax = sc;
+#pragma unroll
+      for (int o = 2; o < 32; o <<= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+      // Lazy rescaling: the reference maximum m moves only when a score exceeds it by more
+      // than kSlack (log2 units), so p = 2^(s - m) <= 2^kSlack = 4 and w = p * scale stays
+      // below 4 * 8734 (the largest scale of 4-bit codes of fp16 data), inside fp16.
+      if (cmax > m + kSlack) {  // warp-uniform; always taken at the first valid token (m = -inf)
+        const float m_new = cmax;
+        const float alpha = fast_exp2(m - m_new);  // 0 when m is -inf
         l *= alpha;
-        accmin *= alpha;
 #pragma unroll
-        for (int i = 0; i < 32; i++) acc[i] *= alpha;
+        for (int e = 0; e < GPL; e++) vmin[e] *= alpha;
 #pragma unroll
-        for (int u = 0; u < S::SUB; u++) {
-          const int tl = warp * (kChunk / kWarps) + u * S::TPW + ts;
-          const bool valid = c * kChunk + tl < L;
-          const float pt = valid ? exp2f(sc[u] - m_new) : 0.f;
-          l += pt;
-          const float w = valid ? pt * __half2float(Vs[tl * S::NG + g]) : 0.f;
-          accmin += valid ? pt * __half2float(Vm[tl * S::NG + g]) : 0.f;
-          const uint4 vw = Vc[tl * S::LPT + p];
-          const uint32_t words[4] = {vw.x, vw.y, vw.z, vw.w};
-#pragma unroll
-          for (int wi = 0; wi < 4; wi++) {
-            const uint32_t lo = words[wi] & 0x0F0F0F0Fu, hi = (words[wi] >> 4) & 0x0F0F0F0Fu;
-#pragma unroll
-            for (int b = 0; b < 4; b++) {
-              acc[8 * wi + 2 * b] = fmaf(w, code_f(lo, b), acc[8 * wi + 2 * b]);
-              acc[8 * wi + 2 * b + 1] = fmaf(w, code_f(hi, b), acc[8 * wi + 2 * b + 1]);
-            }
-          }
+        for (int t = 0; t < MT; t++) {
+          ov[t][0] *= alpha;
+          ov[t][1] *= alpha;
+          ov[t][2] *= alpha;
+          ov[t][3] *= alpha;
         }
         m = m_new;
       }
+      if (cmax != -INFINITY) {  // warp-uniform: some token of the tile is valid
+        const float pt = fast_exp2(sc - m);  // 0 for a masked token
+        l += pt;                         // each token counted by two lanes
+        // w = p * V scale for this lane's (token, groups), packed as fp16 in W
+        uint32_t W;
+        {
+          const int i0 = (t0 + tq) * NG + g0;
+          float w[2];
+#pragma unroll
+          for (int e = 0; e < GPL; e++) {
+            vmin[e] += valid ? pt * __half2float(Vm[i0 + e]) : 0.f;
+            w[e] = valid ? pt * __half2float(Vs[i0 + e]) : 0.f;
+          }
+          W = pack_h2(w[0], w[GPL - 1]);
+        }
+        // ---- w as the B operand: lane (n = gid, c) holds column n at tokens c, c+4 (k slots
+        //      2c, 2c+1) and c+8, c+12 (k slots 2c+8, 2c+9); w(t, n) sits in lane
+        //      4 (t % 8) + 2 (t / 8) + (n / GPL) % 2, half n % GPL ----
+        uint32_t wb0, wb1;
+        {
+          const int src = 4 * c + ((gid / GPL) & (NG > 1 ? 1 : 0));
+          const uint32_t X0 = __shfl_sync(0xffffffffu, W, src), X1 = __shfl_sync(0xffffffffu, W, src + 16);
+          const uint32_t X2 = __shfl_sync(0xffffffffu, W, src + 2), X3 = __shfl_sync(0xffffffffu, W, src + 18);
+          const uint32_t sel = (GPL == 2 && (gid & 1)) ? 0x7632u : 0x5410u;
+          wb0 = gid < NG ? __byte_perm(X0, X1, sel) : 0u;
+          wb1 = gid < NG ? __byte_perm(X2, X3, sel) : 0u;
+        }
+        // ---- V codes as the A operand: lane (gid, c) reads its D/8 dims (bytes
+        //      gid*D/16 ...) of tokens c, c+4, c+8, c+12 and pairs tokens per 16-bit half ----
+        uint32_t v0[VW], v1[VW], v2[VW], v3[VW];
+        const uint8_t *vrow = Vc + (t0 + c) * RB + gid * (D / 16);
+        load_words<VW>(vrow, v0);
+        load_words<VW>(vrow + 4 * RB, v1);
+        load_words<VW>(vrow + 8 * RB, v2);
+        load_words<VW>(vrow + 12 * RB, v3);
+#pragma unroll
+        for (int j = 0; j < VW; j++) {
+#pragma unroll
+          for (int h = 0; h < 2; h++) {
+            const uint32_t sel = h ? 0x7632u : 0x5410u;
+            const uint32_t P = __byte_perm(v0[j], v1[j], sel), Q = __byte_perm(v2[j], v3[j], sel);
+            const uint32_t Ps = P >> 8, Qs = Q >> 8;
+            // tile 4j+2h: rows gid / gid+8 = dims gid*D/8 + 2T + 0 / + 1 (nibbles 0 / 1 of
+            // the byte pair); tile 4j+2h+1: nibbles 2 / 3
+            mma_f16(ov[4 * j + 2 * h], P & kLoNib, P & kHiNib, Q & kLoNib, Q & kHiNib, wb0, wb1);
+            mma_f16(ov[4 * j + 2 * h + 1], Ps & kLoNib, Ps & kHiNib, Qs & kLoNib, Qs & kHiNib, wb0, wb1);
+          }
+        }
+      }
     }
     __syncthreads();  // every warp is done with stage st
-    if (tid == 0 && ok && c + kStages < nchunks) issue(c + kStages);
+    if (tid == 0 && ok && ch + kStages < nchunks) issue(ch + kStages);
   }
 
-  // reduce over the token slots of the warp (lanes with equal p)
+  // ---- per-warp totals, then combine the 4 warps ----
 #pragma unroll
-  for (int o = S::LPT; o < 32; o <<= 1) {
-    l += __shfl_xor_sync(0xffffffffu, l, o);
-    accmin += __shfl_xor_sync(0xffffffffu, accmin, o);
+  for (int o = 1; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  l *= 0.5f;  // every token was counted by both lanes of its pair
 #pragma unroll
-    for (int i = 0; i < 32; i++) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-  }
-  if (ts == 0) {
+  for (int o = (NG > 1 ? 2 : 1); o < 32; o <<= 1)
 #pragma unroll
-    for (int i = 0; i < 32; i++) red_o[warp][p * 32 + i] = acc[i] + accmin;
-    if (p == 0) {
-      red_m[warp] = m;
-      red_l[warp] = l;
+    for (int e = 0; e < GPL; e++) vmin[e] += __shfl_xor_sync(0xffffffffu, vmin[e], o);
+  if constexpr (NG == 1) vmin[0] *= 0.5f;
+  {
+    // lane (gid, c) with c == g/2 owns dims gid*D/8 .. +D/8-1 of group g = gid*D/512:
+    // column g is element (g & 1) of its accumulator pairs; the V-min total of group g sits
+    // in lane (g / GPL) % 2, element g % GPL
+    const int g = gid * D / 512;
+    const int gl = NG > 1 ? (g / GPL) & 1 : 0;
+    float vm = __shfl_sync(0xffffffffu, vmin[0], gl);
+    if constexpr (GPL == 2) {
+      const float vm1 = __shfl_sync(0xffffffffu, vmin[1], gl);
+      vm = (g & 1) ? vm1 : vm;
     }
+    if (c == g / 2) {
+      const bool odd = g & 1;
+      float2 *dst = reinterpret_cast<float2 *>(&red_o[warp][gid * (D / 8)]);
+#pragma unroll
+      for (int t = 0; t < MT; t++)
+        dst[t] = make_float2((odd ? ov[t][1] : ov[t][0]) * kS24 + vm, (odd ? ov[t][3] : ov[t][2]) * kS20 + vm);
+    }
+  }
+  if (lane == 0) {
+    red_m[warp] = m;
+    red_l[warp] = l;
   }
   __syncthreads();
   float M = -INFINITY;
