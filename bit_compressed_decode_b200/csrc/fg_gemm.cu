@@ -326,6 +326,288 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
 }
 
 // ------------------------------------------------------------------------------------
+// Pair kernel: one tcgen05.mma.cta_group::2 spans two SMs.
+//
+//   CTA pair (cluster ranks 2p, 2p+1): 256 output features x 512 tokens x a k-range.  Each
+//   CTA dequantises its own 128 weight rows (the MMA's A = 256 rows is split by rows) and
+//   loads its halves of the two 256-token x tiles (B is split by columns: tokens
+//   tile*256 + half*128 ...).  The even CTA issues two M=256, N=256 MMAs per 16-wide k-step,
+//   one per token tile, into TMEM columns [0, 256) and [256, 512) of BOTH CTAs (each holds
+//   its 128 feature rows).  Per SM and k-tile: 128 dequantised rows (half of the single-SM
+//   kernel's rows per flop) and ~112 KB of shared-memory traffic for 8 MFLOP.
+//   warps 0..7   dequantise (thread: row tid % 128, k half tid / 128), then the epilogue
+//                (warp: TMEM lane quarter warp % 4, token tile warp / 4);
+//   warp 8       TMA of this CTA's x halves, completing on the even CTA's barrier;
+//   warp 9       even CTA: the MMA issuer; odd CTA: forwards "A half ready" per stage (one
+//                cluster-scope release instead of one per dequant warp); TMEM allocation.
+//   Split k-ranges of one pair tile form the cluster's z dimension (cluster 2 x 1 x splits);
+//   partial sums are reduced over distributed shared memory in z-rank order.
+// ------------------------------------------------------------------------------------
+
+constexpr int kPairTok = 512;                  // tokens per pair tile
+constexpr int kPairStages = 4;
+constexpr int kPairA = 128 * 128;              // this CTA's A tile: 128 rows x 128 B
+constexpr int kPairBHalf = 128 * 128;          // this CTA's half of one token tile: 128 tokens x 128 B
+constexpr int kPairStage = kPairA + 2 * kPairBHalf;
+constexpr int kPairRing = kPairStages * kPairStage;
+constexpr int kPairSmem = kPairRing + 1024;
+constexpr int kPairCols = 512;
+constexpr int kPairPrefetch = 4;
+constexpr uint32_t kPairIdesc = umma_idesc_f16_f32(256, 256);
+
+__global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_pair_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                      const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // full (even CTA): the stage is ready -- its 8 dequant warps, the odd CTA's forwarded
+  // "A half done", and its TMA arrival carrying the x bytes of both CTAs (one wait per stage
+  // for the MMA thread, whose issue rate bounds the kernel); a_half (odd CTA): its 8
+  // dequant warps are done; empty: the pair's MMAs are done with the stage.
+  __shared__ __align__(8) uint64_t full[kPairStages], a_half[kPairStages], empty[kPairStages], accum_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t lead = crank & ~1u;
+  const bool leader = crank == lead;
+  const int half = static_cast<int>(crank & 1u);
+  const int n0 = blockIdx.x * 128;  // this CTA's 128 weight rows
+  const int t0 = blockIdx.y * kPairTok, split = blockIdx.z;
+  const int ktiles = a.K / kBK;
+  const int kt0 = static_cast<int>((static_cast<int64_t>(split) * ktiles) / a.splits);
+  const int kt1 = static_cast<int>((static_cast<int64_t>(split + 1) * ktiles) / a.splits);
+  const int nk = kt1 - kt0;
+  volatile int *abortp = &abort_flag;
+  const uint16_t pair_mask = static_cast<uint16_t>(3u << lead);
+
+  auto a_tile = [&](int st) { return smem + st * kPairStage; };
+  auto b_tile = [&](int st, int tile) { return smem + st * kPairStage + kPairA + tile * kPairBHalf; };
+
+  if (tid == 0) {
+    for (int i = 0; i < kPairStages; i++) {
+      mbar_init(smem_u32(&full[i]), kDeqWarps + 2);  // 8 local warps + odd CTA + TMA
+      mbar_init(smem_u32(&a_half[i]), kDeqWarps);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    mbar_init(smem_u32(&accum_bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc_pair(smem_u32(&tmem_slot), kPairCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers initialised and TMEM allocated in both CTAs
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp < kDeqWarps) {
+    // ---------------- dequantise producer: row tid % 128, k half tid / 128 ----------------
+    const int row = tid & 127, hk = tid >> 7;
+    const int n = n0 + row;
+    const bool live = n < a.N;
+    const uint4 *crow = reinterpret_cast<const uint4 *>(a.wc + static_cast<int64_t>(live ? n : 0) * (a.K / 2));
+    const __half *mrow = a.wm + static_cast<int64_t>(live ? n : 0) * (a.K / kBK);
+    const __half *srow = a.ws + static_cast<int64_t>(live ? n : 0) * (a.K / kBK);
+    uint4 cb[kPairPrefetch];
+    __half mb[kPairPrefetch], sb[kPairPrefetch];
+#pragma unroll
+    for (int j = 0; j < kPairPrefetch; j++) {
+      if (j < nk && live) {
+        cb[j] = crow[(kt0 + j) * 2 + hk];
+        mb[j] = mrow[kt0 + j];
+        sb[j] = srow[kt0 + j];
+      } else {
+        cb[j] = make_uint4(0, 0, 0, 0);
+        mb[j] = sb[j] = __ushort_as_half(0);
+      }
+    }
+    // leader: arrive on its own full barrier; odd CTA: on a_half, forwarded by warp 9
+    const uint32_t done_bar0 = smem_u32(leader ? &full[0] : &a_half[0]);
+    for (int i = 0; i < nk; i++) {
+      const int st = i % kPairStages;
+      const uint4 c0 = cb[0];
+      const __half m0 = mb[0], s0 = sb[0];
+#pragma unroll
+      for (int j = 0; j + 1 < kPairPrefetch; j++) {
+        cb[j] = cb[j + 1];
+        mb[j] = mb[j + 1];
+        sb[j] = sb[j + 1];
+      }
+      if (i + kPairPrefetch < nk && live) {
+        const int kt = kt0 + i + kPairPrefetch;
+        cb[kPairPrefetch - 1] = crow[kt * 2 + hk];
+        mb[kPairPrefetch - 1] = mrow[kt];
+        sb[kPairPrefetch - 1] = srow[kt];
+      }
+      if (i >= kPairStages &&
+          !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kPairStages) - 1) & 1, abortp, a.err))
+        break;
+      const __half2 s2 = __half2half2(s0), m2 = __half2half2(m0);
+      uint8_t *at = a_tile(st);
+      const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
+#pragma unroll
+      for (int c = 0; c < 4; c++) {
+        const uint4 v = live ? dequant8(words[c], s2, m2) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(at + sw128_offset(row, 4 * hk + c)) = v;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(done_bar0 + st * 8);
+    }
+  } else if (warp == kTmaWarp) {
+    // ---------------- TMA producer: this CTA's halves of the two token tiles ----------------
+    if (lane == 0) {
+      prefetch_tmap(&xmap);
+      for (int i = 0; i < nk; i++) {
+        const int st = i % kPairStages;
+        if (i >= kPairStages &&
+            !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kPairStages) - 1) & 1, abortp, a.err))
+          break;
+        const uint32_t fb = mapa_shared(smem_u32(&full[st]), lead);
+        if (leader) mbar_arrive_expect_tx(smem_u32(&full[st]), 4 * kPairBHalf);  // both CTAs, both tiles
+#pragma unroll
+        for (int tile = 0; tile < 2; tile++)
+          tma_load_2d_pair(smem_u32(b_tile(st, tile)), &xmap, (kt0 + i) * kBK, t0 + tile * 256 + half * 128, fb);
+      }
+    }
+  } else if (!leader) {
+    // ---------------- odd CTA: forward "A half ready" to the even CTA ----------------
+    // One cluster-scope release per stage instead of one per dequant warp.
+    if (lane == 0) {
+      for (int i = 0; i < nk; i++) {
+        const int st = i % kPairStages;
+        if (!mbar_wait_bounded(smem_u32(&a_half[st]), (i / kPairStages) & 1, abortp, a.err)) break;
+        mbar_arrive_cluster(mapa_shared(smem_u32(&full[st]), lead));
+      }
+    }
+  } else {
+    // ---------------- MMA issuer (even CTA) ----------------
+    // Kept lean: one wait, 8 MMAs and one commit per stage, descriptors precomputed (the
+    // 14-bit start-address field advances by 2 per 32-byte k step without carrying).
+    if (lane == 0) {
+      const uint64_t adesc0 = umma_desc_sw128(smem_u32(a_tile(0)));
+      const uint64_t bdesc0 = umma_desc_sw128(smem_u32(b_tile(0, 0)));
+      constexpr uint64_t kStageStep = kPairStage >> 4, kTileStep = kPairBHalf >> 4;
+      for (int i = 0; i < nk; i++) {
+        const int st = i % kPairStages;
+        if (!mbar_wait_bounded_cluster(smem_u32(&full[st]), (i / kPairStages) & 1, abortp, a.err)) break;
+        tc_fence_after();
+        const uint64_t ad = adesc0 + st * kStageStep, bd = bdesc0 + st * kStageStep;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; kk++) {
+#pragma unroll
+          for (int tile = 0; tile < 2; tile++)
+            umma_f16_pair(tmem + tile * 256, ad + 2 * kk, bd + tile * kTileStep + 2 * kk, kPairIdesc,
+                          (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit_pair(smem_u32(&empty[st]), pair_mask);
+      }
+      umma_commit_pair(smem_u32(&accum_bar), pair_mask);  // also tracks completion if the loop stopped early
+    }
+  }
+
+  // ---------------- epilogue: TMEM -> shared memory -> (cluster sum) -> global ----------------
+  // The 128 x 512 fp32 accumulator goes through the idle ring buffers kRound chunks of
+  // [32 tokens][128 features] at a time.  Chunk ch is finished by z rank ch % splits, which
+  // sums it over the cluster's z ranks in rank order (deterministic; with one split, its own
+  // copy) and writes 8 consecutive features per thread: 16-byte stores covering whole
+  // 256-byte row segments of y.  All threads of all CTAs take the same barriers.
+  bool ready = false;
+  if (warp < kDeqWarps) {
+    ready = mbar_wait_bounded_cluster(smem_u32(&accum_bar), 0, nullptr, a.err) && !*abortp;
+    tc_fence_after();
+  }
+  {
+    constexpr int kChunkFloats = 32 * 128;
+    constexpr int kRound = kPairRing / (kChunkFloats * 4);  // 12 chunks of the 16
+    constexpr int kChunks = kPairCols / 32;
+    const int q = warp & 3, etile = (warp >> 2) & 1;
+    const int zrank = static_cast<int>(crank >> 1);
+    const bool clustered = a.splits > 1;
+    float *buf = reinterpret_cast<float *>(smem);
+    // finishing thread: 8 features f8 .. f8+7 of rows (tokens) mj0 and mj0 + 16 of a chunk
+    const int f8 = (tid & 15) * 8, mj0 = (tid >> 4) & 15;
+    const int nb = n0 + f8;
+    float bias[8];
+#pragma unroll
+    for (int u = 0; u < 8; u++) bias[u] = (a.bias && warp < kDeqWarps && nb < a.N) ? __half2float(a.bias[nb + u]) : 0.f;
+    for (int r0 = 0; r0 < kChunks; r0 += kRound) {
+      if (warp < kDeqWarps) {
+        for (int c8 = 0; c8 < 8; c8++) {
+          const int ch = etile * 8 + c8;
+          if (ch < r0 || ch >= r0 + kRound) continue;
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, v);
+          tmem_wait_ld();
+          float *cbuf = buf + (ch - r0) * kChunkFloats;
+#pragma unroll
+          for (int j = 0; j < 32; j++) cbuf[j * 128 + q * 32 + lane] = __uint_as_float(v[j]);
+        }
+      }
+      __syncwarp();
+      if (clustered) cluster_sync_all(); else __syncthreads();
+      if (warp < kDeqWarps && ready && nb < a.N) {
+        for (int ch = r0; ch < r0 + kRound && ch < kChunks; ch++) {
+          if (ch % a.splits != zrank) continue;
+          float acc[2][8];
+#pragma unroll
+          for (int it = 0; it < 2; it++)
+#pragma unroll
+            for (int u = 0; u < 8; u++) acc[it][u] = 0.f;
+          const uint32_t off = smem_u32(buf + (ch - r0) * kChunkFloats + mj0 * 128 + f8);
+          for (int z = 0; z < a.splits; z++) {  // z-rank order
+            const uint32_t rb = clustered ? mapa_shared(off, (crank & 1u) + 2u * z) : off;
+#pragma unroll
+            for (int it = 0; it < 2; it++) {
+              const float4 p0 = clustered ? ld_shared_cluster_v4(rb + it * 16 * 128 * 4)
+                                          : *reinterpret_cast<const float4 *>(buf + (ch - r0) * kChunkFloats +
+                                                                              (mj0 + 16 * it) * 128 + f8);
+              const float4 p1 = clustered ? ld_shared_cluster_v4(rb + it * 16 * 128 * 4 + 16)
+                                          : *reinterpret_cast<const float4 *>(buf + (ch - r0) * kChunkFloats +
+                                                                              (mj0 + 16 * it) * 128 + f8 + 4);
+              acc[it][0] += p0.x; acc[it][1] += p0.y; acc[it][2] += p0.z; acc[it][3] += p0.w;
+              acc[it][4] += p1.x; acc[it][5] += p1.y; acc[it][6] += p1.z; acc[it][7] += p1.w;
+            }
+          }
+          uint4 rv[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+#pragma unroll
+          for (int it = 0; it < 2; it++) {
+            const int m = t0 + ch * 32 + mj0 + 16 * it;
+            if (a.res && m < a.M) rv[it] = *reinterpret_cast<const uint4 *>(a.res + static_cast<int64_t>(m) * a.N + nb);
+          }
+#pragma unroll
+          for (int it = 0; it < 2; it++) {
+            const int m = t0 + ch * 32 + mj0 + 16 * it;
+            if (m >= a.M) continue;
+            const __half *rh = reinterpret_cast<const __half *>(&rv[it]);
+            uint4 ov;
+            __half *oh = reinterpret_cast<__half *>(&ov);
+#pragma unroll
+            for (int u = 0; u < 8; u++)
+              oh[u] = __float2half_rn(epilogue(acc[it][u], bias[u], __half2float(rh[u]), nb + u, a));
+            *reinterpret_cast<uint4 *>(a.y + static_cast<int64_t>(m) * a.N + nb) = ov;
+          }
+        }
+      }
+      __syncwarp();
+      if (clustered) cluster_sync_all(); else __syncthreads();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer's TMEM and shared memory are no longer in use
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kPairCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------
 
@@ -424,6 +706,96 @@ fg_status launch_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cu
   return fg_launch_check();
 }
 
+
+// ---- pair kernel planning ----
+
+// Pair-kernel clusters (2 x 1 x splits CTAs) that can be resident at once; 0 when such a
+// cluster does not fit on the device.
+int pair_clusters_resident(int splits) {
+  static int cache[64][5];
+  static bool known[64][5] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || splits < 1 || splits > 4) return 0;
+  if (!known[dev][splits]) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(2, 1, splits);
+    lc.blockDim = dim3(kThreads, 1, 1);
+    lc.dynamicSmemBytes = kPairSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = splits;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, w4a16_gemm_pair_kernel, &lc) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    cache[dev][splits] = n > 0 ? n : 0;
+    known[dev][splits] = true;
+  }
+  return cache[dev][splits];
+}
+
+// Splits of the k-range (the cluster's z dimension, at most 4) that minimise
+// waves of resident clusters * k-tiles per CTA, with a small charge per extra split.
+Plan make_pair_plan(int M, int N, int K) {
+  Plan p;
+  p.nt = kPairTok;
+  p.n_tiles = (N + 255) / 256;  // CTA pairs along the features
+  p.t_tiles = (M + kPairTok - 1) / kPairTok;
+  const int ktiles = K / kBK;
+  const int clusters = p.n_tiles * p.t_tiles;
+  double best = 1e30;
+  p.splits = 1;
+  for (int s = 1; s <= 4; s++) {
+    if (s > 1 && ktiles / s < 8) break;
+    const int resident = pair_clusters_resident(s);
+    if (resident == 0) continue;
+    const int waves = (clusters + resident - 1) / resident;
+    const double cost = static_cast<double>(waves) * ((ktiles + s - 1) / s) * (1.0 + 0.05 * (s - 1));
+    if (cost < best - 1e-9) {
+      best = cost;
+      p.splits = s;
+    }
+  }
+  return p;
+}
+
+fg_status pair_attr_once() {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    fg_status rc = fg_cuda_check(
+        cudaFuncSetAttribute(w4a16_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem));
+    if (rc != FG_OK) return rc;
+    attr_set[dev] = true;
+  }
+  return FG_OK;
+}
+
+fg_status launch_pair(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(2 * p.n_tiles, p.t_tiles, p.splits);
+  lc.blockDim = dim3(kThreads, 1, 1);
+  lc.dynamicSmemBytes = kPairSmem;
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = p.splits;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  fg_status rc = fg_cuda_check(cudaLaunchKernelEx(&lc, w4a16_gemm_pair_kernel, map, a));
+  if (rc != FG_OK) return rc;
+  return fg_launch_check();
+}
+
 }  // namespace
 
 // No global scratch: split-k partial sums are reduced inside the cluster.
@@ -436,13 +808,18 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
   if (M == 0) return FG_OK;
   (void)workspace;
   (void)ws_bytes;
-  Plan p = make_plan(M, N, K);
+  const bool pair = M > 256;
+  if (pair) {
+    fg_status rc = pair_attr_once();
+    if (rc != FG_OK) return rc;
+  }
+  Plan p = pair ? make_pair_plan(M, N, K) : make_plan(M, N, K);
   EncodeTiledFn enc = encode_fn();
   if (!enc) return FG_ERR_CUDA;
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t box[2] = {kBK, static_cast<cuuint32_t>(p.nt)};
+  const cuuint32_t box[2] = {kBK, static_cast<cuuint32_t>(pair ? 128 : p.nt)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<fg_half *>(x), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -464,6 +841,7 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
   a.splits = p.splits;
   a.err = fg_error_word_ptr();
   if (!a.err) return FG_ERR_CUDA;
+  if (pair) return launch_pair(map, a, p, st);
   switch (p.nt) {
     case 16: return launch_nt<16>(map, a, p, st);
     case 32: return launch_nt<32>(map, a, p, st);
@@ -487,7 +865,7 @@ extern "C" fg_status fg_linear_w4a16(const fg_half *x, int M, int K, const fg_qt
   if (M == 0) return FG_OK;
   if (!x || !y || !w->codes || !w->mins || !w->scales) return FG_ERR_INVALID;
   if (!fg_aligned16(x) || !fg_aligned16(y) || !fg_aligned16(w->codes)) return FG_ERR_INVALID;
-  if ((flags & FG_EPI_RESIDUAL) && !residual) return FG_ERR_INVALID;
+  if ((flags & FG_EPI_RESIDUAL) && (!residual || !fg_aligned16(residual))) return FG_ERR_INVALID;
   return fg_linear_launch(x, M, K, w, bias, residual, flags, qscale_cols, qscale, y, workspace, workspace_bytes,
                           static_cast<cudaStream_t>(stream));
 }

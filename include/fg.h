@@ -171,9 +171,10 @@ enum {
  * fp16 output.  x: fp16 device [M][K]; w: packed along K, shape [N][K]
  * (PyTorch Linear orientation); bias: fp16 [N] or NULL; residual: fp16 [M][N]
  * (with FG_EPI_RESIDUAL); the first qscale_cols outputs of each row are
- * multiplied by qscale after the bias.  K % 64 == 0, N % 128 == 0.
- * workspace: device scratch of fg_linear_workspace_bytes(M, N, K) bytes
- * (split-K partial sums and tile counters; may be NULL when that is 0).
+ * multiplied by qscale after the bias.  K % 64 == 0, N % 128 == 0; x, y, the
+ * codes and the residual 16-byte aligned (FG_ERR_INVALID otherwise).
+ * workspace: device scratch of fg_linear_workspace_bytes(M, N, K) bytes, which
+ * is 0 (split-K partial sums are reduced on chip); may be NULL.
  * Tensor cores dequantise W tiles in shared memory ([G3]: on-the-fly
  * dequantisation for FP16 compute). */
 FG_API size_t fg_linear_workspace_bytes(int M, int N, int K);

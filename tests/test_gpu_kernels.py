@@ -198,7 +198,11 @@ def test_attention_prompt_rows_causal():
 # ------------------------------------------------------------------ linear -------------
 
 @pytest.mark.parametrize("M,N,K", [(1, 128, 64), (4, 256, 768), (16, 384, 128), (17, 256, 192), (100, 512, 1024),
-                                   (256, 768, 768), (300, 1280, 512), (512, 2304, 768), (40, 768, 3072)])
+                                   (256, 768, 768), (300, 1280, 512), (512, 2304, 768), (40, 768, 3072),
+                                   # M > 256: two-SM (CTA pair) tiles of 256 features x 512 tokens, with a
+                                   # ragged last token tile, a last pair holding only 128 features, and
+                                   # (long k) the split-k cluster reduction
+                                   (257, 256, 128), (600, 640, 2048), (1100, 384, 1024), (520, 640, 4096)])
 def test_linear_matches_oracle(M, N, K):
     x = si.normal_f16(14, 1, (M, K), 1.0)
     w16 = si.normal_f16(14, 2, (N, K), 0.02)
@@ -210,8 +214,9 @@ def test_linear_matches_oracle(M, N, K):
     assert err <= 2e-3 * np.max(np.abs(ref)), err
 
 
-def test_linear_epilogues():
-    M, N, K = 70, 512, 256
+@pytest.mark.parametrize("M,K", [(70, 256), (300, 256), (300, 2048)])
+def test_linear_epilogues(M, K):
+    N = 512
     x = si.normal_f16(15, 1, (M, K), 1.0)
     w16 = si.normal_f16(15, 2, (N, K), 0.05)
     b = si.normal_f16(15, 3, (N,), 0.1)
