@@ -338,8 +338,9 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
 //   warps 0..7   dequantise (thread: row tid % 128, k half tid / 128), then the epilogue
 //                (warp: TMEM lane quarter warp % 4, token tile warp / 4);
 //   warp 8       TMA of this CTA's x halves, completing on the even CTA's barrier;
-//   warp 9       even CTA: the MMA issuer; odd CTA: forwards "A half ready" per stage (one
-//                cluster-scope release instead of one per dequant warp); TMEM allocation.
+//   warp 9       even CTA: the MMA issuer; TMEM allocation in both;
+//   warps 9..12  odd CTA: forward "A half ready" to the even CTA, one stage each (one
+//                cluster-scope release per stage instead of one per dequant warp).
 //   Split k-ranges of one pair tile form the cluster's z dimension (cluster 2 x 1 x splits);
 //   partial sums are reduced over distributed shared memory in z-rank order.
 // ------------------------------------------------------------------------------------
@@ -354,8 +355,13 @@ constexpr int kPairSmem = kPairRing + 1024;
 constexpr int kPairCols = 512;
 constexpr int kPairPrefetch = 4;
 constexpr uint32_t kPairIdesc = umma_idesc_f16_f32(256, 256);
+// warps 0..7 dequant + epilogue, 8 TMA, 9 MMA issuer (even CTA) / TMEM allocation, and in
+// the odd CTA warps 9 .. 9 + kPairStages - 1 forward "A half ready", one stage each: a
+// cluster-scope release arrive occupies its thread for about a k-tile, so one forwarder
+// for all stages would set the pace of the pipeline.
+constexpr int kPairThreads = (kDeqWarps + 1 + kPairStages) * 32;
 
-__global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_pair_kernel(const __grid_constant__ CUtensorMap xmap,
+__global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                       const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -476,15 +482,16 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_pair_kernel(const __gr
     }
   } else if (!leader) {
     // ---------------- odd CTA: forward "A half ready" to the even CTA ----------------
-    // One cluster-scope release per stage instead of one per dequant warp.
-    if (lane == 0) {
-      for (int i = 0; i < nk; i++) {
-        const int st = i % kPairStages;
-        if (!mbar_wait_bounded(smem_u32(&a_half[st]), (i / kPairStages) & 1, abortp, a.err)) break;
+    // Warp 9 + st forwards stage st: one cluster-scope release per stage, up to kPairStages
+    // of them in flight.
+    const int st = warp - kMmaWarp;
+    if (lane == 0 && st < kPairStages) {
+      for (int i = st; i < nk; i += kPairStages) {
+        if (!mbar_poll_bounded<false>(smem_u32(&a_half[st]), (i / kPairStages) & 1, abortp, a.err)) break;
         mbar_arrive_cluster(mapa_shared(smem_u32(&full[st]), lead));
       }
     }
-  } else {
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer (even CTA) ----------------
     // Kept lean: one wait, 8 MMAs and one commit per stage, descriptors precomputed (the
     // 14-bit start-address field advances by 2 per 32-byte k step without carrying).
@@ -494,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_pair_kernel(const __gr
       constexpr uint64_t kStageStep = kPairStage >> 4, kTileStep = kPairBHalf >> 4;
       for (int i = 0; i < nk; i++) {
         const int st = i % kPairStages;
-        if (!mbar_wait_bounded_cluster(smem_u32(&full[st]), (i / kPairStages) & 1, abortp, a.err)) break;
+        if (!mbar_poll_bounded<true>(smem_u32(&full[st]), (i / kPairStages) & 1, abortp, a.err)) break;
         tc_fence_after();
         const uint64_t ad = adesc0 + st * kStageStep, bd = bdesc0 + st * kStageStep;
 #pragma unroll
@@ -720,7 +727,7 @@ int pair_clusters_resident(int splits) {
   if (!known[dev][splits]) {
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(2, 1, splits);
-    lc.blockDim = dim3(kThreads, 1, 1);
+    lc.blockDim = dim3(kPairThreads, 1, 1);
     lc.dynamicSmemBytes = kPairSmem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -781,7 +788,7 @@ fg_status pair_attr_once() {
 fg_status launch_pair(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st) {
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(2 * p.n_tiles, p.t_tiles, p.splits);
-  lc.blockDim = dim3(kThreads, 1, 1);
+  lc.blockDim = dim3(kPairThreads, 1, 1);
   lc.dynamicSmemBytes = kPairSmem;
   lc.stream = st;
   cudaLaunchAttribute attr[1];

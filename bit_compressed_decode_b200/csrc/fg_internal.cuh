@@ -239,6 +239,52 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Non-blocking phase test (no suspension), acquire at CTA or cluster scope.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait by polling, for a thread that has its warp to itself and must react to the
+// phase change at once (try_wait may suspend the thread past the completion).
+template <bool kCluster>
+__device__ __forceinline__ bool mbar_poll_bounded(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                                  unsigned int *err) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; it++) {
+    if (kCluster ? mbar_test_wait_cluster(bar, parity) : mbar_test_wait(bar, parity)) return true;
+    if ((it & 63u) == 63u) {
+      if (abort_flag && *abort_flag) return false;
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > FG_WAIT_TIMEOUT_NS) {
+        if (abort_flag) *abort_flag = 1;
+        if (err) atomicOr(err, FG_DEVERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
 // ---- CTA pairs (cta_group::2): one MMA spans the tensor cores of two SMs --------------
 // The pair is two CTAs of a cluster with ranks 2p and 2p+1; the even CTA issues the MMAs.
 // A (M = 256) is split by rows (128 per CTA), B by columns (N/2 per CTA), and each CTA's
