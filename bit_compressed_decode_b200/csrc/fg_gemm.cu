@@ -356,20 +356,22 @@ constexpr int kPairCols = 512;
 constexpr int kPairPrefetch = 4;
 constexpr uint32_t kPairIdesc = umma_idesc_f16_f32(256, 256);
 // warps 0..7 dequant + epilogue, 8 TMA, 9 MMA issuer (even CTA) / TMEM allocation, and in
-// the odd CTA warps 9 .. 9 + kPairStages - 1 forward "A half ready", one stage each: a
-// cluster-scope release arrive occupies its thread for about a k-tile, so one forwarder
-// for all stages would set the pace of the pipeline.
+// the odd CTA warps 9 .. 9 + kPairStages - 1 forward "A half ready", one stage each.
 constexpr int kPairThreads = (kDeqWarps + 1 + kPairStages) * 32;
 
 __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                       const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // full (even CTA): the stage is ready -- its 8 dequant warps, the odd CTA's forwarded
-  // "A half done", and its TMA arrival carrying the x bytes of both CTAs (one wait per stage
-  // for the MMA thread, whose issue rate bounds the kernel); a_half (odd CTA): its 8
-  // dequant warps are done; empty: the pair's MMAs are done with the stage.
+  // full (even CTA): the stage is ready -- its 8 dequant warps arrive, its TMA thread
+  // arrives expecting the x bytes of both CTAs plus the 16 bytes of the odd CTA's "A half
+  // done" token (one wait per stage for the MMA thread, whose issue rate bounds the
+  // kernel); a_half (odd CTA): its 8 dequant warps are done; empty: the pair's MMAs are
+  // done with the stage.  The odd CTA signals with a 16-byte bulk copy into the even CTA
+  // rather than a remote arrive: a remote mbarrier arrive took over a microsecond to land,
+  // the bulk copy's completion a few hundred nanoseconds.
   __shared__ __align__(8) uint64_t full[kPairStages], a_half[kPairStages], empty[kPairStages], accum_bar;
+  __shared__ __align__(16) uint32_t token_src[4], token_sink[kPairStages][4];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -392,7 +394,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
 
   if (tid == 0) {
     for (int i = 0; i < kPairStages; i++) {
-      mbar_init(smem_u32(&full[i]), kDeqWarps + 2);  // 8 local warps + odd CTA + TMA
+      mbar_init(smem_u32(&full[i]), kDeqWarps + 1);  // 8 local warps + TMA (odd CTA: tx bytes)
       mbar_init(smem_u32(&a_half[i]), kDeqWarps);
       mbar_init(smem_u32(&empty[i]), 1);
     }
@@ -474,7 +476,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
             !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kPairStages) - 1) & 1, abortp, a.err))
           break;
         const uint32_t fb = mapa_shared(smem_u32(&full[st]), lead);
-        if (leader) mbar_arrive_expect_tx(smem_u32(&full[st]), 4 * kPairBHalf);  // both CTAs, both tiles
+        if (leader) mbar_arrive_expect_tx(smem_u32(&full[st]), 4 * kPairBHalf + 16);  // x of both CTAs + token
 #pragma unroll
         for (int tile = 0; tile < 2; tile++)
           tma_load_2d_pair(smem_u32(b_tile(st, tile)), &xmap, (kt0 + i) * kBK, t0 + tile * 256 + half * 128, fb);
@@ -482,13 +484,15 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     }
   } else if (!leader) {
     // ---------------- odd CTA: forward "A half ready" to the even CTA ----------------
-    // Warp 9 + st forwards stage st: one cluster-scope release per stage, up to kPairStages
-    // of them in flight.
+    // Warp 9 + st forwards stage st.  Ordering: the dequant warps' proxy fence and release
+    // (a_half), this thread's acquire, then the bulk copy whose completion the even CTA
+    // acquires at cluster scope before its MMAs read this CTA's A half.
     const int st = warp - kMmaWarp;
     if (lane == 0 && st < kPairStages) {
       for (int i = st; i < nk; i += kPairStages) {
-        if (!mbar_poll_bounded<false>(smem_u32(&a_half[st]), (i / kPairStages) & 1, abortp, a.err)) break;
-        mbar_arrive_cluster(mapa_shared(smem_u32(&full[st]), lead));
+        if (!mbar_wait_bounded(smem_u32(&a_half[st]), (i / kPairStages) & 1, abortp, a.err)) break;
+        bulk_s2s_cluster(mapa_shared(smem_u32(&token_sink[st][0]), lead), smem_u32(&token_src[0]), 16,
+                         mapa_shared(smem_u32(&full[st]), lead));
       }
     }
   } else if (warp == kMmaWarp) {
