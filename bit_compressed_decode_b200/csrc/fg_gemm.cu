@@ -521,28 +521,63 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     }
   }
 
-  // ---------------- epilogue: TMEM -> shared memory -> (cluster sum) -> global ----------------
-  // The 128 x 512 fp32 accumulator goes through the idle ring buffers kRound chunks of
-  // [32 tokens][128 features] at a time.  Chunk ch is finished by z rank ch % splits, which
-  // sums it over the cluster's z ranks in rank order (deterministic; with one split, its own
-  // copy) and writes 8 consecutive features per thread: 16-byte stores covering whole
-  // 256-byte row segments of y.  All threads of all CTAs take the same barriers.
+  // ---------------- epilogue: TMEM -> shared memory -> global ----------------
+  // The 128 x 512 fp32 accumulator is transposed through the idle ring buffers so that every
+  // thread writes 8 consecutive features (16-byte stores covering whole 256-byte row
+  // segments of y).  Without a residual or a k split, bias, q-scale and ReLU are applied
+  // straight out of TMEM (a thread holds one feature) and only fp16 is staged; otherwise
+  // fp32 chunks of [32 tokens][128 features] are staged kRound at a time and chunk ch is
+  // finished by z rank ch % splits, which sums it over the cluster's z ranks in rank order
+  // (deterministic) before the epilogue.  All threads of all CTAs take the same barriers.
   bool ready = false;
   if (warp < kDeqWarps) {
     ready = mbar_wait_bounded_cluster(smem_u32(&accum_bar), 0, nullptr, a.err) && !*abortp;
     tc_fence_after();
   }
-  {
+  const int q = warp & 3, etile = (warp >> 2) & 1;
+  // finishing thread: 8 features f8 .. f8+7, tokens mj0 + 16 it of a 32-token chunk
+  const int f8 = (tid & 15) * 8, mj0 = (tid >> 4) & 15;
+  const int nb = n0 + f8;
+  if (a.splits == 1 && !a.res) {
+    __half *hbuf = reinterpret_cast<__half *>(smem);  // [16 chunks][32 tokens][128 features]
+    if (warp < kDeqWarps) {
+      const int n = n0 + q * 32 + lane;
+      const float bias = (a.bias && n < a.N) ? __half2float(a.bias[n]) : 0.f;
+      const float qs = n < a.qcols ? a.qscale : 1.f;
+      for (int c8 = 0; c8 < 8; c8++) {
+        const int ch = etile * 8 + c8;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, v);
+        tmem_wait_ld();
+        __half *cb = hbuf + ch * (32 * 128) + q * 32 + lane;
+#pragma unroll
+        for (int j = 0; j < 32; j++) {
+          float y = (__uint_as_float(v[j]) + bias) * qs;
+          if (a.relu) y = fmaxf(y, 0.f);
+          cb[j * 128] = __float2half_rn(y);
+        }
+      }
+    }
+    __syncthreads();
+    if (warp < kDeqWarps && ready && nb < a.N) {
+#pragma unroll 4
+      for (int ch = 0; ch < kPairCols / 32; ch++) {
+#pragma unroll
+        for (int it = 0; it < 2; it++) {
+          const int mj = mj0 + 16 * it, m = t0 + ch * 32 + mj;
+          const uint4 ov = *reinterpret_cast<const uint4 *>(hbuf + ch * (32 * 128) + mj * 128 + f8);
+          if (m < a.M) *reinterpret_cast<uint4 *>(a.y + static_cast<int64_t>(m) * a.N + nb) = ov;
+        }
+      }
+    }
+    __syncthreads();
+  } else {
     constexpr int kChunkFloats = 32 * 128;
     constexpr int kRound = kPairRing / (kChunkFloats * 4);  // 12 chunks of the 16
     constexpr int kChunks = kPairCols / 32;
-    const int q = warp & 3, etile = (warp >> 2) & 1;
     const int zrank = static_cast<int>(crank >> 1);
     const bool clustered = a.splits > 1;
     float *buf = reinterpret_cast<float *>(smem);
-    // finishing thread: 8 features f8 .. f8+7 of rows (tokens) mj0 and mj0 + 16 of a chunk
-    const int f8 = (tid & 15) * 8, mj0 = (tid >> 4) & 15;
-    const int nb = n0 + f8;
     float bias[8];
 #pragma unroll
     for (int u = 0; u < 8; u++) bias[u] = (a.bias && warp < kDeqWarps && nb < a.N) ? __half2float(a.bias[nb + u]) : 0.f;
@@ -565,23 +600,30 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
         for (int ch = r0; ch < r0 + kRound && ch < kChunks; ch++) {
           if (ch % a.splits != zrank) continue;
           float acc[2][8];
+          const float *own = buf + (ch - r0) * kChunkFloats + mj0 * 128 + f8;
 #pragma unroll
-          for (int it = 0; it < 2; it++)
+          for (int it = 0; it < 2; it++) {
+            const float4 p0 = *reinterpret_cast<const float4 *>(own + it * 16 * 128);
+            const float4 p1 = *reinterpret_cast<const float4 *>(own + it * 16 * 128 + 4);
+            acc[it][0] = p0.x; acc[it][1] = p0.y; acc[it][2] = p0.z; acc[it][3] = p0.w;
+            acc[it][4] = p1.x; acc[it][5] = p1.y; acc[it][6] = p1.z; acc[it][7] = p1.w;
+          }
+          if (clustered) {
+            // the sum restarts from rank 0 so that every split's rank order is the same
+            const uint32_t off = smem_u32(own);
 #pragma unroll
-            for (int u = 0; u < 8; u++) acc[it][u] = 0.f;
-          const uint32_t off = smem_u32(buf + (ch - r0) * kChunkFloats + mj0 * 128 + f8);
-          for (int z = 0; z < a.splits; z++) {  // z-rank order
-            const uint32_t rb = clustered ? mapa_shared(off, (crank & 1u) + 2u * z) : off;
+            for (int it = 0; it < 2; it++)
 #pragma unroll
-            for (int it = 0; it < 2; it++) {
-              const float4 p0 = clustered ? ld_shared_cluster_v4(rb + it * 16 * 128 * 4)
-                                          : *reinterpret_cast<const float4 *>(buf + (ch - r0) * kChunkFloats +
-                                                                              (mj0 + 16 * it) * 128 + f8);
-              const float4 p1 = clustered ? ld_shared_cluster_v4(rb + it * 16 * 128 * 4 + 16)
-                                          : *reinterpret_cast<const float4 *>(buf + (ch - r0) * kChunkFloats +
-                                                                              (mj0 + 16 * it) * 128 + f8 + 4);
-              acc[it][0] += p0.x; acc[it][1] += p0.y; acc[it][2] += p0.z; acc[it][3] += p0.w;
-              acc[it][4] += p1.x; acc[it][5] += p1.y; acc[it][6] += p1.z; acc[it][7] += p1.w;
+              for (int u = 0; u < 8; u++) acc[it][u] = 0.f;
+            for (int z = 0; z < a.splits; z++) {  // z-rank order
+              const uint32_t rb = mapa_shared(off, (crank & 1u) + 2u * z);
+#pragma unroll
+              for (int it = 0; it < 2; it++) {
+                const float4 p0 = ld_shared_cluster_v4(rb + it * 16 * 128 * 4);
+                const float4 p1 = ld_shared_cluster_v4(rb + it * 16 * 128 * 4 + 16);
+                acc[it][0] += p0.x; acc[it][1] += p0.y; acc[it][2] += p0.z; acc[it][3] += p0.w;
+                acc[it][4] += p1.x; acc[it][5] += p1.y; acc[it][6] += p1.z; acc[it][7] += p1.w;
+              }
             }
           }
           uint4 rv[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
