@@ -338,9 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
 //   warps 0..7   dequantise (thread: row tid % 128, k half tid / 128), then the epilogue
 //                (warp: TMEM lane quarter warp % 4, token tile warp / 4);
 //   warp 8       TMA of this CTA's x halves, completing on the even CTA's barrier;
-//   warp 9       even CTA: the MMA issuer; TMEM allocation in both;
-//   warps 9..12  odd CTA: forward "A half ready" to the even CTA, one stage each (one
-//                cluster-scope release per stage instead of one per dequant warp).
+//   warp 9       even CTA: the MMA issuer; odd CTA: forwards "A half ready" to the even
+//                CTA (a 16-byte bulk copy completing on its barrier); TMEM allocation.
 //   Split k-ranges of one pair tile form the cluster's z dimension (cluster 2 x 1 x splits);
 //   partial sums are reduced over distributed shared memory in z-rank order.
 // ------------------------------------------------------------------------------------
@@ -355,9 +354,10 @@ constexpr int kPairSmem = kPairRing + 1024;
 constexpr int kPairCols = 512;
 constexpr int kPairPrefetch = 4;
 constexpr uint32_t kPairIdesc = umma_idesc_f16_f32(256, 256);
-// warps 0..7 dequant + epilogue, 8 TMA, 9 MMA issuer (even CTA) / TMEM allocation, and in
-// the odd CTA warps 9 .. 9 + kPairStages - 1 forward "A half ready", one stage each.
-constexpr int kPairThreads = (kDeqWarps + 1 + kPairStages) * 32;
+// warps 0..7 dequant + epilogue, 8 TMA, 9 MMA issuer (even CTA) or "A half ready"
+// forwarder (odd CTA), and TMEM allocation.  Ten warps leave room for ~168 registers per
+// thread (the register file is split over the four schedulers).
+constexpr int kPairThreads = (kDeqWarps + 2) * 32;
 
 __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                       const GemmArgs a) {
@@ -484,12 +484,13 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     }
   } else if (!leader) {
     // ---------------- odd CTA: forward "A half ready" to the even CTA ----------------
-    // Warp 9 + st forwards stage st.  Ordering: the dequant warps' proxy fence and release
-    // (a_half), this thread's acquire, then the bulk copy whose completion the even CTA
-    // acquires at cluster scope before its MMAs read this CTA's A half.
-    const int st = warp - kMmaWarp;
-    if (lane == 0 && st < kPairStages) {
-      for (int i = st; i < nk; i += kPairStages) {
+    // Warp 9 forwards every stage; the bulk copy does not hold the thread.  Ordering: the
+    // dequant warps' proxy fence and release (a_half), this thread's acquire, then the bulk
+    // copy whose completion the even CTA acquires at cluster scope before its MMAs read
+    // this CTA's A half.
+    if (warp == kMmaWarp && lane == 0) {
+      for (int i = 0; i < nk; i++) {
+        const int st = i % kPairStages;
         if (!mbar_wait_bounded(smem_u32(&a_half[st]), (i / kPairStages) & 1, abortp, a.err)) break;
         bulk_s2s_cluster(mapa_shared(smem_u32(&token_sink[st][0]), lead), smem_u32(&token_src[0]), 16,
                          mapa_shared(smem_u32(&full[st]), lead));
@@ -583,9 +584,8 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     for (int u = 0; u < 8; u++) bias[u] = (a.bias && warp < kDeqWarps && nb < a.N) ? __half2float(a.bias[nb + u]) : 0.f;
     for (int r0 = 0; r0 < kChunks; r0 += kRound) {
       if (warp < kDeqWarps) {
-        for (int c8 = 0; c8 < 8; c8++) {
-          const int ch = etile * 8 + c8;
-          if (ch < r0 || ch >= r0 + kRound) continue;
+        // warps q and q + 4 share TMEM lanes 32q..32q+31 and take alternate chunks
+        for (int ch = r0 + etile; ch < r0 + kRound && ch < kChunks; ch += 2) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, v);
           tmem_wait_ld();
@@ -597,52 +597,89 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
       __syncwarp();
       if (clustered) cluster_sync_all(); else __syncthreads();
       if (warp < kDeqWarps && ready && nb < a.N) {
-        for (int ch = r0; ch < r0 + kRound && ch < kChunks; ch++) {
-          if (ch % a.splits != zrank) continue;
-          float acc[2][8];
-          const float *own = buf + (ch - r0) * kChunkFloats + mj0 * 128 + f8;
+        // this rank's chunks of the round: ch = zrank + kk * splits; their residual rows are
+        // all requested first, so their memory latency overlaps instead of adding up
+        constexpr int kOwnMax = 6;  // chunks of a 12-chunk round owned by one rank, splits >= 2
+        const int nown = clustered ? kOwnMax : kRound;
+        // first chunk of the round owned by this rank
+        const int ch0 = clustered ? r0 + ((zrank - r0 % a.splits) + a.splits) % a.splits : r0;
+        uint4 resv[kOwnMax][2];
+#pragma unroll
+        for (int kk = 0; kk < kOwnMax; kk++) {
+          const int ch = ch0 + kk * a.splits;
 #pragma unroll
           for (int it = 0; it < 2; it++) {
-            const float4 p0 = *reinterpret_cast<const float4 *>(own + it * 16 * 128);
-            const float4 p1 = *reinterpret_cast<const float4 *>(own + it * 16 * 128 + 4);
-            acc[it][0] = p0.x; acc[it][1] = p0.y; acc[it][2] = p0.z; acc[it][3] = p0.w;
-            acc[it][4] = p1.x; acc[it][5] = p1.y; acc[it][6] = p1.z; acc[it][7] = p1.w;
+            const int m = t0 + ch * 32 + mj0 + 16 * it;
+            resv[kk][it] = (clustered && a.res && ch < r0 + kRound && ch < kChunks && m < a.M)
+                               ? *reinterpret_cast<const uint4 *>(a.res + static_cast<int64_t>(m) * a.N + nb)
+                               : make_uint4(0, 0, 0, 0);
           }
-          if (clustered) {
-            // the sum restarts from rank 0 so that every split's rank order is the same
-            const uint32_t off = smem_u32(own);
+        }
+        // one owned chunk per pass: both items' partial loads (every rank) are in flight
+        // together before either is summed
+        for (int kk = 0; kk < nown; kk++) {
+          float4 part[1][2][4][2];  // [chunk][item][rank][half]
 #pragma unroll
-            for (int it = 0; it < 2; it++)
+          for (int c2 = 0; c2 < 1; c2++) {
+            const int ch = clustered ? ch0 + (kk + c2) * a.splits : r0 + kk + c2;
+            if (ch >= r0 + kRound || ch >= kChunks) continue;
+            const float *own = buf + (ch - r0) * kChunkFloats + mj0 * 128 + f8;
 #pragma unroll
-              for (int u = 0; u < 8; u++) acc[it][u] = 0.f;
-            for (int z = 0; z < a.splits; z++) {  // z-rank order
-              const uint32_t rb = mapa_shared(off, (crank & 1u) + 2u * z);
+            for (int it = 0; it < 2; it++) {
+              if (clustered) {
+                const uint32_t off = smem_u32(own + it * 16 * 128);
 #pragma unroll
-              for (int it = 0; it < 2; it++) {
-                const float4 p0 = ld_shared_cluster_v4(rb + it * 16 * 128 * 4);
-                const float4 p1 = ld_shared_cluster_v4(rb + it * 16 * 128 * 4 + 16);
-                acc[it][0] += p0.x; acc[it][1] += p0.y; acc[it][2] += p0.z; acc[it][3] += p0.w;
-                acc[it][4] += p1.x; acc[it][5] += p1.y; acc[it][6] += p1.z; acc[it][7] += p1.w;
+                for (int z = 0; z < 4; z++) {
+                  if (z < a.splits) {
+                    const uint32_t rb = mapa_shared(off, (crank & 1u) + 2u * z);
+                    part[c2][it][z][0] = ld_shared_cluster_v4(rb);
+                    part[c2][it][z][1] = ld_shared_cluster_v4(rb + 16);
+                  }
+                }
+              } else {
+                part[c2][it][0][0] = *reinterpret_cast<const float4 *>(own + it * 16 * 128);
+                part[c2][it][0][1] = *reinterpret_cast<const float4 *>(own + it * 16 * 128 + 4);
               }
             }
           }
-          uint4 rv[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
 #pragma unroll
-          for (int it = 0; it < 2; it++) {
-            const int m = t0 + ch * 32 + mj0 + 16 * it;
-            if (a.res && m < a.M) rv[it] = *reinterpret_cast<const uint4 *>(a.res + static_cast<int64_t>(m) * a.N + nb);
-          }
+          for (int c2 = 0; c2 < 1; c2++) {
+            const int kc = kk + c2;
+            const int ch = clustered ? ch0 + kc * a.splits : r0 + kc;
+            if (ch >= r0 + kRound || ch >= kChunks) continue;
 #pragma unroll
-          for (int it = 0; it < 2; it++) {
-            const int m = t0 + ch * 32 + mj0 + 16 * it;
-            if (m >= a.M) continue;
-            const __half *rh = reinterpret_cast<const __half *>(&rv[it]);
-            uint4 ov;
-            __half *oh = reinterpret_cast<__half *>(&ov);
+            for (int it = 0; it < 2; it++) {
+              const int m = t0 + ch * 32 + mj0 + 16 * it;
+              if (m >= a.M) continue;
+              // summed from rank 0 up: the same order for every output
+              float acc[8];
 #pragma unroll
-            for (int u = 0; u < 8; u++)
-              oh[u] = __float2half_rn(epilogue(acc[it][u], bias[u], __half2float(rh[u]), nb + u, a));
-            *reinterpret_cast<uint4 *>(a.y + static_cast<int64_t>(m) * a.N + nb) = ov;
+              for (int u = 0; u < 8; u++) acc[u] = 0.f;
+              const int nz = clustered ? a.splits : 1;
+#pragma unroll
+              for (int z = 0; z < 4; z++) {
+                if (z < nz) {
+                  const float4 p0 = part[c2][it][z][0], p1 = part[c2][it][z][1];
+                  acc[0] += p0.x; acc[1] += p0.y; acc[2] += p0.z; acc[3] += p0.w;
+                  acc[4] += p1.x; acc[5] += p1.y; acc[6] += p1.z; acc[7] += p1.w;
+                }
+              }
+              uint4 rv = make_uint4(0, 0, 0, 0);
+              if (clustered) {
+#pragma unroll
+                for (int k2 = 0; k2 < kOwnMax; k2++)
+                  if (k2 == kc) rv = resv[k2][it];
+              } else if (a.res) {
+                rv = *reinterpret_cast<const uint4 *>(a.res + static_cast<int64_t>(m) * a.N + nb);
+              }
+              const __half *rh = reinterpret_cast<const __half *>(&rv);
+              uint4 ov;
+              __half *oh = reinterpret_cast<__half *>(&ov);
+#pragma unroll
+              for (int u = 0; u < 8; u++)
+                oh[u] = __float2half_rn(epilogue(acc[u], bias[u], __half2float(rh[u]), nb + u, a));
+              *reinterpret_cast<uint4 *>(a.y + static_cast<int64_t>(m) * a.N + nb) = ov;
+            }
           }
         }
       }
