@@ -372,6 +372,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
   // the bulk copy's completion a few hundred nanoseconds.
   __shared__ __align__(8) uint64_t full[kPairStages], a_half[kPairStages], empty[kPairStages], accum_bar;
   __shared__ __align__(16) uint32_t token_src[4], token_sink[kPairStages][4];
+  __shared__ __align__(8) uint64_t recv_bar;  // split-k epilogue: this rank's received partials
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -399,6 +400,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
       mbar_init(smem_u32(&empty[i]), 1);
     }
     mbar_init(smem_u32(&accum_bar), 1);
+    mbar_init(smem_u32(&recv_bar), 1);
     abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -572,12 +574,11 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
       }
     }
     __syncthreads();
-  } else {
+  } else if (a.splits == 1) {
+    // residual, no k split: fp32 chunks staged kRound at a time, finished by this CTA
     constexpr int kChunkFloats = 32 * 128;
     constexpr int kRound = kPairRing / (kChunkFloats * 4);  // 12 chunks of the 16
     constexpr int kChunks = kPairCols / 32;
-    const int zrank = static_cast<int>(crank >> 1);
-    const bool clustered = a.splits > 1;
     float *buf = reinterpret_cast<float *>(smem);
     float bias[8];
 #pragma unroll
@@ -594,85 +595,121 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
           for (int j = 0; j < 32; j++) cbuf[j * 128 + q * 32 + lane] = __uint_as_float(v[j]);
         }
       }
-      __syncwarp();
-      if (clustered) cluster_sync_all(); else __syncthreads();
+      __syncthreads();
       if (warp < kDeqWarps && ready && nb < a.N) {
-        // this rank's chunks of the round: ch = zrank + kk * splits; their residual rows are
-        // all requested first, so their memory latency overlaps instead of adding up
-        constexpr int kOwnMax = 6;  // chunks of a 12-chunk round owned by one rank, splits >= 2
-        const int nown = clustered ? kOwnMax : kRound;
-        // first chunk of the round owned by this rank
-        const int ch0 = clustered ? r0 + ((zrank - r0 % a.splits) + a.splits) % a.splits : r0;
-        uint4 resv[kOwnMax][2];
-#pragma unroll
-        for (int kk = 0; kk < kOwnMax; kk++) {
-          const int ch = ch0 + kk * a.splits;
+        for (int ch = r0; ch < r0 + kRound && ch < kChunks; ch++) {
+          const float *own = buf + (ch - r0) * kChunkFloats + mj0 * 128 + f8;
+          uint4 rv[2];
 #pragma unroll
           for (int it = 0; it < 2; it++) {
             const int m = t0 + ch * 32 + mj0 + 16 * it;
-            resv[kk][it] = (clustered && a.res && ch < r0 + kRound && ch < kChunks && m < a.M)
-                               ? *reinterpret_cast<const uint4 *>(a.res + static_cast<int64_t>(m) * a.N + nb)
-                               : make_uint4(0, 0, 0, 0);
+            rv[it] = (a.res && m < a.M) ? *reinterpret_cast<const uint4 *>(a.res + static_cast<int64_t>(m) * a.N + nb)
+                                        : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int it = 0; it < 2; it++) {
+            const int m = t0 + ch * 32 + mj0 + 16 * it;
+            if (m >= a.M) continue;
+            const float4 p0 = *reinterpret_cast<const float4 *>(own + it * 16 * 128);
+            const float4 p1 = *reinterpret_cast<const float4 *>(own + it * 16 * 128 + 4);
+            const float acc[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            const __half *rh = reinterpret_cast<const __half *>(&rv[it]);
+            uint4 ov;
+            __half *oh = reinterpret_cast<__half *>(&ov);
+#pragma unroll
+            for (int u = 0; u < 8; u++)
+              oh[u] = __float2half_rn(epilogue(acc[u], bias[u], __half2float(rh[u]), nb + u, a));
+            *reinterpret_cast<uint4 *>(a.y + static_cast<int64_t>(m) * a.N + nb) = ov;
           }
         }
-        // one owned chunk per pass: both items' partial loads (every rank) are in flight
-        // together before either is summed
-        for (int kk = 0; kk < nown; kk++) {
-          float4 part[1][2][4][2];  // [chunk][item][rank][half]
+      }
+      __syncthreads();
+    }
+  } else {
+    // k split over the cluster's z ranks.  Per round of kR chunks every rank stages its fp32
+    // partial of each chunk, then pushes the chunks it does not own into the owner's receive
+    // slots with bulk copies (completion counted on the owner's recv_bar); the owner sums
+    // its own partial and the received ones in z-rank order (deterministic) and finishes.
+    constexpr int kChunkFloats = 32 * 128;
+    constexpr int kChunkBytes = kChunkFloats * 4;
+    constexpr int kR = 6;                                        // chunks per round
+    constexpr int kSlots = kPairRing / kChunkBytes - kR;         // receive slots: 6
+    constexpr int kChunks = kPairCols / 32;
+    constexpr int kOwnMax = 3;                                   // chunks of a round one rank owns (splits >= 2)
+    static_assert(kSlots >= 6, "a rank owns at most 2 chunks x 3 senders or 3 chunks x 1 sender per round");
+    const int S = a.splits, zrank = static_cast<int>(crank >> 1);
+    float *sendb = reinterpret_cast<float *>(smem);              // [kR] chunks
+    float *recvb = sendb + kR * kChunkFloats;                    // [kSlots] chunks
+    float bias[8];
 #pragma unroll
-          for (int c2 = 0; c2 < 1; c2++) {
-            const int ch = clustered ? ch0 + (kk + c2) * a.splits : r0 + kk + c2;
-            if (ch >= r0 + kRound || ch >= kChunks) continue;
-            const float *own = buf + (ch - r0) * kChunkFloats + mj0 * 128 + f8;
+    for (int u = 0; u < 8; u++) bias[u] = (a.bias && warp < kDeqWarps && nb < a.N) ? __half2float(a.bias[nb + u]) : 0.f;
+    auto first_owned = [&](int owner, int r0) { return r0 + ((owner - r0 % S) + S) % S; };
+    int round = 0;
+    for (int r0 = 0; r0 < kChunks; r0 += kR, round++) {
+      const int rend = min(r0 + kR, kChunks);
+      const int f0 = first_owned(zrank, r0);
+      const int nown = f0 < rend ? (rend - 1 - f0) / S + 1 : 0;
+      if (warp < kDeqWarps) {
+        for (int ch = r0 + etile; ch < rend; ch += 2) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, v);
+          tmem_wait_ld();
+          float *cbuf = sendb + (ch - r0) * kChunkFloats;
+#pragma unroll
+          for (int j = 0; j < 32; j++) cbuf[j * 128 + q * 32 + lane] = __uint_as_float(v[j]);
+        }
+        fence_proxy_async_smem();  // the staged partials are read by bulk copies
+      }
+      if (tid == 0) mbar_arrive_expect_tx(smem_u32(&recv_bar), static_cast<uint32_t>(nown * (S - 1) * kChunkBytes));
+      __syncwarp();
+      cluster_sync_all();  // staged everywhere; every receiver's slots free and its barrier armed
+      if (tid == 0) {
+        for (int ch = r0; ch < rend; ch++) {
+          const int owner = ch % S;
+          if (owner == zrank) continue;
+          const int j = (ch - first_owned(owner, r0)) / S;
+          const int slot = j * (S - 1) + (zrank < owner ? zrank : zrank - 1);
+          const uint32_t dst = (crank & 1u) + 2u * static_cast<uint32_t>(owner);
+          bulk_s2s_cluster(mapa_shared(smem_u32(recvb + slot * kChunkFloats), dst),
+                           smem_u32(sendb + (ch - r0) * kChunkFloats), kChunkBytes, mapa_shared(smem_u32(&recv_bar), dst));
+        }
+      }
+      if (warp < kDeqWarps) {
+        const bool got = mbar_wait_bounded(smem_u32(&recv_bar), round & 1, nullptr, a.err);
+        if (got && ready && nb < a.N) {
+          uint4 resv[kOwnMax][2];
+#pragma unroll
+          for (int j = 0; j < kOwnMax; j++) {
+            const int ch = f0 + j * S;
 #pragma unroll
             for (int it = 0; it < 2; it++) {
-              if (clustered) {
-                const uint32_t off = smem_u32(own + it * 16 * 128);
-#pragma unroll
-                for (int z = 0; z < 4; z++) {
-                  if (z < a.splits) {
-                    const uint32_t rb = mapa_shared(off, (crank & 1u) + 2u * z);
-                    part[c2][it][z][0] = ld_shared_cluster_v4(rb);
-                    part[c2][it][z][1] = ld_shared_cluster_v4(rb + 16);
-                  }
-                }
-              } else {
-                part[c2][it][0][0] = *reinterpret_cast<const float4 *>(own + it * 16 * 128);
-                part[c2][it][0][1] = *reinterpret_cast<const float4 *>(own + it * 16 * 128 + 4);
-              }
+              const int m = t0 + ch * 32 + mj0 + 16 * it;
+              resv[j][it] = (a.res && j < nown && m < a.M)
+                                ? *reinterpret_cast<const uint4 *>(a.res + static_cast<int64_t>(m) * a.N + nb)
+                                : make_uint4(0, 0, 0, 0);
             }
           }
 #pragma unroll
-          for (int c2 = 0; c2 < 1; c2++) {
-            const int kc = kk + c2;
-            const int ch = clustered ? ch0 + kc * a.splits : r0 + kc;
-            if (ch >= r0 + kRound || ch >= kChunks) continue;
+          for (int j = 0; j < kOwnMax; j++) {
+            if (j >= nown) continue;
+            const int ch = f0 + j * S;
 #pragma unroll
             for (int it = 0; it < 2; it++) {
               const int m = t0 + ch * 32 + mj0 + 16 * it;
               if (m >= a.M) continue;
-              // summed from rank 0 up: the same order for every output
+              const int eoff = (mj0 + 16 * it) * 128 + f8;
               float acc[8];
 #pragma unroll
               for (int u = 0; u < 8; u++) acc[u] = 0.f;
-              const int nz = clustered ? a.splits : 1;
-#pragma unroll
-              for (int z = 0; z < 4; z++) {
-                if (z < nz) {
-                  const float4 p0 = part[c2][it][z][0], p1 = part[c2][it][z][1];
-                  acc[0] += p0.x; acc[1] += p0.y; acc[2] += p0.z; acc[3] += p0.w;
-                  acc[4] += p1.x; acc[5] += p1.y; acc[6] += p1.z; acc[7] += p1.w;
-                }
+              for (int z = 0; z < S; z++) {  // z-rank order
+                const float *src = z == zrank ? sendb + (ch - r0) * kChunkFloats + eoff
+                                              : recvb + (j * (S - 1) + (z < zrank ? z : z - 1)) * kChunkFloats + eoff;
+                const float4 p0 = *reinterpret_cast<const float4 *>(src);
+                const float4 p1 = *reinterpret_cast<const float4 *>(src + 4);
+                acc[0] += p0.x; acc[1] += p0.y; acc[2] += p0.z; acc[3] += p0.w;
+                acc[4] += p1.x; acc[5] += p1.y; acc[6] += p1.z; acc[7] += p1.w;
               }
-              uint4 rv = make_uint4(0, 0, 0, 0);
-              if (clustered) {
-#pragma unroll
-                for (int k2 = 0; k2 < kOwnMax; k2++)
-                  if (k2 == kc) rv = resv[k2][it];
-              } else if (a.res) {
-                rv = *reinterpret_cast<const uint4 *>(a.res + static_cast<int64_t>(m) * a.N + nb);
-              }
-              const __half *rh = reinterpret_cast<const __half *>(&rv);
+              const __half *rh = reinterpret_cast<const __half *>(&resv[j][it]);
               uint4 ov;
               __half *oh = reinterpret_cast<__half *>(&ov);
 #pragma unroll
@@ -684,7 +721,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
         }
       }
       __syncwarp();
-      if (clustered) cluster_sync_all(); else __syncthreads();
+      cluster_sync_all();  // every push has landed: send buffers and slots can be reused
     }
   }
 

@@ -255,6 +255,25 @@ def test_linear_split_k_deterministic(M, N, K):
     assert np.max(np.abs(host(y1).astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref))
 
 
+@pytest.mark.parametrize("M,N,K", [(520, 4096, 4096), (600, 7680, 1024), (530, 5120, 1536), (512, 4096, 16384)])
+def test_linear_split_k_residual_sampled(M, N, K):
+    # output-projection / FC2 shapes with a residual: few CTA-pair tiles, so the k-range is
+    # split over a cluster and the partial sums are pushed between ranks; two runs give
+    # identical bits, and sampled rows (the oracle is slow at this size) match the oracle
+    x = si.normal_f16(18, 1, (M, K), 1.0)
+    w16 = si.normal_f16(18, 2, (N, K), 0.02)
+    b = si.normal_f16(18, 3, (N,), 0.1)
+    r = si.normal_f16(18, 4, (M, N), 1.0)
+    wq = fg.fg_quantize(dev(w16), dim=1)
+    y1 = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), residual=dev(r))
+    y2 = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), residual=dev(r))
+    assert torch.equal(y1, y2)
+    rows = np.unique(np.concatenate([np.random.default_rng(M).choice(M, 20, replace=False), [0, 255, 256, 511, M - 1]]))
+    ref = oracle.linear(x[rows], oracle.quantize(w16, 1), bias=b, residual=r[rows])
+    got = host(y1)[rows].astype(np.float64)
+    assert np.max(np.abs(got - ref)) <= 2e-3 * np.max(np.abs(ref))
+
+
 def test_linear_errors():
     x = torch.zeros((4, 64), dtype=torch.float16, device="cuda")
     w = fg.fg_quantize(torch.zeros((64, 64), dtype=torch.float16, device="cuda"), dim=1)
