@@ -438,47 +438,74 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 scale2, __half2 mi
   return r;
 }
 
+// RN(d / 15) for finite d >= 0: d * RN(1/15) corrected by one fused multiply-add on the
+// exact residual d - 15 q0 (Markstein's correction step, P. Markstein, IBM J. Res. Dev. 34,
+// 1990).  Equal to the correctly rounded quotient for every non-negative finite float
+// (checked exhaustively against __fdiv_rn on B200).
+__device__ __forceinline__ float div15_rn(float d) {
+  const float c = 0.0666666701436042785644531250f;  // RN(1/15)
+  const float q0 = __fmul_rn(d, c);
+  const float r = __fmaf_rn(-15.0f, q0, d);
+  return __fmaf_rn(r, c, q0);
+}
+
+// RN(1 / s) for s a positive finite fp16 value widened to fp32: one Newton-Raphson step with
+// a fused multiply-add on the hardware reciprocal approximation (Markstein, same reference).
+// Equal to the correctly rounded reciprocal for every such s (checked exhaustively against
+// __fdiv_rn on B200).
+__device__ __forceinline__ float rcp_rn_f16val(float s) {
+  float r0;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(s));
+  const float e = __fmaf_rn(-s, r0, 1.0f);
+  return __fmaf_rn(e, r0, r0);
+}
+
+// Insert the low 4 bits of v into w at bit position pos.
+__device__ __forceinline__ uint32_t bfi4(uint32_t v, uint32_t w, uint32_t pos) {
+  uint32_t r;
+  asm("bfi.b32 %0, %1, %2, %3, 4;" : "=r"(r) : "r"(v), "r"(w), "r"(pos));
+  return r;
+}
+
 // Cooperative quantisation of one group of 64 fp16 values held by 8 consecutive
 // lanes (lane j of the 8 holds elements 8j..8j+7 in v).  Steps and fp32 operation
 // order as stated in fg.h: min/max over the group, mn += 0, d = mx - mn,
 // scale = fp16_rn(d/15), inv = 1/scale, code = clamp(rint((x - mn) * inv), 0, 15).
+// Min and max are taken on the fp16 values (exact, as on their fp32 widenings), carried
+// between lanes as the pair {min, -max}; rint is the fp32 addition of 1.5 * 2^23 (the
+// nearest integer, ties to even, lands in the low mantissa bits; the quotient lies in
+// [0, 30] because the scale is rounded to fp16).  Inputs must be finite.
 // Returns this lane's 8 codes packed into one 32-bit word (element 8j+2i in the low
 // nibble of byte i) and the group's fp16 min and scale.  All 32 lanes of the warp
 // must call it together.
 __device__ __forceinline__ uint32_t quant_group8(const uint4 v, __half &min_h, __half &scale_h) {
-  float x[8];
-  {
-    const __half2 *h2 = reinterpret_cast<const __half2 *>(&v);
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-      float2 f = __half22float2(h2[i]);
-      x[2 * i] = f.x;
-      x[2 * i + 1] = f.y;
-    }
-  }
-  float mn = x[0], mx = x[0];
-#pragma unroll
-  for (int i = 1; i < 8; i++) {
-    mn = fminf(mn, x[i]);
-    mx = fmaxf(mx, x[i]);
-  }
+  const __half2 *h2 = reinterpret_cast<const __half2 *>(&v);
+  const __half2 lo = __hmin2(__hmin2(h2[0], h2[1]), __hmin2(h2[2], h2[3]));
+  const __half2 hi = __hmax2(__hmax2(h2[0], h2[1]), __hmax2(h2[2], h2[3]));
+  // {min, -max} of this lane's 8 values
+  __half2 mm = __halves2half2(__hmin(__low2half(lo), __high2half(lo)),
+                              __hneg(__hmax(__low2half(hi), __high2half(hi))));
 #pragma unroll
   for (int o = 1; o < 8; o <<= 1) {
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const uint32_t u = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<const uint32_t *>(&mm), o);
+    mm = __hmin2(mm, *reinterpret_cast<const __half2 *>(&u));
   }
+  float mn = __low2float(mm);
+  const float mx = -__high2float(mm);
   mn = __fadd_rn(mn, 0.0f);
   const float d = __fsub_rn(mx, mn);
-  __half sh = __float2half_rn(__fdiv_rn(d, 15.0f));
+  __half sh = __float2half_rn(div15_rn(d));
   const float s = __half2float(sh);
   uint32_t word = 0;
   if (s != 0.0f) {
-    const float inv = __fdiv_rn(1.0f, s);
+    const float inv = rcp_rn_f16val(s);
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-      int c = __float2int_rn(__fmul_rn(__fsub_rn(x[i], mn), inv));
-      c = min(max(c, 0), 15);
-      word |= static_cast<uint32_t>(c) << (4 * i);
+    for (int i = 0; i < 4; i++) {
+      const float2 f = __half22float2(h2[i]);
+      const float r0 = __fadd_rn(__fmul_rn(__fsub_rn(f.x, mn), inv), 12582912.0f);
+      const float r1 = __fadd_rn(__fmul_rn(__fsub_rn(f.y, mn), inv), 12582912.0f);
+      word = bfi4(min(__float_as_uint(r0), 0x4B40000Fu), word, 8 * i);
+      word = bfi4(min(__float_as_uint(r1), 0x4B40000Fu), word, 8 * i + 4);
     }
   } else {
     sh = __ushort_as_half(0);

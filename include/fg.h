@@ -103,7 +103,8 @@ FG_API fg_status fg_qtensor_bytes(int ndim, const int64_t *shape, int dim, int b
 
 /* Quantise fp16 `x` (device, row-major `shape`) along `dim` into out->codes,
  * out->mins, out->scales (device buffers set by the caller; their sizes from
- * fg_qtensor_bytes).  Fills out->ndim/shape/dim/bits/group.
+ * fg_qtensor_bytes).  Fills out->ndim/shape/dim/bits/group.  x must be finite
+ * (a group holding Inf or NaN gets unspecified codes).
  * Errors: FG_ERR_SHAPE if shape[dim] % 64 != 0; FG_ERR_UNSUPPORTED if
  * bits != 4 or group != 64.  [G3] */
 FG_API fg_status fg_quantize(const fg_half *x, int ndim, const int64_t *shape, int dim, int bits, int group,

@@ -72,6 +72,19 @@ def test_quantize_wide_ranges_and_specials():
     _check_quant_equal(x)
 
 
+def test_quantize_every_fp16_range_bit_exact():
+    # one group per positive finite fp16 value v: {0, v} and {-v, v} ranges with the other
+    # elements spread between them -- every reachable scale, including the fp16 subnormal
+    # ones, goes through the quantizer's division and reciprocal
+    v = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float64)
+    t = np.linspace(0.0, 1.0, 64)
+    a = (v[:, None] * t[None, :]).astype(np.float16)                  # min 0, max v
+    b = (v[:, None] * (2.0 * t[None, :] - 1.0)).astype(np.float16)    # min -v, max v
+    b[:, 0] = (-v).astype(np.float16)
+    b[:, -1] = v.astype(np.float16)
+    _check_quant_equal(np.concatenate([a, b], axis=0))
+
+
 @pytest.mark.parametrize("shape,dim", [((6, 128, 5), 1), ((64, 3), 0), ((2, 3, 192, 4), 2)])
 def test_quantize_strided_dims_bit_exact(shape, dim):
     _check_quant_equal(si.normal_f16(8, 2, shape, 1.0), dim=dim)
