@@ -9,50 +9,58 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kMaxVec = 8;  // up to 8 x 8 halves per thread: h <= 16384
 
-__device__ __forceinline__ float block_sum(float v, float *red) {
+// Sum over the CTA.  red holds two slots per warp used alternately (parity), so one barrier
+// per reduction suffices: a slot is rewritten only two reductions later, after the barrier
+// of the reduction in between.
+__device__ __forceinline__ float block_sum(float v, float *red, int parity) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
+  if (lane == 0) red[parity * (kThreads / 32) + warp] = v;
   __syncthreads();
   float t = 0.f;
 #pragma unroll
-  for (int w = 0; w < kThreads / 32; w++) t += red[w];
+  for (int w = 0; w < kThreads / 32; w++) t += red[parity * (kThreads / 32) + w];
   return t;
 }
 
+// One CTA per row; VPT 8-element vectors per thread (h = 8 * 256 * VPT at most).
+template <int VPT>
 __global__ void __launch_bounds__(kThreads) layernorm_kernel(const uint4 *__restrict__ x, int h,
-                                                             const __half *__restrict__ gamma,
-                                                             const __half *__restrict__ beta, float eps,
+                                                             const uint4 *__restrict__ gamma,
+                                                             const uint4 *__restrict__ beta, float eps,
                                                              uint4 *__restrict__ y) {
-  __shared__ float red[kThreads / 32];
+  __shared__ float red[2 * (kThreads / 32)];
   const int nvec = h / 8;
   const uint4 *xr = x + static_cast<int64_t>(blockIdx.x) * nvec;
   uint4 *yr = y + static_cast<int64_t>(blockIdx.x) * nvec;
-  float v[kMaxVec][8];
+  uint4 xv[VPT], gv[VPT], bv[VPT];
+#pragma unroll
+  for (int i = 0; i < VPT; i++) {  // every load is issued before any reduction
+    const int idx = threadIdx.x + i * kThreads;
+    const bool in = idx < nvec;
+    xv[i] = in ? xr[idx] : make_uint4(0, 0, 0, 0);
+    gv[i] = (in && gamma) ? gamma[idx] : make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);  // 1.0
+    bv[i] = (in && beta) ? beta[idx] : make_uint4(0, 0, 0, 0);
+  }
+  float v[VPT][8];
   float sum = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxVec; i++) {
-    const int idx = threadIdx.x + i * kThreads;
-    if (idx < nvec) {
-      uint4 u = xr[idx];
-      const __half2 *h2 = reinterpret_cast<const __half2 *>(&u);
+  for (int i = 0; i < VPT; i++) {
+    const __half2 *h2 = reinterpret_cast<const __half2 *>(&xv[i]);
 #pragma unroll
-      for (int j = 0; j < 4; j++) {
-        float2 f = __half22float2(h2[j]);
-        v[i][2 * j] = f.x;
-        v[i][2 * j + 1] = f.y;
-        sum += f.x + f.y;
-      }
+    for (int j = 0; j < 4; j++) {
+      const float2 f = __half22float2(h2[j]);
+      v[i][2 * j] = f.x;
+      v[i][2 * j + 1] = f.y;
+      sum += f.x + f.y;
     }
   }
-  const float mean = block_sum(sum, red) / h;
+  const float mean = block_sum(sum, red, 0) / h;
   float sq = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxVec; i++) {
-    const int idx = threadIdx.x + i * kThreads;
-    if (idx < nvec) {
+  for (int i = 0; i < VPT; i++) {
+    if (threadIdx.x + i * kThreads < nvec) {
 #pragma unroll
       for (int j = 0; j < 8; j++) {
         const float d = v[i][j] - mean;
@@ -60,20 +68,20 @@ __global__ void __launch_bounds__(kThreads) layernorm_kernel(const uint4 *__rest
       }
     }
   }
-  const float var = block_sum(sq, red) / h;
+  const float var = block_sum(sq, red, 1) / h;
   const float rstd = rsqrtf(var + eps);
 #pragma unroll
-  for (int i = 0; i < kMaxVec; i++) {
+  for (int i = 0; i < VPT; i++) {
     const int idx = threadIdx.x + i * kThreads;
     if (idx < nvec) {
       uint4 out;
       __half2 *o2 = reinterpret_cast<__half2 *>(&out);
+      const __half2 *g2 = reinterpret_cast<const __half2 *>(&gv[i]);
+      const __half2 *b2 = reinterpret_cast<const __half2 *>(&bv[i]);
 #pragma unroll
       for (int j = 0; j < 4; j++) {
-        const int c = idx * 8 + 2 * j;
-        const float g0 = gamma ? __half2float(gamma[c]) : 1.f, g1 = gamma ? __half2float(gamma[c + 1]) : 1.f;
-        const float b0 = beta ? __half2float(beta[c]) : 0.f, b1 = beta ? __half2float(beta[c + 1]) : 0.f;
-        o2[j] = __floats2half2_rn((v[i][2 * j] - mean) * rstd * g0 + b0, (v[i][2 * j + 1] - mean) * rstd * g1 + b1);
+        const float2 g = __half22float2(g2[j]), b = __half22float2(b2[j]);
+        o2[j] = __floats2half2_rn((v[i][2 * j] - mean) * rstd * g.x + b.x, (v[i][2 * j + 1] - mean) * rstd * g.y + b.y);
       }
       yr[idx] = out;
     }
@@ -85,9 +93,14 @@ __global__ void __launch_bounds__(kThreads) layernorm_kernel(const uint4 *__rest
 fg_status fg_layernorm_launch(const fg_half *x, int M, int h, const fg_half *gamma, const fg_half *beta, float eps,
                               fg_half *y, cudaStream_t st) {
   if (M == 0) return FG_OK;
-  layernorm_kernel<<<M, kThreads, 0, st>>>(reinterpret_cast<const uint4 *>(x), h,
-                                           reinterpret_cast<const __half *>(gamma),
-                                           reinterpret_cast<const __half *>(beta), eps, reinterpret_cast<uint4 *>(y));
+  const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+  const uint4 *gv = reinterpret_cast<const uint4 *>(gamma), *bv = reinterpret_cast<const uint4 *>(beta);
+  uint4 *yv = reinterpret_cast<uint4 *>(y);
+  const int vpt = (h / 8 + kThreads - 1) / kThreads;
+  if (vpt <= 1) layernorm_kernel<1><<<M, kThreads, 0, st>>>(xv, h, gv, bv, eps, yv);
+  else if (vpt <= 2) layernorm_kernel<2><<<M, kThreads, 0, st>>>(xv, h, gv, bv, eps, yv);
+  else if (vpt <= 4) layernorm_kernel<4><<<M, kThreads, 0, st>>>(xv, h, gv, bv, eps, yv);
+  else layernorm_kernel<8><<<M, kThreads, 0, st>>>(xv, h, gv, bv, eps, yv);
   return fg_launch_check();
 }
 
@@ -97,5 +110,6 @@ extern "C" fg_status fg_layernorm(const fg_half *x, int M, int h, const fg_half 
   if (h % 8 || h > kThreads * kMaxVec * 8) return FG_ERR_SHAPE;
   if (M == 0) return FG_OK;
   if (!x || !y || !fg_aligned16(x) || !fg_aligned16(y)) return FG_ERR_INVALID;
+  if ((gamma && !fg_aligned16(gamma)) || (beta && !fg_aligned16(beta))) return FG_ERR_INVALID;
   return fg_layernorm_launch(x, M, h, gamma, beta, eps, y, static_cast<cudaStream_t>(stream));
 }

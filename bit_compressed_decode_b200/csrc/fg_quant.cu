@@ -179,41 +179,40 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __half *__restrict
                                                         int64_t ld, int rows, int rows_per_seq,
                                                         const int32_t *__restrict__ positions, KvArgs a,
                                                         unsigned int *err) {
+  // A warp takes one (row, head) item per step: its 2 * d/64 units (k and v groups), 4 at a
+  // time in the four 8-lane slots; unit us = group * 2 + (0 for k, 1 for v).
   const int lane = threadIdx.x & 31;
   const int slot = lane >> 3, j = lane & 7;
   const int ng = a.d >> 6;
-  const int64_t units = static_cast<int64_t>(rows) * a.H * ng * 2;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t u0 = warp * 4; u0 < units; u0 += nwarps * 4) {
-    const int64_t u = u0 + slot;
-    const bool live = u < units;
-    // unit -> (row, head, group, k|v), v units after k units of the same group
-    const int which = static_cast<int>(u & 1);
-    const int64_t q = u >> 1;
-    const int g = static_cast<int>(q % ng);
-    const int hd = static_cast<int>((q / ng) % a.H);
-    const int r = static_cast<int>(q / (static_cast<int64_t>(ng) * a.H));
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (live) {
-      const __half *src = (which ? v : k) + static_cast<int64_t>(r) * ld + hd * a.d + g * 64;
-      val = *reinterpret_cast<const uint4 *>(src + j * 8);
-    }
-    __half mn, sc;
-    const uint32_t w = quant_group8(val, mn, sc);
-    if (!live) continue;
+  const int items = rows * a.H;
+  const int warp = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
+  const int nwarps = static_cast<int>((static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5);
+  for (int item = warp; item < items; item += nwarps) {
+    const int r = item / a.H, hd = item - r * a.H;
     const int s = r / rows_per_seq;
-    const int pos = positions[s] + r % rows_per_seq;
-    if (pos < 0 || pos >= a.maxL) {
-      if (j == 0) atomicOr(err, FG_DEVERR_RANGE);
-      continue;
-    }
+    const int pos = positions[s] + (r - s * rows_per_seq);
+    const bool in_range = pos >= 0 && pos < a.maxL;
     const int64_t slot_idx = (static_cast<int64_t>(s) * a.H + hd) * a.maxL + pos;
-    (which ? a.vc : a.kc)[slot_idx * (a.d / 8) + g * 8 + j] = w;
-    if (j == 0) {
-      const int64_t m = slot_idx * ng + g;
-      (which ? a.vm : a.km)[m] = mn;
-      (which ? a.vs : a.ks)[m] = sc;
+    for (int u0 = 0; u0 < 2 * ng; u0 += 4) {  // warp-uniform
+      const int us = u0 + slot;
+      const bool live = us < 2 * ng;
+      const int which = us & 1, g = us >> 1;
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (live) val = *reinterpret_cast<const uint4 *>((which ? v : k) + static_cast<int64_t>(r) * ld + hd * a.d +
+                                                       g * 64 + j * 8);
+      __half mn, sc;
+      const uint32_t w = quant_group8(val, mn, sc);
+      if (!live) continue;
+      if (!in_range) {
+        if (j == 0) atomicOr(err, FG_DEVERR_RANGE);
+        continue;
+      }
+      (which ? a.vc : a.kc)[slot_idx * (a.d / 8) + g * 8 + j] = w;
+      if (j == 0) {
+        const int64_t m = slot_idx * ng + g;
+        (which ? a.vm : a.km)[m] = mn;
+        (which ? a.vs : a.ks)[m] = sc;
+      }
     }
   }
 }
@@ -350,9 +349,9 @@ fg_status fg_kv_append_launch(const fg_kv_cache *kv, const fg_half *k, const fg_
   a.num_seqs = kv->num_seqs;
   unsigned int *err = fg_error_word_ptr();
   if (!err) return FG_ERR_CUDA;
-  const int64_t units = static_cast<int64_t>(rows) * kv->num_heads * (kv->head_dim / 64) * 2;
-  const int64_t warps = (units + 3) / 4;
-  kv_append_kernel<<<grid_for((warps + 7) / 8, 8), 256, 0, st>>>(
+  const int64_t items = static_cast<int64_t>(rows) * kv->num_heads;  // one warp per (row, head)
+  if (items > INT32_MAX) return FG_ERR_SHAPE;
+  kv_append_kernel<<<grid_for((items + 7) / 8, 8), 256, 0, st>>>(
       reinterpret_cast<const __half *>(k), reinterpret_cast<const __half *>(v), ld, rows, rows_per_seq, positions, a,
       err);
   return fg_launch_check();

@@ -185,7 +185,7 @@ FG_API fg_status fg_linear_w4a16(const fg_half *x, int M, int K, const fg_qtenso
 
 /* y = (x - mean) / sqrt(var + eps) * gamma + beta per row (fp32 statistics,
  * biased variance), fp16 in/out, gamma/beta fp16 [h] (NULL = 1 / 0).
- * h % 8 == 0.  [OPT] */
+ * h % 8 == 0; x, y, gamma and beta 16-byte aligned (FG_ERR_INVALID otherwise).  [OPT] */
 FG_API fg_status fg_layernorm(const fg_half *x, int M, int h, const fg_half *gamma, const fg_half *beta,
                        float eps, fg_half *y, void *stream);
 
