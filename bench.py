@@ -37,6 +37,13 @@ WORKLOADS = {
     # OPT-30B-shaped stack: 48 layers whose W4 blobs stay in pinned host memory and are
     # prefetched layer by layer on a side stream; KV4 caches resident in HBM
     "opt-30b-stack": dict(hidden=7168, heads=56, ffn=28672, nb=4, gbs=64, prompt=512, steps=32, layers=48),
+    # OPT-175B-shaped stack: weights AND KV4 caches in pinned host memory; each layer's cache is
+    # filled into a device staging cache before the layer and its new slots written back after.
+    # The model has 96 layers (about 3.06 GB of host memory each); unless --layers is given the
+    # run takes at most 16, and no more than half the host's available memory holds, every
+    # layer with its own host buffers.
+    "opt-175b-stack": dict(hidden=12288, heads=96, ffn=49152, nb=8, gbs=32, prompt=512, steps=32, layers=16,
+                           model_layers=96, kv_host=True),
 }
 METRIC = "decode tokens/s per OPT layer block (W4 KV4)"
 
@@ -281,24 +288,32 @@ def run_ours(args, wl):
     fg.fg_sync_status()
 
     # ---- timed region (device time, CUDA events on the launching stream) ----
+    # The steps are timed without per-kernel events; a second timed pass over the same steps
+    # with the library's per-kernel events (on the launching stream) gives the breakdown
+    # behind the roofline figures.
     sampler = ClockSampler(dev.index if world == 1 else local)
     sampler.start()
     time.sleep(0.3)
-    fg.fg_profile_enable(True)
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        step(args.warmup + i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    fg.fg_profile_enable(False)
+
+    def timed(profile):
+        fg.fg_profile_enable(profile)
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        fg.fg_profile_enable(False)
+        return replicas.max_over_ranks(e0.elapsed_time(e1), device=dev)
+
+    ms = timed(False)
+    ms_profiled = timed(True)
     clocks = sampler.stop()
     prof = fg.fg_profile_collect()
     fg.fg_sync_status()
-    ms = replicas.max_over_ranks(e0.elapsed_time(e1), device=dev)
     ms_per_step = ms / args.steps
     value = world * S * args.steps / (ms / 1e3)
 
@@ -372,6 +387,7 @@ def run_ours(args, wl):
                            cache.nbytes() / 1e9, totals["w4_bytes"] / 1e6)},
             "roofline": roofline,
             "kernels": kernels,
+            "kernels_pass_ms_per_step": ms_profiled / args.steps,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": sum(v[1] for v in prof.values()),
             "clocks": clocks,
@@ -403,6 +419,17 @@ def run_stack(args, wl):
     S, d = nb * gbs, h // H
     maxL = (P + wl["steps"] + 63) // 64 * 64
     cfg = fg.LayerConfig(h, H, F)
+    ng = d // 64
+    kv_host = bool(wl.get("kv_host"))
+    if kv_host and not args.layers:
+        # as many layers as half the host's available memory holds (pinned buffers are
+        # rounded up to powers of two by torch's host allocator)
+        def p2(n):
+            return 1 << (int(n) - 1).bit_length()
+        per_layer = p2(cfg.blob_bytes()) + 2 * p2(S * H * maxL * d // 2) + 4 * p2(S * H * maxL * ng * 2)
+        with open("/proc/meminfo") as f:
+            avail = next(int(ln.split()[1]) * 1024 for ln in f if ln.startswith("MemAvailable"))
+        nl = max(2, min(nl, int(avail * 0.5) // per_layer))
     g = torch.Generator(device=dev)
     g.manual_seed(2000 + rank)
     # weights: seeded device draws N(0, 0.02) (biases 0, LayerNorm 1/0), quantised by fg_quantize,
@@ -427,16 +454,29 @@ def run_stack(args, wl):
     # KV caches: seeded random codes and group min/scale for the prompt positions (a decode
     # step reads the same bytes whatever they hold; prefilling 48 layers x 512 tokens through
     # the per-row attention kernel would take far longer than the timed steps)
-    ng = d // 64
-    caches = []
-    for _ in range(nl):
-        caches.append(fg.KVCache(S, H, d, maxL, device=dev, arrays=[
+
+    def seeded_cache():
+        return fg.KVCache(S, H, d, maxL, device=dev, arrays=[
             torch.randint(0, 256, (S, H, maxL, d // 2), generator=g, device=dev, dtype=torch.uint8),
             torch.randn((S, H, maxL, ng), generator=g, device=dev, dtype=torch.float16),
             (torch.rand((S, H, maxL, ng), generator=g, device=dev) * 0.2).half(),
             torch.randint(0, 256, (S, H, maxL, d // 2), generator=g, device=dev, dtype=torch.uint8),
             torch.randn((S, H, maxL, ng), generator=g, device=dev, dtype=torch.float16),
-            (torch.rand((S, H, maxL, ng), generator=g, device=dev) * 0.2).half()]))
+            (torch.rand((S, H, maxL, ng), generator=g, device=dev) * 0.2).half()])
+
+    caches, staging = [], []
+    if kv_host:
+        # every layer's cache drawn on the device, then parked in its own pinned host arrays
+        for _ in range(nl):
+            c = seeded_cache()
+            hc = fg.KVCache(S, H, d, maxL, device="cpu", pin_memory=True)
+            for a, b in zip(hc.arrays(), c.arrays()):
+                a.copy_(b)
+            caches.append(hc)
+            del c
+        staging = [fg.KVCache(S, H, d, maxL, device=dev) for _ in range(2)]
+    else:
+        caches = [seeded_cache() for _ in range(nl)]
     compute = torch.cuda.current_stream()
     copy = torch.cuda.Stream(device=dev)
     fg.fg_sync_status()
@@ -446,8 +486,14 @@ def run_stack(args, wl):
     ws = torch.empty(st.workspace_bytes(S), dtype=torch.uint8, device=dev)
 
     def step(i):
-        st.decode(caches, xs[i % 2], pos[i % wl["steps"]], num_gpu_batches=nb, gpu_batch_size=gbs, out=out,
-                  workspace=ws, compute_stream=compute, copy_stream=copy)
+        t = i % wl["steps"]
+        if kv_host:
+            # positions [0, P+t) filled before each layer, slot P+t written back after it
+            st.decode_host_kv(caches, staging, xs[i % 2], pos[t], P + t, P + t, P + t + 1, num_gpu_batches=nb,
+                              gpu_batch_size=gbs, out=out, workspace=ws, compute_stream=compute, copy_stream=copy)
+        else:
+            st.decode(caches, xs[i % 2], pos[t], num_gpu_batches=nb, gpu_batch_size=gbs, out=out,
+                      workspace=ws, compute_stream=compute, copy_stream=copy)
 
     for i in range(args.warmup):
         step(i)
@@ -469,19 +515,36 @@ def run_stack(args, wl):
     ms = replicas.max_over_ranks(e0.elapsed_time(e1), device=dev)
     fg.fg_sync_status()
     blob_gb = cfg.blob_bytes() * nl / 1e9
+    slot_bytes = S * H * 2 * (d // 2 + 4 * ng)          # K and V codes + min/scale of one position
+    fill_gb = wb_gb = 0.0
+    if kv_host:
+        ts = [(args.warmup + i) % wl["steps"] for i in range(args.steps)]
+        fill_gb = sum((P + t) * slot_bytes for t in ts) * nl / args.steps / 1e9
+        wb_gb = slot_bytes * nl / 1e9
     if rank == 0:
-        print(json.dumps({
-            "metric": "decode tokens/s of the OPT layer stack (W4 weights streamed from pinned host, KV4 in HBM)",
+        line = {
+            "metric": ("decode tokens/s of the OPT layer stack (W4 weights and KV4 streamed from pinned host)"
+                       if kv_host else
+                       "decode tokens/s of the OPT layer stack (W4 weights streamed from pinned host, KV4 in HBM)"),
             "value": world * S * args.steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "dtype": "f16", "data": "synthetic",
             "config": {"workload": args.workload, "layers": nl, "block": f"{nb}x{gbs}", "hidden": h, "prompt": P,
                        "weights_streamed_gb_per_step": round(blob_gb, 3),
-                       "kv": "KV4 g64, seeded random codes at the prompt positions (no prefill)",
-                       "kv_gb_in_hbm": round(sum(c.nbytes() for c in caches) / 1e9, 2)},
-            "host_link_gbs": round(blob_gb / (ms / args.steps / 1e3), 1),
+                       "kv": "KV4 g64, seeded random codes at the prompt positions (no prefill)"},
+            "host_link_gbs": round((blob_gb + fill_gb + wb_gb) / (ms / args.steps / 1e3), 1),
             "clocks": clocks,
-        }), flush=True)
+        }
+        if kv_host:
+            line["config"]["kv_fill_gb_per_step"] = round(fill_gb, 3)
+            line["config"]["kv_writeback_gb_per_step"] = round(wb_gb, 4)
+            line["config"]["kv_gb_in_host"] = round(sum(c.nbytes() for c in caches) / 1e9, 2)
+            # the same per-layer time over the model's full depth (every layer moves the same bytes)
+            line["tokens_per_s_full_depth_projected"] = line["value"] * nl / wl["model_layers"]
+            line["config"]["model_layers"] = wl["model_layers"]
+        else:
+            line["config"]["kv_gb_in_hbm"] = round(sum(c.nbytes() for c in caches) / 1e9, 2)
+        print(json.dumps(line), flush=True)
     st.close()
 
 

@@ -90,6 +90,8 @@ _decl("fg_profile_collect", c_int, POINTER(c_float), POINTER(c_int), c_int)
 _decl("fg_stack_create", c_int, POINTER(fg_layer_config), c_int, POINTER(c_void_p), P, P, POINTER(c_void_p))
 _decl("fg_stack_decode", c_int, P, POINTER(fg_kv_cache), P, P, P, c_int, c_int, P, c_size_t, P, P)
 _decl("fg_stack_prefill", c_int, P, POINTER(fg_kv_cache), P, P, P, c_int, c_int, c_int, P, c_size_t, P, P)
+_decl("fg_stack_decode_host_kv", c_int, P, POINTER(fg_kv_cache), POINTER(fg_kv_cache), c_int, c_int, c_int, P, P, P,
+      c_int, c_int, P, c_size_t, P, P)
 _decl("fg_stack_inject_copy_failure", c_int, P, c_int)
 _decl("fg_stack_destroy", c_int, P)
 
@@ -184,7 +186,9 @@ def fg_dequantize(q: QTensor, stream=None) -> torch.Tensor:
 class KVCache:
     """4-bit KV cache of one layer, allocated with torch on ``device``."""
 
-    def __init__(self, num_seqs, num_heads, head_dim, max_len, device="cuda", arrays=None):
+    def __init__(self, num_seqs, num_heads, head_dim, max_len, device="cuda", arrays=None, pin_memory=False):
+        """``pin_memory=True`` with ``device="cpu"`` allocates page-locked host arrays, the form
+        fg_stack_decode_host_kv copies from and back to."""
         self.num_seqs, self.num_heads, self.head_dim, self.max_len = num_seqs, num_heads, head_dim, max_len
         cb, mb = c_size_t(), c_size_t()
         _check(_lib.fg_kv_cache_bytes(num_seqs, num_heads, head_dim, max_len, ctypes.byref(cb), ctypes.byref(mb)),
@@ -193,12 +197,13 @@ class KVCache:
         if arrays is None:
             cshape = (num_seqs, num_heads, max_len, head_dim // 2)
             mshape = (num_seqs, num_heads, max_len, ng)
-            arrays = [torch.zeros(cshape, dtype=torch.uint8, device=device),
-                      torch.zeros(mshape, dtype=torch.float16, device=device),
-                      torch.zeros(mshape, dtype=torch.float16, device=device),
-                      torch.zeros(cshape, dtype=torch.uint8, device=device),
-                      torch.zeros(mshape, dtype=torch.float16, device=device),
-                      torch.zeros(mshape, dtype=torch.float16, device=device)]
+            kw = {"pin_memory": True} if pin_memory else {}
+            arrays = [torch.zeros(cshape, dtype=torch.uint8, device=device, **kw),
+                      torch.zeros(mshape, dtype=torch.float16, device=device, **kw),
+                      torch.zeros(mshape, dtype=torch.float16, device=device, **kw),
+                      torch.zeros(cshape, dtype=torch.uint8, device=device, **kw),
+                      torch.zeros(mshape, dtype=torch.float16, device=device, **kw),
+                      torch.zeros(mshape, dtype=torch.float16, device=device, **kw)]
         self.k_codes, self.k_mins, self.k_scales, self.v_codes, self.v_mins, self.v_scales = arrays
 
     def arrays(self):
@@ -492,6 +497,28 @@ class Stack:
         ps = _stream(copy_stream) if copy_stream is not None else c_void_p(torch.cuda.Stream().cuda_stream)
         _check(_lib.fg_stack_prefill(self._h, kv, _ptr(x), _ptr(out), _ptr(positions), P, num_gpu_batches, gbs,
                                      _ptr(workspace), workspace.numel(), cs, ps), "fg_stack_prefill")
+        return out
+
+    def decode_host_kv(self, host_caches, staging_caches, x, positions, fill_len, wb_begin, wb_end,
+                       num_gpu_batches=1, gpu_batch_size=None, out=None, workspace=None, compute_stream=None,
+                       copy_stream=None):
+        """One decode step with every layer's cache in pinned host memory (fg_stack_decode_host_kv):
+        ``host_caches`` one pinned KVCache per layer, ``staging_caches`` two device KVCaches of the same
+        geometry; positions [0, fill_len) are filled before each layer and [wb_begin, wb_end) written
+        back after it."""
+        S = x.shape[0]
+        gbs = S // num_gpu_batches if gpu_batch_size is None else gpu_batch_size
+        if out is None:
+            out = torch.empty_like(x)
+        if workspace is None:
+            workspace = torch.empty(self.workspace_bytes(S), dtype=torch.uint8, device=x.device)
+        hk = (fg_kv_cache * len(host_caches))(*[c.struct() for c in host_caches])
+        dk = (fg_kv_cache * 2)(*[c.struct() for c in staging_caches])
+        cs = _stream(compute_stream)
+        ps = _stream(copy_stream) if copy_stream is not None else c_void_p(torch.cuda.Stream().cuda_stream)
+        _check(_lib.fg_stack_decode_host_kv(self._h, hk, dk, fill_len, wb_begin, wb_end, _ptr(x), _ptr(out),
+                                            _ptr(positions), num_gpu_batches, gbs, _ptr(workspace),
+                                            workspace.numel(), cs, ps), "fg_stack_decode_host_kv")
         return out
 
     def inject_copy_failure(self, count: int = 1) -> None:

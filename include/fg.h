@@ -310,6 +310,32 @@ FG_API fg_status fg_stack_prefill(fg_stack *st, const fg_kv_cache *kv, const fg_
                            const int32_t *positions, int prompt_len, int num_gpu_batches, int gpu_batch_size,
                            void *workspace, size_t workspace_bytes, void *compute_stream, void *copy_stream);
 
+/* One decode step with every layer's KV cache in host memory, for stacks whose
+ * cache does not fit in HBM ([G1] section 2: the KV cache is offloaded with
+ * the weights; [G3]: it stays in 4-bit form while it moves).
+ * host_kv: array of num_layers caches in pinned host memory (same geometry).
+ * dev_kv: two device caches of that geometry, used as staging: layer l runs on
+ * dev_kv[l%2].  Per layer, copy_stream copies the weight blob and positions
+ * [0, fill_len) of host_kv[l] into staging buffer l%2, one strided
+ * cudaMemcpy2DAsync per cache array; after the layer it copies positions
+ * [wb_begin, wb_end) (the slots this step appended) back to host_kv[l].
+ * Events order the two streams, so the fill of layer l+1 and the write-back of
+ * layer l-1 overlap the compute of layer l.  Slots past a sequence's length in
+ * a staging cache may hold another layer's data; attention never reads them.
+ * The write-back copies whole position slices for every sequence, so a slot in
+ * [wb_begin, wb_end) that this step does not append must lie below fill_len
+ * (with equal positions p: fill_len = p, wb = [p, p+1); ragged: fill_len =
+ * max p + 1, wb = [min p, max p + 1)).  compute_stream waits for the last
+ * write-back, so work enqueued on it afterwards sees every host cache updated.
+ * Other arguments as fg_stack_decode.  Returns FG_ERR_SHAPE when the caches'
+ * geometries differ or the block has more sequences than a cache,
+ * FG_ERR_INVALID for fill/write-back ranges outside [0, max_len). */
+FG_API fg_status fg_stack_decode_host_kv(fg_stack *st, const fg_kv_cache *host_kv, const fg_kv_cache *dev_kv,
+                                  int fill_len, int wb_begin, int wb_end, const fg_half *x_in, fg_half *x_out,
+                                  const int32_t *positions, int num_gpu_batches, int gpu_batch_size,
+                                  void *workspace, size_t workspace_bytes, void *compute_stream,
+                                  void *copy_stream);
+
 /* Test hook: the next `count` blob copies of this stack report a copy
  * failure (no copy is issued), as if cudaMemcpyAsync had failed. */
 FG_API fg_status fg_stack_inject_copy_failure(fg_stack *st, int count);

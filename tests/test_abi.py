@@ -25,7 +25,7 @@ def test_header_declares_the_entry_points():
     names = declared()
     for must in ("fg_quantize", "fg_dequantize", "fg_kv_append", "fg_layer_decode", "fg_layer_prefill",
                  "fg_attention_decode", "fg_linear_w4a16", "fg_sync_status", "fg_stack_decode",
-                 "fg_layer_decode_noalloc"):
+                 "fg_layer_decode_noalloc", "fg_stack_decode_host_kv"):
         assert must in names
 
 
@@ -154,3 +154,9 @@ def test_stack_create_validates():
                ctypes.byref(h)) == 1
     assert _rc("fg_stack_create", ctypes.byref(c), 0, blobs, ctypes.c_void_p(256), ctypes.c_void_p(512),
                ctypes.byref(h)) == 1
+
+
+def test_stack_decode_host_kv_validates_before_cuda():
+    kv = (B.fg_kv_cache * 2)()
+    assert _rc("fg_stack_decode_host_kv", None, kv, kv, 0, 0, 1, None, None, None, 1, 1, None, 0, None,
+               None) == 1                                    # no stack: FG_ERR_INVALID

@@ -221,6 +221,70 @@ def test_stack_copy_failure_is_reported_and_recoverable():
     st.close()
 
 
+@pytest.mark.parametrize("ragged", [False, True])
+def test_stack_host_kv_equals_device_kv(ragged):
+    # Caches spilled to pinned host memory, filled into two device staging caches layer by
+    # layer, give the same bits as the caches resident in HBM: the output of two decode
+    # steps and, after the write-back of the new slots, the host caches themselves.
+    nl, h, H, F, S, P, maxL = 3, 256, 4, 512, 8, 12, 64
+    cfg, _, _, host = _stack_setup(nl, h, H, F, S, P)
+    st = fg.Stack(cfg, host)
+    caches = [fg.KVCache(S, H, h // H, maxL) for _ in range(nl)]
+    st.prefill(caches, dev(si.hidden_block(10, si.STREAM["prompt"], S, P, h)), dev(np.zeros(S, np.int32)))
+    torch.cuda.synchronize()
+    hcaches = [fg.KVCache(S, H, h // H, maxL, device="cpu", pin_memory=True) for _ in range(nl)]
+    for hc, c in zip(hcaches, caches):
+        for a, b in zip(hc.arrays(), c.arrays()):
+            a.copy_(b)
+    # staging caches start with arbitrary bytes (NaN and inf metadata included): slots past a
+    # sequence's length are never read
+    g = torch.Generator(device="cuda").manual_seed(3)
+    staging = [fg.KVCache(S, H, h // H, maxL) for _ in range(2)]
+    for c in staging:
+        for a in c.arrays():
+            a.view(torch.uint8).copy_(torch.randint(0, 256, a.view(torch.uint8).shape, dtype=torch.uint8,
+                                                    device="cuda", generator=g))
+    cs, ps = torch.cuda.Stream(), torch.cuda.Stream()
+    for t in range(2):
+        p = np.full(S, P + t, np.int32) + (np.arange(S, dtype=np.int32) % 3 if ragged else 0)
+        x = dev(si.decode_inputs(10, t, S, h))
+        y = st.decode(caches, x, dev(p), num_gpu_batches=2)
+        torch.cuda.synchronize()
+        # ragged: slots that some sequences skip are filled so the write-back returns them intact
+        fill = int(p.max()) + (1 if ragged else 0)
+        z = st.decode_host_kv(hcaches, staging, x, dev(p), fill, int(p.min()), int(p.max()) + 1,
+                              num_gpu_batches=2, compute_stream=cs, copy_stream=ps)
+        ps.synchronize()
+        cs.synchronize()
+        fg.fg_sync_status()
+        assert torch.equal(y, z)
+    for hc, c in zip(hcaches, caches):
+        for a, b in zip(hc.arrays(), c.arrays()):
+            assert torch.equal(a, b.cpu())
+    st.close()
+
+
+def test_stack_host_kv_rejects_bad_ranges():
+    nl, h, H, F, S = 2, 256, 4, 512, 4
+    cfg, _, _, host = _stack_setup(nl, h, H, F, S, 4)
+    st = fg.Stack(cfg, host)
+    hc = [fg.KVCache(S, H, h // H, 64, device="cpu", pin_memory=True) for _ in range(nl)]
+    dc = [fg.KVCache(S, H, h // H, 64) for _ in range(2)]
+    x, pos = dev(si.decode_inputs(11, 0, S, h)), dev(np.zeros(S, np.int32))
+    with pytest.raises(fg.FgError, match="INVALID"):
+        st.decode_host_kv(hc, dc, x, pos, 65, 0, 1)          # fill past max_len
+    with pytest.raises(fg.FgError, match="INVALID"):
+        st.decode_host_kv(hc, dc, x, pos, 0, 2, 1)           # empty-reversed write-back range
+    short = [fg.KVCache(S, H, h // H, 128) for _ in range(2)]
+    with pytest.raises(fg.FgError, match="SHAPE"):
+        st.decode_host_kv(hc, short, x, pos, 0, 0, 1)        # staging geometry differs
+    hfew = [fg.KVCache(2, H, h // H, 64, device="cpu", pin_memory=True) for _ in range(nl)]
+    few = [fg.KVCache(2, H, h // H, 64) for _ in range(2)]
+    with pytest.raises(fg.FgError, match="SHAPE"):
+        st.decode_host_kv(hfew, few, x, pos, 0, 0, 1)        # block larger than the caches
+    st.close()
+
+
 # ------------------------------------------------------------------ full size -----------
 
 @pytest.mark.slow
