@@ -495,6 +495,22 @@ def run_stack(args, wl):
             st.decode(caches, xs[i % 2], pos[t], num_gpu_batches=nb, gpu_batch_size=gbs, out=out,
                       workspace=ws, compute_stream=compute, copy_stream=copy)
 
+    # host-link peak: a plain pinned -> device cudaMemcpyAsync of 1 GiB on the copy stream
+    # (best of 5), the denominator of the stack's roofline
+    pin = torch.empty(1 << 30, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    link = []
+    for _ in range(5):
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(copy)
+        with torch.cuda.stream(copy):
+            dst.copy_(pin, non_blocking=True)
+        c1.record(copy)
+        c1.synchronize()
+        link.append(c0.elapsed_time(c1))
+    link_peak = (1 << 30) / (min(link) / 1e3) / 1e9
+    del pin, dst
+
     for i in range(args.warmup):
         step(i)
     fg.fg_sync_status()
@@ -533,6 +549,11 @@ def run_stack(args, wl):
                        "weights_streamed_gb_per_step": round(blob_gb, 3),
                        "kv": "KV4 g64, seeded random codes at the prompt positions (no prefill)"},
             "host_link_gbs": round((blob_gb + fill_gb + wb_gb) / (ms / args.steps / 1e3), 1),
+            "roofline": {"bound": "host-link", "achieved": round((blob_gb + fill_gb) / (ms / args.steps / 1e3), 1),
+                         "peak": round(link_peak, 1), "unit": "GB/s",
+                         "frac": round((blob_gb + fill_gb) / (ms / args.steps / 1e3) / link_peak, 4),
+                         "traffic": None,
+                         "peak_source": "measured here: pinned host -> device cudaMemcpyAsync of 1 GiB"},
             "clocks": clocks,
         }
         if kv_host:
@@ -583,7 +604,11 @@ def run_kernel(args, wl):
         x = torch.randn((S, K), generator=g, device=dev, dtype=torch.float16)
         wq = fg.fg_quantize(torch.randn((N, K), generator=g, device=dev, dtype=torch.float16) * 0.02, dim=1)
         y = torch.empty((S, N), dtype=torch.float16, device=dev)
-        run = lambda: fg.fg_linear_w4a16(x, wq, out=y, stream=stream)
+        # --gemm-scratch none: no split-k scratch, so split k-ranges are added on chip
+        gws = torch.empty(16 if args.gemm_scratch == "none" else
+                          max(16, fg.fg_linear_workspace_bytes(x.shape[0], wq.shape[0], x.shape[1])),
+                          dtype=torch.uint8, device=dev)
+        run = lambda: fg.fg_linear_w4a16(x, wq, out=y, workspace=gws, stream=stream)
         work, unit, peak = 2 * S * N * K, "TFLOP/s", peaks["tc_burst"]
     elif args.kernel in ("quantize", "dequantize"):
         n = 1 << args.log2_elems
@@ -628,6 +653,8 @@ def main():
     ap.add_argument("--seqs", type=int, default=0, help="--kernel: sequences (default: the workload's block)")
     ap.add_argument("--log2-elems", type=int, default=28, help="--kernel quantize/dequantize: tensor size")
     ap.add_argument("--layers", type=int, default=0, help="stack workloads: number of layers (default: the model's)")
+    ap.add_argument("--gemm-scratch", choices=("auto", "none"), default="auto",
+                    help="--kernel *_gemm: give the GEMM its split-k scratch (auto) or none (on-chip reduction)")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
     if args.kernel:

@@ -59,6 +59,7 @@ struct GemmArgs {
   int relu, qcols;
   float qscale;
   int splits;
+  float *part;         // pair kernel, k split: fp32 partial sums through global memory, or null
   unsigned int *err;
 };
 
@@ -341,7 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
 //   warp 9       even CTA: the MMA issuer; odd CTA: forwards "A half ready" to the even
 //                CTA (a 16-byte bulk copy completing on its barrier); TMEM allocation.
 //   Split k-ranges of one pair tile form the cluster's z dimension (cluster 2 x 1 x splits);
-//   partial sums are reduced over distributed shared memory in z-rank order.
+//   partial sums are reduced in z-rank order through a global scratch (L2) when the caller
+//   gives one, else over distributed shared memory.
 // ------------------------------------------------------------------------------------
 
 constexpr int kPairTok = 512;                  // tokens per pair tile
@@ -625,6 +627,74 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
       }
       __syncthreads();
     }
+  } else if (a.part) {
+    // k split, partial sums through global memory (they stay in L2): every z rank stores its
+    // fp32 partial [512 tokens][its 128 features] straight from TMEM -- a warp writes 128
+    // contiguous bytes per token -- the cluster synchronises (release / acquire at cluster
+    // scope orders these stores for the other ranks' loads), and the owner of each 32-token
+    // chunk (chunk % splits) adds the splits' partials in z-rank order, as the on-chip
+    // reduction below does, and finishes the chunk.  One barrier instead of a chain of
+    // rounds of distributed-shared-memory copies.
+    constexpr int kChunks = kPairCols / 32;
+    const int S = a.splits, zrank = static_cast<int>(crank >> 1);
+    constexpr int64_t kTileFloats = static_cast<int64_t>(kPairTok) * 256;
+    const float *tilep =
+        a.part + (static_cast<int64_t>(blockIdx.y) * (gridDim.x / 2) + blockIdx.x / 2) * S * kTileFloats;
+    if (warp < kDeqWarps && ready) {
+      float *mine = const_cast<float *>(tilep) + zrank * kTileFloats + half * 128 + q * 32 + lane;
+      for (int c8 = 0; c8 < kChunks / 2; c8++) {
+        const int ch = etile * (kChunks / 2) + c8;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; j++) mine[static_cast<int64_t>(ch * 32 + j) * 256] = __uint_as_float(v[j]);
+      }
+    }
+    __threadfence();
+    cluster_sync_all();
+    if (warp < kDeqWarps && ready && nb < a.N) {
+      float bias[8];
+#pragma unroll
+      for (int u = 0; u < 8; u++) bias[u] = a.bias ? __half2float(a.bias[nb + u]) : 0.f;
+      const float *col = tilep + half * 128 + f8;
+      for (int ch = zrank; ch < kChunks; ch += S) {
+        uint4 rv[2];
+        float acc[2][8];
+#pragma unroll
+        for (int it = 0; it < 2; it++) {
+          const int m = t0 + ch * 32 + mj0 + 16 * it;
+          rv[it] = (a.res && m < a.M) ? *reinterpret_cast<const uint4 *>(a.res + static_cast<int64_t>(m) * a.N + nb)
+                                      : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int u = 0; u < 8; u++) acc[it][u] = 0.f;
+        }
+#pragma unroll
+        for (int z = 0; z < 4; z++) {  // z-rank order
+          if (z >= S) break;
+#pragma unroll
+          for (int it = 0; it < 2; it++) {
+            const float *src = col + z * kTileFloats + static_cast<int64_t>(ch * 32 + mj0 + 16 * it) * 256;
+            const float4 p0 = __ldcg(reinterpret_cast<const float4 *>(src));
+            const float4 p1 = __ldcg(reinterpret_cast<const float4 *>(src + 4));
+            acc[it][0] += p0.x; acc[it][1] += p0.y; acc[it][2] += p0.z; acc[it][3] += p0.w;
+            acc[it][4] += p1.x; acc[it][5] += p1.y; acc[it][6] += p1.z; acc[it][7] += p1.w;
+          }
+        }
+#pragma unroll
+        for (int it = 0; it < 2; it++) {
+          const int m = t0 + ch * 32 + mj0 + 16 * it;
+          if (m >= a.M) continue;
+          const __half *rh = reinterpret_cast<const __half *>(&rv[it]);
+          uint4 ov;
+          __half *oh = reinterpret_cast<__half *>(&ov);
+#pragma unroll
+          for (int u = 0; u < 8; u++)
+            oh[u] = __float2half_rn(epilogue(acc[it][u], bias[u], __half2float(rh[u]), nb + u, a));
+          *reinterpret_cast<uint4 *>(a.y + static_cast<int64_t>(m) * a.N + nb) = ov;
+        }
+      }
+    }
   } else {
     // k split over the cluster's z ranks.  Per round of kR chunks every rank stages its fp32
     // partial of each chunk, then pushes the chunks it does not own into the owner's receive
@@ -836,6 +906,19 @@ fg_status launch_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cu
 
 // ---- pair kernel planning ----
 
+fg_status pair_attr_once() {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    fg_status rc = fg_cuda_check(
+        cudaFuncSetAttribute(w4a16_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem));
+    if (rc != FG_OK) return rc;
+    attr_set[dev] = true;
+  }
+  return FG_OK;
+}
+
 // Pair-kernel clusters (2 x 1 x splits CTAs) that can be resident at once; 0 when such a
 // cluster does not fit on the device.
 int pair_clusters_resident(int splits) {
@@ -844,6 +927,8 @@ int pair_clusters_resident(int splits) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || splits < 1 || splits > 4) return 0;
+  // the occupancy query needs the kernel's shared-memory attribute; a failed query is not cached
+  if (pair_attr_once() != FG_OK) return 0;
   if (!known[dev][splits]) {
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(2, 1, splits);
@@ -859,7 +944,7 @@ int pair_clusters_resident(int splits) {
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, w4a16_gemm_pair_kernel, &lc) != cudaSuccess) {
       cudaGetLastError();
-      n = 0;
+      return 0;
     }
     cache[dev][splits] = n > 0 ? n : 0;
     known[dev][splits] = true;
@@ -892,19 +977,6 @@ Plan make_pair_plan(int M, int N, int K) {
   return p;
 }
 
-fg_status pair_attr_once() {
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    fg_status rc = fg_cuda_check(
-        cudaFuncSetAttribute(w4a16_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem));
-    if (rc != FG_OK) return rc;
-    attr_set[dev] = true;
-  }
-  return FG_OK;
-}
-
 fg_status launch_pair(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st) {
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(2 * p.n_tiles, p.t_tiles, p.splits);
@@ -925,16 +997,20 @@ fg_status launch_pair(const CUtensorMap &map, const GemmArgs &a, const Plan &p, 
 
 }  // namespace
 
-// No global scratch: split-k partial sums are reduced inside the cluster.
-size_t fg_linear_ws_bytes(int, int, int) { return 0; }
+// Optional scratch of the pair kernel's k split: one fp32 partial [512 tokens][256 features]
+// per split of every pair tile.  Without it the partials are reduced inside the cluster.
+size_t fg_linear_ws_bytes(int M, int N, int K) {
+  if (M <= 256 || N <= 0 || K <= 0 || K % kBK) return 0;
+  const Plan p = make_pair_plan(M, N, K);
+  if (p.splits < 2) return 0;
+  return static_cast<size_t>(p.n_tiles) * p.t_tiles * p.splits * kPairTok * 256 * sizeof(float);
+}
 
 fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, const fg_half *bias,
                            const fg_half *residual, int flags, int qscale_cols, float qscale, fg_half *y,
                            void *workspace, size_t ws_bytes, cudaStream_t st) {
   const int N = static_cast<int>(w->shape[0]);
   if (M == 0) return FG_OK;
-  (void)workspace;
-  (void)ws_bytes;
   const bool pair = M > 256;
   if (pair) {
     fg_status rc = pair_attr_once();
@@ -966,6 +1042,10 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
   a.qcols = qscale_cols;
   a.qscale = qscale;
   a.splits = p.splits;
+  a.part = nullptr;
+  if (pair && p.splits > 1 && workspace && fg_aligned16(workspace) &&
+      ws_bytes >= static_cast<size_t>(p.n_tiles) * p.t_tiles * p.splits * kPairTok * 256 * sizeof(float))
+    a.part = static_cast<float *>(workspace);
   a.err = fg_error_word_ptr();
   if (!a.err) return FG_ERR_CUDA;
   if (pair) return launch_pair(map, a, p, st);

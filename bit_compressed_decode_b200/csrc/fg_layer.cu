@@ -122,7 +122,8 @@ fg_status run_layer(const fg_layer_config *c, const fg_layer_weights *w, const f
                     fg_half *x_out, const int32_t *positions, int rows, int rows_per_seq, uint8_t *ws,
                     size_t ws_bytes, cudaStream_t st) {
   const WsLayout L = ws_layout(c, rows);
-  if (ws_bytes < L.total) return FG_ERR_WORKSPACE;
+  // the GEMMs' split-k scratch is optional: they reduce on chip when what is left is short
+  if (ws_bytes < L.gemm) return FG_ERR_WORKSPACE;
   const int h = c->hidden, F = c->ffn;
   fg_half *a = reinterpret_cast<fg_half *>(ws + L.a);
   fg_half *qkv = reinterpret_cast<fg_half *>(ws + L.qkv);
@@ -130,7 +131,7 @@ fg_status run_layer(const fg_layer_config *c, const fg_layer_weights *w, const f
   fg_half *h1 = reinterpret_cast<fg_half *>(ws + L.h1);
   fg_half *f = reinterpret_cast<fg_half *>(ws + L.f);
   void *gws = ws + L.gemm;
-  const size_t gbytes = L.total - L.gemm;
+  const size_t gbytes = ws_bytes - L.gemm;
   const float qscale = 1.0f / sqrtf(static_cast<float>(c->head_dim));
   fg_status rc;
   int ev;
@@ -215,6 +216,13 @@ extern "C" fg_status fg_layer_weights_from_blob(const fg_layer_config *c, void *
   return FG_OK;
 }
 
+// The part of the layer's workspace that a call cannot do without (everything before the
+// GEMMs' optional split-k scratch).
+size_t fg_layer_ws_required(const fg_layer_config *c, int rows) {
+  if (!c || rows <= 0 || !config_ok(c)) return 0;
+  return ws_layout(c, rows).gemm;
+}
+
 extern "C" size_t fg_layer_workspace_bytes(const fg_layer_config *c, int rows) {
   if (!config_ok(c) || rows < 0) return 0;
   return ws_layout(c, rows).total;
@@ -243,7 +251,7 @@ extern "C" fg_status fg_layer_prefill(const fg_layer_config *c, const fg_layer_w
   // Process whole sequences in chunks that fit the workspace given.
   const int S = kv->num_seqs;
   int chunk = S;
-  while (chunk > 0 && ws_layout(c, chunk * prompt_len).total > workspace_bytes) chunk = chunk > 1 ? chunk / 2 : 0;
+  while (chunk > 0 && ws_layout(c, chunk * prompt_len).gemm > workspace_bytes) chunk = chunk > 1 ? chunk / 2 : 0;
   if (chunk == 0) return FG_ERR_WORKSPACE;
   if (static_cast<int64_t>(chunk) * prompt_len > (1 << 30)) return FG_ERR_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

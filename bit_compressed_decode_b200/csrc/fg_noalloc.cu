@@ -43,7 +43,8 @@ extern "C" fg_status fg_layer_decode_noalloc(const fg_layer_config *c, const fg_
                                              const int32_t *positions, int num_gpu_batches, int gpu_batch_size,
                                              void *stream) {
   if (num_gpu_batches < 0 || gpu_batch_size < 0) return FG_ERR_INVALID;
-  const size_t need = fg_layer_workspace_bytes(c, num_gpu_batches * gpu_batch_size);
+  // the activations must fit; the GEMMs use the rest for their optional split-k scratch
+  const size_t need = fg_layer_ws_required(c, num_gpu_batches * gpu_batch_size);
   if (need == 0 && num_gpu_batches * gpu_batch_size > 0) return FG_ERR_UNSUPPORTED;
   if (need > FG_NOALLOC_SCRATCH_BYTES) return FG_ERR_WORKSPACE;
   void *scratch = nullptr;

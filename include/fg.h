@@ -174,8 +174,12 @@ enum {
  * (with FG_EPI_RESIDUAL); the first qscale_cols outputs of each row are
  * multiplied by qscale after the bias.  K % 64 == 0, N % 128 == 0; x, y, the
  * codes and the residual 16-byte aligned (FG_ERR_INVALID otherwise).
- * workspace: device scratch of fg_linear_workspace_bytes(M, N, K) bytes, which
- * is 0 (split-K partial sums are reduced on chip); may be NULL.
+ * workspace: optional device scratch (16-byte aligned) of
+ * fg_linear_workspace_bytes(M, N, K) bytes, 0 when the GEMM does not split its
+ * k-range.  With it the partial sums of a split k-range are added through it
+ * (they stay in L2); with less, or NULL, they are added on chip over
+ * distributed shared memory.  Both add the splits in the same order, so the
+ * result is the same bit for bit.
  * Tensor cores dequantise W tiles in shared memory ([G3]: on-the-fly
  * dequantisation for FP16 compute). */
 FG_API size_t fg_linear_workspace_bytes(int M, int N, int K);
@@ -219,8 +223,11 @@ FG_API size_t fg_layer_blob_bytes(const fg_layer_config *c);
  * (any memory; no data is touched). */
 FG_API fg_status fg_layer_weights_from_blob(const fg_layer_config *c, void *blob, fg_layer_weights *out);
 
-/* Device scratch needed by fg_layer_decode / fg_layer_prefill for `rows`
- * hidden-state rows (the block's sequences, or sequences * prompt length). */
+/* Device scratch for fg_layer_decode / fg_layer_prefill over `rows`
+ * hidden-state rows (the block's sequences, or sequences * prompt length):
+ * the intermediate activations, then the GEMMs' optional split-k scratch
+ * (fg_linear_w4a16).  A call needs at least the activations' part and gives
+ * the GEMMs whatever follows it. */
 FG_API size_t fg_layer_workspace_bytes(const fg_layer_config *c, int rows);
 
 /* One decode step of one layer for every sequence of a block of
@@ -256,9 +263,10 @@ FG_API fg_status fg_layer_prefill(const fg_layer_config *c, const fg_layer_weigh
  * GPU loading the library holds until the process exits; the caller still
  * passes weights, cache, inputs and outputs, as for fg_layer_decode, whose
  * computation this is.
- *   - Returns FG_ERR_WORKSPACE when the block needs more scratch than that
- *     (fg_layer_workspace_bytes(c, S) > FG_NOALLOC_SCRATCH_BYTES), before any
- *     launch.
+ *   - Returns FG_ERR_WORKSPACE when the block's activations need more scratch
+ *     than that, before any launch (fg_layer_workspace_bytes(c, S) above
+ *     FG_NOALLOC_SCRATCH_BYTES only by the GEMMs' split-k scratch is fine: the
+ *     GEMMs then add their partial sums on chip).
  *   - The first call on each device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
  *   - Every call shares the one array and it keeps the last call's contents;

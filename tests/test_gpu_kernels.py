@@ -5,6 +5,10 @@ Tolerance (floating point): attention, W4A16 linear, LayerNorm -- the fp16
 output rounding (2^-11 relative) plus fp32 accumulation, checked as
 max|gpu - oracle| <= tol * max|oracle|.
 """
+import os
+import subprocess
+import sys
+
 import numpy as np
 import pytest
 import torch
@@ -260,10 +264,16 @@ def test_linear_split_k_deterministic(M, N, K):
     x = dev(si.normal_f16(17, 1, (M, K), 1.0))
     w16 = si.normal_f16(17, 2, (N, K), 0.02)
     wq = fg.fg_quantize(dev(w16), dim=1)
-    assert fg.fg_linear_workspace_bytes(M, N, K) == 0       # partial sums stay on chip
     y1 = fg.fg_linear_w4a16(x, wq)
     y2 = fg.fg_linear_w4a16(x, wq)
     assert torch.equal(y1, y2)
+    if M <= 256:
+        assert fg.fg_linear_workspace_bytes(M, N, K) == 0   # one-SM tiles add partials on chip
+    else:
+        # CTA-pair tiles: through the scratch by default, on chip without one; same bits
+        assert fg.fg_linear_workspace_bytes(M, N, K) > 0
+        y3 = fg.fg_linear_w4a16(x, wq, workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+        assert torch.equal(y1, y3)
     ref = oracle.linear(host(x), oracle.quantize(w16, 1))
     assert np.max(np.abs(host(y1).astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref))
 
@@ -281,6 +291,14 @@ def test_linear_split_k_residual_sampled(M, N, K):
     y1 = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), residual=dev(r))
     y2 = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), residual=dev(r))
     assert torch.equal(y1, y2)
+    if K >= 4096:
+        assert fg.fg_linear_workspace_bytes(M, N, K) > 0        # these shapes split the k-range
+    if fg.fg_linear_workspace_bytes(M, N, K):
+        # partial sums added through the scratch (above) or, with too little scratch, on chip
+        # over distributed shared memory: the same order of additions, the same bits
+        y3 = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), residual=dev(r),
+                                workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+        assert torch.equal(y1, y3)
     rows = np.unique(np.concatenate([np.random.default_rng(M).choice(M, 20, replace=False), [0, 255, 256, 511, M - 1]]))
     ref = oracle.linear(x[rows], oracle.quantize(w16, 1), bias=b, residual=r[rows])
     got = host(y1)[rows].astype(np.float64)
@@ -304,3 +322,22 @@ def test_layernorm_matches_oracle(M, h):
     y = fg.fg_layernorm(dev(x), dev(g), dev(b))
     ref = oracle.layernorm(x, g, b)
     assert np.max(np.abs(host(y).astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref))
+
+
+def test_linear_plan_in_a_fresh_process_before_any_launch():
+    # the split-k plan (and so the scratch size) must not depend on whether a GEMM has run in
+    # the process yet: query it first thing in a new interpreter, then after a launch
+    code = (
+        "import torch, bit_compressed_decode_b200 as fg\n"
+        "torch.cuda.init()\n"
+        "a = fg.fg_linear_workspace_bytes(512, 4096, 4096)\n"
+        "x = torch.zeros((512, 4096), dtype=torch.float16, device='cuda')\n"
+        "w = fg.fg_quantize(torch.zeros((4096, 4096), dtype=torch.float16, device='cuda'), dim=1)\n"
+        "fg.fg_linear_w4a16(x, w)\n"
+        "torch.cuda.synchronize()\n"
+        "print(a, fg.fg_linear_workspace_bytes(512, 4096, 4096))\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    before, after = map(int, out.stdout.split()[-2:])
+    assert before == after > 0
