@@ -74,6 +74,7 @@ _decl("fg_kv_cache_bytes", c_int, c_int, c_int, c_int, c_int, POINTER(c_size_t),
 _decl("fg_kv_append", c_int, POINTER(fg_kv_cache), P, P, c_int64, c_int, c_int, P, P)
 _decl("fg_attention_decode", c_int, POINTER(fg_kv_cache), P, c_int64, P, c_int64, c_int, c_int, P, P)
 _decl("fg_linear_workspace_bytes", c_size_t, c_int, c_int, c_int)
+_decl("fg_linear_plan", c_int, c_int, c_int, c_int, POINTER(c_int), POINTER(c_int))
 _decl("fg_linear_w4a16", c_int, P, c_int, c_int, POINTER(fg_qtensor), P, P, c_int, c_int, c_float, P, P, c_size_t, P)
 _decl("fg_layernorm", c_int, P, c_int, c_int, P, P, c_float, P, P)
 _decl("fg_layer_blob_bytes", c_size_t, POINTER(fg_layer_config))
@@ -252,6 +253,13 @@ def fg_attention_decode(cache: KVCache, q: torch.Tensor, positions: torch.Tensor
 
 def fg_linear_workspace_bytes(M: int, N: int, K: int) -> int:
     return int(_lib.fg_linear_workspace_bytes(M, N, K))
+
+
+def fg_linear_plan(M: int, N: int, K: int) -> tuple:
+    """(tokens per output tile, k splits) of the launch fg_linear_w4a16 makes for this shape."""
+    t, s = c_int(), c_int()
+    _check(_lib.fg_linear_plan(M, N, K, ctypes.byref(t), ctypes.byref(s)), "fg_linear_plan")
+    return t.value, s.value
 
 
 def fg_linear_w4a16(x: torch.Tensor, w: QTensor, bias=None, residual=None, relu: bool = False,

@@ -346,23 +346,34 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
 //   gives one, else over distributed shared memory.
 // ------------------------------------------------------------------------------------
 
-constexpr int kPairTok = 512;                  // tokens per pair tile
-constexpr int kPairStages = 4;
 constexpr int kPairA = 128 * 128;              // this CTA's A tile: 128 rows x 128 B
 constexpr int kPairBHalf = 128 * 128;          // this CTA's half of one token tile: 128 tokens x 128 B
-constexpr int kPairStage = kPairA + 2 * kPairBHalf;
-constexpr int kPairRing = kPairStages * kPairStage;
+constexpr int kPairRing = 192 * 1024;          // pipeline ring (both tile sizes)
 constexpr int kPairSmem = kPairRing + 1024;
-constexpr int kPairCols = 512;
 constexpr int kPairPrefetch = 4;
+// NTT 256-token MMA tiles per pair tile: 2 (512 tokens, the A tile feeds two MMAs per k
+// step) or 1 (256 tokens: half the partial sums when the k-range is split, twice the
+// dequantisation per flop)
+template <int NTT>
+struct PairCfg {
+  static constexpr int kTok = 256 * NTT;               // tokens per pair tile
+  static constexpr int kStage = kPairA + NTT * kPairBHalf;
+  static constexpr int kStages = kPairRing / kStage;   // 4 or 6
+  static constexpr int kCols = 256 * NTT;              // TMEM columns (fp32 accumulators)
+  static constexpr int kChunks = kCols / 32;           // 32-token epilogue chunks
+  static_assert(kStages * kStage == kPairRing, "ring");
+};
 constexpr uint32_t kPairIdesc = umma_idesc_f16_f32(256, 256);
 // warps 0..7 dequant + epilogue, 8 TMA, 9 MMA issuer (even CTA) or "A half ready"
 // forwarder (odd CTA), and TMEM allocation.  Ten warps leave room for ~168 registers per
 // thread (the register file is split over the four schedulers).
 constexpr int kPairThreads = (kDeqWarps + 2) * 32;
 
+template <int NTT>
 __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                       const GemmArgs a) {
+  using C = PairCfg<NTT>;
+  constexpr int kPairStages = C::kStages, kPairStage = C::kStage, kPairTok = C::kTok, kPairCols = C::kCols;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // full (even CTA): the stage is ready -- its 8 dequant warps arrive, its TMA thread
@@ -480,9 +491,9 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
             !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kPairStages) - 1) & 1, abortp, a.err))
           break;
         const uint32_t fb = mapa_shared(smem_u32(&full[st]), lead);
-        if (leader) mbar_arrive_expect_tx(smem_u32(&full[st]), 4 * kPairBHalf + 16);  // x of both CTAs + token
+        if (leader) mbar_arrive_expect_tx(smem_u32(&full[st]), 2 * NTT * kPairBHalf + 16);  // x of both CTAs + token
 #pragma unroll
-        for (int tile = 0; tile < 2; tile++)
+        for (int tile = 0; tile < NTT; tile++)
           tma_load_2d_pair(smem_u32(b_tile(st, tile)), &xmap, (kt0 + i) * kBK, t0 + tile * 256 + half * 128, fb);
       }
     }
@@ -516,7 +527,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; kk++) {
 #pragma unroll
-          for (int tile = 0; tile < 2; tile++)
+          for (int tile = 0; tile < NTT; tile++)
             umma_f16_pair(tmem + tile * 256, ad + 2 * kk, bd + tile * kTileStep + 2 * kk, kPairIdesc,
                           (i > 0 || kk > 0) ? 1u : 0u);
         }
@@ -544,13 +555,13 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
   const int f8 = (tid & 15) * 8, mj0 = (tid >> 4) & 15;
   const int nb = n0 + f8;
   if (a.splits == 1 && !a.res) {
-    __half *hbuf = reinterpret_cast<__half *>(smem);  // [16 chunks][32 tokens][128 features]
+    __half *hbuf = reinterpret_cast<__half *>(smem);  // [chunks][32 tokens][128 features]
     if (warp < kDeqWarps) {
       const int n = n0 + q * 32 + lane;
       const float bias = (a.bias && n < a.N) ? __half2float(a.bias[n]) : 0.f;
       const float qs = n < a.qcols ? a.qscale : 1.f;
-      for (int c8 = 0; c8 < 8; c8++) {
-        const int ch = etile * 8 + c8;
+      for (int c8 = 0; c8 < C::kChunks / 2; c8++) {
+        const int ch = etile * (C::kChunks / 2) + c8;
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, v);
         tmem_wait_ld();
@@ -906,13 +917,14 @@ fg_status launch_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cu
 
 // ---- pair kernel planning ----
 
+template <int NTT>
 fg_status pair_attr_once() {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     fg_status rc = fg_cuda_check(
-        cudaFuncSetAttribute(w4a16_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem));
+        cudaFuncSetAttribute(w4a16_gemm_pair_kernel<NTT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem));
     if (rc != FG_OK) return rc;
     attr_set[dev] = true;
   }
@@ -921,6 +933,7 @@ fg_status pair_attr_once() {
 
 // Pair-kernel clusters (2 x 1 x splits CTAs) that can be resident at once; 0 when such a
 // cluster does not fit on the device.
+template <int NTT>
 int pair_clusters_resident(int splits) {
   static int cache[64][5];
   static bool known[64][5] = {};
@@ -928,7 +941,7 @@ int pair_clusters_resident(int splits) {
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || splits < 1 || splits > 4) return 0;
   // the occupancy query needs the kernel's shared-memory attribute; a failed query is not cached
-  if (pair_attr_once() != FG_OK) return 0;
+  if (pair_attr_once<NTT>() != FG_OK) return 0;
   if (!known[dev][splits]) {
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(2, 1, splits);
@@ -942,7 +955,7 @@ int pair_clusters_resident(int splits) {
     lc.attrs = attr;
     lc.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, w4a16_gemm_pair_kernel, &lc) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, w4a16_gemm_pair_kernel<NTT>, &lc) != cudaSuccess) {
       cudaGetLastError();
       return 0;
     }
@@ -952,32 +965,45 @@ int pair_clusters_resident(int splits) {
   return cache[dev][splits];
 }
 
-// Splits of the k-range (the cluster's z dimension, at most 4) that minimise
-// waves of resident clusters * k-tiles per CTA, with a small charge per extra split.
+// Tile size (256 or 512 tokens) and k splits (the cluster's z dimension, at most 4) by a
+// time model in microseconds, measured on B200 for this kernel: a k-tile takes about
+// 0.70 us at 512 tokens and 0.63 us at 256 (half the MMA work, the same dequantisation
+// and pipeline hand-offs); each wave pays its pipeline fill (~5 us) and the epilogue, whose
+// partial sums grow with the tile and the number of splits.
 Plan make_pair_plan(int M, int N, int K) {
   Plan p;
-  p.nt = kPairTok;
   p.n_tiles = (N + 255) / 256;  // CTA pairs along the features
-  p.t_tiles = (M + kPairTok - 1) / kPairTok;
-  const int ktiles = K / kBK;
-  const int clusters = p.n_tiles * p.t_tiles;
-  double best = 1e30;
+  p.nt = 512;
   p.splits = 1;
-  for (int s = 1; s <= 4; s++) {
-    if (s > 1 && ktiles / s < 8) break;
-    const int resident = pair_clusters_resident(s);
-    if (resident == 0) continue;
-    const int waves = (clusters + resident - 1) / resident;
-    const double cost = static_cast<double>(waves) * ((ktiles + s - 1) / s) * (1.0 + 0.05 * (s - 1));
-    if (cost < best - 1e-9) {
-      best = cost;
-      p.splits = s;
+  const int ktiles = K / kBK;
+  double best = 1e30;
+  for (int ntt = 2; ntt >= 1; ntt--) {
+    const int tok = 256 * ntt;
+    const int t_tiles = (M + tok - 1) / tok;
+    const int clusters = p.n_tiles * t_tiles;
+    const double ktime = ntt == 2 ? 0.70 : 0.63;
+    for (int s = 1; s <= 4; s++) {
+      if (s > 1 && ktiles / s < 8) break;
+      const int resident = ntt == 2 ? pair_clusters_resident<2>(s) : pair_clusters_resident<1>(s);
+      if (resident == 0) continue;
+      const int waves = (clusters + resident - 1) / resident;
+      const double epi = 3.0 * ntt + (s > 1 ? 4.0 * ntt + 1.0 * s : 0.0);
+      const double cost = waves * (((ktiles + s - 1) / s) * ktime + 5.0 + epi);
+      if (cost < best - 1e-9) {
+        best = cost;
+        p.nt = tok;
+        p.splits = s;
+      }
     }
   }
+  p.t_tiles = (M + p.nt - 1) / p.nt;
   return p;
 }
 
-fg_status launch_pair(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st) {
+template <int NTT>
+fg_status launch_pair_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st) {
+  fg_status rc = pair_attr_once<NTT>();
+  if (rc != FG_OK) return rc;
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(2 * p.n_tiles, p.t_tiles, p.splits);
   lc.blockDim = dim3(kPairThreads, 1, 1);
@@ -990,20 +1016,26 @@ fg_status launch_pair(const CUtensorMap &map, const GemmArgs &a, const Plan &p, 
   attr[0].val.clusterDim.z = p.splits;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  fg_status rc = fg_cuda_check(cudaLaunchKernelEx(&lc, w4a16_gemm_pair_kernel, map, a));
+  rc = fg_cuda_check(cudaLaunchKernelEx(&lc, w4a16_gemm_pair_kernel<NTT>, map, a));
   if (rc != FG_OK) return rc;
   return fg_launch_check();
 }
 
+fg_status launch_pair(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st) {
+  return p.nt == 256 ? launch_pair_nt<1>(map, a, p, st) : launch_pair_nt<2>(map, a, p, st);
+}
+
 }  // namespace
 
-// Optional scratch of the pair kernel's k split: one fp32 partial [512 tokens][256 features]
+// Optional scratch of the pair kernel's k split: one fp32 partial [tile tokens][256 features]
 // per split of every pair tile.  Without it the partials are reduced inside the cluster.
+size_t pair_part_bytes(const Plan &p) {
+  return p.splits < 2 ? 0 : static_cast<size_t>(p.n_tiles) * p.t_tiles * p.splits * p.nt * 256 * sizeof(float);
+}
+
 size_t fg_linear_ws_bytes(int M, int N, int K) {
   if (M <= 256 || N <= 0 || K <= 0 || K % kBK) return 0;
-  const Plan p = make_pair_plan(M, N, K);
-  if (p.splits < 2) return 0;
-  return static_cast<size_t>(p.n_tiles) * p.t_tiles * p.splits * kPairTok * 256 * sizeof(float);
+  return pair_part_bytes(make_pair_plan(M, N, K));
 }
 
 fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, const fg_half *bias,
@@ -1012,10 +1044,6 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
   const int N = static_cast<int>(w->shape[0]);
   if (M == 0) return FG_OK;
   const bool pair = M > 256;
-  if (pair) {
-    fg_status rc = pair_attr_once();
-    if (rc != FG_OK) return rc;
-  }
   Plan p = pair ? make_pair_plan(M, N, K) : make_plan(M, N, K);
   EncodeTiledFn enc = encode_fn();
   if (!enc) return FG_ERR_CUDA;
@@ -1043,8 +1071,7 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
   a.qscale = qscale;
   a.splits = p.splits;
   a.part = nullptr;
-  if (pair && p.splits > 1 && workspace && fg_aligned16(workspace) &&
-      ws_bytes >= static_cast<size_t>(p.n_tiles) * p.t_tiles * p.splits * kPairTok * 256 * sizeof(float))
+  if (pair && p.splits > 1 && workspace && fg_aligned16(workspace) && ws_bytes >= pair_part_bytes(p))
     a.part = static_cast<float *>(workspace);
   a.err = fg_error_word_ptr();
   if (!a.err) return FG_ERR_CUDA;
@@ -1059,6 +1086,14 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
 }
 
 extern "C" size_t fg_linear_workspace_bytes(int M, int N, int K) { return fg_linear_ws_bytes(M, N, K); }
+
+extern "C" fg_status fg_linear_plan(int M, int N, int K, int *tile_tokens, int *splits) {
+  if (!tile_tokens || !splits || M <= 0 || N <= 0 || K <= 0 || K % kBK || N % 128) return FG_ERR_INVALID;
+  const Plan p = M > 256 ? make_pair_plan(M, N, K) : make_plan(M, N, K);
+  *tile_tokens = p.nt;
+  *splits = p.splits;
+  return FG_OK;
+}
 
 extern "C" fg_status fg_linear_w4a16(const fg_half *x, int M, int K, const fg_qtensor *w, const fg_half *bias,
                                      const fg_half *residual, int flags, int qscale_cols, float qscale, fg_half *y,

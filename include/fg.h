@@ -183,6 +183,13 @@ enum {
  * Tensor cores dequantise W tiles in shared memory ([G3]: on-the-fly
  * dequantisation for FP16 compute). */
 FG_API size_t fg_linear_workspace_bytes(int M, int N, int K);
+/* The launch fg_linear_w4a16 makes for this shape on the current device (no
+ * launch): *tile_tokens = tokens per output tile (16..256 for M <= 256, one SM
+ * per tile; 256 or 512 for larger M, a CTA pair per tile), *splits = CTAs
+ * sharing each tile's k-range (1..8 one-SM, 1..4 pair).  Chosen by a time
+ * model of the kernels: waves of resident clusters x k-tiles per CTA, plus the
+ * pipeline fill and the epilogue. */
+FG_API fg_status fg_linear_plan(int M, int N, int K, int *tile_tokens, int *splits);
 FG_API fg_status fg_linear_w4a16(const fg_half *x, int M, int K, const fg_qtensor *w, const fg_half *bias,
                           const fg_half *residual, int flags, int qscale_cols, float qscale,
                           fg_half *y, void *workspace, size_t workspace_bytes, void *stream);

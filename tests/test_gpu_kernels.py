@@ -341,3 +341,15 @@ def test_linear_plan_in_a_fresh_process_before_any_launch():
     assert out.returncode == 0, out.stderr[-2000:]
     before, after = map(int, out.stdout.split()[-2:])
     assert before == after > 0
+
+
+def test_linear_parity_shapes_cover_every_pair_plan():
+    # the shapes the parity tests above run reach both pair tile sizes (256 and 512 tokens),
+    # each with and without a k split
+    shapes = [(257, 256, 128), (600, 640, 2048), (1100, 384, 1024), (520, 640, 4096), (300, 512, 256),
+              (300, 512, 2048), (512, 4096, 4096), (520, 4096, 4096), (600, 7680, 1024), (530, 5120, 1536),
+              (512, 4096, 16384), (512, 2304, 768), (300, 1280, 512)]
+    plans = {(M, N, K): fg.fg_linear_plan(M, N, K) for M, N, K in shapes}
+    seen = {(t, s > 1) for t, s in plans.values()}
+    for want in [(256, False), (256, True), (512, False), (512, True)]:
+        assert want in seen, (want, plans)
