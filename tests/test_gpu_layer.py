@@ -1,6 +1,6 @@
 """GPU parity of the whole OPT layer (prefill + decode), the block schedule and the stack.
 
-Tolerance (the benchmark spec): max relative error 1e-2 of the layer output
+Tolerance (the stated layer bound): max relative error 1e-2 of the layer output
 against the oracle's float64 evaluation of the same dequantised weights, read
 as max|gpu - ref| <= 1e-2 * max|ref| on D = x_out - x_in (the residual
 stream would otherwise hide errors in the attention and FFN branches).
