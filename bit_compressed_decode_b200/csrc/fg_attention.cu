@@ -163,6 +163,7 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ float red_m[kWarps], red_l[kWarps];
   __shared__ float red_o[kWarps][D];
+  griddep_launch();  // the output projection may start its weight-side prologue
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, c = lane & 3;

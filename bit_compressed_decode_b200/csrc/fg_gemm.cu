@@ -81,6 +81,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
+  griddep_launch();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n0 = blockIdx.x * kBM, t0 = blockIdx.y * NT, split = blockIdx.z;
   const int ktiles = a.K / kBK;
@@ -172,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
     // ---------------- TMA producer for the x tiles ----------------
     if (lane == 0) {
       prefetch_tmap(&xmap);
+      griddep_wait();  // x comes from the previous kernel
       int issued = 0;
       for (int i = 0; i < nk; i++) {
         const int st = i % C::STAGES;
@@ -215,6 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
   // ---------------- epilogue: TMEM -> registers -> global ----------------
   constexpr int kChunks = NT >= 32 ? NT / 32 : 1;  // 32-column chunks of the accumulator
   constexpr int kCW = NT >= 32 ? 32 : NT;          // columns per chunk
+  griddep_wait();  // residual and outputs: after the previous kernel has finished
   bool ready = false;
   if (warp < kDeqWarps) {
     ready = mbar_wait_bounded(smem_u32(&accum_bar), 0, nullptr, a.err) && !*abortp;
@@ -389,6 +392,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
+  griddep_launch();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t crank = cluster_ctarank();
   const uint32_t lead = crank & ~1u;
@@ -485,6 +489,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     // ---------------- TMA producer: this CTA's halves of the two token tiles ----------------
     if (lane == 0) {
       prefetch_tmap(&xmap);
+      griddep_wait();  // x comes from the previous kernel
       for (int i = 0; i < nk; i++) {
         const int st = i % kPairStages;
         if (i >= kPairStages &&
@@ -545,6 +550,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
   // fp32 chunks of [32 tokens][128 features] are staged kRound at a time and chunk ch is
   // finished by z rank ch % splits, which sums it over the cluster's z ranks in rank order
   // (deterministic) before the epilogue.  All threads of all CTAs take the same barriers.
+  griddep_wait();  // residual, outputs and scratch: after the previous kernel has finished
   bool ready = false;
   if (warp < kDeqWarps) {
     ready = mbar_wait_bounded_cluster(smem_u32(&accum_bar), 0, nullptr, a.err) && !*abortp;
@@ -885,8 +891,12 @@ Plan make_plan(int M, int N, int K) {
   return p;
 }
 
+// pdl: launch with programmatic stream serialisation -- the kernel's prologue (barriers,
+// TMEM, weight loads and their dequantisation) may overlap the previous kernel, which the
+// kernel waits for before it touches activations, residual or outputs.  Only for callers
+// whose weights the previous kernel cannot be writing.
 template <int NT>
-fg_status launch_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st) {
+fg_status launch_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st, bool pdl) {
   using C = Cfg<NT>;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -902,13 +912,15 @@ fg_status launch_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cu
   lc.blockDim = dim3(kThreads, 1, 1);
   lc.dynamicSmemBytes = C::SMEM;
   lc.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = p.splits;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
-  lc.numAttrs = 1;
+  lc.numAttrs = pdl ? 2 : 1;
   fg_status rc = fg_cuda_check(cudaLaunchKernelEx(&lc, w4a16_gemm_kernel<NT>, map, a));
   if (rc != FG_OK) return rc;
   return fg_launch_check();
@@ -1001,7 +1013,7 @@ Plan make_pair_plan(int M, int N, int K) {
 }
 
 template <int NTT>
-fg_status launch_pair_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st) {
+fg_status launch_pair_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st, bool pdl) {
   fg_status rc = pair_attr_once<NTT>();
   if (rc != FG_OK) return rc;
   cudaLaunchConfig_t lc = {};
@@ -1009,20 +1021,22 @@ fg_status launch_pair_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &
   lc.blockDim = dim3(kPairThreads, 1, 1);
   lc.dynamicSmemBytes = kPairSmem;
   lc.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = p.splits;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
-  lc.numAttrs = 1;
+  lc.numAttrs = pdl ? 2 : 1;
   rc = fg_cuda_check(cudaLaunchKernelEx(&lc, w4a16_gemm_pair_kernel<NTT>, map, a));
   if (rc != FG_OK) return rc;
   return fg_launch_check();
 }
 
-fg_status launch_pair(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st) {
-  return p.nt == 256 ? launch_pair_nt<1>(map, a, p, st) : launch_pair_nt<2>(map, a, p, st);
+fg_status launch_pair(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st, bool pdl) {
+  return p.nt == 256 ? launch_pair_nt<1>(map, a, p, st, pdl) : launch_pair_nt<2>(map, a, p, st, pdl);
 }
 
 }  // namespace
@@ -1040,7 +1054,7 @@ size_t fg_linear_ws_bytes(int M, int N, int K) {
 
 fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, const fg_half *bias,
                            const fg_half *residual, int flags, int qscale_cols, float qscale, fg_half *y,
-                           void *workspace, size_t ws_bytes, cudaStream_t st) {
+                           void *workspace, size_t ws_bytes, cudaStream_t st, bool pdl) {
   const int N = static_cast<int>(w->shape[0]);
   if (M == 0) return FG_OK;
   const bool pair = M > 256;
@@ -1075,13 +1089,13 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
     a.part = static_cast<float *>(workspace);
   a.err = fg_error_word_ptr();
   if (!a.err) return FG_ERR_CUDA;
-  if (pair) return launch_pair(map, a, p, st);
+  if (pair) return launch_pair(map, a, p, st, pdl);
   switch (p.nt) {
-    case 16: return launch_nt<16>(map, a, p, st);
-    case 32: return launch_nt<32>(map, a, p, st);
-    case 64: return launch_nt<64>(map, a, p, st);
-    case 128: return launch_nt<128>(map, a, p, st);
-    default: return launch_nt<256>(map, a, p, st);
+    case 16: return launch_nt<16>(map, a, p, st, pdl);
+    case 32: return launch_nt<32>(map, a, p, st, pdl);
+    case 64: return launch_nt<64>(map, a, p, st, pdl);
+    case 128: return launch_nt<128>(map, a, p, st, pdl);
+    default: return launch_nt<256>(map, a, p, st, pdl);
   }
 }
 
@@ -1108,6 +1122,7 @@ extern "C" fg_status fg_linear_w4a16(const fg_half *x, int M, int K, const fg_qt
   if (!x || !y || !w->codes || !w->mins || !w->scales) return FG_ERR_INVALID;
   if (!fg_aligned16(x) || !fg_aligned16(y) || !fg_aligned16(w->codes)) return FG_ERR_INVALID;
   if ((flags & FG_EPI_RESIDUAL) && (!residual || !fg_aligned16(residual))) return FG_ERR_INVALID;
+  // weights may come from the kernel just before (fg_quantize): no overlap with it
   return fg_linear_launch(x, M, K, w, bias, residual, flags, qscale_cols, qscale, y, workspace, workspace_bytes,
-                          static_cast<cudaStream_t>(stream));
+                          static_cast<cudaStream_t>(stream), false);
 }

@@ -129,6 +129,15 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 }
 
 // Every thread of every CTA in the cluster arrives (release) and waits (acquire).
+// Programmatic dependent launch.  A kernel launched with the programmatic-serialisation
+// attribute may start while the previous kernel in its stream is still running;
+// griddep_wait() blocks until that kernel has completed and its memory is visible, so it
+// must precede every read of data the previous kernel produced and every write the previous
+// kernel could still be reading.  griddep_launch() lets the next such kernel be scheduled
+// once every CTA of this grid has issued it (without it: once this grid completes).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }

@@ -15,7 +15,7 @@ fg_status fg_layernorm_launch(const fg_half *x, int M, int h, const fg_half *gam
                               fg_half *y, cudaStream_t st);
 fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, const fg_half *bias,
                            const fg_half *residual, int flags, int qscale_cols, float qscale, fg_half *y,
-                           void *workspace, size_t ws_bytes, cudaStream_t st);
+                           void *workspace, size_t ws_bytes, cudaStream_t st, bool pdl);
 size_t fg_linear_ws_bytes(int M, int N, int K);
 fg_status fg_kv_validate(const fg_kv_cache *kv);
 fg_status fg_kv_append_launch(const fg_kv_cache *kv, const fg_half *k, const fg_half *v, int64_t ld, int rows,
@@ -133,6 +133,11 @@ fg_status run_layer(const fg_layer_config *c, const fg_layer_weights *w, const f
   void *gws = ws + L.gemm;
   const size_t gbytes = ws_bytes - L.gemm;
   const float qscale = 1.0f / sqrtf(static_cast<float>(c->head_dim));
+  // Decode steps launch the GEMMs with programmatic dependent launch: a GEMM's prologue
+  // (weight loads and dequantisation; the weights are fixed for the call) overlaps the
+  // kernel before it.  Not for prompts, whose attention can outlast the GEMM's bounded
+  // pipeline waits.
+  const bool pdl = rows_per_seq == 1;
   fg_status rc;
   int ev;
 #define FG_STEP(slot, call)                    \
@@ -142,19 +147,19 @@ fg_status run_layer(const fg_layer_config *c, const fg_layer_weights *w, const f
   // a = LN1(x)
   FG_STEP(0, fg_layernorm_launch(x_in, rows, h, w->ln1_g, w->ln1_b, c->ln_eps, a, st));
   // [q k v] = a Wqkv^T + bqkv; q *= d^-1/2
-  FG_STEP(1, fg_linear_launch(a, rows, h, &w->wqkv, w->bqkv, nullptr, 0, h, qscale, qkv, gws, gbytes, st));
+  FG_STEP(1, fg_linear_launch(a, rows, h, &w->wqkv, w->bqkv, nullptr, 0, h, qscale, qkv, gws, gbytes, st, pdl));
   // append k, v (4-bit) at the sequences' positions
   FG_STEP(2, fg_kv_append_launch(kv, qkv + h, qkv + 2 * h, 3 * h, rows, rows_per_seq, positions, st));
   // o = softmax(q K^T) V over the 4-bit cache
   FG_STEP(3, fg_attention_launch(kv, qkv, 3 * h, o, h, rows, rows_per_seq, positions, st));
   // h1 = x + o Wo^T + bo
-  FG_STEP(4, fg_linear_launch(o, rows, h, &w->wo, w->bo, x_in, FG_EPI_RESIDUAL, 0, 1.f, h1, gws, gbytes, st));
+  FG_STEP(4, fg_linear_launch(o, rows, h, &w->wo, w->bo, x_in, FG_EPI_RESIDUAL, 0, 1.f, h1, gws, gbytes, st, pdl));
   // a = LN2(h1)
   FG_STEP(5, fg_layernorm_launch(h1, rows, h, w->ln2_g, w->ln2_b, c->ln_eps, a, st));
   // f = relu(a W1^T + b1)
-  FG_STEP(6, fg_linear_launch(a, rows, h, &w->w1, w->b1, nullptr, FG_EPI_RELU, 0, 1.f, f, gws, gbytes, st));
+  FG_STEP(6, fg_linear_launch(a, rows, h, &w->w1, w->b1, nullptr, FG_EPI_RELU, 0, 1.f, f, gws, gbytes, st, pdl));
   // x_out = h1 + f W2^T + b2
-  FG_STEP(7, fg_linear_launch(f, rows, F, &w->w2, w->b2, h1, FG_EPI_RESIDUAL, 0, 1.f, x_out, gws, gbytes, st));
+  FG_STEP(7, fg_linear_launch(f, rows, F, &w->w2, w->b2, h1, FG_EPI_RESIDUAL, 0, 1.f, x_out, gws, gbytes, st, pdl));
 #undef FG_STEP
   return FG_OK;
 }

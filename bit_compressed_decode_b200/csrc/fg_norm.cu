@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(kThreads) layernorm_kernel(const uint4 *__rest
                                                              const uint4 *__restrict__ beta, float eps,
                                                              uint4 *__restrict__ y) {
   __shared__ float red[2 * (kThreads / 32)];
+  griddep_launch();  // the GEMM after this kernel may start its weight-side prologue
   const int nvec = h / 8;
   const uint4 *xr = x + static_cast<int64_t>(blockIdx.x) * nvec;
   uint4 *yr = y + static_cast<int64_t>(blockIdx.x) * nvec;

@@ -59,6 +59,12 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_dequantize.argtypes = [P, P, P, I64, I64, I64, P]
         _lib.oracle_linear.restype = I
         _lib.oracle_linear.argtypes = [P, I, I, P, P, P, I, P, P, I, I, D, P]
+        _lib.oracle_quantize_g.restype = I
+        _lib.oracle_quantize_g.argtypes = [P, I64, I64, I64, P, P, P, I]
+        _lib.oracle_dequantize_g.restype = I
+        _lib.oracle_dequantize_g.argtypes = [P, P, P, I64, I64, I64, P, I]
+        _lib.oracle_linear_g.restype = I
+        _lib.oracle_linear_g.argtypes = [P, I, I, P, P, P, I, P, P, I, I, D, P, I]
         _lib.oracle_layernorm.restype = I
         _lib.oracle_layernorm.argtypes = [P, I, I, P, P, D, P]
         _lib.oracle_kv_append.restype = I
@@ -106,11 +112,11 @@ def f64_to_f16(x) -> np.ndarray:
 # --------------------------------------------------------------------------------------
 
 class Packed:
-    """Planar 4-bit tensor: codes uint8 (dim halved), mins/scales float16 (dim / 64)."""
+    """Planar 4-bit tensor: codes uint8 (dim halved), mins/scales float16 (dim / group)."""
 
-    def __init__(self, codes, mins, scales, shape, dim):
+    def __init__(self, codes, mins, scales, shape, dim, group: int = GROUP):
         self.codes, self.mins, self.scales = codes, mins, scales
-        self.shape, self.dim = tuple(shape), dim
+        self.shape, self.dim, self.group = tuple(shape), dim, group
 
 
 def _split(shape, dim):
@@ -120,27 +126,30 @@ def _split(shape, dim):
     return dim, outer, int(shape[dim]), inner
 
 
-def quantize(x, dim: int = -1) -> Packed:
-    """Group-wise (64) asymmetric min-max 4-bit quantisation along ``dim``."""
+def quantize(x, dim: int = -1, group: int = GROUP) -> Packed:
+    """Group-wise asymmetric min-max 4-bit quantisation along ``dim``, groups of 64 or 128
+    consecutive elements ("FlexGen Guide", section 3: groups of 64 or 128)."""
     x = _u16(x)
     dim, outer, n, inner = _split(x.shape, dim)
-    if n % GROUP:
-        raise ValueError("size along dim must be a multiple of 64")
+    if group not in (64, 128):
+        raise ValueError("group must be 64 or 128")
+    if n % group:
+        raise ValueError(f"size along dim must be a multiple of {group}")
     cshape = list(x.shape); cshape[dim] = n // 2
-    mshape = list(x.shape); mshape[dim] = n // GROUP
+    mshape = list(x.shape); mshape[dim] = n // group
     codes = np.empty(cshape, dtype=np.uint8)
     mins = np.empty(mshape, dtype=np.uint16)
     scales = np.empty(mshape, dtype=np.uint16)
-    rc = lib().oracle_quantize(_p(x), outer, n, inner, _p(codes), _p(mins), _p(scales))
+    rc = lib().oracle_quantize_g(_p(x), outer, n, inner, _p(codes), _p(mins), _p(scales), group)
     assert rc == 0
-    return Packed(codes, mins.view(np.float16), scales.view(np.float16), x.shape, dim)
+    return Packed(codes, mins.view(np.float16), scales.view(np.float16), x.shape, dim, group)
 
 
 def dequantize(q: Packed) -> np.ndarray:
     dim, outer, n, inner = _split(q.shape, q.dim)
     y = np.empty(q.shape, dtype=np.uint16)
-    rc = lib().oracle_dequantize(_p(np.ascontiguousarray(q.codes)), _p(_u16(q.mins)), _p(_u16(q.scales)),
-                                 outer, n, inner, _p(y))
+    rc = lib().oracle_dequantize_g(_p(np.ascontiguousarray(q.codes)), _p(_u16(q.mins)), _p(_u16(q.scales)),
+                                   outer, n, inner, _p(y), q.group)
     assert rc == 0
     return y.view(np.float16)
 
@@ -157,10 +166,10 @@ def linear(x, w: Packed, bias=None, residual=None, relu: bool = False,
     N = w.shape[0]
     assert w.shape == (N, K) and w.dim == 1
     y = np.empty((M, N), dtype=np.float64)
-    rc = lib().oracle_linear(_p(x), M, K, _p(np.ascontiguousarray(w.codes)), _p(_u16(w.mins)), _p(_u16(w.scales)), N,
-                             _p(None if bias is None else _u16(bias)),
-                             _p(None if residual is None else _u16(residual)),
-                             int(relu), int(qscale_cols), float(qscale), _p(y))
+    rc = lib().oracle_linear_g(_p(x), M, K, _p(np.ascontiguousarray(w.codes)), _p(_u16(w.mins)), _p(_u16(w.scales)),
+                               N, _p(None if bias is None else _u16(bias)),
+                               _p(None if residual is None else _u16(residual)),
+                               int(relu), int(qscale_cols), float(qscale), _p(y), w.group)
     assert rc == 0
     return y
 

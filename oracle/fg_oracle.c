@@ -46,7 +46,8 @@
 #include <stdlib.h>
 #include <string.h>
 
-#define OR_GROUP 64
+#define OR_GROUP 64       /* the layer's group size */
+#define OR_GROUP_MAX 128  /* quantise/dequantise/linear also take groups of 128 [G3] */
 
 /* ------------------------------------------------------------------------- */
 /* binary16 conversions, written from the IEEE 754 binary16 format:          */
@@ -116,7 +117,7 @@ void oracle_f64_to_f16_array(const double *x, uint16_t *out, int64_t n)
 /* ------------------------------------------------------------------------- */
 
 /*
- * One group of 64 fp16 values x[i*xs] -> 32 packed bytes codes[j*cs]
+ * One group of `group` (64 or 128) fp16 values x[i*xs] -> group/2 packed bytes codes[j*cs]
  * (byte j = code(2j) | code(2j+1) << 4), fp16 min and fp16 scale.
  * Steps, in this order, each one IEEE fp32 operation:
  *   1. mn = min(x), mx = max(x);  mn = mn + 0  (turns -0 into +0)
@@ -129,12 +130,12 @@ void oracle_f64_to_f16_array(const double *x, uint16_t *out, int64_t n)
  *   8. min_h = fp16(mn)      (exact: mn is one of the fp16 inputs)
  */
 static void quantize_group(const uint16_t *x, ptrdiff_t xs, uint8_t *codes, ptrdiff_t cs,
-                           uint16_t *min_out, uint16_t *scale_out)
+                           uint16_t *min_out, uint16_t *scale_out, int group)
 {
-    float v[OR_GROUP];
-    for (int i = 0; i < OR_GROUP; i++) v[i] = oracle_f16_to_f32(x[i * xs]);
+    float v[OR_GROUP_MAX];
+    for (int i = 0; i < group; i++) v[i] = oracle_f16_to_f32(x[i * xs]);
     float mn = v[0], mx = v[0];
-    for (int i = 1; i < OR_GROUP; i++) {
+    for (int i = 1; i < group; i++) {
         if (v[i] < mn) mn = v[i];
         if (v[i] > mx) mx = v[i];
     }
@@ -143,13 +144,13 @@ static void quantize_group(const uint16_t *x, ptrdiff_t xs, uint8_t *codes, ptrd
     float q15 = d / 15.0f;
     uint16_t scale_h = oracle_f32_to_f16(q15);
     float s = oracle_f16_to_f32(scale_h);
-    int q[OR_GROUP];
+    int q[OR_GROUP_MAX];
     if (s == 0.0f) {
         scale_h = 0;
-        for (int i = 0; i < OR_GROUP; i++) q[i] = 0;
+        for (int i = 0; i < group; i++) q[i] = 0;
     } else {
         float inv = 1.0f / s;
-        for (int i = 0; i < OR_GROUP; i++) {
+        for (int i = 0; i < group; i++) {
             float diff = v[i] - mn;
             float t = diff * inv;
             float r = nearbyintf(t);          /* default mode: nearest, ties to even */
@@ -159,7 +160,7 @@ static void quantize_group(const uint16_t *x, ptrdiff_t xs, uint8_t *codes, ptrd
             q[i] = c;
         }
     }
-    for (int j = 0; j < OR_GROUP / 2; j++)
+    for (int j = 0; j < group / 2; j++)
         codes[j * cs] = (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
     *min_out = oracle_f32_to_f16(mn);
     *scale_out = scale_h;
@@ -175,23 +176,47 @@ static uint16_t dequant_one(int q, uint16_t min_h, uint16_t scale_h)
     return oracle_f64_to_f16((double)q * s + m);
 }
 
+static int group_ok(int group) { return group == 64 || group == 128; }
+
 /*
- * x viewed as [outer, n, inner]; groups of 64 consecutive elements along n.
- * codes: [outer, n/2, inner]   mins, scales: [outer, n/64, inner].
- * Returns 0, or -1 when n is not a multiple of 64.
+ * x viewed as [outer, n, inner]; groups of `group` (64 or 128) consecutive elements
+ * along n.  codes: [outer, n/2, inner]   mins, scales: [outer, n/group, inner].
+ * Returns 0, or -1 for another group size or n not a multiple of the group.
  */
-int oracle_quantize(const uint16_t *x, int64_t outer, int64_t n, int64_t inner,
-                    uint8_t *codes, uint16_t *mins, uint16_t *scales)
+int oracle_quantize_g(const uint16_t *x, int64_t outer, int64_t n, int64_t inner,
+                      uint8_t *codes, uint16_t *mins, uint16_t *scales, int group)
 {
-    if (n % OR_GROUP) return -1;
-    int64_t ng = n / OR_GROUP;
+    if (!group_ok(group) || n % group) return -1;
+    int64_t ng = n / group;
     for (int64_t o = 0; o < outer; o++)
         for (int64_t g = 0; g < ng; g++)
             for (int64_t i = 0; i < inner; i++) {
-                const uint16_t *xp = x + (o * n + g * OR_GROUP) * inner + i;
-                uint8_t *cp = codes + (o * (n / 2) + g * (OR_GROUP / 2)) * inner + i;
+                const uint16_t *xp = x + (o * n + g * group) * inner + i;
+                uint8_t *cp = codes + (o * (n / 2) + g * (group / 2)) * inner + i;
                 int64_t m = (o * ng + g) * inner + i;
-                quantize_group(xp, inner, cp, inner, &mins[m], &scales[m]);
+                quantize_group(xp, inner, cp, inner, &mins[m], &scales[m], group);
+            }
+    return 0;
+}
+
+int oracle_quantize(const uint16_t *x, int64_t outer, int64_t n, int64_t inner,
+                    uint8_t *codes, uint16_t *mins, uint16_t *scales)
+{
+    return oracle_quantize_g(x, outer, n, inner, codes, mins, scales, OR_GROUP);
+}
+
+int oracle_dequantize_g(const uint8_t *codes, const uint16_t *mins, const uint16_t *scales,
+                        int64_t outer, int64_t n, int64_t inner, uint16_t *y, int group)
+{
+    if (!group_ok(group) || n % group) return -1;
+    int64_t ng = n / group;
+    for (int64_t o = 0; o < outer; o++)
+        for (int64_t e = 0; e < n; e++)
+            for (int64_t i = 0; i < inner; i++) {
+                uint8_t byte = codes[(o * (n / 2) + e / 2) * inner + i];
+                int q = (e & 1) ? (byte >> 4) : (byte & 15);
+                int64_t m = (o * ng + e / group) * inner + i;
+                y[(o * n + e) * inner + i] = dequant_one(q, mins[m], scales[m]);
             }
     return 0;
 }
@@ -199,17 +224,7 @@ int oracle_quantize(const uint16_t *x, int64_t outer, int64_t n, int64_t inner,
 int oracle_dequantize(const uint8_t *codes, const uint16_t *mins, const uint16_t *scales,
                       int64_t outer, int64_t n, int64_t inner, uint16_t *y)
 {
-    if (n % OR_GROUP) return -1;
-    int64_t ng = n / OR_GROUP;
-    for (int64_t o = 0; o < outer; o++)
-        for (int64_t e = 0; e < n; e++)
-            for (int64_t i = 0; i < inner; i++) {
-                uint8_t byte = codes[(o * (n / 2) + e / 2) * inner + i];
-                int q = (e & 1) ? (byte >> 4) : (byte & 15);
-                int64_t m = (o * ng + e / OR_GROUP) * inner + i;
-                y[(o * n + e) * inner + i] = dequant_one(q, mins[m], scales[m]);
-            }
-    return 0;
+    return oracle_dequantize_g(codes, mins, scales, outer, n, inner, y, OR_GROUP);
 }
 
 /* ------------------------------------------------------------------------- */
@@ -241,16 +256,17 @@ static void linear_row(const float *W, const double *b, const double *x, int N, 
 }
 
 /* Dequantise a [N][K] weight (groups along K) into float (exact for fp16 values). */
-static float *dequant_weight(const uint8_t *codes, const uint16_t *mins, const uint16_t *scales, int N, int K)
+static float *dequant_weight(const uint8_t *codes, const uint16_t *mins, const uint16_t *scales, int N, int K,
+                             int group)
 {
     float *W = (float *)malloc(sizeof(float) * (size_t)N * K);
     if (!W) return NULL;
-    int ng = K / OR_GROUP;
+    int ng = K / group;
     for (int64_t n = 0; n < N; n++)
         for (int k = 0; k < K; k++) {
             uint8_t byte = codes[n * (K / 2) + k / 2];
             int q = (k & 1) ? (byte >> 4) : (byte & 15);
-            int64_t m = n * ng + k / OR_GROUP;
+            int64_t m = n * ng + k / group;
             W[n * K + k] = (float)oracle_f16_to_f64(dequant_one(q, mins[m], scales[m]));
         }
     return W;
@@ -274,13 +290,13 @@ static double *f16_vec(const uint16_t *h, int64_t n, double dflt)
 /* y[m][n] = epilogue(sum_k x[m][k] * deq(W)[n][k] + b[n]) in float64.
    relu: max(0, .);  residual (fp16 [M][N]) added after the activation;
    the first qscale_cols outputs of each row are multiplied by qscale after the bias. */
-int oracle_linear(const uint16_t *x, int M, int K,
-                  const uint8_t *codes, const uint16_t *mins, const uint16_t *scales, int N,
-                  const uint16_t *bias, const uint16_t *residual, int relu,
-                  int qscale_cols, double qscale, double *y)
+int oracle_linear_g(const uint16_t *x, int M, int K,
+                    const uint8_t *codes, const uint16_t *mins, const uint16_t *scales, int N,
+                    const uint16_t *bias, const uint16_t *residual, int relu,
+                    int qscale_cols, double qscale, double *y, int group)
 {
-    if (K % OR_GROUP) return -1;
-    float *W = dequant_weight(codes, mins, scales, N, K);
+    if (!group_ok(group) || K % group) return -1;
+    float *W = dequant_weight(codes, mins, scales, N, K, group);
     double *b = f16_vec(bias, N, 0.0);
     double *xr = (double *)malloc(sizeof(double) * (size_t)K);
     if (!W || !b || !xr) return -2;
@@ -298,6 +314,14 @@ int oracle_linear(const uint16_t *x, int M, int K,
     }
     free(W); free(b); free(xr);
     return 0;
+}
+
+int oracle_linear(const uint16_t *x, int M, int K,
+                  const uint8_t *codes, const uint16_t *mins, const uint16_t *scales, int N,
+                  const uint16_t *bias, const uint16_t *residual, int relu,
+                  int qscale_cols, double qscale, double *y)
+{
+    return oracle_linear_g(x, M, K, codes, mins, scales, N, bias, residual, relu, qscale_cols, qscale, y, OR_GROUP);
 }
 
 int oracle_layernorm(const uint16_t *x, int M, int h, const uint16_t *gamma, const uint16_t *beta,
@@ -331,9 +355,9 @@ static void kv_store(const kv_t *kv, int s, int head, int pos, const uint16_t *k
     int ng = kv->d / OR_GROUP;
     for (int g = 0; g < ng; g++) {
         quantize_group(k16 + g * OR_GROUP, 1, kv->kc + slot * (kv->d / 2) + g * 32, 1,
-                       &kv->km[slot * ng + g], &kv->ks[slot * ng + g]);
+                       &kv->km[slot * ng + g], &kv->ks[slot * ng + g], OR_GROUP);
         quantize_group(v16 + g * OR_GROUP, 1, kv->vc + slot * (kv->d / 2) + g * 32, 1,
-                       &kv->vm[slot * ng + g], &kv->vs[slot * ng + g]);
+                       &kv->vm[slot * ng + g], &kv->vs[slot * ng + g], OR_GROUP);
     }
 }
 
@@ -509,10 +533,10 @@ int oracle_layer_rows(const int *dims, double eps,
     if (c.h != c.H * c.d || c.h % OR_GROUP || c.F % OR_GROUP || c.d % OR_GROUP) return -1;
     for (int r = 0; r < R; r++)
         if (seq_of_row[r] < 0 || seq_of_row[r] >= S || pos_of_row[r] < 0 || pos_of_row[r] >= maxL) return -2;
-    c.Wqkv = dequant_weight(qkv_c, qkv_m, qkv_s, 3 * c.h, c.h);
-    c.Wo = kv_only ? NULL : dequant_weight(o_c, o_m, o_s, c.h, c.h);
-    c.W1 = kv_only ? NULL : dequant_weight(f1_c, f1_m, f1_s, c.F, c.h);
-    c.W2 = kv_only ? NULL : dequant_weight(f2_c, f2_m, f2_s, c.h, c.F);
+    c.Wqkv = dequant_weight(qkv_c, qkv_m, qkv_s, 3 * c.h, c.h, OR_GROUP);
+    c.Wo = kv_only ? NULL : dequant_weight(o_c, o_m, o_s, c.h, c.h, OR_GROUP);
+    c.W1 = kv_only ? NULL : dequant_weight(f1_c, f1_m, f1_s, c.F, c.h, OR_GROUP);
+    c.W2 = kv_only ? NULL : dequant_weight(f2_c, f2_m, f2_s, c.h, c.F, OR_GROUP);
     c.bqkv = f16_vec(bqkv, 3 * c.h, 0.0); c.bo = f16_vec(bo, c.h, 0.0);
     c.b1 = f16_vec(b1, c.F, 0.0); c.b2 = f16_vec(b2, c.h, 0.0);
     c.g1 = f16_vec(ln1_g, c.h, 1.0); c.be1 = f16_vec(ln1_b, c.h, 0.0);

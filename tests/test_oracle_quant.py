@@ -251,3 +251,94 @@ def test_nibble_order_low_is_even():
 def test_rejects_non_multiple_of_64():
     with pytest.raises(ValueError):
         oracle.quantize(np.zeros((2, 96), dtype=np.float16))
+
+
+# ------------------------------------------------------------------ groups of 128 -----------
+# ("FlexGen Guide", section 3: groups of 64 or 128 elements)
+
+def test_ramp_group128_hand_worked(golden_dir):
+    g = _load(golden_dir, "quant_ramp_group128.json")
+    x = (np.arange(128) / 2).astype(np.float16).reshape(1, 128)
+    q = oracle.quantize(x, group=128)
+    assert q.mins.shape == (1, 1) and q.codes.shape == (1, 64)
+    assert int(q.scales.view(np.uint16)[0, 0]) == g["scale_bits"]
+    assert int(q.mins.view(np.uint16)[0, 0]) == g["min_bits"]
+    want = np.repeat(np.arange(16), g["code_run_lengths"])
+    assert np.array_equal(_nibbles(q.codes[0]), want)
+    assert list(q.codes[0, :4]) == g["first_bytes"]
+    y = oracle.dequantize(q).astype(np.float64)[0]
+    assert np.array_equal(y, np.asarray(g["dequant_by_code"])[want])
+    assert np.max(np.abs(y - np.arange(128) / 2)) <= 4.234375 / 2 + 2.0 ** -6
+
+
+def test_group128_of_two_halves_with_the_same_range_equals_group64():
+    # when each 64-half of a 128-group holds the group's min and max, both groupings see the
+    # same (min, max), so the scale and every code agree; a mistake in the 128-grouping
+    # (a wrong stride, half, or metadata slot) breaks the equality
+    rng = np.random.default_rng(5)
+    x = rng.uniform(-3, 5, (4, 512)).astype(np.float16)
+    for r in range(4):
+        for blk in range(4):
+            lo, hi = np.float16(-3.0 - r), np.float16(5.0 + blk)
+            x[r, blk * 128 + 3], x[r, blk * 128 + 64 + 7] = lo, lo
+            x[r, blk * 128 + 50], x[r, blk * 128 + 64 + 60] = hi, hi
+    a = oracle.quantize(x, group=128)
+    b = oracle.quantize(x, group=64)
+    assert np.array_equal(a.codes, b.codes)
+    assert np.array_equal(a.scales.view(np.uint16), b.scales.view(np.uint16)[:, ::2])
+    assert np.array_equal(a.scales.view(np.uint16), b.scales.view(np.uint16)[:, 1::2])
+    assert np.array_equal(a.mins.view(np.uint16), b.mins.view(np.uint16)[:, ::2])
+    assert np.array_equal(oracle.dequantize(a).view(np.uint16), oracle.dequantize(b).view(np.uint16))
+
+
+def test_group128_blocks_land_in_their_metadata_slots():
+    # block j of 128 holds values in [j, j + 0.5]: min of slot j is j, and a 128-group never
+    # mixes two blocks (with groups of 64 the same data gives two equal slots per block)
+    x = np.empty((2, 640), np.float16)
+    for j in range(5):
+        x[:, 128 * j:128 * (j + 1)] = (j + np.linspace(0.0, 0.5, 128)).astype(np.float16)
+    q = oracle.quantize(x, group=128)
+    assert q.mins.shape == (2, 5)
+    assert np.array_equal(q.mins.astype(np.float64), np.tile(np.arange(5.0), (2, 1)))
+    # dims: along a non-last dim equals the transposed tensor along the last dim
+    x3 = si.normal_f16(6, 99, (3, 256, 5), 1.0)
+    a = oracle.quantize(x3, dim=1, group=128)
+    b = oracle.quantize(np.ascontiguousarray(np.transpose(x3, (0, 2, 1))), dim=-1, group=128)
+    assert np.array_equal(a.codes, np.transpose(b.codes, (0, 2, 1)))
+    assert np.array_equal(a.scales.view(np.uint16), np.transpose(b.scales.view(np.uint16), (0, 2, 1)))
+
+
+@pytest.mark.parametrize("value", [0.0, -2.5, 1000.0])
+def test_constant_group128(value):
+    q = oracle.quantize(np.full((1, 128), value, np.float16), group=128)
+    assert np.all(q.codes == 0)
+    assert q.scales.view(np.uint16)[0, 0] == 0
+    assert np.all(oracle.dequantize(q) == np.float16(value))
+
+
+def test_group128_round_trip_bound():
+    x = si.sweep_tensor(seed=2, numel=1 << 16, row=4096)
+    q = oracle.quantize(x, group=128)
+    y = oracle.dequantize(q).astype(np.float64).reshape(-1, 128)
+    G = x.astype(np.float64).reshape(-1, 128)
+    s = q.scales.astype(np.float64).reshape(-1, 1)
+    assert np.array_equal(q.mins.astype(np.float64).reshape(-1), G.min(axis=1) + 0.0)
+    # |x - deq| <= scale/2 (fp32 step rounding) + half an fp16 spacing of the result
+    ulp = np.spacing(np.abs(y).astype(np.float16)).astype(np.float64)
+    assert np.all(np.abs(G - y) <= s / 2 * (1 + 2.0 ** -16) + ulp / 2)
+
+
+def test_group128_linear_indexes_its_groups():
+    # y = x deq(W)^T with W in groups of 128 along K, against numpy on the dequantised weights
+    x = si.normal_f16(7, 1, (5, 384), 1.0)
+    w = si.normal_f16(7, 2, (128, 384), 0.05)
+    q = oracle.quantize(w, dim=1, group=128)
+    ref = x.astype(np.float64) @ oracle.dequantize(q).astype(np.float64).T
+    assert np.allclose(oracle.linear(x, q), ref, rtol=0, atol=1e-5 * np.max(np.abs(ref)))
+
+
+def test_group_sizes_rejected():
+    with pytest.raises(ValueError):
+        oracle.quantize(np.zeros((2, 192), dtype=np.float16), group=128)
+    with pytest.raises(ValueError):
+        oracle.quantize(np.zeros((2, 192), dtype=np.float16), group=96)
