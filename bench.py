@@ -602,7 +602,8 @@ def run_kernel(args, wl):
     elif args.kernel.endswith("_gemm"):
         N, K = {"qkv_gemm": (3 * h, h), "out_gemm": (h, h), "fc1_gemm": (F, h), "fc2_gemm": (h, F)}[args.kernel]
         x = torch.randn((S, K), generator=g, device=dev, dtype=torch.float16)
-        wq = fg.fg_quantize(torch.randn((N, K), generator=g, device=dev, dtype=torch.float16) * 0.02, dim=1)
+        wq = fg.fg_quantize(torch.randn((N, K), generator=g, device=dev, dtype=torch.float16) * 0.02, dim=1,
+                            group=args.group)
         y = torch.empty((S, N), dtype=torch.float16, device=dev)
         # --gemm-scratch none: no split-k scratch, so split k-ranges are added on chip
         gws = torch.empty(16 if args.gemm_scratch == "none" else
@@ -613,12 +614,12 @@ def run_kernel(args, wl):
     elif args.kernel in ("quantize", "dequantize"):
         n = 1 << args.log2_elems
         x = torch.randn((n // 4096, 4096), generator=g, device=dev, dtype=torch.float16) * 0.02
-        q = fg.fg_quantize(x)
+        q = fg.fg_quantize(x, group=args.group)
         if args.kernel == "quantize":
-            run = lambda: fg.fg_quantize(x, out=q, stream=stream)
+            run = lambda: fg.fg_quantize(x, group=args.group, out=q, stream=stream)
         else:
             run = lambda: fg.fg_dequantize(q, stream=stream)
-        work, unit, peak = n * 2.5625, "GB/s", peaks["hbm"]
+        work, unit, peak = n * (2.5 + 4.0 / args.group), "GB/s", peaks["hbm"]
     else:
         raise SystemExit(f"unknown kernel {args.kernel}")
     for _ in range(args.warmup):
@@ -634,7 +635,7 @@ def run_kernel(args, wl):
     t = sorted(a.elapsed_time(b) / 1e3 for a, b in ev)
     med = t[len(t) // 2]
     scale = 1e12 if unit == "TFLOP/s" else 1e9
-    print(json.dumps({"kernel": args.kernel, "workload": args.workload, "seqs": S, "median_us": med * 1e6,
+    print(json.dumps({"kernel": args.kernel, "group": args.group, "workload": args.workload, "seqs": S, "median_us": med * 1e6,
                       "min_us": t[0] * 1e6, "achieved": work / med / scale, "unit": unit, "peak": peak,
                       "frac": work / med / scale / peak}), flush=True)
 
@@ -653,6 +654,8 @@ def main():
     ap.add_argument("--seqs", type=int, default=0, help="--kernel: sequences (default: the workload's block)")
     ap.add_argument("--log2-elems", type=int, default=28, help="--kernel quantize/dequantize: tensor size")
     ap.add_argument("--layers", type=int, default=0, help="stack workloads: number of layers (default: the model's)")
+    ap.add_argument("--group", type=int, choices=(64, 128), default=64,
+                    help="--kernel quantize/dequantize/*_gemm: quantisation group size")
     ap.add_argument("--gemm-scratch", choices=("auto", "none"), default="auto",
                     help="--kernel *_gemm: give the GEMM its split-k scratch (auto) or none (on-chip reduction)")
     args = ap.parse_args()

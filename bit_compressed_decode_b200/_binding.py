@@ -130,9 +130,9 @@ def _need(t: torch.Tensor, dtype, name: str) -> None:
 class QTensor:
     """Packed 4-bit tensor (device): codes uint8, mins/scales float16, grouped along ``dim``."""
 
-    def __init__(self, codes, mins, scales, shape, dim):
+    def __init__(self, codes, mins, scales, shape, dim, group: int = 64):
         self.codes, self.mins, self.scales = codes, mins, scales
-        self.shape, self.dim = tuple(int(s) for s in shape), dim
+        self.shape, self.dim, self.group = tuple(int(s) for s in shape), dim, group
 
     def struct(self) -> fg_qtensor:
         s = fg_qtensor()
@@ -140,7 +140,7 @@ class QTensor:
         s.ndim = len(self.shape)
         for i in range(4):
             s.shape[i] = self.shape[i] if i < len(self.shape) else 1
-        s.dim, s.bits, s.group = self.dim, 4, 64
+        s.dim, s.bits, s.group = self.dim, 4, self.group
         return s
 
 
@@ -165,11 +165,12 @@ def fg_quantize(x: torch.Tensor, dim: int = -1, bits: int = 4, group: int = 64, 
         ms = list(shape); ms[dim] //= group
         out = QTensor(torch.empty(cs, dtype=torch.uint8, device=x.device),
                       torch.empty(ms, dtype=torch.float16, device=x.device),
-                      torch.empty(ms, dtype=torch.float16, device=x.device), shape, dim)
+                      torch.empty(ms, dtype=torch.float16, device=x.device), shape, dim, group)
     s = out.struct()
     arr = (c_int64 * len(shape))(*shape)
     _check(_lib.fg_quantize(_ptr(x), len(shape), arr, dim, bits, group, ctypes.byref(s), _stream(stream)),
            "fg_quantize")
+    out.group = group
     return out
 
 

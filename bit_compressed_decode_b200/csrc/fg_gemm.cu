@@ -59,6 +59,7 @@ struct GemmArgs {
   int relu, qcols;
   float qscale;
   int splits;
+  int gshift;          // log2(group / 64): the weights' min/scale cover 1 (group 64) or 2 (128) k-tiles
   float *part;         // pair kernel, k split: fp32 partial sums through global memory, or null
   unsigned int *err;
 };
@@ -120,8 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
     const bool live = n < a.N;
     const int acc = row >> 7, r = row & 127;
     const uint4 *crow = reinterpret_cast<const uint4 *>(a.wc + static_cast<int64_t>(live ? n : 0) * (a.K / 2));
-    const __half *mrow = a.wm + static_cast<int64_t>(live ? n : 0) * (a.K / kBK);
-    const __half *srow = a.ws + static_cast<int64_t>(live ? n : 0) * (a.K / kBK);
+    const __half *mrow = a.wm + static_cast<int64_t>(live ? n : 0) * ((a.K / kBK) >> a.gshift);
+    const __half *srow = a.ws + static_cast<int64_t>(live ? n : 0) * ((a.K / kBK) >> a.gshift);
     uint4 cb[kPrefetch][2];
     __half mb[kPrefetch], sb[kPrefetch];
 #pragma unroll
@@ -130,8 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
         const int kt = kt0 + j;
         cb[j][0] = crow[kt * 2];
         cb[j][1] = crow[kt * 2 + 1];
-        mb[j] = mrow[kt];
-        sb[j] = srow[kt];
+        mb[j] = mrow[kt >> a.gshift];
+        sb[j] = srow[kt >> a.gshift];
       } else {
         cb[j][0] = cb[j][1] = make_uint4(0, 0, 0, 0);
         mb[j] = sb[j] = __ushort_as_half(0);
@@ -152,8 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
         const int kt = kt0 + i + kPrefetch;
         cb[kPrefetch - 1][0] = crow[kt * 2];
         cb[kPrefetch - 1][1] = crow[kt * 2 + 1];
-        mb[kPrefetch - 1] = mrow[kt];
-        sb[kPrefetch - 1] = srow[kt];
+        mb[kPrefetch - 1] = mrow[kt >> a.gshift];
+        sb[kPrefetch - 1] = srow[kt >> a.gshift];
       }
       if (i >= C::STAGES && !mbar_wait_bounded(smem_u32(&empty[st]), ((i / C::STAGES) - 1) & 1, abortp, a.err))
         break;
@@ -437,16 +438,16 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     const int n = n0 + row;
     const bool live = n < a.N;
     const uint4 *crow = reinterpret_cast<const uint4 *>(a.wc + static_cast<int64_t>(live ? n : 0) * (a.K / 2));
-    const __half *mrow = a.wm + static_cast<int64_t>(live ? n : 0) * (a.K / kBK);
-    const __half *srow = a.ws + static_cast<int64_t>(live ? n : 0) * (a.K / kBK);
+    const __half *mrow = a.wm + static_cast<int64_t>(live ? n : 0) * ((a.K / kBK) >> a.gshift);
+    const __half *srow = a.ws + static_cast<int64_t>(live ? n : 0) * ((a.K / kBK) >> a.gshift);
     uint4 cb[kPairPrefetch];
     __half mb[kPairPrefetch], sb[kPairPrefetch];
 #pragma unroll
     for (int j = 0; j < kPairPrefetch; j++) {
       if (j < nk && live) {
         cb[j] = crow[(kt0 + j) * 2 + hk];
-        mb[j] = mrow[kt0 + j];
-        sb[j] = srow[kt0 + j];
+        mb[j] = mrow[(kt0 + j) >> a.gshift];
+        sb[j] = srow[(kt0 + j) >> a.gshift];
       } else {
         cb[j] = make_uint4(0, 0, 0, 0);
         mb[j] = sb[j] = __ushort_as_half(0);
@@ -467,8 +468,8 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
       if (i + kPairPrefetch < nk && live) {
         const int kt = kt0 + i + kPairPrefetch;
         cb[kPairPrefetch - 1] = crow[kt * 2 + hk];
-        mb[kPairPrefetch - 1] = mrow[kt];
-        sb[kPairPrefetch - 1] = srow[kt];
+        mb[kPairPrefetch - 1] = mrow[kt >> a.gshift];
+        sb[kPairPrefetch - 1] = srow[kt >> a.gshift];
       }
       if (i >= kPairStages &&
           !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kPairStages) - 1) & 1, abortp, a.err))
@@ -1084,6 +1085,7 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
   a.qcols = qscale_cols;
   a.qscale = qscale;
   a.splits = p.splits;
+  a.gshift = w->group == 128 ? 1 : 0;
   a.part = nullptr;
   if (pair && p.splits > 1 && workspace && fg_aligned16(workspace) && ws_bytes >= pair_part_bytes(p))
     a.part = static_cast<float *>(workspace);
@@ -1113,10 +1115,10 @@ extern "C" fg_status fg_linear_w4a16(const fg_half *x, int M, int K, const fg_qt
                                      const fg_half *residual, int flags, int qscale_cols, float qscale, fg_half *y,
                                      void *workspace, size_t workspace_bytes, void *stream) {
   if (!w || M < 0 || K <= 0) return FG_ERR_INVALID;
-  if (w->bits != 4 || w->group != 64) return FG_ERR_UNSUPPORTED;
+  if (w->bits != 4 || (w->group != 64 && w->group != 128)) return FG_ERR_UNSUPPORTED;
   if (w->ndim != 2 || w->dim != 1 || w->shape[1] != K) return FG_ERR_SHAPE;
   const int64_t N = w->shape[0];
-  if (K % 64 || N <= 0 || N % 128 || N > (1 << 30)) return FG_ERR_SHAPE;
+  if (K % w->group || N <= 0 || N % 128 || N > (1 << 30)) return FG_ERR_SHAPE;
   if (flags & ~(FG_EPI_RELU | FG_EPI_RESIDUAL)) return FG_ERR_INVALID;
   if (M == 0) return FG_OK;
   if (!x || !y || !w->codes || !w->mins || !w->scales) return FG_ERR_INVALID;

@@ -477,8 +477,8 @@ __device__ __forceinline__ uint32_t bfi4(uint32_t v, uint32_t w, uint32_t pos) {
   return r;
 }
 
-// Cooperative quantisation of one group of 64 fp16 values held by 8 consecutive
-// lanes (lane j of the 8 holds elements 8j..8j+7 in v).  Steps and fp32 operation
+// Cooperative quantisation of one group of 8 * LANES fp16 values (64 or 128) held by
+// LANES consecutive lanes (lane j of them holds elements 8j..8j+7 in v).  Steps and fp32 operation
 // order as stated in fg.h: min/max over the group, mn += 0, d = mx - mn,
 // scale = fp16_rn(d/15), inv = 1/scale, code = clamp(rint((x - mn) * inv), 0, 15).
 // Min and max are taken on the fp16 values (exact, as on their fp32 widenings), carried
@@ -488,6 +488,7 @@ __device__ __forceinline__ uint32_t bfi4(uint32_t v, uint32_t w, uint32_t pos) {
 // Returns this lane's 8 codes packed into one 32-bit word (element 8j+2i in the low
 // nibble of byte i) and the group's fp16 min and scale.  All 32 lanes of the warp
 // must call it together.
+template <int LANES = 8>  // lanes sharing one group: 8 (group of 64) or 16 (group of 128)
 __device__ __forceinline__ uint32_t quant_group8(const uint4 v, __half &min_h, __half &scale_h) {
   const __half2 *h2 = reinterpret_cast<const __half2 *>(&v);
   const __half2 lo = __hmin2(__hmin2(h2[0], h2[1]), __hmin2(h2[2], h2[3]));
@@ -496,7 +497,7 @@ __device__ __forceinline__ uint32_t quant_group8(const uint4 v, __half &min_h, _
   __half2 mm = __halves2half2(__hmin(__low2half(lo), __high2half(lo)),
                               __hneg(__hmax(__low2half(hi), __high2half(hi))));
 #pragma unroll
-  for (int o = 1; o < 8; o <<= 1) {
+  for (int o = 1; o < LANES; o <<= 1) {
     const uint32_t u = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<const uint32_t *>(&mm), o);
     mm = __hmin2(mm, *reinterpret_cast<const __half2 *>(&u));
   }

@@ -33,34 +33,37 @@ unsigned grid_for(int64_t work_blocks, int per_sm) {
 __device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
 
 // ------------------------------------------------------------------------------------
-// K1: quantise along the last dim.  x: [ngroups][64] fp16 (as uint4 = 8 halves);
-// codes: [ngroups][32] bytes (as uint32 = 8 codes); mins/scales [ngroups].
-// A warp handles 4 groups per step and U steps per loop trip (loads issued first).
+// K1: quantise along the last dim.  x: [ngroups][G] fp16 (as uint4 = 8 halves);
+// codes: [ngroups][G/2] bytes (as uint32 = 8 codes); mins/scales [ngroups].  G/8 lanes
+// per group: a warp handles 32/(G/8) groups per step and U steps per loop trip (loads
+// issued first).
 // ------------------------------------------------------------------------------------
 constexpr int kQU = 4;
 
+template <int G>
 __global__ void __launch_bounds__(256) quantize_lastdim_kernel(const uint4 *__restrict__ x, int64_t ngroups,
                                                                uint32_t *__restrict__ codes,
                                                                __half *__restrict__ mins,
                                                                __half *__restrict__ scales) {
+  constexpr int L = G / 8, GPW = 32 / L;  // lanes per group, groups per warp step
   const int lane = threadIdx.x & 31;
-  const int slot = lane >> 3, j = lane & 7;
+  const int slot = lane / L, j = lane % L;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t g0 = warp * 4 * kQU; g0 < ngroups; g0 += nwarps * 4 * kQU) {
+  for (int64_t g0 = warp * GPW * kQU; g0 < ngroups; g0 += nwarps * GPW * kQU) {
     uint4 v[kQU];
 #pragma unroll
     for (int u = 0; u < kQU; u++) {
-      const int64_t g = g0 + u * 4 + slot;
-      v[u] = g < ngroups ? ld_stream(x + g * 8 + j) : make_uint4(0, 0, 0, 0);
+      const int64_t g = g0 + u * GPW + slot;
+      v[u] = g < ngroups ? ld_stream(x + g * L + j) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < kQU; u++) {
-      const int64_t g = g0 + u * 4 + slot;
+      const int64_t g = g0 + u * GPW + slot;
       __half mn, sc;
-      const uint32_t w = quant_group8(v[u], mn, sc);
+      const uint32_t w = quant_group8<L>(v[u], mn, sc);
       if (g < ngroups) {
-        codes[g * 8 + j] = w;
+        codes[g * L + j] = w;
         if (j == 0) {
           mins[g] = mn;
           scales[g] = sc;
@@ -70,7 +73,9 @@ __global__ void __launch_bounds__(256) quantize_lastdim_kernel(const uint4 *__re
   }
 }
 
-// K2: dequantise along the last dim; one thread per 8 codes (one 16-byte output).
+// K2: dequantise along the last dim; one thread per 8 codes (one 16-byte output).  G/8
+// such chunks share a group's min and scale.
+template <int G>
 __global__ void __launch_bounds__(256) dequantize_lastdim_kernel(const uint32_t *__restrict__ codes,
                                                                  const __half *__restrict__ mins,
                                                                  const __half *__restrict__ scales,
@@ -84,14 +89,14 @@ __global__ void __launch_bounds__(256) dequantize_lastdim_kernel(const uint32_t 
     for (int u = 0; u < 4; u++) {
       const int64_t c = i + u * stride;
       w[u] = __ldcs(codes + c);
-      mn[u] = mins[c >> 3];
-      sc[u] = scales[c >> 3];
+      mn[u] = mins[c / (G / 8)];
+      sc[u] = scales[c / (G / 8)];
     }
 #pragma unroll
     for (int u = 0; u < 4; u++) __stcs(y + i + u * stride, dequant8(w[u], __half2half2(sc[u]), __half2half2(mn[u])));
   }
   for (; i < nchunks; i += stride) {
-    __stcs(y + i, dequant8(__ldcs(codes + i), __half2half2(scales[i >> 3]), __half2half2(mins[i >> 3])));
+    __stcs(y + i, dequant8(__ldcs(codes + i), __half2half2(scales[i / (G / 8)]), __half2half2(mins[i / (G / 8)])));
   }
 }
 
@@ -99,25 +104,26 @@ __global__ void __launch_bounds__(256) dequantize_lastdim_kernel(const uint32_t 
 // Strided variants (grouping dim is not the last one): x viewed as [outer][n][inner],
 // one thread per group, consecutive threads on consecutive inner positions.
 // ------------------------------------------------------------------------------------
+template <int G>
 __global__ void __launch_bounds__(256) quantize_strided_kernel(const __half *__restrict__ x, int64_t outer,
                                                                int64_t n, int64_t inner,
                                                                uint8_t *__restrict__ codes,
                                                                __half *__restrict__ mins,
                                                                __half *__restrict__ scales) {
-  const int64_t ng = n / 64;
+  const int64_t ng = n / G;
   const int64_t total = outer * ng * inner;
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t i = t % inner, g = (t / inner) % ng, o = t / (inner * ng);
-    const __half *xp = x + (o * n + g * 64) * inner + i;
-    float v[64];
+    const __half *xp = x + (o * n + g * G) * inner + i;
+    float v[G];
     float mn, mx;
 #pragma unroll
-    for (int e = 0; e < 64; e++) v[e] = __half2float(xp[e * inner]);
+    for (int e = 0; e < G; e++) v[e] = __half2float(xp[e * inner]);
     mn = v[0];
     mx = v[0];
 #pragma unroll
-    for (int e = 1; e < 64; e++) {
+    for (int e = 1; e < G; e++) {
       mn = fminf(mn, v[e]);
       mx = fmaxf(mx, v[e]);
     }
@@ -125,11 +131,11 @@ __global__ void __launch_bounds__(256) quantize_strided_kernel(const __half *__r
     const float d = __fsub_rn(mx, mn);
     __half sh = __float2half_rn(__fdiv_rn(d, 15.0f));
     const float s = __half2float(sh);
-    uint8_t *cp = codes + (o * (n / 2) + g * 32) * inner + i;
+    uint8_t *cp = codes + (o * (n / 2) + g * (G / 2)) * inner + i;
     if (s != 0.0f) {
       const float inv = __fdiv_rn(1.0f, s);
 #pragma unroll
-      for (int e = 0; e < 64; e += 2) {
+      for (int e = 0; e < G; e += 2) {
         int c0 = min(max(__float2int_rn(__fmul_rn(__fsub_rn(v[e], mn), inv)), 0), 15);
         int c1 = min(max(__float2int_rn(__fmul_rn(__fsub_rn(v[e + 1], mn), inv)), 0), 15);
         cp[(e / 2) * inner] = static_cast<uint8_t>(c0 | (c1 << 4));
@@ -137,7 +143,7 @@ __global__ void __launch_bounds__(256) quantize_strided_kernel(const __half *__r
     } else {
       sh = __ushort_as_half(0);
 #pragma unroll
-      for (int e = 0; e < 64; e += 2) cp[(e / 2) * inner] = 0;
+      for (int e = 0; e < G; e += 2) cp[(e / 2) * inner] = 0;
     }
     const int64_t m = (o * ng + g) * inner + i;
     mins[m] = __float2half_rn(mn);
@@ -145,6 +151,7 @@ __global__ void __launch_bounds__(256) quantize_strided_kernel(const __half *__r
   }
 }
 
+template <int G>
 __global__ void __launch_bounds__(256) dequantize_strided_kernel(const uint8_t *__restrict__ codes,
                                                                  const __half *__restrict__ mins,
                                                                  const __half *__restrict__ scales,
@@ -155,7 +162,7 @@ __global__ void __launch_bounds__(256) dequantize_strided_kernel(const uint8_t *
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t i = t % inner, jb = (t / inner) % (n / 2), o = t / (inner * (n / 2));
     const uint32_t b = codes[t];
-    const int64_t m = (o * (n / 64) + (2 * jb) / 64) * inner + i;
+    const int64_t m = (o * (n / G) + (2 * jb) / G) * inner + i;
     const __half2 s2 = __half2half2(scales[m]), m2 = __half2half2(mins[m]);
     __half2 c = __hsub2(nib2_plus1024((b & 0xFu) | ((b & 0xF0u) << 12)),
                         __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
@@ -236,12 +243,12 @@ bool shape_numel(int ndim, const int64_t *shape, int64_t *numel) {
 extern "C" fg_status fg_qtensor_bytes(int ndim, const int64_t *shape, int dim, int bits, int group,
                                       size_t *codes_bytes, size_t *meta_bytes) {
   if (!shape || ndim < 1 || ndim > 4 || dim < 0 || dim >= ndim) return FG_ERR_INVALID;
-  if (bits != 4 || group != 64) return FG_ERR_UNSUPPORTED;
+  if (bits != 4 || (group != 64 && group != 128)) return FG_ERR_UNSUPPORTED;
   int64_t numel;
   if (!shape_numel(ndim, shape, &numel)) return FG_ERR_INVALID;
-  if (shape[dim] % 64) return FG_ERR_SHAPE;
+  if (shape[dim] % group) return FG_ERR_SHAPE;
   if (codes_bytes) *codes_bytes = static_cast<size_t>(numel / 2);
-  if (meta_bytes) *meta_bytes = static_cast<size_t>(numel / 64) * 2;
+  if (meta_bytes) *meta_bytes = static_cast<size_t>(numel / group) * 2;
   return FG_OK;
 }
 
@@ -268,17 +275,20 @@ extern "C" fg_status fg_quantize(const fg_half *x, int ndim, const int64_t *shap
     if (!fg_aligned16(x) || !fg_aligned16(out->codes) || (reinterpret_cast<uintptr_t>(out->mins) & 1) ||
         (reinterpret_cast<uintptr_t>(out->scales) & 1))
       return FG_ERR_INVALID;
-    const int64_t ngroups = numel / 64;
-    const int64_t warps_needed = (ngroups + 4 * kQU - 1) / (4 * kQU);
-    quantize_lastdim_kernel<<<grid_for((warps_needed + 7) / 8, 8), 256, 0, st>>>(
+    const int64_t ngroups = numel / group;
+    const int gpw = 32 / (group / 8);  // groups per warp step
+    const int64_t warps_needed = (ngroups + gpw * kQU - 1) / (gpw * kQU);
+    auto kern = group == 128 ? quantize_lastdim_kernel<128> : quantize_lastdim_kernel<64>;
+    kern<<<grid_for((warps_needed + 7) / 8, 8), 256, 0, st>>>(
         reinterpret_cast<const uint4 *>(x), ngroups, reinterpret_cast<uint32_t *>(out->codes),
         reinterpret_cast<__half *>(out->mins), reinterpret_cast<__half *>(out->scales));
   } else {
     if ((reinterpret_cast<uintptr_t>(x) & 1) || (reinterpret_cast<uintptr_t>(out->mins) & 1) ||
         (reinterpret_cast<uintptr_t>(out->scales) & 1))
       return FG_ERR_INVALID;
-    const int64_t groups = outer * (n / 64) * inner;
-    quantize_strided_kernel<<<grid_for((groups + 255) / 256, 8), 256, 0, st>>>(
+    const int64_t groups = outer * (n / group) * inner;
+    auto kern = group == 128 ? quantize_strided_kernel<128> : quantize_strided_kernel<64>;
+    kern<<<grid_for((groups + 255) / 256, 8), 256, 0, st>>>(
         reinterpret_cast<const __half *>(x), outer, n, inner, out->codes, reinterpret_cast<__half *>(out->mins),
         reinterpret_cast<__half *>(out->scales));
   }
@@ -301,12 +311,14 @@ extern "C" fg_status fg_dequantize(const fg_qtensor *q, fg_half *y, void *stream
   if (inner == 1) {
     if (!fg_aligned16(y) || (reinterpret_cast<uintptr_t>(q->codes) & 3)) return FG_ERR_INVALID;
     const int64_t nchunks = numel / 8;
-    dequantize_lastdim_kernel<<<grid_for((nchunks + 255) / 256, 8), 256, 0, st>>>(
+    auto kern = q->group == 128 ? dequantize_lastdim_kernel<128> : dequantize_lastdim_kernel<64>;
+    kern<<<grid_for((nchunks + 255) / 256, 8), 256, 0, st>>>(
         reinterpret_cast<const uint32_t *>(q->codes), reinterpret_cast<const __half *>(q->mins),
         reinterpret_cast<const __half *>(q->scales), nchunks, reinterpret_cast<uint4 *>(y));
   } else {
     const int64_t total = outer * (n / 2) * inner;
-    dequantize_strided_kernel<<<grid_for((total + 255) / 256, 8), 256, 0, st>>>(
+    auto kern = q->group == 128 ? dequantize_strided_kernel<128> : dequantize_strided_kernel<64>;
+    kern<<<grid_for((total + 255) / 256, 8), 256, 0, st>>>(
         q->codes, reinterpret_cast<const __half *>(q->mins), reinterpret_cast<const __half *>(q->scales), outer, n,
         inner, reinterpret_cast<__half *>(y));
   }

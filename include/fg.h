@@ -14,8 +14,9 @@
  *        (pre-LayerNorm decoder layer, multi-head attention, ReLU FFN).
  *
  * The 4-bit format (the pages give no formula; this is the reading the whole
- * library and its tests use).  For every group of 64 consecutive fp16 values
- * x_0..x_63 along the grouping dim, each step one IEEE fp32 operation:
+ * library and its tests use).  For every group of G consecutive fp16 values
+ * x_0..x_{G-1} along the grouping dim (G = 64, or 128 where a call says so --
+ * [G3] allows groups of 64 or 128), each step one IEEE fp32 operation:
  *   mn = min(x) + 0 (so -0 becomes +0);  d = max(x) - mn;
  *   scale = fp16_rn(d / 15);  if scale == 0: every code 0, stored scale +0;
  *   inv = 1 / scale;  code_i = clamp(round_half_even((x_i - mn) * inv), 0, 15);
@@ -60,7 +61,7 @@ typedef enum {
     FG_OK = 0,
     FG_ERR_INVALID = 1,     /* null/misaligned pointer, bad enum, negative size */
     FG_ERR_SHAPE = 2,       /* size not a multiple of the group, inconsistent dims */
-    FG_ERR_UNSUPPORTED = 3, /* bits != 4, group != 64, dims the kernels do not cover */
+    FG_ERR_UNSUPPORTED = 3, /* bits != 4, a group size not taken, dims the kernels do not cover */
     FG_ERR_RANGE = 4,       /* a cache position outside [0, max_len) (host or device check) */
     FG_ERR_CUDA = 5,        /* a CUDA runtime call failed (launch, copy, event) */
     FG_ERR_TIMEOUT = 6,     /* a bounded wait inside a kernel gave up */
@@ -94,7 +95,7 @@ typedef struct {
     int64_t shape[4];
     int32_t dim;         /* grouping dim, 0..ndim-1 */
     int32_t bits;        /* 4 */
-    int32_t group;       /* 64 */
+    int32_t group;       /* 64 or 128 */
 } fg_qtensor;
 
 /* Byte sizes of the codes array and of each of the mins/scales arrays. */
@@ -105,8 +106,8 @@ FG_API fg_status fg_qtensor_bytes(int ndim, const int64_t *shape, int dim, int b
  * out->mins, out->scales (device buffers set by the caller; their sizes from
  * fg_qtensor_bytes).  Fills out->ndim/shape/dim/bits/group.  x must be finite
  * (a group holding Inf or NaN gets unspecified codes).
- * Errors: FG_ERR_SHAPE if shape[dim] % 64 != 0; FG_ERR_UNSUPPORTED if
- * bits != 4 or group != 64.  [G3] */
+ * Errors: FG_ERR_SHAPE if shape[dim] % group != 0; FG_ERR_UNSUPPORTED if
+ * bits != 4 or group not 64 or 128.  [G3] */
 FG_API fg_status fg_quantize(const fg_half *x, int ndim, const int64_t *shape, int dim, int bits, int group,
                       fg_qtensor *out, void *stream);
 
@@ -172,7 +173,8 @@ enum {
  * fp16 output.  x: fp16 device [M][K]; w: packed along K, shape [N][K]
  * (PyTorch Linear orientation); bias: fp16 [N] or NULL; residual: fp16 [M][N]
  * (with FG_EPI_RESIDUAL); the first qscale_cols outputs of each row are
- * multiplied by qscale after the bias.  K % 64 == 0, N % 128 == 0; x, y, the
+ * multiplied by qscale after the bias.  w->group 64 or 128 with K % group == 0,
+ * N % 128 == 0; x, y, the
  * codes and the residual 16-byte aligned (FG_ERR_INVALID otherwise).
  * workspace: optional device scratch (16-byte aligned) of
  * fg_linear_workspace_bytes(M, N, K) bytes, 0 when the GEMM does not split its

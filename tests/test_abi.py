@@ -55,8 +55,11 @@ def test_qtensor_bytes_and_errors():
         fg.fg_qtensor_bytes((8, 96))
     with pytest.raises(fg.FgError, match="UNSUPPORTED"):
         fg.fg_qtensor_bytes((8, 64), bits=8)
+    assert fg.fg_qtensor_bytes((8, 256), group=128) == (8 * 256 // 2, 8 * 2 * 2)   # groups of 128
+    with pytest.raises(fg.FgError, match="SHAPE"):
+        fg.fg_qtensor_bytes((8, 192), group=128)
     with pytest.raises(fg.FgError, match="UNSUPPORTED"):
-        fg.fg_qtensor_bytes((8, 128), group=128)
+        fg.fg_qtensor_bytes((8, 256), group=32)
     with pytest.raises(fg.FgError, match="INVALID"):
         fg.fg_qtensor_bytes((1, 2, 3, 4, 64))
 

@@ -41,9 +41,9 @@ def u16(a):
 
 # ------------------------------------------------------------------ quantise ----------
 
-def _check_quant_equal(x16, dim=-1):
-    q = fg.fg_quantize(dev(x16), dim=dim)
-    r = oracle.quantize(x16, dim=dim)
+def _check_quant_equal(x16, dim=-1, group=64):
+    q = fg.fg_quantize(dev(x16), dim=dim, group=group)
+    r = oracle.quantize(x16, dim=dim, group=group)
     torch.cuda.synchronize()
     assert np.array_equal(host(q.codes), r.codes)
     assert np.array_equal(u16(host(q.mins)), u16(r.mins))
@@ -122,6 +122,55 @@ def test_quantize_2pow30_sampled_bit_exact():
     assert np.array_equal(u16(q.scales.view(-1)[torch.from_numpy(sel).cuda()].cpu().numpy()), u16(r.scales[:, 0]))
     y = fg.fg_dequantize(q).view(-1, 64)[torch.from_numpy(sel).cuda()].cpu().numpy()
     assert np.array_equal(u16(y), u16(oracle.dequantize(r)))
+
+
+# ------------------------------------------------------------------ groups of 128 -----
+
+@pytest.mark.parametrize("rows,cols", [(1, 128), (3, 256), (17, 4096), (5, 768 * 4), (1000, 384)])
+def test_quantize_group128_lastdim_bit_exact(rows, cols):
+    _check_quant_equal(si.sweep_tensor(9, rows * cols, row=cols) if rows * cols >= 256
+                       else si.normal_f16(9, 1, (rows, cols), 0.02), group=128)
+
+
+def test_quantize_group128_wide_ranges_bit_exact():
+    rng = np.random.default_rng(6)
+    x = (rng.standard_normal((1024, 128)) * 10.0 ** rng.integers(-7, 4, (1024, 1))).astype(np.float16)
+    x[0] = 0
+    x[1, :64] = -65504
+    x[1, 64:] = 65504
+    x[2] = (np.arange(128) / 2).astype(np.float16)
+    _check_quant_equal(x, group=128)
+
+
+@pytest.mark.parametrize("shape,dim", [((6, 256, 5), 1), ((128, 3), 0), ((2, 3, 384, 4), 2)])
+def test_quantize_group128_strided_bit_exact(shape, dim):
+    _check_quant_equal(si.normal_f16(10, 2, shape, 1.0), dim=dim, group=128)
+
+
+def test_quantize_group128_errors():
+    with pytest.raises(fg.FgError, match="SHAPE"):
+        fg.fg_quantize(torch.zeros((2, 192), dtype=torch.float16, device="cuda"), group=128)
+    with pytest.raises(fg.FgError, match="UNSUPPORTED"):
+        fg.fg_quantize(torch.zeros((2, 192), dtype=torch.float16, device="cuda"), group=96)
+
+
+@pytest.mark.parametrize("M,N,K", [(7, 256, 1024), (200, 384, 2048), (300, 512, 4096), (600, 640, 2048),
+                                   (512, 4096, 4096)])
+def test_linear_group128_weights(M, N, K):
+    # W4 weights in groups of 128 along K on both GEMM kernels (one SM per tile for M <= 256,
+    # CTA pairs above, with k splits for the long-k shapes)
+    x = si.normal_f16(19, 1, (M, K), 1.0)
+    w16 = si.normal_f16(19, 2, (N, K), 0.02)
+    b = si.normal_f16(19, 3, (N,), 0.1)
+    r = si.normal_f16(19, 4, (M, N), 1.0)
+    wq = fg.fg_quantize(dev(w16), dim=1, group=128)
+    wo = oracle.quantize(w16, 1, group=128)
+    assert np.array_equal(host(wq.codes), wo.codes)
+    y = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), residual=dev(r))
+    rows = np.unique(np.concatenate([np.arange(min(M, 8)), [M // 2, M - 1]]))
+    ref = oracle.linear(x[rows], wo, bias=b, residual=r[rows])
+    got = host(y)[rows].astype(np.float64)
+    assert np.max(np.abs(got - ref)) <= 2e-3 * np.max(np.abs(ref))
 
 
 # ------------------------------------------------------------------ KV append ---------
