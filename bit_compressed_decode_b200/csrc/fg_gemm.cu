@@ -6,9 +6,11 @@
 // in 4-bit form and are dequantised on the fly so the tensor cores compute in FP16.
 // Here the dequantisation target is shared memory, in the tensor cores' operand layout:
 //
+// One-SM kernel (M <= 256 tokens; the CTA-pair kernel for larger M is described further down):
 //   CTA tile: 256 output features (two 128-row MMA accumulators) x NT tokens x a k-range.
 //   warps 0..7   dequantise: thread t owns weight row n0+t; per 64-wide k-tile it loads
-//                32 code bytes + the group's fp16 min/scale (prefetched 3 tiles ahead),
+//                32 code bytes + the group's fp16 min/scale (a group covers one k-tile, or
+//                two with groups of 128; prefetched 3 tiles ahead),
 //                expands them with fp16 FMAs (exactly round(min + code*scale)) and stores
 //                128 bytes into the 128-byte-swizzled K-major A tile; then the epilogue.
 //   warp 8       TMA: the x tile [NT tokens x 64] (128-byte swizzle) per k-tile.
@@ -20,7 +22,10 @@
 //   cluster: each CTA copies its partial accumulator, 32 token columns at a time, into
 //   its own shared memory, and the owner of each 32-column chunk adds the partials of
 //   all CTAs of the cluster over distributed shared memory in cluster-rank order
-//   (deterministic) before the epilogue -- no partial sums go through global memory.
+//   (deterministic) before the epilogue -- this kernel's partial sums never go through
+//   global memory.
+// Both kernels may be launched with programmatic dependent launch: they read only weights
+// before griddep_wait(), and activations, residual, outputs and scratch after it.
 // Every mbarrier wait is bounded (FG_WAIT_TIMEOUT_NS) and reports FG_ERR_TIMEOUT.
 #include <stdio.h>
 

@@ -3,9 +3,9 @@
 // Format and fp32 operation order: "FlexGen Guide: High-Throughput LLM Offloading on
 // One GPU", section 3 (Group-Wise 4-Bit Quantization for Weights and KV Cache), read
 // as stated in fg.h.  All three kernels are HBM-bound streaming kernels: 16-byte
-// coalesced loads, a group of 64 values spread over 8 lanes whose min/max is found
-// with warp shuffles, 32-bit packed code stores, grids sized in whole waves of the
-// SM count.
+// coalesced loads, a group of 64 (or 128) values spread over 8 (or 16) lanes whose
+// min/max is found with warp shuffles, 32-bit packed code stores, grids sized in whole
+// waves of the SM count.  The KV cache always uses groups of 64 along head_dim.
 #include "fg_internal.cuh"
 
 namespace {
