@@ -34,6 +34,9 @@ sys.path.insert(0, ROOT)
 WORKLOADS = {
     "opt-6.7b-layer": dict(hidden=4096, heads=32, ffn=16384, nb=8, gbs=64, prompt=512, steps=32),
     "opt-125m-layer": dict(hidden=768, heads=12, ffn=3072, nb=1, gbs=4, prompt=32, steps=8),
+    # prompt processing of the OPT-6.7B-shaped block: one prefill of 512 tokens for each of the
+    # 512 sequences through one layer (the cache filled from position 0)
+    "opt-6.7b-prefill": dict(hidden=4096, heads=32, ffn=16384, nb=8, gbs=64, prompt=512, steps=32, phase="prefill"),
     # OPT-30B-shaped stack: 48 layers whose W4 blobs stay in pinned host memory and are
     # prefetched layer by layer on a side stream; KV4 caches resident in HBM
     "opt-30b-stack": dict(hidden=7168, heads=56, ffn=28672, nb=4, gbs=64, prompt=512, steps=32, layers=48),
@@ -399,6 +402,106 @@ def run_ours(args, wl):
         dist.destroy_process_group()
 
 
+def run_prefill(args, wl):
+    """One step = the prefill of the whole block's prompts through one layer (fg_layer_prefill:
+    the same kernels as decode with every prompt row a query, K/V of the prompt appended as 4-bit
+    codes), timed with CUDA events; then a second pass with per-kernel events."""
+    import torch
+
+    import bit_compressed_decode_b200 as fg
+    import seeded_inputs as si
+    from bit_compressed_decode_b200 import replicas
+
+    rank, world, local = replicas.env_ranks()
+    if world > 1:
+        torch.cuda.set_device(local)
+        replicas.init("nccl", timeout_s=300, device=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    h, H, F, P = wl["hidden"], wl["heads"], wl["ffn"], wl["prompt"]
+    nb, gbs = wl["nb"], wl["gbs"]
+    S, d = nb * gbs, h // H
+    maxL = (P + wl["steps"] + 63) // 64 * 64
+    cfg = fg.LayerConfig(h, H, F)
+    w16 = si.layer_weights_f16(0, h, F)
+    lw = fg.LayerWeights.from_fp16(cfg, w16, device=dev)
+    del w16
+    cache = fg.KVCache(S, H, d, maxL, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(3000 + rank)
+    x = torch.randn((S, P, h), generator=g, device=dev, dtype=torch.float16)
+    out = torch.empty_like(x)
+    zero = torch.zeros(S, dtype=torch.int32, device=dev)
+    # scratch for 64 Ki prompt rows; the library runs the block in chunks of whole sequences
+    ws = torch.empty(cfg.workspace_bytes(65536), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        fg.fg_layer_prefill(cfg, lw, cache, x, zero, num_gpu_batches=nb, gpu_batch_size=gbs, out=out, workspace=ws,
+                            stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    fg.fg_sync_status()
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+
+    def timed(profile):
+        fg.fg_profile_enable(profile)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        fg.fg_profile_enable(False)
+        return replicas.max_over_ranks(e0.elapsed_time(e1), device=dev)
+
+    ms = timed(False)
+    ms_profiled = timed(True)
+    clocks = sampler.stop()
+    prof = fg.fg_profile_collect()
+    fg.fg_sync_status()
+    peaks = load_peaks()
+    rows = S * P
+    work, _ = kernel_work(wl, rows, (P + 1) / 2)   # causal: row t of a prompt reads t + 1 cached tokens
+    kernels = {}
+    for name, (tot_ms, n) in prof.items():
+        if n == 0:
+            continue
+        bound, w = work[name]
+        per_step_s = tot_ms / 1e3 / args.steps
+        if bound == "tensor":
+            ach, unit, peak = w / per_step_s / 1e12, "TFLOP/s", peaks["tc_sustained"]
+        else:
+            ach, unit, peak = w / per_step_s / 1e9, "GB/s", peaks["hbm"]
+        kernels[name] = {"bound": bound, "ms_per_step": round(tot_ms / args.steps, 3), "launches": n,
+                         "share": round(tot_ms / sum(v[0] for v in prof.values()), 4), "achieved": round(ach, 1),
+                         "peak": peak, "unit": unit, "frac": round(ach / peak, 4)}
+    top = max(kernels, key=lambda n: kernels[n]["share"])
+    if rank == 0:
+        print(json.dumps({
+            "metric": "prefill prompt tokens/s per OPT layer block (W4 KV4)",
+            "value": world * rows * args.steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": args.workload, "block": f"{nb}x{gbs}", "prompt": P, "hidden": h, "heads": H,
+                       "ffn": F, "weights": "W4 g64", "kv": "KV4 g64 written from position 0",
+                       "l2": "inputs larger than L2 (prompt activations 2.1 GB per step)"},
+            "roofline": {"kernel": top, "bound": kernels[top]["bound"], "achieved": kernels[top]["achieved"],
+                         "peak": kernels[top]["peak"], "unit": kernels[top]["unit"], "frac": kernels[top]["frac"],
+                         "traffic": None},
+            "kernels": kernels, "kernels_pass_ms_per_step": ms_profiled / args.steps,
+            "gpu_launches": sum(v[1] for v in prof.values()), "clocks": clocks,
+        }), flush=True)
+
+
 def run_stack(args, wl):
     """One decode step = all layers of the stack for every sequence of the block, each layer's
     packed weights copied from pinned host memory (fg_stack_decode, double-buffered prefetch)."""
@@ -662,6 +765,8 @@ def main():
     wl = WORKLOADS[args.workload]
     if args.kernel:
         run_kernel(args, wl)
+    elif wl.get("phase") == "prefill" and args.impl == "ours":
+        run_prefill(args, wl)
     elif "layers" in wl and args.impl == "ours":
         run_stack(args, wl)
     elif args.impl == "reference":
