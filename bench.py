@@ -176,8 +176,9 @@ def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    threads = os.cpu_count() or 1
-    n_seqs = max(1, min(threads, 8))
+    # one sampled sequence per host thread (the oracle splits a step's rows by sequence)
+    n_seqs = max(1, min(os.cpu_count() or 1, 32, wl["nb"] * wl["gbs"]))
+    threads = n_seqs
     sample = OracleSample(wl, n_seqs, threads)
     times = []
     for i in range(args.warmup + args.steps):
@@ -371,12 +372,13 @@ def run_ours(args, wl):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # one sampled sequence per host thread (the oracle splits a step's rows by sequence)
         threads = os.cpu_count() or 1
-        n = max(1, min(threads, 8))
-        osample = OracleSample(wl, n, threads)
+        n = max(1, min(threads, 32, S))
+        osample = OracleSample(wl, n, n)
         t = min(osample.step() for _ in range(2))
-        cpu = {"value": n / t, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"{n} of {S} sequences, one decode step at position {P} ({threads} threads)"}
+        cpu = {"value": n / t, "unit": "tokens/s", "cores": n, "kind": "oracle",
+               "sample": f"{n} of {S} sequences, one decode step at position {P} ({n} threads, one per sequence)"}
 
     if rank == 0:
         line = {
