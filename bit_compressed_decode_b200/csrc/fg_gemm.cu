@@ -338,13 +338,14 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
 // ------------------------------------------------------------------------------------
 // Pair kernel: one tcgen05.mma.cta_group::2 spans two SMs.
 //
-//   CTA pair (cluster ranks 2p, 2p+1): 256 output features x 512 tokens x a k-range.  Each
-//   CTA dequantises its own 128 weight rows (the MMA's A = 256 rows is split by rows) and
-//   loads its halves of the two 256-token x tiles (B is split by columns: tokens
-//   tile*256 + half*128 ...).  The even CTA issues two M=256, N=256 MMAs per 16-wide k-step,
-//   one per token tile, into TMEM columns [0, 256) and [256, 512) of BOTH CTAs (each holds
-//   its 128 feature rows).  Per SM and k-tile: 128 dequantised rows (half of the single-SM
-//   kernel's rows per flop) and ~112 KB of shared-memory traffic for 8 MFLOP.
+//   CTA pair (cluster ranks 2p, 2p+1): 256 output features x NTT * 256 tokens (NTT = 2, or
+//   1 for smaller tiles) x a k-range.  Each CTA dequantises its own 128 weight rows (the
+//   MMA's A = 256 rows is split by rows) and loads its halves of the NTT 256-token x tiles
+//   (B is split by columns: tokens tile*256 + half*128 ...).  The even CTA issues NTT M=256,
+//   N=256 MMAs per 16-wide k-step, one per token tile, into TMEM columns [tile*256, +256) of
+//   BOTH CTAs (each holds its 128 feature rows).  Per SM and k-tile at NTT = 2: 128
+//   dequantised rows (half of the single-SM kernel's rows per flop) and ~112 KB of
+//   shared-memory traffic for 8 MFLOP.
 //   warps 0..7   dequantise (thread: row tid % 128, k half tid / 128), then the epilogue
 //                (warp: TMEM lane quarter warp % 4, token tile warp / 4);
 //   warp 8       TMA of this CTA's x halves, completing on the even CTA's barrier;
