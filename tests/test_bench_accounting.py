@@ -1,0 +1,47 @@
+"""The benchmark's algorithmic work per kernel (the numerators of every roofline fraction)
+against per-unit figures stated independently of it: OPT layer FLOPs (24 S h^2 for the four
+GEMMs with F = 4h), 4-bit bytes (0.5625 per weight: half a byte of code plus 4 bytes of fp16
+min and scale per 64), 144 bytes of K and V per cached token at head_dim 128."""
+import importlib.util
+import os
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    return m
+
+
+def test_opt6p7b_decode_step_work(bench):
+    wl = bench.WORKLOADS["opt-6.7b-layer"]
+    S, h, H = 512, 4096, 32
+    work, totals = bench.kernel_work(wl, S, 512)
+    gemm = sum(w for b, w in work.values() if b == "tensor")
+    assert gemm == 24 * S * h * h                        # 206 GFLOP per step
+    assert totals["kv_bytes_per_token"] == 2 * (64 + 4 * 2) == 144
+    assert totals["w4_bytes"] == 12 * h * h * 9 // 16   # 113.2 MB
+    att = work["attention"][1]
+    assert att == S * H * 512 * 144 + 2 * S * h * 2      # 1.208 GB of KV4 + q and o
+    assert work["kv_append"][1] == S * 2 * h * 2 + S * 2 * (h // 2 + h // 16)
+    units = bench.kernel_units(wl, S, 512)
+    assert units["attention"] == S * H * 512            # traffic of a smaller capture scales by these
+
+
+def test_stack_and_prefill_shapes(bench):
+    for name, layers in (("opt-30b-stack", 48), ("opt-175b-stack", 16)):
+        wl = bench.WORKLOADS[name]
+        assert wl["hidden"] % wl["heads"] == 0 and wl["ffn"] == 4 * wl["hidden"]
+        assert wl["layers"] == layers
+    wl = bench.WORKLOADS["opt-175b-stack"]
+    assert wl["nb"] * wl["gbs"] == 256 and wl["model_layers"] == 96
+    # prefill: row t of a prompt reads t + 1 cached tokens, so P rows read P (P + 1) / 2 in all
+    wl = bench.WORKLOADS["opt-6.7b-prefill"]
+    P = wl["prompt"]
+    work, _ = bench.kernel_work(wl, P, (P + 1) / 2)
+    assert work["attention"][1] == pytest.approx(wl["heads"] * P * (P + 1) / 2 * 144 + 2 * P * wl["hidden"] * 2)
