@@ -6,7 +6,11 @@
 // that must not allocate between steps for latency reasons.  For them this file keeps
 // the layer's scratch (the intermediate activations of one decode step) in a file-scope
 // device array of fixed size, which every GPU that loads the library holds until the
-// process exits.  The computation is exactly fg_layer_decode's.
+// process exits.  The computation is exactly fg_layer_decode's.  Under CUDA's lazy module
+// loading the array's memory is taken when this file's module is loaded, which the first
+// address lookup below triggers: callers make one call before they reserve device memory.
+#include <limits.h>
+
 #include <mutex>
 
 #include "fg_internal.cuh"
@@ -43,9 +47,11 @@ extern "C" fg_status fg_layer_decode_noalloc(const fg_layer_config *c, const fg_
                                              const int32_t *positions, int num_gpu_batches, int gpu_batch_size,
                                              void *stream) {
   if (num_gpu_batches < 0 || gpu_batch_size < 0) return FG_ERR_INVALID;
+  const int64_t rows = static_cast<int64_t>(num_gpu_batches) * gpu_batch_size;
+  if (rows > INT_MAX) return FG_ERR_SHAPE;
   // the activations must fit; the GEMMs use the rest for their optional split-k scratch
-  const size_t need = fg_layer_ws_required(c, num_gpu_batches * gpu_batch_size);
-  if (need == 0 && num_gpu_batches * gpu_batch_size > 0) return FG_ERR_UNSUPPORTED;
+  const size_t need = fg_layer_ws_required(c, static_cast<int>(rows));
+  if (need == 0 && rows > 0) return FG_ERR_UNSUPPORTED;
   if (need > FG_NOALLOC_SCRATCH_BYTES) return FG_ERR_WORKSPACE;
   void *scratch = nullptr;
   fg_status rc = scratch_address(&scratch);

@@ -2,6 +2,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "fg_internal.cuh"
 
 // One error word per device (every device that loads the library holds its own
@@ -18,16 +20,20 @@ fg_status fg_cuda_check(cudaError_t e) {
 
 fg_status fg_launch_check() { return fg_cuda_check(cudaGetLastError()); }
 
+// Per-device cache of the error word's address.  Threads that race on a first call each look
+// the address up (the same value) and store it; readers see either null or that value.
 unsigned int *fg_error_word_ptr() {
-  static unsigned int *cache[64] = {nullptr};
+  static std::atomic<unsigned int *> cache[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!cache[dev]) {
-    void *p = nullptr;
-    if (fg_cuda_check(cudaGetSymbolAddress(&p, fg_device_error_word)) != FG_OK) return nullptr;
-    cache[dev] = static_cast<unsigned int *>(p);
+  unsigned int *p = cache[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void *q = nullptr;
+    if (fg_cuda_check(cudaGetSymbolAddress(&q, fg_device_error_word)) != FG_OK) return nullptr;
+    p = static_cast<unsigned int *>(q);
+    cache[dev].store(p, std::memory_order_release);
   }
-  return cache[dev];
+  return p;
 }
 
 extern "C" const char *fg_last_cuda_error(void) { return g_last_cuda_error; }
