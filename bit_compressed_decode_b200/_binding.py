@@ -94,6 +94,7 @@ _decl("fg_stack_prefill", c_int, P, POINTER(fg_kv_cache), P, P, P, c_int, c_int,
 _decl("fg_stack_decode_host_kv", c_int, P, POINTER(fg_kv_cache), POINTER(fg_kv_cache), c_int, c_int, c_int, P, P, P,
       c_int, c_int, P, c_size_t, P, P)
 _decl("fg_stack_inject_copy_failure", c_int, P, c_int)
+_decl("fg_test_gemm_stall", c_int, c_int, ctypes.c_uint64)
 _decl("fg_stack_destroy", c_int, P)
 
 
@@ -444,6 +445,12 @@ def fg_profile_collect() -> dict:
     cnt = (c_int * n)()
     _check(_lib.fg_profile_collect(ms, cnt, n), "fg_profile_collect")
     return {PROFILE_SLOTS[i]: (float(ms[i]), int(cnt[i])) for i in range(n)}
+
+
+def fg_test_gemm_stall(count: int, wait_limit_ns: int) -> None:
+    """Test hook: the next `count` one-SM GEMM launches stall their first pipeline stage and give
+    up after wait_limit_ns (see fg_test_gemm_stall in fg.h)."""
+    _check(_lib.fg_test_gemm_stall(count, wait_limit_ns), "fg_test_gemm_stall")
 
 
 def fg_sync_status(stream=None) -> None:

@@ -29,6 +29,8 @@
 // Every mbarrier wait is bounded (FG_WAIT_TIMEOUT_NS) and reports FG_ERR_TIMEOUT.
 #include <stdio.h>
 
+#include <atomic>
+
 #include "fg_internal.cuh"
 
 namespace {
@@ -67,6 +69,8 @@ struct GemmArgs {
   int gshift;          // log2(group / 64): the weights' min/scale cover 1 (group 64) or 2 (128) k-tiles
   float *part;         // pair kernel, k split: fp32 partial sums through global memory, or null
   unsigned int *err;
+  uint64_t wait_ns;    // one-SM kernel: limit of every pipeline wait (FG_WAIT_TIMEOUT_NS unless a test shortens it)
+  int stall;           // one-SM kernel, test hook: the dequantising warps withhold their first-stage arrival
 };
 
 // ((acc + bias) * qscale if n < qcols) -> ReLU if set -> + residual (0 when unused).
@@ -161,7 +165,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
         mb[kPrefetch - 1] = mrow[kt >> a.gshift];
         sb[kPrefetch - 1] = srow[kt >> a.gshift];
       }
-      if (i >= C::STAGES && !mbar_wait_bounded(smem_u32(&empty[st]), ((i / C::STAGES) - 1) & 1, abortp, a.err))
+      if (i >= C::STAGES &&
+          !mbar_wait_bounded(smem_u32(&empty[st]), ((i / C::STAGES) - 1) & 1, abortp, a.err, a.wait_ns))
         break;
       const __half2 s2 = __half2half2(s0), m2 = __half2half2(m0);
       uint8_t *at = a_tile(st, acc);
@@ -173,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&full_a[st]));
+      if (lane == 0 && !(a.stall && i == 0)) mbar_arrive(smem_u32(&full_a[st]));
     }
   } else if (warp == kTmaWarp) {
     // ---------------- TMA producer for the x tiles ----------------
@@ -183,7 +188,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
       int issued = 0;
       for (int i = 0; i < nk; i++) {
         const int st = i % C::STAGES;
-        if (i >= C::STAGES && !mbar_wait_bounded(smem_u32(&empty[st]), ((i / C::STAGES) - 1) & 1, abortp, a.err))
+        if (i >= C::STAGES &&
+            !mbar_wait_bounded(smem_u32(&empty[st]), ((i / C::STAGES) - 1) & 1, abortp, a.err, a.wait_ns))
           break;
         const uint32_t bar = smem_u32(&full_b[st]);
         mbar_arrive_expect_tx(bar, C::B_BYTES);
@@ -192,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
       }
       if (*abortp) {  // let copies still in flight land before the CTA exits
         for (int j = issued > C::STAGES ? issued - C::STAGES : 0; j < issued; j++)
-          mbar_wait_bounded(smem_u32(&full_b[j % C::STAGES]), (j / C::STAGES) & 1, nullptr, nullptr);
+          mbar_wait_bounded(smem_u32(&full_b[j % C::STAGES]), (j / C::STAGES) & 1, nullptr, nullptr, a.wait_ns);
       }
     }
   } else {
@@ -201,8 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
       for (int i = 0; i < nk; i++) {
         const int st = i % C::STAGES;
         const uint32_t par = (i / C::STAGES) & 1;
-        if (!mbar_wait_bounded(smem_u32(&full_a[st]), par, abortp, a.err)) break;
-        if (!mbar_wait_bounded(smem_u32(&full_b[st]), par, abortp, a.err)) break;
+        if (!mbar_wait_bounded(smem_u32(&full_a[st]), par, abortp, a.err, a.wait_ns)) break;
+        if (!mbar_wait_bounded(smem_u32(&full_b[st]), par, abortp, a.err, a.wait_ns)) break;
         tc_fence_after();
         const uint32_t bbase = smem_u32(b_tile(st));
 #pragma unroll
@@ -226,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
   griddep_wait();  // residual and outputs: after the previous kernel has finished
   bool ready = false;
   if (warp < kDeqWarps) {
-    ready = mbar_wait_bounded(smem_u32(&accum_bar), 0, nullptr, a.err) && !*abortp;
+    ready = mbar_wait_bounded(smem_u32(&accum_bar), 0, nullptr, a.err, a.wait_ns) && !*abortp;
     tc_fence_after();
   }
   const int acc = (warp & 7) >> 2, q = warp & 3;
@@ -1046,6 +1052,11 @@ fg_status launch_pair(const CUtensorMap &map, const GemmArgs &a, const Plan &p, 
   return p.nt == 256 ? launch_pair_nt<1>(map, a, p, st, pdl) : launch_pair_nt<2>(map, a, p, st, pdl);
 }
 
+// Test hook state (fg_test_gemm_stall): launches of the one-SM kernel still to stall, and
+// their wait limit.
+std::atomic<int> g_stall_count{0};
+std::atomic<uint64_t> g_stall_wait_ns{FG_WAIT_TIMEOUT_NS};
+
 }  // namespace
 
 // Optional scratch of the pair kernel's k split: one fp32 partial [tile tokens][256 features]
@@ -1097,7 +1108,16 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
     a.part = static_cast<float *>(workspace);
   a.err = fg_error_word_ptr();
   if (!a.err) return FG_ERR_CUDA;
+  a.wait_ns = FG_WAIT_TIMEOUT_NS;
+  a.stall = 0;
   if (pair) return launch_pair(map, a, p, st, pdl);
+  int left = g_stall_count.load();
+  while (left > 0 && !g_stall_count.compare_exchange_weak(left, left - 1)) {
+  }
+  if (left > 0) {
+    a.stall = 1;
+    a.wait_ns = g_stall_wait_ns.load();
+  }
   switch (p.nt) {
     case 16: return launch_nt<16>(map, a, p, st, pdl);
     case 32: return launch_nt<32>(map, a, p, st, pdl);
@@ -1108,6 +1128,13 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
 }
 
 extern "C" size_t fg_linear_workspace_bytes(int M, int N, int K) { return fg_linear_ws_bytes(M, N, K); }
+
+extern "C" fg_status fg_test_gemm_stall(int count, uint64_t wait_limit_ns) {
+  if (count < 0 || wait_limit_ns == 0 || wait_limit_ns > FG_WAIT_TIMEOUT_NS) return FG_ERR_INVALID;
+  g_stall_wait_ns.store(wait_limit_ns);
+  g_stall_count.store(count);
+  return FG_OK;
+}
 
 extern "C" fg_status fg_linear_plan(int M, int N, int K, int *tile_tokens, int *splits) {
   if (!tile_tokens || !splits || M <= 0 || N <= 0 || K <= 0 || K % kBK || N % 128) return FG_ERR_INVALID;

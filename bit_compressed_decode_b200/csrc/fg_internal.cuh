@@ -80,16 +80,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for phase `parity` of an mbarrier.  Gives up (returns false) when the
-// shared abort flag is raised by another thread or after FG_WAIT_TIMEOUT_NS,
-// in which case it raises the abort flag and the device error word.
+// shared abort flag is raised by another thread or after limit_ns nanoseconds
+// (FG_WAIT_TIMEOUT_NS unless a test shortens it), in which case it raises the abort
+// flag and the device error word.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                                  unsigned int *err) {
+                                                  unsigned int *err, uint64_t limit_ns = FG_WAIT_TIMEOUT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort_flag && *abort_flag) return false;
-    if (globaltimer_ns() - t0 > FG_WAIT_TIMEOUT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       if (abort_flag) *abort_flag = 1;
       if (err) atomicOr(err, FG_DEVERR_TIMEOUT);
       return false;

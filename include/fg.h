@@ -275,14 +275,21 @@ FG_API fg_status fg_layer_prefill(const fg_layer_config *c, const fg_layer_weigh
  *   - Returns FG_ERR_WORKSPACE when the block's activations need more scratch
  *     than that, before any launch (fg_layer_workspace_bytes(c, S) above
  *     FG_NOALLOC_SCRATCH_BYTES only by the GEMMs' split-k scratch is fine: the
- *     GEMMs then add their partial sums on chip).
- *   - The first call on each device looks up the array's device address with
- *     that device current; make that first call before any stream capture.
+ *     GEMMs then add their partial sums on chip, with the same bits);
+ *     FG_ERR_SHAPE when num_gpu_batches * gpu_batch_size exceeds INT_MAX.
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address with that device current.  Under CUDA's lazy module loading (the
+ *     default) that lookup is also when the array's memory is taken, and each
+ *     kernel's code is loaded at its first launch.  A caller that reserves all
+ *     device memory up front therefore makes one ordinary call first (one step
+ *     on any block; a call with zero sequences sets up the array alone), before
+ *     reserving and before any stream capture.
  *   - Every call shares the one array and it keeps the last call's contents;
  *     nothing in it has to start at zero (each step writes what it reads).
  *     Calls whose work overlaps on the GPU (other streams, other threads)
  *     race on it: serialise them.
- *   - Allocates nothing (keep fg_profile_enable off: profiling creates events). */
+ *   - After that first call it allocates nothing (keep fg_profile_enable off:
+ *     profiling creates events). */
 #define FG_NOALLOC_SCRATCH_BYTES (48u << 20)
 FG_API fg_status fg_layer_decode_noalloc(const fg_layer_config *c, const fg_layer_weights *w,
                                          const fg_kv_cache *kv, const fg_half *x_in, fg_half *x_out,
@@ -352,6 +359,17 @@ FG_API fg_status fg_stack_decode_host_kv(fg_stack *st, const fg_kv_cache *host_k
                                   const int32_t *positions, int num_gpu_batches, int gpu_batch_size,
                                   void *workspace, size_t workspace_bytes, void *compute_stream,
                                   void *copy_stream);
+
+/* Test hook of the kernels' bounded waits (failure detection without a GPU
+ * fault).  The next `count` launches of the one-SM W4A16 GEMM (fg_linear_w4a16
+ * with M <= 256) run with every pipeline wait limited to wait_limit_ns
+ * nanoseconds (1 .. 2e9) instead of 2 s, and their dequantising warps withhold
+ * their arrival on the first pipeline stage, so the tensor-core issuer's wait
+ * for that stage cannot complete.  Such a launch gives up after the limit,
+ * stops issuing, waits for its copies in flight, frees its tensor memory and
+ * flags FG_ERR_TIMEOUT (reported by fg_sync_status); its output is
+ * unspecified.  Later launches run normally. */
+FG_API fg_status fg_test_gemm_stall(int count, uint64_t wait_limit_ns);
 
 /* Test hook: the next `count` blob copies of this stack report a copy
  * failure (no copy is issued), as if cudaMemcpyAsync had failed. */

@@ -150,6 +150,23 @@ def test_noalloc_rejects_oversized_block_on_host():
     assert rc == 7                                          # FG_ERR_WORKSPACE, before any CUDA call
 
 
+def test_noalloc_rejects_row_count_overflow_on_host():
+    cfg = fg.LayerConfig(4096, 32, 16384)
+    c = cfg.struct()
+    w = B.fg_layer_weights()
+    kv = B.fg_kv_cache()
+    rc = _rc("fg_layer_decode_noalloc", ctypes.byref(c), ctypes.byref(w), ctypes.byref(kv), None, None, None, 65536,
+             65536, None)
+    assert rc == 2                                          # FG_ERR_SHAPE: 2^32 rows, before any CUDA call
+
+
+def test_gemm_stall_hook_validates():
+    assert _rc("fg_test_gemm_stall", -1, 1000) == 1
+    assert _rc("fg_test_gemm_stall", 1, 0) == 1             # a zero limit
+    assert _rc("fg_test_gemm_stall", 1, 3_000_000_000) == 1  # above the normal 2 s limit
+    assert _rc("fg_test_gemm_stall", 0, 1000) == 0           # disarm
+
+
 def test_stack_create_validates():
     cfg = fg.LayerConfig(768, 12, 3072)
     c = cfg.struct()
