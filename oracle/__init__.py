@@ -67,10 +67,10 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_linear_g.argtypes = [P, I, I, P, P, P, I, P, P, I, I, D, P, I]
         _lib.oracle_layernorm.restype = I
         _lib.oracle_layernorm.argtypes = [P, I, I, P, P, D, P]
-        _lib.oracle_kv_append.restype = I
-        _lib.oracle_kv_append.argtypes = [P, P, I64, I, P, P, P, P, P, P, P, P, I, I, I, I]
-        _lib.oracle_attention.restype = I
-        _lib.oracle_attention.argtypes = [P, I64, I, P, P, P, P, P, P, P, P, I, I, I, I, P]
+        _lib.oracle_kv_append_g.restype = I
+        _lib.oracle_kv_append_g.argtypes = [P, P, I64, I, P, P, P, P, P, P, P, P, I, I, I, I, I]
+        _lib.oracle_attention_g.restype = I
+        _lib.oracle_attention_g.argtypes = [P, I64, I, P, P, P, P, P, P, P, P, I, I, I, I, P, I]
         _lib.oracle_layer_rows.restype = I
         _lib.oracle_layer_rows.argtypes = ([P, D] + [P] * 16 + [P] * 4 + [P] * 6 + [I, I] + [P, I, P, P, I, P, P, I])
     return _lib
@@ -184,11 +184,14 @@ def layernorm(x, gamma=None, beta=None, eps: float = 1e-5) -> np.ndarray:
 
 
 class KVCache:
-    """4-bit KV cache of one layer: codes [S,H,maxL,d/2], mins/scales [S,H,maxL,d/64]."""
+    """4-bit KV cache of one layer: codes [S,H,maxL,d/2], mins/scales [S,H,maxL,d/group], head_dim
+    quantised in groups of 64 or 128 ("FlexGen Guide", section 3)."""
 
-    def __init__(self, S: int, H: int, d: int, maxL: int):
-        self.S, self.H, self.d, self.maxL = S, H, d, maxL
-        ng = d // GROUP
+    def __init__(self, S: int, H: int, d: int, maxL: int, group: int = GROUP):
+        if group not in (64, 128) or d % group:
+            raise ValueError("group must be 64 or 128 and divide head_dim")
+        self.S, self.H, self.d, self.maxL, self.group = S, H, d, maxL, group
+        ng = d // group
         self.kc = np.zeros((S, H, maxL, d // 2), dtype=np.uint8)
         self.vc = np.zeros((S, H, maxL, d // 2), dtype=np.uint8)
         self.km = np.zeros((S, H, maxL, ng), dtype=np.uint16)
@@ -204,14 +207,14 @@ class KVCache:
 
 
 def kv_append(cache: KVCache, k, v, seq_of_row, pos_of_row, ld: int | None = None) -> None:
-    """Quantises fp16 k, v rows ``[R, H*d]`` into the cache (groups of 64 along head_dim)."""
+    """Quantises fp16 k, v rows ``[R, H*d]`` into the cache (groups of cache.group along head_dim)."""
     k = _u16(k); v = _u16(v)
     R = k.shape[0]
     ld = k.shape[1] if ld is None else ld
     sr = np.ascontiguousarray(seq_of_row, dtype=np.int32)
     pr = np.ascontiguousarray(pos_of_row, dtype=np.int32)
-    rc = lib().oracle_kv_append(_p(k), _p(v), ld, R, _p(sr), _p(pr), *cache.ptrs(),
-                                cache.S, cache.H, cache.d, cache.maxL)
+    rc = lib().oracle_kv_append_g(_p(k), _p(v), ld, R, _p(sr), _p(pr), *cache.ptrs(),
+                                  cache.S, cache.H, cache.d, cache.maxL, cache.group)
     assert rc == 0, rc
 
 
@@ -222,20 +225,21 @@ def attention(cache: KVCache, q, seq_of_row, len_of_row) -> np.ndarray:
     out = np.empty((R, cache.H * cache.d), dtype=np.float64)
     sr = np.ascontiguousarray(seq_of_row, dtype=np.int32)
     lr = np.ascontiguousarray(len_of_row, dtype=np.int32)
-    rc = lib().oracle_attention(_p(q), q.shape[1], R, _p(sr), _p(lr), *cache.ptrs(),
-                                cache.S, cache.H, cache.d, cache.maxL, _p(out))
+    rc = lib().oracle_attention_g(_p(q), q.shape[1], R, _p(sr), _p(lr), *cache.ptrs(),
+                                  cache.S, cache.H, cache.d, cache.maxL, _p(out), cache.group)
     assert rc == 0, rc
     return out
 
 
 class LayerWeights:
-    """One OPT layer's weights, quantised by the oracle along the input dim."""
+    """One OPT layer's weights, quantised by the oracle along the input dim in groups of 64 or 128."""
 
-    def __init__(self, w16: dict):
-        self.wqkv = quantize(w16["wqkv"], 1)
-        self.wo = quantize(w16["wo"], 1)
-        self.w1 = quantize(w16["w1"], 1)
-        self.w2 = quantize(w16["w2"], 1)
+    def __init__(self, w16: dict, group: int = GROUP):
+        self.group = group
+        self.wqkv = quantize(w16["wqkv"], 1, group)
+        self.wo = quantize(w16["wo"], 1, group)
+        self.w1 = quantize(w16["w1"], 1, group)
+        self.w2 = quantize(w16["w2"], 1, group)
         self.b = {k: _u16(w16[k]) for k in ("bqkv", "bo", "b1", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b")}
         self.hidden = self.wqkv.shape[1]
         self.ffn = self.w1.shape[0]
@@ -247,12 +251,15 @@ def layer_rows(weights: LayerWeights, heads: int, cache: KVCache, x, seq_of_row,
 
     Row r belongs to sequence ``seq_of_row[r]`` and is the token at cache
     position ``pos_of_row[r]``: its k, v are appended there, then it attends
-    over positions ``0..pos``.  Returns ``(out [R,h] float64, attn [R,h] or None)``.
+    over positions ``0..pos``.  The weights' group size is the cache's.
+    Returns ``(out [R,h] float64, attn [R,h] or None)``.
     """
     x = _u16(x)
     R, h = x.shape
     d = h // heads
-    dims = np.array([h, heads, d, weights.ffn], dtype=np.int32)
+    if cache.group != weights.group:
+        raise ValueError("the layer's weights and KV cache use one group size")
+    dims = np.array([h, heads, d, weights.ffn, weights.group], dtype=np.int32)
     out = np.zeros((R, h), dtype=np.float64)
     attn = np.zeros((R, h), dtype=np.float64) if want_attn else None
     sr = np.ascontiguousarray(seq_of_row, dtype=np.int32)

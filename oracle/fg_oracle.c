@@ -46,7 +46,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-#define OR_GROUP 64       /* the layer's group size */
+#define OR_GROUP 64       /* the default group size (the layer takes 64 or 128) */
 #define OR_GROUP_MAX 128  /* quantise/dequantise/linear also take groups of 128 [G3] */
 
 /* ------------------------------------------------------------------------- */
@@ -347,46 +347,56 @@ typedef struct {
     uint8_t *kc; uint16_t *km, *ks;
     uint8_t *vc; uint16_t *vm, *vs;
     int S, H, d, maxL;
+    int group;   /* 64 or 128 values of head_dim per group [G3] */
 } kv_t;
 
 static void kv_store(const kv_t *kv, int s, int head, int pos, const uint16_t *k16, const uint16_t *v16)
 {
     int64_t slot = ((int64_t)s * kv->H + head) * kv->maxL + pos;
-    int ng = kv->d / OR_GROUP;
+    int G = kv->group, ng = kv->d / G;
     for (int g = 0; g < ng; g++) {
-        quantize_group(k16 + g * OR_GROUP, 1, kv->kc + slot * (kv->d / 2) + g * 32, 1,
-                       &kv->km[slot * ng + g], &kv->ks[slot * ng + g], OR_GROUP);
-        quantize_group(v16 + g * OR_GROUP, 1, kv->vc + slot * (kv->d / 2) + g * 32, 1,
-                       &kv->vm[slot * ng + g], &kv->vs[slot * ng + g], OR_GROUP);
+        quantize_group(k16 + g * G, 1, kv->kc + slot * (kv->d / 2) + g * (G / 2), 1,
+                       &kv->km[slot * ng + g], &kv->ks[slot * ng + g], G);
+        quantize_group(v16 + g * G, 1, kv->vc + slot * (kv->d / 2) + g * (G / 2), 1,
+                       &kv->vm[slot * ng + g], &kv->vs[slot * ng + g], G);
     }
 }
 
-static void kv_load(const uint8_t *c, const uint16_t *mn, const uint16_t *sc, int64_t slot, int d, double *out)
+static void kv_load(const uint8_t *c, const uint16_t *mn, const uint16_t *sc, int64_t slot, int d, int G,
+                    double *out)
 {
-    int ng = d / OR_GROUP;
+    int ng = d / G;
     for (int i = 0; i < d; i++) {
         uint8_t byte = c[slot * (d / 2) + i / 2];
         int q = (i & 1) ? (byte >> 4) : (byte & 15);
-        int64_t m = slot * ng + i / OR_GROUP;
+        int64_t m = slot * ng + i / G;
         out[i] = oracle_f16_to_f64(dequant_one(q, mn[m], sc[m]));
     }
 }
 
 /* Append fp16 k, v rows [R][H*d] (row stride ld) at positions pos_of_row[r] of
-   sequence seq_of_row[r]. */
-int oracle_kv_append(const uint16_t *k, const uint16_t *v, int64_t ld, int R,
-                     const int *seq_of_row, const int *pos_of_row,
-                     uint8_t *kc, uint16_t *km, uint16_t *ks, uint8_t *vc, uint16_t *vm, uint16_t *vs,
-                     int S, int H, int d, int maxL)
+   sequence seq_of_row[r]; head_dim quantised in groups of `group` (64 or 128). */
+int oracle_kv_append_g(const uint16_t *k, const uint16_t *v, int64_t ld, int R,
+                       const int *seq_of_row, const int *pos_of_row,
+                       uint8_t *kc, uint16_t *km, uint16_t *ks, uint8_t *vc, uint16_t *vm, uint16_t *vs,
+                       int S, int H, int d, int maxL, int group)
 {
-    if (d % OR_GROUP) return -1;
-    kv_t kv = {kc, km, ks, vc, vm, vs, S, H, d, maxL};
+    if (!group_ok(group) || d % group) return -1;
+    kv_t kv = {kc, km, ks, vc, vm, vs, S, H, d, maxL, group};
     for (int r = 0; r < R; r++) {
         if (pos_of_row[r] < 0 || pos_of_row[r] >= maxL || seq_of_row[r] < 0 || seq_of_row[r] >= S) return -2;
         for (int hd = 0; hd < H; hd++)
             kv_store(&kv, seq_of_row[r], hd, pos_of_row[r], k + (int64_t)r * ld + hd * d, v + (int64_t)r * ld + hd * d);
     }
     return 0;
+}
+
+int oracle_kv_append(const uint16_t *k, const uint16_t *v, int64_t ld, int R,
+                     const int *seq_of_row, const int *pos_of_row,
+                     uint8_t *kc, uint16_t *km, uint16_t *ks, uint8_t *vc, uint16_t *vm, uint16_t *vs,
+                     int S, int H, int d, int maxL)
+{
+    return oracle_kv_append_g(k, v, ld, R, seq_of_row, pos_of_row, kc, km, ks, vc, vm, vs, S, H, d, maxL, OR_GROUP);
 }
 
 /* Softmax attention of one query head over cached positions 0..L-1:
@@ -397,7 +407,7 @@ static void attend_head(const kv_t *kv, int s, int head, int L, const double *q,
     int64_t base = ((int64_t)s * kv->H + head) * kv->maxL;
     double mx = -INFINITY;
     for (int j = 0; j < L; j++) {
-        kv_load(kv->kc, kv->km, kv->ks, base + j, d, kbuf);
+        kv_load(kv->kc, kv->km, kv->ks, base + j, d, kv->group, kbuf);
         double acc = 0.0;
         for (int i = 0; i < d; i++) acc += q[i] * kbuf[i];
         scores[j] = acc;
@@ -407,7 +417,7 @@ static void attend_head(const kv_t *kv, int s, int head, int L, const double *q,
     for (int j = 0; j < L; j++) { scores[j] = exp(scores[j] - mx); sum += scores[j]; }
     for (int i = 0; i < d; i++) o[i] = 0.0;
     for (int j = 0; j < L; j++) {
-        kv_load(kv->vc, kv->vm, kv->vs, base + j, d, kbuf);
+        kv_load(kv->vc, kv->vm, kv->vs, base + j, d, kv->group, kbuf);
         double p = scores[j] / sum;
         for (int i = 0; i < d; i++) o[i] += p * kbuf[i];
     }
@@ -415,12 +425,14 @@ static void attend_head(const kv_t *kv, int s, int head, int L, const double *q,
 
 /* q: fp16 rows [R][H*d] (row stride ld); each row attends over positions
    0..len_of_row[r]-1 of sequence seq_of_row[r].  out: float64 [R][H*d]. */
-int oracle_attention(const uint16_t *q16, int64_t ld, int R, const int *seq_of_row, const int *len_of_row,
-                     const uint8_t *kc, const uint16_t *km, const uint16_t *ks,
-                     const uint8_t *vc, const uint16_t *vm, const uint16_t *vs,
-                     int S, int H, int d, int maxL, double *out)
+int oracle_attention_g(const uint16_t *q16, int64_t ld, int R, const int *seq_of_row, const int *len_of_row,
+                       const uint8_t *kc, const uint16_t *km, const uint16_t *ks,
+                       const uint8_t *vc, const uint16_t *vm, const uint16_t *vs,
+                       int S, int H, int d, int maxL, double *out, int group)
 {
-    kv_t kv = {(uint8_t *)kc, (uint16_t *)km, (uint16_t *)ks, (uint8_t *)vc, (uint16_t *)vm, (uint16_t *)vs, S, H, d, maxL};
+    if (!group_ok(group) || d % group) return -1;
+    kv_t kv = {(uint8_t *)kc, (uint16_t *)km, (uint16_t *)ks, (uint8_t *)vc, (uint16_t *)vm, (uint16_t *)vs, S, H, d, maxL,
+               group};
     double *q = malloc(sizeof(double) * d), *kb = malloc(sizeof(double) * d);
     double *sc = malloc(sizeof(double) * (maxL > 0 ? maxL : 1));
     for (int r = 0; r < R; r++) {
@@ -432,6 +444,14 @@ int oracle_attention(const uint16_t *q16, int64_t ld, int R, const int *seq_of_r
     }
     free(q); free(kb); free(sc);
     return 0;
+}
+
+int oracle_attention(const uint16_t *q16, int64_t ld, int R, const int *seq_of_row, const int *len_of_row,
+                     const uint8_t *kc, const uint16_t *km, const uint16_t *ks,
+                     const uint8_t *vc, const uint16_t *vm, const uint16_t *vs,
+                     int S, int H, int d, int maxL, double *out)
+{
+    return oracle_attention_g(q16, ld, R, seq_of_row, len_of_row, kc, km, ks, vc, vm, vs, S, H, d, maxL, out, OR_GROUP);
 }
 
 /* ------------------------------------------------------------------------- */
@@ -510,11 +530,12 @@ static void *layer_worker(void *arg)
 }
 
 /*
- * dims = {hidden, heads, head_dim, ffn}.  Weights as packed 4-bit tensors
- * quantised along the input dim: wqkv [3h][h], wo [h][h], w1 [F][h], w2 [h][F]
- * (codes, mins, scales each); biases and LayerNorm parameters fp16 (NULL = 0,
- * gamma NULL = 1).  The KV cache arrays are read and written in place.
- * kv_only = 1 stops after step 3 (cache fill for prompts).
+ * dims = {hidden, heads, head_dim, ffn, group}.  Weights as packed 4-bit tensors
+ * quantised along the input dim in groups of `group` (64 or 128; the KV cache
+ * uses the same group along head_dim): wqkv [3h][h], wo [h][h], w1 [F][h],
+ * w2 [h][F] (codes, mins, scales each); biases and LayerNorm parameters fp16
+ * (NULL = 0, gamma NULL = 1).  The KV cache arrays are read and written in
+ * place.  kv_only = 1 stops after step 3 (cache fill for prompts).
  */
 int oracle_layer_rows(const int *dims, double eps,
                       const uint8_t *qkv_c, const uint16_t *qkv_m, const uint16_t *qkv_s, const uint16_t *bqkv,
@@ -530,18 +551,19 @@ int oracle_layer_rows(const int *dims, double eps,
     layer_ctx c;
     memset(&c, 0, sizeof(c));
     c.h = dims[0]; c.H = dims[1]; c.d = dims[2]; c.F = dims[3]; c.eps = eps;
-    if (c.h != c.H * c.d || c.h % OR_GROUP || c.F % OR_GROUP || c.d % OR_GROUP) return -1;
+    int G = dims[4];
+    if (!group_ok(G) || c.h != c.H * c.d || c.h % G || c.F % G || c.d % G) return -1;
     for (int r = 0; r < R; r++)
         if (seq_of_row[r] < 0 || seq_of_row[r] >= S || pos_of_row[r] < 0 || pos_of_row[r] >= maxL) return -2;
-    c.Wqkv = dequant_weight(qkv_c, qkv_m, qkv_s, 3 * c.h, c.h, OR_GROUP);
-    c.Wo = kv_only ? NULL : dequant_weight(o_c, o_m, o_s, c.h, c.h, OR_GROUP);
-    c.W1 = kv_only ? NULL : dequant_weight(f1_c, f1_m, f1_s, c.F, c.h, OR_GROUP);
-    c.W2 = kv_only ? NULL : dequant_weight(f2_c, f2_m, f2_s, c.h, c.F, OR_GROUP);
+    c.Wqkv = dequant_weight(qkv_c, qkv_m, qkv_s, 3 * c.h, c.h, G);
+    c.Wo = kv_only ? NULL : dequant_weight(o_c, o_m, o_s, c.h, c.h, G);
+    c.W1 = kv_only ? NULL : dequant_weight(f1_c, f1_m, f1_s, c.F, c.h, G);
+    c.W2 = kv_only ? NULL : dequant_weight(f2_c, f2_m, f2_s, c.h, c.F, G);
     c.bqkv = f16_vec(bqkv, 3 * c.h, 0.0); c.bo = f16_vec(bo, c.h, 0.0);
     c.b1 = f16_vec(b1, c.F, 0.0); c.b2 = f16_vec(b2, c.h, 0.0);
     c.g1 = f16_vec(ln1_g, c.h, 1.0); c.be1 = f16_vec(ln1_b, c.h, 0.0);
     c.g2 = f16_vec(ln2_g, c.h, 1.0); c.be2 = f16_vec(ln2_b, c.h, 0.0);
-    kv_t kv = {kc, km, ks, vc, vm, vs, S, c.H, c.d, maxL};
+    kv_t kv = {kc, km, ks, vc, vm, vs, S, c.H, c.d, maxL, G};
     c.kv = kv;
     c.x = x; c.seq_of_row = seq_of_row; c.pos_of_row = pos_of_row; c.R = R;
     c.kv_only = kv_only; c.out = out; c.attn = attn;

@@ -170,6 +170,26 @@ def test_attention_peaked_selects_token():
     assert np.allclose(o, _deq_v(cache, 0, 0, 2), rtol=0, atol=1e-100 + 1e-12)
 
 
+@pytest.mark.parametrize("d", [128, 256])
+def test_kv_append_group128_layout_matches_quantize(d):
+    # groups of 128 along head_dim ("FlexGen Guide", section 3: groups of 64 or 128): the cache
+    # slot of (sequence, head, position) holds quantize(row, groups of 128) of that head's values
+    S, H, maxL = 2, 2, 64
+    c = oracle.KVCache(S, H, d, maxL, group=128)
+    assert c.km.shape == (S, H, maxL, d // 128)
+    k = si.normal_f16(20, 1, (3, H * d), 1.0)
+    v = si.normal_f16(20, 2, (3, H * d), 1.0)
+    oracle.kv_append(c, k, v, [1, 0, 1], [3, 9, 63])
+    qk = oracle.quantize(k.reshape(3, H, d), dim=-1, group=128)
+    qv = oracle.quantize(v.reshape(3, H, d), dim=-1, group=128)
+    for r, (s, p) in enumerate([(1, 3), (0, 9), (1, 63)]):
+        assert np.array_equal(c.kc[s, :, p], qk.codes[r]) and np.array_equal(c.vc[s, :, p], qv.codes[r])
+        assert np.array_equal(c.ks[s, :, p], qk.scales.view(np.uint16)[r])
+        assert np.array_equal(c.vm[s, :, p], qv.mins.view(np.uint16)[r])
+    with pytest.raises(ValueError):
+        oracle.KVCache(S, H, 64, maxL, group=128)            # a group must fit in head_dim
+
+
 def test_kv_append_layout_matches_quantize():
     S, H, d, maxL = 3, 2, 128, 64
     c = oracle.KVCache(S, H, d, maxL)
@@ -191,7 +211,7 @@ HID = H_ * D_
 FFN = 4 * HID
 
 
-def _wiring_weights(qk_zero: bool):
+def _wiring_weights(qk_zero: bool, HID=HID, FFN=FFN):
     """Permutation-structured layer whose output has a closed form."""
     rng = np.random.default_rng(11)
     pv, po, p1 = rng.permutation(HID), rng.permutation(HID), rng.integers(0, HID, FFN)
@@ -235,8 +255,9 @@ def _closed_form(w16, perms, x_rows, o_rows):
 def _v_rows(w16, perms, x_rows):
     """v = fp16(15*fp16(LN1(x))[pv] + bv) (what is appended to the cache)."""
     pv = perms[0]
+    hid = x_rows.shape[1]
     a = r16(oracle.layernorm(x_rows, w16["ln1_g"], w16["ln1_b"]))
-    return f16(15.0 * a[:, pv] + w16["bqkv"].astype(np.float64)[2 * HID:])
+    return f16(15.0 * a[:, pv] + w16["bqkv"].astype(np.float64)[2 * hid:])
 
 
 def test_layer_single_token_closed_form():
@@ -251,6 +272,34 @@ def test_layer_single_token_closed_form():
     o = oracle.dequantize(oracle.quantize(v.reshape(S, H_, D_), -1)).astype(np.float64).reshape(S, HID)
     assert np.array_equal(attn, r16(o))
     assert np.allclose(y, _closed_form(w16, perms, x, r16(o)), rtol=0, atol=1e-9)
+
+
+def test_layer_group128_single_token_and_uniform_prompt_closed_forms():
+    # The layer with weights and KV cache in groups of 128 (2 heads x 128): the permutation
+    # weights are still stored exactly ({0, 15} per group), one cached token returns its
+    # dequantised group-128 v, and q = k = 0 averages the group-128 v of the prefix.
+    H, D = 2, 128
+    hid, ffn = H * D, 4 * H * D
+    w16, perms = _wiring_weights(qk_zero=True, HID=hid, FFN=ffn)
+    W = oracle.LayerWeights(w16, group=128)
+    S, P = 2, 4
+    x = si.normal_f16(21, 1, (S, P, hid), 1.0)
+    cache = oracle.KVCache(S, H, D, 64, group=128)
+    rows = x.transpose(1, 0, 2).reshape(P * S, hid)
+    seq, pos = np.tile(np.arange(S), P), np.repeat(np.arange(P), S)
+    y, attn = oracle.layer_rows(W, H, cache, rows, seq, pos, want_attn=True)
+    v = _v_rows(w16, perms, rows)
+    vd = oracle.dequantize(oracle.quantize(v.reshape(-1, H, D), -1, group=128)).astype(np.float64).reshape(-1, hid)
+    for r in range(P * S):
+        mine = (seq == seq[r]) & (pos <= pos[r])
+        o = vd[mine].mean(axis=0)
+        # the attention output is o rounded to fp16 (its sum order differs from numpy's mean, so
+        # allow half an fp16 ulp; a wrong group would be off by up to half a quantisation step)
+        assert np.all(np.abs(attn[r] - o) <= 2.0 ** -11 * np.abs(o) + 1e-12)
+        assert np.allclose(y[r], _closed_form(w16, perms, rows[r:r + 1], attn[r][None])[0], rtol=0, atol=1e-9)
+    assert np.array_equal(attn[:S], r16(vd[:S]))          # position 0: the one cached token
+    with pytest.raises(ValueError):
+        oracle.layer_rows(W, H, oracle.KVCache(S, H, D, 64), rows, seq, pos)   # groups must agree
 
 
 def test_layer_uniform_attention_over_prompt():
