@@ -69,8 +69,8 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_layernorm.argtypes = [P, I, I, P, P, D, P]
         _lib.oracle_kv_append_g.restype = I
         _lib.oracle_kv_append_g.argtypes = [P, P, I64, I, P, P, P, P, P, P, P, P, I, I, I, I, I]
-        _lib.oracle_attention_g.restype = I
-        _lib.oracle_attention_g.argtypes = [P, I64, I, P, P, P, P, P, P, P, P, I, I, I, I, P, I]
+        _lib.oracle_attention_x.restype = I
+        _lib.oracle_attention_x.argtypes = [P, I64, I, P, P, P, P, P, P, P, P, I, I, I, I, P, I, I]
         _lib.oracle_layer_rows.restype = I
         _lib.oracle_layer_rows.argtypes = ([P, D] + [P] * 16 + [P] * 4 + [P] * 6 + [I, I] + [P, I, P, P, I, P, P, I])
     return _lib
@@ -218,15 +218,18 @@ def kv_append(cache: KVCache, k, v, seq_of_row, pos_of_row, ld: int | None = Non
     assert rc == 0, rc
 
 
-def attention(cache: KVCache, q, seq_of_row, len_of_row) -> np.ndarray:
-    """Softmax attention of fp16 query rows ``[R, H*d]`` (already scaled) over the cache."""
+def attention(cache: KVCache, q, seq_of_row, len_of_row, exact_dequant: bool = False) -> np.ndarray:
+    """Softmax attention of fp16 query rows ``[R, H*d]`` (already scaled) over the cache.
+
+    K and V are the dequantised fp16 values (``exact_dequant=False``, the layer's reading), or
+    ``min + code * scale`` before that rounding (``exact_dequant=True``)."""
     q = _u16(q)
     R = q.shape[0]
     out = np.empty((R, cache.H * cache.d), dtype=np.float64)
     sr = np.ascontiguousarray(seq_of_row, dtype=np.int32)
     lr = np.ascontiguousarray(len_of_row, dtype=np.int32)
-    rc = lib().oracle_attention_g(_p(q), q.shape[1], R, _p(sr), _p(lr), *cache.ptrs(),
-                                  cache.S, cache.H, cache.d, cache.maxL, _p(out), cache.group)
+    rc = lib().oracle_attention_x(_p(q), q.shape[1], R, _p(sr), _p(lr), *cache.ptrs(),
+                                  cache.S, cache.H, cache.d, cache.maxL, _p(out), cache.group, int(exact_dequant))
     assert rc == 0, rc
     return out
 

@@ -348,6 +348,7 @@ typedef struct {
     uint8_t *vc; uint16_t *vm, *vs;
     int S, H, d, maxL;
     int group;   /* 64 or 128 values of head_dim per group [G3] */
+    int exact;   /* attention reads min + code * scale unrounded (1) or rounded to fp16 (0) */
 } kv_t;
 
 static void kv_store(const kv_t *kv, int s, int head, int pos, const uint16_t *k16, const uint16_t *v16)
@@ -363,14 +364,17 @@ static void kv_store(const kv_t *kv, int s, int head, int pos, const uint16_t *k
 }
 
 static void kv_load(const uint8_t *c, const uint16_t *mn, const uint16_t *sc, int64_t slot, int d, int G,
-                    double *out)
+                    int exact, double *out)
 {
     int ng = d / G;
     for (int i = 0; i < d; i++) {
         uint8_t byte = c[slot * (d / 2) + i / 2];
         int q = (i & 1) ? (byte >> 4) : (byte & 15);
         int64_t m = slot * ng + i / G;
-        out[i] = oracle_f16_to_f64(dequant_one(q, mn[m], sc[m]));
+        if (exact)  /* min + q * scale is exact in float64 (see dequant_one) */
+            out[i] = oracle_f16_to_f64(mn[m]) + (double)q * oracle_f16_to_f64(sc[m]);
+        else
+            out[i] = oracle_f16_to_f64(dequant_one(q, mn[m], sc[m]));
     }
 }
 
@@ -382,7 +386,7 @@ int oracle_kv_append_g(const uint16_t *k, const uint16_t *v, int64_t ld, int R,
                        int S, int H, int d, int maxL, int group)
 {
     if (!group_ok(group) || d % group) return -1;
-    kv_t kv = {kc, km, ks, vc, vm, vs, S, H, d, maxL, group};
+    kv_t kv = {kc, km, ks, vc, vm, vs, S, H, d, maxL, group, 0};
     for (int r = 0; r < R; r++) {
         if (pos_of_row[r] < 0 || pos_of_row[r] >= maxL || seq_of_row[r] < 0 || seq_of_row[r] >= S) return -2;
         for (int hd = 0; hd < H; hd++)
@@ -407,7 +411,7 @@ static void attend_head(const kv_t *kv, int s, int head, int L, const double *q,
     int64_t base = ((int64_t)s * kv->H + head) * kv->maxL;
     double mx = -INFINITY;
     for (int j = 0; j < L; j++) {
-        kv_load(kv->kc, kv->km, kv->ks, base + j, d, kv->group, kbuf);
+        kv_load(kv->kc, kv->km, kv->ks, base + j, d, kv->group, kv->exact, kbuf);
         double acc = 0.0;
         for (int i = 0; i < d; i++) acc += q[i] * kbuf[i];
         scores[j] = acc;
@@ -417,22 +421,25 @@ static void attend_head(const kv_t *kv, int s, int head, int L, const double *q,
     for (int j = 0; j < L; j++) { scores[j] = exp(scores[j] - mx); sum += scores[j]; }
     for (int i = 0; i < d; i++) o[i] = 0.0;
     for (int j = 0; j < L; j++) {
-        kv_load(kv->vc, kv->vm, kv->vs, base + j, d, kv->group, kbuf);
+        kv_load(kv->vc, kv->vm, kv->vs, base + j, d, kv->group, kv->exact, kbuf);
         double p = scores[j] / sum;
         for (int i = 0; i < d; i++) o[i] += p * kbuf[i];
     }
 }
 
 /* q: fp16 rows [R][H*d] (row stride ld); each row attends over positions
-   0..len_of_row[r]-1 of sequence seq_of_row[r].  out: float64 [R][H*d]. */
-int oracle_attention_g(const uint16_t *q16, int64_t ld, int R, const int *seq_of_row, const int *len_of_row,
+   0..len_of_row[r]-1 of sequence seq_of_row[r].  out: float64 [R][H*d].
+   exact = 0: K and V are the dequantised fp16 values (the layer's reading);
+   exact = 1: K and V are min + code * scale before that rounding (the decode
+   kernel's reading: it never forms the fp16 value). */
+int oracle_attention_x(const uint16_t *q16, int64_t ld, int R, const int *seq_of_row, const int *len_of_row,
                        const uint8_t *kc, const uint16_t *km, const uint16_t *ks,
                        const uint8_t *vc, const uint16_t *vm, const uint16_t *vs,
-                       int S, int H, int d, int maxL, double *out, int group)
+                       int S, int H, int d, int maxL, double *out, int group, int exact)
 {
     if (!group_ok(group) || d % group) return -1;
     kv_t kv = {(uint8_t *)kc, (uint16_t *)km, (uint16_t *)ks, (uint8_t *)vc, (uint16_t *)vm, (uint16_t *)vs, S, H, d, maxL,
-               group};
+               group, exact ? 1 : 0};
     double *q = malloc(sizeof(double) * d), *kb = malloc(sizeof(double) * d);
     double *sc = malloc(sizeof(double) * (maxL > 0 ? maxL : 1));
     for (int r = 0; r < R; r++) {
@@ -444,6 +451,14 @@ int oracle_attention_g(const uint16_t *q16, int64_t ld, int R, const int *seq_of
     }
     free(q); free(kb); free(sc);
     return 0;
+}
+
+int oracle_attention_g(const uint16_t *q16, int64_t ld, int R, const int *seq_of_row, const int *len_of_row,
+                       const uint8_t *kc, const uint16_t *km, const uint16_t *ks,
+                       const uint8_t *vc, const uint16_t *vm, const uint16_t *vs,
+                       int S, int H, int d, int maxL, double *out, int group)
+{
+    return oracle_attention_x(q16, ld, R, seq_of_row, len_of_row, kc, km, ks, vc, vm, vs, S, H, d, maxL, out, group, 0);
 }
 
 int oracle_attention(const uint16_t *q16, int64_t ld, int R, const int *seq_of_row, const int *len_of_row,
@@ -563,7 +578,7 @@ int oracle_layer_rows(const int *dims, double eps,
     c.b1 = f16_vec(b1, c.F, 0.0); c.b2 = f16_vec(b2, c.h, 0.0);
     c.g1 = f16_vec(ln1_g, c.h, 1.0); c.be1 = f16_vec(ln1_b, c.h, 0.0);
     c.g2 = f16_vec(ln2_g, c.h, 1.0); c.be2 = f16_vec(ln2_b, c.h, 0.0);
-    kv_t kv = {kc, km, ks, vc, vm, vs, S, c.H, c.d, maxL, G};
+    kv_t kv = {kc, km, ks, vc, vm, vs, S, c.H, c.d, maxL, G, 0};
     c.kv = kv;
     c.x = x; c.seq_of_row = seq_of_row; c.pos_of_row = pos_of_row; c.R = R;
     c.kv_only = kv_only; c.out = out; c.attn = attn;

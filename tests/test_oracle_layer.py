@@ -132,6 +132,44 @@ def test_attention_zero_query_is_mean_of_v():
             assert np.allclose(o[s, h * d:(h + 1) * d], mean, rtol=0, atol=1e-13)
 
 
+def test_attention_exact_dequant_single_token_rounds_to_the_fp16_form():
+    # one cached token: the exact form returns min + code * scale, the fp16 form that value
+    # rounded to fp16 -- so rounding the exact output gives the fp16 output bit for bit
+    S, H, d = 2, 3, 128
+    c = _random_cache(S, H, d, 64, 1)
+    q = si.normal_f16(7, 1, (S, H * d), 1.0)
+    o16 = oracle.attention(c, q, np.arange(S), np.ones(S, dtype=np.int32))
+    ox = oracle.attention(c, q, np.arange(S), np.ones(S, dtype=np.int32), exact_dequant=True)
+    assert np.array_equal(oracle.f64_to_f16(ox).astype(np.float64), o16)
+    assert np.all(np.abs(ox - o16) <= 2.0 ** -11 * np.abs(o16))
+    assert not np.array_equal(ox, o16)                       # the two forms do differ
+
+
+@pytest.mark.parametrize("group", [64, 128])
+def test_attention_exact_dequant_equals_fp16_form_on_representable_groups(group):
+    # groups built as min + code * 2^e (codes 0 and 15 present, min a multiple of 2^e): the
+    # quantiser stores scale 2^e and the codes exactly, and every min + code * scale is an fp16
+    # value, so both forms read the same K and V and agree bit for bit for any query
+    S, H, d, L = 2, 2, 128, 37
+    rng = np.random.default_rng(8)
+    c = oracle.KVCache(S, H, d, 64, group=group)
+    for s in range(S):
+        rows = []
+        for _ in range(2 * L):
+            e = rng.integers(-8, 0, size=d // group)
+            codes = rng.integers(0, 16, size=(d // group, group))
+            codes[:, 0], codes[:, 1] = 0, 15
+            mins = rng.integers(-64, 64, size=d // group) * 2.0 ** e
+            rows.append((mins[:, None] + codes * (2.0 ** e)[:, None]).reshape(d))
+        kv = np.array(rows).astype(np.float16).reshape(2, L, d)
+        k, v = np.tile(kv[0], (1, H)), np.tile(kv[1], (1, H))
+        oracle.kv_append(c, k, v, np.full(L, s), np.arange(L))
+    q = si.normal_f16(8, 1, (S, H * d), 1.0)
+    lens = np.array([L, 20], dtype=np.int32)
+    assert np.array_equal(oracle.attention(c, q, np.arange(S), lens),
+                          oracle.attention(c, q, np.arange(S), lens, exact_dequant=True))
+
+
 def test_attention_two_tokens_logistic():
     # K_0 = 0 (constant group), K_1 = constant c: scores 0 and c*sum(q); softmax of two is logistic
     S, H, d = 1, 1, 64
