@@ -53,9 +53,9 @@ struct AttnArgs {
   unsigned int *err;
 };
 
-template <int D>
+template <int D, int G>
 struct AttnShape {
-  static constexpr int NG = D / 64;                 // 64-groups per head
+  static constexpr int NG = D / G;                  // G-groups (G = 64 or 128) per head
   static constexpr int RB = D / 2;                  // code bytes per token row
   static constexpr int KW = D / 32;                 // K code words per lane per token
   static constexpr int VW = D / 64;                 // V code words per lane per token
@@ -67,7 +67,7 @@ struct AttnShape {
 };
 
 // Byte offset in a K code row of word j of lane class c (lane % 4): the dims that lane
-// class feeds to the score MMAs.  Always inside one 64-group (32 bytes).
+// class feeds to the score MMAs.  Always inside one group (32 or 64 bytes).
 template <int D>
 __device__ __forceinline__ int kword_off(int c, int j) {
   return D == 64 ? 8 * c + 4 * j : 64 * (j >> 2) + 16 * c + 4 * (j & 3);
@@ -154,9 +154,9 @@ __device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
   return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-template <int D>
+template <int D, int G>
 __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs a) {
-  using S = AttnShape<D>;
+  using S = AttnShape<D, G>;
   constexpr int NG = S::NG, RB = S::RB, KW = S::KW, VW = S::VW, MT = S::MT;
   constexpr float kS24 = 16777216.0f, kS20 = 1048576.0f;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
 #pragma unroll
   for (int j = 0; j < KW; j++) {
     const int o = kword_off<D>(c, j);
-    if (col_group<NG>(gid) == o / 32) {
+    if (col_group<NG>(gid) == o / (G / 2)) {
       const uint4 v = *reinterpret_cast<const uint4 *>(qrow + 2 * o);
       const __half *e = reinterpret_cast<const __half *>(&v);
       qlo[j][0] = pack_h2(e[0], e[4]);
@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
   constexpr int GPL = NG == 4 ? 2 : 1;  // groups per lane
   float ql[GPL];                         // sum of q over those groups, times log2(e)
   {
-    constexpr int PER = D / 32, LPG = 64 / PER;  // dims per lane, lanes per group
+    constexpr int PER = D / 32, LPG = G / PER;   // dims per lane, lanes per group
     float qs = 0.f;
 #pragma unroll
     for (int i = 0; i < PER; i++) qs += __half2float(qrow[lane * PER + i]);
@@ -386,10 +386,10 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
     for (int e = 0; e < GPL; e++) vmin[e] += __shfl_xor_sync(0xffffffffu, vmin[e], o);
   if constexpr (NG == 1) vmin[0] *= 0.5f;
   {
-    // lane (gid, c) with c == g/2 owns dims gid*D/8 .. +D/8-1 of group g = gid*D/512:
+    // lane (gid, c) with c == g/2 owns dims gid*D/8 .. +D/8-1 of group g = gid*(D/8)/G:
     // column g is element (g & 1) of its accumulator pairs; the V-min total of group g sits
     // in lane (g / GPL) % 2, element g % GPL
-    const int g = gid * D / 512;
+    const int g = gid * (D / 8) / G;
     const int gl = NG > 1 ? (g / GPL) & 1 : 0;
     float vm = __shfl_sync(0xffffffffu, vmin[0], gl);
     if constexpr (GPL == 2) {
@@ -427,29 +427,38 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
   }
 }
 
-template <int D>
+template <int D, int G>
 fg_status launch(const AttnArgs &a, cudaStream_t st) {
-  using S = AttnShape<D>;
+  using S = AttnShape<D, G>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     fg_status rc = fg_cuda_check(
-        cudaFuncSetAttribute(attn_decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM));
+        cudaFuncSetAttribute(attn_decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM));
     if (rc != FG_OK) return rc;
     attr_set[dev] = true;
   }
   const int64_t ctas = static_cast<int64_t>(a.rows) * a.H;
-  attn_decode_kernel<D><<<static_cast<unsigned>(ctas), kWarps * 32, S::SMEM, st>>>(a);
+  attn_decode_kernel<D, G><<<static_cast<unsigned>(ctas), kWarps * 32, S::SMEM, st>>>(a);
   return fg_launch_check();
 }
 
 }  // namespace
 
 fg_status fg_kv_validate(const fg_kv_cache *kv);
+fg_status fg_attention_prefill_launch(const fg_kv_cache *kv, const fg_half *q, int64_t ldq, fg_half *out,
+                                      int64_t ldo, int rows, int rows_per_seq, const int32_t *positions,
+                                      cudaStream_t st);
 
+// Prompt rows (rows_per_seq > 1) go to the tiled prefill kernel, which reads each K/V tile once
+// for 64 query rows; decode rows, and head dims that kernel does not take, to this one.
 fg_status fg_attention_launch(const fg_kv_cache *kv, const fg_half *q, int64_t ldq, fg_half *out, int64_t ldo,
                               int rows, int rows_per_seq, const int32_t *positions, cudaStream_t st) {
+  if (rows_per_seq > 1) {
+    const fg_status rc = fg_attention_prefill_launch(kv, q, ldq, out, ldo, rows, rows_per_seq, positions, st);
+    if (rc != FG_ERR_UNSUPPORTED) return rc;
+  }
   AttnArgs a;
   a.q = reinterpret_cast<const __half *>(q);
   a.ldq = ldq;
@@ -468,10 +477,18 @@ fg_status fg_attention_launch(const fg_kv_cache *kv, const fg_half *q, int64_t l
   a.maxL = kv->max_len;
   a.err = fg_error_word_ptr();
   if (!a.err) return FG_ERR_CUDA;
-  switch (kv->head_dim) {
-    case 64: return launch<64>(a, st);
-    case 128: return launch<128>(a, st);
-    case 256: return launch<256>(a, st);
+  const int G = fg_kv_group(kv->group);
+  if (G == 64) {
+    switch (kv->head_dim) {
+      case 64: return launch<64, 64>(a, st);
+      case 128: return launch<128, 64>(a, st);
+      case 256: return launch<256, 64>(a, st);
+    }
+  } else if (G == 128) {
+    switch (kv->head_dim) {
+      case 128: return launch<128, 128>(a, st);
+      case 256: return launch<256, 128>(a, st);
+    }
   }
   return FG_ERR_UNSUPPORTED;
 }

@@ -26,6 +26,10 @@ fg_status fg_launch_check();             // cudaGetLastError after a launch
 
 static inline bool fg_aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The 4-bit group of a KV cache or layer config: 0 selects 64; 64 and 128 as given; 0 for any
+// other value (unsupported).
+static inline int fg_kv_group(int group) { return group == 0 ? 64 : (group == 64 || group == 128) ? group : 0; }
+
 // --------------------------------------------------------------------------------------
 // device helpers
 // --------------------------------------------------------------------------------------

@@ -33,6 +33,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 bool config_ok(const fg_layer_config *c) {
   if (!c) return false;
   if (c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256) return false;
+  const int G = fg_kv_group(c->group);
+  if (G == 0 || c->head_dim % G) return false;
   if (c->num_heads < 1 || c->hidden != c->num_heads * c->head_dim) return false;
   if (c->hidden % 128 || c->ffn % 128 || c->ffn <= 0 || c->hidden > 16384) return false;
   return true;
@@ -53,6 +55,7 @@ struct BlobLayout {
 BlobLayout blob_layout(const fg_layer_config *c) {
   BlobLayout L;
   const int64_t h = c->hidden, F = c->ffn;
+  const int64_t G = fg_kv_group(c->group);
   L.mat[0] = {3 * h, h};
   L.mat[1] = {h, h};
   L.mat[2] = {F, h};
@@ -63,9 +66,9 @@ BlobLayout blob_layout(const fg_layer_config *c) {
     L.off[i][0] = p;
     p = align256(p + numel / 2);
     L.off[i][1] = p;
-    p = align256(p + numel / 64 * 2);
+    p = align256(p + numel / G * 2);
     L.off[i][2] = p;
-    p = align256(p + numel / 64 * 2);
+    p = align256(p + numel / G * 2);
   }
   const int64_t vlen[8] = {3 * h, h, F, h, h, h, h, h};
   for (int i = 0; i < 8; i++) {
@@ -108,8 +111,9 @@ bool weights_ok(const fg_layer_config *c, const fg_layer_weights *w) {
   const int64_t h = c->hidden, F = c->ffn;
   const fg_qtensor *m[4] = {&w->wqkv, &w->wo, &w->w1, &w->w2};
   const int64_t shp[4][2] = {{3 * h, h}, {h, h}, {F, h}, {h, F}};
+  const int G = fg_kv_group(c->group);
   for (int i = 0; i < 4; i++) {
-    if (m[i]->ndim != 2 || m[i]->dim != 1 || m[i]->bits != 4 || m[i]->group != 64) return false;
+    if (m[i]->ndim != 2 || m[i]->dim != 1 || m[i]->bits != 4 || m[i]->group != G) return false;
     if (m[i]->shape[0] != shp[i][0] || m[i]->shape[1] != shp[i][1]) return false;
     if (!m[i]->codes || !m[i]->mins || !m[i]->scales || !fg_aligned16(m[i]->codes)) return false;
   }
@@ -167,12 +171,13 @@ fg_status run_layer(const fg_layer_config *c, const fg_layer_weights *w, const f
 fg_kv_cache kv_view(const fg_kv_cache *kv, int s0, int n) {
   fg_kv_cache v = *kv;
   const size_t slots = static_cast<size_t>(s0) * kv->num_heads * kv->max_len;
+  const size_t ng = kv->head_dim / fg_kv_group(kv->group);
   v.k_codes += slots * (kv->head_dim / 2);
   v.v_codes += slots * (kv->head_dim / 2);
-  v.k_mins += slots * (kv->head_dim / 64);
-  v.k_scales += slots * (kv->head_dim / 64);
-  v.v_mins += slots * (kv->head_dim / 64);
-  v.v_scales += slots * (kv->head_dim / 64);
+  v.k_mins += slots * ng;
+  v.k_scales += slots * ng;
+  v.v_mins += slots * ng;
+  v.v_scales += slots * ng;
   v.num_seqs = n;
   return v;
 }
@@ -184,6 +189,7 @@ fg_status check_common(const fg_layer_config *c, const fg_layer_weights *w, cons
   fg_status rc = fg_kv_validate(kv);
   if (rc != FG_OK) return rc;
   if (kv->num_heads != c->num_heads || kv->head_dim != c->head_dim) return FG_ERR_SHAPE;
+  if (fg_kv_group(kv->group) != fg_kv_group(c->group)) return FG_ERR_SHAPE;
   if (nb < 0 || gbs < 0) return FG_ERR_INVALID;
   if (static_cast<int64_t>(nb) * gbs != kv->num_seqs) return FG_ERR_SHAPE;
   if (kv->num_seqs == 0) return FG_OK;
@@ -214,7 +220,7 @@ extern "C" fg_status fg_layer_weights_from_blob(const fg_layer_config *c, void *
     m[i]->shape[2] = m[i]->shape[3] = 1;
     m[i]->dim = 1;
     m[i]->bits = 4;
-    m[i]->group = 64;
+    m[i]->group = fg_kv_group(c->group);
   }
   fg_half **v[8] = {&out->bqkv, &out->bo, &out->b1, &out->b2, &out->ln1_g, &out->ln1_b, &out->ln2_g, &out->ln2_b};
   for (int i = 0; i < 8; i++) *v[i] = reinterpret_cast<fg_half *>(b + L.vec[i]);

@@ -173,8 +173,8 @@ __global__ void __launch_bounds__(256) dequantize_strided_kernel(const uint8_t *
 }
 
 // ------------------------------------------------------------------------------------
-// K5: append new k, v rows to the 4-bit cache.  Work unit = one 64-group of k or v of
-// one head of one row; 8 lanes per unit, 4 units per warp step.
+// K5: append new k, v rows to the 4-bit cache.  Work unit = one G-group (64 or 128) of k or
+// v of one head of one row; G/8 lanes per unit, 32/(G/8) units per warp step.
 // ------------------------------------------------------------------------------------
 struct KvArgs {
   uint32_t *kc, *vc;  // codes as 32-bit words
@@ -182,15 +182,17 @@ struct KvArgs {
   int H, d, maxL, num_seqs;
 };
 
+template <int G>
 __global__ void __launch_bounds__(256) kv_append_kernel(const __half *__restrict__ k, const __half *__restrict__ v,
                                                         int64_t ld, int rows, int rows_per_seq,
                                                         const int32_t *__restrict__ positions, KvArgs a,
                                                         unsigned int *err) {
-  // A warp takes one (row, head) item per step: its 2 * d/64 units (k and v groups), 4 at a
-  // time in the four 8-lane slots; unit us = group * 2 + (0 for k, 1 for v).
+  // A warp takes one (row, head) item per step: its 2 * d/G units (k and v groups), USTEP at
+  // a time in its G/8-lane slots; unit us = group * 2 + (0 for k, 1 for v).
+  constexpr int L = G / 8, USTEP = 32 / L;
   const int lane = threadIdx.x & 31;
-  const int slot = lane >> 3, j = lane & 7;
-  const int ng = a.d >> 6;
+  const int slot = lane / L, j = lane % L;
+  const int ng = a.d / G;
   const int items = rows * a.H;
   const int warp = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
   const int nwarps = static_cast<int>((static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5);
@@ -200,21 +202,21 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __half *__restrict
     const int pos = positions[s] + (r - s * rows_per_seq);
     const bool in_range = pos >= 0 && pos < a.maxL;
     const int64_t slot_idx = (static_cast<int64_t>(s) * a.H + hd) * a.maxL + pos;
-    for (int u0 = 0; u0 < 2 * ng; u0 += 4) {  // warp-uniform
+    for (int u0 = 0; u0 < 2 * ng; u0 += USTEP) {  // warp-uniform
       const int us = u0 + slot;
       const bool live = us < 2 * ng;
       const int which = us & 1, g = us >> 1;
       uint4 val = make_uint4(0, 0, 0, 0);
       if (live) val = *reinterpret_cast<const uint4 *>((which ? v : k) + static_cast<int64_t>(r) * ld + hd * a.d +
-                                                       g * 64 + j * 8);
+                                                       g * G + j * 8);
       __half mn, sc;
-      const uint32_t w = quant_group8(val, mn, sc);
+      const uint32_t w = quant_group8<L>(val, mn, sc);
       if (!live) continue;
       if (!in_range) {
         if (j == 0) atomicOr(err, FG_DEVERR_RANGE);
         continue;
       }
-      (which ? a.vc : a.kc)[slot_idx * (a.d / 8) + g * 8 + j] = w;
+      (which ? a.vc : a.kc)[slot_idx * (a.d / 8) + g * L + j] = w;
       if (j == 0) {
         const int64_t m = slot_idx * ng + g;
         (which ? a.vm : a.km)[m] = mn;
@@ -325,20 +327,23 @@ extern "C" fg_status fg_dequantize(const fg_qtensor *q, fg_half *y, void *stream
   return fg_launch_check();
 }
 
-extern "C" fg_status fg_kv_cache_bytes(int num_seqs, int num_heads, int head_dim, int max_len,
+extern "C" fg_status fg_kv_cache_bytes(int num_seqs, int num_heads, int head_dim, int max_len, int group,
                                        size_t *codes_bytes, size_t *meta_bytes) {
   if (num_seqs < 0 || num_heads < 1 || max_len < 0) return FG_ERR_INVALID;
   if (head_dim != 64 && head_dim != 128 && head_dim != 256) return FG_ERR_UNSUPPORTED;
-  if (max_len % 64) return FG_ERR_SHAPE;
+  const int G = fg_kv_group(group);
+  if (G == 0) return FG_ERR_UNSUPPORTED;
+  if (max_len % 64 || head_dim % G) return FG_ERR_SHAPE;
   const size_t slots = static_cast<size_t>(num_seqs) * num_heads * max_len;
   if (codes_bytes) *codes_bytes = slots * (head_dim / 2);
-  if (meta_bytes) *meta_bytes = slots * (head_dim / 64) * 2;
+  if (meta_bytes) *meta_bytes = slots * (head_dim / G) * 2;
   return FG_OK;
 }
 
 fg_status fg_kv_validate(const fg_kv_cache *kv) {
   if (!kv) return FG_ERR_INVALID;
-  fg_status rc = fg_kv_cache_bytes(kv->num_seqs, kv->num_heads, kv->head_dim, kv->max_len, nullptr, nullptr);
+  fg_status rc = fg_kv_cache_bytes(kv->num_seqs, kv->num_heads, kv->head_dim, kv->max_len, kv->group, nullptr,
+                                   nullptr);
   if (rc != FG_OK) return rc;
   const void *p[6] = {kv->k_codes, kv->k_mins, kv->k_scales, kv->v_codes, kv->v_mins, kv->v_scales};
   for (const void *ptr : p)
@@ -363,9 +368,10 @@ fg_status fg_kv_append_launch(const fg_kv_cache *kv, const fg_half *k, const fg_
   if (!err) return FG_ERR_CUDA;
   const int64_t items = static_cast<int64_t>(rows) * kv->num_heads;  // one warp per (row, head)
   if (items > INT32_MAX) return FG_ERR_SHAPE;
-  kv_append_kernel<<<grid_for((items + 7) / 8, 8), 256, 0, st>>>(
-      reinterpret_cast<const __half *>(k), reinterpret_cast<const __half *>(v), ld, rows, rows_per_seq, positions, a,
-      err);
+  auto kern = fg_kv_group(kv->group) == 128 ? kv_append_kernel<128> : kv_append_kernel<64>;
+  kern<<<grid_for((items + 7) / 8, 8), 256, 0, st>>>(reinterpret_cast<const __half *>(k),
+                                                     reinterpret_cast<const __half *>(v), ld, rows, rows_per_seq,
+                                                     positions, a, err);
   return fg_launch_check();
 }
 

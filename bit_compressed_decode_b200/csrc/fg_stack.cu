@@ -88,7 +88,7 @@ fg_status stack_run(fg_stack *st, const fg_kv_cache *kv, const fg_half *x_in, fg
 
 bool same_geometry(const fg_kv_cache &a, const fg_kv_cache &b) {
   return a.num_seqs == b.num_seqs && a.num_heads == b.num_heads && a.head_dim == b.head_dim &&
-         a.max_len == b.max_len;
+         a.max_len == b.max_len && fg_kv_group(a.group) == fg_kv_group(b.group);
 }
 
 // Positions [p0, p1) of every (sequence, head) row of the six cache arrays, src -> dst,
@@ -97,7 +97,7 @@ fg_status kv_copy(const fg_kv_cache &dst, const fg_kv_cache &src, int p0, int p1
                   cudaStream_t s) {
   if (p1 <= p0) return FG_OK;
   const size_t rows = static_cast<size_t>(src.num_seqs) * src.num_heads;
-  const size_t cpos = src.head_dim / 2, mpos = (src.head_dim / 64) * 2;  // bytes per slot
+  const size_t cpos = src.head_dim / 2, mpos = (src.head_dim / fg_kv_group(src.group)) * 2;  // bytes per slot
   const size_t n = static_cast<size_t>(p1 - p0);
   struct Arr {
     void *d;
