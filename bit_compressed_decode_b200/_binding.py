@@ -24,6 +24,7 @@ STATUS = {0: "FG_OK", 1: "FG_ERR_INVALID", 2: "FG_ERR_SHAPE", 3: "FG_ERR_UNSUPPO
           5: "FG_ERR_CUDA", 6: "FG_ERR_TIMEOUT", 7: "FG_ERR_WORKSPACE"}
 FG_EPI_RELU = 1
 FG_EPI_RESIDUAL = 2
+FG_GEMM_PERSISTENT = 4
 
 
 class FgError(RuntimeError):
@@ -43,12 +44,13 @@ class fg_qtensor(Structure):
 class fg_kv_cache(Structure):
     _fields_ = [("k_codes", c_void_p), ("k_mins", c_void_p), ("k_scales", c_void_p),
                 ("v_codes", c_void_p), ("v_mins", c_void_p), ("v_scales", c_void_p),
-                ("num_seqs", c_int32), ("num_heads", c_int32), ("head_dim", c_int32), ("max_len", c_int32)]
+                ("num_seqs", c_int32), ("num_heads", c_int32), ("head_dim", c_int32), ("max_len", c_int32),
+                ("group", c_int32)]
 
 
 class fg_layer_config(Structure):
     _fields_ = [("hidden", c_int32), ("num_heads", c_int32), ("head_dim", c_int32), ("ffn", c_int32),
-                ("ln_eps", c_float)]
+                ("ln_eps", c_float), ("group", c_int32)]
 
 
 class fg_layer_weights(Structure):
@@ -70,11 +72,11 @@ _decl("fg_last_cuda_error", c_char_p)
 _decl("fg_qtensor_bytes", c_int, c_int, POINTER(c_int64), c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_size_t))
 _decl("fg_quantize", c_int, P, c_int, POINTER(c_int64), c_int, c_int, c_int, POINTER(fg_qtensor), P)
 _decl("fg_dequantize", c_int, POINTER(fg_qtensor), P, P)
-_decl("fg_kv_cache_bytes", c_int, c_int, c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_size_t))
+_decl("fg_kv_cache_bytes", c_int, c_int, c_int, c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_size_t))
 _decl("fg_kv_append", c_int, POINTER(fg_kv_cache), P, P, c_int64, c_int, c_int, P, P)
 _decl("fg_attention_decode", c_int, POINTER(fg_kv_cache), P, c_int64, P, c_int64, c_int, c_int, P, P)
 _decl("fg_linear_workspace_bytes", c_size_t, c_int, c_int, c_int)
-_decl("fg_linear_plan", c_int, c_int, c_int, c_int, POINTER(c_int), POINTER(c_int))
+_decl("fg_linear_plan", c_int, c_int, c_int, c_int, POINTER(c_int), POINTER(c_int), POINTER(c_int))
 _decl("fg_linear_w4a16", c_int, P, c_int, c_int, POINTER(fg_qtensor), P, P, c_int, c_int, c_float, P, P, c_size_t, P)
 _decl("fg_layernorm", c_int, P, c_int, c_int, P, P, c_float, P, P)
 _decl("fg_layer_blob_bytes", c_size_t, POINTER(fg_layer_config))
@@ -187,16 +189,19 @@ def fg_dequantize(q: QTensor, stream=None) -> torch.Tensor:
 # ---------------------------------------------------------------------------------------
 
 class KVCache:
-    """4-bit KV cache of one layer, allocated with torch on ``device``."""
+    """4-bit KV cache of one layer, allocated with torch on ``device``; head_dim quantised in
+    groups of ``group`` (64 or 128)."""
 
-    def __init__(self, num_seqs, num_heads, head_dim, max_len, device="cuda", arrays=None, pin_memory=False):
+    def __init__(self, num_seqs, num_heads, head_dim, max_len, device="cuda", arrays=None, pin_memory=False,
+                 group: int = 64):
         """``pin_memory=True`` with ``device="cpu"`` allocates page-locked host arrays, the form
         fg_stack_decode_host_kv copies from and back to."""
         self.num_seqs, self.num_heads, self.head_dim, self.max_len = num_seqs, num_heads, head_dim, max_len
+        self.group = group
         cb, mb = c_size_t(), c_size_t()
-        _check(_lib.fg_kv_cache_bytes(num_seqs, num_heads, head_dim, max_len, ctypes.byref(cb), ctypes.byref(mb)),
-               "fg_kv_cache_bytes")
-        ng = head_dim // 64
+        _check(_lib.fg_kv_cache_bytes(num_seqs, num_heads, head_dim, max_len, group, ctypes.byref(cb),
+                                      ctypes.byref(mb)), "fg_kv_cache_bytes")
+        ng = head_dim // group
         if arrays is None:
             cshape = (num_seqs, num_heads, max_len, head_dim // 2)
             mshape = (num_seqs, num_heads, max_len, ng)
@@ -215,12 +220,13 @@ class KVCache:
     def view(self, s0: int, n: int) -> "KVCache":
         """The cache of sequences [s0, s0+n) (shares memory)."""
         return KVCache(n, self.num_heads, self.head_dim, self.max_len,
-                       arrays=[a[s0:s0 + n] for a in self.arrays()])
+                       arrays=[a[s0:s0 + n] for a in self.arrays()], group=self.group)
 
     def struct(self) -> fg_kv_cache:
         s = fg_kv_cache()
         (s.k_codes, s.k_mins, s.k_scales, s.v_codes, s.v_mins, s.v_scales) = [a.data_ptr() for a in self.arrays()]
         s.num_seqs, s.num_heads, s.head_dim, s.max_len = self.num_seqs, self.num_heads, self.head_dim, self.max_len
+        s.group = self.group
         return s
 
     def nbytes(self) -> int:
@@ -258,14 +264,33 @@ def fg_linear_workspace_bytes(M: int, N: int, K: int) -> int:
 
 
 def fg_linear_plan(M: int, N: int, K: int) -> tuple:
-    """(tokens per output tile, k splits) of the launch fg_linear_w4a16 makes for this shape."""
-    t, s = c_int(), c_int()
-    _check(_lib.fg_linear_plan(M, N, K, ctypes.byref(t), ctypes.byref(s)), "fg_linear_plan")
+    """(tokens per output tile, k splits) of the classic launch fg_linear_w4a16 makes for this
+    shape (see fg_linear_plan_pairs for the persistent launch)."""
+    t, s, p = c_int(), c_int(), c_int()
+    _check(_lib.fg_linear_plan(M, N, K, ctypes.byref(t), ctypes.byref(s), ctypes.byref(p)), "fg_linear_plan")
     return t.value, s.value
 
 
+def fg_linear_plan_pairs(M: int, N: int, K: int) -> int:
+    """CTA pairs of the persistent launch fg_linear_w4a16(..., persistent=True) takes for this
+    shape given fg_linear_workspace_bytes of scratch (0: not available, the classic launch)."""
+    t, s, p = c_int(), c_int(), c_int()
+    _check(_lib.fg_linear_plan(M, N, K, ctypes.byref(t), ctypes.byref(s), ctypes.byref(p)), "fg_linear_plan")
+    return p.value
+
+
+def fg_linear_classic_scratch_bytes(M: int, N: int, K: int) -> int:
+    """Scratch the classic launch's split k-range adds its partial sums through (0 without a
+    split); with less than that (and less than fg_linear_workspace_bytes) it adds them on chip."""
+    t, s = fg_linear_plan(M, N, K)
+    if M <= 256 or s < 2:
+        return 0
+    return -(-N // 256) * -(-M // t) * s * t * 256 * 4
+
+
 def fg_linear_w4a16(x: torch.Tensor, w: QTensor, bias=None, residual=None, relu: bool = False,
-                    qscale_cols: int = 0, qscale: float = 1.0, out=None, workspace=None, stream=None):
+                    qscale_cols: int = 0, qscale: float = 1.0, out=None, workspace=None, stream=None,
+                    persistent: bool = False):
     _need(x, torch.float16, "x")
     M, K = x.shape
     N = w.shape[0]
@@ -274,7 +299,8 @@ def fg_linear_w4a16(x: torch.Tensor, w: QTensor, bias=None, residual=None, relu:
     need = fg_linear_workspace_bytes(M, N, K)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
-    flags = (FG_EPI_RELU if relu else 0) | (FG_EPI_RESIDUAL if residual is not None else 0)
+    flags = ((FG_EPI_RELU if relu else 0) | (FG_EPI_RESIDUAL if residual is not None else 0) |
+             (FG_GEMM_PERSISTENT if persistent else 0))
     s = w.struct()
     _check(_lib.fg_linear_w4a16(_ptr(x), M, K, ctypes.byref(s), _ptr(bias), _ptr(residual), flags, qscale_cols,
                                 qscale, _ptr(out), _ptr(workspace), 0 if workspace is None else workspace.numel(),
@@ -297,12 +323,13 @@ def fg_layernorm(x: torch.Tensor, gamma=None, beta=None, eps: float = 1e-5, out=
 # ---------------------------------------------------------------------------------------
 
 class LayerConfig:
-    def __init__(self, hidden: int, num_heads: int, ffn: int, ln_eps: float = 1e-5):
-        self.hidden, self.num_heads, self.ffn, self.ln_eps = hidden, num_heads, ffn, ln_eps
+    def __init__(self, hidden: int, num_heads: int, ffn: int, ln_eps: float = 1e-5, group: int = 64):
+        """``group``: the 4-bit group of the layer's weights and KV cache (64 or 128)."""
+        self.hidden, self.num_heads, self.ffn, self.ln_eps, self.group = hidden, num_heads, ffn, ln_eps, group
         self.head_dim = hidden // num_heads
 
     def struct(self) -> fg_layer_config:
-        return fg_layer_config(self.hidden, self.num_heads, self.head_dim, self.ffn, self.ln_eps)
+        return fg_layer_config(self.hidden, self.num_heads, self.head_dim, self.ffn, self.ln_eps, self.group)
 
     def blob_bytes(self) -> int:
         c = self.struct()
@@ -347,10 +374,11 @@ class LayerWeights:
         def sub(ptr, nbytes):
             off = ptr - base
             return self.blob[off:off + nbytes]
+        G = self.cfg.group
         codes = sub(q.codes, n * k // 2).view(n, k // 2)
-        mins = sub(q.mins, n * k // 64 * 2).view(torch.float16).view(n, k // 64)
-        scales = sub(q.scales, n * k // 64 * 2).view(torch.float16).view(n, k // 64)
-        return QTensor(codes, mins, scales, (n, k), 1)
+        mins = sub(q.mins, n * k // G * 2).view(torch.float16).view(n, k // G)
+        scales = sub(q.scales, n * k // G * 2).view(torch.float16).view(n, k // G)
+        return QTensor(codes, mins, scales, (n, k), 1, G)
 
     def vector(self, name: str) -> torch.Tensor:
         ptr = getattr(self._w, name)
@@ -365,7 +393,7 @@ class LayerWeights:
         lw = LayerWeights(cfg, blob)
         for name in _MATS:
             x = torch.as_tensor(w16[name]).to(device=device, dtype=torch.float16).contiguous()
-            fg_quantize(x, dim=1, stream=stream, out=lw.matrix(name))
+            fg_quantize(x, dim=1, group=cfg.group, stream=stream, out=lw.matrix(name))
         for name in _VECS:
             lw.vector(name).copy_(torch.as_tensor(w16[name]).to(device=device, dtype=torch.float16))
         return lw
@@ -390,7 +418,7 @@ def fg_layer_decode(cfg: LayerConfig, w: LayerWeights, cache: KVCache, x: torch.
     return out
 
 
-NOALLOC_SCRATCH_BYTES = 48 << 20
+NOALLOC_SCRATCH_BYTES = 96 << 20
 
 
 def fg_layer_decode_noalloc(cfg: LayerConfig, w: LayerWeights, cache: KVCache, x: torch.Tensor,

@@ -33,6 +33,14 @@
 
 #include "fg_internal.cuh"
 
+// the persistent stream-K launch (fg_gemm_streamk.cu)
+int fg_streamk_pairs();
+size_t fg_streamk_scratch_bytes(int pairs);
+fg_status fg_streamk_launch(const CUtensorMap &map, const uint8_t *wc, const __half *wm, const __half *wsc, int gshift,
+                            const __half *bias, const __half *res, int relu, int qcols, float qscale, __half *y,
+                            int M, int N, int K, int pairs, void *scratch, unsigned int *err, cudaStream_t st,
+                            bool pdl);
+
 namespace {
 
 constexpr int kBK = 64;                      // k-tile = one quantisation group
@@ -878,12 +886,16 @@ int pick_nt(int M) {
 
 struct Plan {
   int nt, n_tiles, t_tiles, splits;
+  double cost;  // pair kernel: modelled microseconds
+  int pairs;    // > 0: the persistent stream-K launch over this many CTA pairs is faster
 };
 
 // Split the k-range over the CTAs of a cluster only to fill the SMs: minimise
 // waves * k-tiles per CTA, with a small charge per extra split for the cluster reduction.
 Plan make_plan(int M, int N, int K) {
   Plan p;
+  p.pairs = 0;
+  p.cost = 0.0;
   p.nt = pick_nt(M);
   p.n_tiles = (N + kBM - 1) / kBM;
   p.t_tiles = (M + p.nt - 1) / p.nt;
@@ -1022,6 +1034,21 @@ Plan make_pair_plan(int M, int N, int K) {
     }
   }
   p.t_tiles = (M + p.nt - 1) / p.nt;
+  p.cost = best;
+  // The persistent stream-K launch (every resident pair takes an equal share of the (tile,
+  // k-tile) iterations of 512-token tiles) runs only when a caller asks for it
+  // (FG_GEMM_PERSISTENT): measured on the decode shapes it is still 1.5-2.6x slower than this
+  // classic launch, so the time model does not choose it.  It needs every tile split into at
+  // most 13 segments (the staging buffers of a split tile's partials).
+  p.pairs = 0;
+  const int sk = fg_streamk_pairs();
+  if (sk > 0) {
+    const int64_t iters = static_cast<int64_t>(p.n_tiles) * ((M + 511) / 512) * ktiles;
+    const int P = static_cast<int>(iters < sk ? iters : sk);
+    const int64_t per = (iters + P - 1) / P;
+    const int64_t segs = per >= ktiles ? 2 : (ktiles + per - 1) / per + 1;  // most segments of a tile
+    if (segs - 1 <= 12) p.pairs = sk;
+  }
   return p;
 }
 
@@ -1061,13 +1088,15 @@ std::atomic<uint64_t> g_stall_wait_ns{FG_WAIT_TIMEOUT_NS};
 
 // Optional scratch of the pair kernel's k split: one fp32 partial [tile tokens][256 features]
 // per split of every pair tile.  Without it the partials are reduced inside the cluster.
-size_t pair_part_bytes(const Plan &p) {
+static size_t pair_part_bytes(const Plan &p) {
   return p.splits < 2 ? 0 : static_cast<size_t>(p.n_tiles) * p.t_tiles * p.splits * p.nt * 256 * sizeof(float);
 }
 
 size_t fg_linear_ws_bytes(int M, int N, int K) {
   if (M <= 256 || N <= 0 || K <= 0 || K % kBK) return 0;
-  return pair_part_bytes(make_pair_plan(M, N, K));
+  const Plan p = make_pair_plan(M, N, K);
+  const size_t classic = pair_part_bytes(p), sk = p.pairs > 0 ? fg_streamk_scratch_bytes(p.pairs) : 0;
+  return classic > sk ? classic : sk;
 }
 
 fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, const fg_half *bias,
@@ -1110,6 +1139,10 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
   if (!a.err) return FG_ERR_CUDA;
   a.wait_ns = FG_WAIT_TIMEOUT_NS;
   a.stall = 0;
+  if (pair && (flags & FG_GEMM_PERSISTENT) && p.pairs > 0 && workspace && fg_aligned16(workspace) &&
+      ws_bytes >= fg_streamk_scratch_bytes(p.pairs))
+    return fg_streamk_launch(map, a.wc, a.wm, a.ws, a.gshift, a.bias, a.res, a.relu, a.qcols, a.qscale, a.y, M, N, K,
+                             p.pairs, workspace, a.err, st, pdl);
   if (pair) return launch_pair(map, a, p, st, pdl);
   int left = g_stall_count.load();
   while (left > 0 && !g_stall_count.compare_exchange_weak(left, left - 1)) {
@@ -1136,11 +1169,18 @@ extern "C" fg_status fg_test_gemm_stall(int count, uint64_t wait_limit_ns) {
   return FG_OK;
 }
 
-extern "C" fg_status fg_linear_plan(int M, int N, int K, int *tile_tokens, int *splits) {
-  if (!tile_tokens || !splits || M <= 0 || N <= 0 || K <= 0 || K % kBK || N % 128) return FG_ERR_INVALID;
-  const Plan p = M > 256 ? make_pair_plan(M, N, K) : make_plan(M, N, K);
+extern "C" fg_status fg_linear_plan(int M, int N, int K, int *tile_tokens, int *splits, int *pairs) {
+  if (!tile_tokens || !splits || !pairs || M <= 0 || N <= 0 || K <= 0 || K % kBK || N % 128) return FG_ERR_INVALID;
+  Plan p;
+  if (M > 256) {
+    p = make_pair_plan(M, N, K);
+  } else {
+    p = make_plan(M, N, K);
+    p.pairs = 0;
+  }
   *tile_tokens = p.nt;
   *splits = p.splits;
+  *pairs = p.pairs;
   return FG_OK;
 }
 
@@ -1152,7 +1192,7 @@ extern "C" fg_status fg_linear_w4a16(const fg_half *x, int M, int K, const fg_qt
   if (w->ndim != 2 || w->dim != 1 || w->shape[1] != K) return FG_ERR_SHAPE;
   const int64_t N = w->shape[0];
   if (K % w->group || N <= 0 || N % 128 || N > (1 << 30)) return FG_ERR_SHAPE;
-  if (flags & ~(FG_EPI_RELU | FG_EPI_RESIDUAL)) return FG_ERR_INVALID;
+  if (flags & ~(FG_EPI_RELU | FG_EPI_RESIDUAL | FG_GEMM_PERSISTENT)) return FG_ERR_INVALID;
   if (M == 0) return FG_OK;
   if (!x || !y || !w->codes || !w->mins || !w->scales) return FG_ERR_INVALID;
   if (!fg_aligned16(x) || !fg_aligned16(y) || !fg_aligned16(w->codes)) return FG_ERR_INVALID;

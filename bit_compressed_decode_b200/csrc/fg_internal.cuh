@@ -26,6 +26,23 @@ fg_status fg_launch_check();             // cudaGetLastError after a launch
 
 static inline bool fg_aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Events of a layer step whose weights (and cache) arrive in slices (the stack's sliced
+// prefetch): `ready` events the step waits for before the kernels that read a slice, `done`
+// events it records once the kernels that read a slice have been enqueued.  Any may be null.
+//   ready: [0] vectors (biases, LayerNorm parameters) before LN1, [1] wqkv before the QKV GEMM,
+//          [2] the KV cache before the KV append, [3] wo, [4] w1, [5] w2 before their GEMMs.
+//   done:  [1] after the QKV GEMM, [2] after attention (the cache), [3] after the output
+//          projection, [4] after FC1, [0] and [5] after FC2 (its bias is the last vector read).
+struct fg_layer_slices {
+  cudaEvent_t ready[6];
+  cudaEvent_t done[6];
+};
+fg_status fg_layer_decode_sliced(const fg_layer_config *c, const fg_layer_weights *w, const fg_kv_cache *kv,
+                                 const fg_half *x_in, fg_half *x_out, const int32_t *positions, int num_gpu_batches,
+                                 int gpu_batch_size, void *workspace, size_t workspace_bytes, cudaStream_t st,
+                                 const fg_layer_slices *sl);
+fg_status fg_layer_blob_slices(const fg_layer_config *c, size_t begin[5], size_t end[5]);
+
 // The 4-bit group of a KV cache or layer config: 0 selects 64; 64 and 128 as given; 0 for any
 // other value (unsupported).
 static inline int fg_kv_group(int group) { return group == 0 ? 64 : (group == 64 || group == 128) ? group : 0; }

@@ -120,11 +120,25 @@ bool weights_ok(const fg_layer_config *c, const fg_layer_weights *w) {
   return true;
 }
 
+}  // namespace
+
+namespace {
+
+fg_status slice_wait(const fg_layer_slices *sl, int i, cudaStream_t st) {
+  if (!sl || !sl->ready[i]) return FG_OK;
+  return fg_cuda_check(cudaStreamWaitEvent(st, sl->ready[i], 0));
+}
+
+fg_status slice_done(const fg_layer_slices *sl, int i, cudaStream_t st) {
+  if (!sl || !sl->done[i]) return FG_OK;
+  return fg_cuda_check(cudaEventRecord(sl->done[i], st));
+}
+
 // The layer over `rows` hidden-state rows; row r is token r % rows_per_seq of
 // sequence r / rows_per_seq of `kv` (a view starting at the first sequence).
 fg_status run_layer(const fg_layer_config *c, const fg_layer_weights *w, const fg_kv_cache *kv, const fg_half *x_in,
                     fg_half *x_out, const int32_t *positions, int rows, int rows_per_seq, uint8_t *ws,
-                    size_t ws_bytes, cudaStream_t st) {
+                    size_t ws_bytes, cudaStream_t st, const fg_layer_slices *sl = nullptr) {
   const WsLayout L = ws_layout(c, rows);
   // the GEMMs' split-k scratch is optional: they reduce on chip when what is left is short
   if (ws_bytes < L.gemm) return FG_ERR_WORKSPACE;
@@ -148,23 +162,38 @@ fg_status run_layer(const fg_layer_config *c, const fg_layer_weights *w, const f
   ev = fg_profile_begin(slot, st);             \
   if ((rc = (call)) != FG_OK) return rc;       \
   fg_profile_end(ev, st);
+#define FG_SLICE(call)                   \
+  if ((rc = (call)) != FG_OK) return rc;
   // a = LN1(x)
+  FG_SLICE(slice_wait(sl, 0, st));
   FG_STEP(0, fg_layernorm_launch(x_in, rows, h, w->ln1_g, w->ln1_b, c->ln_eps, a, st));
   // [q k v] = a Wqkv^T + bqkv; q *= d^-1/2
+  FG_SLICE(slice_wait(sl, 1, st));
   FG_STEP(1, fg_linear_launch(a, rows, h, &w->wqkv, w->bqkv, nullptr, 0, h, qscale, qkv, gws, gbytes, st, pdl));
+  FG_SLICE(slice_done(sl, 1, st));
   // append k, v (4-bit) at the sequences' positions
+  FG_SLICE(slice_wait(sl, 2, st));
   FG_STEP(2, fg_kv_append_launch(kv, qkv + h, qkv + 2 * h, 3 * h, rows, rows_per_seq, positions, st));
   // o = softmax(q K^T) V over the 4-bit cache
   FG_STEP(3, fg_attention_launch(kv, qkv, 3 * h, o, h, rows, rows_per_seq, positions, st));
+  FG_SLICE(slice_done(sl, 2, st));
   // h1 = x + o Wo^T + bo
+  FG_SLICE(slice_wait(sl, 3, st));
   FG_STEP(4, fg_linear_launch(o, rows, h, &w->wo, w->bo, x_in, FG_EPI_RESIDUAL, 0, 1.f, h1, gws, gbytes, st, pdl));
+  FG_SLICE(slice_done(sl, 3, st));
   // a = LN2(h1)
   FG_STEP(5, fg_layernorm_launch(h1, rows, h, w->ln2_g, w->ln2_b, c->ln_eps, a, st));
   // f = relu(a W1^T + b1)
+  FG_SLICE(slice_wait(sl, 4, st));
   FG_STEP(6, fg_linear_launch(a, rows, h, &w->w1, w->b1, nullptr, FG_EPI_RELU, 0, 1.f, f, gws, gbytes, st, pdl));
+  FG_SLICE(slice_done(sl, 4, st));
   // x_out = h1 + f W2^T + b2
+  FG_SLICE(slice_wait(sl, 5, st));
   FG_STEP(7, fg_linear_launch(f, rows, F, &w->w2, w->b2, h1, FG_EPI_RESIDUAL, 0, 1.f, x_out, gws, gbytes, st, pdl));
+  FG_SLICE(slice_done(sl, 5, st));
+  FG_SLICE(slice_done(sl, 0, st));
 #undef FG_STEP
+#undef FG_SLICE
   return FG_OK;
 }
 
@@ -248,6 +277,33 @@ extern "C" fg_status fg_layer_decode(const fg_layer_config *c, const fg_layer_we
   if (!workspace || !fg_aligned16(workspace)) return FG_ERR_INVALID;
   return run_layer(c, w, kv, x_in, x_out, positions, kv->num_seqs, 1, static_cast<uint8_t *>(workspace),
                    workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+// fg_layer_decode whose weights and cache arrive in slices (see fg_layer_slices); the stack's
+// sliced prefetch calls it.
+fg_status fg_layer_decode_sliced(const fg_layer_config *c, const fg_layer_weights *w, const fg_kv_cache *kv,
+                                 const fg_half *x_in, fg_half *x_out, const int32_t *positions, int num_gpu_batches,
+                                 int gpu_batch_size, void *workspace, size_t workspace_bytes, cudaStream_t st,
+                                 const fg_layer_slices *sl) {
+  fg_status rc = check_common(c, w, kv, x_in, x_out, positions, num_gpu_batches, gpu_batch_size);
+  if (rc != FG_OK || kv->num_seqs == 0) return rc;
+  if (!workspace || !fg_aligned16(workspace)) return FG_ERR_INVALID;
+  return run_layer(c, w, kv, x_in, x_out, positions, kv->num_seqs, 1, static_cast<uint8_t *>(workspace),
+                   workspace_bytes, st, sl);
+}
+
+// Byte ranges of the layer blob's slices, in the order a layer step reads them: [0] the vectors,
+// [1] wqkv, [2] wo, [3] w1, [4] w2 (begin[i] .. end[i]).
+fg_status fg_layer_blob_slices(const fg_layer_config *c, size_t begin[5], size_t end[5]) {
+  if (!config_ok(c)) return FG_ERR_UNSUPPORTED;
+  const BlobLayout L = blob_layout(c);
+  begin[0] = L.vec[0];
+  end[0] = L.total;
+  for (int i = 0; i < 4; i++) {
+    begin[1 + i] = L.off[i][0];
+    end[1 + i] = i < 3 ? L.off[i + 1][0] : L.vec[0];
+  }
+  return FG_OK;
 }
 
 extern "C" fg_status fg_layer_prefill(const fg_layer_config *c, const fg_layer_weights *w, const fg_kv_cache *kv,

@@ -49,10 +49,10 @@ extern "C" fg_status fg_layer_decode_noalloc(const fg_layer_config *c, const fg_
   if (num_gpu_batches < 0 || gpu_batch_size < 0) return FG_ERR_INVALID;
   const int64_t rows = static_cast<int64_t>(num_gpu_batches) * gpu_batch_size;
   if (rows > INT_MAX) return FG_ERR_SHAPE;
-  // the activations must fit; the GEMMs use the rest for their optional split-k scratch
-  const size_t need = fg_layer_ws_required(c, static_cast<int>(rows));
-  if (need == 0 && rows > 0) return FG_ERR_UNSUPPORTED;
-  if (need > FG_NOALLOC_SCRATCH_BYTES) return FG_ERR_WORKSPACE;
+  // the whole layer workspace must fit (activations and the GEMMs' scratch), so the GEMMs take
+  // the same launches as fg_layer_decode given its full workspace: the same bits
+  if (rows > 0 && fg_layer_ws_required(c, static_cast<int>(rows)) == 0) return FG_ERR_UNSUPPORTED;
+  if (fg_layer_workspace_bytes(c, static_cast<int>(rows)) > FG_NOALLOC_SCRATCH_BYTES) return FG_ERR_WORKSPACE;
   void *scratch = nullptr;
   fg_status rc = scratch_address(&scratch);
   if (rc != FG_OK) return rc;

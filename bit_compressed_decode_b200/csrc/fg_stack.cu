@@ -4,9 +4,13 @@
 // weights sit in CPU memory and move to the GPU layer by layer; a loaded layer is used
 // for every batch of the block before the next one.  Here two device staging buffers
 // alternate: while layer l computes from buffer l%2 on the compute stream, the copy
-// stream moves layer l+1's blob into the other buffer with one cudaMemcpyAsync.  Two
-// events per buffer order the streams: `ready` (copy done -> compute may start) and
-// `done` (compute done -> the buffer may be overwritten).  For caches larger than HBM
+// stream moves layer l+1's blob into the other buffer.  The blob moves in slices, in the
+// order a layer step reads them -- its vectors, wqkv, wo, w1, w2 -- with one pair of events
+// per slice and buffer: `ready` (slice copied -> the kernels that read it may run) and
+// `done` (those kernels enqueued before it -> the slice may be overwritten).  So a layer's
+// QKV GEMM starts once wqkv has landed while wo, w1 and w2 are still crossing the link
+// (the weight loader that slices weights across batches, TightLLM abstract; the
+// fine-grained offloading pipeline of PIPO, abstract).  For caches larger than HBM
 // (a 175B-class stack), fg_stack_decode_host_kv keeps every layer's 4-bit KV cache in
 // pinned host memory too: the copy stream fills a device KV staging cache with the layer's
 // cached positions next to its blob, and writes only the new token slots back after the
@@ -23,13 +27,25 @@ struct fg_stack {
   int num_layers;
   std::vector<void *> host;
   void *staging[2];
-  cudaEvent_t ready[2], done[2];
-  cudaEvent_t kv_back[2];  // host-KV decode: write-back from KV staging cache b done
+  // per staging buffer: the layer-step slice events (see fg_layer_slices; entry 2 is the
+  // host-KV staging cache), and the host-KV write-back from KV staging cache b
+  fg_layer_slices ev[2];
+  cudaEvent_t kv_back[2];
+  size_t sbegin[5], send[5];  // blob slices: vectors, wqkv, wo, w1, w2
   size_t blob_bytes;
   int inject_failures;
 };
 
 namespace {
+
+// layer-step event index of blob slice i (vectors, wqkv, wo, w1, w2)
+constexpr int kSliceEvent[5] = {0, 1, 3, 4, 5};
+
+// Copies layer l's blob into staging buffer l % 2, slice by slice, on the copy stream: each
+// slice waits until the layer that used the buffer before is done with it.  With a KV fill
+// (host-KV decode), the fill goes after wqkv, before wo.
+fg_status prefetch_sliced(fg_stack *st, int l, cudaStream_t ps, const fg_kv_cache *fill_dst,
+                          const fg_kv_cache *fill_src, int fill_len);
 
 fg_status stack_run(fg_stack *st, const fg_kv_cache *kv, const fg_half *x_in, fg_half *x_out,
                     const int32_t *positions, int prompt_len, int nb, int gbs, void *workspace, size_t ws_bytes,
@@ -47,35 +63,27 @@ fg_status stack_run(fg_stack *st, const fg_kv_cache *kv, const fg_half *x_in, fg
   void *lws = ws + 2 * act;
   const size_t lws_bytes = ws_bytes - 2 * act;
 
-  fg_status rc = FG_OK;
-  auto prefetch = [&](int l) -> fg_status {
-    const int b = l & 1;
-    if (st->inject_failures > 0) {
-      st->inject_failures--;
-      return FG_ERR_CUDA;
-    }
-    fg_status r = fg_cuda_check(cudaStreamWaitEvent(ps, st->done[b], 0));
-    if (r != FG_OK) return r;
-    r = fg_cuda_check(cudaMemcpyAsync(st->staging[b], st->host[l], st->blob_bytes, cudaMemcpyHostToDevice, ps));
-    if (r != FG_OK) return r;
-    return fg_cuda_check(cudaEventRecord(st->ready[b], ps));
-  };
-
-  rc = prefetch(0);
+  fg_status rc = prefetch_sliced(st, 0, ps, nullptr, nullptr, 0);
   for (int l = 0; rc == FG_OK && l < st->num_layers; l++) {
     const int b = l & 1;
-    if (l + 1 < st->num_layers && (rc = prefetch(l + 1)) != FG_OK) break;
-    if ((rc = fg_cuda_check(cudaStreamWaitEvent(cs, st->ready[b], 0))) != FG_OK) break;
+    if (l + 1 < st->num_layers && (rc = prefetch_sliced(st, l + 1, ps, nullptr, nullptr, 0)) != FG_OK) break;
     fg_layer_weights w;
     if ((rc = fg_layer_weights_from_blob(&st->cfg, st->staging[b], &w)) != FG_OK) break;
     const fg_half *in = l == 0 ? x_in : buf[(l - 1) & 1];
     fg_half *out = l == st->num_layers - 1 ? x_out : buf[l & 1];
-    if (prompt_len > 0)
-      rc = fg_layer_prefill(&st->cfg, &w, &kv[l], in, out, positions, prompt_len, nb, gbs, lws, lws_bytes, cs);
-    else
-      rc = fg_layer_decode(&st->cfg, &w, &kv[l], in, out, positions, nb, gbs, lws, lws_bytes, cs);
-    if (rc != FG_OK) break;
-    if ((rc = fg_cuda_check(cudaEventRecord(st->done[b], cs))) != FG_OK) break;
+    if (prompt_len > 0) {
+      // a prompt step waits for the whole blob (its chunks reuse every slice), then frees it
+      for (int i = 0; i < 6 && rc == FG_OK; i++)
+        if (st->ev[b].ready[i] && i != 2) rc = fg_cuda_check(cudaStreamWaitEvent(cs, st->ev[b].ready[i], 0));
+      if (rc == FG_OK)
+        rc = fg_layer_prefill(&st->cfg, &w, &kv[l], in, out, positions, prompt_len, nb, gbs, lws, lws_bytes, cs);
+      for (int i = 0; i < 6 && rc == FG_OK; i++)
+        if (i != 2) rc = fg_cuda_check(cudaEventRecord(st->ev[b].done[i], cs));
+    } else {
+      fg_layer_slices sl = st->ev[b];
+      sl.ready[2] = sl.done[2] = nullptr;  // the cache is resident
+      rc = fg_layer_decode_sliced(&st->cfg, &w, &kv[l], in, out, positions, nb, gbs, lws, lws_bytes, cs, &sl);
+    }
   }
   if (rc != FG_OK) {
     // drain what was enqueued so nothing is left waiting on this stack's buffers
@@ -139,36 +147,21 @@ fg_status stack_run_host_kv(fg_stack *st, const fg_kv_cache *host_kv, const fg_k
   void *lws = ws + 2 * act;
   const size_t lws_bytes = ws_bytes - 2 * act;
 
-  fg_status rc = FG_OK;
-  auto prefetch = [&](int l) -> fg_status {
-    const int b = l & 1;
-    if (st->inject_failures > 0) {
-      st->inject_failures--;
-      return FG_ERR_CUDA;
-    }
-    fg_status r = fg_cuda_check(cudaStreamWaitEvent(ps, st->done[b], 0));
-    if (r == FG_OK) r = fg_cuda_check(cudaStreamWaitEvent(ps, st->kv_back[b], 0));
-    if (r == FG_OK)
-      r = fg_cuda_check(cudaMemcpyAsync(st->staging[b], st->host[l], st->blob_bytes, cudaMemcpyHostToDevice, ps));
-    if (r == FG_OK) r = kv_copy(dev_kv[b], host_kv[l], 0, fill_len, cudaMemcpyHostToDevice, ps);
-    if (r == FG_OK) r = fg_cuda_check(cudaEventRecord(st->ready[b], ps));
-    return r;
-  };
-
-  rc = prefetch(0);
+  fg_status rc = prefetch_sliced(st, 0, ps, &dev_kv[0], &host_kv[0], fill_len);
   for (int l = 0; rc == FG_OK && l < st->num_layers; l++) {
     const int b = l & 1;
-    if (l + 1 < st->num_layers && (rc = prefetch(l + 1)) != FG_OK) break;
-    if ((rc = fg_cuda_check(cudaStreamWaitEvent(cs, st->ready[b], 0))) != FG_OK) break;
+    if (l + 1 < st->num_layers &&
+        (rc = prefetch_sliced(st, l + 1, ps, &dev_kv[(l + 1) & 1], &host_kv[l + 1], fill_len)) != FG_OK)
+      break;
     fg_layer_weights w;
     if ((rc = fg_layer_weights_from_blob(&st->cfg, st->staging[b], &w)) != FG_OK) break;
     const fg_half *in = l == 0 ? x_in : buf[(l - 1) & 1];
     fg_half *out = l == st->num_layers - 1 ? x_out : buf[l & 1];
-    if ((rc = fg_layer_decode(&st->cfg, &w, &dev_kv[b], in, out, positions, nb, gbs, lws, lws_bytes, cs)) != FG_OK)
+    if ((rc = fg_layer_decode_sliced(&st->cfg, &w, &dev_kv[b], in, out, positions, nb, gbs, lws, lws_bytes, cs,
+                                     &st->ev[b])) != FG_OK)
       break;
-    if ((rc = fg_cuda_check(cudaEventRecord(st->done[b], cs))) != FG_OK) break;
-    // write the new slots back to the host cache, after the layer, on the copy stream
-    if ((rc = fg_cuda_check(cudaStreamWaitEvent(ps, st->done[b], 0))) != FG_OK) break;
+    // write the new slots back to the host cache once the layer's attention is done, on the copy stream
+    if ((rc = fg_cuda_check(cudaStreamWaitEvent(ps, st->ev[b].done[2], 0))) != FG_OK) break;
     if ((rc = kv_copy(host_kv[l], dev_kv[b], wb_begin, wb_end, cudaMemcpyDeviceToHost, ps)) != FG_OK) break;
     if ((rc = fg_cuda_check(cudaEventRecord(st->kv_back[b], ps))) != FG_OK) break;
   }
@@ -179,6 +172,37 @@ fg_status stack_run_host_kv(fg_stack *st, const fg_kv_cache *host_kv, const fg_k
     cudaStreamSynchronize(cs);
   }
   return rc;
+}
+
+fg_status prefetch_sliced(fg_stack *st, int l, cudaStream_t ps, const fg_kv_cache *fill_dst,
+                          const fg_kv_cache *fill_src, int fill_len) {
+  const int b = l & 1;
+  if (st->inject_failures > 0) {
+    st->inject_failures--;
+    return FG_ERR_CUDA;
+  }
+  uint8_t *dst = static_cast<uint8_t *>(st->staging[b]);
+  const uint8_t *src = static_cast<const uint8_t *>(st->host[l]);
+  fg_layer_slices &ev = st->ev[b];
+  for (int i = 0; i < 5; i++) {
+    const int e = kSliceEvent[i];
+    fg_status r = fg_cuda_check(cudaStreamWaitEvent(ps, ev.done[e], 0));
+    if (r == FG_OK)
+      r = fg_cuda_check(cudaMemcpyAsync(dst + st->sbegin[i], src + st->sbegin[i], st->send[i] - st->sbegin[i],
+                                        cudaMemcpyHostToDevice, ps));
+    if (r == FG_OK) r = fg_cuda_check(cudaEventRecord(ev.ready[e], ps));
+    if (r != FG_OK) return r;
+    if (i == 1 && fill_dst) {
+      // the layer's KV cache: after the previous layer on this staging cache is done with it
+      // (its attention) and has written its new slots back
+      r = fg_cuda_check(cudaStreamWaitEvent(ps, ev.done[2], 0));
+      if (r == FG_OK) r = fg_cuda_check(cudaStreamWaitEvent(ps, st->kv_back[b], 0));
+      if (r == FG_OK) r = kv_copy(*fill_dst, *fill_src, 0, fill_len, cudaMemcpyHostToDevice, ps);
+      if (r == FG_OK) r = fg_cuda_check(cudaEventRecord(ev.ready[2], ps));
+      if (r != FG_OK) return r;
+    }
+  }
+  return FG_OK;
 }
 
 }  // namespace
@@ -203,13 +227,17 @@ extern "C" fg_status fg_stack_create(const fg_layer_config *c, int num_layers, v
   st->staging[1] = dev_staging1;
   st->blob_bytes = bytes;
   st->inject_failures = 0;
+  fg_layer_blob_slices(c, st->sbegin, st->send);
   for (int i = 0; i < 2; i++) {
-    st->ready[i] = st->done[i] = st->kv_back[i] = nullptr;
+    st->kv_back[i] = nullptr;
+    for (int e = 0; e < 6; e++) st->ev[i].ready[e] = st->ev[i].done[e] = nullptr;
   }
   for (int i = 0; i < 2; i++) {
-    if (fg_cuda_check(cudaEventCreateWithFlags(&st->ready[i], cudaEventDisableTiming)) != FG_OK ||
-        fg_cuda_check(cudaEventCreateWithFlags(&st->done[i], cudaEventDisableTiming)) != FG_OK ||
-        fg_cuda_check(cudaEventCreateWithFlags(&st->kv_back[i], cudaEventDisableTiming)) != FG_OK) {
+    bool ok = fg_cuda_check(cudaEventCreateWithFlags(&st->kv_back[i], cudaEventDisableTiming)) == FG_OK;
+    for (int e = 0; ok && e < 6; e++)
+      ok = fg_cuda_check(cudaEventCreateWithFlags(&st->ev[i].ready[e], cudaEventDisableTiming)) == FG_OK &&
+           fg_cuda_check(cudaEventCreateWithFlags(&st->ev[i].done[e], cudaEventDisableTiming)) == FG_OK;
+    if (!ok) {
       fg_stack_destroy(st);
       return FG_ERR_CUDA;
     }
@@ -255,8 +283,10 @@ extern "C" fg_status fg_stack_inject_copy_failure(fg_stack *st, int count) {
 extern "C" fg_status fg_stack_destroy(fg_stack *st) {
   if (!st) return FG_ERR_INVALID;
   for (int i = 0; i < 2; i++) {
-    if (st->ready[i]) cudaEventDestroy(st->ready[i]);
-    if (st->done[i]) cudaEventDestroy(st->done[i]);
+    for (int e = 0; e < 6; e++) {
+      if (st->ev[i].ready[e]) cudaEventDestroy(st->ev[i].ready[e]);
+      if (st->ev[i].done[e]) cudaEventDestroy(st->ev[i].done[e]);
+    }
     if (st->kv_back[i]) cudaEventDestroy(st->kv_back[i]);
   }
   delete st;

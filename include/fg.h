@@ -119,11 +119,11 @@ FG_API fg_status fg_dequantize(const fg_qtensor *q, fg_half *y, void *stream);
 /* ---------------------------------------------------------------------- */
 
 /* For sequence s, head h, position p the head_dim values of k (and of v) are
- * quantised in groups of 64 along head_dim:
+ * quantised in groups of G = 64 or 128 along head_dim ([G3]):
  *   k_codes  uint8 [num_seqs][num_heads][max_len][head_dim/2]
- *   k_mins, k_scales fp16 [num_seqs][num_heads][max_len][head_dim/64]
+ *   k_mins, k_scales fp16 [num_seqs][num_heads][max_len][head_dim/G]
  * and the same for v.  Device memory, caller-owned.
- * Requirements: head_dim in {64, 128, 256}; max_len % 64 == 0. */
+ * Requirements: head_dim in {64, 128, 256}, a multiple of G; max_len % 64 == 0. */
 typedef struct {
     uint8_t *k_codes;
     fg_half *k_mins;
@@ -135,10 +135,11 @@ typedef struct {
     int32_t num_heads;
     int32_t head_dim;
     int32_t max_len;
+    int32_t group;       /* G: 64 or 128 (0 = 64) */
 } fg_kv_cache;
 
-/* Byte sizes of one codes array and of one mins/scales array. */
-FG_API fg_status fg_kv_cache_bytes(int num_seqs, int num_heads, int head_dim, int max_len,
+/* Byte sizes of one codes array and of one mins/scales array (group 0 = 64). */
+FG_API fg_status fg_kv_cache_bytes(int num_seqs, int num_heads, int head_dim, int max_len, int group,
                             size_t *codes_bytes, size_t *meta_bytes);
 
 /* Quantise and append new k, v rows.  k, v: fp16 device rows, row r at
@@ -165,8 +166,9 @@ FG_API fg_status fg_attention_decode(const fg_kv_cache *kv, const fg_half *q, in
 /* ---------------------------------------------------------------------- */
 
 enum {
-    FG_EPI_RELU = 1,      /* y = max(0, .) after the bias (and q-scale) */
-    FG_EPI_RESIDUAL = 2,  /* y += residual[m][n] after the activation */
+    FG_EPI_RELU = 1,         /* y = max(0, .) after the bias (and q-scale) */
+    FG_EPI_RESIDUAL = 2,     /* y += residual[m][n] after the activation */
+    FG_GEMM_PERSISTENT = 4,  /* M > 256: take the persistent launch (see below) */
 };
 
 /* y[m][n] = epi( sum_k x[m][k] * deq(w)[n][k] + bias[n] ), fp32 accumulation,
@@ -176,22 +178,33 @@ enum {
  * multiplied by qscale after the bias.  w->group 64 or 128 with K % group == 0,
  * N % 128 == 0; x, y, the
  * codes and the residual 16-byte aligned (FG_ERR_INVALID otherwise).
- * workspace: optional device scratch (16-byte aligned) of
- * fg_linear_workspace_bytes(M, N, K) bytes, 0 when the GEMM does not split its
- * k-range.  With it the partial sums of a split k-range are added through it
- * (they stay in L2); with less, or NULL, they are added on chip over
- * distributed shared memory.  Both add the splits in the same order, so the
- * result is the same bit for bit.
  * Tensor cores dequantise W tiles in shared memory ([G3]: on-the-fly
- * dequantisation for FP16 compute). */
+ * dequantisation for FP16 compute).
+ * Launches (see fg_linear_plan): M <= 256 runs one SM per output tile; larger M
+ * runs on CTA pairs: the classic launch (one pair per tile, k-range optionally
+ * split over a cluster), or, with FG_GEMM_PERSISTENT in flags, the persistent
+ * launch (every resident pair takes an equal share of the tiles' k-iterations; a
+ * tile shared between pairs is finished by the pair holding its first
+ * k-segment).  The layer calls use the classic launch.
+ * workspace: optional device scratch (16-byte aligned).  The classic launch's
+ * split k-range adds its partial sums through the scratch when it holds
+ * n_tiles * t_tiles * splits * tile_tokens * 256 * 4 bytes (n_tiles =
+ * ceil(N / 256), t_tiles = ceil(M / tile_tokens)), else over distributed shared
+ * memory; the two add the splits in the same order, so their results are the
+ * same bit for bit.  The persistent launch needs fg_linear_workspace_bytes(M, N,
+ * K) bytes (its shared tiles' partial sums) and falls back to the classic launch
+ * with less; it adds partial sums in another order, so its results may differ
+ * from the classic launch's in the last bits (each is deterministic). */
 FG_API size_t fg_linear_workspace_bytes(int M, int N, int K);
-/* The launch fg_linear_w4a16 makes for this shape on the current device (no
- * launch): *tile_tokens = tokens per output tile (16..256 for M <= 256, one SM
- * per tile; 256 or 512 for larger M, a CTA pair per tile), *splits = CTAs
- * sharing each tile's k-range (1..8 one-SM, 1..4 pair).  Chosen by a time
- * model of the kernels: waves of resident clusters x k-tiles per CTA, plus the
- * pipeline fill and the epilogue. */
-FG_API fg_status fg_linear_plan(int M, int N, int K, int *tile_tokens, int *splits);
+/* The launches fg_linear_w4a16 makes for this shape on the current device (no
+ * launch): the classic launch's *tile_tokens = tokens per output tile (16..256
+ * for M <= 256, one SM per tile; 256 or 512 for larger M, a CTA pair per tile)
+ * and *splits = CTAs sharing each tile's k-range (1..8 one-SM, 1..4 pair),
+ * chosen by a time model of the kernels: waves of resident clusters x k-tiles
+ * per CTA, plus the pipeline fill and the epilogue; *pairs = CTA pairs of the
+ * persistent launch (512-token tiles) that FG_GEMM_PERSISTENT would take, 0
+ * where it is not available (M <= 256, or tiles split too finely). */
+FG_API fg_status fg_linear_plan(int M, int N, int K, int *tile_tokens, int *splits, int *pairs);
 FG_API fg_status fg_linear_w4a16(const fg_half *x, int M, int K, const fg_qtensor *w, const fg_half *bias,
                           const fg_half *residual, int flags, int qscale_cols, float qscale,
                           fg_half *y, void *workspace, size_t workspace_bytes, void *stream);
@@ -212,12 +225,14 @@ typedef struct {
     int32_t head_dim;   /* 64, 128 or 256 */
     int32_t ffn;        /* F, multiple of 128 */
     float ln_eps;       /* 1e-5 for OPT */
+    int32_t group;      /* 4-bit group of the weights and the KV cache: 64 or 128 (0 = 64) [G3] */
 } fg_layer_config;
 
 /* Compressed weights of one layer.  Matrices are packed along their input
- * dim (dim 1): wqkv [3h][h] (rows: q, then k, then v, each head-major),
- * wo [h][h], w1 [F][h], w2 [h][F].  Vectors fp16: bqkv [3h], bo [h], b1 [F],
- * b2 [h], ln1_g/ln1_b/ln2_g/ln2_b [h].  All device pointers. */
+ * dim (dim 1) in groups of the config's group: wqkv [3h][h] (rows: q, then k,
+ * then v, each head-major), wo [h][h], w1 [F][h], w2 [h][F].  Vectors fp16:
+ * bqkv [3h], bo [h], b1 [F], b2 [h], ln1_g/ln1_b/ln2_g/ln2_b [h].  All device
+ * pointers. */
 typedef struct {
     fg_qtensor wqkv, wo, w1, w2;
     fg_half *bqkv, *bo, *b1, *b2;
@@ -234,9 +249,10 @@ FG_API fg_status fg_layer_weights_from_blob(const fg_layer_config *c, void *blob
 
 /* Device scratch for fg_layer_decode / fg_layer_prefill over `rows`
  * hidden-state rows (the block's sequences, or sequences * prompt length):
- * the intermediate activations, then the GEMMs' optional split-k scratch
- * (fg_linear_w4a16).  A call needs at least the activations' part and gives
- * the GEMMs whatever follows it. */
+ * the intermediate activations, then the GEMMs' scratch (fg_linear_w4a16).
+ * A call needs at least the activations' part and gives the GEMMs whatever
+ * follows it; the GEMMs add split k-ranges on chip when it is short, with the
+ * same bits. */
 FG_API size_t fg_layer_workspace_bytes(const fg_layer_config *c, int rows);
 
 /* One decode step of one layer for every sequence of a block of
@@ -250,7 +266,8 @@ FG_API size_t fg_layer_workspace_bytes(const fg_layer_config *c, int rows);
  * Steps: a = LN1(x); [q k v] = a Wqkv^T + bqkv, q *= head_dim^-1/2;
  * append k, v to the 4-bit cache at positions; o = attention over positions
  * 0..pos; h1 = x + o Wo^T + bo; x_out = h1 + relu(LN2(h1) W1^T + b1) W2^T + b2.
- * kv->num_seqs must equal S.  Positions are not advanced by the call. */
+ * kv->num_seqs must equal S and kv->group the config's group.  Positions are
+ * not advanced by the call. */
 FG_API fg_status fg_layer_decode(const fg_layer_config *c, const fg_layer_weights *w, const fg_kv_cache *kv,
                           const fg_half *x_in, fg_half *x_out, const int32_t *positions,
                           int num_gpu_batches, int gpu_batch_size,
@@ -268,14 +285,13 @@ FG_API fg_status fg_layer_prefill(const fg_layer_config *c, const fg_layer_weigh
  * process that reserved all device memory up front, a host that only passes
  * pointers it already owns, or a loop that must not allocate between steps.
  * (The pages have no counterpart: this is a deployment convenience.)  The step's
- * scratch lives in a static device array of FG_NOALLOC_SCRATCH_BYTES that every
- * GPU loading the library holds until the process exits; the caller still
- * passes weights, cache, inputs and outputs, as for fg_layer_decode, whose
- * computation this is.
- *   - Returns FG_ERR_WORKSPACE when the block's activations need more scratch
- *     than that, before any launch (fg_layer_workspace_bytes(c, S) above
- *     FG_NOALLOC_SCRATCH_BYTES only by the GEMMs' split-k scratch is fine: the
- *     GEMMs then add their partial sums on chip, with the same bits);
+ * scratch lives in a static device array of FG_NOALLOC_SCRATCH_BYTES (96 MiB)
+ * that every GPU loading the library holds until the process exits; the caller
+ * still passes weights, cache, inputs and outputs, as for fg_layer_decode, whose
+ * computation this is, bit for bit.
+ *   - Returns FG_ERR_WORKSPACE, before any launch, when the block's whole
+ *     workspace, fg_layer_workspace_bytes(c, S), exceeds the array (the
+ *     OPT-6.7B-shaped block of 512 sequences needs about 78 MB);
  *     FG_ERR_SHAPE when num_gpu_batches * gpu_batch_size exceeds INT_MAX.
  *   - Set-up: the first call on each device looks up the array's device
  *     address with that device current.  Under CUDA's lazy module loading (the
@@ -290,7 +306,7 @@ FG_API fg_status fg_layer_prefill(const fg_layer_config *c, const fg_layer_weigh
  *     race on it: serialise them.
  *   - After that first call it allocates nothing (keep fg_profile_enable off:
  *     profiling creates events). */
-#define FG_NOALLOC_SCRATCH_BYTES (48u << 20)
+#define FG_NOALLOC_SCRATCH_BYTES (96u << 20)
 FG_API fg_status fg_layer_decode_noalloc(const fg_layer_config *c, const fg_layer_weights *w,
                                          const fg_kv_cache *kv, const fg_half *x_in, fg_half *x_out,
                                          const int32_t *positions, int num_gpu_batches, int gpu_batch_size,
