@@ -78,10 +78,17 @@ def test_quantize_validates_before_launch():
 
 def test_kv_cache_bytes_rules():
     cb, mb = ctypes.c_size_t(), ctypes.c_size_t()
-    assert _rc("fg_kv_cache_bytes", 512, 32, 128, 576, ctypes.byref(cb), ctypes.byref(mb)) == 0
+    assert _rc("fg_kv_cache_bytes", 512, 32, 128, 576, 64, ctypes.byref(cb), ctypes.byref(mb)) == 0
     assert cb.value == 512 * 32 * 576 * 64 and mb.value == 512 * 32 * 576 * 2 * 2
-    assert _rc("fg_kv_cache_bytes", 4, 12, 96, 64, ctypes.byref(cb), ctypes.byref(mb)) == 3     # head_dim
-    assert _rc("fg_kv_cache_bytes", 4, 12, 64, 100, ctypes.byref(cb), ctypes.byref(mb)) == 2    # max_len % 64
+    assert _rc("fg_kv_cache_bytes", 512, 32, 128, 576, 0, ctypes.byref(cb), ctypes.byref(mb)) == 0   # 0 = 64
+    assert mb.value == 512 * 32 * 576 * 2 * 2
+    # groups of 128 along head_dim ("FlexGen Guide", section 3: groups of 64 or 128)
+    assert _rc("fg_kv_cache_bytes", 512, 32, 128, 576, 128, ctypes.byref(cb), ctypes.byref(mb)) == 0
+    assert cb.value == 512 * 32 * 576 * 64 and mb.value == 512 * 32 * 576 * 1 * 2
+    assert _rc("fg_kv_cache_bytes", 4, 12, 64, 64, 128, ctypes.byref(cb), ctypes.byref(mb)) == 2    # G > head_dim
+    assert _rc("fg_kv_cache_bytes", 4, 12, 64, 64, 32, ctypes.byref(cb), ctypes.byref(mb)) == 3     # group 32
+    assert _rc("fg_kv_cache_bytes", 4, 12, 96, 64, 64, ctypes.byref(cb), ctypes.byref(mb)) == 3     # head_dim
+    assert _rc("fg_kv_cache_bytes", 4, 12, 64, 100, 64, ctypes.byref(cb), ctypes.byref(mb)) == 2    # max_len % 64
 
 
 def _align(x, a=256):
@@ -118,6 +125,26 @@ def test_layer_blob_layout(h, H, F):
     assert spans[-1][0] + spans[-1][1] <= base + want
 
 
+def test_layer_blob_layout_group128():
+    # groups of 128: the same codes, half the metadata of groups of 64
+    h, H, F = 4096, 32, 16384
+    c64, c128 = fg.LayerConfig(h, H, F), fg.LayerConfig(h, H, F, group=128)
+    want = 0
+    for n, k in ((3 * h, h), (h, h), (F, h), (h, F)):
+        want += _align(n * k // 2) + 2 * _align(n * k // 128 * 2)
+    for n in (3 * h, h, F, h, h, h, h, h):
+        want += _align(2 * n)
+    assert c128.blob_bytes() == want < c64.blob_bytes()
+    blob = np.zeros(want + 256, dtype=np.uint8)
+    base = (blob.ctypes.data + 255) // 256 * 256
+    w = B.fg_layer_weights()
+    c = c128.struct()
+    assert _rc("fg_layer_weights_from_blob", ctypes.byref(c), ctypes.c_void_p(base), ctypes.byref(w)) == 0
+    assert w.wqkv.group == w.w2.group == 128
+    bad = fg.LayerConfig(768, 12, 3072, group=128).struct()  # head_dim 64 cannot hold a group of 128
+    assert B.lib().fg_layer_blob_bytes(ctypes.byref(bad)) == 0
+
+
 def test_opt6p7b_sizes():
     cfg = fg.LayerConfig(4096, 32, 16384)
     # 12 h^2 parameters at 4.5 bits (codes + fp16 min and scale per 64): 113.2 MB + vectors
@@ -130,7 +157,7 @@ def test_opt6p7b_sizes():
 
 
 def test_layer_entry_points_validate_config():
-    bad = B.fg_layer_config(4096, 32, 100, 16384, 1e-5)     # head_dim inconsistent
+    bad = B.fg_layer_config(4096, 32, 100, 16384, 1e-5, 64)     # head_dim inconsistent
     assert B.lib().fg_layer_blob_bytes(ctypes.byref(bad)) == 0
     w = B.fg_layer_weights()
     kv = B.fg_kv_cache()
@@ -144,9 +171,9 @@ def test_noalloc_rejects_oversized_block_on_host():
     c = cfg.struct()
     w = B.fg_layer_weights()
     kv = B.fg_kv_cache()
-    assert cfg.workspace_bytes(1024) > fg.NOALLOC_SCRATCH_BYTES
+    assert cfg.workspace_bytes(2048) > fg.NOALLOC_SCRATCH_BYTES
     rc = _rc("fg_layer_decode_noalloc", ctypes.byref(c), ctypes.byref(w), ctypes.byref(kv), None, None, None, 1,
-             1024, None)
+             2048, None)
     assert rc == 7                                          # FG_ERR_WORKSPACE, before any CUDA call
 
 

@@ -191,6 +191,44 @@ def test_kv_append_bit_exact(H, d):
         assert np.array_equal(u16(host(a)) if a.dtype == torch.float16 else host(a), b)
 
 
+@pytest.mark.parametrize("H,d", [(3, 128), (2, 256)])
+def test_kv_append_group128_bit_exact(H, d):
+    # head_dim quantised in groups of 128 ("FlexGen Guide", section 3: groups of 64 or 128)
+    S, maxL = 4, 128
+    g = fg.KVCache(S, H, d, maxL, group=128)
+    o = oracle.KVCache(S, H, d, maxL, group=128)
+    pos = np.array([0, 63, 64, 127], dtype=np.int32)
+    k = si.normal_f16(26, 1, (S, 3 * H * d), 1.0)
+    kd = dev(k)
+    fg.fg_kv_append(g, kd[:, H * d:], kd[:, 2 * H * d:], dev(pos), ld=3 * H * d)
+    oracle.kv_append(o, k[:, H * d:2 * H * d], k[:, 2 * H * d:], np.arange(S), pos)
+    fg.fg_sync_status()
+    for a, b in zip(g.arrays(), o.arrays()):
+        assert np.array_equal(u16(host(a)) if a.dtype == torch.float16 else host(a), b)
+
+
+@pytest.mark.parametrize("H,d,P", [(2, 128, 1), (2, 256, 1), (3, 128, 90)])
+def test_attention_group128_matches_oracle(H, d, P):
+    # decode rows (P = 1) through the row kernel, prompt rows through the tiled prefill kernel
+    # (head_dim 128), the cache in groups of 128 along head_dim
+    S = 3
+    starts = np.array([0, 70, 200], dtype=np.int32)
+    lens = starts + P
+    maxL = int((lens.max() + 63) // 64 * 64)
+    o, g = _cache_pair(S, H, d, maxL, lens, seed=27, group=128)
+    _garbage_past(g, lens, 28)
+    q = (si.normal_f16(27, 1, (S * P, H * d), 1.0).astype(np.float32) / np.sqrt(d)).astype(np.float16)
+    out = fg.fg_attention_decode(g, dev(q), dev(starts), rows_per_seq=P)
+    fg.fg_sync_status()
+    seq = np.repeat(np.arange(S), P)
+    ref = oracle.attention(o, q, seq, starts[seq] + np.tile(np.arange(P), S) + 1)
+    got = host(out).astype(np.float64)
+    for h in range(H):
+        sl = slice(h * d, (h + 1) * d)
+        err = np.max(np.abs(got[:, sl] - ref[:, sl]), axis=1)
+        assert np.all(err <= 2e-3 * np.max(np.abs(ref[:, sl]), axis=1) + 1e-4), (h, err.max())
+
+
 def test_kv_append_prompt_rows_and_range_error():
     S, H, d, maxL, P = 3, 2, 128, 64, 10
     g = fg.KVCache(S, H, d, maxL)
@@ -212,15 +250,15 @@ def test_kv_append_prompt_rows_and_range_error():
 
 # ------------------------------------------------------------------ attention ---------
 
-def _cache_pair(S, H, d, maxL, lens, seed):
-    o = oracle.KVCache(S, H, d, maxL)
+def _cache_pair(S, H, d, maxL, lens, seed, group=64):
+    o = oracle.KVCache(S, H, d, maxL, group=group)
     for s in range(S):
         L = lens[s]
         k = si.normal_f16(seed, 100 + s, (L, H * d), 1.0)
         v = si.normal_f16(seed, 200 + s, (L, H * d), 1.0)
         oracle.kv_append(o, k, v, np.full(L, s), np.arange(L))
     arrays = [dev(a.view(np.float16) if a.dtype == np.uint16 else a) for a in o.arrays()]
-    return o, fg.KVCache(S, H, d, maxL, arrays=arrays)
+    return o, fg.KVCache(S, H, d, maxL, arrays=arrays, group=group)
 
 
 @pytest.mark.parametrize("H,d", [(4, 64), (3, 128), (2, 256)])
@@ -261,6 +299,74 @@ def test_attention_prompt_rows_causal():
     assert np.max(np.abs(host(out).astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref))
 
 
+def _garbage_past(g, lens, seed):
+    """Random bytes (NaN and inf metadata included) in every cache slot at or past each
+    sequence's length: attention must never let them reach its output."""
+    gen = torch.Generator(device="cuda").manual_seed(seed)
+    for a in g.arrays():
+        u8 = a.view(torch.uint8)
+        noise = torch.randint(0, 256, u8.shape, dtype=torch.uint8, device="cuda", generator=gen)
+        for s, L in enumerate(lens):
+            u8[s, :, L:] = noise[s, :, L:]
+
+
+@pytest.mark.parametrize("H,d,P", [(2, 128, 70), (3, 64, 130), (1, 128, 512), (2, 64, 17), (2, 256, 40)])
+def test_attention_prefill_tiles_match_oracle(H, d, P):
+    # prompt rows through the tiled prefill kernel (head_dim 64 / 128; 256 takes the row kernel):
+    # sequences that start at position 0 and sequences that continue an earlier prompt
+    # (positions 5 and 64), prompt lengths that end mid-tile, garbage in the slots past them
+    S = 3
+    starts = np.array([0, 5, 64], dtype=np.int32)
+    lens = starts + P
+    maxL = int((lens.max() + 63) // 64 * 64)
+    o, g = _cache_pair(S, H, d, maxL, lens, seed=30 + d)
+    _garbage_past(g, lens, 31)
+    q = (si.normal_f16(30, 1, (S * P, H * d), 1.0).astype(np.float32) / np.sqrt(d)).astype(np.float16)
+    out = fg.fg_attention_decode(g, dev(q), dev(starts), rows_per_seq=P)
+    fg.fg_sync_status()
+    seq = np.repeat(np.arange(S), P)
+    ref = oracle.attention(o, q, seq, starts[seq] + np.tile(np.arange(P), S) + 1)
+    got = host(out).astype(np.float64)
+    for h in range(H):
+        sl = slice(h * d, (h + 1) * d)
+        err = np.max(np.abs(got[:, sl] - ref[:, sl]), axis=1)
+        assert np.all(err <= 2e-3 * np.max(np.abs(ref[:, sl]), axis=1) + 1e-4), (h, err.max())
+
+
+@pytest.mark.parametrize("prompt", [False, True])
+def test_attention_mixed_token_magnitudes(prompt):
+    # K and V rows whose magnitudes span 1e-3 .. 1e1 from token to token (groups with very
+    # small and very large scales side by side, scores spread over hundreds of log units),
+    # through the decode and the prefill kernels.  The decode kernel multiplies fp16 operands
+    # without forming the dequantised fp16 K/V value (its p * scale operand is the fp16 one
+    # under test here), so it is held to the oracle's exact-dequantisation form; the prefill
+    # kernel dequantises to fp16 like the layer's reading and is held to that form.
+    S, H, d = 2, 2, 128
+    P = 96 if prompt else 1
+    lens = np.array([150, 200], dtype=np.int32) if not prompt else np.array([P, P + 40], dtype=np.int32)
+    maxL = 256
+    o = oracle.KVCache(S, H, d, maxL)
+    rng = np.random.default_rng(41)
+    for s in range(S):
+        L = int(lens[s])
+        mag = 10.0 ** rng.uniform(-3, 1, size=(L, 1))
+        k = (si.normal_f16(41, 100 + s, (L, H * d), 1.0).astype(np.float64) * mag).astype(np.float16)
+        v = (si.normal_f16(41, 200 + s, (L, H * d), 1.0).astype(np.float64) * mag).astype(np.float16)
+        oracle.kv_append(o, k, v, np.full(L, s), np.arange(L))
+    g = fg.KVCache(S, H, d, maxL, arrays=[dev(a.view(np.float16) if a.dtype == np.uint16 else a) for a in o.arrays()])
+    starts = lens - P
+    q = (si.normal_f16(41, 1, (S * P, H * d), 0.3).astype(np.float32)).astype(np.float16)
+    out = fg.fg_attention_decode(g, dev(q), dev(starts.astype(np.int32)), rows_per_seq=P)
+    fg.fg_sync_status()
+    seq = np.repeat(np.arange(S), P)
+    ref = oracle.attention(o, q, seq, starts[seq] + np.tile(np.arange(P), S) + 1, exact_dequant=not prompt)
+    got = host(out).astype(np.float64)
+    for h in range(H):
+        sl = slice(h * d, (h + 1) * d)
+        err = np.max(np.abs(got[:, sl] - ref[:, sl]), axis=1)
+        assert np.all(err <= 2e-3 * np.max(np.abs(ref[:, sl]), axis=1) + 1e-4), (h, err.max())
+
+
 # ------------------------------------------------------------------ linear -------------
 
 @pytest.mark.parametrize("M,N,K", [(1, 128, 64), (4, 256, 768), (16, 384, 128), (17, 256, 192), (100, 512, 1024),
@@ -274,10 +380,18 @@ def test_linear_matches_oracle(M, N, K):
     w16 = si.normal_f16(14, 2, (N, K), 0.02)
     b = si.normal_f16(14, 3, (N,), 0.1)
     wq = fg.fg_quantize(dev(w16), dim=1)
-    y = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b))
     ref = oracle.linear(x, oracle.quantize(w16, 1), bias=b)
-    err = np.max(np.abs(host(y).astype(np.float64) - ref))
-    assert err <= 2e-3 * np.max(np.abs(ref)), err
+    # the classic launch with its scratch; for M > 256 also without scratch (partial sums added
+    # on chip) and the persistent launch where it is available
+    runs = [dict()]
+    if M > 256:
+        runs.append(dict(workspace=torch.empty(16, dtype=torch.uint8, device="cuda")))
+        if fg.fg_linear_plan_pairs(M, N, K) > 0:
+            runs.append(dict(persistent=True))
+    for kw in runs:
+        y = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), **kw)
+        err = np.max(np.abs(host(y).astype(np.float64) - ref))
+        assert err <= 2e-3 * np.max(np.abs(ref)), (err, kw)
 
 
 @pytest.mark.parametrize("M,K", [(70, 256), (300, 256), (300, 2048)])
@@ -294,6 +408,35 @@ def test_linear_epilogues(M, K):
         y = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), **kw)
         ref = oracle.linear(x, wo, bias=b, **okw)
         assert np.max(np.abs(host(y).astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref)), kw
+
+
+def test_bounded_wait_timeout_is_reported_and_the_gpu_stays_usable():
+    # Failure detection without a GPU fault: one launch of the one-SM GEMM (a CTA on each of
+    # 148 SMs) whose dequantising warps withhold their first-stage arrival, with every pipeline
+    # wait limited to 50 ms.  The MMA issuer's wait gives up, the launch drains its copies,
+    # frees its tensor memory and flags FG_ERR_TIMEOUT; the same GEMM then runs normally on
+    # every SM and matches the oracle.
+    M, N, K = 16, 148 * 256, 512
+    x = si.normal_f16(23, 1, (M, K), 1.0)
+    w16 = si.normal_f16(23, 2, (N, K), 0.02)
+    wq = fg.fg_quantize(dev(w16), dim=1)
+    assert fg.fg_linear_plan(M, N, K) == (16, 1)
+    xd = dev(x)
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    fg.fg_sync_status()
+    fg.fg_test_gemm_stall(1, 50_000_000)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    fg.fg_linear_w4a16(xd, wq, out=y)
+    e1.record()
+    with pytest.raises(fg.FgError, match="TIMEOUT"):
+        fg.fg_sync_status()
+    assert 40.0 <= e0.elapsed_time(e1) < 1000.0          # gave up after about the 50 ms limit
+    fg.fg_sync_status()                                  # the error word was cleared
+    y = fg.fg_linear_w4a16(xd, wq, out=y)
+    fg.fg_sync_status()
+    ref = oracle.linear(x, oracle.quantize(w16, 1))
+    assert np.max(np.abs(host(y).astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref))
 
 
 def test_linear_permutation_weight_exact():
@@ -316,15 +459,20 @@ def test_linear_split_k_deterministic(M, N, K):
     y1 = fg.fg_linear_w4a16(x, wq)
     y2 = fg.fg_linear_w4a16(x, wq)
     assert torch.equal(y1, y2)
+    ref = oracle.linear(host(x), oracle.quantize(w16, 1))
+    assert np.max(np.abs(host(y1).astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref))
     if M <= 256:
         assert fg.fg_linear_workspace_bytes(M, N, K) == 0   # one-SM tiles add partials on chip
     else:
-        # CTA-pair tiles: through the scratch by default, on chip without one; same bits
+        # CTA pairs: the classic launch's split k-range through the scratch (L2) and on chip
+        # (no scratch) add the splits in the same order: the same bits
         assert fg.fg_linear_workspace_bytes(M, N, K) > 0
         y3 = fg.fg_linear_w4a16(x, wq, workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
         assert torch.equal(y1, y3)
-    ref = oracle.linear(host(x), oracle.quantize(w16, 1))
-    assert np.max(np.abs(host(y1).astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref))
+        cb = fg.fg_linear_classic_scratch_bytes(M, N, K)
+        if cb:
+            y4 = fg.fg_linear_w4a16(x, wq, workspace=torch.empty(cb, dtype=torch.uint8, device="cuda"))
+            assert torch.equal(y1, y4)
 
 
 @pytest.mark.parametrize("M,N,K", [(520, 4096, 4096), (600, 7680, 1024), (530, 5120, 1536), (512, 4096, 16384)])
@@ -342,16 +490,69 @@ def test_linear_split_k_residual_sampled(M, N, K):
     assert torch.equal(y1, y2)
     if K >= 4096:
         assert fg.fg_linear_workspace_bytes(M, N, K) > 0        # these shapes split the k-range
-    if fg.fg_linear_workspace_bytes(M, N, K):
-        # partial sums added through the scratch (above) or, with too little scratch, on chip
-        # over distributed shared memory: the same order of additions, the same bits
+    outs = [y1]
+    if fg.fg_linear_classic_scratch_bytes(M, N, K):
+        # partial sums through the scratch (above) or, with too little scratch, on chip over
+        # distributed shared memory: the same order of additions, the same bits
         y3 = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), residual=dev(r),
                                 workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
         assert torch.equal(y1, y3)
+    if fg.fg_linear_plan_pairs(M, N, K) > 0:
+        outs.append(fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), residual=dev(r), persistent=True))
     rows = np.unique(np.concatenate([np.random.default_rng(M).choice(M, 20, replace=False), [0, 255, 256, 511, M - 1]]))
     ref = oracle.linear(x[rows], oracle.quantize(w16, 1), bias=b, residual=r[rows])
+    for y in outs:
+        got = host(y)[rows].astype(np.float64)
+        assert np.max(np.abs(got - ref)) <= 2e-3 * np.max(np.abs(ref))
+
+
+@pytest.mark.parametrize("M,N,K,epi", [
+    (512, 12288, 4096, "qscale"),      # QKV of the OPT-6.7B block: 48 tiles over the pairs, split tiles
+    (512, 4096, 4096, "residual"),     # output projection: every tile split between several pairs
+    (512, 16384, 4096, "relu"),        # FC1
+    (512, 4096, 16384, "residual"),    # FC2: long k-ranges
+    (700, 12288, 4096, "relu"),        # a ragged second token tile
+    (513, 4224, 4096, "none"),         # a last feature pair holding 128 features, 2 token tiles
+    (4096, 2048, 1024, "residual"),    # many whole tiles per pair (a prompt-sized M)
+])
+def test_linear_persistent_launch_matches_oracle(M, N, K, epi):
+    # the persistent stream-K launch (FG_GEMM_PERSISTENT with the full scratch): whole tiles,
+    # split tiles finished by the pair holding their first k-segment, every epilogue;
+    # deterministic, and sampled rows against the oracle
+    assert fg.fg_linear_plan_pairs(M, N, K) > 0
+    x = si.normal_f16(24, 1, (M, K), 1.0)
+    w16 = si.normal_f16(24, 2, (N, K), 0.02)
+    b = si.normal_f16(24, 3, (N,), 0.1)
+    r = si.normal_f16(24, 4, (M, N), 1.0)
+    wq = fg.fg_quantize(dev(w16), dim=1)
+    kw = {"qscale": dict(qscale_cols=N // 3, qscale=0.125), "residual": dict(residual=dev(r)),
+          "relu": dict(relu=True), "none": {}}[epi]
+    okw = {"qscale": dict(qscale_cols=N // 3, qscale=0.125), "residual": dict(residual=r),
+           "relu": dict(relu=True), "none": {}}[epi]
+    y1 = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), persistent=True, **kw)
+    y2 = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), persistent=True, **kw)
+    fg.fg_sync_status()
+    assert torch.equal(y1, y2)
+    rows = np.unique(np.concatenate([np.random.default_rng(M + N).choice(M, 24, replace=False),
+                                     [0, 255, 256, 511, M - 1]]))
+    okw_rows = dict(okw)
+    if "residual" in okw_rows:
+        okw_rows["residual"] = r[rows]
+    ref = oracle.linear(x[rows], oracle.quantize(w16, 1), bias=b, **okw_rows)
     got = host(y1)[rows].astype(np.float64)
     assert np.max(np.abs(got - ref)) <= 2e-3 * np.max(np.abs(ref))
+
+
+def test_linear_persistent_launch_group128():
+    M, N, K = 512, 4096, 4096
+    assert fg.fg_linear_plan_pairs(M, N, K) > 0
+    x = si.normal_f16(25, 1, (M, K), 1.0)
+    w16 = si.normal_f16(25, 2, (N, K), 0.02)
+    wq = fg.fg_quantize(dev(w16), dim=1, group=128)
+    y = fg.fg_linear_w4a16(dev(x), wq, persistent=True)
+    rows = np.array([0, 100, 300, 511])
+    ref = oracle.linear(x[rows], oracle.quantize(w16, 1, group=128))
+    assert np.max(np.abs(host(y)[rows].astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref))
 
 
 def test_linear_errors():
