@@ -798,6 +798,23 @@ def run_kernel(args, wl):
         pos = torch.full((S,), P, dtype=torch.int32, device=dev)
         run = lambda: fg.fg_attention_decode(cache, qkv[:, :h], pos, out=out, stream=stream)
         work, unit, peak = S * H * (P + 1) * 2 * (d // 2 + 4 * ng) + 2 * S * h * 2, "GB/s", peaks["hbm"]
+    elif args.kernel == "prefill_attention":
+        # the prompts' attention of the prefill: S sequences x P prompt rows over a cache holding
+        # those P tokens (seeded codes), causal; 4 d flops per (row, head, visible key)
+        maxL = (P + 63) // 64 * 64
+        ng = d // 64
+        cache = fg.KVCache(S, H, d, maxL, device=dev, arrays=[
+            torch.randint(0, 256, (S, H, maxL, d // 2), generator=g, device=dev, dtype=torch.uint8),
+            torch.randn((S, H, maxL, ng), generator=g, device=dev, dtype=torch.float16),
+            (torch.rand((S, H, maxL, ng), generator=g, device=dev) * 0.2).half(),
+            torch.randint(0, 256, (S, H, maxL, d // 2), generator=g, device=dev, dtype=torch.uint8),
+            torch.randn((S, H, maxL, ng), generator=g, device=dev, dtype=torch.float16),
+            (torch.rand((S, H, maxL, ng), generator=g, device=dev) * 0.2).half()])
+        q = torch.randn((S * P, h), generator=g, device=dev, dtype=torch.float16) * 0.1
+        out = torch.empty((S * P, h), dtype=torch.float16, device=dev)
+        zero = torch.zeros((S,), dtype=torch.int32, device=dev)
+        run = lambda: fg.fg_attention_decode(cache, q, zero, rows_per_seq=P, out=out, stream=stream)
+        work, unit, peak = 4 * d * H * S * P * (P + 1) // 2, "TFLOP/s", peaks["tc_burst"]
     elif args.kernel.endswith("_gemm"):
         N, K = {"qkv_gemm": (3 * h, h), "out_gemm": (h, h), "fc1_gemm": (F, h), "fc2_gemm": (h, F)}[args.kernel]
         x = torch.randn((S, K), generator=g, device=dev, dtype=torch.float16)
@@ -856,8 +873,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="opt-6.7b-layer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel", default=None,
-                    help="time one kernel alone: attention, qkv_gemm, out_gemm, fc1_gemm, fc2_gemm, quantize, "
-                         "dequantize")
+                    help="time one kernel alone: attention, prefill_attention, qkv_gemm, out_gemm, fc1_gemm, "
+                         "fc2_gemm, quantize, dequantize")
     ap.add_argument("--seqs", type=int, default=0, help="--kernel: sequences (default: the workload's block)")
     ap.add_argument("--log2-elems", type=int, default=28, help="--kernel quantize/dequantize: tensor size")
     ap.add_argument("--layers", type=int, default=0, help="stack workloads: number of layers (default: the model's)")

@@ -6,9 +6,10 @@
 // the same pages mention (dev.to guide, "Efficient Attention Implementations").
 //
 // One CTA (4 warps) per (query row, head).  The row's cached K/V codes and group
-// metadata stream through shared memory in chunks of 64 tokens with 1-D bulk copies
+// metadata stream through shared memory in chunks of 128 tokens with 1-D bulk copies
 // (cp.async.bulk, completion on an mbarrier), kStages chunks in flight; each warp takes
-// 16 tokens of every chunk.
+// 16 tokens of every 64 in a chunk (two tiles per chunk), so the per-chunk barrier, wait and
+// refill are paid once per 32 tokens of a warp.
 //
 // Both products run on the tensor cores (mma.sync m16n8k16, fp16 operands, fp32
 // accumulation) directly on the codes, through the group decomposition
@@ -33,8 +34,8 @@
 
 namespace {
 
-constexpr int kChunk = 64;
-constexpr int kStages = 4;
+constexpr int kChunk = 128;
+constexpr int kStages = 2;
 constexpr int kWarps = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kSlack = 2.0f;
@@ -264,7 +265,8 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
       const __half *Ks = Km + kChunk * NG;
       const __half *Vm = Ks + kChunk * NG;
       const __half *Vs = Vm + kChunk * NG;
-      const int t0 = warp * 16;  // this warp's tokens in the chunk: t0 .. t0+15
+      for (int sub = 0; sub < kChunk / 64; sub++) {
+      const int t0 = sub * 64 + warp * 16;  // this warp's tokens of the chunk: t0 .. t0+15
 
       // ---- group sums of q . c for tokens t0+gid and t0+gid+8 ----
       float slo[4], shi[4];
@@ -370,6 +372,7 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
             mma_f16(ov[4 * j + 2 * h + 1], Ps & kLoNib, Ps & kHiNib, Qs & kLoNib, Qs & kHiNib, wb0, wb1);
           }
         }
+      }
       }
     }
     __syncthreads();  // every warp is done with stage st

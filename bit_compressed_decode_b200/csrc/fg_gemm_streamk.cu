@@ -48,7 +48,8 @@ constexpr int kTok = 256 * kNTT;           // tokens per pair tile
 constexpr int kStage = kA + kNTT * kBHalf;
 constexpr int kStages = 4;
 constexpr int kRing = kStages * kStage;    // 192 KB
-constexpr int kSmem = kRing + 1024;
+constexpr int kOutChunk = 32 * 128 * 4;    // one 32-token chunk of this CTA's 128 features, fp32: 16 KB
+constexpr int kSmem = kRing + 2 * kOutChunk + 1024;  // ring + double-buffered output staging + alignment
 constexpr int kCols = 256 * kNTT;          // TMEM columns
 constexpr int kPrefetch = 4;
 constexpr uint32_t kIdesc = umma_idesc_f16_f32(256, 256);
@@ -126,12 +127,6 @@ __device__ __forceinline__ bool wait_sleeping(uint32_t bar, uint32_t parity, vol
   return true;
 }
 
-__device__ __forceinline__ float epi_value(float v, float bias, float res, int n, const SkArgs &a) {
-  v += bias;
-  if (n < a.qcols) v *= a.qscale;
-  if (a.relu) v = fmaxf(v, 0.f);
-  return v + res;
-}
 
 __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_streamk_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                         const SkArgs a) {
@@ -394,26 +389,23 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_streamk_kernel(const _
         fence_proxy_async_smem();
         for (int c = 0; c < D && c < 2 * 8; c++) issue_chunk(c);
       }
+      const int te = (warp - kEpiWarp0) * 32 + lane;   // epilogue thread 0..127
+      const int n0 = (tile % a.nf) * 256 + half * 128;  // this CTA's first feature (N % 128 == 0)
+      float qs = 1.f;
+      if (n < a.qcols) qs = a.qscale;
       for (int t = 0; t < kNTT; t++) {
 #pragma unroll 1
         for (int c32 = 0; c32 < 8; c32++) {
           const int c = t * 8 + c32;
+          float *ost = reinterpret_cast<float *>(smem + kRing + (c & 1) * kOutChunk);  // [32 tokens][128]
           uint32_t v[32];
           tmem_ld_32x32b_x32(lane_base + t * 256 + c32 * 32, v);
           tmem_wait_ld();
           const int ml = t * 256 + c32 * 32;   // first token of the chunk within the tile
-          if (!first) {
-            // a later segment of a split tile: store the partial sum in this pair's slot
-            if (ready) {
-#pragma unroll
-              for (int j = 0; j < 32; j++) mine[static_cast<int64_t>(ml + j) * 128] = __uint_as_float(v[j]);
-            }
-            continue;
-          }
           float acc[32];
 #pragma unroll
           for (int j = 0; j < 32; j++) acc[j] = __uint_as_float(v[j]);
-          if (staged) {
+          if (first && staged) {
             // the other segments, in k order, from the staged chunk
             if (ready && wait_sleeping_cta(smem_u32(&red_bar[c % D]), (c / D) & 1, abortp, a.err)) {
               for (int qi = 0; qi < nq; qi++) {
@@ -424,32 +416,59 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_streamk_kernel(const _
             } else {
               ready = false;
             }
-          } else if (ready) {
+          } else if (first && !whole && ready) {
             for (int q = p + 1; q <= q_last; q++) {  // the other segments, in k order
               const float *src = slot(q) + fl;
 #pragma unroll
               for (int j = 0; j < 32; j++) acc[j] += __ldcg(src + static_cast<int64_t>(ml + j) * 128);
             }
           }
-          if (ready && nlive) {
-            float res[32];
+          // stage the chunk: the raw partial sum of a later segment, or the output before its
+          // residual (bias, q-scale, ReLU applied per feature)
 #pragma unroll
-            for (int j = 0; j < 32; j++) {
-              const int m = tok0 + ml + j;
-              res[j] = (a.res && m < a.M) ? __half2float(a.res[static_cast<int64_t>(m) * a.N + n]) : 0.f;
+          for (int j = 0; j < 32; j++) {
+            float y = acc[j];
+            if (first) {
+              y = (y + bias) * qs;
+              if (a.relu) y = fmaxf(y, 0.f);
             }
-#pragma unroll
-            for (int j = 0; j < 32; j++) {
-              const int m = tok0 + ml + j;
-              if (m < a.M) a.y[static_cast<int64_t>(m) * a.N + n] = __float2half_rn(epi_value(acc[j], bias, res[j], n, a));
-            }
+            ost[j * 128 + fl] = y;
           }
-          if (staged) {
-            // every epilogue thread is done with chunk c's buffers: refill them with chunk c + D
-            epi_sync();
-            if (warp == kEpiWarp0 && lane == 0 && c + D < 2 * 8 && !*abortp) {
-              fence_proxy_async_smem();
-              issue_chunk(c + D);
+          // every epilogue thread has staged chunk c (and is done with its staged partials)
+          epi_sync();
+          if (staged && warp == kEpiWarp0 && lane == 0 && c + D < 2 * 8 && !*abortp) {
+            fence_proxy_async_smem();
+            issue_chunk(c + D);
+          }
+          if (ready) {
+            if (!first) {
+              // 16 KB contiguous in this pair's slot: 8 passes of 16 bytes per thread
+#pragma unroll
+              for (int i = 0; i < 8; i++) {
+                const int e = i * 128 + te;
+                *reinterpret_cast<float4 *>(mine - fl + static_cast<int64_t>(ml + (e >> 5)) * 128 + (e & 31) * 4) =
+                    reinterpret_cast<const float4 *>(ost)[e];
+              }
+            } else if (n0 < a.N) {
+              // 8 features of one token per thread and pass (16-byte stores, residual added here)
+#pragma unroll
+              for (int i = 0; i < 4; i++) {
+                const int e = i * 128 + te, tok = e >> 4, f8 = (e & 15) * 8;
+                const int m = tok0 + ml + tok;
+                if (m >= a.M) continue;
+                const float4 p0 = *reinterpret_cast<const float4 *>(ost + tok * 128 + f8);
+                const float4 p1 = *reinterpret_cast<const float4 *>(ost + tok * 128 + f8 + 4);
+                const float w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                __half *yp = a.y + static_cast<int64_t>(m) * a.N + n0 + f8;
+                uint4 rv = make_uint4(0, 0, 0, 0);
+                if (a.res) rv = *reinterpret_cast<const uint4 *>(a.res + static_cast<int64_t>(m) * a.N + n0 + f8);
+                const __half *rh = reinterpret_cast<const __half *>(&rv);
+                uint4 ov;
+                __half *oh = reinterpret_cast<__half *>(&ov);
+#pragma unroll
+                for (int u = 0; u < 8; u++) oh[u] = __float2half_rn(w[u] + __half2float(rh[u]));
+                *reinterpret_cast<uint4 *>(yp) = ov;
+              }
             }
           }
         }
