@@ -61,8 +61,9 @@ def load_peaks():
     return dict(hbm=6650.0, tc_burst=1590.0, tc_sustained=1400.0, source="fallback")
 
 
-def kernel_work(wl, S, L_avg, group=64):
-    """Algorithmic work per launch of each kernel of one decode step (bytes or flops)."""
+def kernel_work(wl, S, L_avg, group=64, fused_append=True):
+    """Algorithmic work per launch of each kernel of one step (bytes or flops).  Decode rows
+    append their k, v inside the attention kernel (fused_append); prompt rows append apart."""
     h, F, H = wl["hidden"], wl["ffn"], wl["heads"]
     d = h // H
     kv_tok = 2 * (d // 2 + 4 * (d // group))         # K and V codes + fp16 min/scale per (seq, head, token)
@@ -71,7 +72,10 @@ def kernel_work(wl, S, L_avg, group=64):
         "ln1": ("hbm", 2 * S * h * 2 + 4 * h),
         "qkv_gemm": ("tensor", 2 * S * 3 * h * h),
         "kv_append": ("hbm", S * 2 * h * 2 + S * H * kv_tok),  # fp16 k, v in; codes and metadata out
-        "attention": ("hbm", S * H * L_avg * kv_tok + 2 * S * h * 2),
+        # decode attention appends the step's k, v itself: fp16 q, k, v in, o out, the new
+        # codes and metadata written, the cache read up to and including them
+        "attention": ("hbm", S * H * L_avg * kv_tok + 2 * S * h * 2
+                      + ((2 * S * h * 2 + S * H * kv_tok) if fused_append else 0)),
         "out_gemm": ("tensor", 2 * S * h * h),
         "ln2": ("hbm", 2 * S * h * 2 + 4 * h),
         "fc1_gemm": ("tensor", 2 * S * F * h),
@@ -561,7 +565,7 @@ def run_prefill(args, wl):
     fg.fg_sync_status()
     peaks = load_peaks()
     rows = S * P
-    work, _ = kernel_work(wl, rows, (P + 1) / 2)   # causal: row t of a prompt reads t + 1 cached tokens
+    work, _ = kernel_work(wl, rows, (P + 1) / 2, fused_append=False)   # causal: row t of a prompt reads t + 1 cached tokens
     # prompt attention runs tiled on the tensor cores: 4 d flops per (row, head, visible key)
     # (q.k and p.v), causal, so sum over rows of t + 1 keys; bound by the tensor pipe
     work["attention"] = ("tensor", 4 * (h // H) * H * S * P * (P + 1) // 2)
@@ -783,7 +787,7 @@ def run_kernel(args, wl):
     g.manual_seed(7)
     peaks = load_peaks()
     stream = torch.cuda.current_stream()
-    if args.kernel == "attention":
+    if args.kernel in ("attention", "attention_append"):
         maxL = (P + wl["steps"] + 63) // 64 * 64
         ng = d // 64
         cache = fg.KVCache(S, H, d, maxL, device=dev, arrays=[
@@ -796,8 +800,14 @@ def run_kernel(args, wl):
         qkv = torch.randn((S, 3 * h), generator=g, device=dev, dtype=torch.float16) * 0.1
         out = torch.empty((S, h), dtype=torch.float16, device=dev)
         pos = torch.full((S,), P, dtype=torch.int32, device=dev)
-        run = lambda: fg.fg_attention_decode(cache, qkv[:, :h], pos, out=out, stream=stream)
-        work, unit, peak = S * H * (P + 1) * 2 * (d // 2 + 4 * ng) + 2 * S * h * 2, "GB/s", peaks["hbm"]
+        kv_tok = 2 * (d // 2 + 4 * ng)
+        work, unit, peak = S * H * (P + 1) * kv_tok + 2 * S * h * 2, "GB/s", peaks["hbm"]
+        if args.kernel == "attention":
+            run = lambda: fg.fg_attention_decode(cache, qkv[:, :h], pos, out=out, stream=stream)
+        else:  # the decode step's form: the new k, v appended at position P in the same launch
+            run = lambda: fg.fg_attention_decode_append(cache, qkv[:, :h], qkv[:, h:2 * h], qkv[:, 2 * h:], pos,
+                                                        out=out, stream=stream)
+            work += 2 * S * h * 2 + S * H * kv_tok
     elif args.kernel == "prefill_attention":
         # the prompts' attention of the prefill: S sequences x P prompt rows over a cache holding
         # those P tokens (seeded codes), causal; 4 d flops per (row, head, visible key)
@@ -873,7 +883,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="opt-6.7b-layer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel", default=None,
-                    help="time one kernel alone: attention, prefill_attention, qkv_gemm, out_gemm, fc1_gemm, "
+                    help="time one kernel alone: attention, attention_append, prefill_attention, qkv_gemm, out_gemm, fc1_gemm, "
                          "fc2_gemm, quantize, dequantize")
     ap.add_argument("--seqs", type=int, default=0, help="--kernel: sequences (default: the workload's block)")
     ap.add_argument("--log2-elems", type=int, default=28, help="--kernel quantize/dequantize: tensor size")

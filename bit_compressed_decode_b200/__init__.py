@@ -6,7 +6,7 @@ it raises ImportError (there is no CPU path).
 """
 from ._binding import (  # noqa: F401
     FG_EPI_RELU, FG_EPI_RESIDUAL, FG_GEMM_PERSISTENT, LIB_PATH, STATUS, FgError, KVCache, LayerConfig, LayerWeights, QTensor, Stack,
-    fg_attention_decode, fg_dequantize, fg_kv_append, fg_layer_decode, fg_layer_prefill, fg_layernorm,
+    fg_attention_decode, fg_attention_decode_append, fg_dequantize, fg_kv_append, fg_layer_decode, fg_layer_prefill, fg_layernorm,
     fg_linear_w4a16, fg_linear_plan, fg_linear_workspace_bytes, fg_qtensor_bytes, fg_quantize, fg_status_string, fg_sync_status,
     fg_profile_enable, fg_profile_collect, PROFILE_SLOTS, fg_layer_decode_noalloc, NOALLOC_SCRATCH_BYTES,
     fg_linear_plan_pairs, fg_linear_classic_scratch_bytes, fg_test_gemm_stall,

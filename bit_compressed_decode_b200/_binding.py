@@ -75,6 +75,7 @@ _decl("fg_dequantize", c_int, POINTER(fg_qtensor), P, P)
 _decl("fg_kv_cache_bytes", c_int, c_int, c_int, c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_size_t))
 _decl("fg_kv_append", c_int, POINTER(fg_kv_cache), P, P, c_int64, c_int, c_int, P, P)
 _decl("fg_attention_decode", c_int, POINTER(fg_kv_cache), P, c_int64, P, c_int64, c_int, c_int, P, P)
+_decl("fg_attention_decode_append", c_int, POINTER(fg_kv_cache), P, c_int64, P, P, c_int64, P, c_int64, c_int, P, P)
 _decl("fg_linear_workspace_bytes", c_size_t, c_int, c_int, c_int)
 _decl("fg_linear_plan", c_int, c_int, c_int, c_int, POINTER(c_int), POINTER(c_int), POINTER(c_int))
 _decl("fg_linear_w4a16", c_int, P, c_int, c_int, POINTER(fg_qtensor), P, P, c_int, c_int, c_float, P, P, c_size_t, P)
@@ -252,6 +253,23 @@ def fg_attention_decode(cache: KVCache, q: torch.Tensor, positions: torch.Tensor
     s = cache.struct()
     _check(_lib.fg_attention_decode(ctypes.byref(s), _ptr(q), q.stride(0), _ptr(out), out.stride(0), rows,
                                     rows_per_seq, _ptr(positions), _stream(stream)), "fg_attention_decode")
+    return out
+
+
+def fg_attention_decode_append(cache: KVCache, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                               positions: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Append k, v at ``positions`` and attend with q, one launch (decode rows: one per sequence)."""
+    rows = q.shape[0]
+    hd = cache.num_heads * cache.head_dim
+    if k.stride(0) != v.stride(0):
+        raise ValueError("k and v must share a row stride")
+    _need(positions, torch.int32, "positions")
+    if out is None:
+        out = torch.empty((rows, hd), dtype=torch.float16, device=q.device)
+    s = cache.struct()
+    _check(_lib.fg_attention_decode_append(ctypes.byref(s), _ptr(q), q.stride(0), _ptr(k), _ptr(v), k.stride(0),
+                                           _ptr(out), out.stride(0), rows, _ptr(positions), _stream(stream)),
+           "fg_attention_decode_append")
     return out
 
 

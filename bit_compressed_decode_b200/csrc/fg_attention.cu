@@ -52,6 +52,8 @@ struct AttnArgs {
   const int32_t *positions;
   int rows, rows_per_seq, H, maxL;
   unsigned int *err;
+  const __half *kn, *vn;  // decode rows: new k, v (fp16) quantised into the cache first; null: none
+  int64_t ldn;
 };
 
 template <int D, int G>
@@ -155,8 +157,62 @@ __device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
   return *reinterpret_cast<const uint32_t *>(&h);
 }
 
+// The decode row's new k and v (D fp16 values each) in 4-bit form, held by one warp: unit us
+// (group us / 2 of k for even us, of v for odd us) is quantised by G/8 lanes with the group
+// quantiser the append kernel uses, so the cache receives the same bits.
 template <int D, int G>
-__global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs a) {
+struct NewRow {
+  static constexpr int NG = D / G, L = G / 8, USTEP = 32 / L, STEPS = (2 * NG + USTEP - 1) / USTEP;
+  uint4 x[STEPS];
+  uint32_t w[STEPS];
+  __half mn[STEPS], sc[STEPS];
+
+  __device__ __forceinline__ void load(const __half *krow, const __half *vrow, int lane) {
+    const int u = lane / L, j = lane % L;
+#pragma unroll
+    for (int st = 0; st < STEPS; st++) {
+      const int us = st * USTEP + u;
+      x[st] = make_uint4(0, 0, 0, 0);
+      if (us < 2 * NG) x[st] = *reinterpret_cast<const uint4 *>(((us & 1) ? vrow : krow) + (us >> 1) * G + j * 8);
+    }
+  }
+  __device__ __forceinline__ void quantise() {  // all 32 lanes: the quantiser shuffles
+#pragma unroll
+    for (int st = 0; st < STEPS; st++) w[st] = quant_group8<L>(x[st], mn[st], sc[st]);
+  }
+  // one token row: codes as 32-bit words (D/8 per row), NG mins and scales per array
+  __device__ __forceinline__ void write(uint32_t *kc, uint32_t *vc, __half *km, __half *ks, __half *vm, __half *vs,
+                                        int lane) const {
+    const int u = lane / L, j = lane % L;
+#pragma unroll
+    for (int st = 0; st < STEPS; st++) {
+      const int us = st * USTEP + u;
+      if (us >= 2 * NG) continue;
+      const int g = us >> 1;
+      ((us & 1) ? vc : kc)[g * L + j] = w[st];
+      if (j == 0) {
+        ((us & 1) ? vm : km)[g] = mn[st];
+        ((us & 1) ? vs : ks)[g] = sc[st];
+      }
+    }
+  }
+};
+
+// One token row (D/8 code words per array, NG mins and scales per array) copied by a warp.
+template <int D, int NG>
+__device__ __forceinline__ void copy_row(uint32_t *kc, uint32_t *vc, __half *km, __half *ks, __half *vm, __half *vs,
+                                         const uint32_t (&codes)[2][D / 8], const __half (&meta)[4][NG], int lane) {
+#pragma unroll
+  for (int i = lane; i < D / 4; i += 32) (i < D / 8 ? kc[i] : vc[i - D / 8]) = codes[i / (D / 8)][i % (D / 8)];
+  if (lane < 4 * NG) {
+    const int arr = lane / NG, g = lane % NG;
+    __half *dst = arr == 0 ? km : arr == 1 ? ks : arr == 2 ? vm : vs;
+    dst[g] = meta[arr][g];
+  }
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kWarps * 32, D <= 128 ? 5 : 1) attn_decode_kernel(const AttnArgs a) {
   using S = AttnShape<D, G>;
   constexpr int NG = S::NG, RB = S::RB, KW = S::KW, VW = S::VW, MT = S::MT;
   constexpr float kS24 = 16777216.0f, kS20 = 1048576.0f;
@@ -164,6 +220,10 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ float red_m[kWarps], red_l[kWarps];
   __shared__ float red_o[kWarps][D];
+  // fused append: the new k, v rows (fp16, copied with the first chunk) and their 4-bit form
+  __shared__ __align__(16) __half new_x[2][D];
+  __shared__ __align__(16) uint32_t new_codes[2][D / 8];
+  __shared__ __half new_meta[4][NG];  // k min, k scale, v min, v scale
   griddep_launch();  // the output projection may start its weight-side prologue
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -187,7 +247,13 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
     const int ntr = (nt + 7) & ~7;  // whole 16-byte metadata rows; stays below max_len (multiple of 64)
     const uint32_t cb = ntr * RB, mb = ntr * NG * 2;
     const uint32_t bar = smem_u32(&full_bar[st]);
-    mbar_arrive_expect_tx(bar, 2 * cb + 4 * mb);
+    const bool rows = a.kn != nullptr && ch == 0;  // fused append: the new k, v rows come with chunk 0
+    mbar_arrive_expect_tx(bar, 2 * cb + 4 * mb + (rows ? 4 * D : 0));
+    if (rows) {
+      const int64_t o = static_cast<int64_t>(r) * a.ldn + hd * D;
+      bulk_g2s(smem_u32(&new_x[0][0]), a.kn + o, 2 * D, bar);
+      bulk_g2s(smem_u32(&new_x[1][0]), a.vn + o, 2 * D, bar);
+    }
     const int64_t t0 = slot0 + static_cast<int64_t>(ch) * kChunk;
     uint8_t *p = stage_ptr(st);
     bulk_g2s(smem_u32(p), a.kc + t0 * RB, cb, bar);
@@ -206,6 +272,14 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
   __syncthreads();
   if (tid == 0)
     for (int ch = 0; ch < min(kStages, nchunks); ch++) issue(ch);
+  // Fused append (decode): the new token (position L - 1, row tl of the last chunk) is read
+  // only by the warp that owns its 16 tokens of the chunk's 64-token sub-tile.  When that
+  // chunk has landed (the new k, v rows landed with the first chunk), the warp quantises the
+  // rows, puts them in place of whatever the copy brought for that row, and stores them to
+  // the cache after the loop, when no copy of this kernel still reads it.
+  const bool app = a.kn != nullptr;
+  const int tl = (L - 1) % kChunk, app_chunk = (L - 1) / kChunk;
+  const bool app_warp = app && warp == (tl % 64) / 16;
 
   // ---- q as the B operand of the score MMAs, in the dim order of kword_off ----
   // Word j of lane class c holds, per 16-bit half, nibbles (bits 0-3, 4-7, 8-11, 12-15) =
@@ -265,8 +339,27 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
       const __half *Ks = Km + kChunk * NG;
       const __half *Vm = Ks + kChunk * NG;
       const __half *Vs = Vm + kChunk * NG;
+      if (app_warp && ch == app_chunk) {
+        {
+          NewRow<D, G> nr;
+          nr.load(new_x[0], new_x[1], lane);
+          nr.quantise();
+          nr.write(new_codes[0], new_codes[1], new_meta[0], new_meta[1], new_meta[2], new_meta[3], lane);
+        }
+        __syncwarp();
+        // the new row in place of the copied one; the proxy fence orders these writes before
+        // the bulk copy that reuses the stage (issued after the chunk's barrier)
+        uint8_t *b = stage_ptr(st);
+        __half *km = reinterpret_cast<__half *>(b + 2 * S::CODE_B);
+        copy_row<D, NG>(reinterpret_cast<uint32_t *>(b + tl * RB), reinterpret_cast<uint32_t *>(b + S::CODE_B + tl * RB),
+                        km + tl * NG, km + kChunk * NG + tl * NG, km + 2 * kChunk * NG + tl * NG,
+                        km + 3 * kChunk * NG + tl * NG, new_codes, new_meta, lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
       for (int sub = 0; sub < kChunk / 64; sub++) {
       const int t0 = sub * 64 + warp * 16;  // this warp's tokens of the chunk: t0 .. t0+15
+      if (ch * kChunk + t0 >= L) break;     // warp-uniform: none of them (nor later ones) visible
 
       // ---- group sums of q . c for tokens t0+gid and t0+gid+8 ----
       float slo[4], shi[4];
@@ -379,6 +472,15 @@ __global__ void __launch_bounds__(kWarps * 32) attn_decode_kernel(const AttnArgs
     if (tid == 0 && ok && ch + kStages < nchunks) issue(ch + kStages);
   }
 
+  if (app_warp && ok) {  // the new row into the cache (every copy of this kernel has completed)
+    const int64_t slot = slot0 + L - 1;
+    copy_row<D, NG>(reinterpret_cast<uint32_t *>(const_cast<uint8_t *>(a.kc)) + slot * (D / 8),
+                    reinterpret_cast<uint32_t *>(const_cast<uint8_t *>(a.vc)) + slot * (D / 8),
+                    const_cast<__half *>(a.km) + slot * NG, const_cast<__half *>(a.ks) + slot * NG,
+                    const_cast<__half *>(a.vm) + slot * NG, const_cast<__half *>(a.vs) + slot * NG, new_codes,
+                    new_meta, lane);
+  }
+
   // ---- per-warp totals, then combine the 4 warps ----
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -457,7 +559,9 @@ fg_status fg_attention_prefill_launch(const fg_kv_cache *kv, const fg_half *q, i
 // Prompt rows (rows_per_seq > 1) go to the tiled prefill kernel, which reads each K/V tile once
 // for 64 query rows; decode rows, and head dims that kernel does not take, to this one.
 fg_status fg_attention_launch(const fg_kv_cache *kv, const fg_half *q, int64_t ldq, fg_half *out, int64_t ldo,
-                              int rows, int rows_per_seq, const int32_t *positions, cudaStream_t st) {
+                              int rows, int rows_per_seq, const int32_t *positions, cudaStream_t st,
+                              const fg_half *k_new, const fg_half *v_new, int64_t ld_new) {
+  if (k_new && rows_per_seq != 1) return FG_ERR_INVALID;  // the fused append is for decode rows
   if (rows_per_seq > 1) {
     const fg_status rc = fg_attention_prefill_launch(kv, q, ldq, out, ldo, rows, rows_per_seq, positions, st);
     if (rc != FG_ERR_UNSUPPORTED) return rc;
@@ -480,6 +584,9 @@ fg_status fg_attention_launch(const fg_kv_cache *kv, const fg_half *q, int64_t l
   a.maxL = kv->max_len;
   a.err = fg_error_word_ptr();
   if (!a.err) return FG_ERR_CUDA;
+  a.kn = reinterpret_cast<const __half *>(k_new);
+  a.vn = reinterpret_cast<const __half *>(v_new);
+  a.ldn = ld_new;
   const int G = fg_kv_group(kv->group);
   if (G == 64) {
     switch (kv->head_dim) {
@@ -506,5 +613,20 @@ extern "C" fg_status fg_attention_decode(const fg_kv_cache *kv, const fg_half *q
   if (!q || !out || !positions || !fg_aligned16(q) || !fg_aligned16(out)) return FG_ERR_INVALID;
   const int64_t hD = static_cast<int64_t>(kv->num_heads) * kv->head_dim;
   if (ldq < hD || ldo < hD || ldq % 8 || ldo % 8) return FG_ERR_SHAPE;
-  return fg_attention_launch(kv, q, ldq, out, ldo, rows, rows_per_seq, positions, static_cast<cudaStream_t>(stream));
+  return fg_attention_launch(kv, q, ldq, out, ldo, rows, rows_per_seq, positions, static_cast<cudaStream_t>(stream),
+                             nullptr, nullptr, 0);
+}
+
+extern "C" fg_status fg_attention_decode_append(const fg_kv_cache *kv, const fg_half *q, int64_t ldq,
+                                                const fg_half *k, const fg_half *v, int64_t ldkv, fg_half *out,
+                                                int64_t ldo, int rows, const int32_t *positions, void *stream) {
+  fg_status rc = fg_kv_validate(kv);
+  if (rc != FG_OK) return rc;
+  if (rows < 0 || rows > kv->num_seqs) return FG_ERR_SHAPE;
+  if (rows == 0) return FG_OK;
+  if (!q || !out || !k || !v || !positions) return FG_ERR_INVALID;
+  if (!fg_aligned16(q) || !fg_aligned16(out) || !fg_aligned16(k) || !fg_aligned16(v)) return FG_ERR_INVALID;
+  const int64_t hD = static_cast<int64_t>(kv->num_heads) * kv->head_dim;
+  if (ldq < hD || ldo < hD || ldkv < hD || ldq % 8 || ldo % 8 || ldkv % 8) return FG_ERR_SHAPE;
+  return fg_attention_launch(kv, q, ldq, out, ldo, rows, 1, positions, static_cast<cudaStream_t>(stream), k, v, ldkv);
 }

@@ -155,38 +155,42 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
         mb[j] = sb[j] = __ushort_as_half(0);
       }
     }
-    for (int i = 0; i < nk; i++) {
-      const int st = i % C::STAGES;
-      const uint4 c0 = cb[0][0], c1 = cb[0][1];
-      const __half m0 = mb[0], s0 = sb[0];
+    // ring of prefetched codes indexed statically (unrolled by the prefetch depth): a slot
+    // is consumed in place and refilled kPrefetch k-tiles ahead, so no register holding a
+    // load in flight is ever moved (a move would wait for its load)
+    bool go = true;
+    for (int i0 = 0; go && i0 < nk; i0 += kPrefetch) {
 #pragma unroll
-      for (int j = 0; j + 1 < kPrefetch; j++) {
-        cb[j][0] = cb[j + 1][0];
-        cb[j][1] = cb[j + 1][1];
-        mb[j] = mb[j + 1];
-        sb[j] = sb[j + 1];
-      }
-      if (i + kPrefetch < nk && live) {
-        const int kt = kt0 + i + kPrefetch;
-        cb[kPrefetch - 1][0] = crow[kt * 2];
-        cb[kPrefetch - 1][1] = crow[kt * 2 + 1];
-        mb[kPrefetch - 1] = mrow[kt >> a.gshift];
-        sb[kPrefetch - 1] = srow[kt >> a.gshift];
-      }
-      if (i >= C::STAGES &&
-          !mbar_wait_bounded(smem_u32(&empty[st]), ((i / C::STAGES) - 1) & 1, abortp, a.err, a.wait_ns))
-        break;
-      const __half2 s2 = __half2half2(s0), m2 = __half2half2(m0);
-      uint8_t *at = a_tile(st, acc);
-      const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      for (int j = 0; j < kPrefetch; j++) {
+        const int i = i0 + j;
+        if (!go || i >= nk) break;
+        const int st = i % C::STAGES;
+        const uint4 c0 = cb[j][0], c1 = cb[j][1];
+        const __half m0 = mb[j], s0 = sb[j];
+        if (i + kPrefetch < nk && live) {
+          const int kt = kt0 + i + kPrefetch;
+          cb[j][0] = crow[kt * 2];
+          cb[j][1] = crow[kt * 2 + 1];
+          mb[j] = mrow[kt >> a.gshift];
+          sb[j] = srow[kt >> a.gshift];
+        }
+        if (i >= C::STAGES &&
+            !mbar_wait_bounded(smem_u32(&empty[st]), ((i / C::STAGES) - 1) & 1, abortp, a.err, a.wait_ns)) {
+          go = false;
+          break;
+        }
+        const __half2 s2 = __half2half2(s0), m2 = __half2half2(m0);
+        uint8_t *at = a_tile(st, acc);
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-      for (int c = 0; c < 8; c++) {
-        const uint4 v = live ? dequant8(words[c], s2, m2) : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4 *>(at + sw128_offset(r, c)) = v;
+        for (int c = 0; c < 8; c++) {
+          const uint4 v = live ? dequant8(words[c], s2, m2) : make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4 *>(at + sw128_offset(r, c)) = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && !(a.stall && i == 0)) mbar_arrive(smem_u32(&full_a[st]));
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0 && !(a.stall && i == 0)) mbar_arrive(smem_u32(&full_a[st]));
     }
   } else if (warp == kTmaWarp) {
     // ---------------- TMA producer for the x tiles ----------------
@@ -473,38 +477,44 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
         mb[j] = sb[j] = __ushort_as_half(0);
       }
     }
-    // leader: arrive on its own full barrier; odd CTA: on a_half, forwarded by warp 9
+    // leader: arrive on its own full barrier; odd CTA: on a_half, forwarded by warp 9.
+    // The prefetched codes sit in a ring indexed statically (the loop is unrolled by the
+    // prefetch depth): k-tile i's codes are consumed in place, and the slot is refilled
+    // with those of k-tile i + kPairPrefetch.  Shifting the array down instead would move
+    // registers whose loads are still in flight, and each move waits for its load.
     const uint32_t done_bar0 = smem_u32(leader ? &full[0] : &a_half[0]);
-    for (int i = 0; i < nk; i++) {
-      const int st = i % kPairStages;
-      const uint4 c0 = cb[0];
-      const __half m0 = mb[0], s0 = sb[0];
+    bool go = true;
+    for (int i0 = 0; go && i0 < nk; i0 += kPairPrefetch) {
 #pragma unroll
-      for (int j = 0; j + 1 < kPairPrefetch; j++) {
-        cb[j] = cb[j + 1];
-        mb[j] = mb[j + 1];
-        sb[j] = sb[j + 1];
-      }
-      if (i + kPairPrefetch < nk && live) {
-        const int kt = kt0 + i + kPairPrefetch;
-        cb[kPairPrefetch - 1] = crow[kt * 2 + hk];
-        mb[kPairPrefetch - 1] = mrow[kt >> a.gshift];
-        sb[kPairPrefetch - 1] = srow[kt >> a.gshift];
-      }
-      if (i >= kPairStages &&
-          !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kPairStages) - 1) & 1, abortp, a.err))
-        break;
-      const __half2 s2 = __half2half2(s0), m2 = __half2half2(m0);
-      uint8_t *at = a_tile(st);
-      const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
+      for (int j = 0; j < kPairPrefetch; j++) {
+        const int i = i0 + j;
+        if (!go || i >= nk) break;
+        const int st = i % kPairStages;
+        const uint4 c0 = cb[j];
+        const __half m0 = mb[j], s0 = sb[j];
+        if (i + kPairPrefetch < nk && live) {
+          const int kt = kt0 + i + kPairPrefetch;
+          cb[j] = crow[kt * 2 + hk];
+          mb[j] = mrow[kt >> a.gshift];
+          sb[j] = srow[kt >> a.gshift];
+        }
+        if (i >= kPairStages &&
+            !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kPairStages) - 1) & 1, abortp, a.err)) {
+          go = false;
+          break;
+        }
+        const __half2 s2 = __half2half2(s0), m2 = __half2half2(m0);
+        uint8_t *at = a_tile(st);
+        const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
 #pragma unroll
-      for (int c = 0; c < 4; c++) {
-        const uint4 v = live ? dequant8(words[c], s2, m2) : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4 *>(at + sw128_offset(row, 4 * hk + c)) = v;
+        for (int c = 0; c < 4; c++) {
+          const uint4 v = live ? dequant8(words[c], s2, m2) : make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4 *>(at + sw128_offset(row, 4 * hk + c)) = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(done_bar0 + st * 8);
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(done_bar0 + st * 8);
     }
   } else if (warp == kTmaWarp) {
     // ---------------- TMA producer: this CTA's halves of the two token tiles ----------------

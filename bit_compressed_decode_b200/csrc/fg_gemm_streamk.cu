@@ -225,26 +225,31 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_streamk_kernel(const _
       }
     }
     const uint32_t done_bar0 = smem_u32(leader ? &full[0] : &a_half[0]);
-    for (int i = 0; i < nit; i++) {
-      const int st = i % kStages;
-      const uint4 c0 = cb[0];
-      const __half m0 = mb[0], s0 = sb[0];
+    // statically indexed ring of prefetched codes (see the classic pair kernel): a slot is
+    // consumed in place and refilled kPrefetch iterations ahead
+    bool go = true;
+    for (int i0 = 0; go && i0 < nit; i0 += kPrefetch) {
 #pragma unroll
-      for (int j = 0; j + 1 < kPrefetch; j++) {
-        cb[j] = cb[j + 1];
-        mb[j] = mb[j + 1];
-        sb[j] = sb[j + 1];
+      for (int j = 0; j < kPrefetch; j++) {
+        const int i = i0 + j;
+        if (!go || i >= nit) break;
+        const int st = i % kStages;
+        const uint4 c0 = cb[j];
+        const __half m0 = mb[j], s0 = sb[j];
+        if (i + kPrefetch < nit) fetch(cb[j], mb[j], sb[j]);
+        if (i >= kStages && !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kStages) - 1) & 1, abortp, a.err)) {
+          go = false;
+          break;
+        }
+        const __half2 s2 = __half2half2(s0), m2 = __half2half2(m0);
+        uint8_t *at = a_tile(st);
+        const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
+#pragma unroll
+        for (int c = 0; c < 4; c++) *reinterpret_cast<uint4 *>(at + sw128_offset(row, 4 * hk + c)) = dequant8(words[c], s2, m2);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(done_bar0 + st * 8);
       }
-      if (i + kPrefetch < nit) fetch(cb[kPrefetch - 1], mb[kPrefetch - 1], sb[kPrefetch - 1]);
-      if (i >= kStages && !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kStages) - 1) & 1, abortp, a.err)) break;
-      const __half2 s2 = __half2half2(s0), m2 = __half2half2(m0);
-      uint8_t *at = a_tile(st);
-      const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
-#pragma unroll
-      for (int c = 0; c < 4; c++) *reinterpret_cast<uint4 *>(at + sw128_offset(row, 4 * hk + c)) = dequant8(words[c], s2, m2);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(done_bar0 + st * 8);
     }
   } else if (warp == kTmaWarp) {
     // ---------------- TMA: this CTA's halves of the two token tiles, every iteration ----------------

@@ -20,6 +20,7 @@
 
 // Host helpers (fg_status.cu).
 unsigned int *fg_error_word_ptr();  // device address of this device's error word (nullptr on failure)
+int fg_sm_count();                  // streaming multiprocessors of the current device (148 if unknown)
 size_t fg_layer_ws_required(const fg_layer_config *c, int rows);  // workspace a layer call cannot do without
 fg_status fg_cuda_check(cudaError_t e);  // records the error text, maps to FG_ERR_CUDA
 fg_status fg_launch_check();             // cudaGetLastError after a launch

@@ -21,7 +21,8 @@ fg_status fg_kv_validate(const fg_kv_cache *kv);
 fg_status fg_kv_append_launch(const fg_kv_cache *kv, const fg_half *k, const fg_half *v, int64_t ld, int rows,
                               int rows_per_seq, const int32_t *positions, cudaStream_t st);
 fg_status fg_attention_launch(const fg_kv_cache *kv, const fg_half *q, int64_t ldq, fg_half *out, int64_t ldo,
-                              int rows, int rows_per_seq, const int32_t *positions, cudaStream_t st);
+                              int rows, int rows_per_seq, const int32_t *positions, cudaStream_t st,
+                              const fg_half *k_new, const fg_half *v_new, int64_t ld_new);
 
 int fg_profile_begin(int slot, cudaStream_t st);
 void fg_profile_end(int idx, cudaStream_t st);
@@ -171,11 +172,20 @@ fg_status run_layer(const fg_layer_config *c, const fg_layer_weights *w, const f
   FG_SLICE(slice_wait(sl, 1, st));
   FG_STEP(1, fg_linear_launch(a, rows, h, &w->wqkv, w->bqkv, nullptr, 0, h, qscale, qkv, gws, gbytes, st, pdl));
   FG_SLICE(slice_done(sl, 1, st));
-  // append k, v (4-bit) at the sequences' positions
+  // append k, v (4-bit) at the sequences' positions, then o = softmax(q K^T) V over the
+  // 4-bit cache.  When the decode attention is about one wave of (row, head) CTAs or less its
+  // time is launch-bound and the append rides in it (one launch fewer: 58.6 instead of 63.7 us
+  // per step at the OPT-125M block of 4 sequences); above that the separate append kernel
+  // costs less than the per-CTA work it would add (a 512-sequence OPT-6.7B block: 10.7 us
+  // against 18 us).  Prompt rows always append first.
   FG_SLICE(slice_wait(sl, 2, st));
-  FG_STEP(2, fg_kv_append_launch(kv, qkv + h, qkv + 2 * h, 3 * h, rows, rows_per_seq, positions, st));
-  // o = softmax(q K^T) V over the 4-bit cache
-  FG_STEP(3, fg_attention_launch(kv, qkv, 3 * h, o, h, rows, rows_per_seq, positions, st));
+  const bool fuse = rows_per_seq == 1 && static_cast<int64_t>(rows) * c->num_heads <= 4LL * fg_sm_count();
+  if (fuse) {
+    FG_STEP(3, fg_attention_launch(kv, qkv, 3 * h, o, h, rows, 1, positions, st, qkv + h, qkv + 2 * h, 3 * h));
+  } else {
+    FG_STEP(2, fg_kv_append_launch(kv, qkv + h, qkv + 2 * h, 3 * h, rows, rows_per_seq, positions, st));
+    FG_STEP(3, fg_attention_launch(kv, qkv, 3 * h, o, h, rows, rows_per_seq, positions, st, nullptr, nullptr, 0));
+  }
   FG_SLICE(slice_done(sl, 2, st));
   // h1 = x + o Wo^T + bo
   FG_SLICE(slice_wait(sl, 3, st));

@@ -52,6 +52,18 @@ extern "C" const char *fg_status_string(fg_status s) {
   return "FG_ERR_UNKNOWN";
 }
 
+int fg_sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int n = cache[dev].load();
+  if (!n) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev].store(n);
+  }
+  return n;
+}
+
 extern "C" fg_status fg_sync_status(void *stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   fg_status rc = fg_cuda_check(cudaStreamSynchronize(st));

@@ -161,6 +161,20 @@ FG_API fg_status fg_kv_append(const fg_kv_cache *kv, const fg_half *k, const fg_
 FG_API fg_status fg_attention_decode(const fg_kv_cache *kv, const fg_half *q, int64_t ldq, fg_half *out, int64_t ldo,
                               int rows, int rows_per_seq, const int32_t *positions, void *stream);
 
+/* One decode step's KV append and attention in one launch: for each row r
+ * (sequence r, one row per sequence), k and v (fp16 device rows at
+ * k + r*ldkv, v + r*ldkv, num_heads*head_dim values, head-major) are quantised
+ * into the cache at position positions[r], exactly as fg_kv_append does (the
+ * cache receives the same bits), and q's row then attends over positions
+ * 0 .. positions[r] as fg_attention_decode does.  rows <= num_seqs.  A
+ * position outside [0, max_len) appends nothing, writes zeros to the row's
+ * output and flags FG_ERR_RANGE (fg_sync_status).  The k, v rows may share a
+ * buffer with q (the layer passes the k and v thirds of its [q k v] rows).
+ * ([G3]: the cache is written and read in its 4-bit form) */
+FG_API fg_status fg_attention_decode_append(const fg_kv_cache *kv, const fg_half *q, int64_t ldq, const fg_half *k,
+                                     const fg_half *v, int64_t ldkv, fg_half *out, int64_t ldo, int rows,
+                                     const int32_t *positions, void *stream);
+
 /* ---------------------------------------------------------------------- */
 /* W4A16 linear layer and LayerNorm                                         */
 /* ---------------------------------------------------------------------- */

@@ -209,3 +209,31 @@ def test_stack_decode_host_kv_validates_before_cuda():
     kv = (B.fg_kv_cache * 2)()
     assert _rc("fg_stack_decode_host_kv", None, kv, kv, 0, 0, 1, None, None, None, 1, 1, None, 0, None,
                None) == 1                                    # no stack: FG_ERR_INVALID
+
+
+def _fake_kv(S=4, H=2, d=128, maxL=64):
+    """A cache descriptor with aligned, never dereferenced addresses: for checks that must
+    fail on the host, before any CUDA call."""
+    kv = B.fg_kv_cache()
+    for i, name in enumerate(("k_codes", "k_mins", "k_scales", "v_codes", "v_mins", "v_scales")):
+        setattr(kv, name, 0x100000 * (i + 1))
+    kv.num_seqs, kv.num_heads, kv.head_dim, kv.max_len, kv.group = S, H, d, maxL, 64
+    return kv
+
+
+def test_attention_decode_append_validates_on_host():
+    kv = _fake_kv()
+    P = 0x800000                                            # aligned, never dereferenced
+    args = lambda **o: [ctypes.byref(o.get("kv", kv)), o.get("q", P), o.get("ldq", 256), o.get("k", P + 512),
+                        o.get("v", P + 1024), o.get("ldkv", 768), o.get("out", P * 2), o.get("ldo", 256),
+                        o.get("rows", 4), o.get("pos", P * 3), None]
+    assert _rc("fg_attention_decode_append", *args(rows=5)) == 2       # more rows than sequences: SHAPE
+    assert _rc("fg_attention_decode_append", *args(rows=-1)) == 2
+    assert _rc("fg_attention_decode_append", *args(rows=0)) == 0       # nothing to do
+    assert _rc("fg_attention_decode_append", *args(k=None)) == 1       # INVALID
+    assert _rc("fg_attention_decode_append", *args(v=P + 1026)) == 1   # misaligned v
+    assert _rc("fg_attention_decode_append", *args(pos=None)) == 1
+    assert _rc("fg_attention_decode_append", *args(ldkv=128)) == 2     # row stride below heads x head_dim
+    assert _rc("fg_attention_decode_append", *args(ldq=260)) == 2      # stride not a multiple of 8
+    bad = _fake_kv(maxL=100)                                           # max_len not a multiple of 64
+    assert _rc("fg_attention_decode_append", *args(kv=bad)) == 2

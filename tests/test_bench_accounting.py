@@ -27,7 +27,8 @@ def test_opt6p7b_decode_step_work(bench):
     assert totals["kv_bytes_per_token"] == 2 * (64 + 4 * 2) == 144
     assert totals["w4_bytes"] == 12 * h * h * 9 // 16   # 113.2 MB
     att = work["attention"][1]
-    assert att == S * H * 512 * 144 + 2 * S * h * 2      # 1.208 GB of KV4 + q and o
+    # 1.208 GB of KV4 read, q in and o out, and the fused append: k, v in, their codes out
+    assert att == S * H * 512 * 144 + 2 * S * h * 2 + 2 * S * h * 2 + S * H * 144
     assert work["kv_append"][1] == S * 2 * h * 2 + S * 2 * (h // 2 + h // 16)
     units = bench.kernel_units(wl, S, 512)
     assert units["attention"] == S * H * 512            # traffic of a smaller capture scales by these
@@ -43,5 +44,5 @@ def test_stack_and_prefill_shapes(bench):
     # prefill: row t of a prompt reads t + 1 cached tokens, so P rows read P (P + 1) / 2 in all
     wl = bench.WORKLOADS["opt-6.7b-prefill"]
     P = wl["prompt"]
-    work, _ = bench.kernel_work(wl, P, (P + 1) / 2)
+    work, _ = bench.kernel_work(wl, P, (P + 1) / 2, fused_append=False)
     assert work["attention"][1] == pytest.approx(wl["heads"] * P * (P + 1) / 2 * 144 + 2 * P * wl["hidden"] * 2)

@@ -277,6 +277,80 @@ def test_attention_decode_matches_oracle(H, d):
             assert err <= 2e-3 * np.max(np.abs(ref[s, sl])) + 1e-4, (s, h, err)
 
 
+def _seeded_cache(S, H, d, maxL, lens, seed, group):
+    """Oracle cache with lens[s] tokens per sequence (0 allowed), and its device copy."""
+    o = oracle.KVCache(S, H, d, maxL, group=group)
+    for s in range(S):
+        L = int(lens[s])
+        if L:
+            k = si.normal_f16(seed, 100 + s, (L, H * d), 1.0)
+            v = si.normal_f16(seed, 200 + s, (L, H * d), 1.0)
+            oracle.kv_append(o, k, v, np.full(L, s), np.arange(L))
+    arrays = [dev(a.view(np.float16) if a.dtype == np.uint16 else a) for a in o.arrays()]
+    return o, fg.KVCache(S, H, d, maxL, arrays=arrays, group=group)
+
+
+@pytest.mark.parametrize("H,d,group", [(4, 64, 64), (3, 128, 64), (2, 256, 64), (3, 128, 128), (2, 256, 128)])
+def test_attention_decode_append_fused(H, d, group):
+    # One launch appends each sequence's new k, v row and attends over the cache with it.
+    # New rows inside the first chunks the kernel streams (positions < 256) and past them;
+    # garbage in every slot from the new position on (the append must overwrite it, the
+    # attention must not read beyond it).  The cache must hold the oracle's append bits,
+    # the output must equal the append-then-attend launches bit for bit and the oracle's
+    # attention within the decode-attention tolerance.
+    S, maxL = 8, 384
+    pos = np.array([0, 1, 63, 127, 128, 255, 256, 300], dtype=np.int32)
+    o, g = _seeded_cache(S, H, d, maxL, pos, seed=31 + d + group, group=group)
+    _garbage_past(g, pos, 32)
+    g2 = fg.KVCache(S, H, d, maxL, arrays=[a.clone() for a in g.arrays()], group=group)
+    Hd = H * d
+    qkv = si.normal_f16(33, 1, (S, 3 * Hd), 1.0)
+    qkv[:, :Hd] = (qkv[:, :Hd].astype(np.float32) / np.sqrt(d)).astype(np.float16)
+    qd, pd = dev(qkv), dev(pos)
+    out = fg.fg_attention_decode_append(g, qd[:, :Hd], qd[:, Hd:2 * Hd], qd[:, 2 * Hd:], pd)
+    fg.fg_kv_append(g2, qd[:, Hd:2 * Hd], qd[:, 2 * Hd:], pd, ld=3 * Hd)
+    out2 = fg.fg_attention_decode(g2, qd[:, :Hd], pd)
+    fg.fg_sync_status()
+    assert torch.equal(out, out2)
+    for a, b in zip(g.arrays(), g2.arrays()):   # bytes: the planted garbage holds NaNs
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    oracle.kv_append(o, qkv[:, Hd:2 * Hd], qkv[:, 2 * Hd:], np.arange(S), pos)
+    for a, b in zip(g.arrays(), o.arrays()):
+        ha = u16(host(a)) if a.dtype == torch.float16 else host(a)
+        for s in range(S):
+            assert np.array_equal(ha[s, :, :pos[s] + 1], b[s, :, :pos[s] + 1]), s
+    ref = oracle.attention(o, qkv[:, :Hd], np.arange(S), pos + 1)
+    got = host(out).astype(np.float64)
+    for s in range(S):
+        for h in range(H):
+            sl = slice(h * d, (h + 1) * d)
+            err = np.max(np.abs(got[s, sl] - ref[s, sl]))
+            assert err <= 2e-3 * np.max(np.abs(ref[s, sl])) + 1e-4, (s, h, err)
+
+
+def test_attention_decode_append_range_error():
+    # a position at max_len: nothing appended for that sequence, zeros out, FG_ERR_RANGE;
+    # the other sequences are appended and attended as usual
+    S, H, d, maxL = 3, 2, 128, 128
+    pos = np.array([5, 128, 127], dtype=np.int32)
+    o, g = _seeded_cache(S, H, d, maxL, np.minimum(pos, maxL), seed=34, group=64)
+    before = [a.clone() for a in g.arrays()]
+    qkv = si.normal_f16(35, 1, (S, 3 * H * d), 1.0)
+    qd = dev(qkv)
+    Hd = H * d
+    out = fg.fg_attention_decode_append(g, qd[:, :Hd], qd[:, Hd:2 * Hd], qd[:, 2 * Hd:], dev(pos))
+    with pytest.raises(fg.FgError, match="RANGE"):
+        fg.fg_sync_status()
+    assert not host(out)[1].any()
+    for a, b in zip(g.arrays(), before):
+        assert torch.equal(a[1].view(torch.uint8), b[1].view(torch.uint8))   # sequence 1 untouched
+    ok = pos < maxL
+    oracle.kv_append(o, qkv[ok, Hd:2 * Hd], qkv[ok, 2 * Hd:], np.arange(S)[ok], pos[ok])
+    for a, b in zip(g.arrays(), o.arrays()):
+        ha = u16(host(a)) if a.dtype == torch.float16 else host(a)
+        assert np.array_equal(ha[[0, 2]], b[[0, 2]])
+
+
 def test_attention_peaked_scores():
     # large query norms make the softmax nearly one-hot: catches masking and max handling
     S, H, d, maxL = 2, 2, 128, 256
