@@ -211,8 +211,10 @@ __device__ __forceinline__ void copy_row(uint32_t *kc, uint32_t *vc, __half *km,
   }
 }
 
-template <int D, int G>
-__global__ void __launch_bounds__(kWarps * 32, D <= 128 ? 5 : 1) attn_decode_kernel(const AttnArgs a) {
+// APP: decode rows that append their new k, v in this launch (fg_attention_decode_append);
+// without it none of the append's state exists.
+template <int D, int G, bool APP>
+__global__ void __launch_bounds__(kWarps * 32, D <= 128 ? 5 : 3) attn_decode_kernel(const AttnArgs a) {
   using S = AttnShape<D, G>;
   constexpr int NG = S::NG, RB = S::RB, KW = S::KW, VW = S::VW, MT = S::MT;
   constexpr float kS24 = 16777216.0f, kS20 = 1048576.0f;
@@ -221,9 +223,10 @@ __global__ void __launch_bounds__(kWarps * 32, D <= 128 ? 5 : 1) attn_decode_ker
   __shared__ float red_m[kWarps], red_l[kWarps];
   __shared__ float red_o[kWarps][D];
   // fused append: the new k, v rows (fp16, copied with the first chunk) and their 4-bit form
-  __shared__ __align__(16) __half new_x[2][D];
-  __shared__ __align__(16) uint32_t new_codes[2][D / 8];
-  __shared__ __half new_meta[4][NG];  // k min, k scale, v min, v scale
+  constexpr int XD = APP ? D : 8, XG = APP ? NG : 1;  // (minimal arrays without the append)
+  __shared__ __align__(16) __half new_x[2][XD];
+  __shared__ __align__(16) uint32_t new_codes[2][XD / 8];
+  __shared__ __half new_meta[4][XG];  // k min, k scale, v min, v scale
   griddep_launch();  // the output projection may start its weight-side prologue
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(kWarps * 32, D <= 128 ? 5 : 1) attn_decode_ker
     const int ntr = (nt + 7) & ~7;  // whole 16-byte metadata rows; stays below max_len (multiple of 64)
     const uint32_t cb = ntr * RB, mb = ntr * NG * 2;
     const uint32_t bar = smem_u32(&full_bar[st]);
-    const bool rows = a.kn != nullptr && ch == 0;  // fused append: the new k, v rows come with chunk 0
+    const bool rows = APP && ch == 0;  // fused append: the new k, v rows come with chunk 0
     mbar_arrive_expect_tx(bar, 2 * cb + 4 * mb + (rows ? 4 * D : 0));
     if (rows) {
       const int64_t o = static_cast<int64_t>(r) * a.ldn + hd * D;
@@ -277,9 +280,8 @@ __global__ void __launch_bounds__(kWarps * 32, D <= 128 ? 5 : 1) attn_decode_ker
   // chunk has landed (the new k, v rows landed with the first chunk), the warp quantises the
   // rows, puts them in place of whatever the copy brought for that row, and stores them to
   // the cache after the loop, when no copy of this kernel still reads it.
-  const bool app = a.kn != nullptr;
   const int tl = (L - 1) % kChunk, app_chunk = (L - 1) / kChunk;
-  const bool app_warp = app && warp == (tl % 64) / 16;
+  const bool app_warp = APP && warp == (tl % 64) / 16;
 
   // ---- q as the B operand of the score MMAs, in the dim order of kword_off ----
   // Word j of lane class c holds, per 16-bit half, nibbles (bits 0-3, 4-7, 8-11, 12-15) =
@@ -339,7 +341,7 @@ __global__ void __launch_bounds__(kWarps * 32, D <= 128 ? 5 : 1) attn_decode_ker
       const __half *Ks = Km + kChunk * NG;
       const __half *Vm = Ks + kChunk * NG;
       const __half *Vs = Vm + kChunk * NG;
-      if (app_warp && ch == app_chunk) {
+      if constexpr (APP) if (app_warp && ch == app_chunk) {
         {
           NewRow<D, G> nr;
           nr.load(new_x[0], new_x[1], lane);
@@ -472,7 +474,7 @@ __global__ void __launch_bounds__(kWarps * 32, D <= 128 ? 5 : 1) attn_decode_ker
     if (tid == 0 && ok && ch + kStages < nchunks) issue(ch + kStages);
   }
 
-  if (app_warp && ok) {  // the new row into the cache (every copy of this kernel has completed)
+  if constexpr (APP) if (app_warp && ok) {  // the new row into the cache (every copy of this kernel has completed)
     const int64_t slot = slot0 + L - 1;
     copy_row<D, NG>(reinterpret_cast<uint32_t *>(const_cast<uint8_t *>(a.kc)) + slot * (D / 8),
                     reinterpret_cast<uint32_t *>(const_cast<uint8_t *>(a.vc)) + slot * (D / 8),
@@ -532,21 +534,26 @@ __global__ void __launch_bounds__(kWarps * 32, D <= 128 ? 5 : 1) attn_decode_ker
   }
 }
 
-template <int D, int G>
-fg_status launch(const AttnArgs &a, cudaStream_t st) {
+template <int D, int G, bool APP>
+fg_status launch_k(const AttnArgs &a, cudaStream_t st) {
   using S = AttnShape<D, G>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     fg_status rc = fg_cuda_check(
-        cudaFuncSetAttribute(attn_decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM));
+        cudaFuncSetAttribute(attn_decode_kernel<D, G, APP>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM));
     if (rc != FG_OK) return rc;
     attr_set[dev] = true;
   }
   const int64_t ctas = static_cast<int64_t>(a.rows) * a.H;
-  attn_decode_kernel<D, G><<<static_cast<unsigned>(ctas), kWarps * 32, S::SMEM, st>>>(a);
+  attn_decode_kernel<D, G, APP><<<static_cast<unsigned>(ctas), kWarps * 32, S::SMEM, st>>>(a);
   return fg_launch_check();
+}
+
+template <int D, int G>
+fg_status launch(const AttnArgs &a, cudaStream_t st) {
+  return a.kn ? launch_k<D, G, true>(a, st) : launch_k<D, G, false>(a, st);
 }
 
 }  // namespace

@@ -366,7 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
 //   shared-memory traffic for 8 MFLOP.
 //   warps 0..7   dequantise (thread: row tid % 128, k half tid / 128), then the epilogue
 //                (warp: TMEM lane quarter warp % 4, token tile warp / 4);
-//   warp 8       TMA of this CTA's x halves, completing on the even CTA's barrier;
+//   warp 8       TMA of this CTA's x halves, completing on the even CTA's barrier, and of this
+//                CTA's packed weights: the codes of each k-tile (128 rows x 32 B, a ring of
+//                kPairCodeStages slots running ahead of the dequant warps) and the fp16 group
+//                mins and scales, 8 group columns at a time (two buffers) -- one tensor copy
+//                each instead of a scattered 16-byte and two 2-byte loads per thread and k-tile;
 //   warp 9       even CTA: the MMA issuer; odd CTA: forwards "A half ready" to the even
 //                CTA (a 16-byte bulk copy completing on its barrier); TMEM allocation.
 //   Split k-ranges of one pair tile form the cluster's z dimension (cluster 2 x 1 x splits);
@@ -377,8 +381,13 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
 constexpr int kPairA = 128 * 128;              // this CTA's A tile: 128 rows x 128 B
 constexpr int kPairBHalf = 128 * 128;          // this CTA's half of one token tile: 128 tokens x 128 B
 constexpr int kPairRing = 192 * 1024;          // pipeline ring (both tile sizes)
-constexpr int kPairSmem = kPairRing + 1024;
-constexpr int kPairPrefetch = 4;
+constexpr int kPairCodeStages = 6;             // k-tiles of codes staged ahead
+constexpr int kPairCodeBytes = 128 * 32;       // one k-tile of this CTA's codes: 128 rows x 32 B
+constexpr int kPairMetaBytes = 128 * 8 * 2;    // 8 group columns of mins (or scales) x 128 rows
+constexpr int kPairCodeOff = kPairRing;
+constexpr int kPairMetaOff = kPairCodeOff + kPairCodeStages * kPairCodeBytes;  // 2 buffers x (mins, scales)
+constexpr int kPairSmem = kPairMetaOff + 4 * kPairMetaBytes + 1024;            // + alignment slack
+static_assert(kPairSmem <= 227 * 1024 - 1024, "shared memory of the pair kernel");
 // NTT 256-token MMA tiles per pair tile: 2 (512 tokens, the A tile feeds two MMAs per k
 // step) or 1 (256 tokens: half the partial sums when the k-range is split, twice the
 // dequantisation per flop)
@@ -399,6 +408,9 @@ constexpr int kPairThreads = (kDeqWarps + 2) * 32;
 
 template <int NTT>
 __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                      const __grid_constant__ CUtensorMap cmap,
+                                                                      const __grid_constant__ CUtensorMap mmap,
+                                                                      const __grid_constant__ CUtensorMap smap,
                                                                       const GemmArgs a) {
   using C = PairCfg<NTT>;
   constexpr int kPairStages = C::kStages, kPairStage = C::kStage, kPairTok = C::kTok, kPairCols = C::kCols;
@@ -414,6 +426,9 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
   __shared__ __align__(8) uint64_t full[kPairStages], a_half[kPairStages], empty[kPairStages], accum_bar;
   __shared__ __align__(16) uint32_t token_src[4], token_sink[kPairStages][4];
   __shared__ __align__(8) uint64_t recv_bar;  // split-k epilogue: this rank's received partials
+  // staged weights: code_full (TMA) / code_empty (the 8 dequant warps have read the slot);
+  // meta_full / meta_empty likewise for the two metadata buffers
+  __shared__ __align__(8) uint64_t code_full[kPairCodeStages], code_empty[kPairCodeStages], meta_full[2], meta_empty[2];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -443,6 +458,14 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     }
     mbar_init(smem_u32(&accum_bar), 1);
     mbar_init(smem_u32(&recv_bar), 1);
+    for (int i = 0; i < kPairCodeStages; i++) {
+      mbar_init(smem_u32(&code_full[i]), 1);
+      mbar_init(smem_u32(&code_empty[i]), kDeqWarps);
+    }
+    for (int i = 0; i < 2; i++) {
+      mbar_init(smem_u32(&meta_full[i]), 1);
+      mbar_init(smem_u32(&meta_empty[i]), kDeqWarps);
+    }
     abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -456,72 +479,84 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
 
+  // metadata column group (8 group columns) of k-tile kt, relative to the first one of the range
+  const int sj0 = (kt0 >> a.gshift) >> 3;
+  auto meta_unit = [&](int kt) { return ((kt >> a.gshift) >> 3) - sj0; };
   if (warp < kDeqWarps) {
     // ---------------- dequantise producer: row tid % 128, k half tid / 128 ----------------
     const int row = tid & 127, hk = tid >> 7;
-    const int n = n0 + row;
-    const bool live = n < a.N;
-    const uint4 *crow = reinterpret_cast<const uint4 *>(a.wc + static_cast<int64_t>(live ? n : 0) * (a.K / 2));
-    const __half *mrow = a.wm + static_cast<int64_t>(live ? n : 0) * ((a.K / kBK) >> a.gshift);
-    const __half *srow = a.ws + static_cast<int64_t>(live ? n : 0) * ((a.K / kBK) >> a.gshift);
-    uint4 cb[kPairPrefetch];
-    __half mb[kPairPrefetch], sb[kPairPrefetch];
-#pragma unroll
-    for (int j = 0; j < kPairPrefetch; j++) {
-      if (j < nk && live) {
-        cb[j] = crow[(kt0 + j) * 2 + hk];
-        mb[j] = mrow[(kt0 + j) >> a.gshift];
-        sb[j] = srow[(kt0 + j) >> a.gshift];
-      } else {
-        cb[j] = make_uint4(0, 0, 0, 0);
-        mb[j] = sb[j] = __ushort_as_half(0);
-      }
-    }
-    // leader: arrive on its own full barrier; odd CTA: on a_half, forwarded by warp 9.
-    // The prefetched codes sit in a ring indexed statically (the loop is unrolled by the
-    // prefetch depth): k-tile i's codes are consumed in place, and the slot is refilled
-    // with those of k-tile i + kPairPrefetch.  Shifting the array down instead would move
-    // registers whose loads are still in flight, and each move waits for its load.
+    const bool live = n0 + row < a.N;
+    int cur_u = -1;
+    // leader: arrive on its own full barrier; odd CTA: on a_half, forwarded by warp 9
     const uint32_t done_bar0 = smem_u32(leader ? &full[0] : &a_half[0]);
-    bool go = true;
-    for (int i0 = 0; go && i0 < nk; i0 += kPairPrefetch) {
-#pragma unroll
-      for (int j = 0; j < kPairPrefetch; j++) {
-        const int i = i0 + j;
-        if (!go || i >= nk) break;
-        const int st = i % kPairStages;
-        const uint4 c0 = cb[j];
-        const __half m0 = mb[j], s0 = sb[j];
-        if (i + kPairPrefetch < nk && live) {
-          const int kt = kt0 + i + kPairPrefetch;
-          cb[j] = crow[kt * 2 + hk];
-          mb[j] = mrow[kt >> a.gshift];
-          sb[j] = srow[kt >> a.gshift];
-        }
-        if (i >= kPairStages &&
-            !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kPairStages) - 1) & 1, abortp, a.err)) {
-          go = false;
-          break;
-        }
-        const __half2 s2 = __half2half2(s0), m2 = __half2half2(m0);
-        uint8_t *at = a_tile(st);
-        const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
-#pragma unroll
-        for (int c = 0; c < 4; c++) {
-          const uint4 v = live ? dequant8(words[c], s2, m2) : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4 *>(at + sw128_offset(row, 4 * hk + c)) = v;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(done_bar0 + st * 8);
+    for (int i = 0; i < nk; i++) {
+      const int st = i % kPairStages, cs = i % kPairCodeStages;
+      if (!mbar_wait_bounded(smem_u32(&code_full[cs]), (i / kPairCodeStages) & 1, abortp, a.err)) break;
+      const uint4 c0 = *reinterpret_cast<const uint4 *>(smem + kPairCodeOff + cs * kPairCodeBytes + row * 32 + hk * 16);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&code_empty[cs]));  // the slot may be refilled
+      const int mi = (kt0 + i) >> a.gshift, u = meta_unit(kt0 + i);
+      if (u != cur_u) {  // warp-uniform
+        if (cur_u >= 0 && lane == 0) mbar_arrive(smem_u32(&meta_empty[cur_u & 1]));  // read by every lane above
+        if (!mbar_wait_bounded(smem_u32(&meta_full[u & 1]), (u >> 1) & 1, abortp, a.err)) break;
+        cur_u = u;
       }
+      const __half *mb = reinterpret_cast<const __half *>(smem + kPairMetaOff + (u & 1) * 2 * kPairMetaBytes);
+      const __half m0 = mb[row * 8 + (mi & 7)], s0 = mb[kPairMetaBytes / 2 + row * 8 + (mi & 7)];
+      if (i >= kPairStages &&
+          !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kPairStages) - 1) & 1, abortp, a.err))
+        break;
+      const __half2 s2 = __half2half2(s0), m2 = __half2half2(m0);
+      uint8_t *at = a_tile(st);
+      const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
+#pragma unroll
+      for (int c = 0; c < 4; c++) {
+        const uint4 v = live ? dequant8(words[c], s2, m2) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(at + sw128_offset(row, 4 * hk + c)) = v;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(done_bar0 + st * 8);
     }
   } else if (warp == kTmaWarp) {
     // ---------------- TMA producer: this CTA's halves of the two token tiles ----------------
     if (lane == 0) {
       prefetch_tmap(&xmap);
-      griddep_wait();  // x comes from the previous kernel
-      for (int i = 0; i < nk; i++) {
+      prefetch_tmap(&cmap);
+      prefetch_tmap(&mmap);
+      prefetch_tmap(&smap);
+      // this CTA's codes and metadata for k-tiles jc < jmax (and the metadata column group
+      // each first needs), into slots the dequant warps have released
+      int jc = 0, um = 0;
+      bool ok = true;
+      auto feed = [&](int jmax) {
+        for (; ok && jc < jmax && jc < nk; jc++) {
+          if (meta_unit(kt0 + jc) == um) {
+            if (um >= 2 && !mbar_wait_bounded(smem_u32(&meta_empty[um & 1]), ((um >> 1) - 1) & 1, abortp, a.err)) {
+              ok = false;
+              break;
+            }
+            const uint32_t mbar = smem_u32(&meta_full[um & 1]);
+            uint8_t *mb = smem + kPairMetaOff + (um & 1) * 2 * kPairMetaBytes;
+            mbar_arrive_expect_tx(mbar, 2 * kPairMetaBytes);
+            tma_load_2d(smem_u32(mb), &mmap, (sj0 + um) * 8, n0, mbar);
+            tma_load_2d(smem_u32(mb + kPairMetaBytes), &smap, (sj0 + um) * 8, n0, mbar);
+            um++;
+          }
+          const int cs = jc % kPairCodeStages;
+          if (jc >= kPairCodeStages &&
+              !mbar_wait_bounded(smem_u32(&code_empty[cs]), ((jc / kPairCodeStages) - 1) & 1, abortp, a.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t cbar = smem_u32(&code_full[cs]);
+          mbar_arrive_expect_tx(cbar, kPairCodeBytes);
+          tma_load_2d(smem_u32(smem + kPairCodeOff + cs * kPairCodeBytes), &cmap, (kt0 + jc) * 32, n0, cbar);
+        }
+      };
+      feed(kPairCodeStages);  // the weights are fixed for the call: before the dependency wait
+      griddep_wait();         // x comes from the previous kernel
+      for (int i = 0; ok && i < nk; i++) {
         const int st = i % kPairStages;
         if (i >= kPairStages &&
             !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kPairStages) - 1) & 1, abortp, a.err))
@@ -531,6 +566,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
 #pragma unroll
         for (int tile = 0; tile < NTT; tile++)
           tma_load_2d_pair(smem_u32(b_tile(st, tile)), &xmap, (kt0 + i) * kBK, t0 + tile * 256 + half * 128, fb);
+        feed(i + 1 + kPairCodeStages);
       }
     }
   } else if (!leader) {
@@ -1063,7 +1099,7 @@ Plan make_pair_plan(int M, int N, int K) {
 }
 
 template <int NTT>
-fg_status launch_pair_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st, bool pdl) {
+fg_status launch_pair_nt(const CUtensorMap (&maps)[4], const GemmArgs &a, const Plan &p, cudaStream_t st, bool pdl) {
   fg_status rc = pair_attr_once<NTT>();
   if (rc != FG_OK) return rc;
   cudaLaunchConfig_t lc = {};
@@ -1080,13 +1116,13 @@ fg_status launch_pair_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = pdl ? 2 : 1;
-  rc = fg_cuda_check(cudaLaunchKernelEx(&lc, w4a16_gemm_pair_kernel<NTT>, map, a));
+  rc = fg_cuda_check(cudaLaunchKernelEx(&lc, w4a16_gemm_pair_kernel<NTT>, maps[0], maps[1], maps[2], maps[3], a));
   if (rc != FG_OK) return rc;
   return fg_launch_check();
 }
 
-fg_status launch_pair(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cudaStream_t st, bool pdl) {
-  return p.nt == 256 ? launch_pair_nt<1>(map, a, p, st, pdl) : launch_pair_nt<2>(map, a, p, st, pdl);
+fg_status launch_pair(const CUtensorMap (&maps)[4], const GemmArgs &a, const Plan &p, cudaStream_t st, bool pdl) {
+  return p.nt == 256 ? launch_pair_nt<1>(maps, a, p, st, pdl) : launch_pair_nt<2>(maps, a, p, st, pdl);
 }
 
 // Test hook state (fg_test_gemm_stall): launches of the one-SM kernel still to stall, and
@@ -1114,19 +1150,49 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
                            void *workspace, size_t ws_bytes, cudaStream_t st, bool pdl) {
   const int N = static_cast<int>(w->shape[0]);
   if (M == 0) return FG_OK;
-  const bool pair = M > 256;
-  Plan p = pair ? make_pair_plan(M, N, K) : make_plan(M, N, K);
+  const int G = w->group == 128 ? 128 : 64;
+  // M > 256: CTA pairs.  The classic pair kernel stages the group metadata by tensor copies of
+  // 8 group columns, so a row of K/G fp16 values must be whole 16-byte units and the arrays
+  // 16-byte aligned; otherwise (and for M <= 256) the one-SM kernel runs.
+  const bool big = M > 256;
+  const Plan pp = big ? make_pair_plan(M, N, K) : Plan{};
+  const bool sk = big && (flags & FG_GEMM_PERSISTENT) && pp.pairs > 0 && workspace && fg_aligned16(workspace) &&
+                  ws_bytes >= fg_streamk_scratch_bytes(pp.pairs);
+  const bool pair = big && !sk && (K / G) % 8 == 0 && fg_aligned16(w->mins) && fg_aligned16(w->scales);
+  const Plan p = (sk || pair) ? pp : make_plan(M, N, K);
   EncodeTiledFn enc = encode_fn();
   if (!enc) return FG_ERR_CUDA;
-  CUtensorMap map;
+  CUtensorMap maps[4];  // x, and for the classic pair kernel the codes, mins and scales
+  CUtensorMap &map = maps[0];
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t box[2] = {kBK, static_cast<cuuint32_t>(pair ? 128 : p.nt)};
+  const cuuint32_t box[2] = {kBK, static_cast<cuuint32_t>((sk || pair) ? 128 : p.nt)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<fg_half *>(x), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return FG_ERR_INVALID;
+  if (pair) {
+    // codes [N][K/2] bytes, box 32 B (one k-tile) x 128 rows; mins, scales [N][K/G] fp16,
+    // box 8 columns x 128 rows
+    const cuuint64_t cdims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
+    const cuuint64_t cstr[1] = {static_cast<cuuint64_t>(K / 2)};
+    const cuuint32_t cbox[2] = {32, 128};
+    cr = enc(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(w->codes), cdims, cstr, cbox, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return FG_ERR_INVALID;
+    const cuuint64_t mdims[2] = {static_cast<cuuint64_t>(K / G), static_cast<cuuint64_t>(N)};
+    const cuuint64_t mstr[1] = {static_cast<cuuint64_t>(K / G) * 2};
+    const cuuint32_t mbox[2] = {8, 128};
+    const void *meta[2] = {w->mins, w->scales};
+    for (int j = 0; j < 2; j++) {
+      cr = enc(&maps[2 + j], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(meta[j]), mdims, mstr, mbox, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (cr != CUDA_SUCCESS) return FG_ERR_INVALID;
+    }
+  }
   GemmArgs a;
   a.wc = w->codes;
   a.wm = reinterpret_cast<const __half *>(w->mins);
@@ -1149,11 +1215,10 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
   if (!a.err) return FG_ERR_CUDA;
   a.wait_ns = FG_WAIT_TIMEOUT_NS;
   a.stall = 0;
-  if (pair && (flags & FG_GEMM_PERSISTENT) && p.pairs > 0 && workspace && fg_aligned16(workspace) &&
-      ws_bytes >= fg_streamk_scratch_bytes(p.pairs))
+  if (sk)
     return fg_streamk_launch(map, a.wc, a.wm, a.ws, a.gshift, a.bias, a.res, a.relu, a.qcols, a.qscale, a.y, M, N, K,
                              p.pairs, workspace, a.err, st, pdl);
-  if (pair) return launch_pair(map, a, p, st, pdl);
+  if (pair) return launch_pair(maps, a, p, st, pdl);
   int left = g_stall_count.load();
   while (left > 0 && !g_stall_count.compare_exchange_weak(left, left - 1)) {
   }
@@ -1184,6 +1249,11 @@ extern "C" fg_status fg_linear_plan(int M, int N, int K, int *tile_tokens, int *
   Plan p;
   if (M > 256) {
     p = make_pair_plan(M, N, K);
+    if ((K / 64) % 8) {  // the classic launch for groups of 64 runs one SM per tile here
+      const int pairs = p.pairs;
+      p = make_plan(M, N, K);
+      p.pairs = pairs;
+    }
   } else {
     p = make_plan(M, N, K);
     p.pairs = 0;

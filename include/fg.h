@@ -196,7 +196,10 @@ enum {
  * dequantisation for FP16 compute).
  * Launches (see fg_linear_plan): M <= 256 runs one SM per output tile; larger M
  * runs on CTA pairs: the classic launch (one pair per tile, k-range optionally
- * split over a cluster), or, with FG_GEMM_PERSISTENT in flags, the persistent
+ * split over a cluster; it stages the weights' codes and group metadata by
+ * tensor copies, so it needs (K / group) % 8 == 0 and the mins and scales
+ * 16-byte aligned, else the one-SM launch runs), or, with FG_GEMM_PERSISTENT in
+ * flags, the persistent
  * launch (every resident pair takes an equal share of the tiles' k-iterations; a
  * tile shared between pairs is finished by the pair holding its first
  * k-segment).  The layer calls use the classic launch.
@@ -211,8 +214,10 @@ enum {
  * from the classic launch's in the last bits (each is deterministic). */
 FG_API size_t fg_linear_workspace_bytes(int M, int N, int K);
 /* The launches fg_linear_w4a16 makes for this shape on the current device (no
- * launch): the classic launch's *tile_tokens = tokens per output tile (16..256
- * for M <= 256, one SM per tile; 256 or 512 for larger M, a CTA pair per tile)
+ * launch; weights in groups of 64 with 16-byte aligned metadata): the classic
+ * launch's *tile_tokens = tokens per output tile (16..256 for M <= 256, or K
+ * not a multiple of 512, one SM per tile; 256 or 512 for larger M, a CTA pair
+ * per tile)
  * and *splits = CTAs sharing each tile's k-range (1..8 one-SM, 1..4 pair),
  * chosen by a time model of the kernels: waves of resident clusters x k-tiles
  * per CTA, plus the pipeline fill and the epilogue; *pairs = CTA pairs of the
