@@ -297,13 +297,15 @@ def fg_linear_plan_pairs(M: int, N: int, K: int) -> int:
     return p.value
 
 
-def fg_linear_classic_scratch_bytes(M: int, N: int, K: int) -> int:
+def fg_linear_classic_scratch_bytes(M: int, N: int, K: int, flags: bool = True) -> int:
     """Scratch the classic launch's split k-range adds its partial sums through (0 without a
-    split); with less than that (and less than fg_linear_workspace_bytes) it adds them on chip."""
+    split): the fp32 partials and, with flags, the flags that let the split ranks run as
+    separate clusters; with less than the partials it adds them on chip."""
     t, s = fg_linear_plan(M, N, K)
     if M <= 256 or s < 2:
         return 0
-    return -(-N // 256) * -(-M // t) * s * t * 256 * 4
+    tiles = -(-N // 256) * -(-M // t)
+    return tiles * s * t * 256 * 4 + (tiles * s * 2 * 8 if flags else 0)
 
 
 def fg_linear_w4a16(x: torch.Tensor, w: QTensor, bias=None, residual=None, relu: bool = False,

@@ -76,6 +76,9 @@ struct GemmArgs {
   int splits;
   int gshift;          // log2(group / 64): the weights' min/scale cover 1 (group 64) or 2 (128) k-tiles
   float *part;         // pair kernel, k split: fp32 partial sums through global memory, or null
+  unsigned long long *flags;  // with part: the split ranks are separate clusters (one wave) that
+                              // publish their partials with these [tile][rank][CTA half] flags
+  unsigned long long epoch;   // the launch's flag value
   unsigned int *err;
   uint64_t wait_ns;    // one-SM kernel: limit of every pipeline wait (FG_WAIT_TIMEOUT_NS unless a test shortens it)
   int stall;           // one-SM kernel, test hook: the dequantising warps withhold their first-stage arrival
@@ -720,10 +723,10 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     // reduction below does, and finishes the chunk.  One barrier instead of a chain of
     // rounds of distributed-shared-memory copies.
     constexpr int kChunks = kPairCols / 32;
-    const int S = a.splits, zrank = static_cast<int>(crank >> 1);
+    const int S = a.splits, zrank = static_cast<int>(blockIdx.z);
     constexpr int64_t kTileFloats = static_cast<int64_t>(kPairTok) * 256;
-    const float *tilep =
-        a.part + (static_cast<int64_t>(blockIdx.y) * (gridDim.x / 2) + blockIdx.x / 2) * S * kTileFloats;
+    const int64_t tile = static_cast<int64_t>(blockIdx.y) * (gridDim.x / 2) + blockIdx.x / 2;
+    const float *tilep = a.part + tile * S * kTileFloats;
     if (warp < kDeqWarps && ready) {
       float *mine = const_cast<float *>(tilep) + zrank * kTileFloats + half * 128 + q * 32 + lane;
       for (int c8 = 0; c8 < kChunks / 2; c8++) {
@@ -736,7 +739,32 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
       }
     }
     __threadfence();
-    cluster_sync_all();
+    if (a.flags) {
+      // The split ranks are separate clusters, all resident (the launch takes this form only
+      // when the grid is one wave): publish this CTA's partial, then wait for the other ranks'
+      // partials of the same tile half (bounded; a timeout flags FG_ERR_TIMEOUT and skips the sum).
+      __syncthreads();
+      unsigned long long *fl = a.flags + tile * S * 2 + half;  // [tile][rank][half]
+      if (tid == 0) {
+        st_release_u64(fl + 2 * zrank, a.epoch);
+        for (int z = 0; z < S && !*abortp; z++) {
+          if (z == zrank) continue;
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_u64(fl + 2 * z) != a.epoch) {
+            if (globaltimer_ns() - t0 > FG_WAIT_TIMEOUT_NS) {
+              atomicOr(a.err, FG_DEVERR_TIMEOUT);
+              *abortp = 1;
+              break;
+            }
+            __nanosleep(64);
+          }
+        }
+      }
+      __syncthreads();
+      ready = ready && !*abortp;
+    } else {
+      cluster_sync_all();
+    }
     if (warp < kDeqWarps && ready && nb < a.N) {
       float bias[8];
 #pragma unroll
@@ -1065,11 +1093,14 @@ Plan make_pair_plan(int M, int N, int K) {
     const int t_tiles = (M + tok - 1) / tok;
     const int clusters = p.n_tiles * t_tiles;
     const double ktime = ntt == 2 ? 0.70 : 0.63;
+    const int one = ntt == 2 ? pair_clusters_resident<2>(1) : pair_clusters_resident<1>(1);
     for (int s = 1; s <= 4; s++) {
       if (s > 1 && ktiles / s < 8) break;
       const int resident = ntt == 2 ? pair_clusters_resident<2>(s) : pair_clusters_resident<1>(s);
       if (resident == 0) continue;
-      const int waves = (clusters + resident - 1) / resident;
+      // a split grid that fits one wave of single-pair clusters runs its ranks as separate
+      // clusters (given the scratch fg_linear_workspace_bytes asks for): one wave
+      const int waves = (s > 1 && clusters * s <= one) ? 1 : (clusters + resident - 1) / resident;
       const double epi = 3.0 * ntt + (s > 1 ? 4.0 * ntt + 1.0 * s : 0.0);
       const double cost = waves * (((ktiles + s - 1) / s) * ktime + 5.0 + epi);
       if (cost < best - 1e-9) {
@@ -1111,7 +1142,7 @@ fg_status launch_pair_nt(const CUtensorMap (&maps)[4], const GemmArgs &a, const 
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = p.splits;
+  attr[0].val.clusterDim.z = a.flags ? 1 : p.splits;  // split ranks: one cluster, or flags
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
@@ -1128,6 +1159,8 @@ fg_status launch_pair(const CUtensorMap (&maps)[4], const GemmArgs &a, const Pla
 // Test hook state (fg_test_gemm_stall): launches of the one-SM kernel still to stall, and
 // their wait limit.
 std::atomic<int> g_stall_count{0};
+// Launch counter behind the split-rank flags' values (tagged apart from the stream-K kernel's).
+std::atomic<unsigned long long> g_split_epoch{0};
 std::atomic<uint64_t> g_stall_wait_ns{FG_WAIT_TIMEOUT_NS};
 
 }  // namespace
@@ -1137,11 +1170,15 @@ std::atomic<uint64_t> g_stall_wait_ns{FG_WAIT_TIMEOUT_NS};
 static size_t pair_part_bytes(const Plan &p) {
   return p.splits < 2 ? 0 : static_cast<size_t>(p.n_tiles) * p.t_tiles * p.splits * p.nt * 256 * sizeof(float);
 }
+// ... and the flags of the split ranks run as separate clusters: [tile][rank][CTA half]
+static size_t pair_flag_bytes(const Plan &p) {
+  return p.splits < 2 ? 0 : static_cast<size_t>(p.n_tiles) * p.t_tiles * p.splits * 2 * sizeof(unsigned long long);
+}
 
 size_t fg_linear_ws_bytes(int M, int N, int K) {
   if (M <= 256 || N <= 0 || K <= 0 || K % kBK) return 0;
   const Plan p = make_pair_plan(M, N, K);
-  const size_t classic = pair_part_bytes(p), sk = p.pairs > 0 ? fg_streamk_scratch_bytes(p.pairs) : 0;
+  const size_t classic = pair_part_bytes(p) + pair_flag_bytes(p), sk = p.pairs > 0 ? fg_streamk_scratch_bytes(p.pairs) : 0;
   return classic > sk ? classic : sk;
 }
 
@@ -1209,8 +1246,19 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
   a.splits = p.splits;
   a.gshift = w->group == 128 ? 1 : 0;
   a.part = nullptr;
-  if (pair && p.splits > 1 && workspace && fg_aligned16(workspace) && ws_bytes >= pair_part_bytes(p))
+  a.flags = nullptr;
+  a.epoch = 0;
+  if (pair && p.splits > 1 && workspace && fg_aligned16(workspace) && ws_bytes >= pair_part_bytes(p)) {
     a.part = static_cast<float *>(workspace);
+    // With room for the flags and the whole grid resident at once (clusters of one pair), the
+    // split ranks run as separate clusters and meet through the flags: no cluster of 2 x splits
+    // CTAs, which the GPCs may not hold in one wave.
+    const int one = p.nt == 256 ? pair_clusters_resident<1>(1) : pair_clusters_resident<2>(1);
+    if (ws_bytes >= pair_part_bytes(p) + pair_flag_bytes(p) && p.n_tiles * p.t_tiles * p.splits <= one) {
+      a.flags = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + pair_part_bytes(p));
+      a.epoch = 0xF6A4000000000000ull | (g_split_epoch.fetch_add(1) + 1);
+    }
+  }
   a.err = fg_error_word_ptr();
   if (!a.err) return FG_ERR_CUDA;
   a.wait_ns = FG_WAIT_TIMEOUT_NS;

@@ -81,14 +81,6 @@ struct SkArgs {
 
 __device__ __forceinline__ int64_t range_begin(const SkArgs &a, int p) { return static_cast<int64_t>(p) * a.iters / a.P; }
 
-__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
 // Barrier among the epilogue warps only (named barrier 1; the non-aligned form, so a lane that
 // polled alone may arrive apart from its warp).
 __device__ __forceinline__ void epi_sync() { asm volatile("barrier.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); }

@@ -545,8 +545,13 @@ def test_linear_split_k_deterministic(M, N, K):
         assert torch.equal(y1, y3)
         cb = fg.fg_linear_classic_scratch_bytes(M, N, K)
         if cb:
+            # partials and flags (split ranks as separate clusters when the grid is one wave),
+            # and partials only (split ranks in one cluster): the same bits again
             y4 = fg.fg_linear_w4a16(x, wq, workspace=torch.empty(cb, dtype=torch.uint8, device="cuda"))
             assert torch.equal(y1, y4)
+            cp = fg.fg_linear_classic_scratch_bytes(M, N, K, flags=False)
+            y5 = fg.fg_linear_w4a16(x, wq, workspace=torch.empty(cp, dtype=torch.uint8, device="cuda"))
+            assert torch.equal(y1, y5)
 
 
 @pytest.mark.parametrize("M,N,K", [(520, 4096, 4096), (600, 7680, 1024), (530, 5120, 1536), (512, 4096, 16384)])
@@ -566,11 +571,17 @@ def test_linear_split_k_residual_sampled(M, N, K):
         assert fg.fg_linear_workspace_bytes(M, N, K) > 0        # these shapes split the k-range
     outs = [y1]
     if fg.fg_linear_classic_scratch_bytes(M, N, K):
-        # partial sums through the scratch (above) or, with too little scratch, on chip over
-        # distributed shared memory: the same order of additions, the same bits
+        # partial sums through the scratch (above: the split ranks as separate clusters meeting
+        # through flags when the grid is one wave), through the scratch within one cluster, or,
+        # with too little scratch, on chip over distributed shared memory: the same order of
+        # additions, the same bits
         y3 = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), residual=dev(r),
                                 workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
         assert torch.equal(y1, y3)
+        cp = fg.fg_linear_classic_scratch_bytes(M, N, K, flags=False)
+        y4 = fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), residual=dev(r),
+                                workspace=torch.empty(cp, dtype=torch.uint8, device="cuda"))
+        assert torch.equal(y1, y4)
     if fg.fg_linear_plan_pairs(M, N, K) > 0:
         outs.append(fg.fg_linear_w4a16(dev(x), wq, bias=dev(b), residual=dev(r), persistent=True))
     rows = np.unique(np.concatenate([np.random.default_rng(M).choice(M, 20, replace=False), [0, 255, 256, 511, M - 1]]))
