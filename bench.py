@@ -435,7 +435,10 @@ def run_ours(args, wl):
     # ---- roofline of the dominant kernel (and of every kernel) ----
     peaks = load_peaks()
     L_avg = P + (args.warmup + (args.steps - 1) / 2.0) % nsteps_cfg + 1
-    work, totals = kernel_work(wl, S, L_avg, G)
+    # the layer appends decode rows inside the attention kernel only when its (row, head) CTAs
+    # are at most 4 per SM (launch-bound); larger blocks take the separate append kernel
+    fused = S * wl["heads"] <= 4 * torch.cuda.get_device_properties(dev).multi_processor_count
+    work, totals = kernel_work(wl, S, L_avg, G, fused_append=fused)
     kernels = {}
     for name, (tot_ms, cnt) in prof.items():
         if cnt == 0:

@@ -19,7 +19,7 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
 size_t fg_linear_ws_bytes(int M, int N, int K);
 fg_status fg_kv_validate(const fg_kv_cache *kv);
 fg_status fg_kv_append_launch(const fg_kv_cache *kv, const fg_half *k, const fg_half *v, int64_t ld, int rows,
-                              int rows_per_seq, const int32_t *positions, cudaStream_t st);
+                              int rows_per_seq, const int32_t *positions, cudaStream_t st, bool pdl);
 fg_status fg_attention_launch(const fg_kv_cache *kv, const fg_half *q, int64_t ldq, fg_half *out, int64_t ldo,
                               int rows, int rows_per_seq, const int32_t *positions, cudaStream_t st,
                               const fg_half *k_new, const fg_half *v_new, int64_t ld_new);
@@ -183,7 +183,7 @@ fg_status run_layer(const fg_layer_config *c, const fg_layer_weights *w, const f
   if (fuse) {
     FG_STEP(3, fg_attention_launch(kv, qkv, 3 * h, o, h, rows, 1, positions, st, qkv + h, qkv + 2 * h, 3 * h));
   } else {
-    FG_STEP(2, fg_kv_append_launch(kv, qkv + h, qkv + 2 * h, 3 * h, rows, rows_per_seq, positions, st));
+    FG_STEP(2, fg_kv_append_launch(kv, qkv + h, qkv + 2 * h, 3 * h, rows, rows_per_seq, positions, st, pdl));
     FG_STEP(3, fg_attention_launch(kv, qkv, 3 * h, o, h, rows, rows_per_seq, positions, st, nullptr, nullptr, 0));
   }
   FG_SLICE(slice_done(sl, 2, st));

@@ -190,6 +190,9 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __half *__restrict
   // A warp takes one (row, head) item per step: its 2 * d/G units (k and v groups), USTEP at
   // a time in its G/8-lane slots; unit us = group * 2 + (0 for k, 1 for v).
   constexpr int L = G / 8, USTEP = 32 / L;
+  // launched as a dependent of the GEMM that produces k and v (decode steps): they are read
+  // only once it has completed
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int slot = lane / L, j = lane % L;
   const int ng = a.d / G;
@@ -351,8 +354,10 @@ fg_status fg_kv_validate(const fg_kv_cache *kv) {
   return FG_OK;
 }
 
+// pdl: launch as a programmatic dependent of the kernel before (its launch overlaps that
+// kernel's tail; the kernel waits for it before reading k and v).
 fg_status fg_kv_append_launch(const fg_kv_cache *kv, const fg_half *k, const fg_half *v, int64_t ld, int rows,
-                              int rows_per_seq, const int32_t *positions, cudaStream_t st) {
+                              int rows_per_seq, const int32_t *positions, cudaStream_t st, bool pdl) {
   KvArgs a;
   a.kc = reinterpret_cast<uint32_t *>(kv->k_codes);
   a.vc = reinterpret_cast<uint32_t *>(kv->v_codes);
@@ -369,9 +374,19 @@ fg_status fg_kv_append_launch(const fg_kv_cache *kv, const fg_half *k, const fg_
   const int64_t items = static_cast<int64_t>(rows) * kv->num_heads;  // one warp per (row, head)
   if (items > INT32_MAX) return FG_ERR_SHAPE;
   auto kern = fg_kv_group(kv->group) == 128 ? kv_append_kernel<128> : kv_append_kernel<64>;
-  kern<<<grid_for((items + 7) / 8, 8), 256, 0, st>>>(reinterpret_cast<const __half *>(k),
-                                                     reinterpret_cast<const __half *>(v), ld, rows, rows_per_seq,
-                                                     positions, a, err);
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(grid_for((items + 7) / 8, 8), 1, 1);
+  lc.blockDim = dim3(256, 1, 1);
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = pdl ? 1 : 0;
+  const fg_status rc = fg_cuda_check(cudaLaunchKernelEx(&lc, kern, reinterpret_cast<const __half *>(k),
+                                                        reinterpret_cast<const __half *>(v), ld, rows, rows_per_seq,
+                                                        positions, a, err));
+  if (rc != FG_OK) return rc;
   return fg_launch_check();
 }
 
@@ -384,5 +399,5 @@ extern "C" fg_status fg_kv_append(const fg_kv_cache *kv, const fg_half *k, const
   if (rows == 0) return FG_OK;
   if (!k || !v || !positions || !fg_aligned16(k) || !fg_aligned16(v)) return FG_ERR_INVALID;
   if (ld < static_cast<int64_t>(kv->num_heads) * kv->head_dim || ld % 8) return FG_ERR_SHAPE;
-  return fg_kv_append_launch(kv, k, v, ld, rows, rows_per_seq, positions, static_cast<cudaStream_t>(stream));
+  return fg_kv_append_launch(kv, k, v, ld, rows, rows_per_seq, positions, static_cast<cudaStream_t>(stream), false);
 }

@@ -30,6 +30,9 @@ def test_opt6p7b_decode_step_work(bench):
     # 1.208 GB of KV4 read, q in and o out, and the fused append: k, v in, their codes out
     assert att == S * H * 512 * 144 + 2 * S * h * 2 + 2 * S * h * 2 + S * H * 144
     assert work["kv_append"][1] == S * 2 * h * 2 + S * 2 * (h // 2 + h // 16)
+    # a block this large appends in its own kernel: the attention reads the cache, q and o only
+    work, _ = bench.kernel_work(wl, S, 512, fused_append=False)
+    assert work["attention"][1] == S * H * 512 * 144 + 2 * S * h * 2
     units = bench.kernel_units(wl, S, 512)
     assert units["attention"] == S * H * 512            # traffic of a smaller capture scales by these
 
