@@ -63,6 +63,10 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_quantize_g.argtypes = [P, I64, I64, I64, P, P, P, I]
         _lib.oracle_dequantize_g.restype = I
         _lib.oracle_dequantize_g.argtypes = [P, P, P, I64, I64, I64, P, I]
+        _lib.oracle_quantize_gb.restype = I
+        _lib.oracle_quantize_gb.argtypes = [P, I64, I64, I64, P, P, P, I, I]
+        _lib.oracle_dequantize_gb.restype = I
+        _lib.oracle_dequantize_gb.argtypes = [P, P, P, I64, I64, I64, P, I, I]
         _lib.oracle_linear_g.restype = I
         _lib.oracle_linear_g.argtypes = [P, I, I, P, P, P, I, P, P, I, I, D, P, I]
         _lib.oracle_layernorm.restype = I
@@ -112,11 +116,12 @@ def f64_to_f16(x) -> np.ndarray:
 # --------------------------------------------------------------------------------------
 
 class Packed:
-    """Planar 4-bit tensor: codes uint8 (dim halved), mins/scales float16 (dim / group)."""
+    """Planar quantised tensor: codes uint8 (dim x bits / 8: two 4-bit codes or one 8-bit code
+    per byte), mins/scales float16 (dim / group)."""
 
-    def __init__(self, codes, mins, scales, shape, dim, group: int = GROUP):
+    def __init__(self, codes, mins, scales, shape, dim, group: int = GROUP, bits: int = 4):
         self.codes, self.mins, self.scales = codes, mins, scales
-        self.shape, self.dim, self.group = tuple(shape), dim, group
+        self.shape, self.dim, self.group, self.bits = tuple(shape), dim, group, bits
 
 
 def _split(shape, dim):
@@ -126,30 +131,34 @@ def _split(shape, dim):
     return dim, outer, int(shape[dim]), inner
 
 
-def quantize(x, dim: int = -1, group: int = GROUP) -> Packed:
-    """Group-wise asymmetric min-max 4-bit quantisation along ``dim``, groups of 64 or 128
-    consecutive elements ("FlexGen Guide", section 3: groups of 64 or 128)."""
+def quantize(x, dim: int = -1, group: int = GROUP, bits: int = 4) -> Packed:
+    """Group-wise asymmetric min-max quantisation along ``dim``, groups of 64 or 128
+    consecutive elements ("FlexGen Guide", section 3: 4 bits, groups of 64 or 128); bits = 8
+    is the same scheme with 255 steps (INT8 among the post-training formats of the
+    "Optimizing LLM for low memory usage" page)."""
     x = _u16(x)
     dim, outer, n, inner = _split(x.shape, dim)
     if group not in (64, 128):
         raise ValueError("group must be 64 or 128")
+    if bits not in (4, 8):
+        raise ValueError("bits must be 4 or 8")
     if n % group:
         raise ValueError(f"size along dim must be a multiple of {group}")
-    cshape = list(x.shape); cshape[dim] = n // 2
+    cshape = list(x.shape); cshape[dim] = n * bits // 8
     mshape = list(x.shape); mshape[dim] = n // group
     codes = np.empty(cshape, dtype=np.uint8)
     mins = np.empty(mshape, dtype=np.uint16)
     scales = np.empty(mshape, dtype=np.uint16)
-    rc = lib().oracle_quantize_g(_p(x), outer, n, inner, _p(codes), _p(mins), _p(scales), group)
+    rc = lib().oracle_quantize_gb(_p(x), outer, n, inner, _p(codes), _p(mins), _p(scales), group, bits)
     assert rc == 0
-    return Packed(codes, mins.view(np.float16), scales.view(np.float16), x.shape, dim, group)
+    return Packed(codes, mins.view(np.float16), scales.view(np.float16), x.shape, dim, group, bits)
 
 
 def dequantize(q: Packed) -> np.ndarray:
     dim, outer, n, inner = _split(q.shape, q.dim)
     y = np.empty(q.shape, dtype=np.uint16)
-    rc = lib().oracle_dequantize_g(_p(np.ascontiguousarray(q.codes)), _p(_u16(q.mins)), _p(_u16(q.scales)),
-                                   outer, n, inner, _p(y), q.group)
+    rc = lib().oracle_dequantize_gb(_p(np.ascontiguousarray(q.codes)), _p(_u16(q.mins)), _p(_u16(q.scales)),
+                                    outer, n, inner, _p(y), q.group, getattr(q, "bits", 4))
     assert rc == 0
     return y.view(np.float16)
 

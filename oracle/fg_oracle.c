@@ -117,21 +117,25 @@ void oracle_f64_to_f16_array(const double *x, uint16_t *out, int64_t n)
 /* ------------------------------------------------------------------------- */
 
 /*
- * One group of `group` (64 or 128) fp16 values x[i*xs] -> group/2 packed bytes codes[j*cs]
- * (byte j = code(2j) | code(2j+1) << 4), fp16 min and fp16 scale.
- * Steps, in this order, each one IEEE fp32 operation:
+ * One group of `group` (64 or 128) fp16 values x[i*xs] -> its codes, fp16 min and fp16 scale.
+ * bits = 4: group/2 packed bytes codes[j*cs], byte j = code(2j) | code(2j+1) << 4;
+ * bits = 8: group bytes codes[j*cs] = code(j).  With levels = 2^bits - 1 (15 or 255), the
+ * steps, in this order, each one IEEE fp32 operation:
  *   1. mn = min(x), mx = max(x);  mn = mn + 0  (turns -0 into +0)
  *   2. d = mx - mn
- *   3. scale_h = fp16_rn(d / 15)
+ *   3. scale_h = fp16_rn(d / levels)
  *   4. scale_h == 0  ->  every code 0, stored scale +0
  *   5. inv = 1 / scale_h
  *   6. t = (x - mn) * inv    (two roundings, no fused multiply-add)
- *   7. code = clamp(round_half_even(t), 0, 15)
+ *   7. code = clamp(round_half_even(t), 0, levels)
  *   8. min_h = fp16(mn)      (exact: mn is one of the fp16 inputs)
+ * The 8-bit form is the same min-max scheme with 255 steps (INT8 next to INT4 among the
+ * post-training formats the "Optimizing LLM for low memory usage" page lists).
  */
-static void quantize_group(const uint16_t *x, ptrdiff_t xs, uint8_t *codes, ptrdiff_t cs,
-                           uint16_t *min_out, uint16_t *scale_out, int group)
+static void quantize_group_b(const uint16_t *x, ptrdiff_t xs, uint8_t *codes, ptrdiff_t cs,
+                             uint16_t *min_out, uint16_t *scale_out, int group, int bits)
 {
+    const int levels = (1 << bits) - 1;
     float v[OR_GROUP_MAX];
     for (int i = 0; i < group; i++) v[i] = oracle_f16_to_f32(x[i * xs]);
     float mn = v[0], mx = v[0];
@@ -141,8 +145,8 @@ static void quantize_group(const uint16_t *x, ptrdiff_t xs, uint8_t *codes, ptrd
     }
     mn = mn + 0.0f;
     float d = mx - mn;
-    float q15 = d / 15.0f;
-    uint16_t scale_h = oracle_f32_to_f16(q15);
+    float qd = d / (float)levels;
+    uint16_t scale_h = oracle_f32_to_f16(qd);
     float s = oracle_f16_to_f32(scale_h);
     int q[OR_GROUP_MAX];
     if (s == 0.0f) {
@@ -156,19 +160,30 @@ static void quantize_group(const uint16_t *x, ptrdiff_t xs, uint8_t *codes, ptrd
             float r = nearbyintf(t);          /* default mode: nearest, ties to even */
             int c = (int)r;
             if (c < 0) c = 0;
-            if (c > 15) c = 15;
+            if (c > levels) c = levels;
             q[i] = c;
         }
     }
-    for (int j = 0; j < group / 2; j++)
-        codes[j * cs] = (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
+    if (bits == 8) {
+        for (int j = 0; j < group; j++) codes[j * cs] = (uint8_t)q[j];
+    } else {
+        for (int j = 0; j < group / 2; j++)
+            codes[j * cs] = (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
+    }
     *min_out = oracle_f32_to_f16(mn);
     *scale_out = scale_h;
 }
 
+static void quantize_group(const uint16_t *x, ptrdiff_t xs, uint8_t *codes, ptrdiff_t cs,
+                           uint16_t *min_out, uint16_t *scale_out, int group)
+{
+    quantize_group_b(x, xs, codes, cs, min_out, scale_out, group, 4);
+}
+
 /* Dequantised value of one code: fp16_rn(mn + q*s), exact before the rounding
-   (q*s has at most 15 significant bits and every term is a multiple of 2^-24
-   below 2^18, so the float64 sum is exact). */
+   (q*s has at most 19 significant bits -- a code of at most 8 bits times an fp16
+   scale -- and every term is a multiple of 2^-24 below 2^25, so the float64 sum is
+   exact). */
 static uint16_t dequant_one(int q, uint16_t min_h, uint16_t scale_h)
 {
     double s = oracle_f16_to_f64(scale_h);
@@ -177,26 +192,38 @@ static uint16_t dequant_one(int q, uint16_t min_h, uint16_t scale_h)
 }
 
 static int group_ok(int group) { return group == 64 || group == 128; }
+static int bits_ok(int bits) { return bits == 4 || bits == 8; }
 
 /*
  * x viewed as [outer, n, inner]; groups of `group` (64 or 128) consecutive elements
  * along n.  codes: [outer, n/2, inner]   mins, scales: [outer, n/group, inner].
  * Returns 0, or -1 for another group size or n not a multiple of the group.
  */
-int oracle_quantize_g(const uint16_t *x, int64_t outer, int64_t n, int64_t inner,
-                      uint8_t *codes, uint16_t *mins, uint16_t *scales, int group)
+/*
+ * bits-bit codes (4 or 8): x viewed as [outer, n, inner]; groups of `group` consecutive
+ * elements along n.  codes: [outer, n*bits/8, inner]   mins, scales: [outer, n/group, inner].
+ * Returns 0, or -1 for another group size or width, or n not a multiple of the group.
+ */
+int oracle_quantize_gb(const uint16_t *x, int64_t outer, int64_t n, int64_t inner,
+                       uint8_t *codes, uint16_t *mins, uint16_t *scales, int group, int bits)
 {
-    if (!group_ok(group) || n % group) return -1;
-    int64_t ng = n / group;
+    if (!group_ok(group) || !bits_ok(bits) || n % group) return -1;
+    int64_t ng = n / group, nc = n * bits / 8, gc = group * bits / 8;
     for (int64_t o = 0; o < outer; o++)
         for (int64_t g = 0; g < ng; g++)
             for (int64_t i = 0; i < inner; i++) {
                 const uint16_t *xp = x + (o * n + g * group) * inner + i;
-                uint8_t *cp = codes + (o * (n / 2) + g * (group / 2)) * inner + i;
+                uint8_t *cp = codes + (o * nc + g * gc) * inner + i;
                 int64_t m = (o * ng + g) * inner + i;
-                quantize_group(xp, inner, cp, inner, &mins[m], &scales[m], group);
+                quantize_group_b(xp, inner, cp, inner, &mins[m], &scales[m], group, bits);
             }
     return 0;
+}
+
+int oracle_quantize_g(const uint16_t *x, int64_t outer, int64_t n, int64_t inner,
+                      uint8_t *codes, uint16_t *mins, uint16_t *scales, int group)
+{
+    return oracle_quantize_gb(x, outer, n, inner, codes, mins, scales, group, 4);
 }
 
 int oracle_quantize(const uint16_t *x, int64_t outer, int64_t n, int64_t inner,
@@ -205,20 +232,31 @@ int oracle_quantize(const uint16_t *x, int64_t outer, int64_t n, int64_t inner,
     return oracle_quantize_g(x, outer, n, inner, codes, mins, scales, OR_GROUP);
 }
 
-int oracle_dequantize_g(const uint8_t *codes, const uint16_t *mins, const uint16_t *scales,
-                        int64_t outer, int64_t n, int64_t inner, uint16_t *y, int group)
+int oracle_dequantize_gb(const uint8_t *codes, const uint16_t *mins, const uint16_t *scales,
+                         int64_t outer, int64_t n, int64_t inner, uint16_t *y, int group, int bits)
 {
-    if (!group_ok(group) || n % group) return -1;
-    int64_t ng = n / group;
+    if (!group_ok(group) || !bits_ok(bits) || n % group) return -1;
+    int64_t ng = n / group, nc = n * bits / 8;
     for (int64_t o = 0; o < outer; o++)
         for (int64_t e = 0; e < n; e++)
             for (int64_t i = 0; i < inner; i++) {
-                uint8_t byte = codes[(o * (n / 2) + e / 2) * inner + i];
-                int q = (e & 1) ? (byte >> 4) : (byte & 15);
+                int q;
+                if (bits == 8) {
+                    q = codes[(o * nc + e) * inner + i];
+                } else {
+                    uint8_t byte = codes[(o * nc + e / 2) * inner + i];
+                    q = (e & 1) ? (byte >> 4) : (byte & 15);
+                }
                 int64_t m = (o * ng + e / group) * inner + i;
                 y[(o * n + e) * inner + i] = dequant_one(q, mins[m], scales[m]);
             }
     return 0;
+}
+
+int oracle_dequantize_g(const uint8_t *codes, const uint16_t *mins, const uint16_t *scales,
+                        int64_t outer, int64_t n, int64_t inner, uint16_t *y, int group)
+{
+    return oracle_dequantize_gb(codes, mins, scales, outer, n, inner, y, group, 4);
 }
 
 int oracle_dequantize(const uint8_t *codes, const uint16_t *mins, const uint16_t *scales,

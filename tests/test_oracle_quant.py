@@ -342,3 +342,99 @@ def test_group_sizes_rejected():
         oracle.quantize(np.zeros((2, 192), dtype=np.float16), group=128)
     with pytest.raises(ValueError):
         oracle.quantize(np.zeros((2, 192), dtype=np.float16), group=96)
+
+
+# ------------------------------------------------------------------ 8-bit codes -----------
+# The same min-max scheme with 255 steps, one code per byte (INT8 beside INT4 among the
+# post-training formats of the "Optimizing LLM for low memory usage" page).
+
+def _b8_span_group(group, offset=0.0):
+    # integers spanning exactly [0, 255] (both ends present), so that range/255 = 1 exactly
+    x = np.concatenate([[0.0, 255.0], np.round(np.linspace(1, 254, group - 2))]) + offset
+    return x.astype(np.float16).reshape(1, group)
+
+
+@pytest.mark.parametrize("group,offset", [(64, 0.0), (64, 1000.0), (64, -700.0), (128, 0.0), (128, 512.0)])
+def test_b8_integer_span_is_exact(group, offset):
+    # scale = fp16(255 / 255) = 1, inverse 1: every code is the value minus the minimum and
+    # the round trip is exact (closed form; all values are fp16 integers)
+    x = _b8_span_group(group, offset)
+    q = oracle.quantize(x, group=group, bits=8)
+    assert q.codes.shape == (1, group)                         # one code per byte, in order
+    assert float(q.scales[0, 0]) == 1.0 and float(q.mins[0, 0]) == offset
+    assert np.array_equal(q.codes[0].astype(np.float64), x[0].astype(np.float64) - offset)
+    assert np.array_equal(oracle.dequantize(q).view(np.uint16), x.view(np.uint16))
+
+
+def test_b8_ties_round_half_even():
+    # span [0, 255] -> step 1; k + 0.5 rounds to the even neighbour
+    x = np.full((1, 64), 100.0)
+    x[0, :2] = [0.0, 255.0]
+    x[0, 2:8] = [0.5, 1.5, 2.5, 3.5, 128.5, 254.5]
+    q = oracle.quantize(x.astype(np.float16), bits=8)
+    assert list(q.codes[0, :8]) == [0, 255, 0, 2, 2, 4, 128, 254]
+    assert np.all(q.codes[0, 8:] == 100)
+
+
+@pytest.mark.parametrize("value", [0.0, -3.25, 1000.0])
+def test_b8_constant_group(value):
+    x = np.full((1, 64), value, dtype=np.float16)
+    q = oracle.quantize(x, bits=8)
+    assert np.all(q.codes == 0) and float(q.scales[0, 0]) == 0.0
+    assert np.array_equal(oracle.dequantize(q).view(np.uint16), (x + np.float16(0)).view(np.uint16))
+
+
+def _check_b8_round_trip(x2d, group=64):
+    q = oracle.quantize(x2d, group=group, bits=8)
+    y = oracle.dequantize(q).astype(np.float64).reshape(-1, group)
+    G = x2d.astype(np.float64).reshape(-1, group)
+    s = q.scales.astype(np.float64).reshape(-1, 1)
+    mn = q.mins.astype(np.float64).reshape(-1, 1)
+    codes = q.codes.reshape(-1, group).astype(np.float64)
+    assert np.array_equal(mn[:, 0], G.min(axis=1) + 0.0)
+    nz = s[:, 0] > 0
+    assert np.all(codes[~nz] == 0) and np.all(codes[nz].min(axis=1) == 0)
+    # codes follow the values: sorting a group's values sorts its codes
+    order = np.argsort(G, axis=1, kind="stable")
+    assert np.all(np.diff(np.take_along_axis(codes, order, axis=1), axis=1) >= 0)
+    # a normal fp16 scale is within 2^-11 of range/255, so the group maximum lands on 255
+    normal = s[:, 0] >= 2.0 ** -14
+    assert np.all(codes[normal, :][np.arange(normal.sum()), G[normal].argmax(axis=1)] == 255)
+    exact = mn + codes * s
+    assert np.all(np.abs(G - exact)[normal] <= (s / 2 * (1 + 2.0 ** -16))[normal])
+    ulp = np.spacing(np.abs(exact).astype(np.float16)).astype(np.float64)
+    assert np.all(np.abs(y - exact) <= ulp / 2)
+    assert np.all(y[np.arange(len(G)), G.argmin(axis=1)] == G.min(axis=1))
+    return int(normal.sum())
+
+
+def test_b8_round_trip_bound_sweep_recipe():
+    x = si.sweep_tensor(seed=5, numel=1 << 16, row=4096)
+    assert _check_b8_round_trip(x) > 0
+    _check_b8_round_trip(x, group=128)
+
+
+def test_b8_non_last_dim_equals_transposed():
+    x = si.normal_f16(6, 99, (3, 128, 5), 1.0)
+    a = oracle.quantize(x, dim=1, bits=8)
+    b = oracle.quantize(np.ascontiguousarray(np.transpose(x, (0, 2, 1))), dim=-1, bits=8)
+    assert a.codes.shape == (3, 128, 5)
+    assert np.array_equal(a.codes, np.transpose(b.codes, (0, 2, 1)))
+    assert np.array_equal(oracle.dequantize(a).view(np.uint16),
+                          np.transpose(oracle.dequantize(b).view(np.uint16), (0, 2, 1)))
+
+
+def test_b8_codes_are_the_4bit_codes_refined():
+    # with the same range, an 8-bit step is a 4-bit step / 17 (255 = 15 * 17): the integer span
+    # [0, 255] quantised at 4 bits has step 17, so the 4-bit code is the 8-bit code / 17 rounded
+    x = _b8_span_group(64)
+    c8 = oracle.quantize(x, bits=8).codes[0].astype(np.int64)
+    c4 = _nibbles(oracle.quantize(x).codes[0])
+    assert float(oracle.quantize(x).scales[0, 0]) == 17.0
+    assert np.array_equal(c4, np.round(c8 / 17.0).astype(np.int64))
+
+
+def test_bits_rejected():
+    for bits in (2, 3, 16):
+        with pytest.raises(ValueError):
+            oracle.quantize(np.zeros((1, 64), dtype=np.float16), bits=bits)
