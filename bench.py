@@ -176,7 +176,7 @@ class OracleSample:
         return time.perf_counter() - t0
 
 
-def oracle_quant_baseline(kind: str, group: int, log2_elems: int):
+def oracle_quant_baseline(kind: str, group: int, log2_elems: int, bits: int = 4):
     """The oracle's quantise (or dequantise) on the quantize-sweep recipe, timed on this host:
     one thread, then the rows split over every host thread (the oracle's C loops release the
     GIL).  A bounded sample of min(2^log2_elems, 2^26) elements stands in for the full tensor;
@@ -188,17 +188,17 @@ def oracle_quant_baseline(kind: str, group: int, log2_elems: int):
     n = 1 << min(log2_elems, 26)
     x = si.sweep_tensor(0, n, group=group)
     rows = x.shape[0]
-    packed = oracle.quantize(x, group=group) if kind == "dequantize" else None
+    packed = oracle.quantize(x, group=group, bits=bits) if kind == "dequantize" else None
 
     def work(lo, hi):
         if kind == "quantize":
-            oracle.quantize(x[lo:hi], group=group)
+            oracle.quantize(x[lo:hi], group=group, bits=bits)
         else:
             q = oracle.Packed(packed.codes[lo:hi], packed.mins[lo:hi], packed.scales[lo:hi],
-                              (hi - lo, x.shape[1]), 1, group)
+                              (hi - lo, x.shape[1]), 1, group, bits)
             oracle.dequantize(q)
 
-    bytes_ = n * (2.5 + 4.0 / group)
+    bytes_ = n * (2 + bits / 8 + 4.0 / group)
     t0 = time.perf_counter()
     work(0, rows)
     t1 = time.perf_counter() - t0
@@ -846,12 +846,12 @@ def run_kernel(args, wl):
     elif args.kernel in ("quantize", "dequantize"):
         n = 1 << args.log2_elems
         x = torch.randn((n // 4096, 4096), generator=g, device=dev, dtype=torch.float16) * 0.02
-        q = fg.fg_quantize(x, group=args.group)
+        q = fg.fg_quantize(x, group=args.group, bits=args.bits)
         if args.kernel == "quantize":
-            run = lambda: fg.fg_quantize(x, group=args.group, out=q, stream=stream)
+            run = lambda: fg.fg_quantize(x, group=args.group, bits=args.bits, out=q, stream=stream)
         else:
             run = lambda: fg.fg_dequantize(q, stream=stream)
-        work, unit, peak = n * (2.5 + 4.0 / args.group), "GB/s", peaks["hbm"]
+        work, unit, peak = n * (2 + args.bits / 8 + 4.0 / args.group), "GB/s", peaks["hbm"]
     else:
         raise SystemExit(f"unknown kernel {args.kernel}")
     for _ in range(args.warmup):
@@ -873,7 +873,8 @@ def run_kernel(args, wl):
             "frac": work / med / scale / peak}
     if args.kernel in ("quantize", "dequantize") and not args.no_cpu_baseline:
         line["log2_elems"] = args.log2_elems
-        line["cpu_baseline"] = oracle_quant_baseline(args.kernel, args.group, args.log2_elems)
+        line["bits"] = args.bits
+        line["cpu_baseline"] = oracle_quant_baseline(args.kernel, args.group, args.log2_elems, args.bits)
     print(json.dumps(line), flush=True)
 
 
@@ -890,6 +891,7 @@ def main():
                          "fc2_gemm, quantize, dequantize")
     ap.add_argument("--seqs", type=int, default=0, help="--kernel: sequences (default: the workload's block)")
     ap.add_argument("--log2-elems", type=int, default=28, help="--kernel quantize/dequantize: tensor size")
+    ap.add_argument("--bits", type=int, choices=(4, 8), default=4, help="--kernel quantize/dequantize: code width")
     ap.add_argument("--layers", type=int, default=0, help="stack workloads: number of layers (default: the model's)")
     ap.add_argument("--group", type=int, choices=(64, 128), default=64,
                     help="quantisation group size: of the layer's weights and KV cache (layer workloads), or of "

@@ -132,11 +132,12 @@ def _need(t: torch.Tensor, dtype, name: str) -> None:
 # ---------------------------------------------------------------------------------------
 
 class QTensor:
-    """Packed 4-bit tensor (device): codes uint8, mins/scales float16, grouped along ``dim``."""
+    """Packed tensor (device): codes uint8 (two 4-bit or one 8-bit code per byte), mins/scales
+    float16, grouped along ``dim``."""
 
-    def __init__(self, codes, mins, scales, shape, dim, group: int = 64):
+    def __init__(self, codes, mins, scales, shape, dim, group: int = 64, bits: int = 4):
         self.codes, self.mins, self.scales = codes, mins, scales
-        self.shape, self.dim, self.group = tuple(int(s) for s in shape), dim, group
+        self.shape, self.dim, self.group, self.bits = tuple(int(s) for s in shape), dim, group, bits
 
     def struct(self) -> fg_qtensor:
         s = fg_qtensor()
@@ -144,7 +145,7 @@ class QTensor:
         s.ndim = len(self.shape)
         for i in range(4):
             s.shape[i] = self.shape[i] if i < len(self.shape) else 1
-        s.dim, s.bits, s.group = self.dim, 4, self.group
+        s.dim, s.bits, s.group = self.dim, self.bits, self.group
         return s
 
 
@@ -165,11 +166,12 @@ def fg_quantize(x: torch.Tensor, dim: int = -1, bits: int = 4, group: int = 64, 
     dim = dim % len(shape)
     fg_qtensor_bytes(shape, dim, bits, group)
     if out is None:
-        cs = list(shape); cs[dim] //= 2
+        cs = list(shape); cs[dim] = cs[dim] * bits // 8
         ms = list(shape); ms[dim] //= group
         out = QTensor(torch.empty(cs, dtype=torch.uint8, device=x.device),
                       torch.empty(ms, dtype=torch.float16, device=x.device),
-                      torch.empty(ms, dtype=torch.float16, device=x.device), shape, dim, group)
+                      torch.empty(ms, dtype=torch.float16, device=x.device), shape, dim, group, bits)
+    out.bits = bits
     s = out.struct()
     arr = (c_int64 * len(shape))(*shape)
     _check(_lib.fg_quantize(_ptr(x), len(shape), arr, dim, bits, group, ctypes.byref(s), _stream(stream)),

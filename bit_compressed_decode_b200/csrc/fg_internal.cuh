@@ -482,6 +482,12 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 scale2, __half2 mi
   return r;
 }
 
+// 8-bit form of quant_group8: the same group min/max, scale = fp16(RN(d / 255)) (the IEEE
+// division), the same reciprocal and rounding, codes clamped to 255, one byte per code: the
+// lane's 8 codes as two words (byte k of word w = code 4w + k).  All 32 lanes must call it.
+template <int LANES = 8>
+__device__ __forceinline__ uint2 quant_group8_u8(const uint4 v, __half &min_h, __half &scale_h);
+
 // RN(d / 15) for finite d >= 0: d * RN(1/15) corrected by one fused multiply-add on the
 // exact residual d - 15 q0 (Markstein's correction step, P. Markstein, IBM J. Res. Dev. 34,
 // 1990).  Equal to the correctly rounded quotient for every non-negative finite float
@@ -558,4 +564,62 @@ __device__ __forceinline__ uint32_t quant_group8(const uint4 v, __half &min_h, _
   min_h = __float2half_rn(mn);
   scale_h = sh;
   return word;
+}
+
+template <int LANES>
+__device__ __forceinline__ uint2 quant_group8_u8(const uint4 v, __half &min_h, __half &scale_h) {
+  const __half2 *h2 = reinterpret_cast<const __half2 *>(&v);
+  const __half2 lo = __hmin2(__hmin2(h2[0], h2[1]), __hmin2(h2[2], h2[3]));
+  const __half2 hi = __hmax2(__hmax2(h2[0], h2[1]), __hmax2(h2[2], h2[3]));
+  __half2 mm = __halves2half2(__hmin(__low2half(lo), __high2half(lo)),
+                              __hneg(__hmax(__low2half(hi), __high2half(hi))));
+#pragma unroll
+  for (int o = 1; o < LANES; o <<= 1) {
+    const uint32_t u = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<const uint32_t *>(&mm), o);
+    mm = __hmin2(mm, *reinterpret_cast<const __half2 *>(&u));
+  }
+  float mn = __low2float(mm);
+  const float mx = -__high2float(mm);
+  mn = __fadd_rn(mn, 0.0f);
+  const float d = __fsub_rn(mx, mn);
+  __half sh = __float2half_rn(__fdiv_rn(d, 255.0f));
+  const float s = __half2float(sh);
+  uint32_t w[2] = {0u, 0u};
+  if (s != 0.0f) {
+    const float inv = rcp_rn_f16val(s);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      const float2 f = __half22float2(h2[i]);
+      const float r0 = __fadd_rn(__fmul_rn(__fsub_rn(f.x, mn), inv), 12582912.0f);
+      const float r1 = __fadd_rn(__fmul_rn(__fsub_rn(f.y, mn), inv), 12582912.0f);
+      const uint32_t c0 = min(__float_as_uint(r0), 0x4B4000FFu) & 0xFFu;
+      const uint32_t c1 = min(__float_as_uint(r1), 0x4B4000FFu) & 0xFFu;
+      w[i >> 1] |= (c0 | (c1 << 8)) << (16 * (i & 1));
+    }
+  } else {
+    sh = __ushort_as_half(0);
+  }
+  min_h = __float2half_rn(mn);
+  scale_h = sh;
+  return make_uint2(w[0], w[1]);
+}
+
+// Eight 8-bit codes (two words, byte k of word w = code 4w + k) -> eight fp16 values
+// fp16_rn(min + code * scale): a byte placed under the exponent bits 0x64 is the fp16 value
+// 1024 + code (exact), less 1024 is the code, and one half-precision FMA rounds once.
+__device__ __forceinline__ uint4 dequant8_u8(uint2 w, __half2 scale2, __half2 min2) {
+  const __half2 k1024 = __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400));
+  uint4 r;
+  uint32_t *o = reinterpret_cast<uint32_t *>(&r);
+  const uint32_t words[2] = {w.x, w.y};
+#pragma unroll
+  for (int i = 0; i < 2; i++) {
+    const uint32_t a = __byte_perm(words[i], 0x6464u, 0x5140), b = __byte_perm(words[i], 0x6464u, 0x5342);
+    const __half2 ca = __hsub2(*reinterpret_cast<const __half2 *>(&a), k1024);
+    const __half2 cb = __hsub2(*reinterpret_cast<const __half2 *>(&b), k1024);
+    const __half2 ya = __hfma2(ca, scale2, min2), yb = __hfma2(cb, scale2, min2);
+    o[2 * i] = *reinterpret_cast<const uint32_t *>(&ya);
+    o[2 * i + 1] = *reinterpret_cast<const uint32_t *>(&yb);
+  }
+  return r;
 }

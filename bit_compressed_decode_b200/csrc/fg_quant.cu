@@ -1,4 +1,4 @@
-// fg_quant.cu -- group-wise 4-bit quantise (pack), dequantise and the 4-bit KV append.
+// fg_quant.cu -- group-wise 4-bit (and 8-bit) quantise (pack), dequantise and the 4-bit KV append.
 //
 // Format and fp32 operation order: "FlexGen Guide: High-Throughput LLM Offloading on
 // One GPU", section 3 (Group-Wise 4-Bit Quantization for Weights and KV Cache), read
@@ -40,7 +40,7 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
 // ------------------------------------------------------------------------------------
 constexpr int kQU = 4;
 
-template <int G>
+template <int G, int B>  // B: code width, 4 (two codes per byte) or 8 (one)
 __global__ void __launch_bounds__(256) quantize_lastdim_kernel(const uint4 *__restrict__ x, int64_t ngroups,
                                                                uint32_t *__restrict__ codes,
                                                                __half *__restrict__ mins,
@@ -61,12 +61,23 @@ __global__ void __launch_bounds__(256) quantize_lastdim_kernel(const uint4 *__re
     for (int u = 0; u < kQU; u++) {
       const int64_t g = g0 + u * GPW + slot;
       __half mn, sc;
-      const uint32_t w = quant_group8<L>(v[u], mn, sc);
-      if (g < ngroups) {
-        codes[g * L + j] = w;
-        if (j == 0) {
-          mins[g] = mn;
-          scales[g] = sc;
+      if constexpr (B == 8) {
+        const uint2 w = quant_group8_u8<L>(v[u], mn, sc);
+        if (g < ngroups) {
+          reinterpret_cast<uint2 *>(codes)[g * L + j] = w;
+          if (j == 0) {
+            mins[g] = mn;
+            scales[g] = sc;
+          }
+        }
+      } else {
+        const uint32_t w = quant_group8<L>(v[u], mn, sc);
+        if (g < ngroups) {
+          codes[g * L + j] = w;
+          if (j == 0) {
+            mins[g] = mn;
+            scales[g] = sc;
+          }
         }
       }
     }
@@ -75,36 +86,56 @@ __global__ void __launch_bounds__(256) quantize_lastdim_kernel(const uint4 *__re
 
 // K2: dequantise along the last dim; one thread per 8 codes (one 16-byte output).  G/8
 // such chunks share a group's min and scale.
-template <int G>
+template <int G, int B>
 __global__ void __launch_bounds__(256) dequantize_lastdim_kernel(const uint32_t *__restrict__ codes,
                                                                  const __half *__restrict__ mins,
                                                                  const __half *__restrict__ scales,
                                                                  int64_t nchunks, uint4 *__restrict__ y) {
+  // chunk c = 8 codes: one 32-bit word (4-bit codes) or two (8-bit codes)
+  auto deq = [&](int64_t c) {
+    const __half2 s2 = __half2half2(scales[c / (G / 8)]), m2 = __half2half2(mins[c / (G / 8)]);
+    if constexpr (B == 8) return dequant8_u8(__ldcs(reinterpret_cast<const uint2 *>(codes) + c), s2, m2);
+    else return dequant8(__ldcs(codes + c), s2, m2);
+  };
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (; i + 3 * stride < nchunks; i += 4 * stride) {
-    uint32_t w[4];
-    __half mn[4], sc[4];
+  if constexpr (B == 8) {
+    for (; i + 3 * stride < nchunks; i += 4 * stride) {
+      uint2 w[4];
+      __half mn[4], sc[4];
 #pragma unroll
-    for (int u = 0; u < 4; u++) {
-      const int64_t c = i + u * stride;
-      w[u] = __ldcs(codes + c);
-      mn[u] = mins[c / (G / 8)];
-      sc[u] = scales[c / (G / 8)];
+      for (int u = 0; u < 4; u++) {
+        const int64_t c = i + u * stride;
+        w[u] = __ldcs(reinterpret_cast<const uint2 *>(codes) + c);
+        mn[u] = mins[c / (G / 8)];
+        sc[u] = scales[c / (G / 8)];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; u++) __stcs(y + i + u * stride, dequant8_u8(w[u], __half2half2(sc[u]), __half2half2(mn[u])));
     }
+  } else {
+    for (; i + 3 * stride < nchunks; i += 4 * stride) {
+      uint32_t w[4];
+      __half mn[4], sc[4];
 #pragma unroll
-    for (int u = 0; u < 4; u++) __stcs(y + i + u * stride, dequant8(w[u], __half2half2(sc[u]), __half2half2(mn[u])));
+      for (int u = 0; u < 4; u++) {
+        const int64_t c = i + u * stride;
+        w[u] = __ldcs(codes + c);
+        mn[u] = mins[c / (G / 8)];
+        sc[u] = scales[c / (G / 8)];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; u++) __stcs(y + i + u * stride, dequant8(w[u], __half2half2(sc[u]), __half2half2(mn[u])));
+    }
   }
-  for (; i < nchunks; i += stride) {
-    __stcs(y + i, dequant8(__ldcs(codes + i), __half2half2(scales[i / (G / 8)]), __half2half2(mins[i / (G / 8)])));
-  }
+  for (; i < nchunks; i += stride) __stcs(y + i, deq(i));
 }
 
 // ------------------------------------------------------------------------------------
 // Strided variants (grouping dim is not the last one): x viewed as [outer][n][inner],
 // one thread per group, consecutive threads on consecutive inner positions.
 // ------------------------------------------------------------------------------------
-template <int G>
+template <int G, int B>
 __global__ void __launch_bounds__(256) quantize_strided_kernel(const __half *__restrict__ x, int64_t outer,
                                                                int64_t n, int64_t inner,
                                                                uint8_t *__restrict__ codes,
@@ -129,21 +160,27 @@ __global__ void __launch_bounds__(256) quantize_strided_kernel(const __half *__r
     }
     mn = __fadd_rn(mn, 0.0f);
     const float d = __fsub_rn(mx, mn);
-    __half sh = __float2half_rn(__fdiv_rn(d, 15.0f));
+    constexpr int kLevels = (1 << B) - 1;
+    __half sh = __float2half_rn(__fdiv_rn(d, static_cast<float>(kLevels)));
     const float s = __half2float(sh);
-    uint8_t *cp = codes + (o * (n / 2) + g * (G / 2)) * inner + i;
+    uint8_t *cp = codes + (o * (n * B / 8) + g * (G * B / 8)) * inner + i;
     if (s != 0.0f) {
       const float inv = __fdiv_rn(1.0f, s);
 #pragma unroll
       for (int e = 0; e < G; e += 2) {
-        int c0 = min(max(__float2int_rn(__fmul_rn(__fsub_rn(v[e], mn), inv)), 0), 15);
-        int c1 = min(max(__float2int_rn(__fmul_rn(__fsub_rn(v[e + 1], mn), inv)), 0), 15);
-        cp[(e / 2) * inner] = static_cast<uint8_t>(c0 | (c1 << 4));
+        int c0 = min(max(__float2int_rn(__fmul_rn(__fsub_rn(v[e], mn), inv)), 0), kLevels);
+        int c1 = min(max(__float2int_rn(__fmul_rn(__fsub_rn(v[e + 1], mn), inv)), 0), kLevels);
+        if constexpr (B == 8) {
+          cp[e * inner] = static_cast<uint8_t>(c0);
+          cp[(e + 1) * inner] = static_cast<uint8_t>(c1);
+        } else {
+          cp[(e / 2) * inner] = static_cast<uint8_t>(c0 | (c1 << 4));
+        }
       }
     } else {
       sh = __ushort_as_half(0);
 #pragma unroll
-      for (int e = 0; e < G; e += 2) cp[(e / 2) * inner] = 0;
+      for (int e = 0; e < G * B / 8; e++) cp[e * inner] = 0;
     }
     const int64_t m = (o * ng + g) * inner + i;
     mins[m] = __float2half_rn(mn);
@@ -151,12 +188,24 @@ __global__ void __launch_bounds__(256) quantize_strided_kernel(const __half *__r
   }
 }
 
-template <int G>
+template <int G, int B>
 __global__ void __launch_bounds__(256) dequantize_strided_kernel(const uint8_t *__restrict__ codes,
                                                                  const __half *__restrict__ mins,
                                                                  const __half *__restrict__ scales,
                                                                  int64_t outer, int64_t n, int64_t inner,
                                                                  __half *__restrict__ y) {
+  if constexpr (B == 8) {  // one thread per code byte (1 element): fp16_rn(min + code * scale)
+    const int64_t total = outer * n * inner;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+         t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      const int64_t i = t % inner, e = (t / inner) % n, o = t / (inner * n);
+      const int64_t m = (o * (n / G) + e / G) * inner + i;
+      const __half c = __hsub(__ushort_as_half(static_cast<unsigned short>(0x6400u | codes[t])),
+                              __ushort_as_half(0x6400));
+      y[t] = __hfma(c, scales[m], mins[m]);
+    }
+    return;
+  }
   const int64_t total = outer * (n / 2) * inner;  // one thread per code byte (2 elements)
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -248,11 +297,11 @@ bool shape_numel(int ndim, const int64_t *shape, int64_t *numel) {
 extern "C" fg_status fg_qtensor_bytes(int ndim, const int64_t *shape, int dim, int bits, int group,
                                       size_t *codes_bytes, size_t *meta_bytes) {
   if (!shape || ndim < 1 || ndim > 4 || dim < 0 || dim >= ndim) return FG_ERR_INVALID;
-  if (bits != 4 || (group != 64 && group != 128)) return FG_ERR_UNSUPPORTED;
+  if ((bits != 4 && bits != 8) || (group != 64 && group != 128)) return FG_ERR_UNSUPPORTED;
   int64_t numel;
   if (!shape_numel(ndim, shape, &numel)) return FG_ERR_INVALID;
   if (shape[dim] % group) return FG_ERR_SHAPE;
-  if (codes_bytes) *codes_bytes = static_cast<size_t>(numel / 2);
+  if (codes_bytes) *codes_bytes = static_cast<size_t>(numel / 8 * bits);
   if (meta_bytes) *meta_bytes = static_cast<size_t>(numel / group) * 2;
   return FG_OK;
 }
@@ -283,7 +332,8 @@ extern "C" fg_status fg_quantize(const fg_half *x, int ndim, const int64_t *shap
     const int64_t ngroups = numel / group;
     const int gpw = 32 / (group / 8);  // groups per warp step
     const int64_t warps_needed = (ngroups + gpw * kQU - 1) / (gpw * kQU);
-    auto kern = group == 128 ? quantize_lastdim_kernel<128> : quantize_lastdim_kernel<64>;
+    auto kern = bits == 8 ? (group == 128 ? quantize_lastdim_kernel<128, 8> : quantize_lastdim_kernel<64, 8>)
+                          : (group == 128 ? quantize_lastdim_kernel<128, 4> : quantize_lastdim_kernel<64, 4>);
     kern<<<grid_for((warps_needed + 7) / 8, 8), 256, 0, st>>>(
         reinterpret_cast<const uint4 *>(x), ngroups, reinterpret_cast<uint32_t *>(out->codes),
         reinterpret_cast<__half *>(out->mins), reinterpret_cast<__half *>(out->scales));
@@ -292,7 +342,8 @@ extern "C" fg_status fg_quantize(const fg_half *x, int ndim, const int64_t *shap
         (reinterpret_cast<uintptr_t>(out->scales) & 1))
       return FG_ERR_INVALID;
     const int64_t groups = outer * (n / group) * inner;
-    auto kern = group == 128 ? quantize_strided_kernel<128> : quantize_strided_kernel<64>;
+    auto kern = bits == 8 ? (group == 128 ? quantize_strided_kernel<128, 8> : quantize_strided_kernel<64, 8>)
+                          : (group == 128 ? quantize_strided_kernel<128, 4> : quantize_strided_kernel<64, 4>);
     kern<<<grid_for((groups + 255) / 256, 8), 256, 0, st>>>(
         reinterpret_cast<const __half *>(x), outer, n, inner, out->codes, reinterpret_cast<__half *>(out->mins),
         reinterpret_cast<__half *>(out->scales));
@@ -314,15 +365,20 @@ extern "C" fg_status fg_dequantize(const fg_qtensor *q, fg_half *y, void *stream
   const int64_t n = q->shape[q->dim];
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (inner == 1) {
-    if (!fg_aligned16(y) || (reinterpret_cast<uintptr_t>(q->codes) & 3)) return FG_ERR_INVALID;
+    // chunks of 8 codes: one aligned word (4-bit codes) or two (8-bit codes)
+    if (!fg_aligned16(y) || (reinterpret_cast<uintptr_t>(q->codes) & (q->bits == 8 ? 7 : 3))) return FG_ERR_INVALID;
     const int64_t nchunks = numel / 8;
-    auto kern = q->group == 128 ? dequantize_lastdim_kernel<128> : dequantize_lastdim_kernel<64>;
+    auto kern = q->bits == 8
+                    ? (q->group == 128 ? dequantize_lastdim_kernel<128, 8> : dequantize_lastdim_kernel<64, 8>)
+                    : (q->group == 128 ? dequantize_lastdim_kernel<128, 4> : dequantize_lastdim_kernel<64, 4>);
     kern<<<grid_for((nchunks + 255) / 256, 8), 256, 0, st>>>(
         reinterpret_cast<const uint32_t *>(q->codes), reinterpret_cast<const __half *>(q->mins),
         reinterpret_cast<const __half *>(q->scales), nchunks, reinterpret_cast<uint4 *>(y));
   } else {
-    const int64_t total = outer * (n / 2) * inner;
-    auto kern = q->group == 128 ? dequantize_strided_kernel<128> : dequantize_strided_kernel<64>;
+    const int64_t total = outer * (n * q->bits / 8) * inner;  // one thread per code byte
+    auto kern = q->bits == 8
+                    ? (q->group == 128 ? dequantize_strided_kernel<128, 8> : dequantize_strided_kernel<64, 8>)
+                    : (q->group == 128 ? dequantize_strided_kernel<128, 4> : dequantize_strided_kernel<64, 4>);
     kern<<<grid_for((total + 255) / 256, 8), 256, 0, st>>>(
         q->codes, reinterpret_cast<const __half *>(q->mins), reinterpret_cast<const __half *>(q->scales), outer, n,
         inner, reinterpret_cast<__half *>(y));

@@ -61,7 +61,7 @@ typedef enum {
     FG_OK = 0,
     FG_ERR_INVALID = 1,     /* null/misaligned pointer, bad enum, negative size */
     FG_ERR_SHAPE = 2,       /* size not a multiple of the group, inconsistent dims */
-    FG_ERR_UNSUPPORTED = 3, /* bits != 4, a group size not taken, dims the kernels do not cover */
+    FG_ERR_UNSUPPORTED = 3, /* a code width or group size not taken, dims the kernels do not cover */
     FG_ERR_RANGE = 4,       /* a cache position outside [0, max_len) (host or device check) */
     FG_ERR_CUDA = 5,        /* a CUDA runtime call failed (launch, copy, event) */
     FG_ERR_TIMEOUT = 6,     /* a bounded wait inside a kernel gave up */
@@ -84,9 +84,13 @@ FG_API const char *fg_last_cuda_error(void);
 /* ---------------------------------------------------------------------- */
 
 /* A tensor of `shape` quantised in groups of `group` along `dim`.
- * codes:  uint8, shape with shape[dim] halved  (even element in the low nibble)
+ * codes:  uint8; bits = 4: shape with shape[dim] halved (even element in the
+ *         low nibble); bits = 8: shape unchanged, one code per byte
  * mins, scales: fp16, shape with shape[dim] divided by `group`.
- * All three are row-major (C order) and caller-owned (device memory). */
+ * All three are row-major (C order) and caller-owned (device memory).
+ * bits = 8 is the same min-max scheme with 255 steps (INT8 beside INT4 among
+ * the post-training formats of the "Optimizing LLM for low memory usage"
+ * page); the layer, the KV cache and fg_linear_w4a16 take 4-bit codes only. */
 typedef struct {
     uint8_t *codes;
     fg_half *mins;
@@ -94,7 +98,7 @@ typedef struct {
     int32_t ndim;        /* 1..4 */
     int64_t shape[4];
     int32_t dim;         /* grouping dim, 0..ndim-1 */
-    int32_t bits;        /* 4 */
+    int32_t bits;        /* 4 or 8 */
     int32_t group;       /* 64 or 128 */
 } fg_qtensor;
 
@@ -106,8 +110,11 @@ FG_API fg_status fg_qtensor_bytes(int ndim, const int64_t *shape, int dim, int b
  * out->mins, out->scales (device buffers set by the caller; their sizes from
  * fg_qtensor_bytes).  Fills out->ndim/shape/dim/bits/group.  x must be finite
  * (a group holding Inf or NaN gets unspecified codes).
+ * Codes: with levels = 2^bits - 1, scale = fp16_rn(d / levels) for the group
+ * range d, code = clamp(rint_even((x - min) * (1 / scale)), 0, levels), in the
+ * fp32 steps stated at the top of this file for 4 bits (15 replaced by levels).
  * Errors: FG_ERR_SHAPE if shape[dim] % group != 0; FG_ERR_UNSUPPORTED if
- * bits != 4 or group not 64 or 128.  [G3] */
+ * bits is not 4 or 8, or group not 64 or 128.  [G3] */
 FG_API fg_status fg_quantize(const fg_half *x, int ndim, const int64_t *shape, int dim, int bits, int group,
                       fg_qtensor *out, void *stream);
 

@@ -53,8 +53,11 @@ def test_qtensor_bytes_and_errors():
     assert fg.fg_qtensor_bytes((6, 128, 5), dim=1) == (6 * 128 * 5 // 2, 6 * 2 * 5 * 2)
     with pytest.raises(fg.FgError, match="SHAPE"):
         fg.fg_qtensor_bytes((8, 96))
-    with pytest.raises(fg.FgError, match="UNSUPPORTED"):
-        fg.fg_qtensor_bytes((8, 64), bits=8)
+    assert fg.fg_qtensor_bytes((8, 64), bits=8) == (8 * 64, 8 * 2)        # 8-bit codes: one per byte
+    assert fg.fg_qtensor_bytes((6, 128, 5), dim=1, bits=8, group=128) == (6 * 128 * 5, 6 * 5 * 2)
+    for bits in (2, 3, 16):
+        with pytest.raises(fg.FgError, match="UNSUPPORTED"):
+            fg.fg_qtensor_bytes((8, 64), bits=bits)
     assert fg.fg_qtensor_bytes((8, 256), group=128) == (8 * 256 // 2, 8 * 2 * 2)   # groups of 128
     with pytest.raises(fg.FgError, match="SHAPE"):
         fg.fg_qtensor_bytes((8, 192), group=128)

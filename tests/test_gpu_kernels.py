@@ -41,9 +41,9 @@ def u16(a):
 
 # ------------------------------------------------------------------ quantise ----------
 
-def _check_quant_equal(x16, dim=-1, group=64):
-    q = fg.fg_quantize(dev(x16), dim=dim, group=group)
-    r = oracle.quantize(x16, dim=dim, group=group)
+def _check_quant_equal(x16, dim=-1, group=64, bits=4):
+    q = fg.fg_quantize(dev(x16), dim=dim, group=group, bits=bits)
+    r = oracle.quantize(x16, dim=dim, group=group, bits=bits)
     torch.cuda.synchronize()
     assert np.array_equal(host(q.codes), r.codes)
     assert np.array_equal(u16(host(q.mins)), u16(r.mins))
@@ -100,8 +100,60 @@ def test_quantize_empty_and_errors():
     assert q.codes.numel() == 0
     with pytest.raises(fg.FgError, match="SHAPE"):
         fg.fg_quantize(torch.zeros((2, 96), dtype=torch.float16, device="cuda"))
+    for bits in (2, 3, 16):
+        with pytest.raises(fg.FgError, match="UNSUPPORTED"):
+            fg.fg_quantize(torch.zeros((2, 64), dtype=torch.float16, device="cuda"), bits=bits)
+
+
+# ------------------------------------------------------------------ 8-bit codes -----
+# the same min-max scheme with 255 steps, one code per byte
+
+@pytest.mark.parametrize("rows,cols,group", [(1, 64, 64), (3, 128, 64), (17, 4096, 64), (5, 768 * 4, 64),
+                                             (1, 128, 128), (33, 4096, 128), (1000, 384, 128)])
+def test_quantize_b8_lastdim_bit_exact(rows, cols, group):
+    x = si.sweep_tensor(11, rows * cols, row=cols) if rows * cols >= 4096 else si.normal_f16(11, 1, (rows, cols), 0.02)
+    q = _check_quant_equal(x, group=group, bits=8)
+    assert tuple(q.codes.shape) == (rows, cols)
+
+
+def test_quantize_b8_sweep_2pow20_bit_exact():
+    _check_quant_equal(si.sweep_tensor(3, 1 << 20, row=4096), bits=8)
+
+
+def test_quantize_b8_every_fp16_range_bit_exact():
+    # every positive finite fp16 range v, from 0 and from -v: every reachable scale (fp16
+    # subnormal ones included) through the 8-bit division by 255 and the reciprocal
+    v = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float64)
+    t = np.linspace(0.0, 1.0, 64)
+    a = (v[:, None] * t[None, :]).astype(np.float16)
+    b = (v[:, None] * (2.0 * t[None, :] - 1.0)).astype(np.float16)
+    b[:, 0] = (-v).astype(np.float16)
+    b[:, -1] = v.astype(np.float16)
+    _check_quant_equal(np.concatenate([a, b], axis=0), bits=8)
+
+
+def test_quantize_b8_specials():
+    x = np.full((6, 64), 3.0, dtype=np.float16)
+    x[0] = 0
+    x[1] = np.where(np.arange(64) % 3 == 0, np.float16(-0.0), np.float16(0.0))
+    x[2] = 65504
+    x[3, :32] = -65504
+    x[3, 32:] = 65504
+    x[4] = np.concatenate([[0.0, 255.0], np.arange(1, 63)]).astype(np.float16)   # step exactly 1
+    x[5, :8] = [0.0, 255.0, 0.5, 1.5, 2.5, 3.5, 128.5, 254.5]                  # half-even ties
+    q = _check_quant_equal(x, bits=8)
+    assert list(host(q.codes)[5, :8]) == [0, 255, 0, 2, 2, 4, 128, 254]
+
+
+@pytest.mark.parametrize("shape,dim,group", [((6, 128, 5), 1, 64), ((64, 3), 0, 64), ((2, 3, 256, 4), 2, 128)])
+def test_quantize_b8_strided_dims_bit_exact(shape, dim, group):
+    _check_quant_equal(si.normal_f16(12, 2, shape, 1.0), dim=dim, group=group, bits=8)
+
+
+def test_linear_rejects_8bit_weights():
+    wq = fg.fg_quantize(torch.zeros((256, 256), dtype=torch.float16, device="cuda"), dim=1, bits=8)
     with pytest.raises(fg.FgError, match="UNSUPPORTED"):
-        fg.fg_quantize(torch.zeros((2, 64), dtype=torch.float16, device="cuda"), bits=8)
+        fg.fg_linear_w4a16(torch.zeros((4, 256), dtype=torch.float16, device="cuda"), wq)
 
 
 @pytest.mark.slow
