@@ -381,6 +381,15 @@ __global__ void __launch_bounds__(kWarps * 32, D <= 128 ? 5 : 3) attn_decode_ker
           }
         }
       }
+      // V codes of the tile, loaded ahead of the softmax bookkeeping
+      uint32_t v0[VW], v1[VW], v2[VW], v3[VW];
+      {
+        const uint8_t *vrow = Vc + (t0 + c) * RB + gid * (D / 16);
+        load_words<VW>(vrow, v0);
+        load_words<VW>(vrow + 4 * RB, v1);
+        load_words<VW>(vrow + 8 * RB, v2);
+        load_words<VW>(vrow + 12 * RB, v3);
+      }
       // ---- score (log2 units) of token t0+tq ----
       const bool valid = ch * kChunk + t0 + tq < L;
       float sc;
@@ -448,12 +457,6 @@ __global__ void __launch_bounds__(kWarps * 32, D <= 128 ? 5 : 3) attn_decode_ker
         }
         // ---- V codes as the A operand: lane (gid, c) reads its D/8 dims (bytes
         //      gid*D/16 ...) of tokens c, c+4, c+8, c+12 and pairs tokens per 16-bit half ----
-        uint32_t v0[VW], v1[VW], v2[VW], v3[VW];
-        const uint8_t *vrow = Vc + (t0 + c) * RB + gid * (D / 16);
-        load_words<VW>(vrow, v0);
-        load_words<VW>(vrow + 4 * RB, v1);
-        load_words<VW>(vrow + 8 * RB, v2);
-        load_words<VW>(vrow + 12 * RB, v3);
 #pragma unroll
         for (int j = 0; j < VW; j++) {
 #pragma unroll
