@@ -212,10 +212,13 @@ enum {
  * k-segment).  The layer calls use the classic launch.
  * workspace: optional device scratch (16-byte aligned).  The classic launch's
  * split k-range adds its partial sums through the scratch when it holds
- * n_tiles * t_tiles * splits * tile_tokens * 256 * 4 bytes (n_tiles =
+ * P = n_tiles * t_tiles * splits * tile_tokens * 256 * 4 bytes (n_tiles =
  * ceil(N / 256), t_tiles = ceil(M / tile_tokens)), else over distributed shared
- * memory; the two add the splits in the same order, so their results are the
- * same bit for bit.  The persistent launch needs fg_linear_workspace_bytes(M, N,
+ * memory.  With P + n_tiles * t_tiles * splits * 16 bytes (flags after the
+ * partials) and a grid that fits the GPU in one wave, the split ranks run as
+ * separate CTA pairs that meet through the flags; otherwise each tile's ranks
+ * form one cluster.  All of these add the splits in the same order, so their
+ * results are the same bit for bit.  The persistent launch needs fg_linear_workspace_bytes(M, N,
  * K) bytes (its shared tiles' partial sums) and falls back to the classic launch
  * with less; it adds partial sums in another order, so its results may differ
  * from the classic launch's in the last bits (each is deterministic). */
