@@ -75,6 +75,14 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_kv_append_g.argtypes = [P, P, I64, I, P, P, P, P, P, P, P, P, I, I, I, I, I]
         _lib.oracle_attention_x.restype = I
         _lib.oracle_attention_x.argtypes = [P, I64, I, P, P, P, P, P, P, P, P, I, I, I, I, P, I, I]
+        _lib.oracle_w4a8_quantize_weight.restype = I
+        _lib.oracle_w4a8_quantize_weight.argtypes = [P, I, I, P, P, P, P]
+        _lib.oracle_w4a8_weight_int8.restype = I
+        _lib.oracle_w4a8_weight_int8.argtypes = [P, P, P, I, I, P]
+        _lib.oracle_act8_quantize.restype = I
+        _lib.oracle_act8_quantize.argtypes = [P, I, I, P, P]
+        _lib.oracle_linear_w4a8.restype = I
+        _lib.oracle_linear_w4a8.argtypes = [P, P, I, I, P, P, P, P, I, P, P, I, I, D, P, P]
         _lib.oracle_layer_rows.restype = I
         _lib.oracle_layer_rows.argtypes = ([P, D] + [P] * 16 + [P] * 4 + [P] * 6 + [I, I] + [P, I, P, P, I, P, P, I])
     return _lib
@@ -181,6 +189,73 @@ def linear(x, w: Packed, bias=None, residual=None, relu: bool = False,
                                int(relu), int(qscale_cols), float(qscale), _p(y), w.group)
     assert rc == 0
     return y
+
+
+# --------------------------------------------------------------------------------------
+# W4A8: two-level 4-bit weights and per-row 8-bit activations, integer products (the QServe
+# W4A8KV4 entry of the PIPO paper's references, by title; "Optimizing LLM for low memory
+# usage", Quantization and Weight Compression).  The scheme is a reading: fg_oracle.c states it.
+# --------------------------------------------------------------------------------------
+
+class W4A8Weight:
+    """codes uint8 [N, K/2] (low nibble = even k), gmin int8 [N, K/64], gstep uint8 [N, K/64],
+    cscale float32 [N]; the product's 8-bit weight is gmin + code * gstep, the real weight
+    cscale * that."""
+
+    def __init__(self, codes, gmin, gstep, cscale):
+        self.codes, self.gmin, self.gstep, self.cscale = codes, gmin, gstep, cscale
+        self.N, self.K = codes.shape[0], codes.shape[1] * 2
+
+
+def w4a8_quantize_weight(w) -> W4A8Weight:
+    w = _u16(w)
+    N, K = w.shape
+    if K % GROUP:
+        raise ValueError("K must be a multiple of 64")
+    codes = np.empty((N, K // 2), np.uint8)
+    gmin = np.empty((N, K // GROUP), np.int8)
+    gstep = np.empty((N, K // GROUP), np.uint8)
+    cscale = np.empty(N, np.float32)
+    assert lib().oracle_w4a8_quantize_weight(_p(w), N, K, _p(codes), _p(gmin), _p(gstep), _p(cscale)) == 0
+    return W4A8Weight(codes, gmin, gstep, cscale)
+
+
+def w4a8_weight_int8(q: W4A8Weight) -> np.ndarray:
+    """The 8-bit weights [N, K] the integer product uses."""
+    w8 = np.empty((q.N, q.K), np.int8)
+    assert lib().oracle_w4a8_weight_int8(_p(np.ascontiguousarray(q.codes)), _p(np.ascontiguousarray(q.gmin)),
+                                         _p(np.ascontiguousarray(q.gstep)), q.N, q.K, _p(w8)) == 0
+    return w8
+
+
+def act8_quantize(x):
+    """Per-row symmetric 8-bit activations: (a8 int8 [M, K], ascale float32 [M])."""
+    x = _u16(x)
+    M, K = x.shape
+    a8 = np.empty((M, K), np.int8)
+    ascale = np.empty(M, np.float32)
+    assert lib().oracle_act8_quantize(_p(x), M, K, _p(a8), _p(ascale)) == 0
+    return a8, ascale
+
+
+def linear_w4a8(a8, ascale, w: W4A8Weight, bias=None, residual=None, relu: bool = False,
+                qscale_cols: int = 0, qscale: float = 1.0, with_acc: bool = False):
+    """``epi(acc * ascale[t] * cscale[n] + bias)`` in float64 with the exact integer sums
+    ``acc = a8 @ w8.T``; with ``with_acc`` also returns acc (int64)."""
+    a8 = np.ascontiguousarray(a8, dtype=np.int8)
+    ascale = np.ascontiguousarray(ascale, dtype=np.float32)
+    M, K = a8.shape
+    assert K == w.K
+    y = np.empty((M, w.N), np.float64)
+    acc = np.empty((M, w.N), np.int64) if with_acc else None
+    rc = lib().oracle_linear_w4a8(_p(a8), _p(ascale), M, K, _p(np.ascontiguousarray(w.codes)),
+                                  _p(np.ascontiguousarray(w.gmin)), _p(np.ascontiguousarray(w.gstep)),
+                                  _p(np.ascontiguousarray(w.cscale)), w.N,
+                                  _p(None if bias is None else _u16(bias)),
+                                  _p(None if residual is None else _u16(residual)),
+                                  int(relu), int(qscale_cols), float(qscale), _p(y), _p(acc))
+    assert rc == 0
+    return (y, acc) if with_acc else y
 
 
 def layernorm(x, gamma=None, beta=None, eps: float = 1e-5) -> np.ndarray:

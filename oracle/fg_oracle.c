@@ -635,3 +635,151 @@ int oracle_layer_rows(const int *dims, double eps,
     free(c.bqkv); free(c.bo); free(c.b1); free(c.b2); free(c.g1); free(c.be1); free(c.g2); free(c.be2);
     return 0;
 }
+
+/* ------------------------------------------------------------------------- */
+/* W4A8: 4-bit weights, 8-bit activations, integer products                  */
+/* ------------------------------------------------------------------------- */
+/*
+ * What it follows: the W4A8KV4 entry (QServe) in the PIPO paper's list of references,
+ * by its title only; the "Optimizing LLM for low memory usage" page, section
+ * "Quantization and Weight Compression" (weights mapped to INT8 or INT4); [G3] for the
+ * groups of 64 along the input dimension.  The pages give no scheme, so this is the
+ * reading (listed with the others in the design notes):
+ *
+ * Weights [N][K], two levels:
+ *   1. per output row n: amax = max_k |w|; amax == 0 -> cscale = 0, every w8 = 0; else
+ *      inv = 113 / amax and cscale = amax / 113 (each one fp32 division),
+ *      w8 = clamp(round_half_even(w * inv), -113, 113)  (one fp32 multiply);
+ *   2. per group of 64 along k, in the integer domain: mn = min w8, mx = max w8,
+ *      step = max(1, ceil((mx - mn) / 15)), code = floor((2 (w8 - mn) + step) / (2 step))
+ *      (nearest, halves up; at most 15 because mx - mn <= 15 step), two codes per byte,
+ *      even element in the low nibble; gmin = mn (int8), gstep = step (uint8, 1..16).
+ *   The 8-bit weight the product uses is mn + code * step.  113 is the largest bound for
+ *   which that value stays in int8 whatever the group: mn + 15 step <= mx + 14 <= 127.
+ * Activations [M][K], per row t: amax = max_k |x|; amax == 0 -> ascale = 0, a8 = 0; else
+ *   inv = 127 / amax, ascale = amax / 127, a8 = clamp(round_half_even(x * inv), -127, 127),
+ *   the same fp32 operations as level 1.
+ * Product: acc[t][n] = sum_k a8[t][k] * (mn + code * step)[n][k], exact (int64 here);
+ *   y = acc * (ascale[t] * cscale[n]) + bias[n], then the q-scale of the first qscale_cols
+ *   outputs, ReLU and the fp16 residual as in oracle_linear, in float64.
+ */
+#define OR_W8_BOUND 113
+#define OR_A8_BOUND 127
+
+/* round-half-even of x * inv (fp32 multiply), clamped to [-bound, bound] */
+static int q8_of(float x, float inv, int bound)
+{
+    float t = x * inv;
+    int c = (int)nearbyintf(t);
+    if (c < -bound) c = -bound;
+    if (c > bound) c = bound;
+    return c;
+}
+
+/* One row of n fp16 values -> symmetric 8-bit codes and the row's fp32 scale. */
+static void quantize_row_sym8(const uint16_t *x, int64_t n, int bound, int *q, float *scale)
+{
+    float amax = 0.0f;
+    for (int64_t k = 0; k < n; k++) {
+        float a = fabsf(oracle_f16_to_f32(x[k]));
+        if (a > amax) amax = a;
+    }
+    if (amax == 0.0f) {
+        *scale = 0.0f;
+        for (int64_t k = 0; k < n; k++) q[k] = 0;
+        return;
+    }
+    float inv = (float)bound / amax;
+    *scale = amax / (float)bound;
+    for (int64_t k = 0; k < n; k++) q[k] = q8_of(oracle_f16_to_f32(x[k]), inv, bound);
+}
+
+int oracle_w4a8_quantize_weight(const uint16_t *w, int N, int K, uint8_t *codes, int8_t *gmin,
+                                uint8_t *gstep, float *cscale)
+{
+    if (N < 0 || K <= 0 || K % OR_GROUP) return -1;
+    int *w8 = (int *)malloc(sizeof(int) * (size_t)K);
+    if (!w8) return -2;
+    int ng = K / OR_GROUP;
+    for (int64_t n = 0; n < N; n++) {
+        quantize_row_sym8(w + n * K, K, OR_W8_BOUND, w8, &cscale[n]);
+        for (int g = 0; g < ng; g++) {
+            const int *v = w8 + g * OR_GROUP;
+            int mn = v[0], mx = v[0];
+            for (int i = 1; i < OR_GROUP; i++) {
+                if (v[i] < mn) mn = v[i];
+                if (v[i] > mx) mx = v[i];
+            }
+            int step = (mx - mn + 14) / 15;
+            if (step < 1) step = 1;
+            uint8_t *cp = codes + n * (K / 2) + g * (OR_GROUP / 2);
+            for (int j = 0; j < OR_GROUP / 2; j++) {
+                int c0 = (2 * (v[2 * j] - mn) + step) / (2 * step);
+                int c1 = (2 * (v[2 * j + 1] - mn) + step) / (2 * step);
+                cp[j] = (uint8_t)(c0 | (c1 << 4));
+            }
+            gmin[n * ng + g] = (int8_t)mn;
+            gstep[n * ng + g] = (uint8_t)step;
+        }
+    }
+    free(w8);
+    return 0;
+}
+
+/* The 8-bit weights the product uses: w8[n][k] = gmin + code * gstep. */
+int oracle_w4a8_weight_int8(const uint8_t *codes, const int8_t *gmin, const uint8_t *gstep, int N, int K,
+                            int8_t *w8)
+{
+    if (N < 0 || K <= 0 || K % OR_GROUP) return -1;
+    int ng = K / OR_GROUP;
+    for (int64_t n = 0; n < N; n++)
+        for (int k = 0; k < K; k++) {
+            uint8_t byte = codes[n * (K / 2) + k / 2];
+            int q = (k & 1) ? (byte >> 4) : (byte & 15);
+            int64_t g = n * ng + k / OR_GROUP;
+            int v = gmin[g] + q * gstep[g];
+            if (v < -128 || v > 127) return -3;   /* cannot happen for weights quantised above */
+            w8[n * K + k] = (int8_t)v;
+        }
+    return 0;
+}
+
+int oracle_act8_quantize(const uint16_t *x, int M, int K, int8_t *a8, float *ascale)
+{
+    if (M < 0 || K <= 0) return -1;
+    int *q = (int *)malloc(sizeof(int) * (size_t)K);
+    if (!q) return -2;
+    for (int64_t t = 0; t < M; t++) {
+        quantize_row_sym8(x + t * K, K, OR_A8_BOUND, q, &ascale[t]);
+        for (int k = 0; k < K; k++) a8[t * K + k] = (int8_t)q[k];
+    }
+    free(q);
+    return 0;
+}
+
+/* y[t][n] in float64; acc_out (optional) receives the exact integer sums [M][N]. */
+int oracle_linear_w4a8(const int8_t *a8, const float *ascale, int M, int K,
+                       const uint8_t *codes, const int8_t *gmin, const uint8_t *gstep, const float *cscale, int N,
+                       const uint16_t *bias, const uint16_t *residual, int relu, int qscale_cols, double qscale,
+                       double *y, int64_t *acc_out)
+{
+    if (M < 0 || N < 0 || K <= 0 || K % OR_GROUP) return -1;
+    int8_t *W = (int8_t *)malloc((size_t)N * K + 1);
+    if (!W) return -2;
+    if (oracle_w4a8_weight_int8(codes, gmin, gstep, N, K, W)) { free(W); return -3; }
+    for (int64_t t = 0; t < M; t++)
+        for (int64_t n = 0; n < N; n++) {
+            const int8_t *ar = a8 + t * K, *wr = W + n * K;
+            int64_t acc = 0;
+            for (int k = 0; k < K; k++) acc += (int64_t)ar[k] * (int64_t)wr[k];
+            if (acc_out) acc_out[t * N + n] = acc;
+            double v = (double)acc * ((double)ascale[t] * (double)cscale[n]);
+            if (bias) v += oracle_f16_to_f64(bias[n]);
+            if (n < qscale_cols) v *= qscale;
+            if (relu && v < 0.0) v = 0.0;
+            if (residual) v += oracle_f16_to_f64(residual[t * N + n]);
+            y[t * N + n] = v;
+        }
+    free(W);
+    return 0;
+}
