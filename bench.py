@@ -828,6 +828,22 @@ def run_kernel(args, wl):
         zero = torch.zeros((S,), dtype=torch.int32, device=dev)
         run = lambda: fg.fg_attention_decode(cache, q, zero, rows_per_seq=P, out=out, stream=stream)
         work, unit, peak = 4 * d * H * S * P * (P + 1) // 2, "TFLOP/s", peaks["tc_burst"]
+    elif args.kernel.endswith("_gemm_w4a8"):
+        # the W4A8 variant of a decode GEMM: int8 activations (quantised once, outside the timed
+        # launches) times two-level 4-bit weights on the integer tensor cores; the peak is the
+        # measured fp16 GEMM peak x 2, the nominal int8 / fp16 dense ratio (4.5 / 2.25 PFLOP/s)
+        N, K = {"qkv": (3 * h, h), "out": (h, h), "fc1": (F, h), "fc2": (h, F)}[args.kernel[:-len("_gemm_w4a8")]]
+        x = torch.randn((S, K), generator=g, device=dev, dtype=torch.float16)
+        wq = fg.fg_w4a8_quantize_weight(torch.randn((N, K), generator=g, device=dev, dtype=torch.float16) * 0.02)
+        a8, asc = fg.fg_act8_quantize(x)
+        y = torch.empty((S, N), dtype=torch.float16, device=dev)
+        run = lambda: fg.fg_linear_w4a8(a8, asc, wq, out=y, stream=stream)
+        work, unit, peak = 2 * S * N * K, "TOP/s", peaks["tc_burst"] * 2
+    elif args.kernel == "act8_quantize":
+        x = torch.randn((S, F), generator=g, device=dev, dtype=torch.float16)
+        a8, asc = fg.fg_act8_quantize(x)
+        run = lambda: fg.fg_act8_quantize(x, a8, asc, stream=stream)
+        work, unit, peak = S * F * 3 + S * 4, "GB/s", peaks["hbm"]
     elif args.kernel.endswith("_gemm"):
         N, K = {"qkv_gemm": (3 * h, h), "out_gemm": (h, h), "fc1_gemm": (F, h), "fc2_gemm": (h, F)}[args.kernel]
         x = torch.randn((S, K), generator=g, device=dev, dtype=torch.float16)
@@ -866,9 +882,11 @@ def run_kernel(args, wl):
     fg.fg_sync_status()
     t = sorted(a.elapsed_time(b) / 1e3 for a, b in ev)
     med = t[len(t) // 2]
-    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    scale = 1e12 if unit in ("TFLOP/s", "TOP/s") else 1e9
     line = {"kernel": args.kernel, "group": args.group, "workload": args.workload, "seqs": S,
-            "gemm_scratch": args.gemm_scratch if args.kernel.endswith("_gemm") else None, "median_us": med * 1e6,
+            "gemm_scratch": args.gemm_scratch if args.kernel.endswith("_gemm") else None,
+            "plan": fg.fg_linear_w4a8_plan(S, N, K) if args.kernel.endswith("_gemm_w4a8") else None,
+            "median_us": med * 1e6,
             "min_us": t[0] * 1e6, "achieved": work / med / scale, "unit": unit, "peak": peak,
             "frac": work / med / scale / peak}
     if args.kernel in ("quantize", "dequantize") and not args.no_cpu_baseline:

@@ -58,6 +58,11 @@ class fg_layer_weights(Structure):
         (n, c_void_p) for n in ("bqkv", "bo", "b1", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b")]
 
 
+class fg_w4a8_weight(Structure):
+    _fields_ = [("codes", c_void_p), ("gmin", c_void_p), ("gstep", c_void_p), ("cscale", c_void_p),
+                ("N", c_int64), ("K", c_int64)]
+
+
 def _decl(name, restype, *args):
     f = getattr(_lib, name)
     f.restype = restype
@@ -80,6 +85,10 @@ _decl("fg_linear_workspace_bytes", c_size_t, c_int, c_int, c_int)
 _decl("fg_linear_plan", c_int, c_int, c_int, c_int, POINTER(c_int), POINTER(c_int), POINTER(c_int))
 _decl("fg_linear_w4a16", c_int, P, c_int, c_int, POINTER(fg_qtensor), P, P, c_int, c_int, c_float, P, P, c_size_t, P)
 _decl("fg_layernorm", c_int, P, c_int, c_int, P, P, c_float, P, P)
+_decl("fg_w4a8_quantize_weight", c_int, P, POINTER(fg_w4a8_weight), P)
+_decl("fg_act8_quantize", c_int, P, c_int, c_int, P, P, P)
+_decl("fg_linear_w4a8", c_int, P, P, c_int, c_int, POINTER(fg_w4a8_weight), P, P, c_int, c_int, c_float, P, P)
+_decl("fg_linear_w4a8_plan", c_int, c_int, c_int, c_int, POINTER(c_int), POINTER(c_int))
 _decl("fg_layer_blob_bytes", c_size_t, POINTER(fg_layer_config))
 _decl("fg_layer_weights_from_blob", c_int, POINTER(fg_layer_config), P, POINTER(fg_layer_weights))
 _decl("fg_layer_workspace_bytes", c_size_t, POINTER(fg_layer_config), c_int)
@@ -327,6 +336,68 @@ def fg_linear_w4a16(x: torch.Tensor, w: QTensor, bias=None, residual=None, relu:
     _check(_lib.fg_linear_w4a16(_ptr(x), M, K, ctypes.byref(s), _ptr(bias), _ptr(residual), flags, qscale_cols,
                                 qscale, _ptr(out), _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                 _stream(stream)), "fg_linear_w4a16")
+    return out
+
+
+# ---------------------------------------------------------------------------------------
+# W4A8: 4-bit weights, 8-bit activations, integer products ([Q8] in fg.h)
+# ---------------------------------------------------------------------------------------
+
+class W4A8Weight:
+    """Device W4A8 weight: codes uint8 [N, K/2], gmin int8 [N, K/64], gstep uint8 [N, K/64],
+    cscale float32 [N]."""
+
+    def __init__(self, N: int, K: int, device="cuda"):
+        self.N, self.K = N, K
+        self.codes = torch.empty((N, K // 2), dtype=torch.uint8, device=device)
+        self.gmin = torch.empty((N, K // 64), dtype=torch.int8, device=device)
+        self.gstep = torch.empty((N, K // 64), dtype=torch.uint8, device=device)
+        self.cscale = torch.empty(N, dtype=torch.float32, device=device)
+
+    def struct(self) -> fg_w4a8_weight:
+        return fg_w4a8_weight(self.codes.data_ptr(), self.gmin.data_ptr(), self.gstep.data_ptr(),
+                              self.cscale.data_ptr(), self.N, self.K)
+
+
+def fg_w4a8_quantize_weight(w: torch.Tensor, out: W4A8Weight = None, stream=None) -> W4A8Weight:
+    _need(w, torch.float16, "w")
+    N, K = w.shape
+    if out is None:
+        out = W4A8Weight(N, K, device=w.device)
+    s = out.struct()
+    _check(_lib.fg_w4a8_quantize_weight(_ptr(w), ctypes.byref(s), _stream(stream)), "fg_w4a8_quantize_weight")
+    return out
+
+
+def fg_act8_quantize(x: torch.Tensor, a8=None, ascale=None, stream=None):
+    """(a8 int8 [M, K], ascale float32 [M])."""
+    _need(x, torch.float16, "x")
+    M, K = x.shape
+    if a8 is None:
+        a8 = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if ascale is None:
+        ascale = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(_lib.fg_act8_quantize(_ptr(x), M, K, _ptr(a8), _ptr(ascale), _stream(stream)), "fg_act8_quantize")
+    return a8, ascale
+
+
+def fg_linear_w4a8_plan(M: int, N: int, K: int) -> tuple:
+    t, s = c_int(), c_int()
+    _check(_lib.fg_linear_w4a8_plan(M, N, K, ctypes.byref(t), ctypes.byref(s)), "fg_linear_w4a8_plan")
+    return t.value, s.value
+
+
+def fg_linear_w4a8(a8: torch.Tensor, ascale: torch.Tensor, w: W4A8Weight, bias=None, residual=None,
+                   relu: bool = False, qscale_cols: int = 0, qscale: float = 1.0, out=None, stream=None):
+    _need(a8, torch.int8, "a8")
+    _need(ascale, torch.float32, "ascale")
+    M, K = a8.shape
+    if out is None:
+        out = torch.empty((M, w.N), dtype=torch.float16, device=a8.device)
+    flags = (FG_EPI_RELU if relu else 0) | (FG_EPI_RESIDUAL if residual is not None else 0)
+    s = w.struct()
+    _check(_lib.fg_linear_w4a8(_ptr(a8), _ptr(ascale), M, K, ctypes.byref(s), _ptr(bias), _ptr(residual), flags,
+                               qscale_cols, qscale, _ptr(out), _stream(stream)), "fg_linear_w4a8")
     return out
 
 

@@ -12,6 +12,9 @@
  *        CPU memory and moved to the GPU layer by layer.
  *   [OPT] the OPT entry of the PIPO paper's reference list -- the model family
  *        (pre-LayerNorm decoder layer, multi-head attention, ReLU FFN).
+ *   [Q8] the QServe W4A8KV4 entry of the same list (title only) and the
+ *        "Optimizing LLM for low memory usage" page, section "Quantization and
+ *        Weight Compression" (INT8 and INT4 weight formats) -- the W4A8 variant.
  *
  * The 4-bit format (the pages give no formula; this is the reading the whole
  * library and its tests use).  For every group of G consecutive fp16 values
@@ -237,6 +240,53 @@ FG_API fg_status fg_linear_plan(int M, int N, int K, int *tile_tokens, int *spli
 FG_API fg_status fg_linear_w4a16(const fg_half *x, int M, int K, const fg_qtensor *w, const fg_half *bias,
                           const fg_half *residual, int flags, int qscale_cols, float qscale,
                           fg_half *y, void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* W4A8 linear layer: 4-bit weights, 8-bit activations, integer products   */
+/* ---------------------------------------------------------------------- */
+/* [Q8] The pages name W4A8 only through the QServe W4A8KV4 title in the PIPO paper's list of
+ * references, and list INT8 and INT4 among post-training weight formats ("Optimizing LLM for
+ * low memory usage", Quantization and Weight Compression); groups of 64 along the input
+ * dimension as in [G3].  The scheme (a reading of those pages):
+ *   weights [N][K], two levels: per row n, cscale = amax / 113 and w8 = clamp(round_half_even(
+ *     w * (113 / amax)), -113, 113) (each one IEEE fp32 operation; amax = 0 gives cscale 0 and
+ *     w8 0); per group g of 64 along k, gmin = min w8, gstep = max(1, ceil((max w8 - gmin) / 15))
+ *     (1..16) and code = floor((2 (w8 - gmin) + gstep) / (2 gstep)) (0..15), two codes per byte,
+ *     the even element in the low nibble.  The product's weight is gmin + code * gstep, an int8
+ *     for every group (gmin + 15 gstep <= max w8 + 14 <= 127);
+ *   activations [M][K]: per row t, ascale = amax / 127, a8 = clamp(round_half_even(x * (127 /
+ *     amax)), -127, 127) (amax = 0: ascale 0, a8 0);
+ *   y[t][n] = epi( acc * (ascale[t] * cscale[n]) + bias[n] ), acc = sum_k a8[t][k] *
+ *     (gmin + code * gstep)[n][k] exact in int32 on the tensor cores (tcgen05 kind::i8), then one
+ *     fp32 operation at a time: the scale product, acc * it, + bias, q-scale of the first
+ *     qscale_cols outputs, ReLU (FG_EPI_RELU), + residual (FG_EPI_RESIDUAL), round to fp16. */
+typedef struct {
+    uint8_t *codes;   /* [N][K/2] */
+    int8_t *gmin;     /* [N][K/64] */
+    uint8_t *gstep;   /* [N][K/64], 1..16 (other values give unspecified results) */
+    float *cscale;    /* [N] */
+    int64_t N, K;
+} fg_w4a8_weight;
+/* Quantises fp16 weights w [N][K] (device, row-major, 16-byte aligned) into *out (device arrays
+ * the caller owns, codes 16-byte aligned, cscale 4-byte aligned).  K % 64 == 0, N >= 1
+ * (FG_ERR_SHAPE otherwise).  One CTA per row. */
+FG_API fg_status fg_w4a8_quantize_weight(const fg_half *w, const fg_w4a8_weight *out, void *stream);
+/* Quantises fp16 activations x [M][K] (device, 16-byte aligned) to a8 [M][K] (16-byte aligned)
+ * and ascale [M] (fp32).  K % 64 == 0 (FG_ERR_SHAPE otherwise).  One CTA per row. */
+FG_API fg_status fg_act8_quantize(const fg_half *x, int M, int K, int8_t *a8, float *ascale, void *stream);
+/* The W4A8 product above: a8 [M][K] int8 and ascale [M] from fg_act8_quantize, w from
+ * fg_w4a8_quantize_weight with w->K == K, bias fp16 [N] or NULL, residual fp16 [M][N].
+ * K % 128 == 0 and K <= 65536 (the int32 sums stay exact), N % 128 == 0 (FG_ERR_SHAPE);
+ * a8, y and the codes 16-byte aligned, gmin and gstep 2-byte aligned (FG_ERR_INVALID).
+ * One SM per output tile of 256 features x tile_tokens tokens; the k-range may be split over a
+ * cluster whose CTAs add their int32 partial sums exactly, so the result does not depend on
+ * the plan. */
+FG_API fg_status fg_linear_w4a8(const int8_t *a8, const float *ascale, int M, int K, const fg_w4a8_weight *w,
+                         const fg_half *bias, const fg_half *residual, int flags, int qscale_cols,
+                         float qscale, fg_half *y, void *stream);
+/* The launch fg_linear_w4a8 makes for this shape on the current device (no launch):
+ * *tile_tokens 16..256, *splits 1..8 (FG_ERR_INVALID for shapes it rejects). */
+FG_API fg_status fg_linear_w4a8_plan(int M, int N, int K, int *tile_tokens, int *splits);
 
 /* y = (x - mean) / sqrt(var + eps) * gamma + beta per row (fp32 statistics,
  * biased variance), fp16 in/out, gamma/beta fp16 [h] (NULL = 1 / 0).

@@ -240,3 +240,39 @@ def test_attention_decode_append_validates_on_host():
     assert _rc("fg_attention_decode_append", *args(ldq=260)) == 2      # stride not a multiple of 8
     bad = _fake_kv(maxL=100)                                           # max_len not a multiple of 64
     assert _rc("fg_attention_decode_append", *args(kv=bad)) == 2
+
+
+def _fake_w4a8(N=256, K=512):
+    w = B.fg_w4a8_weight()
+    w.codes, w.gmin, w.gstep, w.cscale = 0x100000, 0x200000, 0x300000, 0x400000
+    w.N, w.K = N, K
+    return w
+
+
+def test_w4a8_entry_points_validate_on_host():
+    P = 0x800000                                            # aligned, never dereferenced
+    w = _fake_w4a8()
+    lin = lambda **o: [o.get("a8", P), o.get("ascale", P * 2), o.get("M", 8), o.get("K", 512),
+                       ctypes.byref(o.get("w", w)), None, o.get("res", None), o.get("flags", 0), 0, 1.0,
+                       o.get("y", P * 3), None]
+    assert _rc("fg_linear_w4a8", *lin(K=448)) == 2                     # K differs from the weight's
+    assert _rc("fg_linear_w4a8", *lin(w=_fake_w4a8(K=448), K=448)) == 2  # K not a multiple of 128
+    assert _rc("fg_linear_w4a8", *lin(w=_fake_w4a8(K=65536 + 128), K=65536 + 128)) == 2  # int32 sums
+    assert _rc("fg_linear_w4a8", *lin(w=_fake_w4a8(N=192))) == 2       # N not a multiple of 128
+    assert _rc("fg_linear_w4a8", *lin(M=-1)) == 1
+    assert _rc("fg_linear_w4a8", *lin(M=0)) == 0                       # nothing to do
+    assert _rc("fg_linear_w4a8", *lin(flags=4)) == 1                   # no persistent launch here
+    assert _rc("fg_linear_w4a8", *lin(flags=2)) == 1                   # residual flag without residual
+    assert _rc("fg_linear_w4a8", *lin(a8=P + 8)) == 1                  # misaligned activations
+    assert _rc("fg_linear_w4a8", *lin(y=None)) == 1
+    odd = _fake_w4a8()
+    odd.gmin = 0x200001                                                # metadata read 2 bytes at a time
+    assert _rc("fg_linear_w4a8", *lin(w=odd)) == 1
+    assert _rc("fg_act8_quantize", P, 4, 96, P * 2, P * 3, None) == 2  # K not a multiple of 64
+    assert _rc("fg_act8_quantize", P, 0, 128, P * 2, P * 3, None) == 0
+    assert _rc("fg_act8_quantize", P + 2, 4, 128, P * 2, P * 3, None) == 1
+    assert _rc("fg_w4a8_quantize_weight", P, ctypes.byref(_fake_w4a8(K=96)), None) == 2
+    assert _rc("fg_w4a8_quantize_weight", P, ctypes.byref(_fake_w4a8(N=0)), None) == 2
+    assert _rc("fg_w4a8_quantize_weight", None, ctypes.byref(w), None) == 1
+    t, s = ctypes.c_int(), ctypes.c_int()
+    assert B.lib().fg_linear_w4a8_plan(8, 256, 448, ctypes.byref(t), ctypes.byref(s)) == 1
