@@ -10,6 +10,6 @@ from ._binding import (  # noqa: F401
     fg_linear_w4a16, fg_linear_plan, fg_linear_workspace_bytes, fg_qtensor_bytes, fg_quantize, fg_status_string, fg_sync_status,
     fg_profile_enable, fg_profile_collect, PROFILE_SLOTS, fg_layer_decode_noalloc, NOALLOC_SCRATCH_BYTES,
     fg_linear_plan_pairs, fg_linear_classic_scratch_bytes, fg_test_gemm_stall,
-    W4A8Weight, fg_w4a8_quantize_weight, fg_act8_quantize, fg_linear_w4a8, fg_linear_w4a8_plan,
+    W4A8Weight, fg_w4a8_quantize_weight, fg_act8_quantize, fg_linear_w4a8, fg_linear_w4a8_plan, fg_linear_w4a8_workspace_bytes,
     lib, weights_struct,
 )

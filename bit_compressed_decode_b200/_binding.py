@@ -87,7 +87,9 @@ _decl("fg_linear_w4a16", c_int, P, c_int, c_int, POINTER(fg_qtensor), P, P, c_in
 _decl("fg_layernorm", c_int, P, c_int, c_int, P, P, c_float, P, P)
 _decl("fg_w4a8_quantize_weight", c_int, P, POINTER(fg_w4a8_weight), P)
 _decl("fg_act8_quantize", c_int, P, c_int, c_int, P, P, P)
-_decl("fg_linear_w4a8", c_int, P, P, c_int, c_int, POINTER(fg_w4a8_weight), P, P, c_int, c_int, c_float, P, P)
+_decl("fg_linear_w4a8", c_int, P, P, c_int, c_int, POINTER(fg_w4a8_weight), P, P, c_int, c_int, c_float, P, P,
+      c_size_t, P)
+_decl("fg_linear_w4a8_workspace_bytes", c_size_t, c_int, c_int, c_int)
 _decl("fg_linear_w4a8_plan", c_int, c_int, c_int, c_int, POINTER(c_int), POINTER(c_int))
 _decl("fg_layer_blob_bytes", c_size_t, POINTER(fg_layer_config))
 _decl("fg_layer_weights_from_blob", c_int, POINTER(fg_layer_config), P, POINTER(fg_layer_weights))
@@ -387,17 +389,28 @@ def fg_linear_w4a8_plan(M: int, N: int, K: int) -> tuple:
     return t.value, s.value
 
 
+def fg_linear_w4a8_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_lib.fg_linear_w4a8_workspace_bytes(M, N, K))
+
+
 def fg_linear_w4a8(a8: torch.Tensor, ascale: torch.Tensor, w: W4A8Weight, bias=None, residual=None,
-                   relu: bool = False, qscale_cols: int = 0, qscale: float = 1.0, out=None, stream=None):
+                   relu: bool = False, qscale_cols: int = 0, qscale: float = 1.0, out=None, workspace=None,
+                   stream=None):
+    """``workspace``: None allocates the scratch the CTA-pair launch can use; a tensor is passed
+    as given (a 0-element one means none: k splits are then added on chip)."""
     _need(a8, torch.int8, "a8")
     _need(ascale, torch.float32, "ascale")
     M, K = a8.shape
     if out is None:
         out = torch.empty((M, w.N), dtype=torch.float16, device=a8.device)
+    if workspace is None:
+        need = fg_linear_w4a8_workspace_bytes(M, w.N, K)
+        workspace = torch.empty(need, dtype=torch.uint8, device=a8.device) if need else None
     flags = (FG_EPI_RELU if relu else 0) | (FG_EPI_RESIDUAL if residual is not None else 0)
     s = w.struct()
     _check(_lib.fg_linear_w4a8(_ptr(a8), _ptr(ascale), M, K, ctypes.byref(s), _ptr(bias), _ptr(residual), flags,
-                               qscale_cols, qscale, _ptr(out), _stream(stream)), "fg_linear_w4a8")
+                               qscale_cols, qscale, _ptr(out), _ptr(workspace),
+                               0 if workspace is None else workspace.numel(), _stream(stream)), "fg_linear_w4a8")
     return out
 
 

@@ -80,6 +80,8 @@ struct GemmArgs {
                               // publish their partials with these [tile][rank][CTA half] flags
   unsigned long long epoch;   // the launch's flag value
   unsigned int *err;
+  const float *ascale; // W4A8 pair kernel: per-token activation scales [M]
+  const float *cscale; // W4A8 pair kernel: per-row weight scales [N]
   uint64_t wait_ns;    // one-SM kernel: limit of every pipeline wait (FG_WAIT_TIMEOUT_NS unless a test shortens it)
   int stall;           // one-SM kernel, test hook: the dequantising warps withhold their first-stage arrival
 };
@@ -369,11 +371,13 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemm_kernel(const __grid_co
 //   shared-memory traffic for 8 MFLOP.
 //   warps 0..7   dequantise (thread: row tid % 128, k half tid / 128), then the epilogue
 //                (warp: TMEM lane quarter warp % 4, token tile warp / 4);
-//   warp 8       TMA of this CTA's x halves, completing on the even CTA's barrier, and of this
-//                CTA's packed weights: the codes of each k-tile (128 rows x 32 B, a ring of
-//                kPairCodeStages slots running ahead of the dequant warps) and the fp16 group
-//                mins and scales, 8 group columns at a time (two buffers) -- one tensor copy
-//                each instead of a scattered 16-byte and two 2-byte loads per thread and k-tile;
+//   warp 8       lane 0: TMA of this CTA's x halves, completing on the even CTA's barrier;
+//                lane 1: TMA of this CTA's packed weights: the codes of each k-tile (128 rows x
+//                32 B, a 24 KB ring running ahead of the dequant warps) and the fp16 group mins
+//                and scales, 8 group columns at a time (two buffers) -- one tensor copy each
+//                instead of a scattered 16-byte and two 2-byte loads per thread and k-tile.  A
+//                code slot is released once its codes have been used, after a proxy fence (the
+//                tensor copy that refills it must not overtake the generic-proxy reads);
 //   warp 9       even CTA: the MMA issuer; odd CTA: forwards "A half ready" to the even
 //                CTA (a 16-byte bulk copy completing on its barrier); TMEM allocation.
 //   Split k-ranges of one pair tile form the cluster's z dimension (cluster 2 x 1 x splits);
@@ -404,19 +408,67 @@ struct PairCfg {
   static_assert(kStages * kStage == kPairRing, "ring");
 };
 constexpr uint32_t kPairIdesc = umma_idesc_f16_f32(256, 256);
+// Instruction descriptor of the W4A8 form: kind::i8, signed 8-bit A and B, s32 D, K-major.
+constexpr uint32_t kPairIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(256 >> 3) << 17) |
+                                  (static_cast<uint32_t>(256 >> 4) << 24);
+// The two operand widths of the pair kernel.  W4A16: fp16 operands, k-tiles of 64 (one group),
+// 32 code bytes per row and k-tile, fp16 mins and scales 8 group columns per tensor copy.  W4A8:
+// int8 operands, k-tiles of 128 (two groups, the same 128-byte rows), 64 code bytes per row and
+// k-tile, int8 minima and uint8 steps 16 group columns per tensor copy.  Both stage 24 KB of codes
+// and 2 KB per metadata buffer.
+template <bool I8>
+struct PairW {
+  static constexpr int kK = I8 ? 128 : 64;
+  static constexpr int kCodeRow = I8 ? 64 : 32;
+  static constexpr int kCodeBytes = 128 * kCodeRow;
+  static constexpr int kCodeStages = (kPairCodeStages * kPairCodeBytes) / kCodeBytes;
+  static constexpr int kMetaCols = I8 ? 16 : 8;
+  static_assert(kCodeStages * kCodeBytes == kPairCodeStages * kPairCodeBytes, "code ring");
+  static_assert(kMetaCols * 128 * (I8 ? 1 : 2) == kPairMetaBytes, "metadata buffer");
+};
+
+// D (+)= A * B^T over the pair, int8 operands, int32 accumulation.
+__device__ __forceinline__ void umma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 8 codes of one word (element 2j in the low nibble of byte j) -> the 8 int8 weights
+// gmin + code * step in element order, as two words (code * step <= 240: no carry between
+// bytes; the per-byte add wraps to the two's-complement result, which lies in [-113, 127]).
+__device__ __forceinline__ uint2 widen8_i8(uint32_t w, uint32_t step, uint32_t min4) {
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+  const uint32_t e0 = __byte_perm(lo, hi, 0x5140), e1 = __byte_perm(lo, hi, 0x7362);
+  return make_uint2(__vadd4(e0 * step, min4), __vadd4(e1 * step, min4));
+}
 // warps 0..7 dequant + epilogue, 8 TMA, 9 MMA issuer (even CTA) or "A half ready"
 // forwarder (odd CTA), and TMEM allocation.  Ten warps leave room for ~168 registers per
 // thread (the register file is split over the four schedulers).
 constexpr int kPairThreads = (kDeqWarps + 2) * 32;
 
-template <int NTT>
-__global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const __grid_constant__ CUtensorMap xmap,
-                                                                      const __grid_constant__ CUtensorMap cmap,
-                                                                      const __grid_constant__ CUtensorMap mmap,
-                                                                      const __grid_constant__ CUtensorMap smap,
-                                                                      const GemmArgs a) {
+template <bool I8>
+struct PairAcc {
+  using T = float;
+};
+template <>
+struct PairAcc<true> {
+  using T = int;
+};
+
+// The pair kernel's body for both operand widths (I8: the W4A8 form, whose cmap, mmap and smap
+// cover the codes, the int8 group minima and the uint8 group steps).
+template <int NTT, bool I8>
+__device__ __forceinline__ void gemm_pair_body(const CUtensorMap &xmap, const CUtensorMap &cmap,
+                                               const CUtensorMap &mmap, const CUtensorMap &smap, const GemmArgs &a) {
   using C = PairCfg<NTT>;
+  using W = PairW<I8>;
   constexpr int kPairStages = C::kStages, kPairStage = C::kStage, kPairTok = C::kTok, kPairCols = C::kCols;
+  constexpr int kCS = W::kCodeStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // full (even CTA): the stage is ready -- its 8 dequant warps arrive, its TMA thread
@@ -443,7 +495,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
   const int half = static_cast<int>(crank & 1u);
   const int n0 = blockIdx.x * 128;  // this CTA's 128 weight rows
   const int t0 = blockIdx.y * kPairTok, split = blockIdx.z;
-  const int ktiles = a.K / kBK;
+  const int ktiles = a.K / W::kK;
   const int kt0 = static_cast<int>((static_cast<int64_t>(split) * ktiles) / a.splits);
   const int kt1 = static_cast<int>((static_cast<int64_t>(split + 1) * ktiles) / a.splits);
   const int nk = kt1 - kt0;
@@ -461,7 +513,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     }
     mbar_init(smem_u32(&accum_bar), 1);
     mbar_init(smem_u32(&recv_bar), 1);
-    for (int i = 0; i < kPairCodeStages; i++) {
+    for (int i = 0; i < kCS; i++) {
       mbar_init(smem_u32(&code_full[i]), 1);
       mbar_init(smem_u32(&code_empty[i]), kDeqWarps);
     }
@@ -493,73 +545,64 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     // leader: arrive on its own full barrier; odd CTA: on a_half, forwarded by warp 9
     const uint32_t done_bar0 = smem_u32(leader ? &full[0] : &a_half[0]);
     for (int i = 0; i < nk; i++) {
-      const int st = i % kPairStages, cs = i % kPairCodeStages;
-      if (!mbar_wait_bounded(smem_u32(&code_full[cs]), (i / kPairCodeStages) & 1, abortp, a.err)) break;
-      const uint4 c0 = *reinterpret_cast<const uint4 *>(smem + kPairCodeOff + cs * kPairCodeBytes + row * 32 + hk * 16);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&code_empty[cs]));  // the slot may be refilled
+      const int st = i % kPairStages, cs = i % kCS;
+      if (!mbar_wait_bounded(smem_u32(&code_full[cs]), (i / kCS) & 1, abortp, a.err)) break;
+      const uint8_t *cp = smem + kPairCodeOff + cs * W::kCodeBytes + row * W::kCodeRow + hk * (W::kCodeRow / 2);
+      const uint4 c0 = *reinterpret_cast<const uint4 *>(cp);
+      const uint4 c1 = I8 ? *reinterpret_cast<const uint4 *>(cp + 16) : make_uint4(0, 0, 0, 0);
       const int mi = (kt0 + i) >> a.gshift, u = meta_unit(kt0 + i);
       if (u != cur_u) {  // warp-uniform
         if (cur_u >= 0 && lane == 0) mbar_arrive(smem_u32(&meta_empty[cur_u & 1]));  // read by every lane above
         if (!mbar_wait_bounded(smem_u32(&meta_full[u & 1]), (u >> 1) & 1, abortp, a.err)) break;
         cur_u = u;
       }
-      const __half *mb = reinterpret_cast<const __half *>(smem + kPairMetaOff + (u & 1) * 2 * kPairMetaBytes);
-      const __half m0 = mb[row * 8 + (mi & 7)], s0 = mb[kPairMetaBytes / 2 + row * 8 + (mi & 7)];
+      const uint8_t *mbase = smem + kPairMetaOff + (u & 1) * 2 * kPairMetaBytes;
       if (i >= kPairStages &&
           !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kPairStages) - 1) & 1, abortp, a.err))
         break;
-      const __half2 s2 = __half2half2(s0), m2 = __half2half2(m0);
       uint8_t *at = a_tile(st);
-      const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
+      if constexpr (I8) {
+        // this thread's 64 k values are group 2 kt + hk: column (2 kt + hk) mod 16 of the unit
+        const int col = 2 * ((kt0 + i) & 7) + hk;
+        const uint32_t min4 = static_cast<uint32_t>(mbase[row * 16 + col]) * 0x01010101u;
+        const uint32_t step = mbase[kPairMetaBytes + row * 16 + col];
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-      for (int c = 0; c < 4; c++) {
-        const uint4 v = live ? dequant8(words[c], s2, m2) : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4 *>(at + sw128_offset(row, 4 * hk + c)) = v;
+        for (int c = 0; c < 4; c++) {  // chunk 4 hk + c: k values 16c..16c+15 of the thread's 64
+          const uint2 p = widen8_i8(words[2 * c], step, min4), r = widen8_i8(words[2 * c + 1], step, min4);
+          const uint4 v = live ? make_uint4(p.x, p.y, r.x, r.y) : make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4 *>(at + sw128_offset(row, 4 * hk + c)) = v;
+        }
+      } else {
+        const __half *mb = reinterpret_cast<const __half *>(mbase);
+        const __half m0 = mb[row * 8 + (mi & 7)], s0 = mb[kPairMetaBytes / 2 + row * 8 + (mi & 7)];
+        const __half2 s2 = __half2half2(s0), m2 = __half2half2(m0);
+        const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
+#pragma unroll
+        for (int c = 0; c < 4; c++) {
+          const uint4 v = live ? dequant8(words[c], s2, m2) : make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4 *>(at + sw128_offset(row, 4 * hk + c)) = v;
+        }
       }
+      // The code slot is released only now: the codes have been used (so read), and the proxy
+      // fence orders these generic-proxy reads before the tensor copy that refills the slot.
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(done_bar0 + st * 8);
+      if (lane == 0) {
+        mbar_arrive(done_bar0 + st * 8);
+        mbar_arrive(smem_u32(&code_empty[cs]));
+      }
     }
   } else if (warp == kTmaWarp) {
-    // ---------------- TMA producer: this CTA's halves of the two token tiles ----------------
+    // ---------------- TMA producers ----------------
+    // lane 0: this CTA's halves of the token tiles of x, stage by stage;  lane 1: this CTA's
+    // packed weights -- the codes of each k-tile into the code ring, the group metadata a column
+    // group at a time into its two buffers -- as far ahead as the dequant warps release slots.
+    // On separate lanes a code slot the dequant warps still hold never delays an x copy.
     if (lane == 0) {
       prefetch_tmap(&xmap);
-      prefetch_tmap(&cmap);
-      prefetch_tmap(&mmap);
-      prefetch_tmap(&smap);
-      // this CTA's codes and metadata for k-tiles jc < jmax (and the metadata column group
-      // each first needs), into slots the dequant warps have released
-      int jc = 0, um = 0;
-      bool ok = true;
-      auto feed = [&](int jmax) {
-        for (; ok && jc < jmax && jc < nk; jc++) {
-          if (meta_unit(kt0 + jc) == um) {
-            if (um >= 2 && !mbar_wait_bounded(smem_u32(&meta_empty[um & 1]), ((um >> 1) - 1) & 1, abortp, a.err)) {
-              ok = false;
-              break;
-            }
-            const uint32_t mbar = smem_u32(&meta_full[um & 1]);
-            uint8_t *mb = smem + kPairMetaOff + (um & 1) * 2 * kPairMetaBytes;
-            mbar_arrive_expect_tx(mbar, 2 * kPairMetaBytes);
-            tma_load_2d(smem_u32(mb), &mmap, (sj0 + um) * 8, n0, mbar);
-            tma_load_2d(smem_u32(mb + kPairMetaBytes), &smap, (sj0 + um) * 8, n0, mbar);
-            um++;
-          }
-          const int cs = jc % kPairCodeStages;
-          if (jc >= kPairCodeStages &&
-              !mbar_wait_bounded(smem_u32(&code_empty[cs]), ((jc / kPairCodeStages) - 1) & 1, abortp, a.err)) {
-            ok = false;
-            break;
-          }
-          const uint32_t cbar = smem_u32(&code_full[cs]);
-          mbar_arrive_expect_tx(cbar, kPairCodeBytes);
-          tma_load_2d(smem_u32(smem + kPairCodeOff + cs * kPairCodeBytes), &cmap, (kt0 + jc) * 32, n0, cbar);
-        }
-      };
-      feed(kPairCodeStages);  // the weights are fixed for the call: before the dependency wait
-      griddep_wait();         // x comes from the previous kernel
-      for (int i = 0; ok && i < nk; i++) {
+      griddep_wait();  // x comes from the previous kernel
+      for (int i = 0; i < nk; i++) {
         const int st = i % kPairStages;
         if (i >= kPairStages &&
             !mbar_wait_bounded(smem_u32(&empty[st]), ((i / kPairStages) - 1) & 1, abortp, a.err))
@@ -568,8 +611,31 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
         if (leader) mbar_arrive_expect_tx(smem_u32(&full[st]), 2 * NTT * kPairBHalf + 16);  // x of both CTAs + token
 #pragma unroll
         for (int tile = 0; tile < NTT; tile++)
-          tma_load_2d_pair(smem_u32(b_tile(st, tile)), &xmap, (kt0 + i) * kBK, t0 + tile * 256 + half * 128, fb);
-        feed(i + 1 + kPairCodeStages);
+          tma_load_2d_pair(smem_u32(b_tile(st, tile)), &xmap, (kt0 + i) * W::kK, t0 + tile * 256 + half * 128, fb);
+      }
+    } else if (lane == 1) {
+      // the weights are fixed for the call: no dependency wait
+      prefetch_tmap(&cmap);
+      prefetch_tmap(&mmap);
+      prefetch_tmap(&smap);
+      int um = 0;
+      for (int jc = 0; jc < nk; jc++) {
+        if (meta_unit(kt0 + jc) == um) {  // the first k-tile of a metadata column group
+          if (um >= 2 && !mbar_wait_bounded(smem_u32(&meta_empty[um & 1]), ((um >> 1) - 1) & 1, abortp, a.err))
+            break;
+          const uint32_t mbar = smem_u32(&meta_full[um & 1]);
+          uint8_t *mb = smem + kPairMetaOff + (um & 1) * 2 * kPairMetaBytes;
+          mbar_arrive_expect_tx(mbar, 2 * kPairMetaBytes);
+          tma_load_2d(smem_u32(mb), &mmap, (sj0 + um) * W::kMetaCols, n0, mbar);
+          tma_load_2d(smem_u32(mb + kPairMetaBytes), &smap, (sj0 + um) * W::kMetaCols, n0, mbar);
+          um++;
+        }
+        const int cs = jc % kCS;
+        if (jc >= kCS && !mbar_wait_bounded(smem_u32(&code_empty[cs]), ((jc / kCS) - 1) & 1, abortp, a.err))
+          break;
+        const uint32_t cbar = smem_u32(&code_full[cs]);
+        mbar_arrive_expect_tx(cbar, W::kCodeBytes);
+        tma_load_2d(smem_u32(smem + kPairCodeOff + cs * W::kCodeBytes), &cmap, (kt0 + jc) * W::kCodeRow, n0, cbar);
       }
     }
   } else if (!leader) {
@@ -600,11 +666,16 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
         tc_fence_after();
         const uint64_t ad = adesc0 + st * kStageStep, bd = bdesc0 + st * kStageStep;
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; kk++) {
+        for (int kk = 0; kk < 4; kk++) {  // 32-byte k steps: 16 fp16 or 32 int8 values
 #pragma unroll
-          for (int tile = 0; tile < NTT; tile++)
-            umma_f16_pair(tmem + tile * 256, ad + 2 * kk, bd + tile * kTileStep + 2 * kk, kPairIdesc,
-                          (i > 0 || kk > 0) ? 1u : 0u);
+          for (int tile = 0; tile < NTT; tile++) {
+            if constexpr (I8)
+              umma_i8_pair(tmem + tile * 256, ad + 2 * kk, bd + tile * kTileStep + 2 * kk, kPairIdescI8,
+                           (i > 0 || kk > 0) ? 1u : 0u);
+            else
+              umma_f16_pair(tmem + tile * 256, ad + 2 * kk, bd + tile * kTileStep + 2 * kk, kPairIdesc,
+                            (i > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         umma_commit_pair(smem_u32(&empty[st]), pair_mask);
       }
@@ -626,6 +697,16 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     ready = mbar_wait_bounded_cluster(smem_u32(&accum_bar), 0, nullptr, a.err) && !*abortp;
     tc_fence_after();
   }
+  // Accumulator values travel as 32-bit words: fp32 (W4A16) or s32 sums (W4A8), which k-split
+  // partials add exactly; a W4A8 value becomes the fp32 product acc * (ascale[m] * cscale[n]),
+  // one IEEE operation each, only once it is final.
+  using Acc = typename PairAcc<I8>::T;
+  auto acc_of = [](float word) -> Acc {
+    if constexpr (I8) return __float_as_int(word); else return word;
+  };
+  auto fin = [&](Acc v, int m, float csc) -> float {
+    if constexpr (I8) return __fmul_rn(__int2float_rn(v), __fmul_rn(a.ascale[m], csc)); else return v;
+  };
   const int q = warp & 3, etile = (warp >> 2) & 1;
   // finishing thread: 8 features f8 .. f8+7, tokens mj0 + 16 it of a 32-token chunk
   const int f8 = (tid & 15) * 8, mj0 = (tid >> 4) & 15;
@@ -636,6 +717,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
       const int n = n0 + q * 32 + lane;
       const float bias = (a.bias && n < a.N) ? __half2float(a.bias[n]) : 0.f;
       const float qs = n < a.qcols ? a.qscale : 1.f;
+      const float csc = (I8 && n < a.N) ? a.cscale[n] : 0.f;
       for (int c8 = 0; c8 < C::kChunks / 2; c8++) {
         const int ch = etile * (C::kChunks / 2) + c8;
         uint32_t v[32];
@@ -644,7 +726,8 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
         __half *cb = hbuf + ch * (32 * 128) + q * 32 + lane;
 #pragma unroll
         for (int j = 0; j < 32; j++) {
-          float y = (__uint_as_float(v[j]) + bias) * qs;
+          const int m = t0 + ch * 32 + j;
+          float y = (fin(acc_of(__uint_as_float(v[j])), m < a.M ? m : a.M - 1, csc) + bias) * qs;
           if (a.relu) y = fmaxf(y, 0.f);
           cb[j * 128] = __float2half_rn(y);
         }
@@ -669,9 +752,12 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     constexpr int kRound = kPairRing / (kChunkFloats * 4);  // 12 chunks of the 16
     constexpr int kChunks = kPairCols / 32;
     float *buf = reinterpret_cast<float *>(smem);
-    float bias[8];
+    float bias[8], csc8[8];
 #pragma unroll
-    for (int u = 0; u < 8; u++) bias[u] = (a.bias && warp < kDeqWarps && nb < a.N) ? __half2float(a.bias[nb + u]) : 0.f;
+    for (int u = 0; u < 8; u++) {
+      bias[u] = (a.bias && warp < kDeqWarps && nb < a.N) ? __half2float(a.bias[nb + u]) : 0.f;
+      csc8[u] = (I8 && warp < kDeqWarps && nb < a.N) ? a.cscale[nb + u] : 0.f;
+    }
     for (int r0 = 0; r0 < kChunks; r0 += kRound) {
       if (warp < kDeqWarps) {
         // warps q and q + 4 share TMEM lanes 32q..32q+31 and take alternate chunks
@@ -707,7 +793,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
             __half *oh = reinterpret_cast<__half *>(&ov);
 #pragma unroll
             for (int u = 0; u < 8; u++)
-              oh[u] = __float2half_rn(epilogue(acc[u], bias[u], __half2float(rh[u]), nb + u, a));
+              oh[u] = __float2half_rn(epilogue(fin(acc_of(acc[u]), m, csc8[u]), bias[u], __half2float(rh[u]), nb + u, a));
             *reinterpret_cast<uint4 *>(a.y + static_cast<int64_t>(m) * a.N + nb) = ov;
           }
         }
@@ -766,20 +852,23 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
       cluster_sync_all();
     }
     if (warp < kDeqWarps && ready && nb < a.N) {
-      float bias[8];
+      float bias[8], csc8[8];
 #pragma unroll
-      for (int u = 0; u < 8; u++) bias[u] = a.bias ? __half2float(a.bias[nb + u]) : 0.f;
+      for (int u = 0; u < 8; u++) {
+        bias[u] = a.bias ? __half2float(a.bias[nb + u]) : 0.f;
+        csc8[u] = I8 ? a.cscale[nb + u] : 0.f;
+      }
       const float *col = tilep + half * 128 + f8;
       for (int ch = zrank; ch < kChunks; ch += S) {
         uint4 rv[2];
-        float acc[2][8];
+        Acc acc[2][8];
 #pragma unroll
         for (int it = 0; it < 2; it++) {
           const int m = t0 + ch * 32 + mj0 + 16 * it;
           rv[it] = (a.res && m < a.M) ? *reinterpret_cast<const uint4 *>(a.res + static_cast<int64_t>(m) * a.N + nb)
                                       : make_uint4(0, 0, 0, 0);
 #pragma unroll
-          for (int u = 0; u < 8; u++) acc[it][u] = 0.f;
+          for (int u = 0; u < 8; u++) acc[it][u] = 0;
         }
 #pragma unroll
         for (int z = 0; z < 4; z++) {  // z-rank order
@@ -789,8 +878,9 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
             const float *src = col + z * kTileFloats + static_cast<int64_t>(ch * 32 + mj0 + 16 * it) * 256;
             const float4 p0 = __ldcg(reinterpret_cast<const float4 *>(src));
             const float4 p1 = __ldcg(reinterpret_cast<const float4 *>(src + 4));
-            acc[it][0] += p0.x; acc[it][1] += p0.y; acc[it][2] += p0.z; acc[it][3] += p0.w;
-            acc[it][4] += p1.x; acc[it][5] += p1.y; acc[it][6] += p1.z; acc[it][7] += p1.w;
+            acc[it][0] += acc_of(p0.x); acc[it][1] += acc_of(p0.y); acc[it][2] += acc_of(p0.z);
+            acc[it][3] += acc_of(p0.w); acc[it][4] += acc_of(p1.x); acc[it][5] += acc_of(p1.y);
+            acc[it][6] += acc_of(p1.z); acc[it][7] += acc_of(p1.w);
           }
         }
 #pragma unroll
@@ -802,7 +892,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
           __half *oh = reinterpret_cast<__half *>(&ov);
 #pragma unroll
           for (int u = 0; u < 8; u++)
-            oh[u] = __float2half_rn(epilogue(acc[it][u], bias[u], __half2float(rh[u]), nb + u, a));
+            oh[u] = __float2half_rn(epilogue(fin(acc[it][u], m, csc8[u]), bias[u], __half2float(rh[u]), nb + u, a));
           *reinterpret_cast<uint4 *>(a.y + static_cast<int64_t>(m) * a.N + nb) = ov;
         }
       }
@@ -822,9 +912,12 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     const int S = a.splits, zrank = static_cast<int>(crank >> 1);
     float *sendb = reinterpret_cast<float *>(smem);              // [kR] chunks
     float *recvb = sendb + kR * kChunkFloats;                    // [kSlots] chunks
-    float bias[8];
+    float bias[8], csc8[8];
 #pragma unroll
-    for (int u = 0; u < 8; u++) bias[u] = (a.bias && warp < kDeqWarps && nb < a.N) ? __half2float(a.bias[nb + u]) : 0.f;
+    for (int u = 0; u < 8; u++) {
+      bias[u] = (a.bias && warp < kDeqWarps && nb < a.N) ? __half2float(a.bias[nb + u]) : 0.f;
+      csc8[u] = (I8 && warp < kDeqWarps && nb < a.N) ? a.cscale[nb + u] : 0.f;
+    }
     auto first_owned = [&](int owner, int r0) { return r0 + ((owner - r0 % S) + S) % S; };
     int round = 0;
     for (int r0 = 0; r0 < kChunks; r0 += kR, round++) {
@@ -880,23 +973,23 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
               const int m = t0 + ch * 32 + mj0 + 16 * it;
               if (m >= a.M) continue;
               const int eoff = (mj0 + 16 * it) * 128 + f8;
-              float acc[8];
+              Acc acc[8];
 #pragma unroll
-              for (int u = 0; u < 8; u++) acc[u] = 0.f;
+              for (int u = 0; u < 8; u++) acc[u] = 0;
               for (int z = 0; z < S; z++) {  // z-rank order
                 const float *src = z == zrank ? sendb + (ch - r0) * kChunkFloats + eoff
                                               : recvb + (j * (S - 1) + (z < zrank ? z : z - 1)) * kChunkFloats + eoff;
                 const float4 p0 = *reinterpret_cast<const float4 *>(src);
                 const float4 p1 = *reinterpret_cast<const float4 *>(src + 4);
-                acc[0] += p0.x; acc[1] += p0.y; acc[2] += p0.z; acc[3] += p0.w;
-                acc[4] += p1.x; acc[5] += p1.y; acc[6] += p1.z; acc[7] += p1.w;
+                acc[0] += acc_of(p0.x); acc[1] += acc_of(p0.y); acc[2] += acc_of(p0.z); acc[3] += acc_of(p0.w);
+                acc[4] += acc_of(p1.x); acc[5] += acc_of(p1.y); acc[6] += acc_of(p1.z); acc[7] += acc_of(p1.w);
               }
               const __half *rh = reinterpret_cast<const __half *>(&resv[j][it]);
               uint4 ov;
               __half *oh = reinterpret_cast<__half *>(&ov);
 #pragma unroll
               for (int u = 0; u < 8; u++)
-                oh[u] = __float2half_rn(epilogue(acc[u], bias[u], __half2float(rh[u]), nb + u, a));
+                oh[u] = __float2half_rn(epilogue(fin(acc[u], m, csc8[u]), bias[u], __half2float(rh[u]), nb + u, a));
               *reinterpret_cast<uint4 *>(a.y + static_cast<int64_t>(m) * a.N + nb) = ov;
             }
           }
@@ -914,6 +1007,26 @@ __global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const 
     tc_fence_after();
     tmem_dealloc_pair(tmem, kPairCols);
   }
+}
+
+template <int NTT>
+__global__ void __launch_bounds__(kPairThreads, 1) w4a16_gemm_pair_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                      const __grid_constant__ CUtensorMap cmap,
+                                                                      const __grid_constant__ CUtensorMap mmap,
+                                                                      const __grid_constant__ CUtensorMap smap,
+                                                                      const GemmArgs a) {
+  gemm_pair_body<NTT, false>(xmap, cmap, mmap, smap, a);
+}
+
+// W4A8: xmap covers the int8 activations, cmap the codes, mmap the int8 group minima, smap the
+// uint8 group steps; a.ascale and a.cscale the per-token and per-row fp32 scales.
+template <int NTT>
+__global__ void __launch_bounds__(kPairThreads, 1) w4a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                     const __grid_constant__ CUtensorMap cmap,
+                                                                     const __grid_constant__ CUtensorMap mmap,
+                                                                     const __grid_constant__ CUtensorMap smap,
+                                                                     const GemmArgs a) {
+  gemm_pair_body<NTT, true>(xmap, cmap, mmap, smap, a);
 }
 
 // ------------------------------------------------------------------------------------
@@ -1028,14 +1141,14 @@ fg_status launch_nt(const CUtensorMap &map, const GemmArgs &a, const Plan &p, cu
 
 // ---- pair kernel planning ----
 
-template <int NTT>
+template <int NTT, bool I8 = false>
 fg_status pair_attr_once() {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    fg_status rc = fg_cuda_check(
-        cudaFuncSetAttribute(w4a16_gemm_pair_kernel<NTT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem));
+    fg_status rc = fg_cuda_check(cudaFuncSetAttribute(I8 ? w4a8_gemm_pair_kernel<NTT> : w4a16_gemm_pair_kernel<NTT>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem));
     if (rc != FG_OK) return rc;
     attr_set[dev] = true;
   }
@@ -1081,12 +1194,12 @@ int pair_clusters_resident(int splits) {
 // 0.70 us at 512 tokens and 0.63 us at 256 (half the MMA work, the same dequantisation
 // and pipeline hand-offs); each wave pays its pipeline fill (~5 us) and the epilogue, whose
 // partial sums grow with the tile and the number of splits.
-Plan make_pair_plan(int M, int N, int K) {
+Plan make_pair_plan(int M, int N, int K, int kb = kBK) {
   Plan p;
   p.n_tiles = (N + 255) / 256;  // CTA pairs along the features
   p.nt = 512;
   p.splits = 1;
-  const int ktiles = K / kBK;
+  const int ktiles = K / kb;  // k-tiles of 64 (fp16 operands) or 128 (int8: the same bytes per k-tile)
   double best = 1e30;
   for (int ntt = 2; ntt >= 1; ntt--) {
     const int tok = 256 * ntt;
@@ -1129,9 +1242,9 @@ Plan make_pair_plan(int M, int N, int K) {
   return p;
 }
 
-template <int NTT>
+template <int NTT, bool I8 = false>
 fg_status launch_pair_nt(const CUtensorMap (&maps)[4], const GemmArgs &a, const Plan &p, cudaStream_t st, bool pdl) {
-  fg_status rc = pair_attr_once<NTT>();
+  fg_status rc = pair_attr_once<NTT, I8>();
   if (rc != FG_OK) return rc;
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(2 * p.n_tiles, p.t_tiles, p.splits);
@@ -1147,7 +1260,8 @@ fg_status launch_pair_nt(const CUtensorMap (&maps)[4], const GemmArgs &a, const 
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = pdl ? 2 : 1;
-  rc = fg_cuda_check(cudaLaunchKernelEx(&lc, w4a16_gemm_pair_kernel<NTT>, maps[0], maps[1], maps[2], maps[3], a));
+  rc = fg_cuda_check(cudaLaunchKernelEx(&lc, I8 ? w4a8_gemm_pair_kernel<NTT> : w4a16_gemm_pair_kernel<NTT>, maps[0],
+                                        maps[1], maps[2], maps[3], a));
   if (rc != FG_OK) return rc;
   return fg_launch_check();
 }
@@ -1259,6 +1373,8 @@ fg_status fg_linear_launch(const fg_half *x, int M, int K, const fg_qtensor *w, 
       a.epoch = 0xF6A4000000000000ull | (g_split_epoch.fetch_add(1) + 1);
     }
   }
+  a.ascale = nullptr;
+  a.cscale = nullptr;
   a.err = fg_error_word_ptr();
   if (!a.err) return FG_ERR_CUDA;
   a.wait_ns = FG_WAIT_TIMEOUT_NS;
@@ -1328,4 +1444,92 @@ extern "C" fg_status fg_linear_w4a16(const fg_half *x, int M, int K, const fg_qt
   // weights may come from the kernel just before (fg_quantize): no overlap with it
   return fg_linear_launch(x, M, K, w, bias, residual, flags, qscale_cols, qscale, y, workspace, workspace_bytes,
                           static_cast<cudaStream_t>(stream), false);
+}
+
+// ---- W4A8 on CTA pairs (fg_w4a8.cu takes this launch for M > 256) ----
+// The W4A16 pair launch's planner (k-tiles of 128) and k-split modes: with the scratch of
+// fg_w4a8_pair_ws_bytes the ranks' s32 partials go through it (flags when the grid is one wave),
+// else over distributed shared memory; the sums are exact in every mode.  The group metadata
+// arrive by tensor copies of 16 group columns: rows of K / 64 bytes must be whole 16-byte units.
+bool fg_w4a8_pair_eligible(int M, int K, const fg_w4a8_weight *w) {
+  return M > 256 && (K / 64) % 16 == 0 && fg_aligned16(w->gmin) && fg_aligned16(w->gstep);
+}
+
+size_t fg_w4a8_pair_ws_bytes(int M, int N, int K) {
+  if (M <= 256 || N <= 0 || K <= 0 || K % 128) return 0;
+  const Plan p = make_pair_plan(M, N, K, 128);
+  return pair_part_bytes(p) + pair_flag_bytes(p);
+}
+
+void fg_w4a8_pair_plan(int M, int N, int K, int *tile_tokens, int *splits) {
+  const Plan p = make_pair_plan(M, N, K, 128);
+  *tile_tokens = p.nt;
+  *splits = p.splits;
+}
+
+fg_status fg_w4a8_pair_launch(const int8_t *a8, const float *ascale, int M, int K, const fg_w4a8_weight *w,
+                              const fg_half *bias, const fg_half *residual, int flags, int qscale_cols, float qscale,
+                              fg_half *y, void *workspace, size_t ws_bytes, cudaStream_t st) {
+  const int N = static_cast<int>(w->N);
+  const Plan p = make_pair_plan(M, N, K, 128);
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FG_ERR_CUDA;
+  CUtensorMap maps[4];  // activations, codes, group minima, group steps
+  const cuuint32_t estr[2] = {1, 1};
+  const cuuint64_t xdims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  const cuuint64_t xstr[1] = {static_cast<cuuint64_t>(K)};
+  const cuuint32_t xbox[2] = {128, 128};
+  CUresult cr = enc(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(a8), xdims, xstr, xbox, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return FG_ERR_INVALID;
+  const cuuint64_t cdims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
+  const cuuint64_t cstr[1] = {static_cast<cuuint64_t>(K / 2)};
+  const cuuint32_t cbox[2] = {64, 128};
+  cr = enc(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w->codes, cdims, cstr, cbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return FG_ERR_INVALID;
+  const cuuint64_t mdims[2] = {static_cast<cuuint64_t>(K / 64), static_cast<cuuint64_t>(N)};
+  const cuuint64_t mstr[1] = {static_cast<cuuint64_t>(K / 64)};
+  const cuuint32_t mbox[2] = {16, 128};
+  void *meta[2] = {w->gmin, w->gstep};
+  for (int j = 0; j < 2; j++) {
+    cr = enc(&maps[2 + j], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, meta[j], mdims, mstr, mbox, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return FG_ERR_INVALID;
+  }
+  GemmArgs a;
+  a.wc = w->codes;
+  a.wm = nullptr;
+  a.ws = nullptr;
+  a.bias = reinterpret_cast<const __half *>(bias);
+  a.res = (flags & FG_EPI_RESIDUAL) ? reinterpret_cast<const __half *>(residual) : nullptr;
+  a.y = reinterpret_cast<__half *>(y);
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.relu = (flags & FG_EPI_RELU) ? 1 : 0;
+  a.qcols = qscale_cols;
+  a.qscale = qscale;
+  a.splits = p.splits;
+  a.gshift = 0;
+  a.part = nullptr;
+  a.flags = nullptr;
+  a.epoch = 0;
+  if (p.splits > 1 && workspace && fg_aligned16(workspace) && ws_bytes >= pair_part_bytes(p)) {
+    a.part = static_cast<float *>(workspace);
+    const int one = p.nt == 256 ? pair_clusters_resident<1>(1) : pair_clusters_resident<2>(1);
+    if (ws_bytes >= pair_part_bytes(p) + pair_flag_bytes(p) && p.n_tiles * p.t_tiles * p.splits <= one) {
+      a.flags = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + pair_part_bytes(p));
+      a.epoch = 0xF6A4000000000000ull | (g_split_epoch.fetch_add(1) + 1);
+    }
+  }
+  a.ascale = ascale;
+  a.cscale = w->cscale;
+  a.err = fg_error_word_ptr();
+  if (!a.err) return FG_ERR_CUDA;
+  a.wait_ns = FG_WAIT_TIMEOUT_NS;
+  a.stall = 0;
+  return p.nt == 256 ? launch_pair_nt<1, true>(maps, a, p, st, false) : launch_pair_nt<2, true>(maps, a, p, st, false);
 }

@@ -13,7 +13,11 @@
 //   y[t][n] = epi( acc[t][n] * (ascale[t] * cscale[n]) + bias[n] ), acc = sum_k a8 * w8 exact in
 //     int32, the rest one fp32 operation at a time (q-scale, ReLU, residual as in the W4A16 layer).
 //
-// GEMM kernel, one SM per output tile: 256 output features (two 128-row accumulators) x NT tokens
+// Larger blocks (M > 256) run on CTA pairs: the W4A16 pair kernel (fg_gemm.cu) in its int8 form
+// -- the same pipeline with the codes widened to int8, tcgen05.mma.cta_group::2.kind::i8 and the
+// scales applied once a sum is final.
+//
+// GEMM kernel, one SM per output tile (M <= 256): 256 output features (two 128-row accumulators) x NT tokens
 // x a k-range, k-tiles of 128 (two groups; one 128-byte row of int8 per feature and per token).
 //   warps 0..7  thread t owns weight row n0 + t: per k-tile it loads 64 code bytes and both groups'
 //               (gmin, gstep), widens 8 codes at a time to int8 -- two byte permutes, one 32-bit
@@ -26,6 +30,14 @@
 //   shared memory (exact, so the result does not depend on the split).
 // Every mbarrier wait is bounded (FG_WAIT_TIMEOUT_NS) and reports FG_ERR_TIMEOUT.
 #include "fg_internal.cuh"
+
+// the CTA-pair launch for M > 256 (fg_gemm.cu): the W4A16 pair kernel's int8 form
+bool fg_w4a8_pair_eligible(int M, int K, const fg_w4a8_weight *w);
+size_t fg_w4a8_pair_ws_bytes(int M, int N, int K);
+void fg_w4a8_pair_plan(int M, int N, int K, int *tile_tokens, int *splits);
+fg_status fg_w4a8_pair_launch(const int8_t *a8, const float *ascale, int M, int K, const fg_w4a8_weight *w,
+                              const fg_half *bias, const fg_half *residual, int flags, int qscale_cols, float qscale,
+                              fg_half *y, void *workspace, size_t ws_bytes, cudaStream_t st);
 
 namespace {
 
@@ -592,15 +604,25 @@ extern "C" fg_status fg_act8_quantize(const fg_half *x, int M, int K, int8_t *a8
 
 extern "C" fg_status fg_linear_w4a8_plan(int M, int N, int K, int *tile_tokens, int *splits) {
   if (!tile_tokens || !splits || M <= 0 || N <= 0 || N % 128 || K <= 0 || K % kBK) return FG_ERR_INVALID;
+  if (M > 256 && (K / kGrp) % 16 == 0) {
+    fg_w4a8_pair_plan(M, N, K, tile_tokens, splits);
+    return FG_OK;
+  }
   const Plan8 p = make_plan8(M, N, K);
   *tile_tokens = p.nt;
   *splits = p.splits;
   return FG_OK;
 }
 
+extern "C" size_t fg_linear_w4a8_workspace_bytes(int M, int N, int K) {
+  if (M <= 256 || N <= 0 || K <= 0 || K % kBK || (K / kGrp) % 16) return 0;
+  return fg_w4a8_pair_ws_bytes(M, N, K);
+}
+
 extern "C" fg_status fg_linear_w4a8(const int8_t *a8, const float *ascale, int M, int K, const fg_w4a8_weight *w,
                                     const fg_half *bias, const fg_half *residual, int flags, int qscale_cols,
-                                    float qscale, fg_half *y, void *stream) {
+                                    float qscale, fg_half *y, void *workspace, size_t workspace_bytes,
+                                    void *stream) {
   if (!w || M < 0 || K <= 0) return FG_ERR_INVALID;
   if (!w4a8_shape_ok(w) || w->K != K || K % kBK || K > 65536 || w->N % 128) return FG_ERR_SHAPE;
   if (flags & ~(FG_EPI_RELU | FG_EPI_RESIDUAL)) return FG_ERR_INVALID;
@@ -609,7 +631,10 @@ extern "C" fg_status fg_linear_w4a8(const int8_t *a8, const float *ascale, int M
   if (!fg_aligned16(a8) || !fg_aligned16(y) || !fg_aligned16(w->codes) ||
       (reinterpret_cast<uintptr_t>(w->gmin) & 1u) || (reinterpret_cast<uintptr_t>(w->gstep) & 1u))
     return FG_ERR_INVALID;
-  if ((flags & FG_EPI_RESIDUAL) && !residual) return FG_ERR_INVALID;
+  if ((flags & FG_EPI_RESIDUAL) && (!residual || !fg_aligned16(residual))) return FG_ERR_INVALID;
+  if (fg_w4a8_pair_eligible(M, K, w))
+    return fg_w4a8_pair_launch(a8, ascale, M, K, w, bias, residual, flags, qscale_cols, qscale, y, workspace,
+                               workspace_bytes, static_cast<cudaStream_t>(stream));
   const int N = static_cast<int>(w->N);
   const Plan8 p = make_plan8(M, N, K);
   EncodeTiledFn enc = encode_fn8();

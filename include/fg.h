@@ -277,15 +277,22 @@ FG_API fg_status fg_act8_quantize(const fg_half *x, int M, int K, int8_t *a8, fl
 /* The W4A8 product above: a8 [M][K] int8 and ascale [M] from fg_act8_quantize, w from
  * fg_w4a8_quantize_weight with w->K == K, bias fp16 [N] or NULL, residual fp16 [M][N].
  * K % 128 == 0 and K <= 65536 (the int32 sums stay exact), N % 128 == 0 (FG_ERR_SHAPE);
- * a8, y and the codes 16-byte aligned, gmin and gstep 2-byte aligned (FG_ERR_INVALID).
- * One SM per output tile of 256 features x tile_tokens tokens; the k-range may be split over a
- * cluster whose CTAs add their int32 partial sums exactly, so the result does not depend on
- * the plan. */
+ * a8, y, the residual and the codes 16-byte aligned, gmin and gstep 2-byte aligned
+ * (FG_ERR_INVALID).  M <= 256: one SM per output tile of 256 features x tile_tokens tokens, the
+ * k-range possibly split over a cluster whose CTAs add their int32 partials exactly.  M > 256,
+ * (K / 64) % 16 == 0 and gmin, gstep 16-byte aligned: the CTA-pair launch of fg_linear_w4a16 in
+ * its int8 form (256- or 512-token tiles, k-tiles of 128); its k splits add int32 partials
+ * through the optional workspace (fg_linear_w4a8_workspace_bytes; the split ranks then meet
+ * through flags when the grid fits one wave) or over distributed shared memory.  Integer sums are
+ * exact in every launch, so the result does not depend on the plan or the scratch. */
 FG_API fg_status fg_linear_w4a8(const int8_t *a8, const float *ascale, int M, int K, const fg_w4a8_weight *w,
                          const fg_half *bias, const fg_half *residual, int flags, int qscale_cols,
-                         float qscale, fg_half *y, void *stream);
-/* The launch fg_linear_w4a8 makes for this shape on the current device (no launch):
- * *tile_tokens 16..256, *splits 1..8 (FG_ERR_INVALID for shapes it rejects). */
+                         float qscale, fg_half *y, void *workspace, size_t workspace_bytes, void *stream);
+/* Scratch the CTA-pair launch of fg_linear_w4a8 can use for this shape (0: none). */
+FG_API size_t fg_linear_w4a8_workspace_bytes(int M, int N, int K);
+/* The launch fg_linear_w4a8 makes for this shape on the current device, assuming 16-byte aligned
+ * metadata (no launch): *tile_tokens (16..256 one SM per tile, 256 or 512 a CTA pair per tile) and
+ * *splits (1..8, 1..4 for pairs); FG_ERR_INVALID for shapes it rejects. */
 FG_API fg_status fg_linear_w4a8_plan(int M, int N, int K, int *tile_tokens, int *splits);
 
 /* y = (x - mean) / sqrt(var + eps) * gamma + beta per row (fp32 statistics,

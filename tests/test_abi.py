@@ -254,7 +254,7 @@ def test_w4a8_entry_points_validate_on_host():
     w = _fake_w4a8()
     lin = lambda **o: [o.get("a8", P), o.get("ascale", P * 2), o.get("M", 8), o.get("K", 512),
                        ctypes.byref(o.get("w", w)), None, o.get("res", None), o.get("flags", 0), 0, 1.0,
-                       o.get("y", P * 3), None]
+                       o.get("y", P * 3), None, 0, None]
     assert _rc("fg_linear_w4a8", *lin(K=448)) == 2                     # K differs from the weight's
     assert _rc("fg_linear_w4a8", *lin(w=_fake_w4a8(K=448), K=448)) == 2  # K not a multiple of 128
     assert _rc("fg_linear_w4a8", *lin(w=_fake_w4a8(K=65536 + 128), K=65536 + 128)) == 2  # int32 sums

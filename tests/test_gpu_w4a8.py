@@ -147,3 +147,34 @@ def test_linear_w4a8_decode_shapes_sampled(N, K):
     M = 512
     rows = np.unique(np.concatenate([np.arange(0, M, 64), [1, 255, 256, M - 1]]))
     _run_and_check(M, N, K, seed=37, rows=rows)
+
+
+def test_linear_w4a8_pair_split_modes_agree():
+    # the CTA-pair launch's k split (FC2's shape: 4 split ranks) through the scratch with flags,
+    # through the scratch at a cluster barrier, and over distributed shared memory: the int32
+    # partials add exactly, so all three give the same bits
+    M, N, K = 512, 4096, 16384
+    t, splits = fg.fg_linear_w4a8_plan(M, N, K)
+    assert t in (256, 512) and splits > 1
+    w = _weights(38, N, K)
+    x = _acts(38, M, K)
+    r = dev(si.normal_f16(38, 6, (M, N), 1.0))
+    wq = fg.fg_w4a8_quantize_weight(dev(w))
+    a8, s = fg.fg_act8_quantize(dev(x))
+    tiles = -(-N // 256) * -(-M // t)
+    part = tiles * splits * t * 256 * 4
+    full = fg.fg_linear_w4a8_workspace_bytes(M, N, K)
+    assert full == part + tiles * splits * 2 * 8
+    outs = []
+    for nbytes in (full, part, 0):
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device="cuda")[:nbytes]
+        outs.append(fg.fg_linear_w4a8(a8, s, wq, residual=r, workspace=ws))
+    fg.fg_sync_status()
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+    rows = np.array([0, 100, 511])
+    ref_w = oracle.w4a8_quantize_weight(w)
+    ra8, rs = oracle.act8_quantize(x[rows])
+    rr = host(r)[rows]
+    ref, acc = oracle.linear_w4a8(ra8, rs, ref_w, residual=rr, with_acc=True)
+    tol = _bound(acc, rs, ref_w.cscale, None, rr, 0, 1.0, ref)
+    assert np.all(np.abs(host(outs[0])[rows].astype(np.float64) - ref) <= tol)
