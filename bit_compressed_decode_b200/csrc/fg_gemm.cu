@@ -439,12 +439,14 @@ __device__ __forceinline__ void umma_i8_pair(uint32_t d_tmem, uint64_t a_desc, u
 }
 
 // 8 codes of one word (element 2j in the low nibble of byte j) -> the 8 int8 weights
-// gmin + code * step in element order, as two words (code * step <= 240: no carry between
-// bytes; the per-byte add wraps to the two's-complement result, which lies in [-113, 127]).
-__device__ __forceinline__ uint2 widen8_i8(uint32_t w, uint32_t step, uint32_t min4) {
+// gmin + code * step in element order, as two words.  Each byte is formed in offset binary,
+// code * step + (gmin + 128), which lies in [15, 255] (the weight lies in [-113, 127]), so one
+// 32-bit multiply-add makes four bytes with no carry between them; flipping each byte's top bit
+// turns w + 128 into the two's-complement w.  off4 = (gmin + 128) replicated into the 4 bytes.
+__device__ __forceinline__ uint2 widen8_i8(uint32_t w, uint32_t step, uint32_t off4) {
   const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
   const uint32_t e0 = __byte_perm(lo, hi, 0x5140), e1 = __byte_perm(lo, hi, 0x7362);
-  return make_uint2(__vadd4(e0 * step, min4), __vadd4(e1 * step, min4));
+  return make_uint2((e0 * step + off4) ^ 0x80808080u, (e1 * step + off4) ^ 0x80808080u);
 }
 // warps 0..7 dequant + epilogue, 8 TMA, 9 MMA issuer (even CTA) or "A half ready"
 // forwarder (odd CTA), and TMEM allocation.  Ten warps leave room for ~168 registers per
@@ -564,12 +566,12 @@ __device__ __forceinline__ void gemm_pair_body(const CUtensorMap &xmap, const CU
       if constexpr (I8) {
         // this thread's 64 k values are group 2 kt + hk: column (2 kt + hk) mod 16 of the unit
         const int col = 2 * ((kt0 + i) & 7) + hk;
-        const uint32_t min4 = static_cast<uint32_t>(mbase[row * 16 + col]) * 0x01010101u;
+        const uint32_t off4 = ((static_cast<uint32_t>(mbase[row * 16 + col]) ^ 0x80u)) * 0x01010101u;  // gmin + 128
         const uint32_t step = mbase[kPairMetaBytes + row * 16 + col];
         const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
         for (int c = 0; c < 4; c++) {  // chunk 4 hk + c: k values 16c..16c+15 of the thread's 64
-          const uint2 p = widen8_i8(words[2 * c], step, min4), r = widen8_i8(words[2 * c + 1], step, min4);
+          const uint2 p = widen8_i8(words[2 * c], step, off4), r = widen8_i8(words[2 * c + 1], step, off4);
           const uint4 v = live ? make_uint4(p.x, p.y, r.x, r.y) : make_uint4(0, 0, 0, 0);
           *reinterpret_cast<uint4 *>(at + sw128_offset(row, 4 * hk + c)) = v;
         }
@@ -722,12 +724,20 @@ __device__ __forceinline__ void gemm_pair_body(const CUtensorMap &xmap, const CU
         const int ch = etile * (C::kChunks / 2) + c8;
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, v);
+        // W4A8: lane j loads the scale of token j of the chunk; the warp shares them (every lane
+        // of these warps runs this loop)
+        const int ml = t0 + ch * 32 + lane;
+        const float as_l = I8 ? a.ascale[ml < a.M ? ml : a.M - 1] : 0.f;
         tmem_wait_ld();
         __half *cb = hbuf + ch * (32 * 128) + q * 32 + lane;
 #pragma unroll
         for (int j = 0; j < 32; j++) {
-          const int m = t0 + ch * 32 + j;
-          float y = (fin(acc_of(__uint_as_float(v[j])), m < a.M ? m : a.M - 1, csc) + bias) * qs;
+          float y;
+          if constexpr (I8)
+            y = (__fmul_rn(__int2float_rn(static_cast<int>(v[j])), __fmul_rn(__shfl_sync(0xffffffffu, as_l, j), csc)) +
+                 bias) * qs;
+          else
+            y = (__uint_as_float(v[j]) + bias) * qs;
           if (a.relu) y = fmaxf(y, 0.f);
           cb[j * 128] = __float2half_rn(y);
         }

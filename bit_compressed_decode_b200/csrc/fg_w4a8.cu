@@ -107,11 +107,13 @@ struct Args8 {
 };
 
 // 8 codes of one word (element 2j in the low nibble of byte j) -> the 8 int8 weights
-// gmin + code * step in element order, as two words.
-__device__ __forceinline__ uint2 widen8(uint32_t w, uint32_t step, uint32_t min4) {
+// gmin + code * step in element order, as two words: each byte formed in offset binary,
+// code * step + (gmin + 128) in [15, 255] (no carry between bytes), then its top bit flipped.
+// off4 = (gmin + 128) replicated into the 4 bytes.
+__device__ __forceinline__ uint2 widen8(uint32_t w, uint32_t step, uint32_t off4) {
   const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
   const uint32_t e0 = __byte_perm(lo, hi, 0x5140), e1 = __byte_perm(lo, hi, 0x7362);
-  return make_uint2(__vadd4(e0 * step, min4), __vadd4(e1 * step, min4));
+  return make_uint2((e0 * step + off4) ^ 0x80808080u, (e1 * step + off4) ^ 0x80808080u);
 }
 
 // acc -> fp32 scale, bias, q-scale, ReLU, residual: one IEEE fp32 operation each
@@ -212,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a8_gemm_kernel(const __grid_con
           break;
         }
         // group 2kt in the low byte of m2/s2, group 2kt+1 in the high byte
-        const uint32_t min_lo = (m2 & 0xFFu) * 0x01010101u, min_hi = (m2 >> 8) * 0x01010101u;
+        const uint32_t min_lo = ((m2 & 0xFFu) ^ 0x80u) * 0x01010101u, min_hi = ((m2 >> 8) ^ 0x80u) * 0x01010101u;  // gmin + 128
         const uint32_t step_lo = s2 & 0xFFu, step_hi = s2 >> 8;
         uint8_t *at = a_tile(st, acc);
         const uint32_t words[16] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w,
@@ -438,6 +440,42 @@ __global__ void __launch_bounds__(kActThreads) act8_quant_kernel(const __half *x
   }
 }
 
+// The same with the row held in registers (V 16-byte vectors per thread): one read of x.
+template <int V>
+__global__ void __launch_bounds__(kActThreads) act8_quant_reg_kernel(const __half *x, int K, int8_t *a8,
+                                                                     float *ascale) {
+  __shared__ float red[kActThreads / 32];
+  const int64_t t = blockIdx.x;
+  const uint4 *xr = reinterpret_cast<const uint4 *>(x + t * K);
+  const int nv = K / 8;
+  uint4 v[V];
+  float m = 0.f;
+#pragma unroll
+  for (int u = 0; u < V; u++) {
+    const int i = threadIdx.x + u * kActThreads;
+    v[u] = i < nv ? xr[i] : make_uint4(0, 0, 0, 0);
+    m = absmax8(v[u], m);
+  }
+  const float amax = cta_max<kActThreads>(m, red);
+  const float inv = amax > 0.f ? __fdiv_rn(static_cast<float>(kA8Bound), amax) : 0.f;
+  if (threadIdx.x == 0) ascale[t] = amax > 0.f ? __fdiv_rn(amax, static_cast<float>(kA8Bound)) : 0.f;
+  uint2 *out = reinterpret_cast<uint2 *>(a8 + t * K);
+#pragma unroll
+  for (int u = 0; u < V; u++) {
+    const int i = threadIdx.x + u * kActThreads;
+    if (i >= nv) break;
+    const __half2 *h = reinterpret_cast<const __half2 *>(&v[u]);
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      const float2 f = __half22float2(h[j]);
+      const uint32_t b0 = static_cast<uint8_t>(q8(f.x, inv, kA8Bound)), b1 = static_cast<uint8_t>(q8(f.y, inv, kA8Bound));
+      w[j >> 1] |= (b0 | (b1 << 8)) << ((j & 1) * 16);
+    }
+    out[i] = make_uint2(w[0], w[1]);
+  }
+}
+
 // Weights: one CTA per row of K values (K % 64 == 0).  Level 1 as for the activations with bound
 // 113; level 2 per group of 64: mn, mx of the int8 values, step = max(1, ceil((mx - mn) / 15)),
 // code = floor((2 (w8 - mn) + step) / (2 step)).
@@ -597,8 +635,21 @@ extern "C" fg_status fg_act8_quantize(const fg_half *x, int M, int K, int8_t *a8
   if (M == 0) return FG_OK;
   if (!x || !a8 || !ascale || !fg_aligned16(x) || !fg_aligned16(a8) || (reinterpret_cast<uintptr_t>(ascale) & 3u))
     return FG_ERR_INVALID;
-  act8_quant_kernel<<<M, kActThreads, 0, static_cast<cudaStream_t>(stream)>>>(reinterpret_cast<const __half *>(x), K,
-                                                                             a8, ascale);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const __half *xh = reinterpret_cast<const __half *>(x);
+  const int per = (K / 8 + kActThreads - 1) / kActThreads;  // 16-byte vectors per thread
+  if (per <= 1)
+    act8_quant_reg_kernel<1><<<M, kActThreads, 0, st>>>(xh, K, a8, ascale);
+  else if (per <= 2)
+    act8_quant_reg_kernel<2><<<M, kActThreads, 0, st>>>(xh, K, a8, ascale);
+  else if (per <= 4)
+    act8_quant_reg_kernel<4><<<M, kActThreads, 0, st>>>(xh, K, a8, ascale);
+  else if (per <= 8)
+    act8_quant_reg_kernel<8><<<M, kActThreads, 0, st>>>(xh, K, a8, ascale);
+  else if (per <= 16)
+    act8_quant_reg_kernel<16><<<M, kActThreads, 0, st>>>(xh, K, a8, ascale);
+  else  // rows above 32768 values: two passes (the second from cache)
+    act8_quant_kernel<<<M, kActThreads, 0, st>>>(xh, K, a8, ascale);
   return fg_launch_check();
 }
 

@@ -71,7 +71,7 @@ def test_w4a8_weight_quantiser_bit_exact(N, K):
     _check_weight(wq, oracle.w4a8_quantize_weight(w))
 
 
-@pytest.mark.parametrize("M,K", [(1, 64), (5, 4096), (300, 1024), (3, 49152)])
+@pytest.mark.parametrize("M,K", [(1, 64), (5, 4096), (300, 1024), (2, 7168), (2, 16384), (2, 28672), (3, 49152)])
 def test_act8_quantiser_bit_exact(M, K):
     x = _acts(32, M, K)
     a8, s = fg.fg_act8_quantize(dev(x))
