@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_act8_quantize.argtypes = [P, I, I, P, P]
         _lib.oracle_linear_w4a8.restype = I
         _lib.oracle_linear_w4a8.argtypes = [P, P, I, I, P, P, P, P, I, P, P, I, I, D, P, P]
+        _lib.oracle_layer_rows_w4a8.restype = I
+        _lib.oracle_layer_rows_w4a8.argtypes = ([P, D, P] + [P] * 8 + [P] * 6 + [I, I] + [P, I, P, P, I, P, P, I])
         _lib.oracle_layer_rows.restype = I
         _lib.oracle_layer_rows.argtypes = ([P, D] + [P] * 16 + [P] * 4 + [P] * 6 + [I, I] + [P, I, P, P, I, P, P, I])
     return _lib
@@ -359,6 +361,51 @@ def layer_rows(weights: LayerWeights, heads: int, cache: KVCache, x, seq_of_row,
     args += cache.ptrs() + [cache.S, cache.maxL]
     args += [_p(x), R, _p(sr), _p(pr), int(kv_only), _p(out), _p(attn), int(nthreads)]
     rc = lib().oracle_layer_rows(*args)
+    assert rc == 0, rc
+    return out, attn
+
+
+class W4A8LayerWeights:
+    """One OPT layer's weights in the W4A8 form (w4a8_quantize_weight of each matrix); the KV
+    cache stays 4-bit in groups of 64."""
+
+    def __init__(self, w16: dict):
+        self.group = GROUP
+        self.wqkv = w4a8_quantize_weight(w16["wqkv"])
+        self.wo = w4a8_quantize_weight(w16["wo"])
+        self.w1 = w4a8_quantize_weight(w16["w1"])
+        self.w2 = w4a8_quantize_weight(w16["w2"])
+        self.b = {k: _u16(w16[k]) for k in ("bqkv", "bo", "b1", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b")}
+        self.hidden = self.wqkv.K
+        self.ffn = self.w1.N
+
+
+def layer_rows_w4a8(weights: W4A8LayerWeights, heads: int, cache: KVCache, x, seq_of_row, pos_of_row,
+                    kv_only: bool = False, eps: float = 1e-5, nthreads: int = 1, want_attn: bool = False):
+    """``layer_rows`` with the four products in the W4A8 form (the reading in fg_oracle.c): each
+    product's fp16 input row is quantised to int8 with one scale and multiplied as integers."""
+    x = _u16(x)
+    R, h = x.shape
+    d = h // heads
+    if cache.group != GROUP:
+        raise ValueError("the W4A8 layer's KV cache uses groups of 64")
+    dims = np.array([h, heads, d, weights.ffn], dtype=np.int32)
+    out = np.zeros((R, h), dtype=np.float64)
+    attn = np.zeros((R, h), dtype=np.float64) if want_attn else None
+    sr = np.ascontiguousarray(seq_of_row, dtype=np.int32)
+    pr = np.ascontiguousarray(pos_of_row, dtype=np.int32)
+    w = weights
+    keep = []
+    for t in (w.wqkv, w.wo, w.w1, w.w2):
+        keep += [np.ascontiguousarray(t.codes), np.ascontiguousarray(t.gmin), np.ascontiguousarray(t.gstep),
+                 np.ascontiguousarray(t.cscale, dtype=np.float32)]
+    mats = (ctypes.c_void_p * 16)(*[a.ctypes.data for a in keep])
+    args = [_p(dims), float(eps), ctypes.cast(mats, ctypes.c_void_p)]
+    args += [_p(w.b["bqkv"]), _p(w.b["bo"]), _p(w.b["b1"]), _p(w.b["b2"])]
+    args += [_p(w.b["ln1_g"]), _p(w.b["ln1_b"]), _p(w.b["ln2_g"]), _p(w.b["ln2_b"])]
+    args += cache.ptrs() + [cache.S, cache.maxL]
+    args += [_p(x), R, _p(sr), _p(pr), int(kv_only), _p(out), _p(attn), int(nthreads)]
+    rc = lib().oracle_layer_rows_w4a8(*args)
     assert rc == 0, rc
     return out, attn
 

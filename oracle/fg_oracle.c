@@ -511,10 +511,20 @@ int oracle_attention(const uint16_t *q16, int64_t ld, int R, const int *seq_of_r
 /* One OPT decoder layer, row by row [OPT][G3][G2]                            */
 /* ------------------------------------------------------------------------- */
 
+/* W4A8 pieces defined with the W4A8 section at the end of this file */
+#define OR_W8_BOUND 113
+#define OR_A8_BOUND 127
+static void quantize_row_sym8(const uint16_t *x, int64_t n, int bound, int *q, float *scale);
+int oracle_w4a8_weight_int8(const uint8_t *codes, const int8_t *gmin, const uint8_t *gstep, int N, int K,
+                            int8_t *w8);
+
 typedef struct {
     int h, H, d, F;
     double eps;
-    float *Wqkv, *Wo, *W1, *W2;           /* dequantised, [out][in] */
+    float *Wqkv, *Wo, *W1, *W2;           /* dequantised, [out][in] (W4A16) */
+    int w4a8;                             /* 1: the W4A8 products of the W4A8 section */
+    int8_t *Q[4];                         /* W4A8: the products' int8 weights, [out][in] */
+    const float *cs[4];                   /* W4A8: their row scales */
     double *bqkv, *bo, *b1, *b2, *g1, *be1, *g2, *be2;
     kv_t kv;
     const uint16_t *x;                    /* [R][h] */
@@ -524,6 +534,31 @@ typedef struct {
 } layer_ctx;
 
 typedef struct { layer_ctx *c; int tid; } layer_job;
+
+/* y = x W^T + b for one row of one of the layer's matrices (0 wqkv, 1 wo, 2 w1, 3 w2): float64
+   from the dequantised fp16 weights, or (W4A8) the row's fp16 values quantised to int8 with one
+   fp32 scale, exact integer sums with the int8 weights, then acc * (ascale * cscale[n]) + b[n]
+   in float64.  x16 and q hold K values of scratch. */
+static void layer_linear(const layer_ctx *c, int which, const double *x, int N, int K, const double *b,
+                         double *y, uint16_t *x16, int *q)
+{
+    if (!c->w4a8) {
+        const float *W[4] = {c->Wqkv, c->Wo, c->W1, c->W2};
+        linear_row(W[which], b, x, N, K, y);
+        return;
+    }
+    for (int k = 0; k < K; k++) x16[k] = oracle_f64_to_f16(x[k]);   /* exact: x holds fp16 values */
+    float as;
+    quantize_row_sym8(x16, K, OR_A8_BOUND, q, &as);
+    const int8_t *W = c->Q[which];
+    const float *cs = c->cs[which];
+    for (int n = 0; n < N; n++) {
+        const int8_t *wr = W + (int64_t)n * K;
+        int64_t acc = 0;
+        for (int k = 0; k < K; k++) acc += (int64_t)q[k] * (int64_t)wr[k];
+        y[n] = (double)acc * ((double)as * (double)cs[n]) + (b ? b[n] : 0.0);
+    }
+}
 
 /* The rows of one sequence are processed in the order given, so a prompt
    (positions 0..P-1) appends each token before the next one attends. */
@@ -539,6 +574,9 @@ static void *layer_worker(void *arg)
     double *tmp = malloc(sizeof(double) * h), *kb = malloc(sizeof(double) * d);
     double *sc = malloc(sizeof(double) * c->kv.maxL);
     uint16_t *k16 = malloc(sizeof(uint16_t) * d), *v16 = malloc(sizeof(uint16_t) * d);
+    int KX = F > h ? F : h;
+    uint16_t *x16 = malloc(sizeof(uint16_t) * KX);
+    int *q8 = malloc(sizeof(int) * KX);
     double qscale = 1.0 / sqrt((double)d);
     for (int r = 0; r < c->R; r++) {
         int s = c->seq_of_row[r], pos = c->pos_of_row[r];
@@ -548,7 +586,7 @@ static void *layer_worker(void *arg)
         layernorm_row(x, h, c->g1, c->be1, c->eps, a);
         round16_vec(a, h);
         /* 2. [q k v] = a Wqkv^T + b;  q = fp16(q * d^-1/2), k = fp16(k), v = fp16(v) */
-        linear_row(c->Wqkv, c->bqkv, a, 3 * h, h, qkv);
+        layer_linear(c, 0, a, 3 * h, h, c->bqkv, qkv, x16, q8);
         for (int i = 0; i < h; i++) qkv[i] *= qscale;
         round16_vec(qkv, 3 * h);
         /* 3. append k, v to the 4-bit cache at pos */
@@ -566,20 +604,36 @@ static void *layer_worker(void *arg)
         round16_vec(o, h);
         if (c->attn) memcpy(c->attn + (int64_t)r * h, o, sizeof(double) * h);
         /* 6. h1 = fp16(x + o Wo^T + bo) */
-        linear_row(c->Wo, c->bo, o, h, h, tmp);
+        layer_linear(c, 1, o, h, h, c->bo, tmp, x16, q8);
         for (int i = 0; i < h; i++) h1[i] = round16(x[i] + tmp[i]);
         /* 7. y = h1 + fp16(relu(fp16(LN2(h1)) W1^T + b1)) W2^T + b2 */
         layernorm_row(h1, h, c->g2, c->be2, c->eps, a2);
         round16_vec(a2, h);
-        linear_row(c->W1, c->b1, a2, F, h, f);
+        layer_linear(c, 2, a2, F, h, c->b1, f, x16, q8);
         for (int i = 0; i < F; i++) f[i] = f[i] < 0.0 ? 0.0 : round16(f[i]);
-        linear_row(c->W2, c->b2, f, h, F, tmp);
+        layer_linear(c, 3, f, h, F, c->b2, tmp, x16, q8);
         for (int i = 0; i < h; i++) y[i] = h1[i] + tmp[i];
         memcpy(c->out + (int64_t)r * h, y, sizeof(double) * h);
     }
     free(x); free(a); free(qkv); free(o); free(h1); free(a2); free(f); free(y); free(tmp); free(kb); free(sc);
-    free(k16); free(v16);
+    free(k16); free(v16); free(x16); free(q8);
     return NULL;
+}
+
+/* The rows of the layer over nthreads threads (rows of one sequence stay on one thread). */
+static void run_layer_threads(layer_ctx *c, int nthreads)
+{
+    if (nthreads < 1) nthreads = 1;
+    c->nthreads = nthreads;
+    pthread_t *th = malloc(sizeof(pthread_t) * nthreads);
+    layer_job *jobs = malloc(sizeof(layer_job) * nthreads);
+    for (int t = 0; t < nthreads; t++) {
+        jobs[t].c = c; jobs[t].tid = t;
+        if (t > 0) pthread_create(&th[t], NULL, layer_worker, &jobs[t]);
+    }
+    layer_worker(&jobs[0]);
+    for (int t = 1; t < nthreads; t++) pthread_join(th[t], NULL);
+    free(th); free(jobs);
 }
 
 /*
@@ -620,17 +674,7 @@ int oracle_layer_rows(const int *dims, double eps,
     c.kv = kv;
     c.x = x; c.seq_of_row = seq_of_row; c.pos_of_row = pos_of_row; c.R = R;
     c.kv_only = kv_only; c.out = out; c.attn = attn;
-    if (nthreads < 1) nthreads = 1;
-    c.nthreads = nthreads;
-    pthread_t *th = malloc(sizeof(pthread_t) * nthreads);
-    layer_job *jobs = malloc(sizeof(layer_job) * nthreads);
-    for (int t = 0; t < nthreads; t++) {
-        jobs[t].c = &c; jobs[t].tid = t;
-        if (t > 0) pthread_create(&th[t], NULL, layer_worker, &jobs[t]);
-    }
-    layer_worker(&jobs[0]);
-    for (int t = 1; t < nthreads; t++) pthread_join(th[t], NULL);
-    free(th); free(jobs);
+    run_layer_threads(&c, nthreads);
     free(c.Wqkv); free(c.Wo); free(c.W1); free(c.W2);
     free(c.bqkv); free(c.bo); free(c.b1); free(c.b2); free(c.g1); free(c.be1); free(c.g2); free(c.be2);
     return 0;
@@ -663,9 +707,6 @@ int oracle_layer_rows(const int *dims, double eps,
  *   y = acc * (ascale[t] * cscale[n]) + bias[n], then the q-scale of the first qscale_cols
  *   outputs, ReLU and the fp16 residual as in oracle_linear, in float64.
  */
-#define OR_W8_BOUND 113
-#define OR_A8_BOUND 127
-
 /* round-half-even of x * inv (fp32 multiply), clamped to [-bound, bound] */
 static int q8_of(float x, float inv, int bound)
 {
@@ -781,5 +822,50 @@ int oracle_linear_w4a8(const int8_t *a8, const float *ascale, int M, int K,
             y[t * N + n] = v;
         }
     free(W);
+    return 0;
+}
+
+/*
+ * The OPT layer with W4A8 products ([Q8] reading above): the layer of oracle_layer_rows with each
+ * of its four products replaced by the W4A8 product of its fp16 input row (LayerNorm outputs, the
+ * attention output, the ReLU output), everything else unchanged (the KV cache in groups of 64).
+ * mats[4 * i + j], i = wqkv, wo, w1, w2: j = 0 codes [N][K/2], 1 gmin [N][K/64] (int8), 2 gstep
+ * [N][K/64] (uint8), 3 cscale [N] (float).  dims = {hidden, heads, head_dim, ffn}.
+ */
+int oracle_layer_rows_w4a8(const int *dims, double eps, const void *const *mats,
+                           const uint16_t *bqkv, const uint16_t *bo, const uint16_t *b1, const uint16_t *b2,
+                           const uint16_t *ln1_g, const uint16_t *ln1_b, const uint16_t *ln2_g, const uint16_t *ln2_b,
+                           uint8_t *kc, uint16_t *km, uint16_t *ks, uint8_t *vc, uint16_t *vm, uint16_t *vs,
+                           int S, int maxL,
+                           const uint16_t *x, int R, const int *seq_of_row, const int *pos_of_row,
+                           int kv_only, double *out, double *attn, int nthreads)
+{
+    layer_ctx c;
+    memset(&c, 0, sizeof(c));
+    c.h = dims[0]; c.H = dims[1]; c.d = dims[2]; c.F = dims[3]; c.eps = eps;
+    if (c.h != c.H * c.d || c.h % OR_GROUP || c.F % OR_GROUP || c.d % OR_GROUP) return -1;
+    for (int r = 0; r < R; r++)
+        if (seq_of_row[r] < 0 || seq_of_row[r] >= S || pos_of_row[r] < 0 || pos_of_row[r] >= maxL) return -2;
+    const int NK[4][2] = {{3 * c.h, c.h}, {c.h, c.h}, {c.F, c.h}, {c.h, c.F}};
+    c.w4a8 = 1;
+    for (int i = 0; i < 4; i++) {
+        c.Q[i] = (int8_t *)malloc((size_t)NK[i][0] * NK[i][1]);
+        if (!c.Q[i]) return -3;
+        if (oracle_w4a8_weight_int8((const uint8_t *)mats[4 * i], (const int8_t *)mats[4 * i + 1],
+                                    (const uint8_t *)mats[4 * i + 2], NK[i][0], NK[i][1], c.Q[i]))
+            return -4;
+        c.cs[i] = (const float *)mats[4 * i + 3];
+    }
+    c.bqkv = f16_vec(bqkv, 3 * c.h, 0.0); c.bo = f16_vec(bo, c.h, 0.0);
+    c.b1 = f16_vec(b1, c.F, 0.0); c.b2 = f16_vec(b2, c.h, 0.0);
+    c.g1 = f16_vec(ln1_g, c.h, 1.0); c.be1 = f16_vec(ln1_b, c.h, 0.0);
+    c.g2 = f16_vec(ln2_g, c.h, 1.0); c.be2 = f16_vec(ln2_b, c.h, 0.0);
+    kv_t kv = {kc, km, ks, vc, vm, vs, S, c.H, c.d, maxL, OR_GROUP, 0};
+    c.kv = kv;
+    c.x = x; c.seq_of_row = seq_of_row; c.pos_of_row = pos_of_row; c.R = R;
+    c.kv_only = kv_only; c.out = out; c.attn = attn;
+    run_layer_threads(&c, nthreads);
+    for (int i = 0; i < 4; i++) free(c.Q[i]);
+    free(c.bqkv); free(c.bo); free(c.b1); free(c.b2); free(c.g1); free(c.be1); free(c.g2); free(c.be2);
     return 0;
 }

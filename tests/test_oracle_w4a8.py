@@ -4,8 +4,9 @@ The pages name W4A8 only through the QServe W4A8KV4 title in the PIPO paper's re
 INT8/INT4 formats of the "Optimizing LLM for low memory usage" page (Quantization and Weight
 Compression); the scheme itself is a reading, stated in ``oracle/fg_oracle.c``.  Nothing here
 compares the oracle with itself: the expected values are hand-derived fixtures (tests/golden),
-exhaustive integer invariants of the scheme, closed forms, and numpy's integer matrix product as an
-independent check of the oracle's accumulation loop.
+exhaustive integer invariants of the scheme, closed forms, numpy's integer matrix product as an
+independent check of the oracle's accumulation loop, and -- for the W4A8 layer -- the OPT layer's
+wiring written out in Python from those pinned pieces.
 """
 import json
 import os
@@ -208,3 +209,70 @@ def test_linear_w4a8_close_to_the_real_product():
         w.astype(np.float64) - wq).T
     assert np.all(np.abs(y - ref) <= bound * (1 + 1e-9) + 1e-12)
     assert np.max(np.abs(y - ref)) / np.max(np.abs(ref)) < 0.2
+
+
+# ------------------------------------------------------------------ the W4A8 layer ------
+
+def _f16(a):
+    return oracle.f64_to_f16(np.asarray(a, dtype=np.float64))
+
+
+def _compose_layer(w16, wq, heads, cache, x_rows, seq, pos):
+    """The W4A8 layer written out from its pinned pieces (LayerNorm, the activation quantiser,
+    the W4A8 product, the KV append and attention), row by row in order: the wiring of an OPT
+    pre-LN decoder layer ([OPT]) with every activation handed on in fp16."""
+    h = x_rows.shape[1]
+    d = h // heads
+    outs = []
+    for r in range(x_rows.shape[0]):
+        x = x_rows[r:r + 1]
+        a = _f16(oracle.layernorm(x, w16["ln1_g"], w16["ln1_b"]))
+        a8, s = oracle.act8_quantize(a)
+        qkv = oracle.linear_w4a8(a8, s, wq.wqkv, bias=w16["bqkv"], qscale_cols=h, qscale=1.0 / np.sqrt(d))
+        qkv16 = _f16(qkv)
+        oracle.kv_append(cache, qkv16[:, h:2 * h], qkv16[:, 2 * h:], [seq[r]], [pos[r]])
+        o = _f16(oracle.attention(cache, qkv16[:, :h], [seq[r]], [pos[r] + 1]))
+        o8, so = oracle.act8_quantize(o)
+        h1 = _f16(oracle.linear_w4a8(o8, so, wq.wo, bias=w16["bo"], residual=x))
+        a2 = _f16(oracle.layernorm(h1, w16["ln2_g"], w16["ln2_b"]))
+        a28, s2 = oracle.act8_quantize(a2)
+        f = _f16(oracle.linear_w4a8(a28, s2, wq.w1, bias=w16["b1"], relu=True))
+        f8, sf = oracle.act8_quantize(f)
+        y = oracle.linear_w4a8(f8, sf, wq.w2, bias=w16["b2"], residual=h1)
+        outs.append(y[0])
+    return np.stack(outs)
+
+
+def test_w4a8_layer_equals_its_pinned_pieces():
+    import seeded_inputs as si
+    h, H, F = 128, 2, 256
+    w16 = si.layer_weights_f16(41, h, F, std=0.05, bias_std=0.05, ln_random=True)
+    wq = oracle.W4A8LayerWeights(w16)
+    S, maxL = 2, 64
+    c_layer = oracle.KVCache(S, H, h // H, maxL)
+    c_pieces = oracle.KVCache(S, H, h // H, maxL)
+    seq = np.array([0, 1, 0, 0, 1])
+    pos = np.array([0, 0, 1, 2, 1])
+    x = si.normal_f16(41, 9, (len(seq), h), 1.0)
+    got, _ = oracle.layer_rows_w4a8(wq, H, c_layer, x, seq, pos)
+    ref = _compose_layer(w16, wq, H, c_pieces, x, seq, pos)
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+    for a, b in zip(c_layer.arrays(), c_pieces.arrays()):
+        assert np.array_equal(a, b)
+
+
+def test_w4a8_layer_close_to_the_w4a16_layer():
+    # a sanity bound, not a pin: both forms quantise the same weights with independent errors of
+    # similar size (the W4A8 one with 8-bit activations and integer group steps), so their layer
+    # updates differ by about the quantisation noise -- a dropped term or a wrong sign would not
+    import seeded_inputs as si
+    h, H, F = 256, 4, 1024
+    w16 = si.layer_weights_f16(42, h, F, std=0.02)
+    S, maxL = 3, 64
+    seq = np.array([0, 1, 2])
+    pos = np.array([0, 0, 0])
+    x = si.normal_f16(42, 9, (S, h), 1.0)
+    a, _ = oracle.layer_rows_w4a8(oracle.W4A8LayerWeights(w16), H, oracle.KVCache(S, H, h // H, maxL), x, seq, pos)
+    b, _ = oracle.layer_rows(oracle.LayerWeights(w16), H, oracle.KVCache(S, H, h // H, maxL), x, seq, pos)
+    dx = x.astype(np.float64)
+    assert np.max(np.abs((a - dx) - (b - dx))) <= 0.5 * np.max(np.abs(b - dx))
