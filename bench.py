@@ -34,6 +34,9 @@ sys.path.insert(0, ROOT)
 WORKLOADS = {
     "opt-6.7b-layer": dict(hidden=4096, heads=32, ffn=16384, nb=8, gbs=64, prompt=512, steps=32),
     "opt-125m-layer": dict(hidden=768, heads=12, ffn=3072, nb=1, gbs=4, prompt=32, steps=8),
+    # the same OPT-6.7B-shaped block with the layer's products in the W4A8 form (int8 activations,
+    # one scale per row; two-level 4-bit weights; the KV cache unchanged)
+    "opt-6.7b-layer-w4a8": dict(hidden=4096, heads=32, ffn=16384, nb=8, gbs=64, prompt=512, steps=32, act_bits=8),
     # prompt processing of the OPT-6.7B-shaped block: one prefill of 512 tokens for each of the
     # 512 sequences through one layer (the cache filled from position 0)
     "opt-6.7b-prefill": dict(hidden=4096, heads=32, ffn=16384, nb=8, gbs=64, prompt=512, steps=32, phase="prefill"),
@@ -63,23 +66,28 @@ def load_peaks():
 
 def kernel_work(wl, S, L_avg, group=64, fused_append=True):
     """Algorithmic work per launch of each kernel of one step (bytes or flops).  Decode rows
-    append their k, v inside the attention kernel (fused_append); prompt rows append apart."""
+    append their k, v inside the attention kernel (fused_append); prompt rows append apart.
+    W4A8 layers: the products are int8 ("tensor_i8") and each takes its input from an activation
+    quantiser (fp16 in, int8 and a row scale out)."""
     h, F, H = wl["hidden"], wl["ffn"], wl["heads"]
+    gemm = "tensor_i8" if wl.get("act_bits") == 8 else "tensor"
+    act8 = lambda k: ("hbm", S * k * 3 + S * 4)
     d = h // H
     kv_tok = 2 * (d // 2 + 4 * (d // group))         # K and V codes + fp16 min/scale per (seq, head, token)
     w4 = lambda n, k: n * k // 2 + n * (k // group) * 4  # packed weight bytes
     return {
         "ln1": ("hbm", 2 * S * h * 2 + 4 * h),
-        "qkv_gemm": ("tensor", 2 * S * 3 * h * h),
+        "qkv_gemm": (gemm, 2 * S * 3 * h * h),
         "kv_append": ("hbm", S * 2 * h * 2 + S * H * kv_tok),  # fp16 k, v in; codes and metadata out
         # decode attention appends the step's k, v itself: fp16 q, k, v in, o out, the new
         # codes and metadata written, the cache read up to and including them
         "attention": ("hbm", S * H * L_avg * kv_tok + 2 * S * h * 2
                       + ((2 * S * h * 2 + S * H * kv_tok) if fused_append else 0)),
-        "out_gemm": ("tensor", 2 * S * h * h),
+        "out_gemm": (gemm, 2 * S * h * h),
         "ln2": ("hbm", 2 * S * h * 2 + 4 * h),
-        "fc1_gemm": ("tensor", 2 * S * F * h),
-        "fc2_gemm": ("tensor", 2 * S * h * F),
+        "fc1_gemm": (gemm, 2 * S * F * h),
+        "fc2_gemm": (gemm, 2 * S * h * F),
+        "qkv_act8": act8(h), "out_act8": act8(h), "fc1_act8": act8(h), "fc2_act8": act8(F),
     }, {"w4_bytes": w4(3 * h, h) + w4(h, h) + w4(F, h) + w4(h, F), "kv_bytes_per_token": kv_tok}
 
 
@@ -87,7 +95,7 @@ def kernel_units(wl, S, L_avg):
     """Units one launch of each kernel processes, the scale for traffic taken on a smaller case."""
     h, F, H = wl["hidden"], wl["ffn"], wl["heads"]
     return {"ln1": S, "qkv_gemm": S, "kv_append": S, "attention": S * H * L_avg, "out_gemm": S, "ln2": S,
-            "fc1_gemm": S, "fc2_gemm": S}
+            "fc1_gemm": S, "fc2_gemm": S, "qkv_act8": S, "out_act8": S, "fc1_act8": S, "fc2_act8": S}
 
 
 class ClockSampler:
@@ -161,7 +169,9 @@ class OracleSample:
         h, H, F, P = wl["hidden"], wl["heads"], wl["ffn"], wl["prompt"]
         self.H, self.P, self.n, self.threads = H, P, n_seqs, threads
         maxL = (P + wl["steps"] + 63) // 64 * 64
-        self.W = oracle.LayerWeights(si.layer_weights_f16(seed, h, F))
+        self.w4a8 = wl.get("act_bits") == 8
+        w16 = si.layer_weights_f16(seed, h, F)
+        self.W = oracle.W4A8LayerWeights(w16) if self.w4a8 else oracle.LayerWeights(w16)
         self.cache = oracle.KVCache(n_seqs, H, h // H, maxL)
         for s in range(n_seqs):
             k = si.normal_f16(seed, si.STREAM["k_new"], (P, h), 1.0, start=s * P * h)
@@ -171,8 +181,8 @@ class OracleSample:
 
     def step(self) -> float:
         t0 = time.perf_counter()
-        self.oracle.layer_rows(self.W, self.H, self.cache, self.x, np.arange(self.n), np.full(self.n, self.P),
-                               nthreads=self.threads)
+        run = self.oracle.layer_rows_w4a8 if self.w4a8 else self.oracle.layer_rows
+        run(self.W, self.H, self.cache, self.x, np.arange(self.n), np.full(self.n, self.P), nthreads=self.threads)
         return time.perf_counter() - t0
 
 
@@ -353,7 +363,8 @@ def run_ours(args, wl):
     nsteps_cfg = wl["steps"]
     maxL = (P + nsteps_cfg + 63) // 64 * 64
     G = args.group
-    cfg = fg.LayerConfig(h, H, F, group=G)
+    act_bits = wl.get("act_bits", 16)
+    cfg = fg.LayerConfig(h, H, F, group=G, act_bits=act_bits)
 
     # weights: the shared seeded host generator (same on every rank: replicas)
     w16 = si.layer_weights_f16(0, h, F)
@@ -448,6 +459,9 @@ def run_ours(args, wl):
         if bound == "tensor":
             # the timed region is ~10 ms at full clock: the burst GEMM peak applies
             ach, peak, unit = units / avg_s / 1e12, peaks["tc_burst"], "TFLOP/s"
+        elif bound == "tensor_i8":
+            # int8 products: the measured fp16 peak x 2, the nominal int8 / fp16 dense ratio
+            ach, peak, unit = units / avg_s / 1e12, peaks["tc_burst"] * 2, "TOP/s"
         else:
             ach, peak, unit = units / avg_s / 1e9, peaks["hbm"], "GB/s"
         kernels[name] = {"bound": bound, "avg_us": round(avg_s * 1e6, 2), "launches": cnt,
@@ -455,6 +469,8 @@ def run_ours(args, wl):
                          "achieved": round(ach, 1), "peak": peak, "unit": unit, "frac": round(ach / peak, 4)}
         if bound == "tensor":
             kernels[name]["frac_of_sustained"] = round(ach / peaks["tc_sustained"], 4)
+        elif bound == "tensor_i8":
+            kernels[name]["frac_of_sustained"] = round(ach / (2 * peaks["tc_sustained"]), 4)
     dom = max(kernels, key=lambda k: kernels[k]["share"])
     kd = kernels[dom]
     roofline = {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"],
@@ -480,10 +496,13 @@ def run_ours(args, wl):
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "i8 products, f16 elsewhere" if act_bits == 8 else "f16",
+            "data": "synthetic",
             "config": {"workload": args.workload, "block": f"{nb}x{gbs}", "sequences_per_gpu": S, "hidden": h,
                        "heads": H, "ffn": F, "prompt": P, "positions": f"{P}..{P + nsteps_cfg - 1} (cycled)",
-                       "weights": f"W4 g{G}", "kv": f"KV4 g{G}", "parallelism": f"replicas x{world}",
+                       "weights": f"W4 g{G}" + (" (W4A8 form)" if act_bits == 8 else ""),
+                       "activations": "int8, one scale per row" if act_bits == 8 else "fp16",
+                       "kv": f"KV4 g{G}", "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (KV4 cache %.2f GB + W4 %.0f MB per step)" % (
                            cache.nbytes() / 1e9, totals["w4_bytes"] / 1e6)},
             "roofline": roofline,

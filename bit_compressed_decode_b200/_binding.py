@@ -50,12 +50,13 @@ class fg_kv_cache(Structure):
 
 class fg_layer_config(Structure):
     _fields_ = [("hidden", c_int32), ("num_heads", c_int32), ("head_dim", c_int32), ("ffn", c_int32),
-                ("ln_eps", c_float), ("group", c_int32)]
+                ("ln_eps", c_float), ("group", c_int32), ("act_bits", c_int32)]
 
 
 class fg_layer_weights(Structure):
     _fields_ = [("wqkv", fg_qtensor), ("wo", fg_qtensor), ("w1", fg_qtensor), ("w2", fg_qtensor)] + [
-        (n, c_void_p) for n in ("bqkv", "bo", "b1", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b")]
+        (n, c_void_p) for n in ("bqkv", "bo", "b1", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b")] + [
+        ("cscale", c_void_p * 4)]
 
 
 class fg_w4a8_weight(Structure):
@@ -429,13 +430,17 @@ def fg_layernorm(x: torch.Tensor, gamma=None, beta=None, eps: float = 1e-5, out=
 # ---------------------------------------------------------------------------------------
 
 class LayerConfig:
-    def __init__(self, hidden: int, num_heads: int, ffn: int, ln_eps: float = 1e-5, group: int = 64):
-        """``group``: the 4-bit group of the layer's weights and KV cache (64 or 128)."""
+    def __init__(self, hidden: int, num_heads: int, ffn: int, ln_eps: float = 1e-5, group: int = 64,
+                 act_bits: int = 16):
+        """``group``: the 4-bit group of the layer's weights and KV cache (64 or 128);
+        ``act_bits``: 16 (W4A16) or 8 (W4A8 products, weights in the W4A8 form, group 64)."""
         self.hidden, self.num_heads, self.ffn, self.ln_eps, self.group = hidden, num_heads, ffn, ln_eps, group
+        self.act_bits = act_bits
         self.head_dim = hidden // num_heads
 
     def struct(self) -> fg_layer_config:
-        return fg_layer_config(self.hidden, self.num_heads, self.head_dim, self.ffn, self.ln_eps, self.group)
+        return fg_layer_config(self.hidden, self.num_heads, self.head_dim, self.ffn, self.ln_eps, self.group,
+                               self.act_bits)
 
     def blob_bytes(self) -> int:
         c = self.struct()
@@ -486,6 +491,23 @@ class LayerWeights:
         scales = sub(q.scales, n * k // G * 2).view(torch.float16).view(n, k // G)
         return QTensor(codes, mins, scales, (n, k), 1, G)
 
+    def w4a8_matrix(self, name: str) -> "W4A8Weight":
+        """W4A8Weight view of one matrix inside the blob of a W4A8 layer."""
+        i = _MATS.index(name)
+        q = getattr(self._w, name)
+        base = self.blob.data_ptr()
+        n, k = q.shape[0], q.shape[1]
+        def sub(ptr, nbytes):
+            off = ptr - base
+            return self.blob[off:off + nbytes]
+        m = W4A8Weight.__new__(W4A8Weight)
+        m.N, m.K = n, k
+        m.codes = sub(q.codes, n * k // 2).view(n, k // 2)
+        m.gmin = sub(q.mins, n * k // 64).view(torch.int8).view(n, k // 64)
+        m.gstep = sub(q.scales, n * k // 64).view(n, k // 64)
+        m.cscale = sub(self._w.cscale[i], n * 4).view(torch.float32)
+        return m
+
     def vector(self, name: str) -> torch.Tensor:
         ptr = getattr(self._w, name)
         off = ptr - self.blob.data_ptr()
@@ -499,7 +521,10 @@ class LayerWeights:
         lw = LayerWeights(cfg, blob)
         for name in _MATS:
             x = torch.as_tensor(w16[name]).to(device=device, dtype=torch.float16).contiguous()
-            fg_quantize(x, dim=1, group=cfg.group, stream=stream, out=lw.matrix(name))
+            if cfg.act_bits == 8:
+                fg_w4a8_quantize_weight(x, out=lw.w4a8_matrix(name), stream=stream)
+            else:
+                fg_quantize(x, dim=1, group=cfg.group, stream=stream, out=lw.matrix(name))
         for name in _VECS:
             lw.vector(name).copy_(torch.as_tensor(w16[name]).to(device=device, dtype=torch.float16))
         return lw
@@ -565,7 +590,8 @@ def fg_layer_prefill(cfg: LayerConfig, w: LayerWeights, cache: KVCache, x: torch
     return out
 
 
-PROFILE_SLOTS = ("ln1", "qkv_gemm", "kv_append", "attention", "out_gemm", "ln2", "fc1_gemm", "fc2_gemm")
+PROFILE_SLOTS = ("ln1", "qkv_gemm", "kv_append", "attention", "out_gemm", "ln2", "fc1_gemm", "fc2_gemm",
+                 "qkv_act8", "out_act8", "fc1_act8", "fc2_act8")
 
 
 def fg_profile_enable(enable: bool = True) -> None:

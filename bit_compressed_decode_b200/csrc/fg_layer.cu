@@ -23,6 +23,9 @@ fg_status fg_kv_append_launch(const fg_kv_cache *kv, const fg_half *k, const fg_
 fg_status fg_attention_launch(const fg_kv_cache *kv, const fg_half *q, int64_t ldq, fg_half *out, int64_t ldo,
                               int rows, int rows_per_seq, const int32_t *positions, cudaStream_t st,
                               const fg_half *k_new, const fg_half *v_new, int64_t ld_new);
+size_t fg_w4a8_pair_ws_bytes(int M, int N, int K);
+fg_status fg_layernorm_q8_launch(const fg_half *x, int M, int h, const fg_half *gamma, const fg_half *beta,
+                                 float eps, fg_half *y, int8_t *a8, float *ascale, cudaStream_t st);
 
 int fg_profile_begin(int slot, cudaStream_t st);
 void fg_profile_end(int idx, cudaStream_t st);
@@ -31,8 +34,13 @@ namespace {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+bool w4a8(const fg_layer_config *c) { return c->act_bits == 8; }
+
 bool config_ok(const fg_layer_config *c) {
   if (!c) return false;
+  if (c->act_bits != 0 && c->act_bits != 16 && c->act_bits != 8) return false;
+  if (c->act_bits == 8 && (fg_kv_group(c->group) != 64 || c->hidden % 128 || c->ffn % 128 || c->ffn > 65536))
+    return false;
   if (c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256) return false;
   const int G = fg_kv_group(c->group);
   if (G == 0 || c->head_dim % G) return false;
@@ -47,7 +55,7 @@ struct Matrix {
 
 // Offsets of every array inside the layer blob (256-byte aligned).
 struct BlobLayout {
-  size_t off[4][3];  // [matrix][codes, mins, scales]
+  size_t off[4][4];  // [matrix][codes, mins, scales, row scales]: W4A8: codes, gmin, gstep, cscale
   size_t vec[8];     // bqkv, bo, b1, b2, ln1_g, ln1_b, ln2_g, ln2_b
   size_t total;
   Matrix mat[4];
@@ -62,14 +70,17 @@ BlobLayout blob_layout(const fg_layer_config *c) {
   L.mat[2] = {F, h};
   L.mat[3] = {h, F};
   size_t p = 0;
+  const size_t mbytes = w4a8(c) ? 1 : 2;  // per group: int8 minimum and uint8 step, or fp16 min and scale
   for (int i = 0; i < 4; i++) {
     const size_t numel = static_cast<size_t>(L.mat[i].n * L.mat[i].k);
     L.off[i][0] = p;
     p = align256(p + numel / 2);
     L.off[i][1] = p;
-    p = align256(p + numel / G * 2);
+    p = align256(p + numel / G * mbytes);
     L.off[i][2] = p;
-    p = align256(p + numel / G * 2);
+    p = align256(p + numel / G * mbytes);
+    L.off[i][3] = p;
+    if (w4a8(c)) p = align256(p + static_cast<size_t>(L.mat[i].n) * 4);
   }
   const int64_t vlen[8] = {3 * h, h, F, h, h, h, h, h};
   for (int i = 0; i < 8; i++) {
@@ -81,8 +92,12 @@ BlobLayout blob_layout(const fg_layer_config *c) {
 }
 
 struct WsLayout {
-  size_t a, qkv, o, h1, f, gemm, total;
+  size_t a, qkv, o, h1, f, a8, as, gemm, total;
 };
+
+size_t gemm_ws(const fg_layer_config *c, int rows, int N, int K) {
+  return w4a8(c) ? fg_w4a8_pair_ws_bytes(rows, N, K) : fg_linear_ws_bytes(rows, N, K);
+}
 
 WsLayout ws_layout(const fg_layer_config *c, int rows) {
   WsLayout w;
@@ -98,11 +113,19 @@ WsLayout ws_layout(const fg_layer_config *c, int rows) {
   p = align256(p + R * h * 2);
   w.f = p;
   p = align256(p + R * F * 2);
+  w.a8 = w.as = p;  // W4A8: a product's int8 input [rows][<= F] and its row scales
+  if (w4a8(c)) {
+    p = align256(p + R * (F > h ? F : h));
+    w.as = p;
+    p = align256(p + R * 4);
+  }
   w.gemm = p;
-  size_t g = fg_linear_ws_bytes(rows, 3 * c->hidden, c->hidden);
-  g = g > fg_linear_ws_bytes(rows, c->hidden, c->hidden) ? g : fg_linear_ws_bytes(rows, c->hidden, c->hidden);
-  g = g > fg_linear_ws_bytes(rows, c->ffn, c->hidden) ? g : fg_linear_ws_bytes(rows, c->ffn, c->hidden);
-  g = g > fg_linear_ws_bytes(rows, c->hidden, c->ffn) ? g : fg_linear_ws_bytes(rows, c->hidden, c->ffn);
+  const int N[4] = {3 * c->hidden, c->hidden, c->ffn, c->hidden}, K[4] = {c->hidden, c->hidden, c->hidden, c->ffn};
+  size_t g = 0;
+  for (int i = 0; i < 4; i++) {
+    const size_t gi = gemm_ws(c, rows, N[i], K[i]);
+    g = gi > g ? gi : g;
+  }
   p = align256(p + g);
   w.total = p;
   return w;
@@ -117,6 +140,9 @@ bool weights_ok(const fg_layer_config *c, const fg_layer_weights *w) {
     if (m[i]->ndim != 2 || m[i]->dim != 1 || m[i]->bits != 4 || m[i]->group != G) return false;
     if (m[i]->shape[0] != shp[i][0] || m[i]->shape[1] != shp[i][1]) return false;
     if (!m[i]->codes || !m[i]->mins || !m[i]->scales || !fg_aligned16(m[i]->codes)) return false;
+    if (w4a8(c) && (!w->cscale[i] || (reinterpret_cast<uintptr_t>(w->cscale[i]) & 3u) ||
+                    (reinterpret_cast<uintptr_t>(m[i]->mins) & 1u) || (reinterpret_cast<uintptr_t>(m[i]->scales) & 1u)))
+      return false;
   }
   return true;
 }
@@ -157,6 +183,43 @@ fg_status run_layer(const fg_layer_config *c, const fg_layer_weights *w, const f
   // kernel before it.  Not for prompts, whose attention can outlast the GEMM's bounded
   // pipeline waits.
   const bool pdl = rows_per_seq == 1;
+  // W4A8: each product's fp16 input is quantised to int8 per row into a8 / as first
+  const bool i8 = w4a8(c);
+  int8_t *a8 = reinterpret_cast<int8_t *>(ws + L.a8);
+  float *as = reinterpret_cast<float *>(ws + L.as);
+  const fg_qtensor *mq[4] = {&w->wqkv, &w->wo, &w->w1, &w->w2};
+  fg_w4a8_weight w8[4];
+  for (int i = 0; i < 4; i++) {
+    w8[i].codes = const_cast<uint8_t *>(mq[i]->codes);
+    w8[i].gmin = reinterpret_cast<int8_t *>(mq[i]->mins);
+    w8[i].gstep = reinterpret_cast<uint8_t *>(mq[i]->scales);
+    w8[i].cscale = w->cscale[i];
+    w8[i].N = mq[i]->shape[0];
+    w8[i].K = mq[i]->shape[1];
+  }
+  // the product y = epi(x W_i^T + b): W4A16 on fp16 x, or W4A8 on x quantised to int8 (profile slot qslot)
+  // (qslot < 0: a8 / as already hold x's int8 form, made by the LayerNorm before it)
+  auto product = [&](int i, const fg_half *x, int K, const fg_half *b, const fg_half *res, int flags, int qcols,
+                     float qs, fg_half *y, int slot, int qslot) -> fg_status {
+    fg_status r;
+    if (!i8) {
+      const int e = fg_profile_begin(slot, st);
+      r = fg_linear_launch(x, rows, K, mq[i], b, res, flags, qcols, qs, y, gws, gbytes, st, pdl);
+      fg_profile_end(e, st);
+      return r;
+    }
+    int e;
+    if (qslot >= 0) {
+      e = fg_profile_begin(qslot, st);
+      r = fg_act8_quantize(x, rows, K, a8, as, st);
+      fg_profile_end(e, st);
+      if (r != FG_OK) return r;
+    }
+    e = fg_profile_begin(slot, st);
+    r = fg_linear_w4a8(a8, as, rows, K, &w8[i], b, res, flags, qcols, qs, y, gws, gbytes, st);
+    fg_profile_end(e, st);
+    return r;
+  };
   fg_status rc;
   int ev;
 #define FG_STEP(slot, call)                    \
@@ -167,10 +230,12 @@ fg_status run_layer(const fg_layer_config *c, const fg_layer_weights *w, const f
   if ((rc = (call)) != FG_OK) return rc;
   // a = LN1(x)
   FG_SLICE(slice_wait(sl, 0, st));
-  FG_STEP(0, fg_layernorm_launch(x_in, rows, h, w->ln1_g, w->ln1_b, c->ln_eps, a, st));
+  // (W4A8: with its int8 form)
+  FG_STEP(0, i8 ? fg_layernorm_q8_launch(x_in, rows, h, w->ln1_g, w->ln1_b, c->ln_eps, a, a8, as, st)
+                : fg_layernorm_launch(x_in, rows, h, w->ln1_g, w->ln1_b, c->ln_eps, a, st));
   // [q k v] = a Wqkv^T + bqkv; q *= d^-1/2
   FG_SLICE(slice_wait(sl, 1, st));
-  FG_STEP(1, fg_linear_launch(a, rows, h, &w->wqkv, w->bqkv, nullptr, 0, h, qscale, qkv, gws, gbytes, st, pdl));
+  FG_SLICE(product(0, a, h, w->bqkv, nullptr, 0, h, qscale, qkv, 1, -1));
   FG_SLICE(slice_done(sl, 1, st));
   // append k, v (4-bit) at the sequences' positions, then o = softmax(q K^T) V over the
   // 4-bit cache.  When the decode attention is about one wave of (row, head) CTAs or less its
@@ -189,17 +254,18 @@ fg_status run_layer(const fg_layer_config *c, const fg_layer_weights *w, const f
   FG_SLICE(slice_done(sl, 2, st));
   // h1 = x + o Wo^T + bo
   FG_SLICE(slice_wait(sl, 3, st));
-  FG_STEP(4, fg_linear_launch(o, rows, h, &w->wo, w->bo, x_in, FG_EPI_RESIDUAL, 0, 1.f, h1, gws, gbytes, st, pdl));
+  FG_SLICE(product(1, o, h, w->bo, x_in, FG_EPI_RESIDUAL, 0, 1.f, h1, 4, 9));
   FG_SLICE(slice_done(sl, 3, st));
   // a = LN2(h1)
-  FG_STEP(5, fg_layernorm_launch(h1, rows, h, w->ln2_g, w->ln2_b, c->ln_eps, a, st));
+  FG_STEP(5, i8 ? fg_layernorm_q8_launch(h1, rows, h, w->ln2_g, w->ln2_b, c->ln_eps, a, a8, as, st)
+                : fg_layernorm_launch(h1, rows, h, w->ln2_g, w->ln2_b, c->ln_eps, a, st));
   // f = relu(a W1^T + b1)
   FG_SLICE(slice_wait(sl, 4, st));
-  FG_STEP(6, fg_linear_launch(a, rows, h, &w->w1, w->b1, nullptr, FG_EPI_RELU, 0, 1.f, f, gws, gbytes, st, pdl));
+  FG_SLICE(product(2, a, h, w->b1, nullptr, FG_EPI_RELU, 0, 1.f, f, 6, -1));
   FG_SLICE(slice_done(sl, 4, st));
   // x_out = h1 + f W2^T + b2
   FG_SLICE(slice_wait(sl, 5, st));
-  FG_STEP(7, fg_linear_launch(f, rows, F, &w->w2, w->b2, h1, FG_EPI_RESIDUAL, 0, 1.f, x_out, gws, gbytes, st, pdl));
+  FG_SLICE(product(3, f, F, w->b2, h1, FG_EPI_RESIDUAL, 0, 1.f, x_out, 7, 11));
   FG_SLICE(slice_done(sl, 5, st));
   FG_SLICE(slice_done(sl, 0, st));
 #undef FG_STEP
@@ -253,6 +319,7 @@ extern "C" fg_status fg_layer_weights_from_blob(const fg_layer_config *c, void *
     m[i]->codes = b + L.off[i][0];
     m[i]->mins = reinterpret_cast<fg_half *>(b + L.off[i][1]);
     m[i]->scales = reinterpret_cast<fg_half *>(b + L.off[i][2]);
+    out->cscale[i] = w4a8(c) ? reinterpret_cast<float *>(b + L.off[i][3]) : nullptr;
     m[i]->ndim = 2;
     m[i]->shape[0] = L.mat[i].n;
     m[i]->shape[1] = L.mat[i].k;

@@ -312,17 +312,24 @@ typedef struct {
     int32_t ffn;        /* F, multiple of 128 */
     float ln_eps;       /* 1e-5 for OPT */
     int32_t group;      /* 4-bit group of the weights and the KV cache: 64 or 128 (0 = 64) [G3] */
+    int32_t act_bits;   /* what the products multiply the weights with: 16 (or 0): fp16 activations,
+                         * W4 weights of the format above (W4A16); 8: int8 activations, one scale
+                         * per row, and weights in the W4A8 form of fg_w4a8_quantize_weight
+                         * (W4A8 [Q8]; group 64, the KV cache unchanged) */
 } fg_layer_config;
 
 /* Compressed weights of one layer.  Matrices are packed along their input
  * dim (dim 1) in groups of the config's group: wqkv [3h][h] (rows: q, then k,
  * then v, each head-major), wo [h][h], w1 [F][h], w2 [h][F].  Vectors fp16:
  * bqkv [3h], bo [h], b1 [F], b2 [h], ln1_g/ln1_b/ln2_g/ln2_b [h].  All device
- * pointers. */
+ * pointers.  W4A8 layers (act_bits 8): a matrix's `mins` holds its int8 group
+ * minima and `scales` its uint8 group steps (fg_w4a8_weight's gmin and gstep),
+ * and cscale[i] its fp32 row scales (i: wqkv, wo, w1, w2; NULL for W4A16). */
 typedef struct {
     fg_qtensor wqkv, wo, w1, w2;
     fg_half *bqkv, *bo, *b1, *b2;
     fg_half *ln1_g, *ln1_b, *ln2_g, *ln2_b;
+    float *cscale[4];
 } fg_layer_weights;
 
 /* Size of one layer's contiguous weight blob (every array at a 256-byte
@@ -335,7 +342,13 @@ FG_API fg_status fg_layer_weights_from_blob(const fg_layer_config *c, void *blob
 
 /* Device scratch for fg_layer_decode / fg_layer_prefill over `rows`
  * hidden-state rows (the block's sequences, or sequences * prompt length):
- * the intermediate activations, then the GEMMs' scratch (fg_linear_w4a16).
+ * the intermediate activations, then the GEMMs' scratch (fg_linear_w4a16 /
+ * fg_linear_w4a8).  The activations, each at the next 256-byte aligned
+ * offset from the start, fp16 row-major: a [rows][h] (LN1, then LN2 output),
+ * qkv [rows][3h], o [rows][h] (attention output), h1 [rows][h], f [rows][F]
+ * (ReLU output); W4A8 layers then a8 [rows][max(h, F)] int8 and as [rows]
+ * fp32 (the last product's quantised input and row scales).  After a call
+ * they hold that call's values (of the last chunk of a prefill).
  * A call needs at least the activations' part and gives the GEMMs whatever
  * follows it; the GEMMs add split k-ranges on chip when it is short, with the
  * same bits. */
@@ -353,7 +366,9 @@ FG_API size_t fg_layer_workspace_bytes(const fg_layer_config *c, int rows);
  * append k, v to the 4-bit cache at positions; o = attention over positions
  * 0..pos; h1 = x + o Wo^T + bo; x_out = h1 + relu(LN2(h1) W1^T + b1) W2^T + b2.
  * kv->num_seqs must equal S and kv->group the config's group.  Positions are
- * not advanced by the call. */
+ * not advanced by the call.  W4A8 layers (act_bits 8): each product's input
+ * (a, o, LN2(h1), the ReLU output) is quantised to int8 per row first
+ * (fg_act8_quantize) and multiplied with fg_linear_w4a8. */
 FG_API fg_status fg_layer_decode(const fg_layer_config *c, const fg_layer_weights *w, const fg_kv_cache *kv,
                           const fg_half *x_in, fg_half *x_out, const int32_t *positions,
                           int num_gpu_batches, int gpu_batch_size,
@@ -403,8 +418,10 @@ FG_API fg_status fg_layer_decode_noalloc(const fg_layer_config *c, const fg_laye
  * the call's stream (no synchronisation added).  fg_profile_collect waits for
  * those events and writes, per kernel slot, the summed milliseconds and the
  * number of launches, then forgets them.  Slots: 0 LN1, 1 QKV GEMM, 2 KV
- * append, 3 attention, 4 out-proj GEMM, 5 LN2, 6 FC1 GEMM, 7 FC2 GEMM. */
-#define FG_PROFILE_SLOTS 8
+ * append, 3 attention, 4 out-proj GEMM, 5 LN2, 6 FC1 GEMM, 7 FC2 GEMM; W4A8
+ * layers also 8..11, the activation quantisers before QKV, out-proj, FC1 and
+ * FC2. */
+#define FG_PROFILE_SLOTS 12
 FG_API fg_status fg_profile_enable(int enable);
 FG_API fg_status fg_profile_collect(float *ms, int *count, int nslots);
 

@@ -276,3 +276,22 @@ def test_w4a8_entry_points_validate_on_host():
     assert _rc("fg_w4a8_quantize_weight", None, ctypes.byref(w), None) == 1
     t, s = ctypes.c_int(), ctypes.c_int()
     assert B.lib().fg_linear_w4a8_plan(8, 256, 448, ctypes.byref(t), ctypes.byref(s)) == 1
+
+
+def test_w4a8_layer_config_rules():
+    # the W4A8 form of the layer: group 64 only, act_bits 16 (or 0) or 8
+    h, H, F = 768, 12, 3072
+    w16 = fg.LayerConfig(h, H, F).blob_bytes()
+    w8 = fg.LayerConfig(h, H, F, act_bits=8).blob_bytes()
+    # per matrix: codes N*K/2, int8 minima and uint8 steps N*K/64 each, fp32 row scales 4N (each
+    # array 256-byte aligned) in place of fp16 mins and scales N*K/64 * 2 each
+    a = lambda x: (x + 255) // 256 * 256
+    mats = [(3 * h, h), (h, h), (F, h), (h, F)]
+    vecs = sum(a(n * 2) for n in (3 * h, h, F, h, h, h, h, h))
+    assert w16 == sum(a(n * k // 2) + 2 * a(n * k // 64 * 2) for n, k in mats) + vecs
+    assert w8 == sum(a(n * k // 2) + 2 * a(n * k // 64) + a(4 * n) for n, k in mats) + vecs
+    with pytest.raises(fg.FgError):
+        fg.LayerConfig(1024, 8, 4096, group=128, act_bits=8).blob_bytes()
+    with pytest.raises(fg.FgError):
+        fg.LayerConfig(h, H, F, act_bits=4).blob_bytes()
+    assert fg.LayerConfig(h, H, F, act_bits=8).workspace_bytes(16) > fg.LayerConfig(h, H, F).workspace_bytes(16)
