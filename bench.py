@@ -40,6 +40,8 @@ WORKLOADS = {
     # prompt processing of the OPT-6.7B-shaped block: one prefill of 512 tokens for each of the
     # 512 sequences through one layer (the cache filled from position 0)
     "opt-6.7b-prefill": dict(hidden=4096, heads=32, ffn=16384, nb=8, gbs=64, prompt=512, steps=32, phase="prefill"),
+    "opt-6.7b-prefill-w4a8": dict(hidden=4096, heads=32, ffn=16384, nb=8, gbs=64, prompt=512, steps=32,
+                                  phase="prefill", act_bits=8),
     # OPT-30B-shaped stack: 48 layers whose W4 blobs stay in pinned host memory and are
     # prefetched layer by layer on a side stream; KV4 caches resident in HBM
     "opt-30b-stack": dict(hidden=7168, heads=56, ffn=28672, nb=4, gbs=64, prompt=512, steps=32, layers=48),
@@ -540,7 +542,8 @@ def run_prefill(args, wl):
     nb, gbs = wl["nb"], wl["gbs"]
     S, d = nb * gbs, h // H
     maxL = (P + wl["steps"] + 63) // 64 * 64
-    cfg = fg.LayerConfig(h, H, F)
+    act_bits = wl.get("act_bits", 16)
+    cfg = fg.LayerConfig(h, H, F, act_bits=act_bits)
     w16 = si.layer_weights_f16(0, h, F)
     lw = fg.LayerWeights.from_fp16(cfg, w16, device=dev)
     del w16
@@ -599,6 +602,8 @@ def run_prefill(args, wl):
         per_step_s = tot_ms / 1e3 / args.steps
         if bound == "tensor":
             ach, unit, peak = w / per_step_s / 1e12, "TFLOP/s", peaks["tc_burst"]
+        elif bound == "tensor_i8":
+            ach, unit, peak = w / per_step_s / 1e12, "TOP/s", peaks["tc_burst"] * 2
         else:
             ach, unit, peak = w / per_step_s / 1e9, "GB/s", peaks["hbm"]
         kernels[name] = {"bound": bound, "ms_per_step": round(tot_ms / args.steps, 3), "launches": n,
@@ -612,9 +617,12 @@ def run_prefill(args, wl):
             "metric": "prefill prompt tokens/s per OPT layer block (W4 KV4)",
             "value": world * rows * args.steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "i8 products, f16 elsewhere" if act_bits == 8 else "f16",
+            "data": "synthetic",
             "config": {"workload": args.workload, "block": f"{nb}x{gbs}", "prompt": P, "hidden": h, "heads": H,
-                       "ffn": F, "weights": "W4 g64", "kv": "KV4 g64 written from position 0",
+                       "ffn": F, "weights": "W4 g64" + (" (W4A8 form)" if act_bits == 8 else ""),
+                       "activations": "int8, one scale per row" if act_bits == 8 else "fp16",
+                       "kv": "KV4 g64 written from position 0",
                        "l2": "inputs larger than L2 (prompt activations 2.1 GB per step)"},
             "roofline": {"kernel": top, "bound": kernels[top]["bound"], "achieved": kernels[top]["achieved"],
                          "peak": kernels[top]["peak"], "unit": kernels[top]["unit"], "frac": kernels[top]["frac"],
