@@ -216,3 +216,36 @@ def test_w4a8_decode_step_stage_by_stage(S):
     ry, acc2 = oracle.linear_w4a8(f8, sf, ow.w2, bias=w16["b2"], residual=t["h1"], with_acc=True)
     mag2 = np.abs(acc2) * (sf[:, None].astype(np.float64) * ow.w2.cscale[None, :]) + np.abs(t["h1"].astype(np.float64))
     assert _close(y.cpu().numpy(), ry, mag2 + np.abs(w16["b2"].astype(np.float64))[None, :])
+
+
+def test_w4a8_stack_streamed_equals_resident_layers():
+    # the W4A8 blobs streamed from pinned host memory in slices (the stack's sliced prefetch) give
+    # the same bits as the same layers run from resident device blobs
+    nl, h, H, F, S, P = 3, 256, 4, 512, 8, 12
+    cfg = fg.LayerConfig(h, H, F, act_bits=8)
+    w16 = [si.layer_weights_f16(27 + l, h, F, std=0.05, bias_std=0.05, ln_random=True) for l in range(nl)]
+    dev_w = [fg.LayerWeights.from_fp16(cfg, w) for w in w16]
+    host = [torch.empty(cfg.blob_bytes(), dtype=torch.uint8, pin_memory=True) for _ in range(nl)]
+    for hb, dw in zip(host, dev_w):
+        hb.copy_(dw.blob)
+    st = fg.Stack(cfg, host)
+    caches = [fg.KVCache(S, H, h // H, 64) for _ in range(nl)]
+    st.prefill(caches, dev(si.hidden_block(27, si.STREAM["prompt"], S, P, h)), dev(np.zeros(S, np.int32)))
+    x = dev(si.decode_inputs(27, 0, S, h))
+    pos = dev(np.full(S, P, np.int32))
+    snap = [[a.clone() for a in c.arrays()] for c in caches]
+    y = st.decode(caches, x, pos, num_gpu_batches=2)
+    torch.cuda.synchronize()
+    after = [[a.clone() for a in c.arrays()] for c in caches]
+    for c, s in zip(caches, snap):
+        for a, b in zip(c.arrays(), s):
+            a.copy_(b)
+    z = x
+    for l in range(nl):
+        z = fg.fg_layer_decode(cfg, dev_w[l], caches[l], z, pos, num_gpu_batches=2)
+    fg.fg_sync_status()
+    assert torch.equal(y, z)
+    for c, s in zip(caches, after):
+        for a, b in zip(c.arrays(), s):
+            assert torch.equal(a, b)
+    st.close()

@@ -98,3 +98,25 @@ def test_noalloc_rejects_blocks_beyond_the_scratch(fg_lib):
     x = torch.zeros((S, h), dtype=torch.float16, device="cuda")
     with pytest.raises(fg.FgError, match="WORKSPACE"):
         fg.fg_layer_decode_noalloc(cfg, lw, cache, x, torch.zeros(S, dtype=torch.int32, device="cuda"))
+
+
+def test_noalloc_w4a8_layer_equals_workspace_decode(fg_lib):
+    # the W4A8 form of the layer through the allocation-free entry: same kernels, same bits
+    fg = fg_lib
+    h, H, F, S, P = 768, 12, 3072, 16, 24
+    cfg = fg.LayerConfig(h, H, F, act_bits=8)
+    w16 = si.layer_weights_f16(28, h, F, std=0.05, bias_std=0.05, ln_random=True)
+    lw = fg.LayerWeights.from_fp16(cfg, w16)
+    ref_cache = fg.KVCache(S, H, h // H, 64)
+    fg.fg_layer_prefill(cfg, lw, ref_cache, _dev(si.hidden_block(28, si.STREAM["prompt"], S, P, h)),
+                        _dev(np.zeros(S, np.int32)), num_gpu_batches=2)
+    na_cache = fg.KVCache(S, H, h // H, 64, arrays=[a.clone() for a in ref_cache.arrays()])
+    assert cfg.workspace_bytes(S) <= fg.NOALLOC_SCRATCH_BYTES
+    x = _dev(si.decode_inputs(28, 0, S, h))
+    pos = _dev(np.full(S, P, np.int32))
+    y_ref = fg.fg_layer_decode(cfg, lw, ref_cache, x, pos, num_gpu_batches=2)
+    y_na = fg.fg_layer_decode_noalloc(cfg, lw, na_cache, x, pos, num_gpu_batches=2)
+    fg.fg_sync_status()
+    assert torch.equal(y_ref, y_na)
+    for a, b in zip(ref_cache.arrays(), na_cache.arrays()):
+        assert torch.equal(a, b)
