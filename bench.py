@@ -683,7 +683,8 @@ def run_stack(args, wl):
         host.append(hb)
     del tmp
     torch.cuda.synchronize()
-    st = fg.Stack(cfg, host, device=dev)
+    nbuf = 2 if kv_host else args.staging_buffers   # the host-KV stack alternates two staging caches
+    st = fg.Stack(cfg, host, device=dev, staging_buffers=nbuf)
     # KV caches: seeded random codes and group min/scale for the prompt positions (a decode
     # step reads the same bytes whatever they hold; prefilling 48 layers x 512 tokens through
     # the per-row attention kernel would take far longer than the timed steps)
@@ -780,6 +781,7 @@ def run_stack(args, wl):
             "dtype": "f16", "data": "synthetic",
             "config": {"workload": args.workload, "layers": nl, "block": f"{nb}x{gbs}", "hidden": h, "prompt": P,
                        "weights_streamed_gb_per_step": round(blob_gb, 3),
+                       "staging_buffers": f"{nbuf} x {cfg.blob_bytes() / 1e9:.3f} GB",
                        "kv": "KV4 g64, seeded random codes at the prompt positions (no prefill)"},
             "host_link_gbs": round((blob_gb + fill_gb + wb_gb) / (ms / args.steps / 1e3), 1),
             "roofline": {"bound": "host-link", "achieved": round((blob_gb + fill_gb) / (ms / args.steps / 1e3), 1),
@@ -941,6 +943,8 @@ def main():
     ap.add_argument("--group", type=int, choices=(64, 128), default=64,
                     help="quantisation group size: of the layer's weights and KV cache (layer workloads), or of "
                          "--kernel quantize/dequantize/*_gemm")
+    ap.add_argument("--staging-buffers", type=int, choices=(1, 2), default=2,
+                    help="opt-30b-stack: device staging blobs (2 alternate; 1 is refilled slice by slice)")
     ap.add_argument("--gemm-scratch", choices=("auto", "persistent", "classic", "none"), default="auto",
                     help="--kernel *_gemm: the full scratch (auto), the full scratch and the persistent launch "
                          "(persistent), the classic launch's split-k scratch (classic), or none (splits added on chip)")

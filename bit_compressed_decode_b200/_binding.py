@@ -111,6 +111,7 @@ _decl("fg_stack_decode_host_kv", c_int, P, POINTER(fg_kv_cache), POINTER(fg_kv_c
 _decl("fg_stack_inject_copy_failure", c_int, P, c_int)
 _decl("fg_test_gemm_stall", c_int, c_int, ctypes.c_uint64)
 _decl("fg_stack_destroy", c_int, P)
+_decl("fg_stack_one_buffer_bytes", c_size_t, POINTER(fg_layer_config))
 
 
 def lib():
@@ -628,17 +629,22 @@ def fg_status_string(code: int) -> str:
 class Stack:
     """A stack of layers whose blobs live in (pinned) host tensors; see fg_stack_create."""
 
-    def __init__(self, cfg: LayerConfig, host_blobs, device="cuda"):
+    def __init__(self, cfg: LayerConfig, host_blobs, device="cuda", staging_buffers: int = 2):
+        """``staging_buffers``: 2 (layers alternate between two device blobs) or 1 (one blob,
+        refilled slice by slice as the layer before finishes with each slice)."""
+        if staging_buffers not in (1, 2):
+            raise ValueError("staging_buffers must be 1 or 2")
         self.cfg = cfg
         self.host_blobs = list(host_blobs)
-        nbytes = cfg.blob_bytes()
-        self.staging = [torch.empty(nbytes, dtype=torch.uint8, device=device) for _ in range(2)]
+        c0 = cfg.struct()
+        nbytes = cfg.blob_bytes() if staging_buffers == 2 else int(_lib.fg_stack_one_buffer_bytes(ctypes.byref(c0)))
+        self.staging = [torch.empty(nbytes, dtype=torch.uint8, device=device) for _ in range(staging_buffers)]
         arr = (c_void_p * len(self.host_blobs))(*[b.data_ptr() for b in self.host_blobs])
         self._arr = arr
         h = c_void_p()
         c = cfg.struct()
         _check(_lib.fg_stack_create(ctypes.byref(c), len(self.host_blobs), arr, _ptr(self.staging[0]),
-                                    _ptr(self.staging[1]), ctypes.byref(h)), "fg_stack_create")
+                                    _ptr(self.staging[-1]), ctypes.byref(h)), "fg_stack_create")
         self._h = h
 
     def workspace_bytes(self, rows: int) -> int:

@@ -11,6 +11,11 @@
 // QKV GEMM starts once wqkv has landed while wo, w1 and w2 are still crossing the link
 // (the weight loader that slices weights across batches, TightLLM abstract; the
 // fine-grained offloading pipeline of PIPO, abstract).  For caches larger than HBM
+// With one staging buffer (fg_stack_create given the same buffer twice, of
+// fg_stack_one_buffer_bytes) each matrix of layer l+1 waits for layer l's kernels that read
+// the same matrix: about half the staging memory.  The vectors (biases, LayerNorm parameters),
+// needed first and last by a layer, alternate between the blob's vector slot and a second
+// one after the blob, so layer l+1's vectors never wait for layer l's last GEMM.
 // (a 175B-class stack), fg_stack_decode_host_kv keeps every layer's 4-bit KV cache in
 // pinned host memory too: the copy stream fills a device KV staging cache with the layer's
 // cached positions next to its blob, and writes only the new token slots back after the
@@ -27,6 +32,7 @@ struct fg_stack {
   int num_layers;
   std::vector<void *> host;
   void *staging[2];
+  int nbuf;  // 2: layers alternate between the two staging buffers; 1: one buffer (staging[0])
   // per staging buffer: the layer-step slice events (see fg_layer_slices; entry 2 is the
   // host-KV staging cache), and the host-KV write-back from KV staging cache b
   fg_layer_slices ev[2];
@@ -40,6 +46,37 @@ namespace {
 
 // layer-step event index of blob slice i (vectors, wqkv, wo, w1, w2)
 constexpr int kSliceEvent[5] = {0, 1, 3, 4, 5};
+
+// The staging of layer l: buffer, its events, and where its vectors go.  One buffer: the
+// matrices use staging[0] and ev[0]; the vectors of odd layers sit after the blob and use
+// ev[1]'s vector events.
+struct Staging {
+  uint8_t *blob;
+  fg_layer_slices ev;   // the events the layer step uses
+  size_t vec_shift;     // added to the blob's vector offsets
+  int evb;              // the ev[] entry of the matrices (and of the vectors when vec_ev < 0)
+  int vec_ev;           // the ev[] entry of the vectors
+};
+
+Staging staging_of(const fg_stack *st, int l) {
+  Staging g;
+  if (st->nbuf == 2) {
+    const int b = l & 1;
+    g.blob = static_cast<uint8_t *>(st->staging[b]);
+    g.ev = st->ev[b];
+    g.vec_shift = 0;
+    g.evb = g.vec_ev = b;
+  } else {
+    g.blob = static_cast<uint8_t *>(st->staging[0]);
+    g.ev = st->ev[0];
+    g.evb = 0;
+    g.vec_ev = l & 1;
+    g.ev.ready[0] = st->ev[g.vec_ev].ready[0];
+    g.ev.done[0] = st->ev[g.vec_ev].done[0];
+    g.vec_shift = (l & 1) ? st->blob_bytes - st->sbegin[0] : 0;
+  }
+  return g;
+}
 
 // Copies layer l's blob into staging buffer l % 2, slice by slice, on the copy stream: each
 // slice waits until the layer that used the buffer before is done with it.  With a KV fill
@@ -65,25 +102,31 @@ fg_status stack_run(fg_stack *st, const fg_kv_cache *kv, const fg_half *x_in, fg
 
   fg_status rc = prefetch_sliced(st, 0, ps, nullptr, nullptr, 0);
   for (int l = 0; rc == FG_OK && l < st->num_layers; l++) {
-    const int b = l & 1;
-    if (l + 1 < st->num_layers && (rc = prefetch_sliced(st, l + 1, ps, nullptr, nullptr, 0)) != FG_OK) break;
+    const Staging g = staging_of(st, l);
+    // two buffers: layer l+1's copies are enqueued first (they wait only for layer l-1);
+    // one buffer: after layer l's kernels, whose `done` events the copies then wait for
+    if (st->nbuf == 2 && l + 1 < st->num_layers && (rc = prefetch_sliced(st, l + 1, ps, nullptr, nullptr, 0)) != FG_OK)
+      break;
     fg_layer_weights w;
-    if ((rc = fg_layer_weights_from_blob(&st->cfg, st->staging[b], &w)) != FG_OK) break;
+    if ((rc = fg_layer_weights_from_blob(&st->cfg, g.blob, &w)) != FG_OK) break;
+    fg_half **vecs[8] = {&w.bqkv, &w.bo, &w.b1, &w.b2, &w.ln1_g, &w.ln1_b, &w.ln2_g, &w.ln2_b};
+    for (fg_half **v : vecs) *v = reinterpret_cast<fg_half *>(reinterpret_cast<uint8_t *>(*v) + g.vec_shift);
     const fg_half *in = l == 0 ? x_in : buf[(l - 1) & 1];
     fg_half *out = l == st->num_layers - 1 ? x_out : buf[l & 1];
     if (prompt_len > 0) {
       // a prompt step waits for the whole blob (its chunks reuse every slice), then frees it
       for (int i = 0; i < 6 && rc == FG_OK; i++)
-        if (st->ev[b].ready[i] && i != 2) rc = fg_cuda_check(cudaStreamWaitEvent(cs, st->ev[b].ready[i], 0));
+        if (g.ev.ready[i] && i != 2) rc = fg_cuda_check(cudaStreamWaitEvent(cs, g.ev.ready[i], 0));
       if (rc == FG_OK)
         rc = fg_layer_prefill(&st->cfg, &w, &kv[l], in, out, positions, prompt_len, nb, gbs, lws, lws_bytes, cs);
       for (int i = 0; i < 6 && rc == FG_OK; i++)
-        if (i != 2) rc = fg_cuda_check(cudaEventRecord(st->ev[b].done[i], cs));
+        if (i != 2) rc = fg_cuda_check(cudaEventRecord(g.ev.done[i], cs));
     } else {
-      fg_layer_slices sl = st->ev[b];
+      fg_layer_slices sl = g.ev;
       sl.ready[2] = sl.done[2] = nullptr;  // the cache is resident
       rc = fg_layer_decode_sliced(&st->cfg, &w, &kv[l], in, out, positions, nb, gbs, lws, lws_bytes, cs, &sl);
     }
+    if (rc == FG_OK && st->nbuf == 1 && l + 1 < st->num_layers) rc = prefetch_sliced(st, l + 1, ps, nullptr, nullptr, 0);
   }
   if (rc != FG_OK) {
     // drain what was enqueued so nothing is left waiting on this stack's buffers
@@ -131,6 +174,7 @@ fg_status stack_run_host_kv(fg_stack *st, const fg_kv_cache *host_kv, const fg_k
                             int wb_begin, int wb_end, const fg_half *x_in, fg_half *x_out, const int32_t *positions,
                             int nb, int gbs, void *workspace, size_t ws_bytes, cudaStream_t cs, cudaStream_t ps) {
   if (!st || !host_kv || !dev_kv) return FG_ERR_INVALID;
+  if (st->nbuf != 2) return FG_ERR_UNSUPPORTED;  // the KV staging caches alternate with the blobs
   const int S = nb * gbs;
   if (S == 0) return FG_OK;
   if (!workspace || !fg_aligned16(workspace) || !x_in || !x_out) return FG_ERR_INVALID;
@@ -176,21 +220,24 @@ fg_status stack_run_host_kv(fg_stack *st, const fg_kv_cache *host_kv, const fg_k
 
 fg_status prefetch_sliced(fg_stack *st, int l, cudaStream_t ps, const fg_kv_cache *fill_dst,
                           const fg_kv_cache *fill_src, int fill_len) {
-  const int b = l & 1;
+  const int b = l & 1;  // the KV staging cache and its write-back event (two buffers only)
   if (st->inject_failures > 0) {
     st->inject_failures--;
     return FG_ERR_CUDA;
   }
-  uint8_t *dst = static_cast<uint8_t *>(st->staging[b]);
+  const Staging g = staging_of(st, l);
   const uint8_t *src = static_cast<const uint8_t *>(st->host[l]);
-  fg_layer_slices &ev = st->ev[b];
+  fg_layer_slices &ev = st->ev[g.evb];
   for (int i = 0; i < 5; i++) {
     const int e = kSliceEvent[i];
-    fg_status r = fg_cuda_check(cudaStreamWaitEvent(ps, ev.done[e], 0));
+    const size_t shift = i == 0 ? g.vec_shift : 0;
+    cudaEvent_t ready = i == 0 ? st->ev[g.vec_ev].ready[0] : ev.ready[e];
+    cudaEvent_t done = i == 0 ? st->ev[g.vec_ev].done[0] : ev.done[e];
+    fg_status r = fg_cuda_check(cudaStreamWaitEvent(ps, done, 0));
     if (r == FG_OK)
-      r = fg_cuda_check(cudaMemcpyAsync(dst + st->sbegin[i], src + st->sbegin[i], st->send[i] - st->sbegin[i],
-                                        cudaMemcpyHostToDevice, ps));
-    if (r == FG_OK) r = fg_cuda_check(cudaEventRecord(ev.ready[e], ps));
+      r = fg_cuda_check(cudaMemcpyAsync(g.blob + st->sbegin[i] + shift, src + st->sbegin[i],
+                                        st->send[i] - st->sbegin[i], cudaMemcpyHostToDevice, ps));
+    if (r == FG_OK) r = fg_cuda_check(cudaEventRecord(ready, ps));
     if (r != FG_OK) return r;
     if (i == 1 && fill_dst) {
       // the layer's KV cache: after the previous layer on this staging cache is done with it
@@ -225,6 +272,7 @@ extern "C" fg_status fg_stack_create(const fg_layer_config *c, int num_layers, v
   st->host.assign(host_blobs, host_blobs + num_layers);
   st->staging[0] = dev_staging0;
   st->staging[1] = dev_staging1;
+  st->nbuf = dev_staging0 == dev_staging1 ? 1 : 2;
   st->blob_bytes = bytes;
   st->inject_failures = 0;
   fg_layer_blob_slices(c, st->sbegin, st->send);
@@ -291,4 +339,11 @@ extern "C" fg_status fg_stack_destroy(fg_stack *st) {
   }
   delete st;
   return FG_OK;
+}
+
+extern "C" size_t fg_stack_one_buffer_bytes(const fg_layer_config *c) {
+  const size_t bytes = fg_layer_blob_bytes(c);
+  size_t begin[5], end[5];
+  if (bytes == 0 || fg_layer_blob_slices(c, begin, end) != FG_OK) return 0;
+  return bytes + (end[0] - begin[0]);  // the blob, then a second slot for the vectors
 }

@@ -434,9 +434,18 @@ typedef struct fg_stack fg_stack;  /* opaque */
 /* Prepares a stack of num_layers layers whose blobs live in host memory
  * (host_blobs[l], fg_layer_blob_bytes(c) each; pinned for overlap).
  * dev_staging[0..1]: two device buffers of fg_layer_blob_bytes(c) bytes that
- * the next layer is prefetched into while the current one computes.
+ * the next layer is prefetched into while the current one computes.  The same
+ * buffer given twice, of fg_stack_one_buffer_bytes(c) bytes, selects one
+ * staging buffer: each matrix of layer l+1 is then copied once layer l's
+ * kernels that read that matrix have run, and the vectors (biases, LayerNorm
+ * parameters) alternate between two slots (about half the staging memory;
+ * fg_stack_decode_host_kv needs two buffers and returns FG_ERR_UNSUPPORTED
+ * with one).
  * Creates CUDA events only (no memory allocation).  *out is released with
  * fg_stack_destroy. */
+/* Bytes of the one staging buffer of a one-buffer stack: the blob, then a second slot for the
+ * vectors (0 for a configuration the library rejects). */
+FG_API size_t fg_stack_one_buffer_bytes(const fg_layer_config *c);
 FG_API fg_status fg_stack_create(const fg_layer_config *c, int num_layers, void *const *host_blobs,
                           void *dev_staging0, void *dev_staging1, fg_stack **out);
 

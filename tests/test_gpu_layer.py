@@ -452,3 +452,32 @@ def test_large_layer_shapes_sampled_sequences(shape):
         r, _ = oracle.layer_rows(L.ow, H, oc, x[sample], np.arange(len(sample)), np.full(len(sample), P + t),
                                  nthreads=len(sample))
         assert delta_err(y.cpu().numpy()[sample], x[sample], r) <= TOL, t
+
+
+def test_stack_one_staging_buffer_equals_resident_layers():
+    # one staging blob, refilled slice by slice as the layer before finishes with each slice:
+    # prefill and decode give the same bits as the layers run from resident device blobs
+    nl, h, H, F, S, P = 3, 256, 4, 512, 8, 12
+    cfg, w16, dev_w, host = _stack_setup(nl, h, H, F, S, P, seed=17)
+    st = fg.Stack(cfg, host, staging_buffers=1)
+    caches = [fg.KVCache(S, H, h // H, 64) for _ in range(nl)]
+    prompt = dev(si.hidden_block(17, si.STREAM["prompt"], S, P, h))
+    yp = st.prefill(caches, prompt, dev(np.zeros(S, np.int32)))
+    ref_caches = [fg.KVCache(S, H, h // H, 64) for _ in range(nl)]
+    z = prompt
+    for l in range(nl):
+        z = fg.fg_layer_prefill(cfg, dev_w[l], ref_caches[l], z, dev(np.zeros(S, np.int32)))
+    torch.cuda.synchronize()
+    assert torch.equal(yp, z)
+    x = dev(si.decode_inputs(17, 0, S, h))
+    pos = dev(np.full(S, P, np.int32))
+    y = st.decode(caches, x, pos, num_gpu_batches=2)
+    z = x
+    for l in range(nl):
+        z = fg.fg_layer_decode(cfg, dev_w[l], ref_caches[l], z, pos, num_gpu_batches=2)
+    fg.fg_sync_status()
+    assert torch.equal(y, z)
+    for c, r in zip(caches, ref_caches):
+        for a, b in zip(c.arrays(), r.arrays()):
+            assert torch.equal(a, b)
+    st.close()
