@@ -781,7 +781,7 @@ def run_stack(args, wl):
             "dtype": "f16", "data": "synthetic",
             "config": {"workload": args.workload, "layers": nl, "block": f"{nb}x{gbs}", "hidden": h, "prompt": P,
                        "weights_streamed_gb_per_step": round(blob_gb, 3),
-                       "staging_buffers": f"{nbuf} x {cfg.blob_bytes() / 1e9:.3f} GB",
+                       "staging_buffers": f"{nbuf} x {st.staging[0].numel() / 1e9:.3f} GB",
                        "kv": "KV4 g64, seeded random codes at the prompt positions (no prefill)"},
             "host_link_gbs": round((blob_gb + fill_gb + wb_gb) / (ms / args.steps / 1e3), 1),
             "roofline": {"bound": "host-link", "achieved": round((blob_gb + fill_gb) / (ms / args.steps / 1e3), 1),
