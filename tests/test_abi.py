@@ -295,3 +295,14 @@ def test_w4a8_layer_config_rules():
     with pytest.raises(fg.FgError):
         fg.LayerConfig(h, H, F, act_bits=4).blob_bytes()
     assert fg.LayerConfig(h, H, F, act_bits=8).workspace_bytes(16) > fg.LayerConfig(h, H, F).workspace_bytes(16)
+
+
+def test_stack_one_buffer_bytes():
+    # one staging buffer: the blob, then a second slot for the vectors (biases, LayerNorm parameters)
+    for act_bits in (16, 8):
+        cfg = fg.LayerConfig(768, 12, 3072, act_bits=act_bits)
+        c = cfg.struct()
+        vec = sum((n * 2 + 255) // 256 * 256 for n in (3 * 768, 768, 3072, 768, 768, 768, 768, 768))
+        assert B.lib().fg_stack_one_buffer_bytes(ctypes.byref(c)) == cfg.blob_bytes() + vec
+    bad = fg.LayerConfig(768, 12, 3072, act_bits=4).struct()
+    assert B.lib().fg_stack_one_buffer_bytes(ctypes.byref(bad)) == 0

@@ -117,8 +117,10 @@ def _run_and_check(M, N, K, seed, rows=None, relu=False, qcols=0, qscale=1.0, wi
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 256, 128), (5, 384, 640), (40, 512, 1024), (130, 256, 4096),
-                                   (300, 768, 2048), (16, 256, 16384)])
+                                   (300, 768, 2048), (16, 256, 16384), (600, 256, 768)])
 def test_linear_w4a8_matches_oracle(M, N, K):
+    # (600, 256, 768): more than 256 tokens with K / 64 = 12 metadata columns per row, which the
+    # pair launch's 16-column tensor copies do not take: the one-SM kernel over 3 token tiles
     _run_and_check(M, N, K, seed=33)
 
 
