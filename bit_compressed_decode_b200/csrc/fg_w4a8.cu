@@ -13,11 +13,12 @@
 //   y[t][n] = epi( acc[t][n] * (ascale[t] * cscale[n]) + bias[n] ), acc = sum_k a8 * w8 exact in
 //     int32, the rest one fp32 operation at a time (q-scale, ReLU, residual as in the W4A16 layer).
 //
-// Larger blocks (M > 256) run on CTA pairs: the W4A16 pair kernel (fg_gemm.cu) in its int8 form
-// -- the same pipeline with the codes widened to int8, tcgen05.mma.cta_group::2.kind::i8 and the
-// scales applied once a sum is final.
+// Larger blocks (M > 256, with rows of K / 64 metadata bytes that are whole 16-byte units) run on
+// CTA pairs: the W4A16 pair kernel (fg_gemm.cu) in its int8 form -- the same pipeline with the
+// codes widened to int8, tcgen05.mma.cta_group::2.kind::i8 and the scales applied once a sum is
+// final.
 //
-// GEMM kernel, one SM per output tile (M <= 256): 256 output features (two 128-row accumulators) x NT tokens
+// GEMM kernel, one SM per output tile (every other shape): 256 output features (two 128-row accumulators) x NT tokens
 // x a k-range, k-tiles of 128 (two groups; one 128-byte row of int8 per feature and per token).
 //   warps 0..7  thread t owns weight row n0 + t: per k-tile it loads 64 code bytes and both groups'
 //               (gmin, gstep), widens 8 codes at a time to int8 -- two byte permutes, one 32-bit
