@@ -1450,6 +1450,9 @@ extern "C" fg_status fg_linear_w4a16(const fg_half *x, int M, int K, const fg_qt
   if (M == 0) return FG_OK;
   if (!x || !y || !w->codes || !w->mins || !w->scales) return FG_ERR_INVALID;
   if (!fg_aligned16(x) || !fg_aligned16(y) || !fg_aligned16(w->codes)) return FG_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(bias) & 1u) || (reinterpret_cast<uintptr_t>(w->mins) & 1u) ||
+      (reinterpret_cast<uintptr_t>(w->scales) & 1u))
+    return FG_ERR_INVALID;
   if ((flags & FG_EPI_RESIDUAL) && (!residual || !fg_aligned16(residual))) return FG_ERR_INVALID;
   // weights may come from the kernel just before (fg_quantize): no overlap with it
   return fg_linear_launch(x, M, K, w, bias, residual, flags, qscale_cols, qscale, y, workspace, workspace_bytes,

@@ -681,7 +681,9 @@ extern "C" fg_status fg_linear_w4a8(const int8_t *a8, const float *ascale, int M
   if (M == 0) return FG_OK;
   if (!a8 || !ascale || !y || !w->codes || !w->gmin || !w->gstep || !w->cscale) return FG_ERR_INVALID;
   if (!fg_aligned16(a8) || !fg_aligned16(y) || !fg_aligned16(w->codes) ||
-      (reinterpret_cast<uintptr_t>(w->gmin) & 1u) || (reinterpret_cast<uintptr_t>(w->gstep) & 1u))
+      (reinterpret_cast<uintptr_t>(w->gmin) & 1u) || (reinterpret_cast<uintptr_t>(w->gstep) & 1u) ||
+      (reinterpret_cast<uintptr_t>(w->cscale) & 3u) || (reinterpret_cast<uintptr_t>(ascale) & 3u) ||
+      (reinterpret_cast<uintptr_t>(bias) & 1u))
     return FG_ERR_INVALID;
   if ((flags & FG_EPI_RESIDUAL) && (!residual || !fg_aligned16(residual))) return FG_ERR_INVALID;
   if (fg_w4a8_pair_eligible(M, K, w))

@@ -201,7 +201,8 @@ enum {
  * (with FG_EPI_RESIDUAL); the first qscale_cols outputs of each row are
  * multiplied by qscale after the bias.  w->group 64 or 128 with K % group == 0,
  * N % 128 == 0; x, y, the
- * codes and the residual 16-byte aligned (FG_ERR_INVALID otherwise).
+ * codes and the residual 16-byte aligned, the mins, scales and bias 2-byte
+ * aligned (FG_ERR_INVALID otherwise).
  * Tensor cores dequantise W tiles in shared memory ([G3]: on-the-fly
  * dequantisation for FP16 compute).
  * Launches (see fg_linear_plan): M <= 256 runs one SM per output tile; larger M
@@ -277,8 +278,8 @@ FG_API fg_status fg_act8_quantize(const fg_half *x, int M, int K, int8_t *a8, fl
 /* The W4A8 product above: a8 [M][K] int8 and ascale [M] from fg_act8_quantize, w from
  * fg_w4a8_quantize_weight with w->K == K, bias fp16 [N] or NULL, residual fp16 [M][N].
  * K % 128 == 0 and K <= 65536 (the int32 sums stay exact), N % 128 == 0 (FG_ERR_SHAPE);
- * a8, y, the residual and the codes 16-byte aligned, gmin and gstep 2-byte aligned
- * (FG_ERR_INVALID).  M <= 256: one SM per output tile of 256 features x tile_tokens tokens, the
+ * a8, y, the residual and the codes 16-byte aligned, gmin, gstep and bias 2-byte aligned,
+ * cscale and ascale 4-byte aligned (FG_ERR_INVALID).  M <= 256: one SM per output tile of 256 features x tile_tokens tokens, the
  * k-range possibly split over a cluster whose CTAs add their int32 partials exactly.  M > 256,
  * (K / 64) % 16 == 0 and gmin, gstep 16-byte aligned: the CTA-pair launch of fg_linear_w4a16 in
  * its int8 form (256- or 512-token tiles, k-tiles of 128); its k splits add int32 partials

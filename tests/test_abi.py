@@ -268,6 +268,10 @@ def test_w4a8_entry_points_validate_on_host():
     odd = _fake_w4a8()
     odd.gmin = 0x200001                                                # metadata read 2 bytes at a time
     assert _rc("fg_linear_w4a8", *lin(w=odd)) == 1
+    odd = _fake_w4a8()
+    odd.cscale = 0x400002                                              # fp32 row scales
+    assert _rc("fg_linear_w4a8", *lin(w=odd)) == 1
+    assert _rc("fg_linear_w4a8", *lin(ascale=P * 2 + 2)) == 1          # fp32 token scales
     assert _rc("fg_act8_quantize", P, 4, 96, P * 2, P * 3, None) == 2  # K not a multiple of 64
     assert _rc("fg_act8_quantize", P, 0, 128, P * 2, P * 3, None) == 0
     assert _rc("fg_act8_quantize", P + 2, 4, 128, P * 2, P * 3, None) == 1
