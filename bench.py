@@ -45,6 +45,8 @@ WORKLOADS = {
     # OPT-30B-shaped stack: 48 layers whose W4 blobs stay in pinned host memory and are
     # prefetched layer by layer on a side stream; KV4 caches resident in HBM
     "opt-30b-stack": dict(hidden=7168, heads=56, ffn=28672, nb=4, gbs=64, prompt=512, steps=32, layers=48),
+    "opt-30b-stack-w4a8": dict(hidden=7168, heads=56, ffn=28672, nb=4, gbs=64, prompt=512, steps=32, layers=48,
+                               act_bits=8),
     # OPT-175B-shaped stack: weights AND KV4 caches in pinned host memory; each layer's cache is
     # filled into a device staging cache before the layer and its new slots written back after.
     # The model has 96 layers (about 3.06 GB of host memory each); unless --layers is given the
@@ -651,7 +653,8 @@ def run_stack(args, wl):
     nb, gbs = wl["nb"], wl["gbs"]
     S, d = nb * gbs, h // H
     maxL = (P + wl["steps"] + 63) // 64 * 64
-    cfg = fg.LayerConfig(h, H, F)
+    act_bits = wl.get("act_bits", 16)
+    cfg = fg.LayerConfig(h, H, F, act_bits=act_bits)
     ng = d // 64
     kv_host = bool(wl.get("kv_host"))
     if kv_host and not args.layers:
@@ -672,7 +675,10 @@ def run_stack(args, wl):
     for _ in range(nl):
         for name, shape in (("wqkv", (3 * h, h)), ("wo", (h, h)), ("w1", (F, h)), ("w2", (h, F))):
             w = torch.randn(shape, generator=g, device=dev, dtype=torch.float16) * 0.02
-            fg.fg_quantize(w, dim=1, out=tmp.matrix(name))
+            if act_bits == 8:
+                fg.fg_w4a8_quantize_weight(w, out=tmp.w4a8_matrix(name))
+            else:
+                fg.fg_quantize(w, dim=1, out=tmp.matrix(name))
             del w
         for name in ("bqkv", "bo", "b1", "b2", "ln1_b", "ln2_b"):
             tmp.vector(name).zero_()
@@ -778,7 +784,7 @@ def run_stack(args, wl):
                        "decode tokens/s of the OPT layer stack (W4 weights streamed from pinned host, KV4 in HBM)"),
             "value": world * S * args.steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "dtype": "f16", "data": "synthetic",
+            "dtype": "i8 products, f16 elsewhere" if act_bits == 8 else "f16", "data": "synthetic",
             "config": {"workload": args.workload, "layers": nl, "block": f"{nb}x{gbs}", "hidden": h, "prompt": P,
                        "weights_streamed_gb_per_step": round(blob_gb, 3),
                        "staging_buffers": f"{nbuf} x {st.staging[0].numel() / 1e9:.3f} GB",
