@@ -684,8 +684,15 @@ def run_stack(args, wl):
             tmp.vector(name).zero_()
         tmp.vector("ln1_g").fill_(1.0)
         tmp.vector("ln2_g").fill_(1.0)
-        hb = torch.empty(cfg.blob_bytes(), dtype=torch.uint8, pin_memory=True)
-        hb.copy_(tmp.blob)
+        # --resident-layers R: R layers spread evenly over the stack keep their blob in device
+        # memory (read in place), so the copy of a streamed layer overlaps the compute of the
+        # resident one before it
+        l = len(host)
+        if (l + 1) * args.resident_layers // nl > l * args.resident_layers // nl:
+            hb = tmp.blob.clone()
+        else:
+            hb = torch.empty(cfg.blob_bytes(), dtype=torch.uint8, pin_memory=True)
+            hb.copy_(tmp.blob)
         host.append(hb)
     del tmp
     torch.cuda.synchronize()
@@ -770,7 +777,8 @@ def run_stack(args, wl):
     clocks = sampler.stop()
     ms = replicas.max_over_ranks(e0.elapsed_time(e1), device=dev)
     fg.fg_sync_status()
-    blob_gb = cfg.blob_bytes() * nl / 1e9
+    nres = min(args.resident_layers, nl)
+    blob_gb = cfg.blob_bytes() * (nl - nres) / 1e9
     slot_bytes = S * H * 2 * (d // 2 + 4 * ng)          # K and V codes + min/scale of one position
     fill_gb = wb_gb = 0.0
     if kv_host:
@@ -788,6 +796,7 @@ def run_stack(args, wl):
             "config": {"workload": args.workload, "layers": nl, "block": f"{nb}x{gbs}", "hidden": h, "prompt": P,
                        "weights_streamed_gb_per_step": round(blob_gb, 3),
                        "staging_buffers": f"{nbuf} x {st.staging[0].numel() / 1e9:.3f} GB",
+                       "resident_layers": nres,
                        "kv": "KV4 g64, seeded random codes at the prompt positions (no prefill)"},
             "host_link_gbs": round((blob_gb + fill_gb + wb_gb) / (ms / args.steps / 1e3), 1),
             "roofline": {"bound": "host-link", "achieved": round((blob_gb + fill_gb) / (ms / args.steps / 1e3), 1),
@@ -949,6 +958,8 @@ def main():
     ap.add_argument("--group", type=int, choices=(64, 128), default=64,
                     help="quantisation group size: of the layer's weights and KV cache (layer workloads), or of "
                          "--kernel quantize/dequantize/*_gemm")
+    ap.add_argument("--resident-layers", type=int, default=0,
+                    help="stack workloads: layers whose weight blobs stay in device memory (read in place)")
     ap.add_argument("--staging-buffers", type=int, choices=(1, 2), default=2,
                     help="opt-30b-stack: device staging blobs (2 alternate; 1 is refilled slice by slice)")
     ap.add_argument("--gemm-scratch", choices=("auto", "persistent", "classic", "none"), default="auto",

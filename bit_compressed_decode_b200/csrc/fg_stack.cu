@@ -16,6 +16,9 @@
 // the same matrix: about half the staging memory.  The vectors (biases, LayerNorm parameters),
 // needed first and last by a layer, alternate between the blob's vector slot and a second
 // one after the blob, so layer l+1's vectors never wait for layer l's last GEMM.
+// A layer whose blob the caller placed in device memory stays resident: it is read in place,
+// with no copy and no staging buffer (the FlexGen guide's placement of part of the weights on
+// the GPU, section 1; with 180 GB of HBM most of a 175B model's 4-bit weights fit).
 // (a 175B-class stack), fg_stack_decode_host_kv keeps every layer's 4-bit KV cache in
 // pinned host memory too: the copy stream fills a device KV staging cache with the layer's
 // cached positions next to its blob, and writes only the new token slots back after the
@@ -31,6 +34,7 @@ struct fg_stack {
   fg_layer_config cfg;
   int num_layers;
   std::vector<void *> host;
+  std::vector<char> resident;  // 1: blob l is in device memory and is read in place
   void *staging[2];
   int nbuf;  // 2: layers alternate between the two staging buffers; 1: one buffer (staging[0])
   // per staging buffer: the layer-step slice events (see fg_layer_slices; entry 2 is the
@@ -107,20 +111,25 @@ fg_status stack_run(fg_stack *st, const fg_kv_cache *kv, const fg_half *x_in, fg
     // one buffer: after layer l's kernels, whose `done` events the copies then wait for
     if (st->nbuf == 2 && l + 1 < st->num_layers && (rc = prefetch_sliced(st, l + 1, ps, nullptr, nullptr, 0)) != FG_OK)
       break;
+    const bool res = st->resident[l];
     fg_layer_weights w;
-    if ((rc = fg_layer_weights_from_blob(&st->cfg, g.blob, &w)) != FG_OK) break;
-    fg_half **vecs[8] = {&w.bqkv, &w.bo, &w.b1, &w.b2, &w.ln1_g, &w.ln1_b, &w.ln2_g, &w.ln2_b};
-    for (fg_half **v : vecs) *v = reinterpret_cast<fg_half *>(reinterpret_cast<uint8_t *>(*v) + g.vec_shift);
+    if ((rc = fg_layer_weights_from_blob(&st->cfg, res ? st->host[l] : g.blob, &w)) != FG_OK) break;
+    if (!res) {
+      fg_half **vecs[8] = {&w.bqkv, &w.bo, &w.b1, &w.b2, &w.ln1_g, &w.ln1_b, &w.ln2_g, &w.ln2_b};
+      for (fg_half **v : vecs) *v = reinterpret_cast<fg_half *>(reinterpret_cast<uint8_t *>(*v) + g.vec_shift);
+    }
     const fg_half *in = l == 0 ? x_in : buf[(l - 1) & 1];
     fg_half *out = l == st->num_layers - 1 ? x_out : buf[l & 1];
     if (prompt_len > 0) {
       // a prompt step waits for the whole blob (its chunks reuse every slice), then frees it
-      for (int i = 0; i < 6 && rc == FG_OK; i++)
+      for (int i = 0; i < 6 && rc == FG_OK && !res; i++)
         if (g.ev.ready[i] && i != 2) rc = fg_cuda_check(cudaStreamWaitEvent(cs, g.ev.ready[i], 0));
       if (rc == FG_OK)
         rc = fg_layer_prefill(&st->cfg, &w, &kv[l], in, out, positions, prompt_len, nb, gbs, lws, lws_bytes, cs);
-      for (int i = 0; i < 6 && rc == FG_OK; i++)
+      for (int i = 0; i < 6 && rc == FG_OK && !res; i++)
         if (i != 2) rc = fg_cuda_check(cudaEventRecord(g.ev.done[i], cs));
+    } else if (res) {
+      rc = fg_layer_decode_sliced(&st->cfg, &w, &kv[l], in, out, positions, nb, gbs, lws, lws_bytes, cs, nullptr);
     } else {
       fg_layer_slices sl = g.ev;
       sl.ready[2] = sl.done[2] = nullptr;  // the cache is resident
@@ -197,12 +206,18 @@ fg_status stack_run_host_kv(fg_stack *st, const fg_kv_cache *host_kv, const fg_k
     if (l + 1 < st->num_layers &&
         (rc = prefetch_sliced(st, l + 1, ps, &dev_kv[(l + 1) & 1], &host_kv[l + 1], fill_len)) != FG_OK)
       break;
+    const bool res = st->resident[l];
     fg_layer_weights w;
-    if ((rc = fg_layer_weights_from_blob(&st->cfg, st->staging[b], &w)) != FG_OK) break;
+    if ((rc = fg_layer_weights_from_blob(&st->cfg, res ? st->host[l] : st->staging[b], &w)) != FG_OK) break;
     const fg_half *in = l == 0 ? x_in : buf[(l - 1) & 1];
     fg_half *out = l == st->num_layers - 1 ? x_out : buf[l & 1];
+    fg_layer_slices sl = st->ev[b];
+    if (res) {  // weights in place: only the KV staging cache's events
+      for (int i = 0; i < 6; i++)
+        if (i != 2) sl.ready[i] = sl.done[i] = nullptr;
+    }
     if ((rc = fg_layer_decode_sliced(&st->cfg, &w, &dev_kv[b], in, out, positions, nb, gbs, lws, lws_bytes, cs,
-                                     &st->ev[b])) != FG_OK)
+                                     &sl)) != FG_OK)
       break;
     // write the new slots back to the host cache once the layer's attention is done, on the copy stream
     if ((rc = fg_cuda_check(cudaStreamWaitEvent(ps, st->ev[b].done[2], 0))) != FG_OK) break;
@@ -228,6 +243,14 @@ fg_status prefetch_sliced(fg_stack *st, int l, cudaStream_t ps, const fg_kv_cach
   const Staging g = staging_of(st, l);
   const uint8_t *src = static_cast<const uint8_t *>(st->host[l]);
   fg_layer_slices &ev = st->ev[g.evb];
+  if (st->resident[l]) {  // weights in place; the layer's KV cache still goes to its staging cache
+    if (!fill_dst) return FG_OK;
+    fg_status r = fg_cuda_check(cudaStreamWaitEvent(ps, ev.done[2], 0));
+    if (r == FG_OK) r = fg_cuda_check(cudaStreamWaitEvent(ps, st->kv_back[b], 0));
+    if (r == FG_OK) r = kv_copy(*fill_dst, *fill_src, 0, fill_len, cudaMemcpyHostToDevice, ps);
+    if (r == FG_OK) r = fg_cuda_check(cudaEventRecord(ev.ready[2], ps));
+    return r;
+  }
   for (int i = 0; i < 5; i++) {
     const int e = kSliceEvent[i];
     const size_t shift = i == 0 ? g.vec_shift : 0;
@@ -270,6 +293,19 @@ extern "C" fg_status fg_stack_create(const fg_layer_config *c, int num_layers, v
   st->cfg = *c;
   st->num_layers = num_layers;
   st->host.assign(host_blobs, host_blobs + num_layers);
+  st->resident.assign(num_layers, 0);
+  for (int l = 0; l < num_layers; l++) {
+    cudaPointerAttributes pa;
+    if (cudaPointerGetAttributes(&pa, host_blobs[l]) == cudaSuccess) {
+      st->resident[l] = pa.type == cudaMemoryTypeDevice;
+    } else {
+      cudaGetLastError();  // plain host memory on older runtimes
+    }
+    if (st->resident[l] && (reinterpret_cast<uintptr_t>(host_blobs[l]) & 255)) {
+      delete st;
+      return FG_ERR_INVALID;
+    }
+  }
   st->staging[0] = dev_staging0;
   st->staging[1] = dev_staging1;
   st->nbuf = dev_staging0 == dev_staging1 ? 1 : 2;

@@ -433,7 +433,10 @@ FG_API fg_status fg_profile_collect(float *ms, int *count, int nslots);
 typedef struct fg_stack fg_stack;  /* opaque */
 
 /* Prepares a stack of num_layers layers whose blobs live in host memory
- * (host_blobs[l], fg_layer_blob_bytes(c) each; pinned for overlap).
+ * (host_blobs[l], fg_layer_blob_bytes(c) each; pinned for overlap).  A blob
+ * in device memory (256-byte aligned) keeps its layer resident: read in
+ * place, no copy, no staging buffer [G1: part of the weights placed on the
+ * GPU].
  * dev_staging[0..1]: two device buffers of fg_layer_blob_bytes(c) bytes that
  * the next layer is prefetched into while the current one computes.  The same
  * buffer given twice, of fg_stack_one_buffer_bytes(c) bytes, selects one

@@ -481,3 +481,58 @@ def test_stack_one_staging_buffer_equals_resident_layers():
         for a, b in zip(c.arrays(), r.arrays()):
             assert torch.equal(a, b)
     st.close()
+
+
+@pytest.mark.parametrize("buffers", [2, 1])
+def test_stack_with_resident_layers_equals_streamed(buffers):
+    # layers whose blobs sit in device memory are read in place (no copy, no staging buffer);
+    # mixed with streamed ones, prefill and decode give the bits of the all-streamed stack
+    nl, h, H, F, S, P = 4, 256, 4, 512, 8, 12
+    cfg, w16, dev_w, host = _stack_setup(nl, h, H, F, S, P, seed=19)
+    mixed = [dw.blob if l in (0, 2) else hb for l, (dw, hb) in enumerate(zip(dev_w, host))]
+    runs = []
+    for blobs in (host, mixed):
+        st = fg.Stack(cfg, blobs, staging_buffers=buffers)
+        caches = [fg.KVCache(S, H, h // H, 64) for _ in range(nl)]
+        yp = st.prefill(caches, dev(si.hidden_block(19, si.STREAM["prompt"], S, P, h)), dev(np.zeros(S, np.int32)))
+        y = st.decode(caches, dev(si.decode_inputs(19, 0, S, h)), dev(np.full(S, P, np.int32)), num_gpu_batches=2)
+        fg.fg_sync_status()
+        runs.append((yp.clone(), y.clone(), [[a.clone() for a in c.arrays()] for c in caches]))
+        st.close()
+    assert torch.equal(runs[0][0], runs[1][0]) and torch.equal(runs[0][1], runs[1][1])
+    for c0, c1 in zip(runs[0][2], runs[1][2]):
+        for a, b in zip(c0, c1):
+            assert torch.equal(a, b)
+
+
+def test_stack_host_kv_with_resident_layers():
+    # host-spilled caches with the weights of layers 0 and 2 resident in device memory (read in
+    # place; their KV caches still filled into the staging caches and written back): the same
+    # bits as the HBM-resident caches and all-streamed weights
+    nl, h, H, F, S, P, maxL = 3, 256, 4, 512, 8, 12, 64
+    cfg, w16, dev_w, host = _stack_setup(nl, h, H, F, S, P, seed=21)
+    st = fg.Stack(cfg, host)
+    caches = [fg.KVCache(S, H, h // H, maxL) for _ in range(nl)]
+    st.prefill(caches, dev(si.hidden_block(21, si.STREAM["prompt"], S, P, h)), dev(np.zeros(S, np.int32)))
+    torch.cuda.synchronize()
+    hcaches = [fg.KVCache(S, H, h // H, maxL, device="cpu", pin_memory=True) for _ in range(nl)]
+    for hc, c in zip(hcaches, caches):
+        for a, b in zip(hc.arrays(), c.arrays()):
+            a.copy_(b)
+    mixed = fg.Stack(cfg, [dev_w[0].blob, host[1], dev_w[2].blob])
+    staging = [fg.KVCache(S, H, h // H, maxL) for _ in range(2)]
+    cs, ps = torch.cuda.Stream(), torch.cuda.Stream()
+    p = np.full(S, P, np.int32)
+    x = dev(si.decode_inputs(21, 0, S, h))
+    y = st.decode(caches, x, dev(p), num_gpu_batches=2)
+    z = mixed.decode_host_kv(hcaches, staging, x, dev(p), P, P, P + 1, num_gpu_batches=2, compute_stream=cs,
+                             copy_stream=ps)
+    ps.synchronize()
+    cs.synchronize()
+    fg.fg_sync_status()
+    assert torch.equal(y, z)
+    for hc, c in zip(hcaches, caches):
+        for a, b in zip(hc.arrays(), c.arrays()):
+            assert torch.equal(a, b.cpu())
+    st.close()
+    mixed.close()
