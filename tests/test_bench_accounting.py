@@ -49,3 +49,17 @@ def test_stack_and_prefill_shapes(bench):
     P = wl["prompt"]
     work, _ = bench.kernel_work(wl, P, (P + 1) / 2, fused_append=False)
     assert work["attention"][1] == pytest.approx(wl["heads"] * P * (P + 1) / 2 * 144 + 2 * P * wl["hidden"] * 2)
+
+
+def test_w4a8_decode_step_work(bench):
+    # the W4A8 form: the same 24 S h^2 of products, now integer ("tensor_i8", against the int8
+    # peak), and the activation quantisers of the attention and ReLU outputs: fp16 in, int8 and
+    # one fp32 scale per row out
+    wl = bench.WORKLOADS["opt-6.7b-layer-w4a8"]
+    S, h, F = 512, 4096, 16384
+    work, _ = bench.kernel_work(wl, S, 512)
+    assert sum(w for b, w in work.values() if b == "tensor_i8") == 24 * S * h * h
+    assert not any(b == "tensor" for b, _ in work.values())
+    assert work["out_act8"] == ("hbm", S * h * 3 + S * 4)
+    assert work["fc2_act8"] == ("hbm", S * F * 3 + S * 4)
+    assert bench.kernel_units(wl, S, 512)["fc2_act8"] == S
