@@ -10,7 +10,7 @@
 // `done` (those kernels enqueued before it -> the slice may be overwritten).  So a layer's
 // QKV GEMM starts once wqkv has landed while wo, w1 and w2 are still crossing the link
 // (the weight loader that slices weights across batches, TightLLM abstract; the
-// fine-grained offloading pipeline of PIPO, abstract).  For caches larger than HBM
+// fine-grained offloading pipeline of PIPO, abstract).
 // With one staging buffer (fg_stack_create given the same buffer twice, of
 // fg_stack_one_buffer_bytes) each matrix of layer l+1 waits for layer l's kernels that read
 // the same matrix: about half the staging memory.  The vectors (biases, LayerNorm parameters),
@@ -19,10 +19,11 @@
 // A layer whose blob the caller placed in device memory stays resident: it is read in place,
 // with no copy and no staging buffer (the FlexGen guide's placement of part of the weights on
 // the GPU, section 1; with 180 GB of HBM most of a 175B model's 4-bit weights fit).
-// (a 175B-class stack), fg_stack_decode_host_kv keeps every layer's 4-bit KV cache in
-// pinned host memory too: the copy stream fills a device KV staging cache with the layer's
-// cached positions next to its blob, and writes only the new token slots back after the
-// layer (the pages' guide, section 2: KV cache offloaded alongside the weights).
+// For caches larger than HBM (a 175B-class stack), fg_stack_decode_host_kv keeps every
+// layer's 4-bit KV cache in pinned host memory too: the copy stream fills a device KV staging
+// cache with the layer's cached positions next to its blob, and writes only the new token
+// slots back after the layer (the pages' guide, section 2: KV cache offloaded alongside the
+// weights).
 #include <stdlib.h>
 
 #include <new>
