@@ -84,9 +84,9 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_linear_w4a8.restype = I
         _lib.oracle_linear_w4a8.argtypes = [P, P, I, I, P, P, P, P, I, P, P, I, I, D, P, P]
         _lib.oracle_layer_rows_w4a8.restype = I
-        _lib.oracle_layer_rows_w4a8.argtypes = ([P, D, P] + [P] * 8 + [P] * 6 + [I, I] + [P, I, P, P, I, P, P, I, I])
+        _lib.oracle_layer_rows_w4a8.argtypes = ([P, D, P] + [P] * 8 + [P] * 6 + [I, I] + [P, I, P, P, I, P, P, I])
         _lib.oracle_layer_rows.restype = I
-        _lib.oracle_layer_rows.argtypes = ([P, D] + [P] * 16 + [P] * 4 + [P] * 6 + [I, I] + [P, I, P, P, I, P, P, I, I])
+        _lib.oracle_layer_rows.argtypes = ([P, D] + [P] * 16 + [P] * 4 + [P] * 6 + [I, I] + [P, I, P, P, I, P, P, I])
     return _lib
 
 
@@ -335,14 +335,12 @@ class LayerWeights:
 
 
 def layer_rows(weights: LayerWeights, heads: int, cache: KVCache, x, seq_of_row, pos_of_row,
-               kv_only: bool = False, eps: float = 1e-5, nthreads: int = 1, want_attn: bool = False,
-               keep_cache: bool = False):
+               kv_only: bool = False, eps: float = 1e-5, nthreads: int = 1, want_attn: bool = False):
     """Runs the OPT layer on hidden-state rows ``x [R, h]`` in order.
 
     Row r belongs to sequence ``seq_of_row[r]`` and is the token at cache
     position ``pos_of_row[r]``: its k, v are appended there, then it attends
     over positions ``0..pos``.  The weights' group size is the cache's.
-    ``keep_cache``: the cache already holds every row's k, v (nothing is appended).
     Returns ``(out [R,h] float64, attn [R,h] or None)``.
     """
     x = _u16(x)
@@ -361,7 +359,7 @@ def layer_rows(weights: LayerWeights, heads: int, cache: KVCache, x, seq_of_row,
         args += [_p(np.ascontiguousarray(t.codes)), _p(_u16(t.mins)), _p(_u16(t.scales)), _p(w.b[b])]
     args += [_p(w.b["ln1_g"]), _p(w.b["ln1_b"]), _p(w.b["ln2_g"]), _p(w.b["ln2_b"])]
     args += cache.ptrs() + [cache.S, cache.maxL]
-    args += [_p(x), R, _p(sr), _p(pr), int(kv_only), _p(out), _p(attn), int(nthreads), int(keep_cache)]
+    args += [_p(x), R, _p(sr), _p(pr), int(kv_only), _p(out), _p(attn), int(nthreads)]
     rc = lib().oracle_layer_rows(*args)
     assert rc == 0, rc
     return out, attn
@@ -383,8 +381,7 @@ class W4A8LayerWeights:
 
 
 def layer_rows_w4a8(weights: W4A8LayerWeights, heads: int, cache: KVCache, x, seq_of_row, pos_of_row,
-                    kv_only: bool = False, eps: float = 1e-5, nthreads: int = 1, want_attn: bool = False,
-                    keep_cache: bool = False):
+                    kv_only: bool = False, eps: float = 1e-5, nthreads: int = 1, want_attn: bool = False):
     """``layer_rows`` with the four products in the W4A8 form (the reading in fg_oracle.c): each
     product's fp16 input row is quantised to int8 with one scale and multiplied as integers."""
     x = _u16(x)
@@ -407,7 +404,7 @@ def layer_rows_w4a8(weights: W4A8LayerWeights, heads: int, cache: KVCache, x, se
     args += [_p(w.b["bqkv"]), _p(w.b["bo"]), _p(w.b["b1"]), _p(w.b["b2"])]
     args += [_p(w.b["ln1_g"]), _p(w.b["ln1_b"]), _p(w.b["ln2_g"]), _p(w.b["ln2_b"])]
     args += cache.ptrs() + [cache.S, cache.maxL]
-    args += [_p(x), R, _p(sr), _p(pr), int(kv_only), _p(out), _p(attn), int(nthreads), int(keep_cache)]
+    args += [_p(x), R, _p(sr), _p(pr), int(kv_only), _p(out), _p(attn), int(nthreads)]
     rc = lib().oracle_layer_rows_w4a8(*args)
     assert rc == 0, rc
     return out, attn

@@ -530,7 +530,6 @@ typedef struct {
     const uint16_t *x;                    /* [R][h] */
     const int *seq_of_row, *pos_of_row;
     int R, kv_only, nthreads;
-    int keep_cache;                       /* 1: the cache already holds every row's k, v (no append) */
     double *out, *attn;                   /* [R][h] each (attn may be NULL) */
 } layer_ctx;
 
@@ -590,8 +589,8 @@ static void *layer_worker(void *arg)
         layer_linear(c, 0, a, 3 * h, h, c->bqkv, qkv, x16, q8);
         for (int i = 0; i < h; i++) qkv[i] *= qscale;
         round16_vec(qkv, 3 * h);
-        /* 3. append k, v to the 4-bit cache at pos (unless the cache given already holds them) */
-        for (int hd = 0; hd < H && !c->keep_cache; hd++) {
+        /* 3. append k, v to the 4-bit cache at pos */
+        for (int hd = 0; hd < H; hd++) {
             for (int i = 0; i < d; i++) {
                 k16[i] = oracle_f64_to_f16(qkv[h + hd * d + i]);
                 v16[i] = oracle_f64_to_f16(qkv[2 * h + hd * d + i]);
@@ -643,9 +642,7 @@ static void run_layer_threads(layer_ctx *c, int nthreads)
  * uses the same group along head_dim): wqkv [3h][h], wo [h][h], w1 [F][h],
  * w2 [h][F] (codes, mins, scales each); biases and LayerNorm parameters fp16
  * (NULL = 0, gamma NULL = 1).  The KV cache arrays are read and written in
- * place.  kv_only = 1 stops after step 3 (cache fill for prompts).  keep_cache = 1 skips
- * step 3: the cache given already holds every row's k, v (a comparison that attends over
- * another implementation's KV codes, which a one-ulp difference in k or v can move by a step).
+ * place.  kv_only = 1 stops after step 3 (cache fill for prompts).
  */
 int oracle_layer_rows(const int *dims, double eps,
                       const uint8_t *qkv_c, const uint16_t *qkv_m, const uint16_t *qkv_s, const uint16_t *bqkv,
@@ -656,11 +653,10 @@ int oracle_layer_rows(const int *dims, double eps,
                       uint8_t *kc, uint16_t *km, uint16_t *ks, uint8_t *vc, uint16_t *vm, uint16_t *vs,
                       int S, int maxL,
                       const uint16_t *x, int R, const int *seq_of_row, const int *pos_of_row,
-                      int kv_only, double *out, double *attn, int nthreads, int keep_cache)
+                      int kv_only, double *out, double *attn, int nthreads)
 {
     layer_ctx c;
     memset(&c, 0, sizeof(c));
-    c.keep_cache = keep_cache;
     c.h = dims[0]; c.H = dims[1]; c.d = dims[2]; c.F = dims[3]; c.eps = eps;
     int G = dims[4];
     if (!group_ok(G) || c.h != c.H * c.d || c.h % G || c.F % G || c.d % G) return -1;
@@ -842,11 +838,10 @@ int oracle_layer_rows_w4a8(const int *dims, double eps, const void *const *mats,
                            uint8_t *kc, uint16_t *km, uint16_t *ks, uint8_t *vc, uint16_t *vm, uint16_t *vs,
                            int S, int maxL,
                            const uint16_t *x, int R, const int *seq_of_row, const int *pos_of_row,
-                           int kv_only, double *out, double *attn, int nthreads, int keep_cache)
+                           int kv_only, double *out, double *attn, int nthreads)
 {
     layer_ctx c;
     memset(&c, 0, sizeof(c));
-    c.keep_cache = keep_cache;
     c.h = dims[0]; c.H = dims[1]; c.d = dims[2]; c.F = dims[3]; c.eps = eps;
     if (c.h != c.H * c.d || c.h % OR_GROUP || c.F % OR_GROUP || c.d % OR_GROUP) return -1;
     for (int r = 0; r < R; r++)

@@ -276,25 +276,3 @@ def test_w4a8_layer_close_to_the_w4a16_layer():
     b, _ = oracle.layer_rows(oracle.LayerWeights(w16), H, oracle.KVCache(S, H, h // H, maxL), x, seq, pos)
     dx = x.astype(np.float64)
     assert np.max(np.abs((a - dx) - (b - dx))) <= 0.5 * np.max(np.abs(b - dx))
-
-
-def test_layer_keep_cache_attends_over_the_given_cache():
-    # keep_cache skips the append: over a cache that already holds the rows' own k, v (from a
-    # normal run) both forms of the layer give the same rows as the normal run
-    import seeded_inputs as si
-    h, H, F = 128, 2, 256
-    w16 = si.layer_weights_f16(43, h, F, std=0.05, bias_std=0.05)
-    seq = np.array([0, 0, 1, 0])
-    pos = np.array([0, 1, 0, 2])
-    x = si.normal_f16(43, 9, (len(seq), h), 1.0)
-    for run, W in ((oracle.layer_rows_w4a8, oracle.W4A8LayerWeights(w16)), (oracle.layer_rows, oracle.LayerWeights(w16))):
-        c = oracle.KVCache(2, H, h // H, 64)
-        ref, _ = run(W, H, c, x, seq, pos)
-        kept = oracle.KVCache(2, H, h // H, 64)
-        for a, b in zip(kept.arrays(), c.arrays()):
-            a[...] = b
-        order = np.array([3, 2, 1, 0])                       # any order: nothing is written
-        got, _ = run(W, H, kept, x[order], seq[order], pos[order], keep_cache=True)
-        assert np.array_equal(got, ref[order])
-        for a, b in zip(kept.arrays(), c.arrays()):
-            assert np.array_equal(a, b)
