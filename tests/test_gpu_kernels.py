@@ -579,13 +579,14 @@ def test_linear_permutation_weight_exact():
 @pytest.mark.parametrize("M,N,K", [(8, 256, 8192), (512, 4096, 4096), (40, 384, 16384)])
 def test_linear_split_k_deterministic(M, N, K):
     # few output tiles and a long k-range take the cluster split-k path; two runs give identical bits
-    x = dev(si.normal_f16(17, 1, (M, K), 1.0))
+    xs = si.normal_f16(17, 1, (M, K), 1.0)
+    x = dev(xs)
     w16 = si.normal_f16(17, 2, (N, K), 0.02)
     wq = fg.fg_quantize(dev(w16), dim=1)
     y1 = fg.fg_linear_w4a16(x, wq)
     y2 = fg.fg_linear_w4a16(x, wq)
     assert torch.equal(y1, y2)
-    ref = oracle.linear(host(x), oracle.quantize(w16, 1))
+    ref = oracle.linear(xs, oracle.quantize(w16, 1))
     assert np.max(np.abs(host(y1).astype(np.float64) - ref)) <= 2e-3 * np.max(np.abs(ref))
     if M <= 256:
         assert fg.fg_linear_workspace_bytes(M, N, K) == 0   # one-SM tiles add partials on chip
