@@ -36,13 +36,15 @@ def host(t):
 
 def _weights(seed, N, K):
     """N(0, 0.02) weights with rows of very different magnitudes, an all-zero row, a row with one
-    outlier, and a constant group (the pages' workload: trained-like weights with outliers)."""
+    outlier, a constant group and a row of fp16 subnormals (trained-like weights with outliers)."""
     w = si.normal_f16(seed, 1, (N, K), 0.02).astype(np.float32)
     w *= np.float32(10.0) ** si.normal_f16(seed, 2, (N, 1), 1.0).astype(np.float32).clip(-3, 1)
     w = w.astype(np.float16)
     w[1] = 0
     w[2, K // 3] = 8.0
     w[3, 64:128] = 0.5
+    if N > 5:
+        w[5] = (w[5].astype(np.float32) * np.float32(5e-5)).astype(np.float16)   # fp16 subnormals
     return w
 
 
@@ -52,6 +54,8 @@ def _acts(seed, M, K):
     x = x.astype(np.float16)
     if M > 1:
         x[1] = 0
+    if M > 2:
+        x[2] = (x[2].astype(np.float32) * np.float32(1e-5)).astype(np.float16)   # fp16 subnormals
     return x
 
 
