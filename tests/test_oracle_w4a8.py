@@ -112,6 +112,7 @@ def test_w4a8_row_scale_and_bound():
     w = (rng.standard_normal((9, 256)) * rng.uniform(1e-3, 10, (9, 1))).astype(np.float16)
     w[4] = 0                                                  # an all-zero row
     w[5, 7] = -w[5].astype(np.float32).__abs__().max() * 2    # the row's largest magnitude negative
+    w[6] = (rng.standard_normal(256) * 2e-6).astype(np.float16)  # fp16 subnormals only
     q = oracle.w4a8_quantize_weight(w)
     wf = w.astype(np.float64)
     amax = np.abs(wf).max(axis=1)
