@@ -666,6 +666,18 @@ def run_stack(args, wl):
         with open("/proc/meminfo") as f:
             avail = next(int(ln.split()[1]) * 1024 for ln in f if ln.startswith("MemAvailable"))
         nl = max(2, min(nl, int(avail * 0.5) // per_layer))
+    # --resident-layers: that many layers (or, with "auto", as many as the device memory left
+    # after the KV caches, the staging blobs and caches and 4 GiB of scratch holds) keep their
+    # blobs in HBM, spread evenly over the stack
+    from bit_compressed_decode_b200 import placement
+    if args.resident_layers == "auto":
+        kv_layer = S * H * maxL * 2 * (d // 2 + 4 * ng)
+        reserve = (2 * kv_layer if kv_host else nl * kv_layer) + 2 * cfg.blob_bytes() + (4 << 30)
+        nres = placement.resident_count(torch.cuda.mem_get_info(dev)[0], cfg.blob_bytes(), nl,
+                                         reserve_bytes=reserve)
+    else:
+        nres = min(int(args.resident_layers), nl)
+    resident = placement.spread(nres, nl)
     g = torch.Generator(device=dev)
     g.manual_seed(2000 + rank)
     # weights: seeded device draws N(0, 0.02) (biases 0, LayerNorm 1/0), quantised by fg_quantize,
@@ -684,11 +696,9 @@ def run_stack(args, wl):
             tmp.vector(name).zero_()
         tmp.vector("ln1_g").fill_(1.0)
         tmp.vector("ln2_g").fill_(1.0)
-        # --resident-layers R: R layers spread evenly over the stack keep their blob in device
-        # memory (read in place), so the copy of a streamed layer overlaps the compute of the
-        # resident one before it
-        l = len(host)
-        if (l + 1) * args.resident_layers // nl > l * args.resident_layers // nl:
+        # a resident layer keeps its blob in device memory (read in place); spread evenly, the
+        # copy of a streamed layer overlaps the compute of the resident one before it
+        if resident[len(host)]:
             hb = tmp.blob.clone()
         else:
             hb = torch.empty(cfg.blob_bytes(), dtype=torch.uint8, pin_memory=True)
@@ -777,7 +787,6 @@ def run_stack(args, wl):
     clocks = sampler.stop()
     ms = replicas.max_over_ranks(e0.elapsed_time(e1), device=dev)
     fg.fg_sync_status()
-    nres = min(args.resident_layers, nl)
     blob_gb = cfg.blob_bytes() * (nl - nres) / 1e9
     slot_bytes = S * H * 2 * (d // 2 + 4 * ng)          # K and V codes + min/scale of one position
     fill_gb = wb_gb = 0.0
@@ -799,11 +808,14 @@ def run_stack(args, wl):
                        "resident_layers": nres,
                        "kv": "KV4 g64, seeded random codes at the prompt positions (no prefill)"},
             "host_link_gbs": round((blob_gb + fill_gb + wb_gb) / (ms / args.steps / 1e3), 1),
-            "roofline": {"bound": "host-link", "achieved": round((blob_gb + fill_gb) / (ms / args.steps / 1e3), 1),
-                         "peak": round(link_peak, 1), "unit": "GB/s",
-                         "frac": round((blob_gb + fill_gb) / (ms / args.steps / 1e3) / link_peak, 4),
-                         "traffic": None,
-                         "peak_source": "measured here: pinned host -> device cudaMemcpyAsync of 1 GiB"},
+            "roofline": ({"bound": "host-link", "achieved": round((blob_gb + fill_gb) / (ms / args.steps / 1e3), 1),
+                          "peak": round(link_peak, 1), "unit": "GB/s",
+                          "frac": round((blob_gb + fill_gb) / (ms / args.steps / 1e3) / link_peak, 4),
+                          "traffic": None,
+                          "peak_source": "measured here: pinned host -> device cudaMemcpyAsync of 1 GiB"}
+                         if blob_gb + fill_gb > 0 else
+                         {"bound": None, "note": "every layer resident in HBM: nothing crosses the host link; "
+                                                 "the layer kernels' own rooflines apply (see the decode workloads)"}),
             "clocks": clocks,
         }
         if kv_host:
@@ -958,8 +970,9 @@ def main():
     ap.add_argument("--group", type=int, choices=(64, 128), default=64,
                     help="quantisation group size: of the layer's weights and KV cache (layer workloads), or of "
                          "--kernel quantize/dequantize/*_gemm")
-    ap.add_argument("--resident-layers", type=int, default=0,
-                    help="stack workloads: layers whose weight blobs stay in device memory (read in place)")
+    ap.add_argument("--resident-layers", default="0",
+                    help="stack workloads: layers whose weight blobs stay in device memory (read in place), "
+                         "or 'auto': as many as the device memory left holds")
     ap.add_argument("--staging-buffers", type=int, choices=(1, 2), default=2,
                     help="opt-30b-stack: device staging blobs (2 alternate; 1 is refilled slice by slice)")
     ap.add_argument("--gemm-scratch", choices=("auto", "persistent", "classic", "none"), default="auto",
